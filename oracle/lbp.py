@@ -1,0 +1,367 @@
+"""Plain fp64 statement of the hot path: IBP, ReLU relaxation, CROWN back-substitution,
+concretisation over an L-infinity box, intermediate-bound passes and the final decision.
+
+TEST INFRASTRUCTURE (see the package docstring): only tests, the smoke check and
+the benchmark's CPU-baseline leg use this module.
+
+Page: "Scaling Neural Network Verification with Tensor Parallelism and Fully
+Sharded Data Parallelism" (gist.science summary of arXiv 2606.09377), cited as
+[SNNV <section>]:
+  * [SNNV §1]   the task: prove a property for every input of a domain, with the
+                weights and the linear relaxation matrices A of IBP / CROWN /
+                alpha-CROWN held on one accelerator;
+  * [SNNV §2.1] CROWN's backward pass needs intermediate bounds to fix the ReLU
+                relaxation slopes lambda_i; IBP is the cheap, looser but still sound
+                substitute for them;
+  * [SNNV §3], [SNNV §4.3] per-neuron alpha tensors (the ReLU lower slopes);
+  * [SNNV §4.2] soundness means a one-sided over-approximation.
+
+Everything is computed in float64 from the fp32 inputs promoted exactly. The
+oracle works centre by centre, and within a centre on all specification rows at
+once; matrix products use numpy's matmul as a library step. Rows are independent,
+so a pass may be split into row blocks purely to bound memory.
+
+Network format: a list of nodes in topological order (``src`` < own index), node 0
+the input; ops ``input``, ``dense`` (W [n_out, n_in], b), ``conv`` (W [Co, Ci, k, k],
+b [Co], stride, pad), ``relu``, ``add`` (src + src2). Activations are flattened in
+C order (channel, row, column).
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+F = np.float64
+
+
+# ----------------------------------------------------------------------------- shapes
+
+def shapes(net) -> List[tuple]:
+    out = []
+    for nd in net:
+        if nd.op == "input":
+            out.append(tuple(nd.shape))
+        elif nd.op == "dense":
+            out.append((nd.W.shape[0],))
+        elif nd.op == "conv":
+            c, h, w = out[nd.src]
+            k = nd.W.shape[2]
+            out.append((nd.W.shape[0], (h + 2 * nd.pad - k) // nd.stride + 1,
+                        (w + 2 * nd.pad - k) // nd.stride + 1))
+        elif nd.op in ("relu", "add"):
+            out.append(out[nd.src])
+        else:
+            raise ValueError(nd.op)
+    return out
+
+
+def _size(shape) -> int:
+    return int(np.prod(shape))
+
+
+# ----------------------------------------------------------------------------- convolution
+
+def conv2d(x: np.ndarray, W: np.ndarray, stride: int, pad: int) -> np.ndarray:
+    """Cross-correlation by its definition, without bias.
+
+    out[n, o, i, j] = sum_{c, p, q} W[o, c, p, q] * x[n, c, i*stride - pad + p, j*stride - pad + q],
+    with x read as zero outside the image. x: [N, Ci, H, W] -> [N, Co, Ho, Wo].
+    """
+    N, Ci, H, Wd = x.shape
+    Co, _, k, _ = W.shape
+    Ho = (H + 2 * pad - k) // stride + 1
+    Wo = (Wd + 2 * pad - k) // stride + 1
+    xp = np.zeros((N, Ci, H + 2 * pad, Wd + 2 * pad), F)
+    xp[:, :, pad:pad + H, pad:pad + Wd] = x
+    out = np.zeros((N, Co, Ho, Wo), F)
+    Wf = W.astype(F)
+    for p in range(k):
+        for q in range(k):
+            patch = xp[:, :, p:p + stride * (Ho - 1) + 1:stride, q:q + stride * (Wo - 1) + 1:stride]
+            out += np.einsum("nchw,oc->nohw", patch, Wf[:, :, p, q], optimize=True)
+    return out
+
+
+def conv2d_adjoint(y: np.ndarray, W: np.ndarray, stride: int, pad: int, in_hw) -> np.ndarray:
+    """Adjoint (transpose) of :func:`conv2d`: <conv2d(x), y> = <x, conv2d_adjoint(y)> for all x, y.
+
+    y: [N, Co, Ho, Wo] -> [N, Ci, H, W]. Each output position scatters its
+    coefficient back onto the input positions it read.
+    """
+    N, Co, Ho, Wo = y.shape
+    _, Ci, k, _ = W.shape
+    H, Wd = in_hw
+    gp = np.zeros((N, Ci, H + 2 * pad, Wd + 2 * pad), F)
+    Wf = W.astype(F)
+    for p in range(k):
+        for q in range(k):
+            gp[:, :, p:p + stride * (Ho - 1) + 1:stride, q:q + stride * (Wo - 1) + 1:stride] += \
+                np.einsum("nohw,oc->nchw", y, Wf[:, :, p, q], optimize=True)
+    return gp[:, :, pad:pad + H, pad:pad + Wd]
+
+
+# ----------------------------------------------------------------------------- forward
+
+def forward(net, x: np.ndarray) -> List[np.ndarray]:
+    """Plain fp64 evaluation; x [N, n0]. Returns every node's output, flattened [N, n_v]."""
+    sh = shapes(net)
+    x = np.asarray(x, F)
+    N = x.shape[0]
+    outs: List[np.ndarray] = []
+    for v, nd in enumerate(net):
+        if nd.op == "input":
+            o = x
+        elif nd.op == "dense":
+            o = outs[nd.src] @ nd.W.astype(F).T + nd.b.astype(F)
+        elif nd.op == "conv":
+            xs = outs[nd.src].reshape((N,) + sh[nd.src])
+            o = conv2d(xs, nd.W, nd.stride, nd.pad) + nd.b.astype(F)[None, :, None, None]
+            o = o.reshape(N, -1)
+        elif nd.op == "relu":
+            o = np.maximum(outs[nd.src], 0.0)
+        elif nd.op == "add":
+            o = outs[nd.src] + outs[nd.src2]
+        outs.append(o)
+    return outs
+
+
+# ----------------------------------------------------------------------------- IBP
+
+def ibp(net, centres: np.ndarray, eps: float):
+    """Interval bound propagation in centre/radius form [SNNV §2.1, §4.2].
+
+    The input box is centre c, radius eps (no clipping to any data range: the page
+    only speaks of "a specified domain" [SNNV §1]; the plain reading is the L-inf ball).
+    Affine node: centre' = W c + b, radius' = |W| r (the exact image of a box under an
+    affine map, coordinate-wise). ReLU: clamp both ends, then back to centre/radius.
+    Add: centres add, radii add.
+
+    Returns (centre, radius) lists over nodes, each [B, n_v] float64.
+    """
+    sh = shapes(net)
+    c0 = np.asarray(centres, F)
+    B = c0.shape[0]
+    cs: List[np.ndarray] = []
+    rs: List[np.ndarray] = []
+    for v, nd in enumerate(net):
+        if nd.op == "input":
+            c, r = c0, np.full_like(c0, F(eps))
+        elif nd.op == "dense":
+            Wf = nd.W.astype(F)
+            c = cs[nd.src] @ Wf.T + nd.b.astype(F)
+            r = rs[nd.src] @ np.abs(Wf).T
+        elif nd.op == "conv":
+            ci = cs[nd.src].reshape((B,) + sh[nd.src])
+            ri = rs[nd.src].reshape((B,) + sh[nd.src])
+            c = (conv2d(ci, nd.W, nd.stride, nd.pad) + nd.b.astype(F)[None, :, None, None]).reshape(B, -1)
+            r = conv2d(ri, np.abs(nd.W.astype(F)), nd.stride, nd.pad).reshape(B, -1)
+        elif nd.op == "relu":
+            lo = np.maximum(cs[nd.src] - rs[nd.src], 0.0)
+            hi = np.maximum(cs[nd.src] + rs[nd.src], 0.0)
+            c, r = (hi + lo) / 2.0, (hi - lo) / 2.0
+        elif nd.op == "add":
+            c, r = cs[nd.src] + cs[nd.src2], rs[nd.src] + rs[nd.src2]
+        cs.append(c)
+        rs.append(r)
+    return cs, rs
+
+
+# ----------------------------------------------------------------------------- relaxation
+
+def relax_params(l: np.ndarray, u: np.ndarray, alpha: Optional[np.ndarray] = None):
+    """Linear relaxation of h = ReLU(z) for l <= z <= u [SNNV §2.1: slopes lambda_i; §3: alpha].
+
+    Returns (lo, up, t): lower relaxation h >= lo * z, upper relaxation h <= up * z + t.
+      * u <= 0 (inactive, tested first): lo = up = t = 0 (h = 0 exactly);
+      * else l >= 0 (active):            lo = up = 1, t = 0 (h = z exactly);
+      * else (unstable, l < 0 < u):      up = u / (u - l), t = -up * l (the chord), and
+                                          lo = alpha clamped to [0, 1] when alpha is given,
+                                          otherwise the adaptive choice lo = 1 if u >= -l else 0.
+    """
+    l = np.asarray(l, F)
+    u = np.asarray(u, F)
+    lo = np.zeros_like(l)
+    up = np.zeros_like(l)
+    t = np.zeros_like(l)
+    inactive = u <= 0.0
+    active = (~inactive) & (l >= 0.0)
+    unstable = (~inactive) & (~active)
+    lo[active] = 1.0
+    up[active] = 1.0
+    s = u[unstable] / (u[unstable] - l[unstable])
+    up[unstable] = s
+    t[unstable] = -s * l[unstable]
+    if alpha is None:
+        lo[unstable] = np.where(u[unstable] >= -l[unstable], 1.0, 0.0)
+    else:
+        a = np.asarray(alpha, F)
+        if np.isnan(a).any():
+            raise ValueError("alpha contains NaN")
+        lo[unstable] = np.clip(a[unstable], 0.0, 1.0)
+    return lo, up, t
+
+
+# ----------------------------------------------------------------------------- CROWN
+
+def backward(net, start: int, lam0: np.ndarray, relax: Dict[int, tuple], const0=None):
+    """Back-substitute lower-bound rows from node ``start`` to the input [SNNV §1, §2.1].
+
+    lam0 [R, n_start]: the rows' coefficients over node ``start``'s output. For every
+    row the result (lam_in [R, n0], const [R]) satisfies, for each x in the domain,
+    lam0 . node_start(x) >= lam_in . x + const, given the relaxations in ``relax``
+    (relu node -> (lo, up, t) vectors for this centre).
+
+    Nodes are visited in reverse topological order; a node's coefficient matrix is
+    complete once all its consumers (which have larger indices) have been visited.
+      dense z = W h + b:  const += lam . b;  lam_h += lam W
+      conv:               const += sum over (c, i, j) of lam[c, i, j] * b[c];  lam_h += conv^T(lam)
+      relu h = ReLU(z):   positive coefficients take the lower relaxation, negative ones the
+                          upper: lam_z = lo * max(lam, 0) + up * min(lam, 0);
+                          const += min(lam, 0) . t
+      add y = a + b:      lam_a += lam; lam_b += lam
+    """
+    sh = shapes(net)
+    R = lam0.shape[0]
+    pend: Dict[int, np.ndarray] = {start: np.asarray(lam0, F)}
+    const = np.zeros(R, F) if const0 is None else np.asarray(const0, F).copy()
+
+    def put(v, m):
+        if v in pend:
+            pend[v] = pend[v] + m
+        else:
+            pend[v] = m
+
+    for v in range(start, -1, -1):
+        if v not in pend:
+            continue
+        lam = pend.pop(v)
+        nd = net[v]
+        if nd.op == "input":
+            return lam, const
+        if nd.op == "dense":
+            const = const + lam @ nd.b.astype(F)
+            put(nd.src, lam @ nd.W.astype(F))
+        elif nd.op == "conv":
+            co = nd.W.shape[0]
+            lam4 = lam.reshape((R,) + sh[v])
+            const = const + lam4.reshape(R, co, -1).sum(axis=2) @ nd.b.astype(F)
+            put(nd.src, conv2d_adjoint(lam4, nd.W, nd.stride, nd.pad, sh[nd.src][1:]).reshape(R, -1))
+        elif nd.op == "relu":
+            lo, up, t = relax[v]
+            pos = np.maximum(lam, 0.0)
+            neg = np.minimum(lam, 0.0)
+            const = const + neg @ t
+            put(nd.src, pos * lo + neg * up)
+        elif nd.op == "add":
+            put(nd.src, lam)
+            put(nd.src2, lam)
+    raise AssertionError("input node not reached")
+
+
+def concretize(lam_in: np.ndarray, const: np.ndarray, centre: np.ndarray, eps: float) -> np.ndarray:
+    """Minimum of lam_in . x + const over the box |x - centre|_inf <= eps [SNNV §1]:
+    lam_in . centre - eps * sum |lam_in| + const (attained at x = centre - eps * sign(lam_in))."""
+    c = np.asarray(centre, F)
+    return lam_in @ c - F(eps) * np.abs(lam_in).sum(axis=1) + const
+
+
+def crown_pass(net, start: int, lam0: np.ndarray, relax, centre, eps, row_block: int = 4096):
+    """backward + concretize for a block of rows; rows are independent, so large passes
+    are evaluated ``row_block`` rows at a time (memory only: each row's arithmetic is unchanged)."""
+    R = lam0.shape[0]
+    out = np.empty(R, F)
+    for r0 in range(0, R, row_block):
+        r1 = min(R, r0 + row_block)
+        lam_in, cst = backward(net, start, lam0[r0:r1], relax)
+        out[r0:r1] = concretize(lam_in, cst, centre, eps)
+    return out
+
+
+# ----------------------------------------------------------------------------- full verify
+
+@dataclasses.dataclass
+class OracleResult:
+    lb: np.ndarray            # [B, R] final lower bound max(IBP, CROWN)
+    ub: Optional[np.ndarray]  # [B, R] final upper bound min(IBP, CROWN) (both sides only)
+    lb_ibp: np.ndarray        # [B, R]
+    ub_ibp: np.ndarray        # [B, R]
+    lb_crown: np.ndarray      # [B, R]
+    ub_crown: Optional[np.ndarray]
+    verified: np.ndarray      # [B, R] bool, lb > 0
+    pre_bounds: Dict[int, tuple]  # relu node -> (l, u) [B, n] used for its relaxation
+    ibp_bounds: Dict[int, tuple]  # every node -> (l, u) [B, n] from the single IBP pass
+
+
+def _first_affine_on_input(net, p: int) -> bool:
+    nd = net[p]
+    return nd.op in ("dense", "conv") and nd.src == 0
+
+
+def verify(net, centres, eps, C, crown_relus: Optional[Sequence[int]] = None,
+           alphas: Optional[Dict[int, np.ndarray]] = None, both_sides: bool = False,
+           row_block: int = 4096) -> OracleResult:
+    """IBP, then CROWN intermediate bounds, then the specification pass and decision.
+
+    Readings taken where the page is silent (it names the methods only, [SNNV §1, §2.1]):
+      * one IBP pass over the whole network with the plain IBP bounds (later layers
+        are not re-propagated from refined bounds);
+      * for each ReLU node k in topological order whose pre-activation node p is in
+        ``crown_relus`` (None = every ReLU): a CROWN pass from rows [I; -I] over p gives
+        l_cr (first half) and -u_cr (second half); IBP-unstable neurons (l < 0 < u) take
+        l = max(l_ibp, l_cr), u = min(u_ibp, u_cr); IBP-stable neurons keep the IBP bounds
+        (their relaxation is exact either way). When p is a single affine node fed by
+        the input, IBP already gives the exact range and no pass is run;
+      * every other ReLU keeps its IBP bounds (the IBP substitution of [SNNV §2.1]);
+      * specification rows C_b [R, n_L] act on the last node: the CROWN lower bound
+        comes from back-substituting C_b; the IBP bound from C applied to the last
+        node's interval, C c - |C| r; the final lower bound is the larger (both are sound)
+        and a row is verified iff it is > 0 [SNNV §1]. Upper bounds, when asked for,
+        are -lower(-C) and C c + |C| r, the final one the smaller;
+      * alpha (relu node -> [B, n]) is shared by all rows and passes; missing = adaptive.
+    """
+    centres = np.asarray(centres, F)
+    B = centres.shape[0]
+    C = np.asarray(C, F)
+    R = C.shape[1]
+    sh = shapes(net)
+    L = len(net) - 1
+    cs, rs = ibp(net, centres, eps)
+    ibp_b = {v: (cs[v] - rs[v], cs[v] + rs[v]) for v in range(len(net))}
+    relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
+    crown_set = set(relus if crown_relus is None else crown_relus)
+    alphas = alphas or {}
+
+    pre = {k: (ibp_b[net[k].src][0].copy(), ibp_b[net[k].src][1].copy()) for k in relus}
+    lb_cr = np.empty((B, R), F)
+    ub_cr = np.empty((B, R), F) if both_sides else None
+    for b in range(B):
+        relax: Dict[int, tuple] = {}
+        for k in relus:
+            p = net[k].src
+            if k in crown_set and not _first_affine_on_input(net, p):
+                n = _size(sh[p])
+                eye = np.eye(n, dtype=F)
+                lbs = crown_pass(net, p, np.concatenate([eye, -eye]), relax, centres[b], eps, row_block)
+                l_cr, u_cr = lbs[:n], -lbs[n:]
+                l0, u0 = pre[k][0][b], pre[k][1][b]
+                unst = (l0 < 0.0) & (u0 > 0.0)
+                pre[k][0][b] = np.where(unst, np.maximum(l0, l_cr), l0)
+                pre[k][1][b] = np.where(unst, np.minimum(u0, u_cr), u0)
+            a = alphas.get(k)
+            relax[k] = relax_params(pre[k][0][b], pre[k][1][b], None if a is None else a[b])
+        Cb = C[b if C.shape[0] > 1 else 0]
+        rows = np.concatenate([Cb, -Cb]) if both_sides else Cb
+        lbs = crown_pass(net, L, rows, relax, centres[b], eps, row_block)
+        lb_cr[b] = lbs[:R]
+        if both_sides:
+            ub_cr[b] = -lbs[R:]
+    Cfull = np.broadcast_to(C, (B,) + C.shape[1:])
+    zc, zr = cs[L], rs[L]
+    lb_ibp = np.einsum("brn,bn->br", Cfull, zc) - np.einsum("brn,bn->br", np.abs(Cfull), zr)
+    ub_ibp = np.einsum("brn,bn->br", Cfull, zc) + np.einsum("brn,bn->br", np.abs(Cfull), zr)
+    lb = np.maximum(lb_ibp, lb_cr)
+    ub = np.minimum(ub_ibp, ub_cr) if both_sides else None
+    return OracleResult(lb=lb, ub=ub, lb_ibp=lb_ibp, ub_ibp=ub_ibp, lb_crown=lb_cr, ub_crown=ub_cr,
+                        verified=lb > 0.0, pre_bounds=pre, ibp_bounds=ibp_b)
