@@ -1,0 +1,302 @@
+#!/usr/bin/env python
+"""Throughput benchmark: verified specs/sec of one full bound-propagation step on B200.
+
+A step is one vf_verify_batch call over the whole batch: IBP over every node, CROWN passes
+for the intermediate bounds, the specification pass and the decision. Default workload:
+ReLU MLP 784-256-256-256-10, 1024 centres, eps = 2/255, 9 margin rows per centre, CROWN
+intermediate bounds for z2 and z3 (synthetic, seeded; see linear_bound_propagation_b200.synth).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1..5]
+
+Prints one JSON line (rank 0). With N > 1 (torchrun) every rank runs an independent replica
+of the workload on its own GPU (no collective on the data path; the barrier and the max over
+ranks are for timing only), so `value` counts the specs of all ranks ("scaling": "weak").
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_bound_propagation_b200 import synth  # noqa: E402
+
+METRIC = "verified specs/sec (IBP+CROWN bounds) at 1 B200; % tensor-pipe / HBM roofline"
+UNIT = "specs/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}, \
+            "fallback"
+
+
+def threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def workload_config(w, cfg):
+    R = w.C.shape[1]
+    return {"workload": w.name, "centres": int(w.centres.shape[0]), "spec_rows": int(R),
+            "eps": float(w.eps), "both_sides": bool(w.both_sides),
+            "intermediate_bounds": "crown for relus " + (str(w.crown_relus) if w.crown_relus else "all (first layer exact by IBP)"),
+            "l2": "flushed between timed steps (256 MiB write)", "parallelism": "replicas (one full workload per GPU)",
+            "config_index": cfg}
+
+
+def oracle_sample(w, target_s):
+    """Time the oracle on the first n centres of the workload, n sized to about target_s seconds."""
+    import oracle.lbp as O
+    R = w.C.shape[1] * (2 if w.both_sides else 1)
+
+    def run(n):
+        t0 = time.perf_counter()
+        O.verify(w.net, w.centres[:n], w.eps, w.C[:n] if w.C.shape[0] > 1 else w.C, crown_relus=w.crown_relus,
+                 both_sides=w.both_sides)
+        return time.perf_counter() - t0
+
+    B = w.centres.shape[0]
+    t1 = run(1)
+    n = int(max(1, min(B, target_s / max(t1, 1e-6))))
+    t = run(n) if n > 1 else t1
+    return {"value": n * R / t, "unit": UNIT, "cores": threads_used(), "kind": "oracle",
+            "sample": f"first {n} of {B} centres of {w.name} ({n * R} specs), fp64 numpy oracle, {t:.2f} s"}, n, t
+
+
+def start_clocks():
+    path = tempfile.mktemp(suffix=".csv")
+    q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+    dev = os.environ.get("LOCAL_RANK", "0")
+    try:
+        f = open(path, "w")
+        p = subprocess.Popen(["nvidia-smi", "-i", str(dev), f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                              "-lms", "200"], stdout=f, stderr=subprocess.DEVNULL)
+        return p, f, path
+    except Exception:
+        return None, None, path
+
+
+def stop_clocks(handle):
+    p, f, path = handle
+    if p is None:
+        return None
+    p.terminate()
+    try:
+        p.wait(timeout=5)
+    except Exception:
+        p.kill()
+    f.close()
+    sm, mx, reasons = [], 0.0, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    with open(path) as fh:
+        for line in fh:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+    os.unlink(path)
+    if not sm:
+        return None
+    return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = synth.workload(args.config)
+    base, n, t = oracle_sample(w, args.cpu_sample_s)
+    R = w.C.shape[1] * (2 if w.both_sides else 1)
+    import oracle.lbp as O
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        O.verify(w.net, w.centres[:n], w.eps, w.C[:n] if w.C.shape[0] > 1 else w.C, crown_relus=w.crown_relus,
+                 both_sides=w.both_sides)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    value = n * R * len(times) / sum(times)
+    base["value"] = value
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * sum(times) / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, args.config), "cpu_baseline": base,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from linear_bound_propagation_b200 import vf
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = synth.workload(args.config)
+    B, R = w.centres.shape[0], w.C.shape[1]
+    Rs = R * (2 if w.both_sides else 1)
+    net = vf.Net(w.net, workspace_bytes=int(args.workspace_gb * (1 << 30)))
+    dev = torch.device("cuda", local)
+    centres = torch.from_numpy(w.centres).to(dev)
+    C = torch.from_numpy(w.C).to(dev)
+    stream = torch.cuda.current_stream()
+    out = {"lb": torch.empty(B, R, device=dev), "lb_ibp": torch.empty(B, R, device=dev),
+           "verified": torch.empty(B, R, device=dev, dtype=torch.uint8)}
+    if w.both_sides:
+        out["ub"] = torch.empty(B, R, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev)
+    kw = dict(crown_relus=w.crown_relus, both_sides=w.both_sides, out=out)
+
+    for _ in range(args.warmup):
+        net.verify(centres, w.eps, C, **kw)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+
+    clk = start_clocks()
+    launches0 = net.launch_count()
+    net.profile(True)
+    net.profile_read(reset=True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        net.verify(centres, w.eps, C, **kw)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = stop_clocks(clk)
+    launches = net.launch_count() - launches0
+    n_k, k_ms, k_flops = net.profile_read(reset=True)
+    net.profile(False)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * B * Rs * args.steps / (total_ms / 1000.0)
+    verified = int(out["verified"].sum().item())
+
+    # End to end through the public API with host buffers: pinned H2D of centres and C, the
+    # verify call, D2H of lb and verified, every step inside the timed region.
+    h_centres = torch.from_numpy(w.centres).pin_memory()
+    h_C = torch.from_numpy(w.C).pin_memory()
+    h_lb = torch.empty(B, R).pin_memory()
+    h_ver = torch.empty(B, R, dtype=torch.uint8).pin_memory()
+    d_c = torch.empty_like(centres)
+    d_C = torch.empty_like(C)
+    for _ in range(2):
+        d_c.copy_(h_centres, non_blocking=True)
+        d_C.copy_(h_C, non_blocking=True)
+        net.verify(d_c, w.eps, d_C, **kw)
+        h_lb.copy_(out["lb"], non_blocking=True)
+        h_ver.copy_(out["verified"], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = 0.0
+    for i in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        d_c.copy_(h_centres, non_blocking=True)
+        d_C.copy_(h_C, non_blocking=True)
+        net.verify(d_c, w.eps, d_C, **kw)
+        h_lb.copy_(out["lb"], non_blocking=True)
+        h_ver.copy_(out["verified"], non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms += a.elapsed_time(b)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = h_centres.numel() * 4 + h_C.numel() * 4
+    d2h = h_lb.numel() * 4 + h_ver.numel()
+
+    p, src = peaks()
+    sm_mhz = float(p.get("sm_max_mhz", 1965.0))
+    props = torch.cuda.get_device_properties(dev)
+    ffma_peak = props.multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
+    avg_ms = k_ms / max(n_k, 1)
+    achieved = (k_flops / max(n_k, 1)) / (avg_ms / 1000.0) / 1e12 if n_k else 0.0
+    roof = {"bound": "alu", "achieved": achieved, "peak": ffma_peak, "unit": "TFLOP/s",
+            "frac": achieved / ffma_peak, "traffic": None, "kernel": "dense_back_ffma (CROWN Lambda.W contraction)",
+            "launches": n_k, "avg_launch_ms": avg_ms, "share_of_step": k_ms / total_ms if total_ms else None,
+            "peak_source": f"fp32 FFMA: {props.multi_processor_count} SMs x 128 lanes x 2 flop x {sm_mhz:.0f} MHz "
+                           f"({src} max clock)"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": workload_config(w, args.config), "roofline": roof,
+                "e2e": {"value": world * B * Rs * args.steps / (e2e_ms / 1000.0), "unit": UNIT,
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "gpu_launches": launches, "clocks": clocks, "verified_specs": verified, "total_specs": B * Rs}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample(w, args.cpu_sample_s)[0]
+        print(json.dumps(line), flush=True)
+    net.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--workspace-gb", type=float, default=16.0)
+    ap.add_argument("--cpu-sample-s", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,158 @@
+/*
+ * vf.h -- C ABI of libvf.so: linear bound propagation (IBP + CROWN with alpha-slope
+ * ReLU relaxation) for ReLU networks over an L-infinity input box, on one NVIDIA B200.
+ *
+ * Source page for the method: "Scaling Neural Network Verification with Tensor
+ * Parallelism and Fully Sharded Data Parallelism" (gist.science summary of arXiv
+ * 2606.09377). Its technical summary, section 1 (problem definition), states the task:
+ * prove that a network satisfies a property for every input of a domain, using bound
+ * propagation (IBP, CROWN, alpha-CROWN) whose weight matrices and linear relaxation
+ * matrices A sit on one accelerator. Section 2.1 states that CROWN's backward pass
+ * needs intermediate bounds to fix the ReLU relaxation slopes and that IBP can stand in
+ * for them; sections 3 and 4.3 name the per-neuron alpha tensors (ReLU slopes).
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked [device] must be CUDA device memory of the current device;
+ *    [host] pointers are host memory. All floating point data is fp32, row-major.
+ *  - A network's activations are flattened in C order (channel, row, column).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Calls
+ *    only enqueue work on it; outputs are valid once the stream reaches that point.
+ *  - Return value: VF_OK (0) or a vf_status error code. On error nothing further is
+ *    enqueued and vf_last_error() (per thread) describes the failure. No entry point
+ *    aborts or throws across the ABI. Asynchronous CUDA faults surface as VF_ERR_CUDA
+ *    on a later call or from vf_sync().
+ *  - The caller owns every buffer it passes; the library owns only what vf_net_create
+ *    allocates (device copies of the weights, derived tables and the workspace), which
+ *    vf_net_destroy frees. A vf_net is not thread-safe: one call at a time per handle.
+ */
+#ifndef VF_H
+#define VF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    VF_OK = 0,
+    VF_ERR_ARG = 1,         /* null pointer, bad enum, negative size */
+    VF_ERR_SHAPE = 2,       /* inconsistent node shapes or sizes */
+    VF_ERR_WORKSPACE = 3,   /* the workspace given to vf_net_create is too small for this call */
+    VF_ERR_NONFINITE = 4,   /* NaN/Inf in eps, centres, C, weights or alpha */
+    VF_ERR_CUDA = 5,        /* a CUDA runtime call or kernel failed */
+    VF_ERR_TIMEOUT = 6,     /* reserved: a bounded device wait gave up */
+    VF_ERR_UNSUPPORTED = 7  /* valid request outside what this build implements */
+} vf_status;
+
+/* Node kinds. A network is an array of nodes in topological order: every `src`/`src2`
+ * index is smaller than the node's own index; node 0 is the only VF_INPUT. */
+typedef enum {
+    VF_INPUT = 0,   /* shape (c, h, w); use (n, 1, 1) for a flat input */
+    VF_DENSE = 1,   /* z = W h + b,  W [n_out, n_in], b [n_out]; h is src flattened */
+    VF_CONV2D = 2,  /* cross-correlation, W [c_out, c_in, k, k], b [c_out], stride, pad (zeros) */
+    VF_RELU = 3,    /* h = max(z, 0) of src */
+    VF_ADD = 4      /* src + src2 (same shape) */
+} vf_op;
+
+typedef struct {
+    int op;                /* vf_op */
+    int src, src2;         /* producer node indices; src2 only for VF_ADD (else -1) */
+    int c, h, w;           /* VF_INPUT only: input shape */
+    int n_out;             /* VF_DENSE: output width; VF_CONV2D: output channels */
+    int k, stride, pad;    /* VF_CONV2D only */
+    const float* W;        /* [host or device] weights, layout above; copied at create */
+    const float* b;        /* [host or device] bias; copied at create */
+} vf_node_desc;
+
+typedef struct vf_net vf_net;
+
+/* Build a network handle on the current CUDA device. Weights are copied (host or
+ * device source, detected per pointer) and checked for finiteness; derived tables
+ * (|W|, [W; -W] start rows for intermediate passes) are built once here.
+ * `workspace_bytes` is the device scratch the handle reserves for every later call
+ * (allocated here, once); 0 selects 4 GiB. Calls whose fixed buffers do not fit return
+ * VF_ERR_WORKSPACE; CROWN row blocks are otherwise sized to fit the workspace. */
+int vf_net_create(const vf_node_desc* nodes /*[host] n_nodes*/, int n_nodes, size_t workspace_bytes,
+                  vf_net** out_net /*[host]*/);
+void vf_net_destroy(vf_net* net);
+
+/* Number of neurons of node v (its flattened output size), or -1 if v is out of range. */
+int vf_net_node_size(const vf_net* net, int v);
+/* Sum of vf_net_node_size over all nodes: the row length of vf_ibp's bound arrays per centre block. */
+long long vf_net_total_size(const vf_net* net);
+
+/* IBP pass (technical summary, section 2.1: the cheap, sound interval substitute).
+ * Box: centres[b] +/- eps (no clipping). For every node v, writes its interval bounds
+ * into lb_all/ub_all at offset B * (sum of sizes of nodes before v), as a [B, n_v] block.
+ * centres [device] [B, n0]; lb_all, ub_all [device] [B * vf_net_total_size(net)]. */
+int vf_ibp(vf_net* net, const float* centres, int B, float eps, float* lb_all, float* ub_all, void* stream);
+
+/* CROWN back-substitution of lower-bound rows (section 1: the linear relaxation
+ * matrices A; section 2.1: the relaxation slopes come from intermediate bounds).
+ * Rows: lambda0 [device] [B or 1, R, n_start] (centre stride lambda0_bstride elements;
+ * 0 = one block shared by all centres) are coefficients over node `start_node`'s output.
+ * Each ReLU reached uses the bounds of its source node found in lb_all/ub_all (layout of
+ * vf_ibp) and alpha[v] [device] [B, n_v] for ReLU node v (NULL array or NULL entry =
+ * adaptive slope 1 iff u >= -l; given slopes are clamped to [0, 1]).
+ * Outputs: lambda_in [device] [B, R, n0] and const_out [device] [B, R] such that, for
+ * every input x in any domain, row . node_start(x) >= lambda_in . x + const_out.
+ * Upper bounds: pass -lambda0 and negate the result. */
+int vf_crown_backward(vf_net* net, int start_node, const float* lambda0, int R, long long lambda0_bstride,
+                      const float* lb_all, const float* ub_all, const float* const* alpha /*[host] n_nodes or NULL*/,
+                      int B, float* lambda_in, float* const_out, void* stream);
+
+/* Concretisation over the box centres[b] +/- eps (section 1: "all inputs in the domain"):
+ * lb[b, r] = lambda[b, r, :] . centres[b, :] - eps * sum_i |lambda[b, r, i]| + cst[b, r].
+ * lambda [device] [B, R, n0], cst [device] [B, R] (or NULL = 0), centres [device] [B, n0],
+ * lb [device] [B, R]. No handle needed; no scratch memory. */
+int vf_concretize(const float* lambda, const float* cst, const float* centres, float eps, int B, int R, int n0,
+                  float* lb, void* stream);
+
+typedef struct {
+    /* [host] n_nodes entries or NULL. For each ReLU node v: 1 = refine the bounds of its
+     * source by a CROWN pass (rows [I; -I]) before use, 0 = keep the IBP bounds (the IBP
+     * substitution of section 2.1). NULL = CROWN for every ReLU. A source that is a single
+     * affine node fed by the input already has exact IBP bounds and is never re-run. */
+    const int* relu_crown;
+    /* [host] n_nodes entries of [device] [B, n_v] slopes, or NULL (all adaptive). */
+    const float* const* alpha;
+    int both_sides;          /* 1: also compute upper bounds (rows -C) */
+    int skip_finite_check;   /* 1: skip the device NaN/Inf scan of centres, C and alpha */
+    /* [device] optional outputs [B * vf_net_total_size(net)] in the vf_ibp layout: the
+     * bounds used for each ReLU source after refinement (other nodes: IBP bounds). */
+    float* pre_lb;
+    float* pre_ub;
+} vf_opts;
+
+/* Whole verification step (section 1): IBP, CROWN intermediate bounds, specification
+ * pass, decision. C [device] [B or 1, R, n_L] over the last node (centre stride
+ * C_bstride elements; 0 = shared). Outputs [device], [B, R] each:
+ *   lb = max(IBP lower, CROWN lower); ub (both_sides only, else may be NULL) =
+ *   min(IBP upper, CROWN upper); lb_ibp (or NULL) the IBP lower bound; verified (or NULL)
+ *   1 iff lb > 0. opts [host] may be NULL (all defaults). */
+int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
+                    const vf_opts* opts, float* lb, float* ub, float* lb_ibp, uint8_t* verified, void* stream);
+
+/* Synchronise `stream` and report any pending asynchronous CUDA error. */
+int vf_sync(void* stream);
+
+/* Per-thread description of the last error (empty string if none). */
+const char* vf_last_error(void);
+
+/* Kernel timing, for benchmarks. While enabled, the library brackets each launch of
+ * the CROWN back-substitution contraction with CUDA events on the launching stream.
+ * vf_profile_read synchronises those events and returns the number of such launches,
+ * their summed device time in ms, and their summed algorithmic flops (2*M*K*N each),
+ * since the last reset. */
+int vf_profile_enable(vf_net* net, int enable);
+int vf_profile_read(vf_net* net, long long* launches, double* total_ms, double* flops, int reset);
+
+/* Number of kernel launches the library has enqueued on this handle since creation. */
+long long vf_launch_count(const vf_net* net);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VF_H */

@@ -1,0 +1,342 @@
+// Relaxation parameters, intermediate-pass bookkeeping, specification rows, concretisation
+// and the final decision: the elementwise and row-reduction kernels around the contractions.
+//
+// Page: "Scaling Neural Network Verification with Tensor Parallelism and Fully Sharded Data
+// Parallelism", technical summary §1 (prove the property for every input of the domain),
+// §2.1 (ReLU relaxation slopes from intermediate bounds; IBP as their substitute) and §3/§4.3
+// (per-neuron alpha slopes). Every row reduction here runs in a fixed order, so repeated calls
+// give bitwise-identical results.
+#include "vf_internal.cuh"
+
+namespace vf {
+
+namespace {
+
+unsigned grid_for(long long n, int threads) {
+    long long g = (n + threads - 1) / threads;
+    if (g > 148LL * 32) g = 148LL * 32;
+    return (unsigned)(g < 1 ? 1 : g);
+}
+
+#define GRID_STRIDE(i, n) \
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (n); i += (long long)gridDim.x * blockDim.x)
+
+// ReLU relaxation for l <= z <= u: inactive (u <= 0, tested first) {0, 0, 0}; active (l >= 0)
+// {1, 1, 0}; unstable: upper chord up = u / (u - l), t = -up * l; lower slope alpha clamped
+// to [0, 1], or the adaptive choice 1 if u >= -l else 0.
+__global__ void relax_params_k(const float* __restrict__ l, const float* __restrict__ u,
+                               const float* __restrict__ alpha, long long n, float4* __restrict__ P) {
+    GRID_STRIDE(i, n) {
+        const float lo_b = l[i], up_b = u[i];
+        float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (up_b <= 0.f) {
+        } else if (lo_b >= 0.f) {
+            p.x = 1.f;
+            p.y = 1.f;
+        } else {
+            const float s = up_b / (up_b - lo_b);
+            p.y = s;
+            p.z = -s * lo_b;
+            if (alpha != nullptr)
+                p.x = fminf(fmaxf(alpha[i], 0.f), 1.f);
+            else
+                p.x = (up_b >= -lo_b) ? 1.f : 0.f;
+        }
+        P[i] = p;
+    }
+}
+
+// Identity-trick start of an intermediate pass over node p (n_p neurons, rows [I; -I]):
+// the first back-substitution step through p adds +-b_p[j] to row j's constant.
+__global__ void cst_identity_bias_k(float* __restrict__ cst, long long M, PassGeom pg, const float* __restrict__ bias,
+                                    long long n_p, long long per_channel) {
+    GRID_STRIDE(m, M) {
+        const long long r = (pg.pass_m0 + m) % pg.R_pass;
+        const long long j = r % n_p;
+        const float sg = (r < n_p) ? 1.f : -1.f;
+        cst[m] += sg * bias[j / per_channel];
+    }
+}
+
+__global__ void ident_rows_k(float* __restrict__ out, long long ld, long long M, PassGeom pg, long long n_p,
+                             int accumulate) {
+    GRID_STRIDE(e, M * n_p) {
+        const long long m = e / n_p, c = e % n_p;
+        const long long r = (pg.pass_m0 + m) % pg.R_pass;
+        const float v = (c == r % n_p) ? ((r < n_p) ? 1.f : -1.f) : 0.f;
+        float* o = out + m * ld + c;
+        *o = accumulate ? (*o + v) : v;
+    }
+}
+
+// Rows +-(row j of the convolution's matrix) over the conv's input: the identity-trick first
+// step of an intermediate pass that starts at a convolution. One CTA per row.
+__global__ void conv_start_rows_k(float* __restrict__ out, long long ld, long long M, PassGeom pg,
+                                  const float* __restrict__ W, ConvGeom g, int accumulate) {
+    const long long n_p = (long long)g.co * g.ho * g.wo;
+    const long long nin = (long long)g.ci * g.h * g.w;
+    for (long long m = blockIdx.x; m < M; m += gridDim.x) {
+        float* o = out + m * ld;
+        if (!accumulate) {
+            for (long long c = threadIdx.x; c < nin; c += blockDim.x) o[c] = 0.f;
+            __syncthreads();
+        }
+        const long long r = (pg.pass_m0 + m) % pg.R_pass;
+        const long long j = r % n_p;
+        const float sg = (r < n_p) ? 1.f : -1.f;
+        const int co = (int)(j / (g.ho * g.wo));
+        const int oi = (int)((j / g.wo) % g.ho);
+        const int oj = (int)(j % g.wo);
+        const int nk = g.ci * g.k * g.k;
+        for (int e = threadIdx.x; e < nk; e += blockDim.x) {
+            const int q = e % g.k, p = (e / g.k) % g.k, ci = e / (g.k * g.k);
+            const int y = oi * g.stride - g.pad + p, x = oj * g.stride - g.pad + q;
+            if (y < 0 || y >= g.h || x < 0 || x >= g.w) continue;
+            o[((long long)ci * g.h + y) * g.w + x] += sg * W[(((long long)co * g.ci + ci) * g.k + p) * g.k + q];
+        }
+        __syncthreads();
+    }
+}
+
+__device__ __forceinline__ float block_sum256(float v, float* red) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float t = 0.f;
+    if (threadIdx.x == 0)
+        for (int i = 0; i < 8; ++i) t += red[i];
+    __syncthreads();
+    return t;
+}
+
+// out[m, :] (=, +=) relax(A[m, :]); cst[m] += relaxation constant. One CTA per row; may run
+// in place (each element is read and written by the same thread).
+__global__ void __launch_bounds__(256)
+relax_rows_k(RowRef A, Relax rx, long long M, int n, PassGeom pg, float* out, long long ld_out, int accumulate,
+             float* __restrict__ cst) {
+    __shared__ float red[8];
+    for (long long m = blockIdx.x; m < M; m += gridDim.x) {
+        const float* a = A.row(m);
+        const long long b = (pg.pass_m0 + m) / pg.R_pass;
+        float* o = out + m * ld_out;
+        float cs = 0.f;
+        for (int j = threadIdx.x; j < n; j += 256) {
+            const float x = a[j];
+            float r = x;
+            if (rx.P != nullptr) {
+                const float4 p = rx.P[b * n + j];
+                r = (x >= 0.f) ? x * p.x : x * p.y;
+                if (rx.count_const) cs = fmaf(fminf(x, 0.f), p.z, cs);
+            }
+            o[j] = accumulate ? (o[j] + r) : r;
+        }
+        if (rx.P != nullptr && rx.count_const && cst != nullptr) {
+            const float t = block_sum256(cs, red);
+            if (threadIdx.x == 0) cst[m] += t;
+        }
+    }
+}
+
+// cst[m] += A[m, :] . c_b - eps * |A[m, :]|_1 : concretisation of materialised input rows.
+__global__ void __launch_bounds__(256)
+concretize_rows_k(RowRef A, long long M, int n0, PassGeom pg, const float* __restrict__ centres, float eps,
+                  float* __restrict__ cst) {
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * 8;
+    for (long long m = blockIdx.x * 8LL + (threadIdx.x >> 5); m < M; m += warps) {
+        const float* a = A.row(m);
+        const float* c = centres + ((pg.pass_m0 + m) / pg.R_pass) * (long long)n0;
+        float s = 0.f;
+        for (int i = lane; i < n0; i += 32) s += fmaf(a[i], c[i], -eps * fabsf(a[i]));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) cst[m] += s;
+    }
+}
+
+__global__ void finish_rows_k(const float* __restrict__ cst, const float* __restrict__ part, int ntiles, long long M,
+                              float* __restrict__ out) {
+    GRID_STRIDE(m, M) {
+        float v = cst[m];
+        for (int t = 0; t < ntiles; ++t) v += part[(long long)t * M + m];
+        out[m] = v;
+    }
+}
+
+// Intermediate bounds after a pass over node p (rows [I; -I] per centre): IBP-unstable neurons
+// take l = max(l, lb_j), u = min(u, -lb_{n + j}); IBP-stable ones keep their (exact) relaxation.
+__global__ void intersect_k(float* __restrict__ l, float* __restrict__ u, const float* __restrict__ pass_out, int B,
+                            long long n) {
+    GRID_STRIDE(i, (long long)B * n) {
+        const long long b = i / n, j = i % n;
+        const float l0 = l[i], u0 = u[i];
+        if (l0 < 0.f && u0 > 0.f) {
+            l[i] = fmaxf(l0, pass_out[b * 2 * n + j]);
+            u[i] = fminf(u0, -pass_out[b * 2 * n + n + j]);
+        }
+    }
+}
+
+__global__ void spec_rows_k(const float* __restrict__ C, long long C_bstride, int BC, int R, int nL,
+                            float* __restrict__ S) {
+    GRID_STRIDE(e, (long long)BC * R * nL) {
+        const long long bc = e / ((long long)R * nL);
+        const long long rest = e % ((long long)R * nL);
+        const float v = C[bc * C_bstride + rest];
+        S[bc * 2LL * R * nL + rest] = v;
+        S[bc * 2LL * R * nL + (long long)R * nL + rest] = -v;
+    }
+}
+
+// IBP bound of the specification: C applied to the last node's interval, C c -+ |C| r.
+__global__ void __launch_bounds__(256)
+spec_ibp_k(const float* __restrict__ C, long long C_bstride, int B, int R, int nL, const float* __restrict__ zc,
+           const float* __restrict__ zr, float* __restrict__ lb, float* __restrict__ ub) {
+    const int lane = threadIdx.x & 31;
+    const long long rows = (long long)B * R;
+    for (long long w = blockIdx.x * 8LL + (threadIdx.x >> 5); w < rows; w += (long long)gridDim.x * 8) {
+        const long long b = w / R, r = w % R;
+        const float* cr = C + b * C_bstride + r * nL;
+        float sc = 0.f, sr = 0.f;
+        for (int j = lane; j < nL; j += 32) {
+            sc = fmaf(cr[j], zc[b * nL + j], sc);
+            sr = fmaf(fabsf(cr[j]), zr[b * nL + j], sr);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            sc += __shfl_xor_sync(0xffffffffu, sc, off);
+            sr += __shfl_xor_sync(0xffffffffu, sr, off);
+        }
+        if (lane == 0) {
+            lb[w] = sc - sr;
+            ub[w] = sc + sr;
+        }
+    }
+}
+
+__global__ void decide_k(const float* __restrict__ lb_ibp, const float* __restrict__ ub_ibp,
+                         const float* __restrict__ pass_out, int B, int R, int both, float* __restrict__ lb,
+                         float* __restrict__ ub, float* __restrict__ lb_ibp_out, uint8_t* __restrict__ verified) {
+    GRID_STRIDE(i, (long long)B * R) {
+        const long long b = i / R, r = i % R;
+        const long long Rp = both ? 2LL * R : (long long)R;
+        const float l = fmaxf(lb_ibp[i], pass_out[b * Rp + r]);
+        lb[i] = l;
+        if (both) ub[i] = fminf(ub_ibp[i], -pass_out[b * Rp + R + r]);
+        if (lb_ibp_out != nullptr) lb_ibp_out[i] = lb_ibp[i];
+        if (verified != nullptr) verified[i] = (l > 0.f) ? 1 : 0;
+    }
+}
+
+__global__ void finite_scan_k(const float* __restrict__ p, long long n, int* flag) {
+    GRID_STRIDE(i, n) {
+        if (!isfinite(p[i])) atomicOr(flag, 1);
+    }
+}
+
+__global__ void __launch_bounds__(256)
+concretize_api_k(const float* __restrict__ lambda, const float* __restrict__ cst, const float* __restrict__ centres,
+                 float eps, int B, int R, int n0, float* __restrict__ lb) {
+    const int lane = threadIdx.x & 31;
+    const long long rows = (long long)B * R;
+    for (long long w = blockIdx.x * 8LL + (threadIdx.x >> 5); w < rows; w += (long long)gridDim.x * 8) {
+        const float* a = lambda + w * n0;
+        const float* c = centres + (w / R) * (long long)n0;
+        float s = 0.f;
+        for (int i = lane; i < n0; i += 32) s += fmaf(a[i], c[i], -eps * fabsf(a[i]));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) lb[w] = s + (cst != nullptr ? cst[w] : 0.f);
+    }
+}
+
+unsigned rows_grid(long long rows_per_cta_units) {
+    long long g = rows_per_cta_units;
+    if (g > 148LL * 16) g = 148LL * 16;
+    return (unsigned)(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+cudaError_t launch_relax_params(const float* l, const float* u, const float* alpha, long long n, float4* P,
+                                cudaStream_t s) {
+    relax_params_k<<<grid_for(n, 256), 256, 0, s>>>(l, u, alpha, n, P);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cst_identity_bias(float* cst, long long M, PassGeom pg, const float* bias, long long n_p,
+                                     long long per_channel, cudaStream_t s) {
+    cst_identity_bias_k<<<grid_for(M, 256), 256, 0, s>>>(cst, M, pg, bias, n_p, per_channel);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ident_rows(float* out, long long ld, long long M, PassGeom pg, long long n_p, int accumulate,
+                              cudaStream_t s) {
+    ident_rows_k<<<grid_for(M * n_p, 256), 256, 0, s>>>(out, ld, M, pg, n_p, accumulate);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_conv_start_rows(float* out, long long ld, long long M, PassGeom pg, const float* W,
+                                   const ConvGeom& g, int accumulate, cudaStream_t s) {
+    conv_start_rows_k<<<rows_grid(M), 256, 0, s>>>(out, ld, M, pg, W, g, accumulate);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_relax_rows(const RowRef& A, Relax rx, long long M, int n, PassGeom pg, float* out,
+                              long long ld_out, int accumulate, float* cst, cudaStream_t s) {
+    relax_rows_k<<<rows_grid(M), 256, 0, s>>>(A, rx, M, n, pg, out, ld_out, accumulate, cst);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_concretize_rows(const RowRef& A, long long M, int n0, PassGeom pg, const float* centres, float eps,
+                                   float* cst, cudaStream_t s) {
+    concretize_rows_k<<<rows_grid((M + 7) / 8), 256, 0, s>>>(A, M, n0, pg, centres, eps, cst);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finish_rows(const float* cst, const float* part, int ntiles, long long M, float* out,
+                               cudaStream_t s) {
+    finish_rows_k<<<grid_for(M, 256), 256, 0, s>>>(cst, part, ntiles, M, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_intersect(float* l, float* u, const float* l_ibp, const float* u_ibp, const float* pass_out, int B,
+                             long long n, cudaStream_t s) {
+    (void)l_ibp;
+    (void)u_ibp;
+    intersect_k<<<grid_for((long long)B * n, 256), 256, 0, s>>>(l, u, pass_out, B, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_spec_rows(const float* C, long long C_bstride, int BC, int R, int nL, float* S, cudaStream_t s) {
+    spec_rows_k<<<grid_for((long long)BC * R * nL, 256), 256, 0, s>>>(C, C_bstride, BC, R, nL, S);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_spec_ibp(const float* C, long long C_bstride, int B, int R, int nL, const float* zc, const float* zr,
+                            float* lb, float* ub, cudaStream_t s) {
+    spec_ibp_k<<<rows_grid(((long long)B * R + 7) / 8), 256, 0, s>>>(C, C_bstride, B, R, nL, zc, zr, lb, ub);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decide(const float* lb_ibp, const float* ub_ibp, const float* pass_out, int B, int R, int both,
+                          float* lb, float* ub, float* lb_ibp_out, uint8_t* verified, cudaStream_t s) {
+    decide_k<<<grid_for((long long)B * R, 256), 256, 0, s>>>(lb_ibp, ub_ibp, pass_out, B, R, both, lb, ub, lb_ibp_out,
+                                                             verified);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finite_scan(const float* p, long long n, int* flag, cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    finite_scan_k<<<grid_for(n, 256), 256, 0, s>>>(p, n, flag);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_concretize_api(const float* lambda, const float* cst, const float* centres, float eps, int B, int R,
+                                  int n0, float* lb, cudaStream_t s) {
+    concretize_api_k<<<rows_grid(((long long)B * R + 7) / 8), 256, 0, s>>>(lambda, cst, centres, eps, B, R, n0, lb);
+    return cudaGetLastError();
+}
+
+}  // namespace vf

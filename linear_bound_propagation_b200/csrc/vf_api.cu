@@ -1,0 +1,956 @@
+// Host side of libvf.so: the C ABI declared in include/vf.h, the network handle, the workspace
+// arena and the executor that schedules the bound-propagation kernels on one stream.
+//
+// Page: "Scaling Neural Network Verification with Tensor Parallelism and Fully Sharded Data
+// Parallelism" (gist.science summary of arXiv 2606.09377), technical summary:
+//   §1   the task (a property for every input of a domain) and the A matrices that must fit one
+//        accelerator -- here they are streamed through a fixed workspace in row blocks;
+//   §2.1 CROWN needs intermediate bounds for the ReLU relaxation slopes; IBP can replace them;
+//   §3, §4.3 per-neuron alpha slopes.
+//
+// Execution of one verify call (everything enqueued on the caller's stream, no host sync
+// except the optional finiteness scan):
+//   1. IBP over every node (centre/radius form).
+//   2. For each ReLU in topological order: optionally a CROWN pass over its source with rows
+//      [I; -I] per centre (the first step through the source is the "identity trick": rows
+//      become +-W rows with no contraction), then intersection with IBP, then the relaxation
+//      parameters {lo, up, t} per neuron.
+//   3. The specification pass (rows C, or [C; -C] for both sides) back to the input.
+//   4. Decision: max(IBP, CROWN) lower bound, verified iff > 0.
+// Passes are cut into row blocks sized to the workspace; rows are independent, so blocking
+// changes nothing in any row's arithmetic.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "vf.h"
+#include "vf_internal.cuh"
+
+using namespace vf;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[1024];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+#define CU(call)                                                                                              \
+    do {                                                                                                      \
+        cudaError_t e_ = (call);                                                                              \
+        if (e_ != cudaSuccess) return fail(VF_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_));             \
+    } while (0)
+
+#define TRY(call)                       \
+    do {                                \
+        int r_ = (call);                \
+        if (r_ != VF_OK) return r_;     \
+    } while (0)
+
+struct Node {
+    int op = 0, src = -1, src2 = -1;
+    int c = 0, h = 0, w = 0;
+    long long n = 0;
+    int k = 0, stride = 1, pad = 0;
+    float* W = nullptr;
+    float* Wabs = nullptr;
+    float* b = nullptr;
+    float* pmW = nullptr;  // dense only: [W; -W], the rows of the identity-trick first step
+    int consumers = 0;
+};
+
+}  // namespace
+
+struct vf_net {
+    std::vector<Node> nodes;
+    int device = 0;
+    int num_sms = 148;
+    long long total = 0;
+    char* ws = nullptr;
+    size_t ws_bytes = 0;
+    long long launches = 0;
+    long long fail_at = 0;  // test hook: VF_TEST_FAIL_AT=<n> fails the n-th launch on the host
+    bool prof = false;
+    std::vector<cudaEvent_t> ev_free;
+    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev_used;
+    double prof_flops = 0.0;
+    long long prof_launches = 0;
+    double prof_ms = 0.0;
+};
+
+namespace {
+
+ConvGeom conv_geom(const vf_net* net, const Node& nd) {
+    const Node& s = net->nodes[nd.src];
+    ConvGeom g;
+    g.ci = s.c;
+    g.h = s.h;
+    g.w = s.w;
+    g.co = nd.c;
+    g.ho = nd.h;
+    g.wo = nd.w;
+    g.k = nd.k;
+    g.stride = nd.stride;
+    g.pad = nd.pad;
+    return g;
+}
+
+// Counts launches and turns launch errors into VF_ERR_CUDA.
+int launched(vf_net* net, cudaError_t e, const char* what) {
+    net->launches++;
+    if (e != cudaSuccess) return fail(VF_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return VF_OK;
+}
+
+// Test hook: with VF_TEST_FAIL_AT=<n> in the environment at vf_net_create, the n-th launch of
+// the handle is not issued and the call fails with VF_ERR_CUDA (host-side fault injection).
+#define LAUNCH(net, expr)                                                                           \
+    do {                                                                                            \
+        if ((net)->fail_at > 0 && (net)->launches + 1 == (net)->fail_at) {                          \
+            (net)->launches++;                                                                      \
+            return fail(VF_ERR_CUDA, "injected failure before launch %lld", (net)->launches);       \
+        }                                                                                           \
+        TRY(launched((net), (expr), #expr));                                                        \
+    } while (0)
+
+cudaEvent_t take_event(vf_net* net) {
+    if (!net->ev_free.empty()) {
+        cudaEvent_t e = net->ev_free.back();
+        net->ev_free.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+struct Arena {
+    char* base;
+    size_t cap, off = 0;
+    template <typename T>
+    T* take(size_t count) {
+        size_t o = (off + 255) & ~size_t(255);
+        size_t bytes = count * sizeof(T);
+        if (o + bytes > cap) return nullptr;
+        off = o + bytes;
+        return reinterpret_cast<T*>(base + o);
+    }
+    size_t left() const {
+        size_t o = (off + 255) & ~size_t(255);
+        return o >= cap ? 0 : cap - o;
+    }
+};
+
+// -------------------------------------------------------------------------------------------
+// Walker: back-substitutes one row block of one pass through the node graph.
+// -------------------------------------------------------------------------------------------
+enum EntryKind { E_NONE = 0, E_BUF = 1, E_VIRT = 2, E_IDENT = 3 };
+
+struct Entry {
+    int kind = E_NONE;
+    int buf = -1;  // E_BUF: pool index
+    RowRef ref{nullptr, 0, 0, kHugeRows, 0};
+    Relax rx{nullptr, 0};
+};
+
+struct Walker {
+    vf_net* net;
+    cudaStream_t s;
+    bool dry;                 // only count buffers
+    long long M;              // rows in this block
+    PassGeom pg;
+    float* cst;               // [M]
+    float* part;              // [tiles, M] partials of a fused concretisation
+    int part_tiles = 0;       // set when the fused concretisation ran
+    std::vector<float*> bufs;
+    std::vector<int> ref;
+    long long ld_buf;
+    int live = 0, max_live = 0;
+    const float* centres = nullptr;
+    float eps = 0.f;
+    float* ext_in = nullptr;  // vf_crown_backward: rows over the input go here ([M, n0], ld n0)
+    bool ext_written = false;
+    const std::vector<const float4*>* relax;  // per node: relaxation params of ReLU nodes
+    std::vector<Entry> pend;
+
+    int alloc_buf(int* out) {
+        for (size_t i = 0; i < ref.size(); ++i)
+            if (ref[i] == 0) {
+                ref[i] = 1;
+                live++;
+                max_live = std::max(max_live, live);
+                *out = (int)i;
+                return VF_OK;
+            }
+        if (dry) {
+            ref.push_back(1);
+            bufs.push_back(nullptr);
+            live++;
+            max_live = std::max(max_live, live);
+            *out = (int)ref.size() - 1;
+            return VF_OK;
+        }
+        return fail(VF_ERR_WORKSPACE, "row-block buffer pool exhausted");
+    }
+    void release(Entry& e) {
+        if (e.kind == E_BUF && --ref[e.buf] == 0) live--;
+        e = Entry();
+    }
+    RowRef local(int b) const { return RowRef{dry ? nullptr : bufs[b], 0, ld_buf, kHugeRows, 0}; }
+    Entry buf_entry(int b) const {
+        Entry e;
+        e.kind = E_BUF;
+        e.buf = b;
+        e.ref = local(b);
+        return e;
+    }
+
+    // Make pend[v] a plain (unrelaxed, unshared) buffer so contributions can be added to it.
+    int make_plain(int v, int* out) {
+        Entry& e = pend[v];
+        const long long n = net->nodes[v].n;
+        if (e.kind == E_BUF && e.rx.P == nullptr && ref[e.buf] == 1) {
+            *out = e.buf;
+            return VF_OK;
+        }
+        if (e.kind == E_BUF && ref[e.buf] == 1) {  // relax in place
+            if (!dry)
+                LAUNCH(net, launch_relax_rows(e.ref, e.rx, M, (int)n, pg, bufs[e.buf], ld_buf, 0, cst, s));
+            e.rx = Relax{nullptr, 0};
+            *out = e.buf;
+            return VF_OK;
+        }
+        int nb;
+        TRY(alloc_buf(&nb));
+        if (!dry) {
+            if (e.kind == E_IDENT)
+                LAUNCH(net, launch_ident_rows(bufs[nb], ld_buf, M, pg, n, 0, s));
+            else
+                LAUNCH(net, launch_relax_rows(e.ref, e.rx, M, (int)n, pg, bufs[nb], ld_buf, 0, cst, s));
+        }
+        release(e);
+        pend[v] = buf_entry(nb);
+        *out = nb;
+        return VF_OK;
+    }
+
+    // pend[v] += x (x is consumed).
+    int add_into(int v, Entry x) {
+        if (pend[v].kind == E_NONE) {
+            pend[v] = x;
+            return VF_OK;
+        }
+        const long long n = net->nodes[v].n;
+        int b;
+        TRY(make_plain(v, &b));
+        if (!dry) {
+            if (x.kind == E_IDENT)
+                LAUNCH(net, launch_ident_rows(bufs[b], ld_buf, M, pg, n, 1, s));
+            else
+                LAUNCH(net, launch_relax_rows(x.ref, x.rx, M, (int)n, pg, bufs[b], ld_buf, 1, cst, s));
+        }
+        release(x);
+        return VF_OK;
+    }
+
+    // Where an affine node's back-substituted rows over its source go.
+    int target(int src, float** out, long long* ld, int* mode) {
+        if (src == 0 && ext_in != nullptr && pend[0].kind == E_NONE) {
+            *out = ext_in;
+            *ld = net->nodes[0].n;
+            *mode = ext_written ? OUT_ACCUM : OUT_STORE;
+            ext_written = true;
+            return VF_OK;
+        }
+        if (pend[src].kind == E_NONE) {
+            int nb;
+            TRY(alloc_buf(&nb));
+            pend[src] = buf_entry(nb);
+            *out = dry ? nullptr : bufs[nb];
+            *ld = ld_buf;
+            *mode = OUT_STORE;
+            return VF_OK;
+        }
+        int b;
+        TRY(make_plain(src, &b));
+        *out = dry ? nullptr : bufs[b];
+        *ld = ld_buf;
+        *mode = OUT_ACCUM;
+        return VF_OK;
+    }
+
+    void prof_begin(cudaEvent_t* e0) {
+        if (net->prof && !dry) {
+            *e0 = take_event(net);
+            cudaEventRecord(*e0, s);
+        }
+    }
+    void prof_end(cudaEvent_t e0, double flops) {
+        if (net->prof && !dry) {
+            cudaEvent_t e1 = take_event(net);
+            cudaEventRecord(e1, s);
+            net->ev_used.push_back({e0, e1});
+            net->prof_flops += flops;
+        }
+    }
+
+    int process(int v) {
+        Entry e = pend[v];
+        pend[v] = Entry();
+        if (e.kind == E_NONE) return VF_OK;
+        const Node& nd = net->nodes[v];
+        switch (nd.op) {
+            case VF_INPUT: {
+                if (e.kind == E_IDENT || e.rx.P != nullptr) {
+                    pend[0] = e;
+                    int b;
+                    TRY(make_plain(0, &b));
+                    e = pend[0];
+                    pend[0] = Entry();
+                }
+                if (ext_in != nullptr) {
+                    if (!dry)
+                        LAUNCH(net, launch_relax_rows(e.ref, Relax{nullptr, 0}, M, (int)nd.n, pg, ext_in, nd.n,
+                                                      ext_written ? 1 : 0, nullptr, s));
+                    ext_written = true;
+                } else if (!dry) {
+                    LAUNCH(net, launch_concretize_rows(e.ref, M, (int)nd.n, pg, centres, eps, cst, s));
+                }
+                release(e);
+                return VF_OK;
+            }
+            case VF_RELU: {
+                if (e.kind == E_IDENT || e.rx.P != nullptr) {
+                    pend[v] = e;
+                    int b;
+                    TRY(make_plain(v, &b));
+                    e = pend[v];
+                    pend[v] = Entry();
+                }
+                e.rx = Relax{(*relax)[v], 1};
+                return add_into(nd.src, e);
+            }
+            case VF_ADD: {
+                Entry y = e;
+                y.rx.count_const = 0;
+                if (e.kind == E_BUF) ref[e.buf]++;
+                TRY(add_into(nd.src, e));
+                return add_into(nd.src2, y);
+            }
+            case VF_DENSE: {
+                const Node& sn = net->nodes[nd.src];
+                if (e.kind == E_IDENT) {
+                    if (!dry) LAUNCH(net, launch_cst_identity_bias(cst, M, pg, nd.b, nd.n, 1, s));
+                    Entry x;
+                    x.kind = E_VIRT;
+                    x.ref = RowRef{nd.pmW, 0, sn.n, 2 * nd.n, pg.pass_m0};
+                    return add_into(nd.src, x);
+                }
+                const bool fuse = (nd.src == 0 && ext_in == nullptr && net->nodes[0].consumers == 1 &&
+                                   pend[0].kind == E_NONE);
+                float* out = nullptr;
+                long long ld = 0;
+                int mode = OUT_CONCRETIZE;
+                if (!fuse) TRY(target(nd.src, &out, &ld, &mode));
+                if (fuse) part_tiles = dense_back_tiles_n((int)sn.n);
+                if (!dry) {
+                    cudaEvent_t e0 = nullptr;
+                    prof_begin(&e0);
+                    LAUNCH(net, launch_dense_back(e.ref, e.rx, nd.W, nd.b, M, (int)nd.n, (int)sn.n, pg, mode, out, ld,
+                                                  cst, centres, eps, part, s));
+                    prof_end(e0, 2.0 * (double)M * (double)nd.n * (double)sn.n);
+                }
+                release(e);
+                return VF_OK;
+            }
+            case VF_CONV2D: {
+                const ConvGeom g = conv_geom(net, nd);
+                if (e.kind == E_IDENT) {
+                    if (!dry)
+                        LAUNCH(net, launch_cst_identity_bias(cst, M, pg, nd.b, nd.n, (long long)nd.h * nd.w, s));
+                    float* out = nullptr;
+                    long long ld = 0;
+                    int mode = OUT_STORE;
+                    TRY(target(nd.src, &out, &ld, &mode));
+                    if (!dry)
+                        LAUNCH(net, launch_conv_start_rows(out, ld, M, pg, nd.W, g, mode == OUT_ACCUM ? 1 : 0, s));
+                    return VF_OK;
+                }
+                const bool fuse = (nd.src == 0 && ext_in == nullptr && net->nodes[0].consumers == 1 &&
+                                   pend[0].kind == E_NONE);
+                float* out = nullptr;
+                long long ld = 0;
+                int mode = OUT_CONCRETIZE;
+                if (!fuse) TRY(target(nd.src, &out, &ld, &mode));
+                if (!dry) {
+                    cudaEvent_t e0 = nullptr;
+                    prof_begin(&e0);
+                    LAUNCH(net, launch_conv_back(e.ref, e.rx, nd.W, nd.b, M, g, pg, mode, out, ld, cst, centres, eps,
+                                                 net->num_sms, s));
+                    prof_end(e0, 2.0 * (double)M * (double)net->nodes[nd.src].n * (double)g.co * g.k * g.k /
+                                     ((double)g.stride * g.stride));
+                }
+                release(e);
+                return VF_OK;
+            }
+        }
+        return fail(VF_ERR_ARG, "bad node kind");
+    }
+
+    // Back-substitute from node `start` whose rows are `init`, down to the input.
+    int run(int start, Entry init) {
+        pend.assign(net->nodes.size(), Entry());
+        part_tiles = 0;
+        ext_written = false;
+        live = 0;
+        for (auto& r : ref) r = 0;
+        if (!dry) CU(cudaMemsetAsync(cst, 0, sizeof(float) * M, s));
+        pend[start] = init;
+        for (int v = start; v >= 0; --v) TRY(process(v));
+        return VF_OK;
+    }
+};
+
+long long max_node_size(const vf_net* net, bool include_input) {
+    long long m = 1;
+    for (size_t v = include_input ? 0 : 1; v < net->nodes.size(); ++v) m = std::max(m, net->nodes[v].n);
+    return m;
+}
+
+// A source whose IBP bounds are already the exact range: the input itself, or one affine node
+// fed directly by the input (its interval c +- |W| eps is attained coordinate by coordinate).
+bool exact_source(const vf_net* net, int p) {
+    const Node& nd = net->nodes[p];
+    return p == 0 || ((nd.op == VF_DENSE || nd.op == VF_CONV2D) && nd.src == 0);
+}
+
+// Rows over the input are held in a buffer unless its only consumer is one affine node, whose
+// contraction then writes (or concretises) them directly.
+bool input_buffered(const vf_net* net) {
+    if (net->nodes[0].consumers != 1) return true;
+    for (size_t v = 1; v < net->nodes.size(); ++v)
+        if (net->nodes[v].src == 0 || net->nodes[v].src2 == 0)
+            return !(net->nodes[v].op == VF_DENSE || net->nodes[v].op == VF_CONV2D);
+    return true;
+}
+
+// Buffers a pass needs at once, by a dry run of the walker.
+int pool_size(vf_net* net, int start, Entry init, const std::vector<const float4*>* relax, bool ext, int* nb) {
+    Walker w;
+    w.net = net;
+    w.s = nullptr;
+    w.dry = true;
+    w.M = 1;
+    w.pg = PassGeom{0, 1};
+    w.cst = nullptr;
+    w.part = nullptr;
+    w.ld_buf = 1;
+    w.relax = relax;
+    float dummy = 0.f;
+    w.ext_in = ext ? &dummy : nullptr;
+    TRY(w.run(start, init));
+    *nb = w.max_live;
+    return VF_OK;
+}
+
+struct IbpState {
+    std::vector<float*> c, r;
+};
+
+int run_ibp(vf_net* net, const float* centres, int B, float eps, Arena& ar, IbpState& st, cudaStream_t s) {
+    const size_t N = net->nodes.size();
+    st.c.assign(N, nullptr);
+    st.r.assign(N, nullptr);
+    for (size_t v = 0; v < N; ++v) {
+        const Node& nd = net->nodes[v];
+        const long long cnt = (long long)B * nd.n;
+        if (v == 0) {
+            st.c[0] = const_cast<float*>(centres);
+            st.r[0] = ar.take<float>(cnt);
+            if (!st.r[0]) return fail(VF_ERR_WORKSPACE, "workspace too small for IBP buffers");
+            LAUNCH(net, launch_fill(st.r[0], cnt, eps, s));
+            continue;
+        }
+        st.c[v] = ar.take<float>(cnt);
+        st.r[v] = ar.take<float>(cnt);
+        if (!st.c[v] || !st.r[v]) return fail(VF_ERR_WORKSPACE, "workspace too small for IBP buffers");
+        const int sv = nd.src;
+        switch (nd.op) {
+            case VF_DENSE:
+                LAUNCH(net, launch_ibp_dense(st.c[sv], st.r[sv], nd.W, nd.Wabs, nd.b, B, (int)net->nodes[sv].n,
+                                             (int)nd.n, st.c[v], st.r[v], s));
+                break;
+            case VF_CONV2D:
+                LAUNCH(net, launch_ibp_conv(st.c[sv], st.r[sv], nd.W, nd.Wabs, nd.b, B, conv_geom(net, nd), st.c[v],
+                                            st.r[v], s));
+                break;
+            case VF_RELU:
+                LAUNCH(net, launch_ibp_relu(st.c[sv], st.r[sv], cnt, st.c[v], st.r[v], s));
+                break;
+            case VF_ADD:
+                LAUNCH(net, launch_ibp_add(st.c[sv], st.r[sv], st.c[nd.src2], st.r[nd.src2], cnt, st.c[v], st.r[v], s));
+                break;
+        }
+    }
+    return VF_OK;
+}
+
+long long offset_of(const vf_net* net, int v, int B) {
+    long long o = 0;
+    for (int u = 0; u < v; ++u) o += net->nodes[u].n;
+    return o * B;
+}
+
+int check_finite_dev(vf_net* net, const std::vector<std::pair<const float*, long long>>& arrays, Arena& ar,
+                     cudaStream_t s) {
+    int* flag = ar.take<int>(1);
+    if (!flag) return fail(VF_ERR_WORKSPACE, "workspace too small");
+    CU(cudaMemsetAsync(flag, 0, sizeof(int), s));
+    for (auto& a : arrays)
+        if (a.first != nullptr) LAUNCH(net, launch_finite_scan(a.first, a.second, flag, s));
+    int h = 0;
+    CU(cudaMemcpyAsync(&h, flag, sizeof(int), cudaMemcpyDeviceToHost, s));
+    CU(cudaStreamSynchronize(s));
+    if (h) return fail(VF_ERR_NONFINITE, "NaN or Inf in centres, C or alpha");
+    return VF_OK;
+}
+
+// Runs every row block of one pass. `init` describes the start rows (global addressing).
+int run_pass(vf_net* net, int start, Entry init, long long rows, long long R_pass, Arena& ar,
+             const std::vector<const float4*>& relax, const float* centres, float eps, float* pass_out, float* ext_in,
+             float* const_out, cudaStream_t s) {
+    const bool ext = ext_in != nullptr;
+    int nb = 0;
+    TRY(pool_size(net, start, init, &relax, ext, &nb));
+    const long long nmax = max_node_size(net, input_buffered(net));
+    const int tiles = dense_back_tiles_n((int)net->nodes[0].n);
+    Arena a2 = ar;
+    const size_t per_row = sizeof(float) * (1 + (size_t)tiles + (size_t)nb * nmax) + 64;
+    long long chunk = (long long)(a2.left() / per_row);
+    if (chunk > rows) chunk = rows;
+    if (chunk >= 256) chunk -= chunk % 128;
+    if (chunk < 1) return fail(VF_ERR_WORKSPACE, "workspace too small for one row of the pass");
+    Walker w;
+    w.net = net;
+    w.s = s;
+    w.dry = false;
+    w.cst = a2.take<float>(chunk);
+    w.part = a2.take<float>((size_t)chunk * tiles);
+    w.ld_buf = nmax;
+    w.bufs.assign(nb, nullptr);
+    w.ref.assign(nb, 0);
+    for (int i = 0; i < nb; ++i) w.bufs[i] = a2.take<float>((size_t)chunk * nmax);
+    if (!w.cst || !w.part) return fail(VF_ERR_WORKSPACE, "workspace too small");
+    for (int i = 0; i < nb; ++i)
+        if (!w.bufs[i]) return fail(VF_ERR_WORKSPACE, "workspace too small");
+    w.relax = &relax;
+    w.centres = centres;
+    w.eps = eps;
+    for (long long m0 = 0; m0 < rows; m0 += chunk) {
+        w.M = std::min(chunk, rows - m0);
+        w.pg = PassGeom{m0, R_pass};
+        Entry e = init;
+        if (e.kind == E_VIRT) e.ref.m0 = m0;
+        w.ext_in = ext ? ext_in + m0 * net->nodes[0].n : nullptr;
+        TRY(w.run(start, e));
+        if (pass_out != nullptr) LAUNCH(net, launch_finish_rows(w.cst, w.part, w.part_tiles, w.M, pass_out + m0, s));
+        if (const_out != nullptr) CU(cudaMemcpyAsync(const_out + m0, w.cst, sizeof(float) * w.M,
+                                                     cudaMemcpyDeviceToDevice, s));
+    }
+    return VF_OK;
+}
+
+int check_net(const vf_net* net) {
+    if (net == nullptr) return fail(VF_ERR_ARG, "net is NULL");
+    return VF_OK;
+}
+
+// Relaxation parameters for every ReLU from bounds arrays (vf_ibp layout) and optional alpha.
+int build_relax(vf_net* net, int B, const std::vector<const float*>& L, const std::vector<const float*>& U,
+                const float* const* alpha, Arena& ar, std::vector<const float4*>& relax, cudaStream_t s) {
+    relax.assign(net->nodes.size(), nullptr);
+    for (size_t v = 0; v < net->nodes.size(); ++v) {
+        const Node& nd = net->nodes[v];
+        if (nd.op != VF_RELU) continue;
+        float4* P = ar.take<float4>((size_t)B * nd.n);
+        if (!P) return fail(VF_ERR_WORKSPACE, "workspace too small for relaxation parameters");
+        LAUNCH(net, launch_relax_params(L[nd.src], U[nd.src], alpha ? alpha[v] : nullptr, (long long)B * nd.n, P, s));
+        relax[v] = P;
+    }
+    return VF_OK;
+}
+
+}  // namespace
+
+// ===================================== C ABI ===============================================
+
+extern "C" {
+
+const char* vf_last_error(void) { return g_err.c_str(); }
+
+int vf_sync(void* stream) {
+    CU(cudaStreamSynchronize((cudaStream_t)stream));
+    CU(cudaGetLastError());
+    return VF_OK;
+}
+
+void vf_net_destroy(vf_net* net) {
+    if (net == nullptr) return;
+    for (auto& nd : net->nodes) {
+        cudaFree(nd.W);
+        cudaFree(nd.Wabs);
+        cudaFree(nd.b);
+        cudaFree(nd.pmW);
+    }
+    for (auto e : net->ev_free) cudaEventDestroy(e);
+    for (auto& p : net->ev_used) {
+        cudaEventDestroy(p.first);
+        cudaEventDestroy(p.second);
+    }
+    cudaFree(net->ws);
+    delete net;
+}
+
+static int upload(const float* src, long long count, bool abs_copy, float** out, std::vector<float>& host) {
+    host.resize((size_t)count);
+    CU(cudaMemcpy(host.data(), src, sizeof(float) * count, cudaMemcpyDefault));
+    for (long long i = 0; i < count; ++i)
+        if (!std::isfinite(host[i])) return fail(VF_ERR_NONFINITE, "non-finite weight or bias");
+    if (abs_copy)
+        for (auto& x : host) x = std::fabs(x);
+    CU(cudaMalloc(out, sizeof(float) * count));
+    CU(cudaMemcpy(*out, host.data(), sizeof(float) * count, cudaMemcpyHostToDevice));
+    return VF_OK;
+}
+
+static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_net* net) {
+    CU(cudaGetDevice(&net->device));
+    CU(cudaDeviceGetAttribute(&net->num_sms, cudaDevAttrMultiProcessorCount, net->device));
+    if (const char* f = getenv("VF_TEST_FAIL_AT")) net->fail_at = atoll(f);
+    net->nodes.resize(n_nodes);
+    std::vector<float> host;
+    for (int v = 0; v < n_nodes; ++v) {
+        Node& nd = net->nodes[v];
+        const vf_node_desc& x = d[v];
+        nd.op = x.op;
+        if (v == 0) {
+            if (x.op != VF_INPUT) return fail(VF_ERR_ARG, "node 0 must be VF_INPUT");
+            if (x.c <= 0 || x.h <= 0 || x.w <= 0) return fail(VF_ERR_SHAPE, "bad input shape");
+            nd.c = x.c;
+            nd.h = x.h;
+            nd.w = x.w;
+            nd.n = (long long)x.c * x.h * x.w;
+            continue;
+        }
+        if (x.op == VF_INPUT) return fail(VF_ERR_ARG, "only node 0 may be VF_INPUT");
+        if (x.src < 0 || x.src >= v) return fail(VF_ERR_ARG, "node %d: src %d not an earlier node", v, x.src);
+        nd.src = x.src;
+        const Node& s = net->nodes[x.src];
+        net->nodes[x.src].consumers++;
+        switch (x.op) {
+            case VF_DENSE: {
+                if (x.n_out <= 0 || !x.W || !x.b) return fail(VF_ERR_ARG, "node %d: dense needs n_out, W, b", v);
+                nd.c = x.n_out;
+                nd.h = nd.w = 1;
+                nd.n = x.n_out;
+                const long long cnt = nd.n * s.n;
+                TRY(upload(x.W, cnt, false, &nd.W, host));
+                TRY(upload(x.W, cnt, true, &nd.Wabs, host));
+                TRY(upload(x.b, nd.n, false, &nd.b, host));
+                // [W; -W] for the first step of a pass that starts at this node
+                std::vector<float> pm((size_t)(2 * cnt));
+                CU(cudaMemcpy(pm.data(), nd.W, sizeof(float) * cnt, cudaMemcpyDeviceToHost));
+                for (long long i = 0; i < cnt; ++i) pm[cnt + i] = -pm[i];
+                CU(cudaMalloc(&nd.pmW, sizeof(float) * 2 * cnt));
+                CU(cudaMemcpy(nd.pmW, pm.data(), sizeof(float) * 2 * cnt, cudaMemcpyHostToDevice));
+                break;
+            }
+            case VF_CONV2D: {
+                if (x.n_out <= 0 || x.k <= 0 || x.stride <= 0 || x.pad < 0 || !x.W || !x.b)
+                    return fail(VF_ERR_ARG, "node %d: conv needs n_out, k, stride, pad, W, b", v);
+                const int ho = (s.h + 2 * x.pad - x.k) / x.stride + 1;
+                const int wo = (s.w + 2 * x.pad - x.k) / x.stride + 1;
+                if (ho <= 0 || wo <= 0) return fail(VF_ERR_SHAPE, "node %d: empty conv output", v);
+                nd.c = x.n_out;
+                nd.h = ho;
+                nd.w = wo;
+                nd.k = x.k;
+                nd.stride = x.stride;
+                nd.pad = x.pad;
+                nd.n = (long long)nd.c * ho * wo;
+                const long long cnt = (long long)x.n_out * s.c * x.k * x.k;
+                TRY(upload(x.W, cnt, false, &nd.W, host));
+                TRY(upload(x.W, cnt, true, &nd.Wabs, host));
+                TRY(upload(x.b, nd.c, false, &nd.b, host));
+                ConvGeom g = conv_geom(net, nd);
+                if (conv_back_smem_bytes(g) > 220 * 1024)
+                    return fail(VF_ERR_UNSUPPORTED, "node %d: convolution too large for one CTA's shared memory", v);
+                break;
+            }
+            case VF_RELU:
+                nd.c = s.c;
+                nd.h = s.h;
+                nd.w = s.w;
+                nd.n = s.n;
+                break;
+            case VF_ADD: {
+                if (x.src2 < 0 || x.src2 >= v) return fail(VF_ERR_ARG, "node %d: src2 not an earlier node", v);
+                const Node& s2 = net->nodes[x.src2];
+                if (s2.c != s.c || s2.h != s.h || s2.w != s.w) return fail(VF_ERR_SHAPE, "node %d: add shapes differ", v);
+                nd.src2 = x.src2;
+                net->nodes[x.src2].consumers++;
+                nd.c = s.c;
+                nd.h = s.h;
+                nd.w = s.w;
+                nd.n = s.n;
+                break;
+            }
+            default:
+                return fail(VF_ERR_ARG, "node %d: unknown op %d", v, x.op);
+        }
+    }
+    const int last = n_nodes - 1;
+    if (net->nodes[last].op != VF_DENSE && net->nodes[last].op != VF_CONV2D)
+        return fail(VF_ERR_UNSUPPORTED, "the last node must be dense or conv");
+    net->total = 0;
+    for (auto& nd : net->nodes) net->total += nd.n;
+    net->ws_bytes = ws_bytes ? ws_bytes : (size_t(4) << 30);
+    CU(cudaMalloc(&net->ws, net->ws_bytes));
+    return VF_OK;
+}
+
+int vf_net_create(const vf_node_desc* nodes, int n_nodes, size_t workspace_bytes, vf_net** out_net) {
+    if (!nodes || !out_net || n_nodes < 2) return fail(VF_ERR_ARG, "nodes/out_net NULL or fewer than 2 nodes");
+    *out_net = nullptr;
+    vf_net* net = new vf_net();
+    int r = create_impl(nodes, n_nodes, workspace_bytes, net);
+    if (r != VF_OK) {
+        std::string keep = g_err;
+        vf_net_destroy(net);
+        g_err = keep;
+        return r;
+    }
+    *out_net = net;
+    return VF_OK;
+}
+
+int vf_net_node_size(const vf_net* net, int v) {
+    if (!net || v < 0 || v >= (int)net->nodes.size()) return -1;
+    return (int)net->nodes[v].n;
+}
+
+long long vf_net_total_size(const vf_net* net) { return net ? net->total : -1; }
+
+long long vf_launch_count(const vf_net* net) { return net ? net->launches : -1; }
+
+int vf_ibp(vf_net* net, const float* centres, int B, float eps, float* lb_all, float* ub_all, void* stream) {
+    TRY(check_net(net));
+    if (!centres || !lb_all || !ub_all || B < 0) return fail(VF_ERR_ARG, "NULL pointer or negative B");
+    if (!std::isfinite(eps) || eps < 0.f) return fail(VF_ERR_NONFINITE, "eps must be finite and >= 0");
+    if (B == 0) return VF_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    Arena ar{net->ws, net->ws_bytes};
+    IbpState st;
+    TRY(run_ibp(net, centres, B, eps, ar, st, s));
+    for (size_t v = 0; v < net->nodes.size(); ++v) {
+        const long long off = offset_of(net, (int)v, B);
+        LAUNCH(net, launch_bounds_from_cr(st.c[v], st.r[v], (long long)B * net->nodes[v].n, lb_all + off, ub_all + off, s));
+    }
+    return VF_OK;
+}
+
+int vf_crown_backward(vf_net* net, int start_node, const float* lambda0, int R, long long lambda0_bstride,
+                      const float* lb_all, const float* ub_all, const float* const* alpha, int B, float* lambda_in,
+                      float* const_out, void* stream) {
+    TRY(check_net(net));
+    if (!lambda0 || !lb_all || !ub_all || !lambda_in || !const_out) return fail(VF_ERR_ARG, "NULL pointer");
+    if (start_node < 0 || start_node >= (int)net->nodes.size()) return fail(VF_ERR_ARG, "start_node out of range");
+    if (R < 0 || B < 0 || lambda0_bstride < 0) return fail(VF_ERR_ARG, "negative size");
+    if (B == 0 || R == 0) return VF_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    Arena ar{net->ws, net->ws_bytes};
+    const long long n0 = net->nodes[0].n;
+    const long long ns = net->nodes[start_node].n;
+    if (start_node == 0) {  // nothing to back-substitute
+        for (int b = 0; b < B; ++b)
+            CU(cudaMemcpyAsync(lambda_in + (long long)b * R * n0, lambda0 + b * lambda0_bstride,
+                               sizeof(float) * R * n0, cudaMemcpyDeviceToDevice, s));
+        CU(cudaMemsetAsync(const_out, 0, sizeof(float) * B * R, s));
+        return VF_OK;
+    }
+    std::vector<const float*> L(net->nodes.size()), U(net->nodes.size());
+    for (size_t v = 0; v < net->nodes.size(); ++v) {
+        L[v] = lb_all + offset_of(net, (int)v, B);
+        U[v] = ub_all + offset_of(net, (int)v, B);
+    }
+    std::vector<const float4*> relax;
+    TRY(build_relax(net, B, L, U, alpha, ar, relax, s));
+    Entry init;
+    init.kind = E_VIRT;
+    init.ref = RowRef{lambda0, lambda0_bstride, ns, R, 0};
+    return run_pass(net, start_node, init, (long long)B * R, R, ar, relax, nullptr, 0.f, nullptr, lambda_in, const_out,
+                    s);
+}
+
+int vf_concretize(const float* lambda, const float* cst, const float* centres, float eps, int B, int R, int n0,
+                  float* lb, void* stream) {
+    if (!lambda || !centres || !lb) return fail(VF_ERR_ARG, "NULL pointer");
+    if (B < 0 || R < 0 || n0 <= 0) return fail(VF_ERR_ARG, "bad sizes");
+    if (!std::isfinite(eps) || eps < 0.f) return fail(VF_ERR_NONFINITE, "eps must be finite and >= 0");
+    if (B == 0 || R == 0) return VF_OK;
+    CU(launch_concretize_api(lambda, cst, centres, eps, B, R, n0, lb, (cudaStream_t)stream));
+    return VF_OK;
+}
+
+int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
+                    const vf_opts* opts, float* lb, float* ub, float* lb_ibp, uint8_t* verified, void* stream) {
+    TRY(check_net(net));
+    vf_opts o{};
+    if (opts) o = *opts;
+    if (!centres || !C || !lb) return fail(VF_ERR_ARG, "centres, C and lb must not be NULL");
+    if (o.both_sides && !ub) return fail(VF_ERR_ARG, "both_sides needs ub");
+    if (B < 0 || R < 0 || C_bstride < 0) return fail(VF_ERR_ARG, "negative size");
+    if (!std::isfinite(eps) || eps < 0.f) return fail(VF_ERR_NONFINITE, "eps must be finite and >= 0");
+    if (B == 0 || R == 0) return VF_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int nn = (int)net->nodes.size();
+    const int last = nn - 1;
+    const int nL = (int)net->nodes[last].n;
+    const long long n0 = net->nodes[0].n;
+    const int BC = C_bstride > 0 ? B : 1;
+    Arena ar{net->ws, net->ws_bytes};
+
+    if (!o.skip_finite_check) {
+        std::vector<std::pair<const float*, long long>> arrs = {{centres, (long long)B * n0},
+                                                                {C, (long long)(BC - 1) * C_bstride + (long long)R * nL}};
+        if (o.alpha)
+            for (int v = 0; v < nn; ++v)
+                if (net->nodes[v].op == VF_RELU && o.alpha[v]) arrs.push_back({o.alpha[v], (long long)B * net->nodes[v].n});
+        Arena tmp = ar;
+        TRY(check_finite_dev(net, arrs, tmp, s));
+    }
+
+    IbpState st;
+    TRY(run_ibp(net, centres, B, eps, ar, st, s));
+
+    // Bounds used for every ReLU source: start from IBP, refined in place by CROWN passes.
+    std::vector<const float*> L(nn, nullptr), U(nn, nullptr);
+    std::vector<float*> Lw(nn, nullptr), Uw(nn, nullptr);
+    for (int v = 0; v < nn; ++v) {
+        if (net->nodes[v].op != VF_RELU) continue;
+        const int p = net->nodes[v].src;
+        const long long cnt = (long long)B * net->nodes[p].n;
+        Lw[p] = ar.take<float>(cnt);
+        Uw[p] = ar.take<float>(cnt);
+        if (!Lw[p] || !Uw[p]) return fail(VF_ERR_WORKSPACE, "workspace too small for intermediate bounds");
+        LAUNCH(net, launch_bounds_from_cr(st.c[p], st.r[p], cnt, Lw[p], Uw[p], s));
+        L[p] = Lw[p];
+        U[p] = Uw[p];
+    }
+    std::vector<const float4*> relax(nn, nullptr);
+    std::vector<float4*> P(nn, nullptr);
+    long long max_pass_rows = 0;
+    for (int v = 0; v < nn; ++v)
+        if (net->nodes[v].op == VF_RELU) {
+            P[v] = ar.take<float4>((size_t)B * net->nodes[v].n);
+            if (!P[v]) return fail(VF_ERR_WORKSPACE, "workspace too small for relaxation parameters");
+            relax[v] = P[v];
+            max_pass_rows = std::max(max_pass_rows, 2 * net->nodes[v].n);
+        }
+    const int Rp = o.both_sides ? 2 * R : R;
+    float* pass_out = ar.take<float>((size_t)B * std::max<long long>(max_pass_rows, Rp));
+    float* lbI = ar.take<float>((size_t)B * R);
+    float* ubI = ar.take<float>((size_t)B * R);
+    float* S = o.both_sides ? ar.take<float>((size_t)BC * Rp * nL) : nullptr;
+    if (!pass_out || !lbI || !ubI || (o.both_sides && !S)) return fail(VF_ERR_WORKSPACE, "workspace too small");
+
+    for (int k = 0; k < nn; ++k) {
+        const Node& nd = net->nodes[k];
+        if (nd.op != VF_RELU) continue;
+        const int p = nd.src;
+        const bool crown = (o.relu_crown == nullptr) || (o.relu_crown[k] != 0);
+        if (crown && !exact_source(net, p)) {
+            Entry init;
+            init.kind = E_IDENT;
+            const long long np = net->nodes[p].n;
+            TRY(run_pass(net, p, init, (long long)B * 2 * np, 2 * np, ar, relax, centres, eps, pass_out, nullptr,
+                         nullptr, s));
+            LAUNCH(net, launch_intersect(Lw[p], Uw[p], nullptr, nullptr, pass_out, B, np, s));
+        }
+        LAUNCH(net, launch_relax_params(Lw[p], Uw[p], o.alpha ? o.alpha[k] : nullptr, (long long)B * nd.n, P[k], s));
+    }
+
+    // Specification pass.
+    Entry init;
+    init.kind = E_VIRT;
+    if (o.both_sides) {
+        LAUNCH(net, launch_spec_rows(C, C_bstride, BC, R, nL, S, s));
+        init.ref = RowRef{S, BC > 1 ? (long long)Rp * nL : 0, nL, Rp, 0};
+    } else {
+        init.ref = RowRef{C, C_bstride, nL, R, 0};
+    }
+    TRY(run_pass(net, last, init, (long long)B * Rp, Rp, ar, relax, centres, eps, pass_out, nullptr, nullptr, s));
+    LAUNCH(net, launch_spec_ibp(C, C_bstride, B, R, nL, st.c[last], st.r[last], lbI, ubI, s));
+    LAUNCH(net, launch_decide(lbI, ubI, pass_out, B, R, o.both_sides, lb, ub, lb_ibp, verified, s));
+
+    if (o.pre_lb || o.pre_ub) {
+        for (int v = 0; v < nn; ++v) {
+            const long long off = offset_of(net, v, B);
+            const long long cnt = (long long)B * net->nodes[v].n;
+            if (Lw[v]) {
+                if (o.pre_lb) CU(cudaMemcpyAsync(o.pre_lb + off, Lw[v], sizeof(float) * cnt, cudaMemcpyDeviceToDevice, s));
+                if (o.pre_ub) CU(cudaMemcpyAsync(o.pre_ub + off, Uw[v], sizeof(float) * cnt, cudaMemcpyDeviceToDevice, s));
+            } else {
+                float* tl = o.pre_lb ? o.pre_lb + off : nullptr;
+                float* tu = o.pre_ub ? o.pre_ub + off : nullptr;
+                if (tl && tu) LAUNCH(net, launch_bounds_from_cr(st.c[v], st.r[v], cnt, tl, tu, s));
+            }
+        }
+    }
+    return VF_OK;
+}
+
+int vf_profile_enable(vf_net* net, int enable) {
+    TRY(check_net(net));
+    net->prof = enable != 0;
+    return VF_OK;
+}
+
+int vf_profile_read(vf_net* net, long long* launches, double* total_ms, double* flops, int reset) {
+    TRY(check_net(net));
+    for (auto& p : net->ev_used) {
+        CU(cudaEventSynchronize(p.second));
+        float ms = 0.f;
+        CU(cudaEventElapsedTime(&ms, p.first, p.second));
+        net->prof_ms += ms;
+        net->prof_launches++;
+        net->ev_free.push_back(p.first);
+        net->ev_free.push_back(p.second);
+    }
+    net->ev_used.clear();
+    if (launches) *launches = net->prof_launches;
+    if (total_ms) *total_ms = net->prof_ms;
+    if (flops) *flops = net->prof_flops;
+    if (reset) {
+        net->prof_launches = 0;
+        net->prof_ms = 0.0;
+        net->prof_flops = 0.0;
+    }
+    return VF_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+// Internal declarations shared by the CUDA kernels (k_*.cu) and the host executor (vf_api.cu).
+// Nothing here is part of the public ABI (include/vf.h).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace vf {
+
+// Read-only addressing of coefficient rows. Local row m of a launch maps to global
+// row g = m + m0, stored at ptr + (g / RA) * sB + (g % RA) * ld. A chunk-local buffer
+// uses m0 = 0, sB = 0, RA = kHugeRows; a block shared by all centres (the [W; -W] start
+// rows of an intermediate pass, or a specification matrix C with centre stride 0) uses
+// m0 = the chunk's first global row, RA = rows per centre and sB = 0 (or the C stride).
+constexpr long long kHugeRows = (1LL << 62);
+
+struct RowRef {
+    const float* ptr;
+    long long sB, ld, RA, m0;
+    __host__ __device__ __forceinline__ const float* row(long long m) const {
+        long long g = m + m0;
+        return ptr + (g / RA) * sB + (g % RA) * ld;
+    }
+};
+
+// ReLU relaxation applied to coefficients as they are loaded: P[b * n + j] holds
+// {lo, up, t, 0} for centre b and neuron j (lower slope used by coefficients >= 0,
+// upper slope and intercept used by coefficients < 0). P == nullptr: no relaxation.
+struct Relax {
+    const float4* P;
+    int count_const;  // also add sum_j min(x_j, 0) * t_j to the row constant
+};
+
+// Rows of one CROWN pass are processed in chunks; row m of a chunk is global row
+// pass_m0 + m, which belongs to centre (pass_m0 + m) / R_pass.
+struct PassGeom {
+    long long pass_m0;
+    long long R_pass;
+};
+
+enum OutMode { OUT_STORE = 0, OUT_ACCUM = 1, OUT_CONCRETIZE = 2 };
+
+struct ConvGeom {
+    int ci, h, w;     // input (source) shape
+    int co, ho, wo;   // output shape
+    int k, stride, pad;
+};
+
+// ---- contractions (k_back.cu, k_back_conv.cu) ----------------------------------------
+// out[m, :] (=, +=) relax(A[m, :]) . W  with W = the node's [K = n_out, N = n_in] weights;
+// cst[m] += sum_k (relax const) + relax(A)[m, k] * bias[k]   (when cst != nullptr);
+// OUT_CONCRETIZE: part[tile_n * M + m] = sum_{n in tile} v * c_b[n] - eps * |v|.
+int dense_back_tiles_n(int N);
+cudaError_t launch_dense_back(const RowRef& A, Relax rx, const float* W, const float* bias, long long M, int K,
+                              int N, PassGeom pg, int out_mode, float* out, long long ld_out, float* cst,
+                              const float* centres, float eps, float* part, cudaStream_t s);
+
+// Transposed convolution of relaxed rows over the conv output back onto its input.
+// cst[m] += relax const + bias term; OUT_CONCRETIZE adds the concretised row to cst[m].
+size_t conv_back_smem_bytes(const ConvGeom& g);
+cudaError_t launch_conv_back(const RowRef& A, Relax rx, const float* W, const float* bias, long long M,
+                             const ConvGeom& g, PassGeom pg, int out_mode, float* out, long long ld_out, float* cst,
+                             const float* centres, float eps, int num_sms, cudaStream_t s);
+
+// ---- IBP (k_ibp.cu) -------------------------------------------------------------------
+cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
+                             int B, int K, int N, float* zc, float* zr, cudaStream_t s);
+cudaError_t launch_ibp_conv(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
+                            int B, const ConvGeom& g, float* zc, float* zr, cudaStream_t s);
+cudaError_t launch_ibp_relu(const float* c, const float* r, long long n, float* oc, float* orad, cudaStream_t s);
+cudaError_t launch_ibp_add(const float* c1, const float* r1, const float* c2, const float* r2, long long n,
+                           float* oc, float* orad, cudaStream_t s);
+cudaError_t launch_fill(float* p, long long n, float v, cudaStream_t s);
+cudaError_t launch_bounds_from_cr(const float* c, const float* r, long long n, float* lb, float* ub, cudaStream_t s);
+
+// ---- relaxation, pass bookkeeping, decision (k_misc.cu) ------------------------------
+cudaError_t launch_relax_params(const float* l, const float* u, const float* alpha, long long n, float4* P,
+                                cudaStream_t s);
+cudaError_t launch_cst_identity_bias(float* cst, long long M, PassGeom pg, const float* bias, long long n_p,
+                                     long long per_channel, cudaStream_t s);
+cudaError_t launch_ident_rows(float* out, long long ld, long long M, PassGeom pg, long long n_p, int accumulate,
+                              cudaStream_t s);
+cudaError_t launch_conv_start_rows(float* out, long long ld, long long M, PassGeom pg, const float* W,
+                                   const ConvGeom& g, int accumulate, cudaStream_t s);
+cudaError_t launch_relax_rows(const RowRef& A, Relax rx, long long M, int n, PassGeom pg, float* out, long long ld_out,
+                              int accumulate, float* cst, cudaStream_t s);
+cudaError_t launch_concretize_rows(const RowRef& A, long long M, int n0, PassGeom pg, const float* centres, float eps,
+                                   float* cst, cudaStream_t s);
+cudaError_t launch_finish_rows(const float* cst, const float* part, int ntiles, long long M, float* out,
+                               cudaStream_t s);
+cudaError_t launch_intersect(float* l, float* u, const float* l_ibp, const float* u_ibp, const float* pass_out,
+                             int B, long long n, cudaStream_t s);
+cudaError_t launch_spec_rows(const float* C, long long C_bstride, int BC, int R, int nL, float* S, cudaStream_t s);
+cudaError_t launch_spec_ibp(const float* C, long long C_bstride, int B, int R, int nL, const float* zc, const float* zr,
+                            float* lb, float* ub, cudaStream_t s);
+cudaError_t launch_decide(const float* lb_ibp, const float* ub_ibp, const float* pass_out, int B, int R, int both,
+                          float* lb, float* ub, float* lb_ibp_out, uint8_t* verified, cudaStream_t s);
+cudaError_t launch_finite_scan(const float* p, long long n, int* flag, cudaStream_t s);
+cudaError_t launch_concretize_api(const float* lambda, const float* cst, const float* centres, float eps, int B, int R,
+                                  int n0, float* lb, cudaStream_t s);
+
+}  // namespace vf

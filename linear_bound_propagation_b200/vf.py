@@ -1,0 +1,252 @@
+"""Thin ctypes binding of libvf.so (include/vf.h): argument marshalling only.
+
+Every step of the bound computation runs in the CUDA library; this module only passes
+device pointers (``tensor.data_ptr()``), sizes and the current CUDA stream. PyTorch is
+used for device memory and streams. If the library is missing the first call raises --
+there is no other implementation behind these names.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvf.so")
+
+VF_OK, VF_ERR_ARG, VF_ERR_SHAPE, VF_ERR_WORKSPACE, VF_ERR_NONFINITE, VF_ERR_CUDA, VF_ERR_TIMEOUT, \
+    VF_ERR_UNSUPPORTED = range(8)
+VF_INPUT, VF_DENSE, VF_CONV2D, VF_RELU, VF_ADD = range(5)
+
+SYMBOLS = ["vf_net_create", "vf_net_destroy", "vf_net_node_size", "vf_net_total_size", "vf_ibp",
+           "vf_crown_backward", "vf_concretize", "vf_verify_batch", "vf_sync", "vf_last_error",
+           "vf_profile_enable", "vf_profile_read", "vf_launch_count"]
+
+
+class VfError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"vf error {code}: {msg}")
+        self.code = code
+
+
+class NodeDesc(ctypes.Structure):
+    _fields_ = [("op", ctypes.c_int), ("src", ctypes.c_int), ("src2", ctypes.c_int),
+                ("c", ctypes.c_int), ("h", ctypes.c_int), ("w", ctypes.c_int),
+                ("n_out", ctypes.c_int), ("k", ctypes.c_int), ("stride", ctypes.c_int), ("pad", ctypes.c_int),
+                ("W", ctypes.c_void_p), ("b", ctypes.c_void_p)]
+
+
+class Opts(ctypes.Structure):
+    _fields_ = [("relu_crown", ctypes.POINTER(ctypes.c_int)), ("alpha", ctypes.POINTER(ctypes.c_void_p)),
+                ("both_sides", ctypes.c_int), ("skip_finite_check", ctypes.c_int),
+                ("pre_lb", ctypes.c_void_p), ("pre_ub", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libvf.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m linear_bound_propagation_b200._build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, LL, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
+    L.vf_net_create.argtypes = [ctypes.POINTER(NodeDesc), I, ctypes.c_size_t, ctypes.POINTER(P)]
+    L.vf_net_destroy.argtypes = [P]
+    L.vf_net_destroy.restype = None
+    L.vf_net_node_size.argtypes = [P, I]
+    L.vf_net_total_size.argtypes = [P]
+    L.vf_net_total_size.restype = LL
+    L.vf_ibp.argtypes = [P, P, I, F, P, P, P]
+    L.vf_crown_backward.argtypes = [P, I, P, I, LL, P, P, ctypes.POINTER(P), I, P, P, P]
+    L.vf_concretize.argtypes = [P, P, P, F, I, I, I, P, P]
+    L.vf_verify_batch.argtypes = [P, P, I, F, P, I, LL, ctypes.POINTER(Opts), P, P, P, P, P]
+    L.vf_sync.argtypes = [P]
+    L.vf_last_error.restype = ctypes.c_char_p
+    L.vf_profile_enable.argtypes = [P, I]
+    L.vf_profile_read.argtypes = [P, ctypes.POINTER(LL), ctypes.POINTER(ctypes.c_double),
+                                  ctypes.POINTER(ctypes.c_double), I]
+    L.vf_launch_count.argtypes = [P]
+    L.vf_launch_count.restype = LL
+    _lib = L
+    return L
+
+
+def _check(code):
+    if code != VF_OK:
+        raise VfError(code, lib().vf_last_error().decode())
+
+
+def _stream_ptr(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    assert t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class Net:
+    """A network handle on the current CUDA device (vf_net_create / vf_net_destroy)."""
+
+    def __init__(self, nodes: Sequence, workspace_bytes: int = 0):
+        L = lib()
+        descs = (NodeDesc * len(nodes))()
+        keep = []
+        for v, nd in enumerate(nodes):
+            d = descs[v]
+            d.src, d.src2 = -1, -1
+            if nd.op == "input":
+                d.op = VF_INPUT
+                shp = tuple(nd.shape)
+                d.c, d.h, d.w = (shp + (1, 1))[:3] if len(shp) == 1 else shp
+            elif nd.op in ("dense", "conv"):
+                W = np.ascontiguousarray(nd.W, np.float32)
+                b = np.ascontiguousarray(nd.b, np.float32)
+                keep += [W, b]
+                d.op = VF_DENSE if nd.op == "dense" else VF_CONV2D
+                d.src = nd.src
+                d.n_out = W.shape[0]
+                if nd.op == "conv":
+                    d.k, d.stride, d.pad = W.shape[2], nd.stride, nd.pad
+                d.W = W.ctypes.data
+                d.b = b.ctypes.data
+            elif nd.op == "relu":
+                d.op, d.src = VF_RELU, nd.src
+            elif nd.op == "add":
+                d.op, d.src, d.src2 = VF_ADD, nd.src, nd.src2
+            else:
+                raise ValueError(nd.op)
+        h = ctypes.c_void_p()
+        _check(L.vf_net_create(descs, len(nodes), workspace_bytes, ctypes.byref(h)))
+        self.h = h
+        self.n_nodes = len(nodes)
+        self.sizes = [L.vf_net_node_size(h, v) for v in range(len(nodes))]
+        self.total = L.vf_net_total_size(h)
+        self.relu_ids = [v for v, nd in enumerate(nodes) if nd.op == "relu"]
+
+    def close(self):
+        if getattr(self, "h", None):
+            lib().vf_net_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def offset(self, v: int, B: int) -> int:
+        return B * sum(self.sizes[:v])
+
+    # --------------------------------------------------------------------- entry points
+    def ibp(self, centres: torch.Tensor, eps: float, stream=None):
+        B = centres.shape[0]
+        lb = torch.empty(B * self.total, device=centres.device, dtype=torch.float32)
+        ub = torch.empty_like(lb)
+        _check(lib().vf_ibp(self.h, _ptr(centres), B, float(eps), _ptr(lb), _ptr(ub), _stream_ptr(stream)))
+        return lb, ub
+
+    def node_block(self, flat: torch.Tensor, v: int, B: int) -> torch.Tensor:
+        o = self.offset(v, B)
+        return flat[o:o + B * self.sizes[v]].view(B, self.sizes[v])
+
+    def crown_backward(self, start_node: int, lambda0: torch.Tensor, lb_all, ub_all, B: int,
+                       alpha: Optional[Dict[int, torch.Tensor]] = None, stream=None):
+        R = lambda0.shape[-2]
+        bstride = 0 if lambda0.dim() == 2 or lambda0.shape[0] == 1 else R * lambda0.shape[-1]
+        lam_in = torch.empty(B, R, self.sizes[0], device=lambda0.device, dtype=torch.float32)
+        cst = torch.empty(B, R, device=lambda0.device, dtype=torch.float32)
+        arr = self._alpha_array(alpha)
+        _check(lib().vf_crown_backward(self.h, start_node, _ptr(lambda0), R, bstride, _ptr(lb_all), _ptr(ub_all),
+                                       arr, B, _ptr(lam_in), _ptr(cst), _stream_ptr(stream)))
+        return lam_in, cst
+
+    def _alpha_array(self, alpha):
+        if not alpha:
+            return None
+        arr = (ctypes.c_void_p * self.n_nodes)()
+        for v, a in alpha.items():
+            arr[v] = a.data_ptr()
+        return arr
+
+    def verify(self, centres: torch.Tensor, eps: float, C: torch.Tensor, crown_relus: Optional[Sequence[int]] = None,
+               alpha: Optional[Dict[int, torch.Tensor]] = None, both_sides: bool = False, want_pre: bool = False,
+               skip_finite_check: bool = False, stream=None, out=None):
+        """vf_verify_batch. C: [B or 1, R, n_L]. Returns dict of device tensors."""
+        B = centres.shape[0]
+        R = C.shape[1]
+        dev = centres.device
+        bstride = 0 if C.shape[0] == 1 else R * C.shape[2]
+        if out is None:
+            out = {"lb": torch.empty(B, R, device=dev), "lb_ibp": torch.empty(B, R, device=dev),
+                   "verified": torch.empty(B, R, device=dev, dtype=torch.uint8)}
+            if both_sides:
+                out["ub"] = torch.empty(B, R, device=dev)
+            if want_pre:
+                out["pre_lb"] = torch.empty(B * self.total, device=dev)
+                out["pre_ub"] = torch.empty(B * self.total, device=dev)
+        o = Opts()
+        keep = []
+        if crown_relus is not None:
+            flags = (ctypes.c_int * self.n_nodes)()
+            for v in crown_relus:
+                flags[v] = 1
+            o.relu_crown = ctypes.cast(flags, ctypes.POINTER(ctypes.c_int))
+            keep.append(flags)
+        arr = self._alpha_array(alpha)
+        if arr is not None:
+            o.alpha = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+            keep.append(arr)
+        o.both_sides = 1 if both_sides else 0
+        o.skip_finite_check = 1 if skip_finite_check else 0
+        o.pre_lb = out["pre_lb"].data_ptr() if "pre_lb" in out else None
+        o.pre_ub = out["pre_ub"].data_ptr() if "pre_ub" in out else None
+        _check(lib().vf_verify_batch(self.h, _ptr(centres), B, float(eps), _ptr(C), R, bstride, ctypes.byref(o),
+                                     _ptr(out["lb"]), _ptr(out.get("ub")), _ptr(out.get("lb_ibp")),
+                                     _ptr(out.get("verified")), _stream_ptr(stream)))
+        return out
+
+    def profile(self, enable: bool):
+        _check(lib().vf_profile_enable(self.h, 1 if enable else 0))
+
+    def profile_read(self, reset: bool = True):
+        n = ctypes.c_longlong()
+        ms = ctypes.c_double()
+        fl = ctypes.c_double()
+        _check(lib().vf_profile_read(self.h, ctypes.byref(n), ctypes.byref(ms), ctypes.byref(fl), 1 if reset else 0))
+        return n.value, ms.value, fl.value
+
+    def launch_count(self) -> int:
+        return lib().vf_launch_count(self.h)
+
+
+def concretize(lam: torch.Tensor, cst: Optional[torch.Tensor], centres: torch.Tensor, eps: float, stream=None):
+    B, R, n0 = lam.shape
+    lb = torch.empty(B, R, device=lam.device)
+    _check(lib().vf_concretize(_ptr(lam), _ptr(cst), _ptr(centres), float(eps), B, R, n0, _ptr(lb),
+                               _stream_ptr(stream)))
+    return lb
+
+
+def sync(stream=None):
+    _check(lib().vf_sync(_stream_ptr(stream)))
+
+
+def verify_host(net: Net, centres_host: torch.Tensor, eps: float, C_host: torch.Tensor, **kw):
+    """End-to-end call with host inputs: copies centres and C to the device (from pinned host
+    memory when given), runs vf_verify_batch, and copies lb and verified back to the host."""
+    dev = torch.device("cuda")
+    centres = centres_host.to(dev, non_blocking=True)
+    C = C_host.to(dev, non_blocking=True)
+    out = net.verify(centres, eps, C, **kw)
+    return {k: v.to("cpu") for k, v in out.items() if k in ("lb", "ub", "verified")}

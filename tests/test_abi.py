@@ -1,0 +1,41 @@
+"""The C ABI library loads on a machine without a GPU and exports every entry point that
+include/vf.h declares (no compute calls here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+from linear_bound_propagation_b200 import _build, vf
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "vf.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vf_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_builds_and_loads():
+    path = _build.build()
+    assert os.path.exists(path)
+    ctypes.CDLL(path)
+
+
+def test_every_declared_symbol_is_exported():
+    path = _build.build()
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (vf_\w+)$", out, flags=re.M))
+    decl = declared_symbols()
+    assert decl, "no declarations parsed"
+    missing = [s for s in decl if s not in exported]
+    assert not missing, missing
+    assert set(vf.SYMBOLS) <= set(decl)
+    L = vf.lib()
+    for s in decl:
+        assert hasattr(L, s)
+
+
+def test_last_error_without_gpu_call():
+    L = vf.lib()
+    assert isinstance(L.vf_last_error(), bytes)

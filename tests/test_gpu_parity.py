@@ -1,0 +1,197 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on seeded inputs.
+
+Sizes are chosen so that the oracle finishes in seconds while the GPU kernels still see
+several tiles and ragged tails (row counts and widths that are not multiples of the tiles).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.lbp as O
+from linear_bound_propagation_b200 import synth
+from tests._parity import ambiguous_centres, max_violation, sound_on_samples
+
+pytestmark = pytest.mark.gpu
+
+vf = pytest.importorskip("linear_bound_propagation_b200.vf")
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def run_both(net, centres, eps, C, crown_relus=None, alphas=None, both=False, workspace=0):
+    ora = O.verify(net, centres, eps, C, crown_relus=crown_relus, alphas=alphas, both_sides=both)
+    g = vf.Net(net, workspace_bytes=workspace)
+    a_dev = {k: _dev(v.astype(np.float32)) for k, v in (alphas or {}).items()} or None
+    out = g.verify(_dev(centres), eps, _dev(C), crown_relus=crown_relus, alpha=a_dev, both_sides=both, want_pre=True)
+    torch.cuda.synchronize()
+    out = {k: v.cpu().numpy() for k, v in out.items()}
+    return g, ora, out
+
+
+def _row_violation(gpu, ora):
+    """Per-centre max of |gpu - oracle| / tol."""
+    gpu = np.asarray(gpu, np.float64).reshape(gpu.shape[0], -1)
+    ora = np.asarray(ora, np.float64).reshape(ora.shape[0], -1)
+    return np.max(np.abs(gpu - ora) / (1e-4 * (np.abs(ora) + 1.0)), axis=1)
+
+
+def assert_parity(net, centres, eps, C, g, ora, out, alphas=None, both=False):
+    """Element-wise parity on every centre; a centre may differ only if the oracle's bounds put an
+    adaptive-slope decision within rounding of its tie, and then its bounds must still be sound."""
+    amb = ambiguous_centres(ora, net, alphas)
+    B = centres.shape[0]
+    bad = _row_violation(out["lb"], ora.lb) > 1.0
+    assert max_violation(out["lb_ibp"], ora.lb_ibp) <= 1.0
+    if both:
+        bad |= _row_violation(out["ub"], ora.ub) > 1.0
+    for k in [v for v, nd in enumerate(net) if nd.op == "relu"]:
+        p = net[k].src
+        gl = g.node_block(torch.from_numpy(out["pre_lb"]), p, B).numpy()
+        gu = g.node_block(torch.from_numpy(out["pre_ub"]), p, B).numpy()
+        bad |= _row_violation(gl, ora.pre_bounds[k][0]) > 1.0
+        bad |= _row_violation(gu, ora.pre_bounds[k][1]) > 1.0
+    assert not np.any(bad & ~amb), f"parity violated on centres {np.nonzero(bad & ~amb)[0]}"
+    assert (bad & amb).sum() <= max(1, B // 4), f"too many tie-ambiguous centres differ: {(bad & amb).sum()}"
+    ok = ~bad
+    clear = ok[:, None] & (np.abs(ora.lb) > 1e-4 * (np.abs(ora.lb) + 1))
+    assert np.array_equal(out["verified"][clear].astype(bool), ora.verified[clear])
+    if bad.any():
+        assert sound_on_samples(net, centres[bad], eps, C[bad] if C.shape[0] > 1 else C, out["lb"][bad],
+                                out.get("ub")[bad] if both else None)
+
+
+def test_cfg1_full():
+    w = synth.workload(1)
+    g, ora, out = run_both(w.net, w.centres, w.eps, w.C, both=True)
+    assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out, both=True)
+
+
+def test_cfg2_subset_ragged():
+    w = synth.workload(2, B=19)
+    g, ora, out = run_both(w.net, w.centres, w.eps, w.C)
+    assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out)
+
+
+def test_cfg3_subset():
+    w = synth.workload(3, B=3)
+    g, ora, out = run_both(w.net, w.centres, w.eps, w.C)
+    assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out)
+
+
+def test_resnet_small_all_paths():
+    rng = np.random.default_rng(41)
+    net = synth.resnet_cfg4(rng, image=(3, 12, 12), widths=(5, 6, 7), fc=20, classes=7)
+    centres = rng.random((3, 3 * 12 * 12)).astype(np.float32)
+    C = synth.margin_spec(rng.integers(0, 7, 3), 7)
+    g, ora, out = run_both(net, centres, np.float32(0.01).item(), C, both=True)
+    assert_parity(net, centres, 0.01, C, g, ora, out, both=True)
+
+
+@pytest.mark.parametrize("eps", [0.5 / 255, 1.0 / 255, 2.0 / 255])
+def test_cfg5_subset_each_eps(eps):
+    w = synth.workload(5, B=2, eps=eps)
+    g, ora, out = run_both(w.net, w.centres, w.eps, w.C, crown_relus=w.crown_relus)
+    assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out)
+
+
+def test_odd_mlp_given_alpha_and_chunking_is_bitwise_stable():
+    rng = np.random.default_rng(7)
+    net = synth.mlp([13, 37, 29, 33, 7], rng)
+    B = 5
+    centres = rng.random((B, 13)).astype(np.float32)
+    C = synth.margin_spec(rng.integers(0, 7, B), 7)
+    relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
+    alphas = {relus[1]: rng.random((B, 29)) * 1.4 - 0.2}
+    g, ora, out = run_both(net, centres, 0.08, C, alphas=alphas, both=True)
+    assert_parity(net, centres, 0.08, C, g, ora, out, alphas=alphas, both=True)
+    # a workspace so small that every pass runs in many row blocks: bitwise identical
+    g2, _, out2 = run_both(net, centres, 0.08, C, alphas=alphas, both=True, workspace=300_000)
+    for k in ("lb", "ub", "pre_lb", "pre_ub"):
+        assert np.array_equal(out[k], out2[k]), k
+    # repeated call on the same handle: bitwise identical
+    a_dev = {k: _dev(v.astype(np.float32)) for k, v in alphas.items()}
+    o3 = g.verify(_dev(centres), 0.08, _dev(C), alpha=a_dev, both_sides=True)
+    assert np.array_equal(o3["lb"].cpu().numpy(), out["lb"])
+
+
+def test_ibp_entry_point():
+    w = synth.workload(3, B=4)
+    g = vf.Net(w.net)
+    lb, ub = g.ibp(_dev(w.centres), w.eps)
+    torch.cuda.synchronize()
+    ib = O.ibp(w.net, w.centres, w.eps)
+    for v in range(len(w.net)):
+        gl = g.node_block(lb, v, 4).cpu().numpy()
+        gu = g.node_block(ub, v, 4).cpu().numpy()
+        assert max_violation(gl, ib[0][v] - ib[1][v]) <= 1.0, v
+        assert max_violation(gu, ib[0][v] + ib[1][v]) <= 1.0, v
+
+
+def test_crown_backward_and_concretize_entry_points():
+    w = synth.workload(2, B=6)
+    g = vf.Net(w.net)
+    cen = _dev(w.centres)
+    lb, ub = g.ibp(cen, w.eps)
+    last = len(w.net) - 1
+    lam_in, cst = g.crown_backward(last, _dev(w.C), lb, ub, 6)
+    lbc = vf.concretize(lam_in, cst, cen, w.eps)
+    torch.cuda.synchronize()
+    ib = O.ibp(w.net, w.centres, w.eps)
+    for b in range(6):
+        relax = {k: O.relax_params(ib[0][w.net[k].src][b] - ib[1][w.net[k].src][b],
+                                   ib[0][w.net[k].src][b] + ib[1][w.net[k].src][b])
+                 for k, nd in enumerate(w.net) if nd.op == "relu"}
+        L, c = O.backward(w.net, last, w.C[b].astype(np.float64), relax)
+        assert max_violation(lam_in[b].cpu().numpy(), L) <= 1.0
+        assert max_violation(cst[b].cpu().numpy(), c) <= 1.0
+        assert max_violation(lbc[b].cpu().numpy(), O.concretize(L, c, w.centres[b], w.eps)) <= 1.0
+
+
+def test_concretize_ragged_sizes():
+    rng = np.random.default_rng(3)
+    for (B, R, n0) in [(1, 1, 1), (3, 5, 33), (2, 7, 1000)]:
+        lam = rng.standard_normal((B, R, n0)).astype(np.float32)
+        cst = rng.standard_normal((B, R)).astype(np.float32)
+        c = rng.random((B, n0)).astype(np.float32)
+        got = vf.concretize(_dev(lam), _dev(cst), _dev(c), 0.1).cpu().numpy()
+        ref = np.stack([O.concretize(lam[b].astype(np.float64), cst[b], c[b], np.float32(0.1).item()) for b in range(B)])
+        assert max_violation(got, ref) <= 1.0
+
+
+def test_errors_are_codes_not_faults():
+    w = synth.workload(1, B=4)
+    g = vf.Net(w.net)
+    bad = w.centres.copy()
+    bad[1, 2] = np.nan
+    with pytest.raises(vf.VfError) as e:
+        g.verify(_dev(bad), w.eps, _dev(w.C))
+    assert e.value.code == vf.VF_ERR_NONFINITE
+    with pytest.raises(vf.VfError) as e:
+        g.verify(_dev(w.centres), float("nan"), _dev(w.C))
+    assert e.value.code == vf.VF_ERR_NONFINITE
+    tiny = vf.Net(w.net, workspace_bytes=4096)
+    with pytest.raises(vf.VfError) as e:
+        tiny.verify(_dev(w.centres), w.eps, _dev(w.C))
+    assert e.value.code == vf.VF_ERR_WORKSPACE
+    # the handle still works after errors
+    out = g.verify(_dev(w.centres), w.eps, _dev(w.C))
+    torch.cuda.synchronize()
+    assert torch.isfinite(out["lb"]).all()
+
+
+def test_host_fault_injection(monkeypatch):
+    w = synth.workload(2, B=3)
+    monkeypatch.setenv("VF_TEST_FAIL_AT", "5")
+    g = vf.Net(w.net)
+    with pytest.raises(vf.VfError) as e:
+        g.verify(_dev(w.centres), w.eps, _dev(w.C))
+    assert e.value.code == vf.VF_ERR_CUDA and "injected" in str(e.value)
+    monkeypatch.delenv("VF_TEST_FAIL_AT")
+    g2 = vf.Net(w.net)
+    out = g2.verify(_dev(w.centres), w.eps, _dev(w.C))
+    vf.sync()
+    assert torch.isfinite(out["lb"]).all()
