@@ -42,7 +42,7 @@ typedef enum {
     VF_ERR_WORKSPACE = 3,   /* the workspace given to vf_net_create is too small for this call */
     VF_ERR_NONFINITE = 4,   /* NaN/Inf in eps, centres, C, weights or alpha */
     VF_ERR_CUDA = 5,        /* a CUDA runtime call or kernel failed */
-    VF_ERR_TIMEOUT = 6,     /* reserved: a bounded device wait gave up */
+    VF_ERR_TIMEOUT = 6,     /* a kernel gave up a bounded device wait (see vf_net_check) */
     VF_ERR_UNSUPPORTED = 7  /* valid request outside what this build implements */
 } vf_status;
 
@@ -137,6 +137,11 @@ int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const f
 
 /* Synchronise `stream` and report any pending asynchronous CUDA error. */
 int vf_sync(void* stream);
+
+/* Device-wide synchronising check of the handle's kernels: VF_ERR_TIMEOUT if any kernel launched
+ * for `net` gave up a bounded wait (tensor-core pipeline barriers) since the last check, in which
+ * case that call's outputs are not valid; clears the flag. */
+int vf_net_check(vf_net* net);
 
 /* Per-thread description of the last error (empty string if none). */
 const char* vf_last_error(void);

@@ -32,6 +32,7 @@
 
 #include "vf.h"
 #include "vf_internal.cuh"
+#include "vf_tc.cuh"
 
 using namespace vf;
 
@@ -70,6 +71,8 @@ struct Node {
     float* Wabs = nullptr;
     float* b = nullptr;
     float* pmW = nullptr;  // dense only: [W; -W], the rows of the identity-trick first step
+    float* WtHi = nullptr; // dense only: W^T [n_in, n_out] truncated to tf32 (3xTF32 head)
+    float* WtLo = nullptr; // dense only: W^T - WtHi (3xTF32 remainder)
     int consumers = 0;
 };
 
@@ -84,6 +87,8 @@ struct vf_net {
     size_t ws_bytes = 0;
     long long launches = 0;
     long long fail_at = 0;  // test hook: VF_TEST_FAIL_AT=<n> fails the n-th launch on the host
+    int dense_kernel = 0;   // 0: tensor cores where the shapes allow, 1: FFMA only (VF_DENSE_KERNEL=ffma)
+    int* d_err = nullptr;   // device flag raised by a kernel whose bounded wait expired
     bool prof = false;
     std::vector<cudaEvent_t> ev_free;
     std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev_used;
@@ -366,12 +371,18 @@ struct Walker {
                 long long ld = 0;
                 int mode = OUT_CONCRETIZE;
                 if (!fuse) TRY(target(nd.src, &out, &ld, &mode));
-                if (fuse) part_tiles = dense_back_tiles_n((int)sn.n);
+                const bool tc = net->dense_kernel == 0 && nd.WtHi != nullptr &&
+                                dense_back_tc_supported(e.ref, M, (int)nd.n, (int)sn.n, pg);
+                if (fuse) part_tiles = tc ? dense_back_tc_tiles_n((int)sn.n) : dense_back_tiles_n((int)sn.n);
                 if (!dry) {
                     cudaEvent_t e0 = nullptr;
                     prof_begin(&e0);
-                    LAUNCH(net, launch_dense_back(e.ref, e.rx, nd.W, nd.b, M, (int)nd.n, (int)sn.n, pg, mode, out, ld,
-                                                  cst, centres, eps, part, s));
+                    if (tc)
+                        LAUNCH(net, launch_dense_back_tc(e.ref, e.rx, nd.WtHi, nd.WtLo, nd.b, M, (int)nd.n, (int)sn.n, pg,
+                                                         mode, out, ld, cst, centres, eps, part, net->d_err, s));
+                    else
+                        LAUNCH(net, launch_dense_back(e.ref, e.rx, nd.W, nd.b, M, (int)nd.n, (int)sn.n, pg, mode, out,
+                                                      ld, cst, centres, eps, part, s));
                     prof_end(e0, 2.0 * (double)M * (double)nd.n * (double)sn.n);
                 }
                 release(e);
@@ -536,8 +547,8 @@ int run_pass(vf_net* net, int start, Entry init, long long rows, long long R_pas
     const bool ext = ext_in != nullptr;
     int nb = 0;
     TRY(pool_size(net, start, init, &relax, ext, &nb));
-    const long long nmax = max_node_size(net, input_buffered(net));
-    const int tiles = dense_back_tiles_n((int)net->nodes[0].n);
+    const long long nmax = (max_node_size(net, input_buffered(net)) + 31) / 32 * 32;  // 128-byte rows
+    const int tiles = std::max(dense_back_tiles_n((int)net->nodes[0].n), dense_back_tc_tiles_n((int)net->nodes[0].n));
     Arena a2 = ar;
     const size_t per_row = sizeof(float) * (1 + (size_t)tiles + (size_t)nb * nmax) + 64;
     long long chunk = (long long)(a2.left() / per_row);
@@ -608,6 +619,17 @@ int vf_sync(void* stream) {
     return VF_OK;
 }
 
+int vf_net_check(vf_net* net) {
+    if (net == nullptr) return fail(VF_ERR_ARG, "net is NULL");
+    int h = 0;
+    CU(cudaMemcpy(&h, net->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+    if (h) {
+        CU(cudaMemset(net->d_err, 0, sizeof(int)));
+        return fail(VF_ERR_TIMEOUT, "a kernel's bounded wait expired; its results were discarded");
+    }
+    return VF_OK;
+}
+
 void vf_net_destroy(vf_net* net) {
     if (net == nullptr) return;
     for (auto& nd : net->nodes) {
@@ -615,7 +637,10 @@ void vf_net_destroy(vf_net* net) {
         cudaFree(nd.Wabs);
         cudaFree(nd.b);
         cudaFree(nd.pmW);
+        cudaFree(nd.WtHi);
+        cudaFree(nd.WtLo);
     }
+    cudaFree(net->d_err);
     for (auto e : net->ev_free) cudaEventDestroy(e);
     for (auto& p : net->ev_used) {
         cudaEventDestroy(p.first);
@@ -641,6 +666,9 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
     CU(cudaGetDevice(&net->device));
     CU(cudaDeviceGetAttribute(&net->num_sms, cudaDevAttrMultiProcessorCount, net->device));
     if (const char* f = getenv("VF_TEST_FAIL_AT")) net->fail_at = atoll(f);
+    if (const char* f = getenv("VF_DENSE_KERNEL")) net->dense_kernel = (strcmp(f, "ffma") == 0) ? 1 : 0;
+    CU(cudaMalloc(&net->d_err, sizeof(int)));
+    CU(cudaMemset(net->d_err, 0, sizeof(int)));
     net->nodes.resize(n_nodes);
     std::vector<float> host;
     for (int v = 0; v < n_nodes; ++v) {
@@ -677,6 +705,27 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
                 for (long long i = 0; i < cnt; ++i) pm[cnt + i] = -pm[i];
                 CU(cudaMalloc(&nd.pmW, sizeof(float) * 2 * cnt));
                 CU(cudaMemcpy(nd.pmW, pm.data(), sizeof(float) * 2 * cnt, cudaMemcpyHostToDevice));
+                if (nd.n % 4 == 0) {  // TMA rows of W^T need a 16-byte stride
+                    // 3xTF32 split of W^T: head = fp32 with the 13 low mantissa bits cleared (exact tf32),
+                    // remainder = W - head (exact in fp32).
+                    const long long nin = s.n, nout = nd.n;
+                    std::vector<float> hi((size_t)cnt), lo((size_t)cnt);
+                    for (long long o = 0; o < nout; ++o)
+                        for (long long i = 0; i < nin; ++i) {
+                            const float wv = pm[o * nin + i];
+                            uint32_t bits;
+                            std::memcpy(&bits, &wv, 4);
+                            bits &= 0xFFFFE000u;
+                            float h;
+                            std::memcpy(&h, &bits, 4);
+                            hi[i * nout + o] = h;
+                            lo[i * nout + o] = wv - h;
+                        }
+                    CU(cudaMalloc(&nd.WtHi, sizeof(float) * cnt));
+                    CU(cudaMalloc(&nd.WtLo, sizeof(float) * cnt));
+                    CU(cudaMemcpy(nd.WtHi, hi.data(), sizeof(float) * cnt, cudaMemcpyHostToDevice));
+                    CU(cudaMemcpy(nd.WtLo, lo.data(), sizeof(float) * cnt, cudaMemcpyHostToDevice));
+                }
                 break;
             }
             case VF_CONV2D: {

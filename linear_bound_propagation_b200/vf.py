@@ -23,7 +23,7 @@ VF_INPUT, VF_DENSE, VF_CONV2D, VF_RELU, VF_ADD = range(5)
 
 SYMBOLS = ["vf_net_create", "vf_net_destroy", "vf_net_node_size", "vf_net_total_size", "vf_ibp",
            "vf_crown_backward", "vf_concretize", "vf_verify_batch", "vf_sync", "vf_last_error",
-           "vf_profile_enable", "vf_profile_read", "vf_launch_count"]
+           "vf_profile_enable", "vf_profile_read", "vf_launch_count", "vf_net_check"]
 
 
 class VfError(RuntimeError):
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
     L.vf_profile_enable.argtypes = [P, I]
     L.vf_profile_read.argtypes = [P, ctypes.POINTER(LL), ctypes.POINTER(ctypes.c_double),
                                   ctypes.POINTER(ctypes.c_double), I]
+    L.vf_net_check.argtypes = [P]
     L.vf_launch_count.argtypes = [P]
     L.vf_launch_count.restype = LL
     _lib = L
@@ -225,6 +226,10 @@ class Net:
         fl = ctypes.c_double()
         _check(lib().vf_profile_read(self.h, ctypes.byref(n), ctypes.byref(ms), ctypes.byref(fl), 1 if reset else 0))
         return n.value, ms.value, fl.value
+
+    def check(self):
+        """Synchronise and raise if a kernel of this handle gave up a bounded wait."""
+        _check(lib().vf_net_check(self.h))
 
     def launch_count(self) -> int:
         return lib().vf_launch_count(self.h)

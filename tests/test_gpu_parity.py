@@ -28,6 +28,7 @@ def run_both(net, centres, eps, C, crown_relus=None, alphas=None, both=False, wo
     a_dev = {k: _dev(v.astype(np.float32)) for k, v in (alphas or {}).items()} or None
     out = g.verify(_dev(centres), eps, _dev(C), crown_relus=crown_relus, alpha=a_dev, both_sides=both, want_pre=True)
     torch.cuda.synchronize()
+    g.check()
     out = {k: v.cpu().numpy() for k, v in out.items()}
     return g, ora, out
 
@@ -96,6 +97,27 @@ def test_cfg5_subset_each_eps(eps):
     w = synth.workload(5, B=2, eps=eps)
     g, ora, out = run_both(w.net, w.centres, w.eps, w.C, crown_relus=w.crown_relus)
     assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out)
+
+
+@pytest.mark.parametrize("kernel", ["tc", "ffma"])
+def test_cfg2_both_dense_kernels(monkeypatch, kernel):
+    """The tensor-core (3xTF32) and FFMA contractions each match the oracle on the bench network."""
+    monkeypatch.setenv("VF_DENSE_KERNEL", kernel)
+    w = synth.workload(2, B=11)
+    g, ora, out = run_both(w.net, w.centres, w.eps, w.C, both=True)
+    assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out, both=True)
+
+
+def test_tc_path_wide_mlp_shapes(monkeypatch):
+    """Shapes that hit the tensor-core tiling edge cases: K not a multiple of 32, N not a multiple
+    of the N tile, N below 16 (falls back), several N tiles with concretisation partials."""
+    rng = np.random.default_rng(11)
+    net = synth.mlp([300, 196, 68, 260, 36, 12], rng)
+    B = 3
+    centres = rng.random((B, 300)).astype(np.float32)
+    C = synth.margin_spec(rng.integers(0, 12, B), 12)
+    g, ora, out = run_both(net, centres, 0.02, C, both=True)
+    assert_parity(net, centres, 0.02, C, g, ora, out, both=True)
 
 
 def test_odd_mlp_given_alpha_and_chunking_is_bitwise_stable():
