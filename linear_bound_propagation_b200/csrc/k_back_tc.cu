@@ -16,14 +16,22 @@
 // network creation. Three MMAs accumulate r_hi W_hi + r_hi W_lo + r_lo W_hi in fp32, which
 // leaves an error near 2^-21 relative per product instead of tf32's 2^-11.
 //
-// Roles in a CTA of 6 warps (one 128-row x BN-column output tile):
-//   warp 0: TMA producer (raw A tile, W_hi and W_lo tiles) and TMEM allocator;
-//   warp 1: one thread issues the MMAs and commits them to mbarriers;
-//   warps 2-5: one thread per row -- relax + split A into the swizzled smem operand layout, keep
-//              the row constant, then read the accumulator from TMEM and write the epilogue.
-// All waits are bounded: on expiry a shared abort flag stops every role, the producer waits (also
-// bounded) for its copies in flight, TMEM is freed and the kernel reports through *err.
+// Roles in a CTA of 6 warps (one 128-row x BN-column output tile, BN <= 256):
+//   warp 0: TMA producer and TMEM allocator. Two smem rings: raw A tiles (128 x 32 fp32, 128-byte
+//           swizzle) together with the relaxation table slice of the tile's centres, and the
+//           W^T head/remainder tiles (BN x 32 each);
+//   warp 1: one thread issues kind::tf32 MMAs with A read from TMEM and B from smem, committing
+//           each k-block to the barriers that release its A and B stages;
+//   warps 2-5: one thread per tile row (= TMEM lane): relax the row's 32 coefficients of the
+//           k-block, keep the row constant, split into head/remainder and store both into a TMEM
+//           A stage (4 stages of 64 columns); afterwards read the accumulator (TMEM columns
+//           0..BN-1) and write the epilogue, staged through smem so global stores are coalesced.
+// TMEM: 512 columns per CTA (one CTA per SM). All waits are bounded: on expiry a shared abort
+// flag stops every role, the producer waits (also bounded) for its copies in flight, the MMA
+// thread for its MMAs, TMEM is freed and the kernel reports through *err.
 #include <cuda.h>
+
+#include <algorithm>
 
 #include "vf_internal.cuh"
 #include "vf_tc.cuh"
@@ -92,15 +100,6 @@ __device__ __forceinline__ uint32_t idesc_tf32(int n) {
     return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc)
-        : "memory");
-}
-
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
@@ -124,13 +123,46 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+        "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
 __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
+
+constexpr int MAX_STAGES = 6;
+constexpr int A_STAGES = 4;          // TMEM stages of the split A operand (64 columns each)
+constexpr uint32_t TMEM_COLS = 512;  // accumulator in [0, 256), A stages in [256, 512)
 
 struct TcParams {
     long long M;
-    int K, N, BN, n_stages, ntiles_n;
-    int a_row_mode;        // 0: local rows y = m; 1: shared block y = (m0 + m) % RA
-    long long a_m0, a_RA;  // for mode 1
+    int K, N, BN, ntiles_n;
+    int b_stages, r_stages, nbp;  // B ring depth, raw-A ring depth, centres per P box
+    int b_off, r_off, p_off;      // byte offsets of the rings in dynamic smem
+    int a_row_mode;               // 0: local rows y = m; 1: shared block y = (m0 + m) % RA
+    long long a_m0, a_RA;
+    long long B;                  // number of centres (rows of P)
     PassGeom pg;
     int out_mode;
     float* out;
@@ -139,42 +171,49 @@ struct TcParams {
     const float* centres;
     float eps;
     float* part;
-    const float* bias;
-    Relax rx;
+    int count_const;
     int* err;
 };
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmBhi,
-              const __grid_constant__ CUtensorMap tmBlo, TcParams p) {
+dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmP,
+              const __grid_constant__ CUtensorMap tmBhi, const __grid_constant__ CUtensorMap tmBlo, TcParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // 1024-byte aligned carve-up: per stage [A (raw, then hi in place) | A_lo | B_hi | B_lo]
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int bbytes = p.BN * BK * 4;
-    const int stage_bytes = 2 * TILE_A + 2 * bbytes;
-    __shared__ uint64_t full_bar[4], xform_bar[4], empty_bar[4], acc_bar;
+    const int pbytes = p.nbp * BK * 16;
+    __shared__ uint64_t b_full[MAX_STAGES], b_empty[MAX_STAGES], r_full[MAX_STAGES], r_empty[MAX_STAGES];
+    __shared__ uint64_t a_full[A_STAGES], a_empty[A_STAGES], acc_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int S = p.n_stages;
+    const int BS = p.b_stages, RS = p.r_stages;
     const int nk = (p.K + BK - 1) / BK;
     const long long m_tile = blockIdx.x;
     const int n_tile = blockIdx.y;
+    const long long b_first = (p.pg.pass_m0 + m_tile * BM) / p.pg.R_pass;
 
     if (threadIdx.x == 0) {
         abort_sh = 0;
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full_bar[s], 1);
-            mbar_init(&xform_bar[s], 128);
-            mbar_init(&empty_bar[s], 1);
+        for (int s = 0; s < BS; ++s) {
+            mbar_init(&b_full[s], 1);
+            mbar_init(&b_empty[s], 1);
+        }
+        for (int s = 0; s < RS; ++s) {
+            mbar_init(&r_full[s], 1);
+            mbar_init(&r_empty[s], 128);
+        }
+        for (int s = 0; s < A_STAGES; ++s) {
+            mbar_init(&a_full[s], 128);
+            mbar_init(&a_empty[s], 1);
         }
         mbar_init(&acc_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_sh)),
-                     "r"(256)
+                     "r"(TMEM_COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -186,98 +225,111 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 
     if (warp == 0) {
         if (lane == 0) {
+            // ----------------------------------------------------------- TMA producer
             const int ya = (p.a_row_mode == 0) ? (int)(m_tile * BM) : (int)((p.a_m0 + m_tile * BM) % p.a_RA);
             const int yb = n_tile * p.BN;
-            int issued = 0;
+            int r_issued = 0, b_issued = 0;
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % S;
-                if (kb >= S && !mbar_wait(&empty_bar[s], ((kb / S) - 1) & 1, abort_flag)) break;
-                uint8_t* st = base + (size_t)s * stage_bytes;
-                mbar_expect_tx(&full_bar[s], TILE_A + 2 * bbytes);
-                tma_load_2d(st, &tmA, &full_bar[s], kb * BK, ya);
-                tma_load_2d(st + 2 * TILE_A, &tmBhi, &full_bar[s], kb * BK, yb);
-                tma_load_2d(st + 2 * TILE_A + bbytes, &tmBlo, &full_bar[s], kb * BK, yb);
-                issued = kb + 1;
+                const int sr = kb % RS, sb = kb % BS;
+                if (kb >= RS && !mbar_wait(&r_empty[sr], ((kb / RS) - 1) & 1, abort_flag)) break;
+                mbar_expect_tx(&r_full[sr], TILE_A + pbytes);
+                tma_load_2d(base + p.r_off + sr * TILE_A, &tmA, &r_full[sr], kb * BK, ya);
+                tma_load_2d(base + p.p_off + sr * pbytes, &tmP, &r_full[sr], kb * BK * 4, (int)b_first);
+                r_issued = kb + 1;
+                if (kb >= BS && !mbar_wait(&b_empty[sb], ((kb / BS) - 1) & 1, abort_flag)) break;
+                uint8_t* bst = base + p.b_off + (size_t)sb * 2 * bbytes;
+                mbar_expect_tx(&b_full[sb], 2 * bbytes);
+                tma_load_2d(bst, &tmBhi, &b_full[sb], kb * BK, yb);
+                tma_load_2d(bst + bbytes, &tmBlo, &b_full[sb], kb * BK, yb);
+                b_issued = kb + 1;
             }
-            if (*abort_flag) {
-                // drain: wait (bounded) for every copy this thread issued that nobody consumed
-                for (int kb = (issued > S ? issued - S : 0); kb < issued; ++kb) {
+            if (*abort_flag) {  // drain copies still in flight before the CTA can exit
+                for (int kb = (r_issued > RS ? r_issued - RS : 0); kb < r_issued; ++kb) {
                     const long long t0 = clock64();
-                    while (!mbar_test(&full_bar[kb % S], (kb / S) & 1) && clock64() - t0 < WAIT_CYCLES) {
+                    while (!mbar_test(&r_full[kb % RS], (kb / RS) & 1) && clock64() - t0 < WAIT_CYCLES) {
+                    }
+                }
+                for (int kb = (b_issued > BS ? b_issued - BS : 0); kb < b_issued; ++kb) {
+                    const long long t0 = clock64();
+                    while (!mbar_test(&b_full[kb % BS], (kb / BS) & 1) && clock64() - t0 < WAIT_CYCLES) {
                     }
                 }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
+            // ----------------------------------------------------------- MMA issuer
             const uint32_t idesc = idesc_tf32(p.BN);
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % S;
-                const uint32_t ph = (kb / S) & 1;
-                if (!mbar_wait(&xform_bar[s], ph, abort_flag)) break;
-                if (!mbar_wait(&full_bar[s], ph, abort_flag)) break;
+                const int sa = kb % A_STAGES, sb = kb % BS;
+                if (!mbar_wait(&a_full[sa], (kb / A_STAGES) & 1, abort_flag)) break;
+                if (!mbar_wait(&b_full[sb], (kb / BS) & 1, abort_flag)) break;
                 tc_fence_after();
-                uint8_t* st = base + (size_t)s * stage_bytes;
-                const uint64_t da_hi = sw128_desc(smem_u32(st));
-                const uint64_t da_lo = sw128_desc(smem_u32(st + TILE_A));
-                const uint64_t db_hi = sw128_desc(smem_u32(st + 2 * TILE_A));
-                const uint64_t db_lo = sw128_desc(smem_u32(st + 2 * TILE_A + bbytes));
+                uint8_t* bst = base + p.b_off + (size_t)sb * 2 * bbytes;
+                const uint64_t db_hi = sw128_desc(smem_u32(bst));
+                const uint64_t db_lo = sw128_desc(smem_u32(bst + bbytes));
+                const uint32_t ta_hi = tmem + 256 + sa * 64;
+                const uint32_t ta_lo = ta_hi + 32;
 #pragma unroll
                 for (int kk = 0; kk < BK / 8; ++kk) {
-                    const uint64_t off = (uint64_t)(kk * 32) >> 4;  // 8 tf32 = 32 bytes along K
+                    const uint64_t off = (uint64_t)(kk * 32) >> 4;  // 8 tf32 = 32 bytes along K in smem
                     const uint32_t first = (kb > 0 || kk > 0) ? 1u : 0u;
-                    mma_tf32(tmem, da_lo + off, db_hi + off, idesc, first);
-                    mma_tf32(tmem, da_hi + off, db_lo + off, idesc, 1u);
-                    mma_tf32(tmem, da_hi + off, db_hi + off, idesc, 1u);
+                    mma_tf32_ts(tmem, ta_lo + kk * 8, db_hi + off, idesc, first);
+                    mma_tf32_ts(tmem, ta_hi + kk * 8, db_lo + off, idesc, 1u);
+                    mma_tf32_ts(tmem, ta_hi + kk * 8, db_hi + off, idesc, 1u);
                 }
-                mma_commit(&empty_bar[s]);
+                mma_commit(&a_empty[sa]);
+                mma_commit(&b_empty[sb]);
             }
             mma_commit(&acc_bar);
-            // never free TMEM under MMAs still in flight, even after an abort
-            const long long t0 = clock64();
+            const long long t0 = clock64();  // never free TMEM under MMAs still in flight
             while (!mbar_test(&acc_bar, 0) && clock64() - t0 < WAIT_CYCLES) {
             }
         }
     } else {
-        // ------------------------------------------------------------ transform + epilogue
-        const int q = warp & 3;                  // TMEM lane quarter this warp may access
-        const int row = q * 32 + lane;           // row of the tile owned by this thread
+        // ------------------------------------------------------------- transform + epilogue
+        const int q = warp & 3;         // TMEM lane quarter this warp may access
+        const int row = q * 32 + lane;  // tile row owned by this thread (TMEM lane)
         const long long m = m_tile * BM + row;
         const bool valid = m < p.M;
         const long long b = (p.pg.pass_m0 + m) / p.pg.R_pass;
+        const int cb = valid ? (int)(b - b_first) : 0;
         const bool do_cst = (p.cst != nullptr) && n_tile == 0;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         float cacc = 0.f;
-        const float4* P = p.rx.P;
         for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % S;
-            if (!mbar_wait(&full_bar[s], (kb / S) & 1, abort_flag)) break;
-            uint8_t* st = base + (size_t)s * stage_bytes;
-            float4* arow = reinterpret_cast<float4*>(st + row * 128);
-            float4* lrow = reinterpret_cast<float4*>(st + TILE_A + row * 128);
-            const int k0 = kb * BK;
+            const int sr = kb % RS, sa = kb % A_STAGES;
+            bool ok = mbar_wait(&r_full[sr], (kb / RS) & 1, abort_flag);
+            float hi[32], lo[32];
+            if (ok) {
+                const float4* arow = reinterpret_cast<const float4*>(base + p.r_off + sr * TILE_A + row * 128);
+                const float4* prow = reinterpret_cast<const float4*>(base + p.p_off + sr * pbytes) + cb * BK;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const int pc = c ^ (row & 7);  // 128-byte swizzle: chunk c of this row sits at pc
-                float4 x = arow[pc];
-                float v[4] = {x.x, x.y, x.z, x.w};
+                for (int c = 0; c < 8; ++c) {
+                    const float4 x = arow[c ^ (row & 7)];  // 128-byte swizzle of the TMA tile
+                    const float xv[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int k = k0 + c * 4 + j;
-                    float r = v[j];
-                    if (P != nullptr && valid && k < p.K) {
-                        const float4 pr = __ldg(&P[b * p.K + k]);
-                        r = (v[j] >= 0.f) ? v[j] * pr.x : v[j] * pr.y;
-                        if (p.rx.count_const) cacc = fmaf(fminf(v[j], 0.f), pr.z, cacc);
+                    for (int j = 0; j < 4; ++j) {
+                        const float4 pr = prow[c * 4 + j];
+                        const float v = xv[j];
+                        const float r = (v >= 0.f) ? v * pr.x : v * pr.y;
+                        if (p.count_const) cacc = fmaf(fminf(v, 0.f), pr.z, cacc);
+                        cacc = fmaf(r, pr.w, cacc);
+                        const float h = tf32_hi(r);
+                        hi[c * 4 + j] = h;
+                        lo[c * 4 + j] = r - h;
                     }
-                    if (do_cst && p.bias != nullptr && valid && k < p.K) cacc = fmaf(r, __ldg(&p.bias[k]), cacc);
-                    v[j] = r;
                 }
-                const float4 hi = make_float4(tf32_hi(v[0]), tf32_hi(v[1]), tf32_hi(v[2]), tf32_hi(v[3]));
-                arow[pc] = hi;
-                lrow[pc] = make_float4(v[0] - hi.x, v[1] - hi.y, v[2] - hi.z, v[3] - hi.w);
+                mbar_arrive(&r_empty[sr]);
+                if (kb >= A_STAGES) ok = mbar_wait(&a_empty[sa], ((kb / A_STAGES) - 1) & 1, abort_flag);
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive(&xform_bar[s]);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const uint32_t ta = tmem + lane_base + 256 + sa * 64;
+            tmem_st32(ta, hi);
+            tmem_st32(ta + 32, lo);
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            tc_fence_before();
+            mbar_arrive(&a_full[sa]);
         }
         if (do_cst && valid && !*abort_flag) p.cst[m] += cacc;
 
@@ -285,27 +337,45 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         const bool acc_ready = __all_sync(0xffffffffu, mbar_wait(&acc_bar, 0, abort_flag));
         if (acc_ready) {
             tc_fence_after();
-            const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
             const int n0 = n_tile * p.BN;
-            float conc = 0.f;
-            const float* crow = (p.out_mode == OUT_CONCRETIZE && valid) ? p.centres + b * (long long)p.N : nullptr;
-            float* orow = (p.out_mode != OUT_CONCRETIZE && valid) ? p.out + m * p.ld_out : nullptr;
-            for (int c0 = 0; c0 < p.BN; c0 += 32) {
-                float v[32];
-                tmem_ld32(lane_addr + c0, v);
-                if (!valid) continue;
+            if (p.out_mode == OUT_CONCRETIZE) {
+                float conc = 0.f;
+                const float* crow = p.centres + (valid ? b : 0) * (long long)p.N;
+                for (int c0 = 0; c0 < p.BN; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + c0, v);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int n = n0 + c0 + j;
-                    if (c0 + j >= p.BN || n >= p.N) break;
-                    if (crow != nullptr) {
-                        conc += fmaf(v[j], __ldg(&crow[n]), -p.eps * fabsf(v[j]));
-                    } else {
-                        orow[n] = (p.out_mode == OUT_ACCUM ? orow[n] : 0.f) + v[j];
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = n0 + c0 + j;
+                        if (valid && c0 + j < p.BN && n < p.N) conc += fmaf(v[j], __ldg(&crow[n]), -p.eps * fabsf(v[j]));
                     }
                 }
+                if (valid) p.part[(long long)n_tile * p.M + m] = conc;
+            } else {
+                // stage each 32x32 block through smem (the raw-A ring is idle now) so that every
+                // warp store covers one contiguous 128-byte row segment
+                float* stg = reinterpret_cast<float*>(base + p.r_off) + q * (32 * 33);
+                const long long row0 = m_tile * BM + q * 32;
+                for (int c0 = 0; c0 < p.BN; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + c0, v);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = v[j];
+                    __syncwarp();
+                    const int n = n0 + c0 + lane;
+                    const bool col_ok = (c0 + lane < p.BN) && (n < p.N);
+#pragma unroll 4
+                    for (int j = 0; j < 32; ++j) {
+                        const long long mr = row0 + j;
+                        if (col_ok && mr < p.M) {
+                            float* o = p.out + mr * p.ld_out + n;
+                            const float val = stg[j * 33 + lane];
+                            *o = (p.out_mode == OUT_ACCUM) ? (*o + val) : val;
+                        }
+                    }
+                    __syncwarp();
+                }
             }
-            if (p.out_mode == OUT_CONCRETIZE && valid) p.part[(long long)n_tile * p.M + m] = conc;
         }
     }
 
@@ -313,7 +383,7 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
     }
     if (threadIdx.x == 0 && abort_sh && p.err != nullptr) atomicExch(p.err, 1);
 }
@@ -338,16 +408,18 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2-D fp32 tensor map: inner dimension `cols` (contiguous), `rows` rows `ld` elements apart,
-// box of 32 x box_rows, 128-byte swizzle, zero fill outside.
-bool make_map(CUtensorMap* map, const float* ptr, long long cols, long long rows, long long ld, int box_rows) {
+// box of box_cols x box_rows, 128-byte swizzle (box_cols = 32) or none, zero fill outside.
+bool make_map(CUtensorMap* map, const float* ptr, long long cols, long long rows, long long ld, int box_rows,
+              int box_cols, bool swizzle) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)(ld * 4)};
-    cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -359,6 +431,9 @@ int pick_bn(int N, int* ntiles) {
     return bn;
 }
 
+// Centres a 128-row tile can span when a pass has R rows per centre.
+long long centres_per_tile(long long R) { return 127 / R + 2; }
+
 }  // namespace
 
 int dense_back_tc_tiles_n(int N) {
@@ -367,16 +442,17 @@ int dense_back_tc_tiles_n(int N) {
     return t;
 }
 
-bool dense_back_tc_supported(const RowRef& A, long long M, int K, int N, PassGeom pg) {
+bool dense_back_tc_supported(const RowRef& A, Relax rx, long long M, int K, int N, PassGeom pg) {
+    if (rx.P == nullptr) return false;                     // the bias rides in the relaxation table
     if (K % 4 != 0 || K < 32 || N < 16) return false;
+    if (centres_per_tile(pg.R_pass) > 32) return false;
     if ((reinterpret_cast<uintptr_t>(A.ptr) & 15) != 0 || (A.ld % 4) != 0) return false;
-    if (A.RA == kHugeRows && A.sB == 0 && A.m0 == 0) return M < (1LL << 31);  // chunk-local rows
-    if (A.sB == 0 && A.RA % BM == 0 && A.m0 % BM == 0) return true;            // one block shared by all centres
-    (void)pg;
+    if (A.RA == kHugeRows && A.sB == 0 && A.m0 == 0) return M >= BM && M < (1LL << 31);  // chunk-local rows
+    if (A.sB == 0 && A.RA % BM == 0 && A.m0 % BM == 0) return true;  // one block shared by all centres
     return false;
 }
 
-cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, const float* Wt_lo, const float* bias,
+cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, const float* Wt_lo, long long B,
                                  long long M, int K, int N, PassGeom pg, int out_mode, float* out, long long ld_out,
                                  float* cst, const float* centres, float eps, float* part, int* err, cudaStream_t s) {
     if (M <= 0) return cudaSuccess;
@@ -384,11 +460,22 @@ cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, 
     p.M = M;
     p.K = K;
     p.N = N;
+    p.B = B;
     p.BN = pick_bn(N, &p.ntiles_n);
-    const int stage_bytes = 2 * TILE_A + 2 * p.BN * BK * 4;
-    p.n_stages = stage_bytes * 4 + 1024 <= 220 * 1024 ? 4 : (stage_bytes * 3 + 1024 <= 220 * 1024 ? 3 : 2);
-    const size_t smem = (size_t)stage_bytes * p.n_stages + 1024;
-    CUtensorMap ta, tbh, tbl;
+    p.nbp = (int)std::min<long long>(centres_per_tile(pg.R_pass), B);
+    const int bstage = 2 * p.BN * BK * 4;
+    const int rstage = TILE_A + p.nbp * BK * 16;
+    const int budget = 220 * 1024 - 1024;
+    p.b_stages = 2;
+    p.r_stages = 2;
+    while (p.b_stages < 4 && (p.b_stages + 1) * bstage + p.r_stages * rstage <= budget) p.b_stages++;
+    while (p.r_stages < MAX_STAGES && p.b_stages * bstage + (p.r_stages + 1) * rstage <= budget) p.r_stages++;
+    if (p.b_stages * bstage + p.r_stages * rstage > budget) return cudaErrorInvalidValue;
+    p.b_off = 0;
+    p.r_off = p.b_stages * bstage;                        // multiple of 1024 (BN is a multiple of 16)
+    p.p_off = p.r_off + p.r_stages * TILE_A;              // TILE_A is a multiple of 1024
+    const size_t smem = (size_t)p.p_off + (size_t)p.r_stages * p.nbp * BK * 16 + 1024;
+    CUtensorMap ta, tp, tbh, tbl;
     long long a_rows;
     if (A.RA == kHugeRows) {
         p.a_row_mode = 0;
@@ -399,8 +486,9 @@ cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, 
         p.a_RA = A.RA;
         a_rows = A.RA;
     }
-    if (!make_map(&ta, A.ptr, K, a_rows, A.ld, BM) || !make_map(&tbh, Wt_hi, K, N, K, p.BN) ||
-        !make_map(&tbl, Wt_lo, K, N, K, p.BN))
+    if (!make_map(&ta, A.ptr, K, a_rows, A.ld, BM, 32, true) ||
+        !make_map(&tp, reinterpret_cast<const float*>(rx.P), 4LL * K, B, 4LL * K, p.nbp, 128, false) ||
+        !make_map(&tbh, Wt_hi, K, N, K, p.BN, 32, true) || !make_map(&tbl, Wt_lo, K, N, K, p.BN, 32, true))
         return cudaErrorInvalidValue;
     p.pg = pg;
     p.out_mode = out_mode;
@@ -410,8 +498,7 @@ cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, 
     p.centres = centres;
     p.eps = eps;
     p.part = part;
-    p.bias = bias;
-    p.rx = rx;
+    p.count_const = rx.count_const;
     p.err = err;
     static bool attr = false;
     if (!attr) {
@@ -420,7 +507,7 @@ cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, 
         attr = true;
     }
     dim3 grid((unsigned)((M + BM - 1) / BM), (unsigned)p.ntiles_n);
-    dense_back_tc<<<grid, NUM_THREADS, smem, s>>>(ta, tbh, tbl, p);
+    dense_back_tc<<<grid, NUM_THREADS, smem, s>>>(ta, tp, tbh, tbl, p);
     return cudaGetLastError();
 }
 

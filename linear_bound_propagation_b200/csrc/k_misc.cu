@@ -23,9 +23,12 @@ unsigned grid_for(long long n, int threads) {
 
 // ReLU relaxation for l <= z <= u: inactive (u <= 0, tested first) {0, 0, 0}; active (l >= 0)
 // {1, 1, 0}; unstable: upper chord up = u / (u - l), t = -up * l; lower slope alpha clamped
-// to [0, 1], or the adaptive choice 1 if u >= -l else 0.
+// to [0, 1], or the adaptive choice 1 if u >= -l else 0. The fourth lane carries the bias of
+// the affine node that produced z (0 if none), which the next back-substitution step adds to
+// the row constant together with the relaxation intercept.
 __global__ void relax_params_k(const float* __restrict__ l, const float* __restrict__ u,
-                               const float* __restrict__ alpha, long long n, float4* __restrict__ P) {
+                               const float* __restrict__ alpha, long long n, float4* __restrict__ P,
+                               const float* __restrict__ bias, long long n_per_centre, long long per_channel) {
     GRID_STRIDE(i, n) {
         const float lo_b = l[i], up_b = u[i];
         float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -42,6 +45,7 @@ __global__ void relax_params_k(const float* __restrict__ l, const float* __restr
             else
                 p.x = (up_b >= -lo_b) ? 1.f : 0.f;
         }
+        p.w = (bias != nullptr) ? bias[(i % n_per_centre) / per_channel] : 0.f;
         P[i] = p;
     }
 }
@@ -260,8 +264,8 @@ unsigned rows_grid(long long rows_per_cta_units) {
 }  // namespace
 
 cudaError_t launch_relax_params(const float* l, const float* u, const float* alpha, long long n, float4* P,
-                                cudaStream_t s) {
-    relax_params_k<<<grid_for(n, 256), 256, 0, s>>>(l, u, alpha, n, P);
+                                const float* bias, long long n_per_centre, long long per_channel, cudaStream_t s) {
+    relax_params_k<<<grid_for(n, 256), 256, 0, s>>>(l, u, alpha, n, P, bias, n_per_centre, per_channel);
     return cudaGetLastError();
 }
 

@@ -187,6 +187,7 @@ struct Walker {
     int live = 0, max_live = 0;
     const float* centres = nullptr;
     float eps = 0.f;
+    long long n_centres = 0;  // rows of the relaxation tables
     float* ext_in = nullptr;  // vf_crown_backward: rows over the input go here ([M, n0], ld n0)
     bool ext_written = false;
     const std::vector<const float4*>* relax;  // per node: relaxation params of ReLU nodes
@@ -372,13 +373,13 @@ struct Walker {
                 int mode = OUT_CONCRETIZE;
                 if (!fuse) TRY(target(nd.src, &out, &ld, &mode));
                 const bool tc = net->dense_kernel == 0 && nd.WtHi != nullptr &&
-                                dense_back_tc_supported(e.ref, M, (int)nd.n, (int)sn.n, pg);
+                                dense_back_tc_supported(e.ref, e.rx, M, (int)nd.n, (int)sn.n, pg);
                 if (fuse) part_tiles = tc ? dense_back_tc_tiles_n((int)sn.n) : dense_back_tiles_n((int)sn.n);
                 if (!dry) {
                     cudaEvent_t e0 = nullptr;
                     prof_begin(&e0);
                     if (tc)
-                        LAUNCH(net, launch_dense_back_tc(e.ref, e.rx, nd.WtHi, nd.WtLo, nd.b, M, (int)nd.n, (int)sn.n, pg,
+                        LAUNCH(net, launch_dense_back_tc(e.ref, e.rx, nd.WtHi, nd.WtLo, n_centres, M, (int)nd.n, (int)sn.n, pg,
                                                          mode, out, ld, cst, centres, eps, part, net->d_err, s));
                     else
                         LAUNCH(net, launch_dense_back(e.ref, e.rx, nd.W, nd.b, M, (int)nd.n, (int)sn.n, pg, mode, out,
@@ -571,6 +572,7 @@ int run_pass(vf_net* net, int start, Entry init, long long rows, long long R_pas
     w.relax = &relax;
     w.centres = centres;
     w.eps = eps;
+    w.n_centres = rows / R_pass;
     for (long long m0 = 0; m0 < rows; m0 += chunk) {
         w.M = std::min(chunk, rows - m0);
         w.pg = PassGeom{m0, R_pass};
@@ -599,7 +601,10 @@ int build_relax(vf_net* net, int B, const std::vector<const float*>& L, const st
         if (nd.op != VF_RELU) continue;
         float4* P = ar.take<float4>((size_t)B * nd.n);
         if (!P) return fail(VF_ERR_WORKSPACE, "workspace too small for relaxation parameters");
-        LAUNCH(net, launch_relax_params(L[nd.src], U[nd.src], alpha ? alpha[v] : nullptr, (long long)B * nd.n, P, s));
+        const Node& sn = net->nodes[nd.src];
+        const bool aff = sn.op == VF_DENSE || sn.op == VF_CONV2D;
+        LAUNCH(net, launch_relax_params(L[nd.src], U[nd.src], alpha ? alpha[v] : nullptr, (long long)B * nd.n, P,
+                                        aff ? sn.b : nullptr, nd.n, sn.op == VF_CONV2D ? (long long)sn.h * sn.w : 1, s));
         relax[v] = P;
     }
     return VF_OK;
@@ -940,7 +945,10 @@ int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const f
                          nullptr, s));
             LAUNCH(net, launch_intersect(Lw[p], Uw[p], nullptr, nullptr, pass_out, B, np, s));
         }
-        LAUNCH(net, launch_relax_params(Lw[p], Uw[p], o.alpha ? o.alpha[k] : nullptr, (long long)B * nd.n, P[k], s));
+        const Node& sn = net->nodes[p];
+        const bool aff = sn.op == VF_DENSE || sn.op == VF_CONV2D;
+        LAUNCH(net, launch_relax_params(Lw[p], Uw[p], o.alpha ? o.alpha[k] : nullptr, (long long)B * nd.n, P[k],
+                                        aff ? sn.b : nullptr, nd.n, sn.op == VF_CONV2D ? (long long)sn.h * sn.w : 1, s));
     }
 
     // Specification pass.

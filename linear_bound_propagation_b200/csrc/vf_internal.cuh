@@ -73,8 +73,10 @@ cudaError_t launch_fill(float* p, long long n, float v, cudaStream_t s);
 cudaError_t launch_bounds_from_cr(const float* c, const float* r, long long n, float* lb, float* ub, cudaStream_t s);
 
 // ---- relaxation, pass bookkeeping, decision (k_misc.cu) ------------------------------
+// P[i] = {lo, up, t, bias of the affine source}; bias may be null (then 0); neuron j = i % n_per_centre
+// takes bias[j / per_channel] (per_channel = H*W for a convolution, 1 for a dense node).
 cudaError_t launch_relax_params(const float* l, const float* u, const float* alpha, long long n, float4* P,
-                                cudaStream_t s);
+                                const float* bias, long long n_per_centre, long long per_channel, cudaStream_t s);
 cudaError_t launch_cst_identity_bias(float* cst, long long M, PassGeom pg, const float* bias, long long n_p,
                                      long long per_channel, cudaStream_t s);
 cudaError_t launch_ident_rows(float* out, long long ld, long long M, PassGeom pg, long long n_p, int accumulate,

@@ -6,11 +6,13 @@ namespace vf {
 
 // True when the rows can be fed by a 2-D TMA map: 16-byte aligned rows of a chunk-local buffer,
 // or one block of rows shared by all centres whose size is a multiple of the 128-row tile.
-bool dense_back_tc_supported(const RowRef& A, long long M, int K, int N, PassGeom pg);
+// The tensor-core path also needs a relaxation table (it carries the bias in its 4th lane).
+bool dense_back_tc_supported(const RowRef& A, Relax rx, long long M, int K, int N, PassGeom pg);
 int dense_back_tc_tiles_n(int N);
 // Wt_hi / Wt_lo: the node's W transposed to [N, K] (K contiguous) and split into tf32 head and
-// fp32 remainder. Same outputs as launch_dense_back; *err is set if a bounded wait expires.
-cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, const float* Wt_lo, const float* bias,
+// fp32 remainder; B = number of centres (rows of rx.P). Same outputs as launch_dense_back, with
+// the bias taken from rx.P[.].w; *err is set if a bounded wait expires.
+cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, const float* Wt_lo, long long B,
                                  long long M, int K, int N, PassGeom pg, int out_mode, float* out, long long ld_out,
                                  float* cst, const float* centres, float eps, float* part, int* err, cudaStream_t s);
 
