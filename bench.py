@@ -128,6 +128,56 @@ def stop_clocks(handle):
     return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# Nominal dense-throughput ratios used to derive a per-dtype peak from the measured bf16 one.
+TF32_OVER_BF16 = 1.1 / 2.25
+
+
+def roofline(kstats, step_total_ms, n_sms):
+    """Roofline entry for the dominant contraction kind of the step.
+
+    Tensor-core dense steps (3xTF32): algorithmic flops 2*M*K*N per launch against the tf32 peak
+    divided by 3 (three tf32 MMAs per fp32-accurate product); the tf32 peak is the measured bf16
+    burst peak times the nominal tf32/bf16 ratio. FFMA and convolution kernels: fp32 FFMA peak =
+    SMs x 128 lanes x 2 flop x max SM clock ("alu")."""
+    p, src = peaks()
+    kind = max(kstats, key=lambda k: kstats[k][1])
+    n_k, k_ms, k_flops = kstats[kind]
+    avg_ms = k_ms / max(n_k, 1)
+    achieved = (k_flops / max(n_k, 1)) / (avg_ms / 1000.0) / 1e12 if n_k else 0.0
+    sm_mhz = float(p.get("sm_max_mhz", 1965.0))
+    if kind == 1:
+        tf32 = float(p["bf16_tflops"]) * TF32_OVER_BF16
+        peak = tf32 / 3.0
+        bound, name = "tensor", "dense_back_tc (tcgen05 kind::tf32, 3xTF32 CROWN Lambda.W contraction)"
+        psrc = (f"tf32 = {src} bf16 burst {p['bf16_tflops']:.0f} TFLOP/s x nominal 1.1/2.25 = {tf32:.0f}; "
+                f"3xTF32 effective = tf32 / 3")
+    else:
+        peak = n_sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+        bound = "alu"
+        name = "dense_back_ffma" if kind == 2 else "conv_back_ffma"
+        psrc = f"fp32 FFMA: {n_sms} SMs x 128 lanes x 2 flop x {sm_mhz:.0f} MHz ({src} max clock)"
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": None, "kernel": name, "launches": n_k, "avg_launch_ms": avg_ms,
+            "share_of_step": k_ms / step_total_ms if step_total_ms else None, "peak_source": psrc}
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Largest `value` over all ranks of the default process group (timing only, never data)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_throughput(world: int, specs_per_rank_step: int, steps: int, total_ms: float) -> float:
+    """Whole-job specs/s: every rank processes its own full workload each step; the job takes the
+    slowest rank's time."""
+    return world * specs_per_rank_step * steps / (total_ms / 1000.0)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -206,15 +256,13 @@ def run_ours(args):
     torch.cuda.synchronize()
     clocks = stop_clocks(clk)
     launches = net.launch_count() - launches0
-    n_k, k_ms, k_flops = net.profile_read(reset=True)
+    kstats = {k: net.profile_read(kind=k, reset=False) for k in (1, 2, 3)}
+    net.profile_read(reset=True)
     net.profile(False)
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * B * Rs * args.steps / (total_ms / 1000.0)
+    total_ms = max_over_ranks(total_ms, dev)
+    value = weak_throughput(world, B * Rs, args.steps, total_ms)
     verified = int(out["verified"].sum().item())
 
     # End to end through the public API with host buffers: pinned H2D of centres and C, the
@@ -246,31 +294,17 @@ def run_ours(args):
         b.record(stream)
         b.synchronize()
         e2e_ms += a.elapsed_time(b)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
     h2d = h_centres.numel() * 4 + h_C.numel() * 4
     d2h = h_lb.numel() * 4 + h_ver.numel()
 
-    p, src = peaks()
-    sm_mhz = float(p.get("sm_max_mhz", 1965.0))
-    props = torch.cuda.get_device_properties(dev)
-    ffma_peak = props.multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
-    avg_ms = k_ms / max(n_k, 1)
-    achieved = (k_flops / max(n_k, 1)) / (avg_ms / 1000.0) / 1e12 if n_k else 0.0
-    roof = {"bound": "alu", "achieved": achieved, "peak": ffma_peak, "unit": "TFLOP/s",
-            "frac": achieved / ffma_peak, "traffic": None, "kernel": "dense_back_ffma (CROWN Lambda.W contraction)",
-            "launches": n_k, "avg_launch_ms": avg_ms, "share_of_step": k_ms / total_ms if total_ms else None,
-            "peak_source": f"fp32 FFMA: {props.multi_processor_count} SMs x 128 lanes x 2 flop x {sm_mhz:.0f} MHz "
-                           f"({src} max clock)"}
-
+    roof = roofline(kstats, total_ms, torch.cuda.get_device_properties(dev).multi_processor_count)
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": workload_config(w, args.config), "roofline": roof,
-                "e2e": {"value": world * B * Rs * args.steps / (e2e_ms / 1000.0), "unit": UNIT,
+                "e2e": {"value": weak_throughput(world, B * Rs, args.steps, e2e_ms), "unit": UNIT,
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches, "clocks": clocks, "verified_specs": verified, "total_specs": B * Rs}
         if world == 1 and not args.no_cpu_baseline:

@@ -146,13 +146,14 @@ int vf_net_check(vf_net* net);
 /* Per-thread description of the last error (empty string if none). */
 const char* vf_last_error(void);
 
-/* Kernel timing, for benchmarks. While enabled, the library brackets each launch of
- * the CROWN back-substitution contraction with CUDA events on the launching stream.
- * vf_profile_read synchronises those events and returns the number of such launches,
- * their summed device time in ms, and their summed algorithmic flops (2*M*K*N each),
- * since the last reset. */
+/* Kernel timing, for benchmarks. While enabled, the library brackets each launch of a CROWN
+ * back-substitution contraction with CUDA events on the launching stream. vf_profile_read
+ * synchronises those events and returns, for one kind of contraction, the number of launches,
+ * their summed device time in ms and their summed algorithmic flops (2*M*K*N for dense steps;
+ * 2*M*n_in*C_out*k*k/stride^2 for convolutions) since the last reset (reset != 0 clears all kinds). */
+enum { VF_KERNEL_ALL = 0, VF_KERNEL_DENSE_TC = 1, VF_KERNEL_DENSE_FFMA = 2, VF_KERNEL_CONV = 3 };
 int vf_profile_enable(vf_net* net, int enable);
-int vf_profile_read(vf_net* net, long long* launches, double* total_ms, double* flops, int reset);
+int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms, double* flops, int reset);
 
 /* Number of kernel launches the library has enqueued on this handle since creation. */
 long long vf_launch_count(const vf_net* net);

@@ -91,10 +91,15 @@ struct vf_net {
     int* d_err = nullptr;   // device flag raised by a kernel whose bounded wait expired
     bool prof = false;
     std::vector<cudaEvent_t> ev_free;
-    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev_used;
-    double prof_flops = 0.0;
-    long long prof_launches = 0;
-    double prof_ms = 0.0;
+    struct Timed {
+        cudaEvent_t e0, e1;
+        int kind;
+        double flops;
+    };
+    std::vector<Timed> ev_used;
+    double prof_flops[4] = {0, 0, 0, 0};
+    long long prof_launches[4] = {0, 0, 0, 0};
+    double prof_ms[4] = {0, 0, 0, 0};
 };
 
 namespace {
@@ -305,12 +310,11 @@ struct Walker {
             cudaEventRecord(*e0, s);
         }
     }
-    void prof_end(cudaEvent_t e0, double flops) {
+    void prof_end(cudaEvent_t e0, int kind, double flops) {
         if (net->prof && !dry) {
             cudaEvent_t e1 = take_event(net);
             cudaEventRecord(e1, s);
-            net->ev_used.push_back({e0, e1});
-            net->prof_flops += flops;
+            net->ev_used.push_back({e0, e1, kind, flops});
         }
     }
 
@@ -384,7 +388,7 @@ struct Walker {
                     else
                         LAUNCH(net, launch_dense_back(e.ref, e.rx, nd.W, nd.b, M, (int)nd.n, (int)sn.n, pg, mode, out,
                                                       ld, cst, centres, eps, part, s));
-                    prof_end(e0, 2.0 * (double)M * (double)nd.n * (double)sn.n);
+                    prof_end(e0, tc ? VF_KERNEL_DENSE_TC : VF_KERNEL_DENSE_FFMA, 2.0 * (double)M * (double)nd.n * (double)sn.n);
                 }
                 release(e);
                 return VF_OK;
@@ -413,8 +417,8 @@ struct Walker {
                     prof_begin(&e0);
                     LAUNCH(net, launch_conv_back(e.ref, e.rx, nd.W, nd.b, M, g, pg, mode, out, ld, cst, centres, eps,
                                                  net->num_sms, s));
-                    prof_end(e0, 2.0 * (double)M * (double)net->nodes[nd.src].n * (double)g.co * g.k * g.k /
-                                     ((double)g.stride * g.stride));
+                    prof_end(e0, VF_KERNEL_CONV, 2.0 * (double)M * (double)net->nodes[nd.src].n * (double)g.co * g.k *
+                                                     g.k / ((double)g.stride * g.stride));
                 }
                 release(e);
                 return VF_OK;
@@ -648,8 +652,8 @@ void vf_net_destroy(vf_net* net) {
     cudaFree(net->d_err);
     for (auto e : net->ev_free) cudaEventDestroy(e);
     for (auto& p : net->ev_used) {
-        cudaEventDestroy(p.first);
-        cudaEventDestroy(p.second);
+        cudaEventDestroy(p.e0);
+        cudaEventDestroy(p.e1);
     }
     cudaFree(net->ws);
     delete net;
@@ -987,26 +991,31 @@ int vf_profile_enable(vf_net* net, int enable) {
     return VF_OK;
 }
 
-int vf_profile_read(vf_net* net, long long* launches, double* total_ms, double* flops, int reset) {
+int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms, double* flops, int reset) {
     TRY(check_net(net));
-    for (auto& p : net->ev_used) {
-        CU(cudaEventSynchronize(p.second));
+    if (kind < 0 || kind > 3) return fail(VF_ERR_ARG, "bad kernel kind");
+    for (auto& t : net->ev_used) {
+        CU(cudaEventSynchronize(t.e1));
         float ms = 0.f;
-        CU(cudaEventElapsedTime(&ms, p.first, p.second));
-        net->prof_ms += ms;
-        net->prof_launches++;
-        net->ev_free.push_back(p.first);
-        net->ev_free.push_back(p.second);
+        CU(cudaEventElapsedTime(&ms, t.e0, t.e1));
+        for (int k : {0, t.kind}) {
+            net->prof_ms[k] += ms;
+            net->prof_launches[k]++;
+            net->prof_flops[k] += t.flops;
+        }
+        net->ev_free.push_back(t.e0);
+        net->ev_free.push_back(t.e1);
     }
     net->ev_used.clear();
-    if (launches) *launches = net->prof_launches;
-    if (total_ms) *total_ms = net->prof_ms;
-    if (flops) *flops = net->prof_flops;
-    if (reset) {
-        net->prof_launches = 0;
-        net->prof_ms = 0.0;
-        net->prof_flops = 0.0;
-    }
+    if (launches) *launches = net->prof_launches[kind];
+    if (total_ms) *total_ms = net->prof_ms[kind];
+    if (flops) *flops = net->prof_flops[kind];
+    if (reset)
+        for (int k = 0; k < 4; ++k) {
+            net->prof_launches[k] = 0;
+            net->prof_ms[k] = 0.0;
+            net->prof_flops[k] = 0.0;
+        }
     return VF_OK;
 }
 

@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libvf.so")
 VF_OK, VF_ERR_ARG, VF_ERR_SHAPE, VF_ERR_WORKSPACE, VF_ERR_NONFINITE, VF_ERR_CUDA, VF_ERR_TIMEOUT, \
     VF_ERR_UNSUPPORTED = range(8)
 VF_INPUT, VF_DENSE, VF_CONV2D, VF_RELU, VF_ADD = range(5)
+VF_KERNEL_ALL, VF_KERNEL_DENSE_TC, VF_KERNEL_DENSE_FFMA, VF_KERNEL_CONV = range(4)
 
 SYMBOLS = ["vf_net_create", "vf_net_destroy", "vf_net_node_size", "vf_net_total_size", "vf_ibp",
            "vf_crown_backward", "vf_concretize", "vf_verify_batch", "vf_sync", "vf_last_error",
@@ -70,7 +71,7 @@ def lib() -> ctypes.CDLL:
     L.vf_sync.argtypes = [P]
     L.vf_last_error.restype = ctypes.c_char_p
     L.vf_profile_enable.argtypes = [P, I]
-    L.vf_profile_read.argtypes = [P, ctypes.POINTER(LL), ctypes.POINTER(ctypes.c_double),
+    L.vf_profile_read.argtypes = [P, I, ctypes.POINTER(LL), ctypes.POINTER(ctypes.c_double),
                                   ctypes.POINTER(ctypes.c_double), I]
     L.vf_net_check.argtypes = [P]
     L.vf_launch_count.argtypes = [P]
@@ -220,11 +221,14 @@ class Net:
     def profile(self, enable: bool):
         _check(lib().vf_profile_enable(self.h, 1 if enable else 0))
 
-    def profile_read(self, reset: bool = True):
+    def profile_read(self, kind: int = 0, reset: bool = True):
+        """(launches, total device ms, algorithmic flops) of one contraction kind since the last reset:
+        0 all, 1 dense tensor-core (3xTF32), 2 dense FFMA, 3 convolution."""
         n = ctypes.c_longlong()
         ms = ctypes.c_double()
         fl = ctypes.c_double()
-        _check(lib().vf_profile_read(self.h, ctypes.byref(n), ctypes.byref(ms), ctypes.byref(fl), 1 if reset else 0))
+        _check(lib().vf_profile_read(self.h, kind, ctypes.byref(n), ctypes.byref(ms), ctypes.byref(fl),
+                                     1 if reset else 0))
         return n.value, ms.value, fl.value
 
     def check(self):
