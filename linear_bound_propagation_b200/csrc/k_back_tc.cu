@@ -44,7 +44,7 @@ constexpr int BM = 128;
 constexpr int BK = 32;                 // one 128-byte swizzle row of fp32
 constexpr int TILE_A = BM * BK * 4;    // 16 KB
 constexpr int MAX_BN = 256;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 352;  // 11 warps, see the role map above the kernel
 constexpr long long WAIT_CYCLES = 4000000000LL;  // ~2 s at boost clock
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -158,11 +158,14 @@ constexpr uint32_t TMEM_COLS = 512;  // accumulator in [0, 256), A stages in [25
 struct TcParams {
     long long M;
     int K, N, BN, ntiles_n;
-    int b_stages, r_stages, nbp;  // B ring depth, raw-A ring depth, centres per P box
-    int b_off, r_off, p_off;      // byte offsets of the rings in dynamic smem
-    int a_row_mode;               // 0: local rows y = m; 1: shared block y = (m0 + m) % RA
+    long long ntiles;               // (M tiles) x (N tiles); CTA i takes tiles i, i + grid, ...
+    int b_stages, r_stages, nbp;    // B ring depth, raw-A ring depth, centres per P box
+    int nbw;                        // centres a warp's 32 rows can span (epilogue staging)
+    int b_off, r_off, p_off, s_off; // byte offsets of the rings and the epilogue staging
+    int s_floats;                   // epilogue staging floats per warp
+    int a_row_mode;                 // 0: local rows y = m; 1: shared block y = (m0 + m) % RA
     long long a_m0, a_RA;
-    long long B;                  // number of centres (rows of P)
+    long long B;                    // number of centres (rows of P and of centres)
     PassGeom pg;
     int out_mode;
     float* out;
@@ -175,6 +178,10 @@ struct TcParams {
     int* err;
 };
 
+// Warp roles (11 warps): 0 raw-A/P producer + TMEM owner, 1 MMA issuer, 2-5 transform,
+// 6-9 epilogue, 10 W producer.
+constexpr int W_RAW = 0, W_MMA = 1, W_XF0 = 2, W_EPI0 = 6, W_B = 10;
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmP,
               const __grid_constant__ CUtensorMap tmBhi, const __grid_constant__ CUtensorMap tmBlo, TcParams p) {
@@ -183,16 +190,14 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     const int bbytes = p.BN * BK * 4;
     const int pbytes = p.nbp * BK * 16;
     __shared__ uint64_t b_full[MAX_STAGES], b_empty[MAX_STAGES], r_full[MAX_STAGES], r_empty[MAX_STAGES];
-    __shared__ uint64_t a_full[A_STAGES], a_empty[A_STAGES], acc_bar;
+    __shared__ uint64_t a_full[A_STAGES], a_empty[A_STAGES], acc_full, acc_empty, done_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int BS = p.b_stages, RS = p.r_stages;
     const int nk = (p.K + BK - 1) / BK;
-    const long long m_tile = blockIdx.x;
-    const int n_tile = blockIdx.y;
-    const long long b_first = (p.pg.pass_m0 + m_tile * BM) / p.pg.R_pass;
+    const int ntn = p.ntiles_n;
 
     if (threadIdx.x == 0) {
         abort_sh = 0;
@@ -208,10 +213,12 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             mbar_init(&a_full[s], 128);
             mbar_init(&a_empty[s], 1);
         }
-        mbar_init(&acc_bar, 1);
+        mbar_init(&acc_full, 1);
+        mbar_init(&acc_empty, 128);
+        mbar_init(&done_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) {
+    if (warp == W_RAW) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_sh)),
                      "r"(TMEM_COLS)
                      : "memory");
@@ -223,142 +230,195 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     const uint32_t tmem = tmem_base_sh;
     volatile int* abort_flag = &abort_sh;
 
-    if (warp == 0) {
+    if (warp == W_RAW) {
         if (lane == 0) {
-            // ----------------------------------------------------------- TMA producer
-            const int ya = (p.a_row_mode == 0) ? (int)(m_tile * BM) : (int)((p.a_m0 + m_tile * BM) % p.a_RA);
-            const int yb = n_tile * p.BN;
-            int r_issued = 0, b_issued = 0;
-            for (int kb = 0; kb < nk; ++kb) {
-                const int sr = kb % RS, sb = kb % BS;
-                if (kb >= RS && !mbar_wait(&r_empty[sr], ((kb / RS) - 1) & 1, abort_flag)) break;
-                mbar_expect_tx(&r_full[sr], TILE_A + pbytes);
-                tma_load_2d(base + p.r_off + sr * TILE_A, &tmA, &r_full[sr], kb * BK, ya);
-                tma_load_2d(base + p.p_off + sr * pbytes, &tmP, &r_full[sr], kb * BK * 4, (int)b_first);
-                r_issued = kb + 1;
-                if (kb >= BS && !mbar_wait(&b_empty[sb], ((kb / BS) - 1) & 1, abort_flag)) break;
-                uint8_t* bst = base + p.b_off + (size_t)sb * 2 * bbytes;
-                mbar_expect_tx(&b_full[sb], 2 * bbytes);
-                tma_load_2d(bst, &tmBhi, &b_full[sb], kb * BK, yb);
-                tma_load_2d(bst + bbytes, &tmBlo, &b_full[sb], kb * BK, yb);
-                b_issued = kb + 1;
-            }
-            if (*abort_flag) {  // drain copies still in flight before the CTA can exit
-                for (int kb = (r_issued > RS ? r_issued - RS : 0); kb < r_issued; ++kb) {
-                    const long long t0 = clock64();
-                    while (!mbar_test(&r_full[kb % RS], (kb / RS) & 1) && clock64() - t0 < WAIT_CYCLES) {
-                    }
-                }
-                for (int kb = (b_issued > BS ? b_issued - BS : 0); kb < b_issued; ++kb) {
-                    const long long t0 = clock64();
-                    while (!mbar_test(&b_full[kb % BS], (kb / BS) & 1) && clock64() - t0 < WAIT_CYCLES) {
-                    }
+            // ------------------------------------------- raw coefficient tiles + relaxation slices
+            long long g = 0;
+            for (long long t = blockIdx.x; t < p.ntiles && !*abort_flag; t += gridDim.x) {
+                const long long m_tile = t / ntn;
+                const int ya = (p.a_row_mode == 0) ? (int)(m_tile * BM) : (int)((p.a_m0 + m_tile * BM) % p.a_RA);
+                const int b_first = (int)((p.pg.pass_m0 + m_tile * BM) / p.pg.R_pass);
+                for (int kb = 0; kb < nk; ++kb, ++g) {
+                    const int sr = (int)(g % RS);
+                    if (g >= RS && !mbar_wait(&r_empty[sr], (uint32_t)((g / RS) - 1) & 1, abort_flag)) break;
+                    mbar_expect_tx(&r_full[sr], TILE_A + pbytes);
+                    tma_load_2d(base + p.r_off + sr * TILE_A, &tmA, &r_full[sr], kb * BK, ya);
+                    tma_load_2d(base + p.p_off + sr * pbytes, &tmP, &r_full[sr], kb * BK * 4, b_first);
                 }
             }
+            if (*abort_flag)  // drain: wait (bounded) for copies nobody will consume
+                for (long long h = (g > RS ? g - RS : 0); h < g; ++h) {
+                    const long long t0 = clock64();
+                    while (!mbar_test(&r_full[h % RS], (uint32_t)(h / RS) & 1) && clock64() - t0 < WAIT_CYCLES) {
+                    }
+                }
         }
-    } else if (warp == 1) {
+    } else if (warp == W_B) {
         if (lane == 0) {
-            // ----------------------------------------------------------- MMA issuer
+            // ------------------------------------------------------------ W^T head/remainder tiles
+            long long g = 0;
+            for (long long t = blockIdx.x; t < p.ntiles && !*abort_flag; t += gridDim.x) {
+                const int yb = (int)(t % ntn) * p.BN;
+                for (int kb = 0; kb < nk; ++kb, ++g) {
+                    const int sb = (int)(g % BS);
+                    if (g >= BS && !mbar_wait(&b_empty[sb], (uint32_t)((g / BS) - 1) & 1, abort_flag)) break;
+                    uint8_t* bst = base + p.b_off + (size_t)sb * 2 * bbytes;
+                    mbar_expect_tx(&b_full[sb], 2 * bbytes);
+                    tma_load_2d(bst, &tmBhi, &b_full[sb], kb * BK, yb);
+                    tma_load_2d(bst + bbytes, &tmBlo, &b_full[sb], kb * BK, yb);
+                }
+            }
+            if (*abort_flag)
+                for (long long h = (g > BS ? g - BS : 0); h < g; ++h) {
+                    const long long t0 = clock64();
+                    while (!mbar_test(&b_full[h % BS], (uint32_t)(h / BS) & 1) && clock64() - t0 < WAIT_CYCLES) {
+                    }
+                }
+        }
+    } else if (warp == W_MMA) {
+        if (lane == 0) {
+            // ------------------------------------------------------------------------ MMA issuer
             const uint32_t idesc = idesc_tf32(p.BN);
-            for (int kb = 0; kb < nk; ++kb) {
-                const int sa = kb % A_STAGES, sb = kb % BS;
-                if (!mbar_wait(&a_full[sa], (kb / A_STAGES) & 1, abort_flag)) break;
-                if (!mbar_wait(&b_full[sb], (kb / BS) & 1, abort_flag)) break;
+            long long g = 0, tiles_done = 0;
+            for (long long t = blockIdx.x; t < p.ntiles && !*abort_flag; t += gridDim.x, ++tiles_done) {
+                if (tiles_done > 0 && !mbar_wait(&acc_empty, (uint32_t)(tiles_done - 1) & 1, abort_flag)) break;
                 tc_fence_after();
-                uint8_t* bst = base + p.b_off + (size_t)sb * 2 * bbytes;
-                const uint64_t db_hi = sw128_desc(smem_u32(bst));
-                const uint64_t db_lo = sw128_desc(smem_u32(bst + bbytes));
-                const uint32_t ta_hi = tmem + 256 + sa * 64;
-                const uint32_t ta_lo = ta_hi + 32;
+                for (int kb = 0; kb < nk; ++kb, ++g) {
+                    const int sa = (int)(g % A_STAGES), sb = (int)(g % BS);
+                    if (!mbar_wait(&a_full[sa], (uint32_t)(g / A_STAGES) & 1, abort_flag)) break;
+                    if (!mbar_wait(&b_full[sb], (uint32_t)(g / BS) & 1, abort_flag)) break;
+                    tc_fence_after();
+                    uint8_t* bst = base + p.b_off + (size_t)sb * 2 * bbytes;
+                    const uint64_t db_hi = sw128_desc(smem_u32(bst));
+                    const uint64_t db_lo = sw128_desc(smem_u32(bst + bbytes));
+                    const uint32_t ta_hi = tmem + 256 + sa * 64;
+                    const uint32_t ta_lo = ta_hi + 32;
 #pragma unroll
-                for (int kk = 0; kk < BK / 8; ++kk) {
-                    const uint64_t off = (uint64_t)(kk * 32) >> 4;  // 8 tf32 = 32 bytes along K in smem
-                    const uint32_t first = (kb > 0 || kk > 0) ? 1u : 0u;
-                    mma_tf32_ts(tmem, ta_lo + kk * 8, db_hi + off, idesc, first);
-                    mma_tf32_ts(tmem, ta_hi + kk * 8, db_lo + off, idesc, 1u);
-                    mma_tf32_ts(tmem, ta_hi + kk * 8, db_hi + off, idesc, 1u);
+                    for (int kk = 0; kk < BK / 8; ++kk) {
+                        const uint64_t off = (uint64_t)(kk * 32) >> 4;  // 8 tf32 = 32 bytes along K in smem
+                        const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+                        mma_tf32_ts(tmem, ta_lo + kk * 8, db_hi + off, idesc, acc);
+                        mma_tf32_ts(tmem, ta_hi + kk * 8, db_lo + off, idesc, 1u);
+                        mma_tf32_ts(tmem, ta_hi + kk * 8, db_hi + off, idesc, 1u);
+                    }
+                    mma_commit(&a_empty[sa]);
+                    mma_commit(&b_empty[sb]);
                 }
-                mma_commit(&a_empty[sa]);
-                mma_commit(&b_empty[sb]);
+                mma_commit(&acc_full);
             }
-            mma_commit(&acc_bar);
-            const long long t0 = clock64();  // never free TMEM under MMAs still in flight
-            while (!mbar_test(&acc_bar, 0) && clock64() - t0 < WAIT_CYCLES) {
+            // never free TMEM under MMAs still in flight, even after an abort: one last commit
+            // tracks every MMA this thread issued
+            mma_commit(&done_bar);
+            const long long t0 = clock64();
+            while (!mbar_test(&done_bar, 0) && clock64() - t0 < WAIT_CYCLES) {
             }
         }
-    } else {
-        // ------------------------------------------------------------- transform + epilogue
+    } else if (warp < W_EPI0) {
+        // ------------------------------------------------------------------------- transform
         const int q = warp & 3;         // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;  // tile row owned by this thread (TMEM lane)
-        const long long m = m_tile * BM + row;
-        const bool valid = m < p.M;
-        const long long b = (p.pg.pass_m0 + m) / p.pg.R_pass;
-        const int cb = valid ? (int)(b - b_first) : 0;
-        const bool do_cst = (p.cst != nullptr) && n_tile == 0;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        float cacc = 0.f;
-        for (int kb = 0; kb < nk; ++kb) {
-            const int sr = kb % RS, sa = kb % A_STAGES;
-            bool ok = mbar_wait(&r_full[sr], (kb / RS) & 1, abort_flag);
-            float hi[32], lo[32];
-            if (ok) {
-                const float4* arow = reinterpret_cast<const float4*>(base + p.r_off + sr * TILE_A + row * 128);
-                const float4* prow = reinterpret_cast<const float4*>(base + p.p_off + sr * pbytes) + cb * BK;
+        long long g = 0;
+        for (long long t = blockIdx.x; t < p.ntiles; t += gridDim.x) {
+            const long long m_tile = t / ntn;
+            const int n_tile = (int)(t % ntn);
+            const long long m = m_tile * BM + row;
+            const bool valid = m < p.M;
+            const long long b = (p.pg.pass_m0 + m) / p.pg.R_pass;
+            const long long b_first = (p.pg.pass_m0 + m_tile * BM) / p.pg.R_pass;
+            const int cb = valid ? (int)(b - b_first) : 0;
+            float cacc = 0.f;
+            bool alive = true;
+            for (int kb = 0; kb < nk; ++kb, ++g) {
+                const int sr = (int)(g % RS), sa = (int)(g % A_STAGES);
+                bool ok = mbar_wait(&r_full[sr], (uint32_t)(g / RS) & 1, abort_flag);
+                float hi[32], lo[32];
+                if (ok) {
+                    const float4* arow = reinterpret_cast<const float4*>(base + p.r_off + sr * TILE_A + row * 128);
+                    const float4* prow = reinterpret_cast<const float4*>(base + p.p_off + sr * pbytes) + cb * BK;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float4 x = arow[c ^ (row & 7)];  // 128-byte swizzle of the TMA tile
-                    const float xv[4] = {x.x, x.y, x.z, x.w};
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 x = arow[c ^ (row & 7)];  // 128-byte swizzle of the TMA tile
+                        const float xv[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float4 pr = prow[c * 4 + j];
-                        const float v = xv[j];
-                        const float r = (v >= 0.f) ? v * pr.x : v * pr.y;
-                        if (p.count_const) cacc = fmaf(fminf(v, 0.f), pr.z, cacc);
-                        cacc = fmaf(r, pr.w, cacc);
-                        const float h = tf32_hi(r);
-                        hi[c * 4 + j] = h;
-                        lo[c * 4 + j] = r - h;
+                        for (int j = 0; j < 4; ++j) {
+                            const float4 pr = prow[c * 4 + j];
+                            const float v = xv[j];
+                            const float r = (v >= 0.f) ? v * pr.x : v * pr.y;
+                            if (p.count_const) cacc = fmaf(fminf(v, 0.f), pr.z, cacc);
+                            cacc = fmaf(r, pr.w, cacc);
+                            const float h = tf32_hi(r);
+                            hi[c * 4 + j] = h;
+                            lo[c * 4 + j] = r - h;
+                        }
                     }
+                    mbar_arrive(&r_empty[sr]);
+                    if (g >= A_STAGES) ok = mbar_wait(&a_empty[sa], (uint32_t)((g / A_STAGES) - 1) & 1, abort_flag);
                 }
-                mbar_arrive(&r_empty[sr]);
-                if (kb >= A_STAGES) ok = mbar_wait(&a_empty[sa], ((kb / A_STAGES) - 1) & 1, abort_flag);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    alive = false;
+                    break;
+                }
+                const uint32_t ta = tmem + lane_base + 256 + sa * 64;
+                tmem_st32(ta, hi);
+                tmem_st32(ta + 32, lo);
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tc_fence_before();
+                mbar_arrive(&a_full[sa]);
             }
-            if (!__all_sync(0xffffffffu, ok)) break;
-            const uint32_t ta = tmem + lane_base + 256 + sa * 64;
-            tmem_st32(ta, hi);
-            tmem_st32(ta + 32, lo);
-            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-            tc_fence_before();
-            mbar_arrive(&a_full[sa]);
+            if (!alive) break;
+            if (p.cst != nullptr && n_tile == 0 && valid) p.cst[m] += cacc;
         }
-        if (do_cst && valid && !*abort_flag) p.cst[m] += cacc;
-
-        // epilogue: accumulator rows from TMEM
-        const bool acc_ready = __all_sync(0xffffffffu, mbar_wait(&acc_bar, 0, abort_flag));
-        if (acc_ready) {
-            tc_fence_after();
+    } else {
+        // -------------------------------------------------------------------------- epilogue
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        float* stg = reinterpret_cast<float*>(base + p.s_off) + q * p.s_floats;
+        long long tiles_done = 0;
+        for (long long t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++tiles_done) {
+            const long long m_tile = t / ntn;
+            const int n_tile = (int)(t % ntn);
             const int n0 = n_tile * p.BN;
+            const long long m = m_tile * BM + row;
+            const bool valid = m < p.M;
+            const long long row0 = m_tile * BM + q * 32;  // first row of this warp
             if (p.out_mode == OUT_CONCRETIZE) {
+                // this warp's rows span centres bw .. bw + nbw - 1: stage their slice of the centres
+                const long long bw = (p.pg.pass_m0 + row0) / p.pg.R_pass;
+                for (int i = lane; i < p.nbw * p.BN; i += 32) {
+                    const long long bb = bw + i / p.BN;
+                    const int n = n0 + i % p.BN;
+                    stg[i] = (bb < p.B && n < p.N) ? __ldg(&p.centres[bb * p.N + n]) : 0.f;
+                }
+                __syncwarp();
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(&acc_full, (uint32_t)tiles_done & 1, abort_flag))) break;
+            tc_fence_after();
+            if (p.out_mode == OUT_CONCRETIZE) {
+                const long long b = (p.pg.pass_m0 + m) / p.pg.R_pass;
+                const long long bw = (p.pg.pass_m0 + row0) / p.pg.R_pass;
+                const float* crow = stg + (valid ? (int)(b - bw) : 0) * p.BN;
                 float conc = 0.f;
-                const float* crow = p.centres + (valid ? b : 0) * (long long)p.N;
                 for (int c0 = 0; c0 < p.BN; c0 += 32) {
                     float v[32];
                     tmem_ld32(tmem + lane_base + c0, v);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int n = n0 + c0 + j;
-                        if (valid && c0 + j < p.BN && n < p.N) conc += fmaf(v[j], __ldg(&crow[n]), -p.eps * fabsf(v[j]));
-                    }
+                    for (int j = 0; j < 32; ++j)
+                        if (c0 + j < p.BN && n0 + c0 + j < p.N) conc += fmaf(v[j], crow[c0 + j], -p.eps * fabsf(v[j]));
                 }
+                tc_fence_before();
+                mbar_arrive(&acc_empty);
                 if (valid) p.part[(long long)n_tile * p.M + m] = conc;
+                __syncwarp();  // the staged centres are reused by the next tile
             } else {
-                // stage each 32x32 block through smem (the raw-A ring is idle now) so that every
-                // warp store covers one contiguous 128-byte row segment
-                float* stg = reinterpret_cast<float*>(base + p.r_off) + q * (32 * 33);
-                const long long row0 = m_tile * BM + q * 32;
                 for (int c0 = 0; c0 < p.BN; c0 += 32) {
                     float v[32];
                     tmem_ld32(tmem + lane_base + c0, v);
+                    if (c0 + 32 >= p.BN) {  // accumulator fully read: hand TMEM back to the MMA
+                        tc_fence_before();
+                        mbar_arrive(&acc_empty);
+                    }
 #pragma unroll
                     for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = v[j];
                     __syncwarp();
@@ -381,7 +441,7 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == W_RAW) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
     }
@@ -463,18 +523,23 @@ cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, 
     p.B = B;
     p.BN = pick_bn(N, &p.ntiles_n);
     p.nbp = (int)std::min<long long>(centres_per_tile(pg.R_pass), B);
+    p.nbw = (int)std::min<long long>(31 / pg.R_pass + 2, B);
+    p.ntiles = ((M + BM - 1) / BM) * p.ntiles_n;
+    p.s_floats = std::max(32 * 33, p.nbw * p.BN);
+    const int sbytes = 4 * p.s_floats * 4;
     const int bstage = 2 * p.BN * BK * 4;
     const int rstage = TILE_A + p.nbp * BK * 16;
-    const int budget = 220 * 1024 - 1024;
+    const int budget = 220 * 1024 - 1024 - sbytes;
     p.b_stages = 2;
     p.r_stages = 2;
-    while (p.b_stages < 4 && (p.b_stages + 1) * bstage + p.r_stages * rstage <= budget) p.b_stages++;
+    while (p.b_stages < 4 && (p.b_stages + 1) * bstage + (p.r_stages + 1) * rstage <= budget) p.b_stages++;
     while (p.r_stages < MAX_STAGES && p.b_stages * bstage + (p.r_stages + 1) * rstage <= budget) p.r_stages++;
     if (p.b_stages * bstage + p.r_stages * rstage > budget) return cudaErrorInvalidValue;
     p.b_off = 0;
     p.r_off = p.b_stages * bstage;                        // multiple of 1024 (BN is a multiple of 16)
     p.p_off = p.r_off + p.r_stages * TILE_A;              // TILE_A is a multiple of 1024
-    const size_t smem = (size_t)p.p_off + (size_t)p.r_stages * p.nbp * BK * 16 + 1024;
+    p.s_off = p.p_off + p.r_stages * p.nbp * BK * 16;     // multiple of 512
+    const size_t smem = (size_t)p.s_off + sbytes + 1024;
     CUtensorMap ta, tp, tbh, tbl;
     long long a_rows;
     if (A.RA == kHugeRows) {
@@ -506,8 +571,14 @@ cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, 
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    dim3 grid((unsigned)((M + BM - 1) / BM), (unsigned)p.ntiles_n);
-    dense_back_tc<<<grid, NUM_THREADS, smem, s>>>(ta, tp, tbh, tbl, p);
+    static int num_sms = 0;
+    if (num_sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    const long long grid = std::min<long long>(p.ntiles, num_sms);  // persistent: one CTA per SM
+    dense_back_tc<<<(unsigned)grid, NUM_THREADS, smem, s>>>(ta, tp, tbh, tbl, p);
     return cudaGetLastError();
 }
 
