@@ -525,7 +525,8 @@ cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, 
     p.nbp = (int)std::min<long long>(centres_per_tile(pg.R_pass), B);
     p.nbw = (int)std::min<long long>(31 / pg.R_pass + 2, B);
     p.ntiles = ((M + BM - 1) / BM) * p.ntiles_n;
-    p.s_floats = std::max(32 * 33, p.nbw * p.BN);
+    // epilogue staging per warp: a 32x33 block for stores, or the centre rows for concretisation
+    p.s_floats = (out_mode == OUT_CONCRETIZE) ? p.nbw * p.BN : 32 * 33;
     const int sbytes = 4 * p.s_floats * 4;
     const int bstage = 2 * p.BN * BK * 4;
     const int rstage = TILE_A + p.nbp * BK * 16;
