@@ -181,6 +181,7 @@ struct TcParams {
 // Warp roles (11 warps): 0 raw-A/P producer + TMEM owner, 1 MMA issuer, 2-5 transform,
 // 6-9 epilogue, 10 W producer.
 constexpr int W_RAW = 0, W_MMA = 1, W_XF0 = 2, W_EPI0 = 6, W_B = 10;
+static_assert(W_EPI0 - W_XF0 == 4 && W_B == W_EPI0 + 4, "four transform and four epilogue warps");
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmP,
