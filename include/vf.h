@@ -155,6 +155,34 @@ enum { VF_KERNEL_ALL = 0, VF_KERNEL_DENSE_TC = 1, VF_KERNEL_DENSE_FFMA = 2, VF_K
 int vf_profile_enable(vf_net* net, int enable);
 int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms, double* flops, int reset);
 
+/* Size, in floats, of the fixed scratch array used by vf_concretize_dense_noalloc (16 MiB). */
+#define VF_NOALLOC_SCRATCH_FLOATS (1LL << 22)
+
+/* Concretised back-substitution through one dense layer, for callers that cannot allocate device
+ * memory: code whose device memory belongs to another allocator (a host framework's pool that forbids
+ * cudaMalloc), code under a fixed device-memory budget, and code that must avoid the device-wide
+ * synchronisation a cudaMalloc/cudaFree can cause. The page has no counterpart of this entry point; it
+ * is the same arithmetic as vf_crown_backward from the layer followed by vf_concretize, without a handle
+ * or workspace.
+ *
+ * Rows lambda [device] [B or 1, R, n_out] (centre stride lambda_bstride elements, 0 = shared) are
+ * coefficients over z = W x + b, W [device] [n_out, n_in], b [device] [n_out]; x ranges over the box
+ * centres[b] +/- eps, centres [device] [B, n_in]. Output lb [device] [B, R]:
+ *   lb[b, r] = sum_i (lambda_r W)_i centres[b, i] - eps * sum_i |(lambda_r W)_i| + lambda_r . b.
+ *
+ * Scratch: a file-scope __device__ array of VF_NOALLOC_SCRATCH_FLOATS floats that every GPU loading the
+ * library holds until exit; this call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine). It needs B*R*(1 + ceil(n_in / T)) floats with T = 64 for n_in <= 64, else 128; larger
+ * requests return VF_ERR_WORKSPACE without launching anything (split the rows into several calls).
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress, which may load
+ * the library's device code), so make that first call before any stream capture. All calls share the
+ * one array and it keeps the last call's contents (the row constants are cleared by each call): calls
+ * whose execution overlaps on the GPU -- on different streams, or from different threads -- race and
+ * must be serialised by the caller. Errors: VF_ERR_ARG, VF_ERR_NONFINITE (eps), VF_ERR_WORKSPACE,
+ * VF_ERR_CUDA, described by vf_last_error(). */
+int vf_concretize_dense_noalloc(const float* lambda, long long lambda_bstride, int R, const float* W, const float* b,
+                                const float* centres, float eps, int B, int n_in, int n_out, float* lb, void* stream);
+
 /* Number of kernel launches the library has enqueued on this handle since creation. */
 long long vf_launch_count(const vf_net* net);
 

@@ -616,6 +616,11 @@ int build_relax(vf_net* net, int B, const std::vector<const float*>& L, const st
 
 }  // namespace
 
+int vf::set_last_error(int code, const char* msg) {
+    g_err = msg;
+    return code;
+}
+
 // ===================================== C ABI ===============================================
 
 extern "C" {

@@ -100,4 +100,7 @@ cudaError_t launch_finite_scan(const float* p, long long n, int* flag, cudaStrea
 cudaError_t launch_concretize_api(const float* lambda, const float* cst, const float* centres, float eps, int B, int R,
                                   int n0, float* lb, cudaStream_t s);
 
+// Records `msg` as this thread's vf_last_error() text and returns `code`.
+int set_last_error(int code, const char* msg);
+
 }  // namespace vf

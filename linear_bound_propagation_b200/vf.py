@@ -24,7 +24,9 @@ VF_KERNEL_ALL, VF_KERNEL_DENSE_TC, VF_KERNEL_DENSE_FFMA, VF_KERNEL_CONV = range(
 
 SYMBOLS = ["vf_net_create", "vf_net_destroy", "vf_net_node_size", "vf_net_total_size", "vf_ibp",
            "vf_crown_backward", "vf_concretize", "vf_verify_batch", "vf_sync", "vf_last_error",
-           "vf_profile_enable", "vf_profile_read", "vf_launch_count", "vf_net_check"]
+           "vf_profile_enable", "vf_profile_read", "vf_launch_count", "vf_net_check",
+           "vf_concretize_dense_noalloc"]
+NOALLOC_SCRATCH_FLOATS = 1 << 22
 
 
 class VfError(RuntimeError):
@@ -74,6 +76,7 @@ def lib() -> ctypes.CDLL:
     L.vf_profile_read.argtypes = [P, I, ctypes.POINTER(LL), ctypes.POINTER(ctypes.c_double),
                                   ctypes.POINTER(ctypes.c_double), I]
     L.vf_net_check.argtypes = [P]
+    L.vf_concretize_dense_noalloc.argtypes = [P, LL, I, P, P, P, F, I, I, I, P, P]
     L.vf_launch_count.argtypes = [P]
     L.vf_launch_count.restype = LL
     _lib = L
@@ -245,6 +248,22 @@ def concretize(lam: torch.Tensor, cst: Optional[torch.Tensor], centres: torch.Te
     _check(lib().vf_concretize(_ptr(lam), _ptr(cst), _ptr(centres), float(eps), B, R, n0, _ptr(lb),
                                _stream_ptr(stream)))
     return lb
+
+
+def concretize_dense_noalloc(lam: torch.Tensor, W: torch.Tensor, b: torch.Tensor, centres: torch.Tensor, eps: float,
+                             out: Optional[torch.Tensor] = None, stream=None):
+    """vf_concretize_dense_noalloc: rows lam [B or 1, R, n_out] over z = W x + b, x in centres +/- eps.
+    The library allocates nothing for this call (its scratch is a fixed device array); `out` may be
+    passed to keep the call free of any allocation on the Python side too."""
+    B = centres.shape[0]
+    R = lam.shape[-2]
+    n_out, n_in = W.shape
+    bstride = 0 if lam.dim() == 2 or lam.shape[0] == 1 else R * n_out
+    if out is None:
+        out = torch.empty(B, R, device=centres.device)
+    _check(lib().vf_concretize_dense_noalloc(_ptr(lam), bstride, R, _ptr(W), _ptr(b), _ptr(centres), float(eps), B,
+                                             n_in, n_out, _ptr(out), _stream_ptr(stream)))
+    return out
 
 
 def sync(stream=None):
