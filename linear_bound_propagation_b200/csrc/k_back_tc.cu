@@ -108,8 +108,9 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
+// tcgen05.ld of 32 consecutive columns of this warp's 32 lanes, without waiting for completion
+// (issue several, then tmem_wait_ld once).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
         "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
@@ -118,10 +119,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
     asm volatile(
@@ -401,40 +400,62 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 const long long bw = (p.pg.pass_m0 + row0) / p.pg.R_pass;
                 const float* crow = stg + (valid ? (int)(b - bw) : 0) * p.BN;
                 float conc = 0.f;
-                for (int c0 = 0; c0 < p.BN; c0 += 32) {
-                    float v[32];
-                    tmem_ld32(tmem + lane_base + c0, v);
+                // 64 columns in flight per wait (2 loads of 32), then the arithmetic
+                for (int c0 = 0; c0 < p.BN; c0 += 64) {
+                    uint32_t v[2][32];
+                    tmem_ld32_nowait(tmem + lane_base + c0, v[0]);
+                    if (c0 + 32 < p.BN) tmem_ld32_nowait(tmem + lane_base + c0 + 32, v[1]);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (c0 + j < p.BN && n0 + c0 + j < p.N) conc += fmaf(v[j], crow[c0 + j], -p.eps * fabsf(v[j]));
+                    for (int u = 0; u < 2; ++u) {
+                        const int cu = c0 + 32 * u;
+                        if (cu >= p.BN) break;
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 cc = *reinterpret_cast<const float4*>(crow + cu + j);
+                            const float cv[4] = {cc.x, cc.y, cc.z, cc.w};
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj) {
+                                const float x = __uint_as_float(v[u][j + jj]);
+                                if (cu + j + jj < p.BN && n0 + cu + j + jj < p.N) conc += fmaf(x, cv[jj], -p.eps * fabsf(x));
+                            }
+                        }
+                    }
                 }
                 tc_fence_before();
                 mbar_arrive(&acc_empty);
                 if (valid) p.part[(long long)n_tile * p.M + m] = conc;
                 __syncwarp();  // the staged centres are reused by the next tile
             } else {
-                for (int c0 = 0; c0 < p.BN; c0 += 32) {
-                    float v[32];
-                    tmem_ld32(tmem + lane_base + c0, v);
-                    if (c0 + 32 >= p.BN) {  // accumulator fully read: hand TMEM back to the MMA
+                for (int c0 = 0; c0 < p.BN; c0 += 64) {
+                    uint32_t v[2][32];
+                    tmem_ld32_nowait(tmem + lane_base + c0, v[0]);
+                    if (c0 + 32 < p.BN) tmem_ld32_nowait(tmem + lane_base + c0 + 32, v[1]);
+                    tmem_wait_ld();
+                    if (c0 + 64 >= p.BN) {  // accumulator fully read: hand TMEM back to the MMA
                         tc_fence_before();
                         mbar_arrive(&acc_empty);
                     }
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = v[j];
-                    __syncwarp();
-                    const int n = n0 + c0 + lane;
-                    const bool col_ok = (c0 + lane < p.BN) && (n < p.N);
+                    for (int u = 0; u < 2; ++u) {
+                        const int cu = c0 + 32 * u;
+                        if (cu >= p.BN) break;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(v[u][j]);
+                        __syncwarp();
+                        const int n = n0 + cu + lane;
+                        const bool col_ok = (cu + lane < p.BN) && (n < p.N);
 #pragma unroll 4
-                    for (int j = 0; j < 32; ++j) {
-                        const long long mr = row0 + j;
-                        if (col_ok && mr < p.M) {
-                            float* o = p.out + mr * p.ld_out + n;
-                            const float val = stg[j * 33 + lane];
-                            *o = (p.out_mode == OUT_ACCUM) ? (*o + val) : val;
+                        for (int j = 0; j < 32; ++j) {
+                            const long long mr = row0 + j;
+                            if (col_ok && mr < p.M) {
+                                float* o = p.out + mr * p.ld_out + n;
+                                const float val = stg[j * 33 + lane];
+                                *o = (p.out_mode == OUT_ACCUM) ? (*o + val) : val;
+                            }
                         }
+                        __syncwarp();
                     }
-                    __syncwarp();
                 }
             }
         }

@@ -13,64 +13,75 @@ namespace vf {
 
 namespace {
 
-// z[m, n] = sum_k h[m, k] * W[n, k] for centre (W) and radius (|W|) at once; 64x64 tiles.
+// z[m, n] = sum_k h[m, k] * W[n, k]: blockIdx.z = 0 computes the centre (h = centre, W, + bias), 1 the
+// radius (h = radius, |W|). Tiles of 16 rows x 64 columns, 256 threads (one row x 4 columns each), the next
+// k-slice prefetched into registers while the current one is used. With rowsum_abs != nullptr the source is
+// the input box with radius eps in every coordinate: the radius is eps * sum_k |W[n, k]| without a product.
 __global__ void __launch_bounds__(256)
 ibp_dense_k(const float* __restrict__ hc, const float* __restrict__ hr, const float* __restrict__ W,
-            const float* __restrict__ Wabs, const float* __restrict__ bias, int B, int K, int N, float* __restrict__ zc,
-            float* __restrict__ zr) {
-    constexpr int T = 64, KB = 16;
-    __shared__ float Ac[KB][T + 1], Ar[KB][T + 1], Bw[KB][T + 1], Ba[KB][T + 1];
+            const float* __restrict__ Wabs, const float* __restrict__ bias, const float* __restrict__ rowsum_abs,
+            float eps, int B, int K, int N, float* __restrict__ zc, float* __restrict__ zr) {
+    constexpr int TM = 16, TN = 64, KB = 32;
+    __shared__ float As[KB][TM + 1], Bs[KB][TN + 1];
     const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
-    const int m0 = blockIdx.x * T, n0 = blockIdx.y * T;
-    float ac[4][4], ar[4][4];
+    const int m0 = blockIdx.x * TM, n0 = blockIdx.y * TN;
+    const bool rad = blockIdx.z == 1;
+    if (rad && rowsum_abs != nullptr) {
+        const int m = m0 + ty;
+        for (int j = 0; j < 4; ++j) {
+            const int n = n0 + tx + 16 * j;
+            if (m < B && n < N) zr[(long long)m * N + n] = eps * rowsum_abs[n];
+        }
+        return;
+    }
+    const float* h = rad ? hr : hc;
+    const float* w = rad ? Wabs : W;
+    float a_reg[2], b_reg[8];
+    auto load = [&](int k0) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 2; ++i) {
+            const int e = tid + 256 * i, row = e / KB, kk = e % KB, m = m0 + row, k = k0 + kk;
+            a_reg[i] = (m < B && k < K) ? h[(long long)m * K + k] : 0.f;
+        }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) ac[i][j] = ar[i][j] = 0.f;
+        for (int i = 0; i < 8; ++i) {
+            const int e = tid + 256 * i, row = e / KB, kk = e % KB, n = n0 + row, k = k0 + kk;
+            b_reg[i] = (n < N && k < K) ? w[(long long)n * K + k] : 0.f;
+        }
+    };
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    load(0);
     for (int k0 = 0; k0 < K; k0 += KB) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 2; ++i) {
             const int e = tid + 256 * i;
-            const int row = e / KB, kk = e % KB, k = k0 + kk;
-            const int m = m0 + row, n = n0 + row;
-            const bool mk = (m < B) && (k < K), nk = (n < N) && (k < K);
-            Ac[kk][row] = mk ? hc[(long long)m * K + k] : 0.f;
-            Ar[kk][row] = mk ? hr[(long long)m * K + k] : 0.f;
-            Bw[kk][row] = nk ? W[(long long)n * K + k] : 0.f;
-            Ba[kk][row] = nk ? Wabs[(long long)n * K + k] : 0.f;
+            As[e % KB][e / KB] = a_reg[i];
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = tid + 256 * i;
+            Bs[e % KB][e / KB] = b_reg[i];
         }
         __syncthreads();
+        if (k0 + KB < K) load(k0 + KB);
 #pragma unroll
         for (int kk = 0; kk < KB; ++kk) {
-            float a_c[4], a_r[4], b_w[4], b_a[4];
+            const float a = As[kk][ty];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                a_c[i] = Ac[kk][ty + 16 * i];
-                a_r[i] = Ar[kk][ty + 16 * i];
-                b_w[i] = Bw[kk][tx + 16 * i];
-                b_a[i] = Ba[kk][tx + 16 * i];
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    ac[i][j] = fmaf(a_c[i], b_w[j], ac[i][j]);
-                    ar[i][j] = fmaf(a_r[i], b_a[j], ar[i][j]);
-                }
+            for (int j = 0; j < 4; ++j) acc[j] = fmaf(a, Bs[kk][tx + 16 * j], acc[j]);
         }
         __syncthreads();
     }
+    const int m = m0 + ty;
+    if (m >= B) return;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int m = m0 + ty + 16 * i;
-        if (m >= B) continue;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int n = n0 + tx + 16 * j;
-            if (n >= N) continue;
-            zc[(long long)m * N + n] = ac[i][j] + bias[n];
-            zr[(long long)m * N + n] = ar[i][j];
-        }
+    for (int j = 0; j < 4; ++j) {
+        const int n = n0 + tx + 16 * j;
+        if (n >= N) continue;
+        if (rad)
+            zr[(long long)m * N + n] = acc[j];
+        else
+            zc[(long long)m * N + n] = acc[j] + bias[n];
     }
 }
 
@@ -148,9 +159,10 @@ unsigned grid_for(long long n, int threads) {
 }  // namespace
 
 cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
-                             int B, int K, int N, float* zc, float* zr, cudaStream_t s) {
-    dim3 grid((B + 63) / 64, (N + 63) / 64);
-    ibp_dense_k<<<grid, 256, 0, s>>>(hc, hr, W, Wabs, bias, B, K, N, zc, zr);
+                             const float* rowsum_abs, float eps, int B, int K, int N, float* zc, float* zr,
+                             cudaStream_t s) {
+    dim3 grid((B + 15) / 16, (N + 63) / 64, 2);
+    ibp_dense_k<<<grid, 256, 0, s>>>(hc, hr, W, Wabs, bias, rowsum_abs, eps, B, K, N, zc, zr);
     return cudaGetLastError();
 }
 

@@ -73,6 +73,7 @@ struct Node {
     float* pmW = nullptr;  // dense only: [W; -W], the rows of the identity-trick first step
     float* WtHi = nullptr; // dense only: W^T [n_in, n_out] truncated to tf32 (3xTF32 head)
     float* WtLo = nullptr; // dense only: W^T - WtHi (3xTF32 remainder)
+    float* rowsum_abs = nullptr;  // dense only: sum_k |W[n, k]| (IBP radius of a layer fed by the input box)
     int consumers = 0;
 };
 
@@ -507,8 +508,8 @@ int run_ibp(vf_net* net, const float* centres, int B, float eps, Arena& ar, IbpS
         const int sv = nd.src;
         switch (nd.op) {
             case VF_DENSE:
-                LAUNCH(net, launch_ibp_dense(st.c[sv], st.r[sv], nd.W, nd.Wabs, nd.b, B, (int)net->nodes[sv].n,
-                                             (int)nd.n, st.c[v], st.r[v], s));
+                LAUNCH(net, launch_ibp_dense(st.c[sv], st.r[sv], nd.W, nd.Wabs, nd.b, sv == 0 ? nd.rowsum_abs : nullptr,
+                                             eps, B, (int)net->nodes[sv].n, (int)nd.n, st.c[v], st.r[v], s));
                 break;
             case VF_CONV2D:
                 LAUNCH(net, launch_ibp_conv(st.c[sv], st.r[sv], nd.W, nd.Wabs, nd.b, B, conv_geom(net, nd), st.c[v],
@@ -653,6 +654,7 @@ void vf_net_destroy(vf_net* net) {
         cudaFree(nd.pmW);
         cudaFree(nd.WtHi);
         cudaFree(nd.WtLo);
+        cudaFree(nd.rowsum_abs);
     }
     cudaFree(net->d_err);
     for (auto e : net->ev_free) cudaEventDestroy(e);
@@ -713,6 +715,17 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
                 TRY(upload(x.W, cnt, false, &nd.W, host));
                 TRY(upload(x.W, cnt, true, &nd.Wabs, host));
                 TRY(upload(x.b, nd.n, false, &nd.b, host));
+                {  // row sums of |W| (host copy of W is still in `host` from the |W| upload above)
+                    std::vector<float> rs((size_t)nd.n, 0.f), wabs((size_t)cnt);
+                    CU(cudaMemcpy(wabs.data(), nd.Wabs, sizeof(float) * cnt, cudaMemcpyDeviceToHost));
+                    for (long long o = 0; o < nd.n; ++o) {
+                        float acc = 0.f;
+                        for (long long i = 0; i < s.n; ++i) acc += wabs[o * s.n + i];
+                        rs[o] = acc;
+                    }
+                    CU(cudaMalloc(&nd.rowsum_abs, sizeof(float) * nd.n));
+                    CU(cudaMemcpy(nd.rowsum_abs, rs.data(), sizeof(float) * nd.n, cudaMemcpyHostToDevice));
+                }
                 // [W; -W] for the first step of a pass that starts at this node
                 std::vector<float> pm((size_t)(2 * cnt));
                 CU(cudaMemcpy(pm.data(), nd.W, sizeof(float) * cnt, cudaMemcpyDeviceToHost));

@@ -62,8 +62,10 @@ cudaError_t launch_conv_back(const RowRef& A, Relax rx, const float* W, const fl
                              const float* centres, float eps, int num_sms, cudaStream_t s);
 
 // ---- IBP (k_ibp.cu) -------------------------------------------------------------------
+// rowsum_abs (optional): sum_k |W[n, k]|, used with `eps` when the source is the input box (radius eps everywhere).
 cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
-                             int B, int K, int N, float* zc, float* zr, cudaStream_t s);
+                             const float* rowsum_abs, float eps, int B, int K, int N, float* zc, float* zr,
+                             cudaStream_t s);
 cudaError_t launch_ibp_conv(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
                             int B, const ConvGeom& g, float* zc, float* zr, cudaStream_t s);
 cudaError_t launch_ibp_relu(const float* c, const float* r, long long n, float* oc, float* orad, cudaStream_t s);
