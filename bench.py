@@ -220,7 +220,7 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    w = synth.workload(args.config)
+    w = synth.workload(args.config, B=args.centres)
     B, R = w.centres.shape[0], w.C.shape[1]
     Rs = R * (2 if w.both_sides else 1)
     net = vf.Net(w.net, workspace_bytes=int(args.workspace_gb * (1 << 30)))
@@ -273,7 +273,7 @@ def run_ours(args):
     h_ver = torch.empty(B, R, dtype=torch.uint8).pin_memory()
     d_c = torch.empty_like(centres)
     d_C = torch.empty_like(C)
-    for _ in range(2):
+    for _ in range(0 if args.no_e2e else 2):
         d_c.copy_(h_centres, non_blocking=True)
         d_C.copy_(h_C, non_blocking=True)
         net.verify(d_c, w.eps, d_C, **kw)
@@ -282,7 +282,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = 0.0
-    for i in range(args.steps):
+    for i in range(0 if args.no_e2e else args.steps):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -304,7 +304,7 @@ def run_ours(args):
                 "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": workload_config(w, args.config), "roofline": roof,
-                "e2e": {"value": weak_throughput(world, B * Rs, args.steps, e2e_ms), "unit": UNIT,
+                "e2e": None if args.no_e2e else {"value": weak_throughput(world, B * Rs, args.steps, e2e_ms), "unit": UNIT,
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches, "clocks": clocks, "verified_specs": verified, "total_specs": B * Rs}
         if world == 1 and not args.no_cpu_baseline:
@@ -325,6 +325,9 @@ def main():
     ap.add_argument("--workspace-gb", type=float, default=16.0)
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--centres", type=int, default=None,
+                    help="use only the first N centres of the workload (profiling captures of a small case)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-staged end-to-end leg")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

@@ -168,6 +168,14 @@ __global__ void finish_rows_k(const float* __restrict__ cst, const float* __rest
     }
 }
 
+__global__ void add_partials_k(float* __restrict__ cst, const float* __restrict__ part, int ntiles, long long M) {
+    GRID_STRIDE(m, M) {
+        float v = 0.f;
+        for (int t = 0; t < ntiles; ++t) v += part[(long long)t * M + m];
+        cst[m] += v;
+    }
+}
+
 // Intermediate bounds after a pass over node p (rows [I; -I] per centre): IBP-unstable neurons
 // take l = max(l, lb_j), u = min(u, -lb_{n + j}); IBP-stable ones keep their (exact) relaxation.
 __global__ void intersect_k(float* __restrict__ l, float* __restrict__ u, const float* __restrict__ pass_out, int B,
@@ -302,6 +310,11 @@ cudaError_t launch_concretize_rows(const RowRef& A, long long M, int n0, PassGeo
 cudaError_t launch_finish_rows(const float* cst, const float* part, int ntiles, long long M, float* out,
                                cudaStream_t s) {
     finish_rows_k<<<grid_for(M, 256), 256, 0, s>>>(cst, part, ntiles, M, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_add_partials(float* cst, const float* part, int ntiles, long long M, cudaStream_t s) {
+    add_partials_k<<<grid_for(M, 256), 256, 0, s>>>(cst, part, ntiles, M);
     return cudaGetLastError();
 }
 

@@ -413,13 +413,15 @@ struct Walker {
                 long long ld = 0;
                 int mode = OUT_CONCRETIZE;
                 if (!fuse) TRY(target(nd.src, &out, &ld, &mode));
+                if (fuse) part_tiles = conv_back_tiles(g);
                 if (!dry) {
                     cudaEvent_t e0 = nullptr;
                     prof_begin(&e0);
-                    LAUNCH(net, launch_conv_back(e.ref, e.rx, nd.W, nd.b, M, g, pg, mode, out, ld, cst, centres, eps,
+                    LAUNCH(net, launch_conv_back(e.ref, e.rx, nd.W, nd.b, M, g, pg, mode, out, ld, part, centres, eps,
                                                  net->num_sms, s));
                     prof_end(e0, VF_KERNEL_CONV, 2.0 * (double)M * (double)net->nodes[nd.src].n * (double)g.co * g.k *
                                                      g.k / ((double)g.stride * g.stride));
+                    if (!fuse) LAUNCH(net, launch_add_partials(cst, part, conv_back_tiles(g), M, s));
                 }
                 release(e);
                 return VF_OK;
@@ -554,7 +556,9 @@ int run_pass(vf_net* net, int start, Entry init, long long rows, long long R_pas
     int nb = 0;
     TRY(pool_size(net, start, init, &relax, ext, &nb));
     const long long nmax = (max_node_size(net, input_buffered(net)) + 31) / 32 * 32;  // 128-byte rows
-    const int tiles = std::max(dense_back_tiles_n((int)net->nodes[0].n), dense_back_tc_tiles_n((int)net->nodes[0].n));
+    int tiles = std::max(dense_back_tiles_n((int)net->nodes[0].n), dense_back_tc_tiles_n((int)net->nodes[0].n));
+    for (size_t v = 1; v < net->nodes.size(); ++v)  // per-tile partials of every convolution step
+        if (net->nodes[v].op == VF_CONV2D) tiles = std::max(tiles, conv_back_tiles(conv_geom(net, net->nodes[v])));
     Arena a2 = ar;
     const size_t per_row = sizeof(float) * (1 + (size_t)tiles + (size_t)nb * nmax) + 64;
     long long chunk = (long long)(a2.left() / per_row);
@@ -773,8 +777,10 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
                 TRY(upload(x.W, cnt, true, &nd.Wabs, host));
                 TRY(upload(x.b, nd.c, false, &nd.b, host));
                 ConvGeom g = conv_geom(net, nd);
-                if (conv_back_smem_bytes(g) > 220 * 1024)
-                    return fail(VF_ERR_UNSUPPORTED, "node %d: convolution too large for one CTA's shared memory", v);
+                if (!conv_back_supported(g))
+                    return fail(VF_ERR_UNSUPPORTED,
+                                "node %d: convolution geometry not supported (stride 1/2/4, pad <= k-1, output covered "
+                                "by the input, staged tile within shared memory)", v);
                 break;
             }
             case VF_RELU:

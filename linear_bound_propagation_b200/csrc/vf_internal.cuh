@@ -54,11 +54,14 @@ cudaError_t launch_dense_back(const RowRef& A, Relax rx, const float* W, const f
                               int N, PassGeom pg, int out_mode, float* out, long long ld_out, float* cst,
                               const float* centres, float eps, float* part, cudaStream_t s);
 
-// Transposed convolution of relaxed rows over the conv output back onto its input.
-// cst[m] += relax const + bias term; OUT_CONCRETIZE adds the concretised row to cst[m].
+// Transposed convolution of relaxed rows over the conv output back onto its input. Writes per-tile
+// partials cpart[tile * M + m] (tile < conv_back_tiles(g)) holding the row-constant terms the tile owns
+// and, with OUT_CONCRETIZE, the tile's concretised outputs; launch_add_partials folds them into cst.
 size_t conv_back_smem_bytes(const ConvGeom& g);
+int conv_back_tiles(const ConvGeom& g);
+bool conv_back_supported(const ConvGeom& g);
 cudaError_t launch_conv_back(const RowRef& A, Relax rx, const float* W, const float* bias, long long M,
-                             const ConvGeom& g, PassGeom pg, int out_mode, float* out, long long ld_out, float* cst,
+                             const ConvGeom& g, PassGeom pg, int out_mode, float* out, long long ld_out, float* cpart,
                              const float* centres, float eps, int num_sms, cudaStream_t s);
 
 // ---- IBP (k_ibp.cu) -------------------------------------------------------------------
@@ -91,6 +94,8 @@ cudaError_t launch_concretize_rows(const RowRef& A, long long M, int n0, PassGeo
                                    float* cst, cudaStream_t s);
 cudaError_t launch_finish_rows(const float* cst, const float* part, int ntiles, long long M, float* out,
                                cudaStream_t s);
+// cst[m] += sum_{t < ntiles} part[t * M + m], in increasing t.
+cudaError_t launch_add_partials(float* cst, const float* part, int ntiles, long long M, cudaStream_t s);
 cudaError_t launch_intersect(float* l, float* u, const float* l_ibp, const float* u_ibp, const float* pass_out,
                              int B, long long n, cudaStream_t s);
 cudaError_t launch_spec_rows(const float* C, long long C_bstride, int BC, int R, int nL, float* S, cudaStream_t s);
