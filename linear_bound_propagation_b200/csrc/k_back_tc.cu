@@ -175,6 +175,7 @@ struct TcParams {
     float* part;
     int count_const;
     int* err;
+    int test_stall;  // test hook: CTA 0 never issues its first raw-tile copy, so a bounded wait expires
 };
 
 // Warp roles (11 warps): 0 raw-A/P producer + TMEM owner, 1 MMA issuer, 2-5 transform,
@@ -241,6 +242,7 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 for (int kb = 0; kb < nk; ++kb, ++g) {
                     const int sr = (int)(g % RS);
                     if (g >= RS && !mbar_wait(&r_empty[sr], (uint32_t)((g / RS) - 1) & 1, abort_flag)) break;
+                    if (p.test_stall && blockIdx.x == 0 && g == 0) continue;  // copy never issued (test hook)
                     mbar_expect_tx(&r_full[sr], TILE_A + pbytes);
                     tma_load_2d(base + p.r_off + sr * TILE_A, &tmA, &r_full[sr], kb * BK, ya);
                     tma_load_2d(base + p.p_off + sr * pbytes, &tmP, &r_full[sr], kb * BK * 4, b_first);
@@ -248,6 +250,7 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             }
             if (*abort_flag)  // drain: wait (bounded) for copies nobody will consume
                 for (long long h = (g > RS ? g - RS : 0); h < g; ++h) {
+                    if (p.test_stall && blockIdx.x == 0 && h == 0) continue;  // never issued
                     const long long t0 = clock64();
                     while (!mbar_test(&r_full[h % RS], (uint32_t)(h / RS) & 1) && clock64() - t0 < WAIT_CYCLES) {
                     }
@@ -536,7 +539,8 @@ bool dense_back_tc_supported(const RowRef& A, Relax rx, long long M, int K, int 
 
 cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, const float* Wt_lo, long long B,
                                  long long M, int K, int N, PassGeom pg, int out_mode, float* out, long long ld_out,
-                                 float* cst, const float* centres, float eps, float* part, int* err, cudaStream_t s) {
+                                 float* cst, const float* centres, float eps, float* part, int* err, int test_stall,
+                                 cudaStream_t s) {
     if (M <= 0) return cudaSuccess;
     TcParams p{};
     p.M = M;
@@ -588,6 +592,7 @@ cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, 
     p.part = part;
     p.count_const = rx.count_const;
     p.err = err;
+    p.test_stall = test_stall;
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(dense_back_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);

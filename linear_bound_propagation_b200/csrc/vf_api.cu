@@ -90,6 +90,7 @@ struct vf_net {
     long long fail_at = 0;  // test hook: VF_TEST_FAIL_AT=<n> fails the n-th launch on the host
     int dense_kernel = 0;   // 0: tensor cores where the shapes allow, 1: FFMA only (VF_DENSE_KERNEL=ffma)
     int* d_err = nullptr;   // device flag raised by a kernel whose bounded wait expired
+    int tc_stall = 0;       // test hook: VF_TEST_TC_STALL=1 makes one tensor-core launch time out
     bool prof = false;
     std::vector<cudaEvent_t> ev_free;
     struct Timed {
@@ -383,10 +384,12 @@ struct Walker {
                 if (!dry) {
                     cudaEvent_t e0 = nullptr;
                     prof_begin(&e0);
-                    if (tc)
+                    if (tc) {
                         LAUNCH(net, launch_dense_back_tc(e.ref, e.rx, nd.WtHi, nd.WtLo, n_centres, M, (int)nd.n, (int)sn.n, pg,
-                                                         mode, out, ld, cst, centres, eps, part, net->d_err, s));
-                    else
+                                                         mode, out, ld, cst, centres, eps, part, net->d_err,
+                                                         net->tc_stall, s));
+                        net->tc_stall = 0;  // the test hook withholds one copy, once
+                    } else
                         LAUNCH(net, launch_dense_back(e.ref, e.rx, nd.W, nd.b, M, (int)nd.n, (int)sn.n, pg, mode, out,
                                                       ld, cst, centres, eps, part, s));
                     prof_end(e0, tc ? VF_KERNEL_DENSE_TC : VF_KERNEL_DENSE_FFMA, 2.0 * (double)M * (double)nd.n * (double)sn.n);
@@ -687,6 +690,7 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
     CU(cudaDeviceGetAttribute(&net->num_sms, cudaDevAttrMultiProcessorCount, net->device));
     if (const char* f = getenv("VF_TEST_FAIL_AT")) net->fail_at = atoll(f);
     if (const char* f = getenv("VF_DENSE_KERNEL")) net->dense_kernel = (strcmp(f, "ffma") == 0) ? 1 : 0;
+    if (const char* f = getenv("VF_TEST_TC_STALL")) net->tc_stall = atoi(f) != 0;
     CU(cudaMalloc(&net->d_err, sizeof(int)));
     CU(cudaMemset(net->d_err, 0, sizeof(int)));
     net->nodes.resize(n_nodes);

@@ -11,9 +11,11 @@ bool dense_back_tc_supported(const RowRef& A, Relax rx, long long M, int K, int 
 int dense_back_tc_tiles_n(int N);
 // Wt_hi / Wt_lo: the node's W transposed to [N, K] (K contiguous) and split into tf32 head and
 // fp32 remainder; B = number of centres (rows of rx.P). Same outputs as launch_dense_back, with
-// the bias taken from rx.P[.].w; *err is set if a bounded wait expires.
+// the bias taken from rx.P[.].w; *err is set if a bounded wait expires. test_stall != 0 (tests only)
+// withholds one copy in CTA 0 so that its bounded wait expires and the abort path runs.
 cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, const float* Wt_lo, long long B,
                                  long long M, int K, int N, PassGeom pg, int out_mode, float* out, long long ld_out,
-                                 float* cst, const float* centres, float eps, float* part, int* err, cudaStream_t s);
+                                 float* cst, const float* centres, float eps, float* part, int* err, int test_stall,
+                                 cudaStream_t s);
 
 }  // namespace vf

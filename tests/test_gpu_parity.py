@@ -217,3 +217,21 @@ def test_host_fault_injection(monkeypatch):
     out = g2.verify(_dev(w.centres), w.eps, _dev(w.C))
     vf.sync()
     assert torch.isfinite(out["lb"]).all()
+
+
+def test_bounded_wait_expiry_is_reported_and_context_survives(monkeypatch):
+    """A tensor-core launch whose copy is withheld (test hook) gives up its bounded wait after about
+    two seconds of clock, frees its resources and raises the device flag: vf_net_check reports
+    VF_ERR_TIMEOUT. The context stays usable: a fresh handle then matches the oracle."""
+    w = synth.workload(2, B=4)
+    monkeypatch.setenv("VF_TEST_TC_STALL", "1")
+    g = vf.Net(w.net)
+    g.verify(_dev(w.centres), w.eps, _dev(w.C))
+    torch.cuda.synchronize()
+    with pytest.raises(vf.VfError) as e:
+        g.check()
+    assert e.value.code == vf.VF_ERR_TIMEOUT
+    g.check()  # the flag was cleared by the first check
+    monkeypatch.delenv("VF_TEST_TC_STALL")
+    g2, ora, out = run_both(w.net, w.centres, w.eps, w.C)
+    assert_parity(w.net, w.centres, w.eps, w.C, g2, ora, out)
