@@ -135,6 +135,28 @@ typedef struct {
 int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
                     const vf_opts* opts, float* lb, float* ub, float* lb_ibp, uint8_t* verified, void* stream);
 
+/* alpha-CROWN (technical summary, section 1: alpha-CROWN; sections 3 and 4.3: the per-neuron alpha
+ * tensors, i.e. the lower ReLU slopes): tightens the CROWN lower bounds of the specification rows by
+ * optimising, separately for every (centre, row), the lower slope of each unstable ReLU (0 < u/(u-l) < 1)
+ * within [0, 1], by `iters` steps of projected gradient ascent with Adam (betas 0.9, 0.999, step `lr`)
+ * from the adaptive slopes. Intermediate bounds are computed as in vf_verify_batch (opts->relu_crown,
+ * opts->alpha) and stay fixed. Any slope in [0, 1] gives a sound bound, so every iterate is sound.
+ * Networks: dense ReLU chains (input, dense, relu, ..., dense); others return VF_ERR_UNSUPPORTED, as
+ * does opts->both_sides (pass -C for upper bounds).
+ * Outputs [device]: lb [B, R] the best CROWN lower bound over the iterates (not intersected with IBP);
+ * lb_start [B, R] (or NULL) the bound at the adaptive start; alpha_out (or NULL) the final slopes, one
+ * [B, R, n_v] block per ReLU node v in node order. C [device] [B or 1, R, n_L] with centre stride C_bstride. */
+int vf_alpha_crown(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
+                   const vf_opts* opts, int iters, float lr, float* lb, float* lb_start, float* alpha_out,
+                   void* stream);
+
+/* The specification rows' CROWN lower bounds at given per-row slopes alpha [device] (layout of
+ * vf_alpha_crown's alpha_out; entries of stable neurons are ignored) and their gradient with respect to
+ * those slopes, grad [device] (same layout; zero for stable neurons and where the coefficient over the
+ * ReLU output is negative). Same networks and options as vf_alpha_crown. */
+int vf_alpha_grad(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
+                  const vf_opts* opts, const float* alpha, float* lb, float* grad, void* stream);
+
 /* Synchronise `stream` and report any pending asynchronous CUDA error. */
 int vf_sync(void* stream);
 

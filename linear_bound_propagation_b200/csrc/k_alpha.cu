@@ -1,0 +1,177 @@
+// alpha-CROWN: per-row lower ReLU slopes for the specification bound, their gradient and the Adam
+// ascent step.
+//
+// Page: "Scaling Neural Network Verification with Tensor Parallelism and Fully Sharded Data
+// Parallelism", technical summary §1 (alpha-CROWN among the bound-propagation methods) and §3 / §4.3
+// (the per-neuron alpha tensors, i.e. the lower ReLU slopes, that alpha-CROWN optimises).
+//
+// For a specification row the bound is a function of the lower slopes of the unstable neurons
+// (0 < up < 1). Back-substitution applies, at each ReLU, lam_z = slope * lam_h with slope = alpha for
+// lam_h >= 0 (unstable neurons) and the intercept term min(lam_h, 0) * t. Its gradient runs the chain in
+// the other direction: at the input G = c - eps * sign(lam_in); through a dense node G_z = G_h W^T + b;
+// at a ReLU d lb / d alpha_i = G_z,i * lam_h,i for lam_h,i >= 0 (unstable i), and
+// G_h = G_z * slope + [lam_h < 0] * t.
+#include <math.h>
+
+#include "vf_internal.cuh"
+
+namespace vf {
+
+namespace {
+
+unsigned grid_for(long long n, int threads) {
+    long long g = (n + threads - 1) / threads;
+    if (g > 148LL * 32) g = 148LL * 32;
+    return (unsigned)(g < 1 ? 1 : g);
+}
+
+__device__ __forceinline__ bool unstable(const float4& p) { return p.y > 0.f && p.y < 1.f; }
+
+__device__ __forceinline__ float block_sum256(float v, float* red) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float t = 0.f;
+    if (threadIdx.x == 0)
+        for (int i = 0; i < 8; ++i) t += red[i];
+    __syncthreads();
+    return t;
+}
+
+// Z[m, :] = slope * H[m, :] with per-row slopes for unstable neurons (alpha == nullptr: the table's
+// own lower slope); cst[m] += sum min(H, 0) * t + Z * bias (bias in P.w). One CTA per row.
+__global__ void __launch_bounds__(256)
+relax_alpha_rows_k(const float* __restrict__ H, long long M, int n, const float4* __restrict__ P, PassGeom pg,
+                   const float* __restrict__ alpha, float* __restrict__ Z, float* __restrict__ cst) {
+    __shared__ float red[8];
+    for (long long m = blockIdx.x; m < M; m += gridDim.x) {
+        const long long b = (pg.pass_m0 + m) / pg.R_pass;
+        const float* h = H + m * n;
+        float* z = Z + m * n;
+        float cs = 0.f;
+        for (int i = threadIdx.x; i < n; i += 256) {
+            const float x = h[i];
+            const float4 p = P[b * n + i];
+            const float lo = (alpha != nullptr && unstable(p)) ? alpha[m * n + i] : p.x;
+            const float r = (x >= 0.f) ? x * lo : x * p.y;
+            cs = fmaf(fminf(x, 0.f), p.z, cs);
+            cs = fmaf(r, p.w, cs);
+            z[i] = r;
+        }
+        const float t = block_sum256(cs, red);
+        if (threadIdx.x == 0) cst[m] += t;
+    }
+}
+
+// lb[m] = cst[m] + lam . c - eps |lam|_1 and G[m, i] = c_i - eps * sign(lam_i). One warp per row.
+__global__ void __launch_bounds__(256)
+concretize_grad_k(const float* __restrict__ lam, long long M, int n0, PassGeom pg, const float* __restrict__ centres,
+                  float eps, const float* __restrict__ cst, float* __restrict__ lb, float* __restrict__ G) {
+    const int lane = threadIdx.x & 31;
+    for (long long m = blockIdx.x * 8LL + (threadIdx.x >> 5); m < M; m += (long long)gridDim.x * 8) {
+        const float* a = lam + m * n0;
+        const float* c = centres + ((pg.pass_m0 + m) / pg.R_pass) * (long long)n0;
+        float s = 0.f;
+        for (int i = lane; i < n0; i += 32) {
+            const float x = a[i];
+            s += fmaf(x, c[i], -eps * fabsf(x));
+            if (G != nullptr) G[m * n0 + i] = c[i] - eps * ((x > 0.f) ? 1.f : ((x < 0.f) ? -1.f : 0.f));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) lb[m] = s + cst[m];
+    }
+}
+
+// Through one ReLU of the chain, in place: g = d lb / d alpha (unstable, lam_h >= 0), then
+// G <- G * slope + [H < 0] * t (slope from the current alpha), then (adam_step > 0) one Adam ascent step
+// on alpha, projected to [0, 1]. grad_out (optional) receives g.
+__global__ void relax_grad_adam_k(float* __restrict__ G, const float* __restrict__ H, long long M, int n,
+                                  const float4* __restrict__ P, PassGeom pg, float* __restrict__ alpha,
+                                  float* __restrict__ grad_out, float* __restrict__ m1, float* __restrict__ m2,
+                                  int adam_step, float lr, float c1, float c2) {
+    const long long total = M * n;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const long long m = e / n;
+        const int i = (int)(e % n);
+        const float4 p = P[((pg.pass_m0 + m) / pg.R_pass) * n + i];
+        const bool un = unstable(p);
+        const float x = H[e];
+        const float a = (alpha != nullptr && un) ? alpha[e] : p.x;
+        const float gz = G[e];
+        const float g = (un && x >= 0.f) ? gz * x : 0.f;
+        G[e] = gz * ((x >= 0.f) ? a : p.y) + ((x < 0.f) ? p.z : 0.f);
+        if (grad_out != nullptr) grad_out[e] = g;
+        if (adam_step > 0 && un && alpha != nullptr) {
+            const float v1 = 0.9f * m1[e] + 0.1f * g;
+            const float v2 = 0.999f * m2[e] + 0.001f * g * g;
+            m1[e] = v1;
+            m2[e] = v2;
+            const float step = lr * (v1 * c1) / (sqrtf(v2 * c2) + 1e-8f);
+            alpha[e] = fminf(fmaxf(a + step, 0.f), 1.f);
+        }
+    }
+}
+
+// alpha[m, i] = P[b, i].x (the adaptive start) and zero Adam moments.
+__global__ void alpha_init_k(float* __restrict__ alpha, float* __restrict__ m1, float* __restrict__ m2, long long M,
+                             int n, const float4* __restrict__ P, PassGeom pg) {
+    const long long total = M * n;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const long long m = e / n;
+        alpha[e] = P[((pg.pass_m0 + m) / pg.R_pass) * n + (e % n)].x;
+        m1[e] = 0.f;
+        m2[e] = 0.f;
+    }
+}
+
+__global__ void best_update_k(float* __restrict__ best, const float* __restrict__ cur, long long M, int first) {
+    for (long long m = blockIdx.x * (long long)blockDim.x + threadIdx.x; m < M; m += (long long)gridDim.x * blockDim.x)
+        best[m] = first ? cur[m] : fmaxf(best[m], cur[m]);
+}
+
+}  // namespace
+
+cudaError_t launch_relax_alpha_rows(const float* H, long long M, int n, const float4* P, PassGeom pg,
+                                    const float* alpha, float* Z, float* cst, cudaStream_t s) {
+    long long g = M < 148LL * 16 ? M : 148LL * 16;
+    relax_alpha_rows_k<<<(unsigned)(g < 1 ? 1 : g), 256, 0, s>>>(H, M, n, P, pg, alpha, Z, cst);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_concretize_grad(const float* lam, long long M, int n0, PassGeom pg, const float* centres, float eps,
+                                   const float* cst, float* lb, float* G, cudaStream_t s) {
+    long long g = (M + 7) / 8;
+    if (g > 148LL * 16) g = 148LL * 16;
+    concretize_grad_k<<<(unsigned)(g < 1 ? 1 : g), 256, 0, s>>>(lam, M, n0, pg, centres, eps, cst, lb, G);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_relax_grad_adam(float* G, const float* H, long long M, int n, const float4* P, PassGeom pg,
+                                   float* alpha, float* grad_out, float* m1, float* m2, int adam_step, float lr,
+                                   cudaStream_t s) {
+    float c1 = 1.f, c2 = 1.f;
+    if (adam_step > 0) {
+        c1 = 1.f / (1.f - powf(0.9f, (float)adam_step));
+        c2 = 1.f / (1.f - powf(0.999f, (float)adam_step));
+    }
+    relax_grad_adam_k<<<grid_for(M * n, 256), 256, 0, s>>>(G, H, M, n, P, pg, alpha, grad_out, m1, m2, adam_step, lr,
+                                                            c1, c2);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_alpha_init(float* alpha, float* m1, float* m2, long long M, int n, const float4* P, PassGeom pg,
+                              cudaStream_t s) {
+    alpha_init_k<<<grid_for(M * n, 256), 256, 0, s>>>(alpha, m1, m2, M, n, P, pg);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_best_update(float* best, const float* cur, long long M, int first, cudaStream_t s) {
+    best_update_k<<<grid_for(M, 256), 256, 0, s>>>(best, cur, M, first);
+    return cudaGetLastError();
+}
+
+}  // namespace vf

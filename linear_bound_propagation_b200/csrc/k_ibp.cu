@@ -166,6 +166,13 @@ cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, c
     return cudaGetLastError();
 }
 
+cudaError_t launch_rows_times_wt(const float* A, const float* W, const float* bias, int M, int K, int N, float* out,
+                                 cudaStream_t s) {
+    dim3 grid((M + 15) / 16, (N + 63) / 64, 1);  // only the centre product: out = A W^T + bias
+    ibp_dense_k<<<grid, 256, 0, s>>>(A, A, W, W, bias, nullptr, 0.f, M, K, N, out, out);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_ibp_conv(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
                             int B, const ConvGeom& g, float* zc, float* zr, cudaStream_t s) {
     const long long total = (long long)B * g.co * g.ho * g.wo;

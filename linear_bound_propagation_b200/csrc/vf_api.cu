@@ -622,6 +622,183 @@ int build_relax(vf_net* net, int B, const std::vector<const float*>& L, const st
     return VF_OK;
 }
 
+// Bounds of every ReLU source (IBP, refined by CROWN passes where asked) and the relaxation tables.
+struct Bounds {
+    std::vector<float*> Lw, Uw;
+    std::vector<const float4*> relax;
+};
+
+int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf_opts& o, Arena& ar, IbpState& st,
+                   Bounds& bd, cudaStream_t s) {
+    const int nn = (int)net->nodes.size();
+    TRY(run_ibp(net, centres, B, eps, ar, st, s));
+    bd.Lw.assign(nn, nullptr);
+    bd.Uw.assign(nn, nullptr);
+    for (int v = 0; v < nn; ++v) {
+        if (net->nodes[v].op != VF_RELU) continue;
+        const int p = net->nodes[v].src;
+        const long long cnt = (long long)B * net->nodes[p].n;
+        bd.Lw[p] = ar.take<float>(cnt);
+        bd.Uw[p] = ar.take<float>(cnt);
+        if (!bd.Lw[p] || !bd.Uw[p]) return fail(VF_ERR_WORKSPACE, "workspace too small for intermediate bounds");
+        LAUNCH(net, launch_bounds_from_cr(st.c[p], st.r[p], cnt, bd.Lw[p], bd.Uw[p], s));
+    }
+    bd.relax.assign(nn, nullptr);
+    std::vector<float4*> P(nn, nullptr);
+    long long max_pass_rows = 1;
+    for (int v = 0; v < nn; ++v)
+        if (net->nodes[v].op == VF_RELU) {
+            P[v] = ar.take<float4>((size_t)B * net->nodes[v].n);
+            if (!P[v]) return fail(VF_ERR_WORKSPACE, "workspace too small for relaxation parameters");
+            bd.relax[v] = P[v];
+            max_pass_rows = std::max(max_pass_rows, 2 * net->nodes[v].n);
+        }
+    Arena tmp = ar;  // pass outputs are transient
+    float* pass_out = tmp.take<float>((size_t)B * max_pass_rows);
+    if (!pass_out) return fail(VF_ERR_WORKSPACE, "workspace too small");
+    for (int k = 0; k < nn; ++k) {
+        const Node& nd = net->nodes[k];
+        if (nd.op != VF_RELU) continue;
+        const int p = nd.src;
+        const bool crown = (o.relu_crown == nullptr) || (o.relu_crown[k] != 0);
+        if (crown && !exact_source(net, p)) {
+            Entry init;
+            init.kind = E_IDENT;
+            const long long np = net->nodes[p].n;
+            TRY(run_pass(net, p, init, (long long)B * 2 * np, 2 * np, tmp, bd.relax, centres, eps, pass_out, nullptr,
+                         nullptr, s));
+            LAUNCH(net, launch_intersect(bd.Lw[p], bd.Uw[p], nullptr, nullptr, pass_out, B, np, s));
+        }
+        const Node& sn = net->nodes[p];
+        const bool aff = sn.op == VF_DENSE || sn.op == VF_CONV2D;
+        LAUNCH(net, launch_relax_params(bd.Lw[p], bd.Uw[p], o.alpha ? o.alpha[k] : nullptr, (long long)B * nd.n, P[k],
+                                        aff ? sn.b : nullptr, nd.n, sn.op == VF_CONV2D ? (long long)sn.h * sn.w : 1, s));
+    }
+    return VF_OK;
+}
+
+// A ReLU MLP laid out input -> dense -> relu -> dense -> ... -> dense (nodes in that order).
+bool dense_chain(const vf_net* net) {
+    const int nn = (int)net->nodes.size();
+    for (int v = 1; v < nn; ++v) {
+        const Node& nd = net->nodes[v];
+        if (nd.src != v - 1) return false;
+        if (nd.op != ((v % 2 == 1) ? VF_DENSE : VF_RELU)) return false;
+    }
+    return net->nodes[nn - 1].op == VF_DENSE;
+}
+
+// alpha-CROWN on the specification rows of a dense chain: per-row lower slopes of unstable neurons.
+// grad_mode: one evaluation at alpha_in, writing lb and d lb / d alpha (grad_out) -- no update.
+// Otherwise: iters Adam ascent steps from the adaptive slopes, lb = best bound seen per row,
+// lb_start (optional) = the bound at the adaptive start, alpha_out (optional) = the final slopes.
+// Slope arrays: for each ReLU node in order, a [B, R, n] block.
+int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
+               const vf_opts& o, int iters, float lr, bool grad_mode, const float* alpha_in, float* grad_out,
+               float* lb, float* lb_start, float* alpha_out, cudaStream_t s) {
+    const int nn = (int)net->nodes.size();
+    const int L = nn - 1;
+    const long long n0 = net->nodes[0].n;
+    const int nL = (int)net->nodes[L].n;
+    Arena ar{net->ws, net->ws_bytes};
+    IbpState st;
+    Bounds bd;
+    TRY(prepare_bounds(net, centres, B, eps, o, ar, st, bd, s));
+    std::vector<int> relus;
+    long long sum_n = 0, nmax = 1;
+    std::vector<long long> aoff(nn, 0);  // offset of each ReLU's [B, R, n] slope block
+    for (int v = 2; v < L; v += 2) {
+        relus.push_back(v);
+        aoff[v] = (long long)B * R * sum_n;
+        sum_n += net->nodes[v].n;
+        nmax = std::max(nmax, net->nodes[v].n);
+    }
+    const long long gmax = std::max<long long>(nmax, n0);
+    const long long rows = (long long)B * R;
+    // per-row floats: H (sum_n) + Z (nmax) + lam_in (n0) + two gradient buffers (gmax) + cst + lb
+    // (+ slopes and two Adam moments, 3 * sum_n, when optimising)
+    const size_t per_row = sizeof(float) * (sum_n + nmax + n0 + 2 * gmax + 2 + (grad_mode ? 0 : 3 * sum_n)) +
+                           64 * (relus.size() + 8);
+    long long chunk = (long long)(ar.left() / per_row);
+    if (chunk > rows) chunk = rows;
+    if (chunk < 1) return fail(VF_ERR_WORKSPACE, "workspace too small for alpha optimisation");
+    std::vector<float*> H(nn, nullptr), A(nn, nullptr), M1(nn, nullptr), M2(nn, nullptr);
+    for (int u : relus) {
+        H[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+        if (!grad_mode) {
+            A[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+            M1[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+            M2[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+        }
+    }
+    float* Z = ar.take<float>((size_t)chunk * nmax);
+    float* lam_in = ar.take<float>((size_t)chunk * n0);
+    float* G0 = ar.take<float>((size_t)chunk * gmax);
+    float* G1 = ar.take<float>((size_t)chunk * gmax);
+    float* cst = ar.take<float>(chunk);
+    float* lbc = ar.take<float>(chunk);
+    if (!Z || !lam_in || !G0 || !G1 || !cst || !lbc) return fail(VF_ERR_WORKSPACE, "workspace too small");
+    for (int u : relus)
+        if (!H[u] || (!grad_mode && (!A[u] || !M1[u] || !M2[u]))) return fail(VF_ERR_WORKSPACE, "workspace too small");
+
+    for (long long m0 = 0; m0 < rows; m0 += chunk) {
+        const long long Mc = std::min(chunk, rows - m0);
+        const PassGeom pg{m0, R};
+        std::vector<float*> al(nn, nullptr);
+        for (int u : relus) {
+            const long long nu = net->nodes[u].n;
+            if (grad_mode) {
+                al[u] = const_cast<float*>(alpha_in) + aoff[u] + m0 * nu;
+            } else {
+                al[u] = A[u];
+                LAUNCH(net, launch_alpha_init(A[u], M1[u], M2[u], Mc, (int)nu, bd.relax[u], pg, s));
+            }
+        }
+        const int evals = grad_mode ? 1 : iters + 1;
+        for (int it = 0; it < evals; ++it) {
+            // down: back-substitution of the rows with the current slopes, keeping lam over every ReLU
+            CU(cudaMemsetAsync(cst, 0, sizeof(float) * Mc, s));
+            const Node& last = net->nodes[L];
+            LAUNCH(net, launch_dense_back(RowRef{C, C_bstride, nL, R, m0}, Relax{nullptr, 0}, last.W, last.b, Mc, nL,
+                                          (int)net->nodes[L - 1].n, pg, OUT_STORE, H[L - 1], net->nodes[L - 1].n, cst,
+                                          nullptr, 0.f, nullptr, s));
+            for (int u = L - 1; u >= 2; u -= 2) {
+                const int nu = (int)net->nodes[u].n;
+                const Node& d = net->nodes[u - 1];
+                const int nd_in = (int)net->nodes[u - 2].n;
+                LAUNCH(net, launch_relax_alpha_rows(H[u], Mc, nu, bd.relax[u], pg, al[u], Z, cst, s));
+                float* out = (u - 2 == 0) ? lam_in : H[u - 2];
+                LAUNCH(net, launch_dense_back(RowRef{Z, 0, nu, kHugeRows, 0}, Relax{nullptr, 0}, d.W, nullptr, Mc, nu,
+                                              nd_in, pg, OUT_STORE, out, nd_in, nullptr, nullptr, 0.f, nullptr, s));
+            }
+            LAUNCH(net, launch_concretize_grad(lam_in, Mc, (int)n0, pg, centres, eps, cst, lbc, G0, s));
+            if (it == 0 && lb_start) CU(cudaMemcpyAsync(lb_start + m0, lbc, sizeof(float) * Mc, cudaMemcpyDeviceToDevice, s));
+            LAUNCH(net, launch_best_update(lb + m0, lbc, Mc, it == 0 ? 1 : 0, s));
+            if (!grad_mode && it == iters) break;
+            // up: gradient with respect to every ReLU's slopes (and one Adam ascent step)
+            float* G = G0;
+            float* Gn = G1;
+            for (int d = 1; d + 1 < L; d += 2) {
+                const Node& dn = net->nodes[d];
+                const int u = d + 1;
+                const int nu = (int)net->nodes[u].n;
+                LAUNCH(net, launch_rows_times_wt(G, dn.W, dn.b, (int)Mc, (int)net->nodes[d - 1].n, nu, Gn, s));
+                float* gout = grad_mode ? grad_out + aoff[u] + m0 * nu : nullptr;
+                LAUNCH(net, launch_relax_grad_adam(Gn, H[u], Mc, nu, bd.relax[u], pg, al[u], gout, M1[u], M2[u],
+                                                   grad_mode ? 0 : it + 1, lr, s));
+                std::swap(G, Gn);
+            }
+        }
+        if (!grad_mode && alpha_out)
+            for (int u : relus) {
+                const long long nu = net->nodes[u].n;
+                CU(cudaMemcpyAsync(alpha_out + aoff[u] + m0 * nu, A[u], sizeof(float) * Mc * nu,
+                                   cudaMemcpyDeviceToDevice, s));
+            }
+    }
+    return VF_OK;
+}
+
 }  // namespace
 
 int vf::set_last_error(int code, const char* msg) {
@@ -931,57 +1108,17 @@ int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const f
     }
 
     IbpState st;
-    TRY(run_ibp(net, centres, B, eps, ar, st, s));
-
-    // Bounds used for every ReLU source: start from IBP, refined in place by CROWN passes.
-    std::vector<const float*> L(nn, nullptr), U(nn, nullptr);
-    std::vector<float*> Lw(nn, nullptr), Uw(nn, nullptr);
-    for (int v = 0; v < nn; ++v) {
-        if (net->nodes[v].op != VF_RELU) continue;
-        const int p = net->nodes[v].src;
-        const long long cnt = (long long)B * net->nodes[p].n;
-        Lw[p] = ar.take<float>(cnt);
-        Uw[p] = ar.take<float>(cnt);
-        if (!Lw[p] || !Uw[p]) return fail(VF_ERR_WORKSPACE, "workspace too small for intermediate bounds");
-        LAUNCH(net, launch_bounds_from_cr(st.c[p], st.r[p], cnt, Lw[p], Uw[p], s));
-        L[p] = Lw[p];
-        U[p] = Uw[p];
-    }
-    std::vector<const float4*> relax(nn, nullptr);
-    std::vector<float4*> P(nn, nullptr);
-    long long max_pass_rows = 0;
-    for (int v = 0; v < nn; ++v)
-        if (net->nodes[v].op == VF_RELU) {
-            P[v] = ar.take<float4>((size_t)B * net->nodes[v].n);
-            if (!P[v]) return fail(VF_ERR_WORKSPACE, "workspace too small for relaxation parameters");
-            relax[v] = P[v];
-            max_pass_rows = std::max(max_pass_rows, 2 * net->nodes[v].n);
-        }
+    Bounds bd;
+    TRY(prepare_bounds(net, centres, B, eps, o, ar, st, bd, s));
+    std::vector<float*>& Lw = bd.Lw;
+    std::vector<float*>& Uw = bd.Uw;
+    std::vector<const float4*>& relax = bd.relax;
     const int Rp = o.both_sides ? 2 * R : R;
-    float* pass_out = ar.take<float>((size_t)B * std::max<long long>(max_pass_rows, Rp));
+    float* pass_out = ar.take<float>((size_t)B * Rp);
     float* lbI = ar.take<float>((size_t)B * R);
     float* ubI = ar.take<float>((size_t)B * R);
     float* S = o.both_sides ? ar.take<float>((size_t)BC * Rp * nL) : nullptr;
     if (!pass_out || !lbI || !ubI || (o.both_sides && !S)) return fail(VF_ERR_WORKSPACE, "workspace too small");
-
-    for (int k = 0; k < nn; ++k) {
-        const Node& nd = net->nodes[k];
-        if (nd.op != VF_RELU) continue;
-        const int p = nd.src;
-        const bool crown = (o.relu_crown == nullptr) || (o.relu_crown[k] != 0);
-        if (crown && !exact_source(net, p)) {
-            Entry init;
-            init.kind = E_IDENT;
-            const long long np = net->nodes[p].n;
-            TRY(run_pass(net, p, init, (long long)B * 2 * np, 2 * np, ar, relax, centres, eps, pass_out, nullptr,
-                         nullptr, s));
-            LAUNCH(net, launch_intersect(Lw[p], Uw[p], nullptr, nullptr, pass_out, B, np, s));
-        }
-        const Node& sn = net->nodes[p];
-        const bool aff = sn.op == VF_DENSE || sn.op == VF_CONV2D;
-        LAUNCH(net, launch_relax_params(Lw[p], Uw[p], o.alpha ? o.alpha[k] : nullptr, (long long)B * nd.n, P[k],
-                                        aff ? sn.b : nullptr, nd.n, sn.op == VF_CONV2D ? (long long)sn.h * sn.w : 1, s));
-    }
 
     // Specification pass.
     Entry init;
@@ -1011,6 +1148,37 @@ int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const f
         }
     }
     return VF_OK;
+}
+
+int vf_alpha_crown(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
+                   const vf_opts* opts, int iters, float lr, float* lb, float* lb_start, float* alpha_out,
+                   void* stream) {
+    TRY(check_net(net));
+    vf_opts o{};
+    if (opts) o = *opts;
+    if (!centres || !C || !lb) return fail(VF_ERR_ARG, "centres, C and lb must not be NULL");
+    if (B < 0 || R < 0 || C_bstride < 0 || iters < 0) return fail(VF_ERR_ARG, "negative size");
+    if (!std::isfinite(eps) || eps < 0.f || !std::isfinite(lr) || lr < 0.f)
+        return fail(VF_ERR_NONFINITE, "eps and lr must be finite and >= 0");
+    if (!dense_chain(net)) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation needs a dense ReLU chain");
+    if (o.both_sides) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation bounds the lower side; pass -C for upper");
+    if (B == 0 || R == 0) return VF_OK;
+    return spec_alpha(net, centres, B, eps, C, R, C_bstride, o, iters, lr, false, nullptr, nullptr, lb, lb_start,
+                      alpha_out, (cudaStream_t)stream);
+}
+
+int vf_alpha_grad(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
+                  const vf_opts* opts, const float* alpha, float* lb, float* grad, void* stream) {
+    TRY(check_net(net));
+    vf_opts o{};
+    if (opts) o = *opts;
+    if (!centres || !C || !lb || !alpha || !grad) return fail(VF_ERR_ARG, "NULL pointer");
+    if (B < 0 || R < 0 || C_bstride < 0) return fail(VF_ERR_ARG, "negative size");
+    if (!std::isfinite(eps) || eps < 0.f) return fail(VF_ERR_NONFINITE, "eps must be finite and >= 0");
+    if (!dense_chain(net)) return fail(VF_ERR_UNSUPPORTED, "alpha gradients need a dense ReLU chain");
+    if (B == 0 || R == 0) return VF_OK;
+    return spec_alpha(net, centres, B, eps, C, R, C_bstride, o, 0, 0.f, true, alpha, grad, lb, nullptr, nullptr,
+                      (cudaStream_t)stream);
 }
 
 int vf_profile_enable(vf_net* net, int enable) {

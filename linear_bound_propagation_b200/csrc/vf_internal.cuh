@@ -107,6 +107,22 @@ cudaError_t launch_finite_scan(const float* p, long long n, int* flag, cudaStrea
 cudaError_t launch_concretize_api(const float* lambda, const float* cst, const float* centres, float eps, int B, int R,
                                   int n0, float* lb, cudaStream_t s);
 
+// out[m, n] = sum_k A[m, k] * W[n, k] + bias[n]  (A [M, K], W [N, K] row-major).
+cudaError_t launch_rows_times_wt(const float* A, const float* W, const float* bias, int M, int K, int N, float* out,
+                                 cudaStream_t s);
+
+// ---- alpha-CROWN (k_alpha.cu) -----------------------------------------------------------
+cudaError_t launch_relax_alpha_rows(const float* H, long long M, int n, const float4* P, PassGeom pg,
+                                    const float* alpha, float* Z, float* cst, cudaStream_t s);
+cudaError_t launch_concretize_grad(const float* lam, long long M, int n0, PassGeom pg, const float* centres, float eps,
+                                   const float* cst, float* lb, float* G, cudaStream_t s);
+cudaError_t launch_relax_grad_adam(float* G, const float* H, long long M, int n, const float4* P, PassGeom pg,
+                                   float* alpha, float* grad_out, float* m1, float* m2, int adam_step, float lr,
+                                   cudaStream_t s);
+cudaError_t launch_alpha_init(float* alpha, float* m1, float* m2, long long M, int n, const float4* P, PassGeom pg,
+                              cudaStream_t s);
+cudaError_t launch_best_update(float* best, const float* cur, long long M, int first, cudaStream_t s);
+
 // Records `msg` as this thread's vf_last_error() text and returns `code`.
 int set_last_error(int code, const char* msg);
 

@@ -25,7 +25,7 @@ VF_KERNEL_ALL, VF_KERNEL_DENSE_TC, VF_KERNEL_DENSE_FFMA, VF_KERNEL_CONV = range(
 SYMBOLS = ["vf_net_create", "vf_net_destroy", "vf_net_node_size", "vf_net_total_size", "vf_ibp",
            "vf_crown_backward", "vf_concretize", "vf_verify_batch", "vf_sync", "vf_last_error",
            "vf_profile_enable", "vf_profile_read", "vf_launch_count", "vf_net_check",
-           "vf_concretize_dense_noalloc"]
+           "vf_concretize_dense_noalloc", "vf_alpha_crown", "vf_alpha_grad"]
 NOALLOC_SCRATCH_FLOATS = 1 << 22
 
 
@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
                                   ctypes.POINTER(ctypes.c_double), I]
     L.vf_net_check.argtypes = [P]
     L.vf_concretize_dense_noalloc.argtypes = [P, LL, I, P, P, P, F, I, I, I, P, P]
+    L.vf_alpha_crown.argtypes = [P, P, I, F, P, I, LL, ctypes.POINTER(Opts), I, F, P, P, P, P]
+    L.vf_alpha_grad.argtypes = [P, P, I, F, P, I, LL, ctypes.POINTER(Opts), P, P, P, P]
     L.vf_launch_count.argtypes = [P]
     L.vf_launch_count.restype = LL
     _lib = L
@@ -220,6 +222,45 @@ class Net:
                                      _ptr(out["lb"]), _ptr(out.get("ub")), _ptr(out.get("lb_ibp")),
                                      _ptr(out.get("verified")), _stream_ptr(stream)))
         return out
+
+    def _opts(self, crown_relus=None):
+        o = Opts()
+        keep = None
+        if crown_relus is not None:
+            keep = (ctypes.c_int * self.n_nodes)()
+            for v in crown_relus:
+                keep[v] = 1
+            o.relu_crown = ctypes.cast(keep, ctypes.POINTER(ctypes.c_int))
+        return o, keep
+
+    def alpha_size(self, B: int, R: int) -> int:
+        """Length of a per-row slope array: one [B, R, n_v] block per ReLU node v in node order."""
+        return B * R * sum(self.sizes[v] for v in self.relu_ids)
+
+    def alpha_crown(self, centres: torch.Tensor, eps: float, C: torch.Tensor, iters: int = 20, lr: float = 0.1,
+                    crown_relus=None, want_alpha: bool = False, stream=None):
+        """vf_alpha_crown: returns dict(lb=best bound [B, R], lb_start=[B, R], alpha=final slopes or None)."""
+        B, R = centres.shape[0], C.shape[1]
+        bstride = 0 if C.shape[0] == 1 else R * C.shape[2]
+        lb = torch.empty(B, R, device=centres.device)
+        lb0 = torch.empty(B, R, device=centres.device)
+        al = torch.empty(self.alpha_size(B, R), device=centres.device) if want_alpha else None
+        o, keep = self._opts(crown_relus)
+        _check(lib().vf_alpha_crown(self.h, _ptr(centres), B, float(eps), _ptr(C), R, bstride, ctypes.byref(o), iters,
+                                    float(lr), _ptr(lb), _ptr(lb0), _ptr(al), _stream_ptr(stream)))
+        return {"lb": lb, "lb_start": lb0, "alpha": al}
+
+    def alpha_grad(self, centres: torch.Tensor, eps: float, C: torch.Tensor, alpha: torch.Tensor, crown_relus=None,
+                   stream=None):
+        """vf_alpha_grad: (lb [B, R], grad with alpha's layout) at the given per-row slopes."""
+        B, R = centres.shape[0], C.shape[1]
+        bstride = 0 if C.shape[0] == 1 else R * C.shape[2]
+        lb = torch.empty(B, R, device=centres.device)
+        grad = torch.empty_like(alpha)
+        o, keep = self._opts(crown_relus)
+        _check(lib().vf_alpha_grad(self.h, _ptr(centres), B, float(eps), _ptr(C), R, bstride, ctypes.byref(o),
+                                   _ptr(alpha), _ptr(lb), _ptr(grad), _stream_ptr(stream)))
+        return lb, grad
 
     def profile(self, enable: bool):
         _check(lib().vf_profile_enable(self.h, 1 if enable else 0))

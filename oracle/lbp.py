@@ -365,3 +365,109 @@ def verify(net, centres, eps, C, crown_relus: Optional[Sequence[int]] = None,
     ub = np.minimum(ub_ibp, ub_cr) if both_sides else None
     return OracleResult(lb=lb, ub=ub, lb_ibp=lb_ibp, ub_ibp=ub_ibp, lb_crown=lb_cr, ub_crown=ub_cr,
                         verified=lb > 0.0, pre_bounds=pre, ibp_bounds=ibp_b)
+
+
+# ----------------------------------------------------------------------------- alpha-CROWN
+
+def _dense_chain(net):
+    """Node ids of a ReLU MLP written as input -> dense -> relu -> ... -> dense, else None."""
+    if net[0].op != "input":
+        return None
+    for v in range(1, len(net)):
+        nd = net[v]
+        if nd.src != v - 1 or nd.op not in ("dense", "relu"):
+            return None
+        if (nd.op == "dense") == (v % 2 == 0):
+            return None
+    return [v for v in range(len(net)) if net[v].op == "dense"]
+
+
+def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows):
+    """Lower bounds of `rows` (R x n_L) over the box, with one lower slope per (row, unstable neuron)
+    [SNNV §3, §4.3: per-neuron alpha tensors], and their gradients with respect to those slopes.
+
+    relax: relu node -> (lo, up, t) vectors (the intermediate-bound relaxation); alpha_rows: relu node
+    -> [R, n] slopes in [0, 1], used in place of `lo` for unstable neurons (0 < up < 1). Returns
+    (lb [R], grads {relu node: [R, n]}, zero where the neuron is stable).
+
+    Forward: the back-substitution of `backward` with row-specific lower slopes. Gradient: reverse
+    mode through that chain (layer order from the input up): with G the gradient of lb with respect
+    to the coefficients over a node's output,
+      input:   G = centre - eps * sign(lam_in)             (from lam . centre - eps |lam|)
+      dense:   G_z = G_h W^T + b                           (lam_h = lam_z W,  const += lam_z . b)
+      relu:    dlb/dalpha_i = G_z,i * lam_h,i * [lam_h,i >= 0]   for unstable i
+               G_h = G_z * slope + [lam_h < 0] * t         (lam_z = slope * lam_h, const += min(lam_h, 0) t)
+    """
+    chain = _dense_chain(net)
+    if chain is None:
+        raise ValueError("alpha optimisation is defined here for dense ReLU chains")
+    L = len(net) - 1
+    lam = np.asarray(rows, F)
+    R = lam.shape[0]
+    const = np.zeros(R, F)
+    saved = {}  # relu node -> (lam_h, slope) used on the way down
+    for v in range(L, 0, -1):
+        nd = net[v]
+        if nd.op == "dense":
+            const = const + lam @ nd.b.astype(F)
+            lam = lam @ nd.W.astype(F)
+        else:
+            lo, up, t = relax[v]
+            unst = (up > 0.0) & (up < 1.0)
+            lo_rows = np.where(unst[None, :], np.asarray(alpha_rows[v], F), lo[None, :])
+            slope = np.where(lam >= 0.0, lo_rows, up[None, :])
+            const = const + np.minimum(lam, 0.0) @ t
+            saved[v] = (lam, slope, unst)
+            lam = lam * slope
+    c = np.asarray(centre, F)
+    lb = lam @ c - F(eps) * np.abs(lam).sum(axis=1) + const
+    G = c[None, :] - F(eps) * np.sign(lam)
+    grads = {}
+    for v in range(1, L + 1):
+        nd = net[v]
+        if nd.op == "dense":
+            G = G @ nd.W.astype(F).T + nd.b.astype(F)[None, :]
+        else:
+            lam_h, slope, unst = saved[v]
+            t = relax[v][2]
+            grads[v] = np.where(unst[None, :] & (lam_h >= 0.0), G * lam_h, 0.0)
+            G = G * slope + np.where(lam_h < 0.0, t[None, :], 0.0)
+    return lb, grads
+
+
+def alpha_crown(net, centres, eps, C, iters=10, lr=0.1, crown_relus=None, betas=(0.9, 0.999)):
+    """Projected gradient ascent (Adam) on per-row lower slopes of the specification pass, starting
+    from the adaptive slopes, keeping each row's best bound [SNNV §1 alpha-CROWN; §3 alpha tensors].
+    Intermediate bounds are those of `verify` (adaptive slopes). Returns (best lb [B, R], lb at the
+    adaptive start [B, R])."""
+    res = verify(net, centres, eps, C, crown_relus=crown_relus)
+    B, R = res.lb.shape
+    C = np.asarray(C, F)
+    relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
+    best = np.empty((B, R), F)
+    start = np.empty((B, R), F)
+    b1, b2 = betas
+    for b in range(B):
+        relax = {k: relax_params(res.pre_bounds[k][0][b], res.pre_bounds[k][1][b]) for k in relus}
+        rows = C[b if C.shape[0] > 1 else 0]
+        alpha = {k: np.repeat(relax[k][0][None, :], R, axis=0) for k in relus}
+        m1 = {k: np.zeros_like(a) for k, a in alpha.items()}
+        m2 = {k: np.zeros_like(a) for k, a in alpha.items()}
+        best_b = None
+        for it in range(iters + 1):
+            lb, g = spec_bound_alpha(net, centres[b], eps, rows, relax, alpha)
+            if it == 0:
+                start[b] = lb
+                best_b = lb.copy()
+            else:
+                best_b = np.maximum(best_b, lb)
+            if it == iters:
+                break
+            for k in relus:
+                m1[k] = b1 * m1[k] + (1 - b1) * g[k]
+                m2[k] = b2 * m2[k] + (1 - b2) * g[k] * g[k]
+                mh = m1[k] / (1 - b1 ** (it + 1))
+                vh = m2[k] / (1 - b2 ** (it + 1))
+                alpha[k] = np.clip(alpha[k] + lr * mh / (np.sqrt(vh) + 1e-8), 0.0, 1.0)
+        best[b] = best_b
+    return best, start
