@@ -74,6 +74,8 @@ struct Node {
     float* WtHi = nullptr; // dense only: W^T [n_in, n_out] truncated to tf32 (3xTF32 head)
     float* WtLo = nullptr; // dense only: W^T - WtHi (3xTF32 remainder)
     float* rowsum_abs = nullptr;  // dense only: sum_k |W[n, k]| (IBP radius of a layer fed by the input box)
+    float* Wwin = nullptr;        // conv only: weights in the tap-major layout of the windowed kernel
+    WinWeights ww{nullptr, 0, 0, 4};
     int consumers = 0;
 };
 
@@ -91,6 +93,7 @@ struct vf_net {
     int dense_kernel = 0;   // 0: tensor cores where the shapes allow, 1: FFMA only (VF_DENSE_KERNEL=ffma)
     int* d_err = nullptr;   // device flag raised by a kernel whose bounded wait expired
     int tc_stall = 0;       // test hook: VF_TEST_TC_STALL=1 makes one tensor-core launch time out
+    int windows = 1;        // receptive-field windows in passes that start at a convolution (VF_CONV_WINDOWS=0: off)
     bool prof = false;
     std::vector<cudaEvent_t> ev_free;
     struct Timed {
@@ -177,7 +180,35 @@ struct Entry {
     int buf = -1;  // E_BUF: pool index
     RowRef ref{nullptr, 0, 0, kHugeRows, 0};
     Relax rx{nullptr, 0};
+    bool windowed = false;  // rows held as a receptive-field window `win` of the node's map
+    Win win{0, 0, 0, 0, 0, 0, 0};
 };
+
+// Receptive-field windows (rows of a pass that starts at a convolution, see k_win.cu).
+Win full_win(const Node& nd) { return Win{nd.c, nd.h, nd.w, 0, 0, 0, 0}; }
+long long win_len(const Win& w) { return (long long)w.C * w.hh * w.hw; }
+bool win_eq(const Win& a, const Win& b) {
+    return a.C == b.C && a.hh == b.hh && a.hw == b.hw && a.ay == b.ay && a.by == b.by && a.ax == b.ax && a.bx == b.bx;
+}
+// Field over a convolution's input of rows in window `wa` over its output.
+Win win_back(const Win& wa, const ConvGeom& g) {
+    return Win{g.ci,
+               g.stride * (wa.hh - 1) + g.k,
+               g.stride * (wa.hw - 1) + g.k,
+               g.stride * wa.ay,
+               g.stride * wa.by - g.pad,
+               g.stride * wa.ax,
+               g.stride * wa.bx - g.pad};
+}
+// A window is kept only while it holds at most half of the node's map.
+bool win_small(const Win& w, const Node& nd) { return nd.h > 1 && 2 * win_len(w) <= nd.n; }
+// Smallest window containing both (same channel count and origin slopes), else false.
+bool win_union(const Win& a, const Win& b, Win* u) {
+    if (a.C != b.C || a.ay != b.ay || a.ax != b.ax) return false;
+    const int by = std::min(a.by, b.by), bx = std::min(a.bx, b.bx);
+    *u = Win{a.C, std::max(a.by + a.hh, b.by + b.hh) - by, std::max(a.bx + a.hw, b.bx + b.hw) - bx, a.ay, by, a.ax, bx};
+    return true;
+}
 
 struct Walker {
     vf_net* net;
@@ -199,8 +230,13 @@ struct Walker {
     bool ext_written = false;
     const std::vector<const float4*>* relax;  // per node: relaxation params of ReLU nodes
     std::vector<Entry> pend;
+    bool win_on = false;      // rows may be held as receptive-field windows (pass starts at a convolution)
+    PassStart ps{1, 1, 1};    // the pass's start node
+    long long max_len = 0;    // longest row a pool buffer has held
 
-    int alloc_buf(int* out) {
+    int alloc_buf(int* out, long long len) {
+        max_len = std::max(max_len, len);
+        if (!dry && len > ld_buf) return fail(VF_ERR_WORKSPACE, "row of %lld floats exceeds the row buffers", len);
         for (size_t i = 0; i < ref.size(); ++i)
             if (ref[i] == 0) {
                 ref[i] = 1;
@@ -232,33 +268,53 @@ struct Walker {
         return e;
     }
 
-    // Make pend[v] a plain (unrelaxed, unshared) buffer so contributions can be added to it.
-    int make_plain(int v, int* out) {
+    // Make pend[v] a plain (unrelaxed, unshared) buffer so contributions can be added to it, held as
+    // window *want (which contains the entry's window), or as the whole map when want is null.
+    int make_plain(int v, int* out, const Win* want = nullptr) {
         Entry& e = pend[v];
-        const long long n = net->nodes[v].n;
-        if (e.kind == E_BUF && e.rx.P == nullptr && ref[e.buf] == 1) {
+        const Node& nd = net->nodes[v];
+        const long long n = nd.n;
+        const bool same = want ? (e.windowed && win_eq(e.win, *want)) : !e.windowed;
+        if (e.kind == E_BUF && same && ref[e.buf] == 1) {
+            if (e.rx.P != nullptr) {  // relax in place
+                if (!dry) {
+                    if (e.windowed)
+                        LAUNCH(net, launch_rewin_rows(e.ref, e.rx, M, nd.c, nd.h, nd.w, pg, ps, e.win, e.win,
+                                                      bufs[e.buf], ld_buf, 0, cst, s));
+                    else
+                        LAUNCH(net, launch_relax_rows(e.ref, e.rx, M, (int)n, pg, bufs[e.buf], ld_buf, 0, cst, s));
+                }
+                e.rx = Relax{nullptr, 0};
+            }
             *out = e.buf;
             return VF_OK;
         }
-        if (e.kind == E_BUF && ref[e.buf] == 1) {  // relax in place
-            if (!dry)
-                LAUNCH(net, launch_relax_rows(e.ref, e.rx, M, (int)n, pg, bufs[e.buf], ld_buf, 0, cst, s));
-            e.rx = Relax{nullptr, 0};
-            *out = e.buf;
-            return VF_OK;
-        }
+        if (e.kind == E_IDENT && want != nullptr) return fail(VF_ERR_ARG, "internal: identity rows cannot be windowed");
         int nb;
-        TRY(alloc_buf(&nb));
+        TRY(alloc_buf(&nb, want ? win_len(*want) : n));
         if (!dry) {
             if (e.kind == E_IDENT)
                 LAUNCH(net, launch_ident_rows(bufs[nb], ld_buf, M, pg, n, 0, s));
-            else
+            else if (!e.windowed && want == nullptr)
                 LAUNCH(net, launch_relax_rows(e.ref, e.rx, M, (int)n, pg, bufs[nb], ld_buf, 0, cst, s));
+            else
+                LAUNCH(net, launch_rewin_rows(e.ref, e.rx, M, nd.c, nd.h, nd.w, pg, ps, e.windowed ? e.win : full_win(nd),
+                                              want ? *want : full_win(nd), bufs[nb], ld_buf, 0, cst, s));
         }
         release(e);
         pend[v] = buf_entry(nb);
+        if (want != nullptr) {
+            pend[v].windowed = true;
+            pend[v].win = *want;
+        }
         *out = nb;
         return VF_OK;
+    }
+
+    // The window that holds both pend[v] and rows in window x (null: the whole map).
+    bool merged_win(int v, const Win* x, Win* u) const {
+        const Entry& e = pend[v];
+        return x != nullptr && e.windowed && win_union(e.win, *x, u) && win_small(*u, net->nodes[v]);
     }
 
     // pend[v] += x (x is consumed).
@@ -267,21 +323,31 @@ struct Walker {
             pend[v] = x;
             return VF_OK;
         }
-        const long long n = net->nodes[v].n;
+        const Node& nd = net->nodes[v];
+        const long long n = nd.n;
+        Win u;
+        const bool wu = merged_win(v, x.windowed ? &x.win : nullptr, &u);
         int b;
-        TRY(make_plain(v, &b));
+        TRY(make_plain(v, &b, wu ? &u : nullptr));
         if (!dry) {
             if (x.kind == E_IDENT)
                 LAUNCH(net, launch_ident_rows(bufs[b], ld_buf, M, pg, n, 1, s));
-            else
+            else if (!x.windowed && !wu)
                 LAUNCH(net, launch_relax_rows(x.ref, x.rx, M, (int)n, pg, bufs[b], ld_buf, 1, cst, s));
+            else
+                LAUNCH(net, launch_rewin_rows(x.ref, x.rx, M, nd.c, nd.h, nd.w, pg, ps, x.windowed ? x.win : full_win(nd),
+                                              wu ? u : full_win(nd), bufs[b], ld_buf, 1, cst, s));
         }
         release(x);
         return VF_OK;
     }
 
-    // Where an affine node's back-substituted rows over its source go.
-    int target(int src, float** out, long long* ld, int* mode) {
+    // Where an affine node's back-substituted rows over its source go. nat: the window the rows
+    // occupy (null: the whole map); *dst receives the window of the destination (the whole map when
+    // the entry there is not windowed).
+    int target(int src, float** out, long long* ld, int* mode, const Win* nat = nullptr, Win* dst = nullptr) {
+        const Node& sn = net->nodes[src];
+        if (dst != nullptr) *dst = full_win(sn);
         if (src == 0 && ext_in != nullptr && pend[0].kind == E_NONE) {
             *out = ext_in;
             *ld = net->nodes[0].n;
@@ -290,16 +356,25 @@ struct Walker {
             return VF_OK;
         }
         if (pend[src].kind == E_NONE) {
+            const bool wnd = nat != nullptr && win_small(*nat, sn);
             int nb;
-            TRY(alloc_buf(&nb));
+            TRY(alloc_buf(&nb, wnd ? win_len(*nat) : sn.n));
             pend[src] = buf_entry(nb);
+            if (wnd) {
+                pend[src].windowed = true;
+                pend[src].win = *nat;
+                if (dst != nullptr) *dst = *nat;
+            }
             *out = dry ? nullptr : bufs[nb];
             *ld = ld_buf;
             *mode = OUT_STORE;
             return VF_OK;
         }
+        Win u;
+        const bool wu = merged_win(src, nat, &u);
         int b;
-        TRY(make_plain(src, &b));
+        TRY(make_plain(src, &b, wu ? &u : nullptr));
+        if (wu && dst != nullptr) *dst = u;
         *out = dry ? nullptr : bufs[b];
         *ld = ld_buf;
         *mode = OUT_ACCUM;
@@ -327,7 +402,7 @@ struct Walker {
         const Node& nd = net->nodes[v];
         switch (nd.op) {
             case VF_INPUT: {
-                if (e.kind == E_IDENT || e.rx.P != nullptr) {
+                if (e.kind == E_IDENT || e.rx.P != nullptr || e.windowed) {
                     pend[0] = e;
                     int b;
                     TRY(make_plain(0, &b));
@@ -349,7 +424,7 @@ struct Walker {
                 if (e.kind == E_IDENT || e.rx.P != nullptr) {
                     pend[v] = e;
                     int b;
-                    TRY(make_plain(v, &b));
+                    TRY(make_plain(v, &b, e.windowed ? &e.win : nullptr));
                     e = pend[v];
                     pend[v] = Entry();
                 }
@@ -365,6 +440,13 @@ struct Walker {
             }
             case VF_DENSE: {
                 const Node& sn = net->nodes[nd.src];
+                if (e.windowed) {  // dense rows span the whole map
+                    pend[v] = e;
+                    int b;
+                    TRY(make_plain(v, &b));
+                    e = pend[v];
+                    pend[v] = Entry();
+                }
                 if (e.kind == E_IDENT) {
                     if (!dry) LAUNCH(net, launch_cst_identity_bias(cst, M, pg, nd.b, nd.n, 1, s));
                     Entry x;
@@ -405,16 +487,49 @@ struct Walker {
                     float* out = nullptr;
                     long long ld = 0;
                     int mode = OUT_STORE;
+                    if (win_on) {  // the k x k field of each start neuron
+                        const Win nat{g.ci, g.k, g.k, g.stride, -g.pad, g.stride, -g.pad};
+                        Win dst;
+                        TRY(target(nd.src, &out, &ld, &mode, &nat, &dst));
+                        if (!dry)
+                            LAUNCH(net, launch_conv_start_rows_win(out, ld, M, pg, ps, nd.W, g, dst,
+                                                                   mode == OUT_ACCUM ? 1 : 0, s));
+                        return VF_OK;
+                    }
                     TRY(target(nd.src, &out, &ld, &mode));
                     if (!dry)
                         LAUNCH(net, launch_conv_start_rows(out, ld, M, pg, nd.W, g, mode == OUT_ACCUM ? 1 : 0, s));
                     return VF_OK;
+                }
+                WinLaunch wl;
+                if (e.windowed && !conv_back_win_plan(g, nd.ww, e.win, &wl)) {  // staging too large
+                    pend[v] = e;
+                    int b;
+                    TRY(make_plain(v, &b));
+                    e = pend[v];
+                    pend[v] = Entry();
                 }
                 const bool fuse = (nd.src == 0 && ext_in == nullptr && net->nodes[0].consumers == 1 &&
                                    pend[0].kind == E_NONE);
                 float* out = nullptr;
                 long long ld = 0;
                 int mode = OUT_CONCRETIZE;
+                if (e.windowed) {
+                    const Win nat = win_back(e.win, g);
+                    Win dst = nat;
+                    if (!fuse) TRY(target(nd.src, &out, &ld, &mode, &nat, &dst));
+                    if (!dry) {
+                        cudaEvent_t e0 = nullptr;
+                        prof_begin(&e0);
+                        LAUNCH(net, launch_conv_back_win(e.ref, e.rx, nd.ww, nd.b, M, g, pg, ps, e.win, dst, mode, out, ld,
+                                                         cst, centres, eps, s));
+                        const double pos = (double)std::min<long long>((long long)dst.hh * dst.hw, (long long)g.h * g.w);
+                        prof_end(e0, VF_KERNEL_CONV, 2.0 * (double)M * pos * g.ci * g.co * g.k * g.k /
+                                                         ((double)g.stride * g.stride));
+                    }
+                    release(e);
+                    return VF_OK;
+                }
                 if (!fuse) TRY(target(nd.src, &out, &ld, &mode));
                 if (fuse) part_tiles = conv_back_tiles(g);
                 if (!dry) {
@@ -470,8 +585,9 @@ bool input_buffered(const vf_net* net) {
     return true;
 }
 
-// Buffers a pass needs at once, by a dry run of the walker.
-int pool_size(vf_net* net, int start, Entry init, const std::vector<const float4*>* relax, bool ext, int* nb) {
+// Buffers a pass needs at once and the longest row they hold, by a dry run of the walker.
+int pool_size(vf_net* net, int start, Entry init, const std::vector<const float4*>* relax, bool ext, bool win_on,
+              int* nb, long long* max_len) {
     Walker w;
     w.net = net;
     w.s = nullptr;
@@ -482,10 +598,12 @@ int pool_size(vf_net* net, int start, Entry init, const std::vector<const float4
     w.part = nullptr;
     w.ld_buf = 1;
     w.relax = relax;
+    w.win_on = win_on;
     float dummy = 0.f;
     w.ext_in = ext ? &dummy : nullptr;
     TRY(w.run(start, init));
     *nb = w.max_live;
+    *max_len = w.max_len;
     return VF_OK;
 }
 
@@ -556,9 +674,14 @@ int run_pass(vf_net* net, int start, Entry init, long long rows, long long R_pas
              const std::vector<const float4*>& relax, const float* centres, float eps, float* pass_out, float* ext_in,
              float* const_out, cudaStream_t s) {
     const bool ext = ext_in != nullptr;
+    const Node& sn = net->nodes[start];
+    // rows held as receptive-field windows: identity-trick passes that start at a convolution
+    const bool win_on = net->windows && !ext && init.kind == E_IDENT && sn.op == VF_CONV2D;
     int nb = 0;
-    TRY(pool_size(net, start, init, &relax, ext, &nb));
-    const long long nmax = (max_node_size(net, input_buffered(net)) + 31) / 32 * 32;  // 128-byte rows
+    long long max_len = 0;
+    TRY(pool_size(net, start, init, &relax, ext, win_on, &nb, &max_len));
+    long long nmax = (max_node_size(net, input_buffered(net)) + 31) / 32 * 32;  // 128-byte rows
+    if (win_on) nmax = std::max<long long>(32, (max_len + 31) / 32 * 32);
     int tiles = std::max(dense_back_tiles_n((int)net->nodes[0].n), dense_back_tc_tiles_n((int)net->nodes[0].n));
     for (size_t v = 1; v < net->nodes.size(); ++v)  // per-tile partials of every convolution step
         if (net->nodes[v].op == VF_CONV2D) tiles = std::max(tiles, conv_back_tiles(conv_geom(net, net->nodes[v])));
@@ -585,6 +708,8 @@ int run_pass(vf_net* net, int start, Entry init, long long rows, long long R_pas
     w.centres = centres;
     w.eps = eps;
     w.n_centres = rows / R_pass;
+    w.win_on = win_on;
+    w.ps = PassStart{sn.n, sn.h, sn.w};
     for (long long m0 = 0; m0 < rows; m0 += chunk) {
         w.M = std::min(chunk, rows - m0);
         w.pg = PassGeom{m0, R_pass};
@@ -839,6 +964,7 @@ void vf_net_destroy(vf_net* net) {
         cudaFree(nd.WtHi);
         cudaFree(nd.WtLo);
         cudaFree(nd.rowsum_abs);
+        cudaFree(nd.Wwin);
     }
     cudaFree(net->d_err);
     for (auto e : net->ev_free) cudaEventDestroy(e);
@@ -868,6 +994,7 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
     if (const char* f = getenv("VF_TEST_FAIL_AT")) net->fail_at = atoll(f);
     if (const char* f = getenv("VF_DENSE_KERNEL")) net->dense_kernel = (strcmp(f, "ffma") == 0) ? 1 : 0;
     if (const char* f = getenv("VF_TEST_TC_STALL")) net->tc_stall = atoi(f) != 0;
+    if (const char* f = getenv("VF_CONV_WINDOWS")) net->windows = atoi(f) != 0;
     CU(cudaMalloc(&net->d_err, sizeof(int)));
     CU(cudaMemset(net->d_err, 0, sizeof(int)));
     net->nodes.resize(n_nodes);
@@ -958,6 +1085,22 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
                 TRY(upload(x.W, cnt, true, &nd.Wabs, host));
                 TRY(upload(x.b, nd.c, false, &nd.b, host));
                 ConvGeom g = conv_geom(net, nd);
+                {  // tap-major copy [k*k][co][ci_pad] (+4 floats of skew per tap) for the windowed kernel
+                    const int cb = win_ci_block(g.ci);
+                    const int ci_pad = (g.ci + cb - 1) / cb * cb;
+                    const int ts = g.co * ci_pad + 4;
+                    std::vector<float> wt((size_t)g.k * g.k * ts, 0.f), w0((size_t)cnt);
+                    CU(cudaMemcpy(w0.data(), nd.W, sizeof(float) * cnt, cudaMemcpyDeviceToHost));
+                    for (int co = 0; co < g.co; ++co)
+                        for (int ci = 0; ci < g.ci; ++ci)
+                            for (int p = 0; p < g.k; ++p)
+                                for (int q = 0; q < g.k; ++q)
+                                    wt[(size_t)(p * g.k + q) * ts + (size_t)co * ci_pad + ci] =
+                                        w0[(((size_t)co * g.ci + ci) * g.k + p) * g.k + q];
+                    CU(cudaMalloc(&nd.Wwin, sizeof(float) * wt.size()));
+                    CU(cudaMemcpy(nd.Wwin, wt.data(), sizeof(float) * wt.size(), cudaMemcpyHostToDevice));
+                    nd.ww = WinWeights{nd.Wwin, ts, ci_pad, cb};
+                }
                 if (!conv_back_supported(g))
                     return fail(VF_ERR_UNSUPPORTED,
                                 "node %d: convolution geometry not supported (stride 1/2/4, pad <= k-1, output covered "

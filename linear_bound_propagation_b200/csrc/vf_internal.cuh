@@ -64,6 +64,56 @@ cudaError_t launch_conv_back(const RowRef& A, Relax rx, const float* W, const fl
                              const ConvGeom& g, PassGeom pg, int out_mode, float* out, long long ld_out, float* cpart,
                              const float* centres, float eps, int num_sms, cudaStream_t s);
 
+// ---- receptive-field windows (k_win.cu) ----------------------------------------------
+// In a pass that starts at a convolution node p, the row of start neuron j = (c_j, y_j, x_j) is nonzero
+// only inside the receptive field of (y_j, x_j) on every map below p. Such rows are stored as a window
+// [C][hh][hw] whose origin on the map is (ay * y_j + by, ax * x_j + bx). Entries that fall outside the
+// map are held as zeros. ay = ax = by = bx = 0 with hh, hw the map's height and width is the whole map,
+// i.e. the plain row layout.
+struct Win {
+    int C, hh, hw;
+    int ay, by, ax, bx;
+};
+// The start node of the pass: neurons per centre, output height and width. Row r of a centre starts
+// from +e_j (r < n) or -e_j (r >= n), j = r mod n.
+struct PassStart {
+    long long n;
+    int h, w;
+};
+// Start rows +-(row j of the convolution's matrix) over the convolution's input, written into window
+// `wd`, which must contain the k x k field of every start neuron.
+cudaError_t launch_conv_start_rows_win(float* out, long long ld, long long M, PassGeom pg, PassStart ps, const float* W,
+                                       const ConvGeom& g, const Win& wd, int accumulate, cudaStream_t s);
+// Weights of a convolution in the layout of the windowed transposed convolution: tap (p, q) at
+// Wt + (p * k + q) * tap_stride holds [co][ci_pad] (ci padded to a multiple of cb, the input channels a
+// thread accumulates at once); tap_stride = co * ci_pad + 4 floats.
+struct WinWeights {
+    const float* Wt;
+    int tap_stride, ci_pad, cb;
+};
+int win_ci_block(int ci);
+constexpr int kWinSmemLimit = 220 * 1024;
+struct WinLaunch {
+    int nwarps, stage_floats, w_in_smem, ctas_per_sm;
+    size_t smem;
+};
+// Launch shape of the windowed transposed convolution for rows in window `wa`; false when one row's
+// staging does not fit in shared memory.
+bool conv_back_win_plan(const ConvGeom& g, const WinWeights& ww, const Win& wa, WinLaunch* L);
+// Transposed convolution of windowed rows: A over the conv output in window `wa` (relaxed on load by rx,
+// bias added to cst) onto the conv input in window `wd` (which must contain the receptive field of `wa`).
+// OUT_CONCRETIZE adds the concretised rows to cst instead of storing them. cst[m] receives one sum per
+// launch and row.
+cudaError_t launch_conv_back_win(const RowRef& A, Relax rx, const WinWeights& ww, const float* bias, long long M,
+                                 const ConvGeom& g, PassGeom pg, PassStart ps, const Win& wa, const Win& wd,
+                                 int out_mode, float* out, long long ld_out, float* cst, const float* centres, float eps,
+                                 cudaStream_t s);
+// Re-windowing of rows over one map of C x H x W: out (=, +=) relax(A) moved from window `wa` into `wd`
+// (which must contain `wa`); relaxation constants (rx.count_const) go to cst.
+cudaError_t launch_rewin_rows(const RowRef& A, Relax rx, long long M, int C, int H, int W, PassGeom pg, PassStart ps,
+                              const Win& wa, const Win& wd, float* out, long long ld_out, int accumulate, float* cst,
+                              cudaStream_t s);
+
 // ---- IBP (k_ibp.cu) -------------------------------------------------------------------
 // rowsum_abs (optional): sum_k |W[n, k]|, used with `eps` when the source is the input box (radius eps everywhere).
 cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,

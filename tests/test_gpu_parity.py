@@ -77,19 +77,56 @@ def test_cfg2_subset_ragged():
     assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out)
 
 
-def test_cfg3_subset():
+@pytest.mark.parametrize("windows", ["1", "0"])
+def test_cfg3_subset(monkeypatch, windows):
+    monkeypatch.setenv("VF_CONV_WINDOWS", windows)
     w = synth.workload(3, B=3)
     g, ora, out = run_both(w.net, w.centres, w.eps, w.C)
     assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out)
 
 
-def test_resnet_small_all_paths():
+@pytest.mark.parametrize("windows", ["1", "0"])
+def test_resnet_small_all_paths(monkeypatch, windows):
+    monkeypatch.setenv("VF_CONV_WINDOWS", windows)
     rng = np.random.default_rng(41)
     net = synth.resnet_cfg4(rng, image=(3, 12, 12), widths=(5, 6, 7), fc=20, classes=7)
     centres = rng.random((3, 3 * 12 * 12)).astype(np.float32)
     C = synth.margin_spec(rng.integers(0, 7, 3), 7)
     g, ora, out = run_both(net, centres, np.float32(0.01).item(), C, both=True)
     assert_parity(net, centres, 0.01, C, g, ora, out, both=True)
+
+
+def _conv_flops(net, centres, eps, C, both):
+    g = vf.Net(net)
+    g.profile(True)
+    g.profile_read(reset=True)
+    out = g.verify(_dev(centres), eps, _dev(C), both_sides=both, want_pre=True)
+    torch.cuda.synchronize()
+    g.check()
+    fl = g.profile_read(kind=3)[2]
+    return fl, {k: v.cpu().numpy() for k, v in out.items()}
+
+
+def test_receptive_field_windows_through_residual_adds(monkeypatch):
+    """A residual net on a map large enough that windows survive the residual adds (union of the two
+    branches' windows, identity shortcuts that share rows, windows that outgrow the map and return to
+    whole-map rows). Windowed and whole-map passes both match the oracle, and the windowed run does
+    less convolution work."""
+    rng = np.random.default_rng(43)
+    net = synth.resnet_cfg4(rng, image=(3, 20, 20), widths=(3, 4, 5), fc=12, classes=5)
+    B = 2
+    centres = rng.random((B, 3 * 20 * 20)).astype(np.float32)
+    C = synth.margin_spec(rng.integers(0, 5, B), 5)
+    eps = 0.01
+    ora = O.verify(net, centres, eps, C, both_sides=True)
+    res = {}
+    for windows in ("1", "0"):
+        monkeypatch.setenv("VF_CONV_WINDOWS", windows)
+        fl, out = _conv_flops(net, centres, eps, C, True)
+        g = vf.Net(net)
+        assert_parity(net, centres, eps, C, g, ora, out, both=True)
+        res[windows] = fl
+    assert res["1"] < 0.7 * res["0"], res
 
 
 @pytest.mark.parametrize("eps", [0.5 / 255, 1.0 / 255, 2.0 / 255])
