@@ -154,7 +154,7 @@ def roofline(kstats, step_total_ms, n_sms):
     else:
         peak = n_sms * 128 * 2 * sm_mhz * 1e6 / 1e12
         bound = "alu"
-        name = "dense_back_ffma" if kind == 2 else "conv_back_ffma"
+        name = {2: "dense_back_ffma", 3: "conv_back_ffma", 4: "conv_back_win_k (receptive-field windows)"}[kind]
         psrc = f"fp32 FFMA: {n_sms} SMs x 128 lanes x 2 flop x {sm_mhz:.0f} MHz ({src} max clock)"
     return {"bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": None, "kernel": name, "launches": n_k, "avg_launch_ms": avg_ms,
@@ -256,7 +256,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     clocks = stop_clocks(clk)
     launches = net.launch_count() - launches0
-    kstats = {k: net.profile_read(kind=k, reset=False) for k in (1, 2, 3)}
+    kstats = {k: net.profile_read(kind=k, reset=False) for k in (1, 2, 3, 4)}
     net.profile_read(reset=True)
     net.profile(False)
     step_ms = [a.elapsed_time(b) for a, b in ev]

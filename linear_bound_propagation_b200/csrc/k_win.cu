@@ -72,6 +72,26 @@ conv_start_rows_win_k(float* __restrict__ out, long long ld, long long M, PassGe
     }
 }
 
+// Identity start rows (+-e_j) in window `wd` of the start node's map (the identity shortcut of a pass that
+// starts at a residual add). One warp per row.
+__global__ void __launch_bounds__(256)
+ident_rows_win_k(float* __restrict__ out, long long ld, long long M, PassGeom pg, PassStart ps, Win wd,
+                 int accumulate) {
+    const int nwin = wd.C * wd.hh * wd.hw;
+    const int lane = threadIdx.x & 31;
+    for (long long m = blockIdx.x * 8LL + (threadIdx.x >> 5); m < M; m += (long long)gridDim.x * 8) {
+        const StartPos sp = start_pos(ps, pg, m);
+        const int dy = sp.yj - (wd.ay * sp.yj + wd.by), dx = sp.xj - (wd.ax * sp.xj + wd.bx);
+        const int hit = (sp.cj * wd.hh + dy) * wd.hw + dx;  // inside the window by construction
+        float* o = out + m * ld;
+        if (accumulate) {
+            if (lane == 0) o[hit] += sp.sg;
+        } else {
+            for (int e = lane; e < nwin; e += 32) o[e] = (e == hit) ? sp.sg : 0.f;
+        }
+    }
+}
+
 // Transposed convolution on windowed rows. One warp per row, `nwarps` rows per CTA. The relaxed row
 // window over the conv output is staged in shared memory ([co][hh][hw], zeros off the map); each lane
 // then owns output positions of the destination window and CB input channels at a time, gathering its
@@ -289,6 +309,13 @@ cudaError_t launch_conv_back_win(const RowRef& A, Relax rx, const WinWeights& ww
             return launch_back_cb<16>(A, rx, ww, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst, centres, eps, L,
                                       s);
     }
+}
+
+cudaError_t launch_ident_rows_win(float* out, long long ld, long long M, PassGeom pg, PassStart ps, const Win& wd,
+                                  int accumulate, cudaStream_t s) {
+    if (M <= 0) return cudaSuccess;
+    ident_rows_win_k<<<warp_rows_grid(M, 8, 8), 256, 0, s>>>(out, ld, M, pg, ps, wd, accumulate);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_rewin_rows(const RowRef& A, Relax rx, long long M, int C, int H, int W, PassGeom pg, PassStart ps,

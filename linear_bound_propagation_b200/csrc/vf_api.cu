@@ -94,6 +94,7 @@ struct vf_net {
     int* d_err = nullptr;   // device flag raised by a kernel whose bounded wait expired
     int tc_stall = 0;       // test hook: VF_TEST_TC_STALL=1 makes one tensor-core launch time out
     int windows = 1;        // receptive-field windows in passes that start at a convolution (VF_CONV_WINDOWS=0: off)
+    int conv_whole_warp = 0;  // whole-map rows through the one-warp-per-row kernel (VF_CONV_KERNEL=warp)
     bool prof = false;
     std::vector<cudaEvent_t> ev_free;
     struct Timed {
@@ -102,9 +103,9 @@ struct vf_net {
         double flops;
     };
     std::vector<Timed> ev_used;
-    double prof_flops[4] = {0, 0, 0, 0};
-    long long prof_launches[4] = {0, 0, 0, 0};
-    double prof_ms[4] = {0, 0, 0, 0};
+    double prof_flops[5] = {0, 0, 0, 0, 0};
+    long long prof_launches[5] = {0, 0, 0, 0, 0};
+    double prof_ms[5] = {0, 0, 0, 0, 0};
 };
 
 namespace {
@@ -186,6 +187,8 @@ struct Entry {
 
 // Receptive-field windows (rows of a pass that starts at a convolution, see k_win.cu).
 Win full_win(const Node& nd) { return Win{nd.c, nd.h, nd.w, 0, 0, 0, 0}; }
+// The 1 x 1 window at the start position: identity start rows on a node shaped like the start node.
+Win ident_win(const Node& nd) { return Win{nd.c, 1, 1, 1, 0, 1, 0}; }
 long long win_len(const Win& w) { return (long long)w.C * w.hh * w.hw; }
 bool win_eq(const Win& a, const Win& b) {
     return a.C == b.C && a.hh == b.hh && a.hw == b.hw && a.ay == b.ay && a.by == b.by && a.ax == b.ax && a.bx == b.bx;
@@ -289,11 +292,12 @@ struct Walker {
             *out = e.buf;
             return VF_OK;
         }
-        if (e.kind == E_IDENT && want != nullptr) return fail(VF_ERR_ARG, "internal: identity rows cannot be windowed");
         int nb;
         TRY(alloc_buf(&nb, want ? win_len(*want) : n));
         if (!dry) {
-            if (e.kind == E_IDENT)
+            if (e.kind == E_IDENT && want != nullptr)
+                LAUNCH(net, launch_ident_rows_win(bufs[nb], ld_buf, M, pg, ps, *want, 0, s));
+            else if (e.kind == E_IDENT)
                 LAUNCH(net, launch_ident_rows(bufs[nb], ld_buf, M, pg, n, 0, s));
             else if (!e.windowed && want == nullptr)
                 LAUNCH(net, launch_relax_rows(e.ref, e.rx, M, (int)n, pg, bufs[nb], ld_buf, 0, cst, s));
@@ -311,10 +315,23 @@ struct Walker {
         return VF_OK;
     }
 
+    // Window of entry e at node v; false for whole-map rows.
+    bool entry_win(int v, const Entry& e, Win* w) const {
+        if (e.windowed) {
+            *w = e.win;
+            return true;
+        }
+        if (e.kind == E_IDENT && win_on && e.rx.P == nullptr && win_small(ident_win(net->nodes[v]), net->nodes[v])) {
+            *w = ident_win(net->nodes[v]);
+            return true;
+        }
+        return false;
+    }
+
     // The window that holds both pend[v] and rows in window x (null: the whole map).
     bool merged_win(int v, const Win* x, Win* u) const {
-        const Entry& e = pend[v];
-        return x != nullptr && e.windowed && win_union(e.win, *x, u) && win_small(*u, net->nodes[v]);
+        Win ew;
+        return x != nullptr && entry_win(v, pend[v], &ew) && win_union(ew, *x, u) && win_small(*u, net->nodes[v]);
     }
 
     // pend[v] += x (x is consumed).
@@ -325,12 +342,15 @@ struct Walker {
         }
         const Node& nd = net->nodes[v];
         const long long n = nd.n;
-        Win u;
-        const bool wu = merged_win(v, x.windowed ? &x.win : nullptr, &u);
+        Win xw, u;
+        const bool xwin = entry_win(v, x, &xw);
+        const bool wu = merged_win(v, xwin ? &xw : nullptr, &u);
         int b;
         TRY(make_plain(v, &b, wu ? &u : nullptr));
         if (!dry) {
-            if (x.kind == E_IDENT)
+            if (x.kind == E_IDENT && wu)
+                LAUNCH(net, launch_ident_rows_win(bufs[b], ld_buf, M, pg, ps, u, 1, s));
+            else if (x.kind == E_IDENT)
                 LAUNCH(net, launch_ident_rows(bufs[b], ld_buf, M, pg, n, 1, s));
             else if (!x.windowed && !wu)
                 LAUNCH(net, launch_relax_rows(x.ref, x.rx, M, (int)n, pg, bufs[b], ld_buf, 1, cst, s));
@@ -422,9 +442,11 @@ struct Walker {
             }
             case VF_RELU: {
                 if (e.kind == E_IDENT || e.rx.P != nullptr) {
+                    Win ew;
+                    const bool wnd = entry_win(v, e, &ew);
                     pend[v] = e;
                     int b;
-                    TRY(make_plain(v, &b, e.windowed ? &e.win : nullptr));
+                    TRY(make_plain(v, &b, wnd ? &ew : nullptr));
                     e = pend[v];
                     pend[v] = Entry();
                 }
@@ -481,6 +503,7 @@ struct Walker {
             }
             case VF_CONV2D: {
                 const ConvGeom g = conv_geom(net, nd);
+                const Node& sn = net->nodes[nd.src];
                 if (e.kind == E_IDENT) {
                     if (!dry)
                         LAUNCH(net, launch_cst_identity_bias(cst, M, pg, nd.b, nd.n, (long long)nd.h * nd.w, s));
@@ -502,6 +525,11 @@ struct Walker {
                     return VF_OK;
                 }
                 WinLaunch wl;
+                if (!e.windowed && e.kind != E_IDENT && net->conv_whole_warp &&
+                    conv_back_win_plan(g, nd.ww, full_win(nd), &wl)) {  // whole-map rows as one full window
+                    e.windowed = true;
+                    e.win = full_win(nd);
+                }
                 if (e.windowed && !conv_back_win_plan(g, nd.ww, e.win, &wl)) {  // staging too large
                     pend[v] = e;
                     int b;
@@ -516,7 +544,7 @@ struct Walker {
                 int mode = OUT_CONCRETIZE;
                 if (e.windowed) {
                     const Win nat = win_back(e.win, g);
-                    Win dst = nat;
+                    Win dst = win_small(nat, sn) ? nat : full_win(sn);
                     if (!fuse) TRY(target(nd.src, &out, &ld, &mode, &nat, &dst));
                     if (!dry) {
                         cudaEvent_t e0 = nullptr;
@@ -524,7 +552,7 @@ struct Walker {
                         LAUNCH(net, launch_conv_back_win(e.ref, e.rx, nd.ww, nd.b, M, g, pg, ps, e.win, dst, mode, out, ld,
                                                          cst, centres, eps, s));
                         const double pos = (double)std::min<long long>((long long)dst.hh * dst.hw, (long long)g.h * g.w);
-                        prof_end(e0, VF_KERNEL_CONV, 2.0 * (double)M * pos * g.ci * g.co * g.k * g.k /
+                        prof_end(e0, VF_KERNEL_CONV_WIN, 2.0 * (double)M * pos * g.ci * g.co * g.k * g.k /
                                                          ((double)g.stride * g.stride));
                     }
                     release(e);
@@ -675,8 +703,9 @@ int run_pass(vf_net* net, int start, Entry init, long long rows, long long R_pas
              float* const_out, cudaStream_t s) {
     const bool ext = ext_in != nullptr;
     const Node& sn = net->nodes[start];
-    // rows held as receptive-field windows: identity-trick passes that start at a convolution
-    const bool win_on = net->windows && !ext && init.kind == E_IDENT && sn.op == VF_CONV2D;
+    // rows held as receptive-field windows: identity-trick passes that start at a convolution or a residual add
+    const bool win_on =
+        net->windows && !ext && init.kind == E_IDENT && (sn.op == VF_CONV2D || sn.op == VF_ADD) && sn.h > 1;
     int nb = 0;
     long long max_len = 0;
     TRY(pool_size(net, start, init, &relax, ext, win_on, &nb, &max_len));
@@ -995,6 +1024,7 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
     if (const char* f = getenv("VF_DENSE_KERNEL")) net->dense_kernel = (strcmp(f, "ffma") == 0) ? 1 : 0;
     if (const char* f = getenv("VF_TEST_TC_STALL")) net->tc_stall = atoi(f) != 0;
     if (const char* f = getenv("VF_CONV_WINDOWS")) net->windows = atoi(f) != 0;
+    if (const char* f = getenv("VF_CONV_KERNEL")) net->conv_whole_warp = (strcmp(f, "warp") == 0) ? 1 : 0;
     CU(cudaMalloc(&net->d_err, sizeof(int)));
     CU(cudaMemset(net->d_err, 0, sizeof(int)));
     net->nodes.resize(n_nodes);
@@ -1332,7 +1362,7 @@ int vf_profile_enable(vf_net* net, int enable) {
 
 int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms, double* flops, int reset) {
     TRY(check_net(net));
-    if (kind < 0 || kind > 3) return fail(VF_ERR_ARG, "bad kernel kind");
+    if (kind < 0 || kind > 4) return fail(VF_ERR_ARG, "bad kernel kind");
     for (auto& t : net->ev_used) {
         CU(cudaEventSynchronize(t.e1));
         float ms = 0.f;
@@ -1350,7 +1380,7 @@ int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms
     if (total_ms) *total_ms = net->prof_ms[kind];
     if (flops) *flops = net->prof_flops[kind];
     if (reset)
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 5; ++k) {
             net->prof_launches[k] = 0;
             net->prof_ms[k] = 0.0;
             net->prof_flops[k] = 0.0;

@@ -108,6 +108,10 @@ cudaError_t launch_conv_back_win(const RowRef& A, Relax rx, const WinWeights& ww
                                  const ConvGeom& g, PassGeom pg, PassStart ps, const Win& wa, const Win& wd,
                                  int out_mode, float* out, long long ld_out, float* cst, const float* centres, float eps,
                                  cudaStream_t s);
+// Identity start rows +-e_j written into window `wd` (which must contain position (y_j, x_j)) of a map with
+// the start node's shape.
+cudaError_t launch_ident_rows_win(float* out, long long ld, long long M, PassGeom pg, PassStart ps, const Win& wd,
+                                  int accumulate, cudaStream_t s);
 // Re-windowing of rows over one map of C x H x W: out (=, +=) relax(A) moved from window `wa` into `wd`
 // (which must contain `wa`); relaxation constants (rx.count_const) go to cst.
 cudaError_t launch_rewin_rows(const RowRef& A, Relax rx, long long M, int C, int H, int W, PassGeom pg, PassStart ps,

@@ -103,7 +103,7 @@ def _conv_flops(net, centres, eps, C, both):
     out = g.verify(_dev(centres), eps, _dev(C), both_sides=both, want_pre=True)
     torch.cuda.synchronize()
     g.check()
-    fl = g.profile_read(kind=3)[2]
+    fl = g.profile_read(kind=3, reset=False)[2] + g.profile_read(kind=4)[2]  # whole-map + windowed
     return fl, {k: v.cpu().numpy() for k, v in out.items()}
 
 
