@@ -243,6 +243,228 @@ rewin_rows_k(RowRef A, Relax rx, long long M, int C, int H, int Wd, PassGeom pg,
     }
 }
 
+// Position-blocked variant of the windowed transposed convolution for stride S and KS = ceil(k / S) taps
+// per axis and stride class. The staged row window carries a zero halo, so every tap read stays inside
+// the stage and needs no test. Input positions of the receptive field are grouped by stride class
+// (y mod S, x mod S); within a class all positions use the same taps. A lane owns PM positions of one
+// class (spaced G apart along x, so neighbouring lanes read neighbouring stage words) times CB input
+// channels, i.e. PM*CB accumulators that share each staged weight and each staged coefficient.
+struct WinClasses {
+    int cum[5];  // items before class i (class = pc * S + qc), cum[S*S] = items per row and chunk
+    int ny[4], nx[4], G[4];
+};
+
+__device__ __forceinline__ int fdiv(int n, float inv) { return __float2int_rz(((float)n + 0.5f) * inv); }
+
+// a[i] for a small runtime i, by selects (keeps the parameter arrays out of local memory)
+template <int N>
+__device__ __forceinline__ int pick(const int (&a)[N], int i) {
+    int v = a[0];
+#pragma unroll
+    for (int j = 1; j < N; ++j) v = (i == j) ? a[j] : v;
+    return v;
+}
+
+template <int S, int KS, int CB, int PM>
+__global__ void __launch_bounds__(256, 2)
+conv_back_win2_k(RowRef A, Relax rx, const float* __restrict__ Wt, int tap_stride, int ci_pad, int w_all,
+                 const float* __restrict__ bias, long long M, ConvGeom g, PassGeom pg, PassStart ps, Win wa, Win wd,
+                 int out_mode, float* __restrict__ out, long long ld_out, float* __restrict__ cst,
+                 const float* __restrict__ centres, float eps, int nwarps, int HH, int HW, int stage_floats,
+                 WinClasses cl, float inv_hwd, int zero_fill) {
+    extern __shared__ float4 smem4[];
+    float* sm = reinterpret_cast<float*>(smem4);
+    constexpr int OFF = KS - 1;
+    const int kk = g.k * g.k;
+    const int slab_ts = g.co * CB + 4;
+    const int nW = w_all ? kk * tap_stride : kk * slab_ts;
+    const int TSs = w_all ? tap_stride : slab_ts;  // smem stride between taps
+    const int COS = w_all ? ci_pad : CB;           // smem stride between output channels
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float* As = sm + nW + warp * stage_floats;
+    const int HHW = HH * HW;
+    const int nst = wa.C * HHW;
+    const int hw_o = g.ho * g.wo;
+    const long long nOut = (long long)g.co * hw_o;
+    const int npos_d = wd.hh * wd.hw;
+    const int nchunks = ci_pad / CB;
+    const int NYT = S * (wa.hh - 1) + g.k, NXT = S * (wa.hw - 1) + g.k;  // receptive field on the input map
+    const long long S_in = (long long)g.h * g.w;
+    if (w_all) {
+        const float4* src = reinterpret_cast<const float4*>(Wt);
+        for (int e = threadIdx.x; e < nW / 4; e += blockDim.x) smem4[e] = src[e];
+    }
+    // the halo of the stage is zero for every row: clear it once, then rows write the interior only
+    for (int e = lane; e < nst; e += 32) As[e] = 0.f;
+    const int na = wa.C * wa.hh * wa.hw;
+    const float inv_a = 1.f / (float)(wa.hh * wa.hw), inv_aw = 1.f / (float)wa.hw;
+    for (long long m0 = (long long)blockIdx.x * nwarps; m0 < M; m0 += (long long)gridDim.x * nwarps) {
+        const long long m = m0 + warp;
+        const bool active = warp < nwarps && m < M;
+        StartPos sp{0, 0, 0, 1.f, 0};
+        int aoy = 0, aox = 0, fy0 = 0, fx0 = 0, doy = 0, dox = 0;
+        float cs = 0.f, conc = 0.f;
+        if (active) {
+            sp = start_pos(ps, pg, m);
+            aoy = wa.ay * sp.yj + wa.by;
+            aox = wa.ax * sp.xj + wa.bx;
+            fy0 = S * aoy - g.pad;
+            fx0 = S * aox - g.pad;
+            doy = wd.ay * sp.yj + wd.by;
+            dox = wd.ax * sp.xj + wd.bx;
+            const float* arow = A.row(m);
+            // four entries per lane at a time: all their loads are issued before any is used
+            const float4* Pb = rx.P != nullptr ? rx.P + sp.b * nOut : nullptr;
+            for (int e0 = lane; e0 < na; e0 += 128) {
+                float xv[4];
+                float4 pr[4];
+                int co[4], sidx[4];
+                bool on[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + 32 * u;
+                    const int c = fdiv(e, inv_a);
+                    const int r2 = e - c * (wa.hh * wa.hw);
+                    const int wy = fdiv(r2, inv_aw);
+                    const int wx = r2 - wy * wa.hw;
+                    const int y = aoy + wy, x = aox + wx;
+                    on[u] = e < na && y >= 0 && y < g.ho && x >= 0 && x < g.wo;
+                    co[u] = c;
+                    sidx[u] = c * HHW + (wy + OFF) * HW + wx + OFF;
+                    xv[u] = on[u] ? arow[e] : 0.f;
+                    pr[u] = (on[u] && Pb != nullptr) ? Pb[(long long)c * hw_o + y * g.wo + x] : make_float4(1.f, 1.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (e0 + 32 * u >= na) break;
+                    float v = 0.f;
+                    if (on[u]) {
+                        v = (xv[u] >= 0.f) ? xv[u] * pr[u].x : xv[u] * pr[u].y;
+                        if (Pb != nullptr && rx.count_const) cs = fmaf(fminf(xv[u], 0.f), pr[u].z, cs);
+                        if (bias != nullptr) cs = fmaf(v, bias[co[u]], cs);
+                    }
+                    As[sidx[u]] = v;
+                }
+            }
+            if (zero_fill) {  // destination entries outside the receptive field
+                float* orow = out + m * ld_out;
+                for (int e = lane; e < npos_d; e += 32) {
+                    const int yd = fdiv(e, inv_hwd);
+                    const int y = doy + yd - fy0, x = dox + (e - yd * wd.hw) - fx0;
+                    if (y >= 0 && y < NYT && x >= 0 && x < NXT) continue;
+                    for (int ci = 0; ci < g.ci; ++ci) orow[(long long)ci * npos_d + e] = 0.f;
+                }
+            }
+        }
+        for (int chunk = 0; chunk < nchunks; ++chunk) {
+            if (!w_all) {  // this chunk's weight slab [tap][co][CB]
+                __syncthreads();
+                for (int e = threadIdx.x; e < kk * g.co * (CB / 4); e += blockDim.x) {
+                    const int c4 = e % (CB / 4), rest = e / (CB / 4);
+                    const int co = rest % g.co, tap = rest / g.co;
+                    smem4[(tap * slab_ts + co * CB) / 4 + c4] =
+                        reinterpret_cast<const float4*>(Wt + (size_t)tap * tap_stride + (size_t)co * ci_pad + chunk * CB)[c4];
+                }
+            }
+            __syncthreads();
+            if (!active) continue;
+            const float* Wc = sm + (w_all ? chunk * CB : 0);
+            for (int it = lane; it < cl.cum[S * S]; it += 32) {
+                int cls = 0, base = 0;
+#pragma unroll
+                for (int c2 = 1; c2 < S * S; ++c2)
+                    if (it >= cl.cum[c2]) {
+                        cls = c2;
+                        base = cl.cum[c2];
+                    }
+                const int pc = cls / S, qc = cls % S;
+                const int Gc = pick(cl.G, qc), nxc = pick(cl.nx, qc);
+                const int local = it - base;
+                const int yq = local / Gc, grp = local - yq * Gc;
+                float acc[PM][CB];
+#pragma unroll
+                for (int i = 0; i < PM; ++i)
+#pragma unroll
+                    for (int c = 0; c < CB; ++c) acc[i][c] = 0.f;
+                bool okp[PM];
+#pragma unroll
+                for (int i = 0; i < PM; ++i) okp[i] = grp + i * Gc < nxc;
+#pragma unroll
+                for (int tp = 0; tp < KS; ++tp) {
+                    const int p = pc + S * tp;
+                    if (p >= g.k) break;
+                    const float* arow_s = As + (yq - tp + OFF) * HW + grp;
+#pragma unroll
+                    for (int tq = 0; tq < KS; ++tq) {
+                        const int q = qc + S * tq;
+                        if (q >= g.k) break;
+                        const float* ab = arow_s + (OFF - tq);
+                        const float4* wb = reinterpret_cast<const float4*>(Wc + (p * g.k + q) * TSs);
+#pragma unroll 2
+                        for (int co = 0; co < g.co; ++co) {
+                            float a[PM];
+#pragma unroll
+                            for (int i = 0; i < PM; ++i) {  // a lane's unused slots read its first (valid) position
+                                const float v = ab[co * HHW + (okp[i] ? i * Gc : 0)];
+                                a[i] = okp[i] ? v : 0.f;
+                            }
+#pragma unroll
+                            for (int c4 = 0; c4 < CB / 4; ++c4) {
+                                const float4 w4 = wb[(co * COS) / 4 + c4];
+#pragma unroll
+                                for (int i = 0; i < PM; ++i) {
+                                    acc[i][4 * c4 + 0] = fmaf(a[i], w4.x, acc[i][4 * c4 + 0]);
+                                    acc[i][4 * c4 + 1] = fmaf(a[i], w4.y, acc[i][4 * c4 + 1]);
+                                    acc[i][4 * c4 + 2] = fmaf(a[i], w4.z, acc[i][4 * c4 + 2]);
+                                    acc[i][4 * c4 + 3] = fmaf(a[i], w4.w, acc[i][4 * c4 + 3]);
+                                }
+                            }
+                        }
+                    }
+                }
+                const int Y = fy0 + pc + S * yq;
+#pragma unroll
+                for (int i = 0; i < PM; ++i) {
+                    if (!okp[i]) continue;
+                    const int X = fx0 + qc + S * (grp + i * Gc);
+                    const bool onmap = Y >= 0 && Y < g.h && X >= 0 && X < g.w;
+                    if (out_mode == OUT_CONCRETIZE) {
+                        if (!onmap) continue;
+                        const float* cp = centres + sp.b * (long long)g.ci * S_in + (long long)Y * g.w + X;
+#pragma unroll
+                        for (int c = 0; c < CB; ++c) {
+                            const int ci = chunk * CB + c;
+                            if (ci < g.ci) conc += fmaf(acc[i][c], cp[ci * S_in], -eps * fabsf(acc[i][c]));
+                        }
+                    } else {
+                        const int yd = Y - doy, xd = X - dox;
+                        if (yd < 0 || yd >= wd.hh || xd < 0 || xd >= wd.hw) continue;
+                        float* o = out + m * ld_out + yd * wd.hw + xd;
+#pragma unroll
+                        for (int c = 0; c < CB; ++c) {
+                            const int ci = chunk * CB + c;
+                            if (ci >= g.ci) break;
+                            const float v = onmap ? acc[i][c] : 0.f;
+                            float* oc = o + (long long)ci * npos_d;
+                            *oc = (out_mode == OUT_ACCUM) ? *oc + v : v;
+                        }
+                    }
+                }
+            }
+        }
+        if (active) {
+            const float tot = warp_sum(cs + conc);
+            if (lane == 0 && cst != nullptr) cst[m] += tot;
+        }
+    }
+}
+
+struct Win2Launch {
+    int nwarps, HH, HW, stage_floats, w_all, ctas_per_sm, zero_fill;
+    size_t smem;
+    WinClasses cl;
+};
+
 template <int CB>
 cudaError_t launch_back_cb(const RowRef& A, Relax rx, const WinWeights& ww, const float* bias, long long M,
                            const ConvGeom& g, PassGeom pg, PassStart ps, const Win& wa, const Win& wd, int out_mode,
@@ -259,6 +481,108 @@ cudaError_t launch_back_cb(const RowRef& A, Relax rx, const WinWeights& ww, cons
         A, rx, ww.Wt, ww.tap_stride, ww.ci_pad, L.w_in_smem, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst,
         centres, eps, L.nwarps, L.stage_floats);
     return cudaGetLastError();
+}
+
+template <int S, int KS, int CB, int PM>
+cudaError_t launch_back2(const RowRef& A, Relax rx, const WinWeights& ww, const float* bias, long long M,
+                         const ConvGeom& g, PassGeom pg, PassStart ps, const Win& wa, const Win& wd, int out_mode,
+                         float* out, long long ld_out, float* cst, const float* centres, float eps,
+                         const Win2Launch& L, cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(conv_back_win2_k<S, KS, CB, PM>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kWinSmemLimit);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    const float inv_hwd = 1.f / (float)wd.hw;
+    int per_sm = 0;  // resident CTAs per SM (registers and shared memory)
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, conv_back_win2_k<S, KS, CB, PM>,
+                                                                  32 * L.nwarps, L.smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    conv_back_win2_k<S, KS, CB, PM><<<warp_rows_grid(M, L.nwarps, std::min(per_sm, 8)), 32 * L.nwarps, L.smem, s>>>(
+        A, rx, ww.Wt, ww.tap_stride, ww.ci_pad, L.w_all, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst,
+        centres, eps, L.nwarps, L.HH, L.HW, L.stage_floats, L.cl, inv_hwd, L.zero_fill);
+    return cudaGetLastError();
+}
+
+template <int S, int KS, int CB>
+cudaError_t launch_back2_pm(const RowRef& A, Relax rx, const WinWeights& ww, const float* bias, long long M,
+                            const ConvGeom& g, PassGeom pg, PassStart ps, const Win& wa, const Win& wd, int out_mode,
+                            float* out, long long ld_out, float* cst, const float* centres, float eps,
+                            const Win2Launch& L, int pm, cudaStream_t s) {
+    if (pm == 4)
+        return launch_back2<S, KS, CB, 4>(A, rx, ww, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst, centres,
+                                          eps, L, s);
+    return launch_back2<S, KS, CB, 1>(A, rx, ww, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst, centres, eps,
+                                      L, s);
+}
+
+template <int S, int KS>
+cudaError_t launch_back2_cb(const RowRef& A, Relax rx, const WinWeights& ww, const float* bias, long long M,
+                            const ConvGeom& g, PassGeom pg, PassStart ps, const Win& wa, const Win& wd, int out_mode,
+                            float* out, long long ld_out, float* cst, const float* centres, float eps,
+                            const Win2Launch& L, int pm, cudaStream_t s) {
+    switch (ww.cb) {
+        case 4:
+            return launch_back2_pm<S, KS, 4>(A, rx, ww, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst,
+                                             centres, eps, L, pm, s);
+        case 8:
+            return launch_back2_pm<S, KS, 8>(A, rx, ww, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst,
+                                             centres, eps, L, pm, s);
+        default:
+            return launch_back2_pm<S, KS, 16>(A, rx, ww, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst,
+                                              centres, eps, L, pm, s);
+    }
+}
+
+// Launch shape of the position-blocked kernel; false when (stride, taps) has no instance or a row's
+// staging does not fit.
+bool conv_back_win2_plan(const ConvGeom& g, const WinWeights& ww, const Win& wa, const Win& wd, int out_mode,
+                         Win2Launch* L, int* pm) {
+    const int S = g.stride, KS = (g.k + g.stride - 1) / g.stride;
+    if (!((S == 1 && (KS == 1 || KS == 3)) || (S == 2 && (KS == 1 || KS == 2)))) return false;
+    L->HH = wa.hh + KS - 1 + (g.k - 1) / S;
+    L->HW = wa.hw + KS - 1 + (g.k - 1) / S;
+    L->stage_floats = (wa.C * L->HH * L->HW + 3) / 4 * 4;
+    const size_t stage = (size_t)L->stage_floats * sizeof(float);
+    const size_t w_all = (size_t)g.k * g.k * ww.tap_stride * sizeof(float);
+    const size_t w_slab = (size_t)g.k * g.k * (g.co * ww.cb + 4) * sizeof(float);
+    const size_t lim = (size_t)kWinSmemLimit;
+    int nw = w_all < lim ? (int)std::min<size_t>(8, (lim - w_all) / stage) : 0;
+    if (nw >= 4) {
+        L->w_all = 1;
+        L->smem = w_all + (size_t)nw * stage;
+    } else {
+        if (w_slab >= lim) return false;
+        nw = (int)std::min<size_t>(8, (lim - w_slab) / stage);
+        if (nw < 1) return false;
+        L->w_all = 0;
+        L->smem = w_slab + (size_t)nw * stage;
+    }
+    L->nwarps = nw;
+    L->ctas_per_sm = std::max(1, std::min(8, (int)(233472 / (L->smem + 1024))));
+    const int NYT = S * (wa.hh - 1) + g.k, NXT = S * (wa.hw - 1) + g.k;
+    *pm = (NYT * NXT >= 256) ? 4 : 1;
+    int acc = 0;
+    for (int pc = 0; pc < S; ++pc)
+        for (int qc = 0; qc < S; ++qc) {
+            const int c = pc * S + qc;
+            L->cl.ny[pc] = (NYT - pc + S - 1) / S;
+            L->cl.nx[qc] = (NXT - qc + S - 1) / S;
+            L->cl.G[qc] = (L->cl.nx[qc] + *pm - 1) / *pm;
+            L->cl.cum[c] = acc;
+            acc += L->cl.ny[pc] * L->cl.G[qc];
+        }
+    L->cl.cum[S * S] = acc;
+    for (int c = S * S + 1; c < 5; ++c) L->cl.cum[c] = acc;
+    // a STORE into a destination larger than the receptive field must zero the rest of it
+    const int doff_y = wd.ay == S * wa.ay ? (S * wa.by - g.pad) - wd.by : 1;
+    const int doff_x = wd.ax == S * wa.ax ? (S * wa.bx - g.pad) - wd.bx : 1;
+    const bool exact = doff_y == 0 && doff_x == 0 && wd.hh == NYT && wd.hw == NXT;
+    L->zero_fill = (out_mode == OUT_STORE && !exact) ? 1 : 0;
+    return true;
 }
 
 }  // namespace
@@ -298,6 +622,22 @@ cudaError_t launch_conv_back_win(const RowRef& A, Relax rx, const WinWeights& ww
                                  int out_mode, float* out, long long ld_out, float* cst, const float* centres, float eps,
                                  cudaStream_t s) {
     if (M <= 0) return cudaSuccess;
+    Win2Launch L2;
+    int pm = 1;
+    if (!ww.per_position && conv_back_win2_plan(g, ww, wa, wd, out_mode, &L2, &pm)) {
+        const int KS = (g.k + g.stride - 1) / g.stride;
+        if (g.stride == 1 && KS == 1)
+            return launch_back2_cb<1, 1>(A, rx, ww, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst, centres,
+                                         eps, L2, pm, s);
+        if (g.stride == 1)
+            return launch_back2_cb<1, 3>(A, rx, ww, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst, centres,
+                                         eps, L2, pm, s);
+        if (KS == 1)
+            return launch_back2_cb<2, 1>(A, rx, ww, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst, centres,
+                                         eps, L2, pm, s);
+        return launch_back2_cb<2, 2>(A, rx, ww, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst, centres, eps,
+                                     L2, pm, s);
+    }
     WinLaunch L;
     if (!conv_back_win_plan(g, ww, wa, &L)) return cudaErrorInvalidConfiguration;
     switch (ww.cb) {

@@ -75,7 +75,7 @@ struct Node {
     float* WtLo = nullptr; // dense only: W^T - WtHi (3xTF32 remainder)
     float* rowsum_abs = nullptr;  // dense only: sum_k |W[n, k]| (IBP radius of a layer fed by the input box)
     float* Wwin = nullptr;        // conv only: weights in the tap-major layout of the windowed kernel
-    WinWeights ww{nullptr, 0, 0, 4};
+    WinWeights ww{nullptr, 0, 0, 4, 0};
     int consumers = 0;
 };
 
@@ -95,6 +95,7 @@ struct vf_net {
     int tc_stall = 0;       // test hook: VF_TEST_TC_STALL=1 makes one tensor-core launch time out
     int windows = 1;        // receptive-field windows in passes that start at a convolution (VF_CONV_WINDOWS=0: off)
     int conv_whole_warp = 0;  // whole-map rows through the one-warp-per-row kernel (VF_CONV_KERNEL=warp)
+    int conv_win_per_position = 0;  // windowed rows without position blocking (VF_CONV_WIN_KERNEL=1)
     bool prof = false;
     std::vector<cudaEvent_t> ev_free;
     struct Timed {
@@ -1025,6 +1026,7 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
     if (const char* f = getenv("VF_TEST_TC_STALL")) net->tc_stall = atoi(f) != 0;
     if (const char* f = getenv("VF_CONV_WINDOWS")) net->windows = atoi(f) != 0;
     if (const char* f = getenv("VF_CONV_KERNEL")) net->conv_whole_warp = (strcmp(f, "warp") == 0) ? 1 : 0;
+    if (const char* f = getenv("VF_CONV_WIN_KERNEL")) net->conv_win_per_position = (strcmp(f, "1") == 0) ? 1 : 0;
     CU(cudaMalloc(&net->d_err, sizeof(int)));
     CU(cudaMemset(net->d_err, 0, sizeof(int)));
     net->nodes.resize(n_nodes);
@@ -1129,7 +1131,7 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
                                         w0[(((size_t)co * g.ci + ci) * g.k + p) * g.k + q];
                     CU(cudaMalloc(&nd.Wwin, sizeof(float) * wt.size()));
                     CU(cudaMemcpy(nd.Wwin, wt.data(), sizeof(float) * wt.size(), cudaMemcpyHostToDevice));
-                    nd.ww = WinWeights{nd.Wwin, ts, ci_pad, cb};
+                    nd.ww = WinWeights{nd.Wwin, ts, ci_pad, cb, net->conv_win_per_position};
                 }
                 if (!conv_back_supported(g))
                     return fail(VF_ERR_UNSUPPORTED,

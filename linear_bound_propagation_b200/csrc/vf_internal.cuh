@@ -90,6 +90,7 @@ cudaError_t launch_conv_start_rows_win(float* out, long long ld, long long M, Pa
 struct WinWeights {
     const float* Wt;
     int tap_stride, ci_pad, cb;
+    int per_position;  // 1: always the per-position kernel (no position blocking)
 };
 int win_ci_block(int ci);
 constexpr int kWinSmemLimit = 220 * 1024;

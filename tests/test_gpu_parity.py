@@ -107,7 +107,35 @@ def _conv_flops(net, centres, eps, C, both):
     return fl, {k: v.cpu().numpy() for k, v in out.items()}
 
 
-def test_receptive_field_windows_through_residual_adds(monkeypatch):
+def test_window_kernels_on_mixed_geometries(monkeypatch):
+    """Convolutions with 5x5 stride-1, 3x3 stride-2 and 4x4 stride-4 kernels: the stride/tap combinations
+    without a position-blocked instance take the per-position windowed kernel, the others the blocked
+    one; both window kernels and the whole-map path match the oracle."""
+    rng = np.random.default_rng(44)
+    net = [synth.Node(synth.INPUT, shape=(3, 16, 16))]
+    v = synth._relu(net, synth._conv(net, rng, 0, 3, 4, 5, 1, 2))
+    v = synth._relu(net, synth._conv(net, rng, v, 4, 6, 3, 2, 1))
+    v = synth._relu(net, synth._conv(net, rng, v, 6, 5, 4, 4, 0))
+    v = synth._relu(net, synth._dense(net, rng, v, 5 * 2 * 2, 9))
+    synth._dense(net, rng, v, 9, 4)
+    B = 3
+    centres = rng.random((B, 3 * 16 * 16)).astype(np.float32)
+    C = synth.margin_spec(rng.integers(0, 4, B), 4)
+    eps = 0.01
+    ora = O.verify(net, centres, eps, C, both_sides=True)
+    for windows, kernel in (("1", "2"), ("1", "1"), ("0", "2")):
+        monkeypatch.setenv("VF_CONV_WINDOWS", windows)
+        monkeypatch.setenv("VF_CONV_WIN_KERNEL", kernel)
+        g = vf.Net(net)
+        out = g.verify(_dev(centres), eps, _dev(C), both_sides=True, want_pre=True)
+        torch.cuda.synchronize()
+        g.check()
+        out = {k: v.cpu().numpy() for k, v in out.items()}
+        assert_parity(net, centres, eps, C, g, ora, out, both=True)
+
+
+@pytest.mark.parametrize("kernel", ["2", "1"])
+def test_receptive_field_windows_through_residual_adds(monkeypatch, kernel):
     """A residual net on a map large enough that windows survive the residual adds (union of the two
     branches' windows, identity shortcuts that share rows, windows that outgrow the map and return to
     whole-map rows). Windowed and whole-map passes both match the oracle, and the windowed run does
@@ -118,6 +146,7 @@ def test_receptive_field_windows_through_residual_adds(monkeypatch):
     centres = rng.random((B, 3 * 20 * 20)).astype(np.float32)
     C = synth.margin_spec(rng.integers(0, 5, B), 5)
     eps = 0.01
+    monkeypatch.setenv("VF_CONV_WIN_KERNEL", kernel)
     ora = O.verify(net, centres, eps, C, both_sides=True)
     res = {}
     for windows in ("1", "0"):
