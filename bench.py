@@ -131,8 +131,14 @@ def stop_clocks(handle):
 # Nominal dense-throughput ratios used to derive a per-dtype peak from the measured bf16 one.
 TF32_OVER_BF16 = 1.1 / 2.25
 
+# DRAM bytes per launch of the dominant kernel: dram__bytes_read.sum + dram__bytes_write.sum from one ncu
+# capture of the full-size workload, summed over the six contraction launches of one timed step and divided
+# by six. Keyed by workload name and kernel kind; reported only for that pair, and to be dropped whenever
+# the kernel changes.
+TRAFFIC_PER_LAUNCH = {("mlp_784-256x3-10_B1024", 1): 1098.6e6 / 6}
 
-def roofline(kstats, step_total_ms, n_sms):
+
+def roofline(kstats, step_total_ms, n_sms, workload=None):
     """Roofline entry for the dominant contraction kind of the step.
 
     Tensor-core dense steps (3xTF32): algorithmic flops 2*M*K*N per launch against the tf32 peak
@@ -157,7 +163,7 @@ def roofline(kstats, step_total_ms, n_sms):
         name = {2: "dense_back_ffma", 3: "conv_back_ffma", 4: "conv_back_win_k (receptive-field windows)"}[kind]
         psrc = f"fp32 FFMA: {n_sms} SMs x 128 lanes x 2 flop x {sm_mhz:.0f} MHz ({src} max clock)"
     return {"bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-            "traffic": None, "kernel": name, "launches": n_k, "avg_launch_ms": avg_ms,
+            "traffic": TRAFFIC_PER_LAUNCH.get((workload, kind)), "kernel": name, "launches": n_k, "avg_launch_ms": avg_ms,
             "share_of_step": k_ms / step_total_ms if step_total_ms else None, "peak_source": psrc}
 
 
@@ -298,7 +304,8 @@ def run_ours(args):
     h2d = h_centres.numel() * 4 + h_C.numel() * 4
     d2h = h_lb.numel() * 4 + h_ver.numel()
 
-    roof = roofline(kstats, total_ms, torch.cuda.get_device_properties(dev).multi_processor_count)
+    roof = roofline(kstats, total_ms, torch.cuda.get_device_properties(dev).multi_processor_count,
+                    w.name if args.centres is None else None)
     alpha = None
     if args.alpha_iters > 0 and all(nd.op in ("input", "dense", "relu") for nd in w.net) and not w.both_sides:
         # alpha-CROWN leg: the same workload, intermediate bounds as above, then per-row slope optimisation
