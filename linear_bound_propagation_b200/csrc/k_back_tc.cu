@@ -121,6 +121,35 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[3
         : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// 16 consecutive columns (the tail of a tile whose width is 16 mod 32).
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// s1 += sum_j v_j * c_j and s2 += sum_j |v_j| over the first CNT values of a TMEM chunk, four independent
+// partial sums each (columns at or beyond N hold exact zeros in both the accumulator and the staged centres).
+template <int CNT>
+__device__ __forceinline__ void conc_chunk(const uint32_t (&v)[32], const float* c, float (&s1)[4], float (&s2)[4]) {
+#pragma unroll
+    for (int j = 0; j < CNT; j += 4) {
+        const float4 cc = *reinterpret_cast<const float4*>(c + j);
+        const float x0 = __uint_as_float(v[j]), x1 = __uint_as_float(v[j + 1]);
+        const float x2 = __uint_as_float(v[j + 2]), x3 = __uint_as_float(v[j + 3]);
+        s1[0] = fmaf(x0, cc.x, s1[0]);
+        s1[1] = fmaf(x1, cc.y, s1[1]);
+        s1[2] = fmaf(x2, cc.z, s1[2]);
+        s1[3] = fmaf(x3, cc.w, s1[3]);
+        s2[0] += fabsf(x0);
+        s2[1] += fabsf(x1);
+        s2[2] += fabsf(x2);
+        s2[3] += fabsf(x3);
+    }
+}
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
     asm volatile(
@@ -402,31 +431,34 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 const long long b = (p.pg.pass_m0 + m) / p.pg.R_pass;
                 const long long bw = (p.pg.pass_m0 + row0) / p.pg.R_pass;
                 const float* crow = stg + (valid ? (int)(b - bw) : 0) * p.BN;
-                float conc = 0.f;
-                // 64 columns in flight per wait (2 loads of 32), then the arithmetic
-                for (int c0 = 0; c0 < p.BN; c0 += 64) {
+                // sum_n v c_n and sum_n |v| over the tile's BN columns (BN is a multiple of 16): 64
+                // columns in flight per wait, then a 32- and a 16-column tail
+                float s1[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+                int c0 = 0;
+                for (; c0 + 64 <= p.BN; c0 += 64) {
                     uint32_t v[2][32];
                     tmem_ld32_nowait(tmem + lane_base + c0, v[0]);
-                    if (c0 + 32 < p.BN) tmem_ld32_nowait(tmem + lane_base + c0 + 32, v[1]);
+                    tmem_ld32_nowait(tmem + lane_base + c0 + 32, v[1]);
                     tmem_wait_ld();
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int cu = c0 + 32 * u;
-                        if (cu >= p.BN) break;
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const float4 cc = *reinterpret_cast<const float4*>(crow + cu + j);
-                            const float cv[4] = {cc.x, cc.y, cc.z, cc.w};
-#pragma unroll
-                            for (int jj = 0; jj < 4; ++jj) {
-                                const float x = __uint_as_float(v[u][j + jj]);
-                                if (cu + j + jj < p.BN && n0 + cu + j + jj < p.N) conc += fmaf(x, cv[jj], -p.eps * fabsf(x));
-                            }
-                        }
-                    }
+                    conc_chunk<32>(v[0], crow + c0, s1, s2);
+                    conc_chunk<32>(v[1], crow + c0 + 32, s1, s2);
+                }
+                if (c0 + 32 <= p.BN) {
+                    uint32_t v[32];
+                    tmem_ld32_nowait(tmem + lane_base + c0, v);
+                    tmem_wait_ld();
+                    conc_chunk<32>(v, crow + c0, s1, s2);
+                    c0 += 32;
+                }
+                if (c0 < p.BN) {
+                    uint32_t v[32];
+                    tmem_ld16_nowait(tmem + lane_base + c0, v);
+                    tmem_wait_ld();
+                    conc_chunk<16>(v, crow + c0, s1, s2);
                 }
                 tc_fence_before();
                 mbar_arrive(&acc_empty);
+                const float conc = ((s1[0] + s1[1]) + (s1[2] + s1[3])) - p.eps * ((s2[0] + s2[1]) + (s2[2] + s2[3]));
                 if (valid) p.part[(long long)n_tile * p.M + m] = conc;
                 __syncwarp();  // the staged centres are reused by the next tile
             } else {
