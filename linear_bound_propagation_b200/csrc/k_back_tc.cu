@@ -69,10 +69,24 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait that may suspend the thread in hardware for up to ~20 us while the phase is pending, so a
+// waiting warp takes no issue slots from the warps sharing its scheduler.
+__device__ __forceinline__ bool mbar_test_suspend(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait; returns false (and raises the CTA abort flag) when it gives up or sees abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_test(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_test(bar, parity)) {
+    while (!mbar_test_suspend(bar, parity)) {
         if (*abort_flag) return false;
         if (clock64() - t0 > WAIT_CYCLES) {
             *abort_flag = 1;
