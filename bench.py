@@ -135,7 +135,7 @@ TF32_OVER_BF16 = 1.1 / 2.25
 # capture of the full-size workload, summed over the six contraction launches of one timed step and divided
 # by six. Keyed by workload name and kernel kind; reported only for that pair, and to be dropped whenever
 # the kernel changes.
-TRAFFIC_PER_LAUNCH = {}  # re-captured after each change of the kernel
+TRAFFIC_PER_LAUNCH = {("mlp_784-256x3-10_B1024", 1): 1099.0e6 / 6}
 
 
 def roofline(kstats, step_total_ms, n_sms, workload=None):
