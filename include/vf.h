@@ -131,7 +131,12 @@ typedef struct {
  * C_bstride elements; 0 = shared). Outputs [device], [B, R] each:
  *   lb = max(IBP lower, CROWN lower); ub (both_sides only, else may be NULL) =
  *   min(IBP upper, CROWN upper); lb_ibp (or NULL) the IBP lower bound; verified (or NULL)
- *   1 iff lb > 0. opts [host] may be NULL (all defaults). */
+ *   1 iff lb > 0. opts [host] may be NULL (all defaults).
+ * An intermediate pass only needs rows for the neurons whose IBP interval contains 0 (the
+ * others keep their IBP bounds), so passes run over those neurons alone; sizing them reads
+ * the per-centre counts back once per call, which synchronises `stream` (as does the finite
+ * check unless skipped). VF_COMPACT=0 in the environment at vf_net_create keeps every pass
+ * at rows [I; -I]. */
 int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
                     const vf_opts* opts, float* lb, float* ub, float* lb_ibp, uint8_t* verified, void* stream);
 

@@ -55,9 +55,8 @@ __global__ void relax_params_k(const float* __restrict__ l, const float* __restr
 __global__ void cst_identity_bias_k(float* __restrict__ cst, long long M, PassGeom pg, const float* __restrict__ bias,
                                     long long n_p, long long per_channel) {
     GRID_STRIDE(m, M) {
-        const long long r = (pg.pass_m0 + m) % pg.R_pass;
-        const long long j = r % n_p;
-        const float sg = (r < n_p) ? 1.f : -1.f;
+        float sg;
+        const long long j = start_neuron(pg, n_p, m, &sg);
         cst[m] += sg * bias[j / per_channel];
     }
 }
@@ -66,8 +65,9 @@ __global__ void ident_rows_k(float* __restrict__ out, long long ld, long long M,
                              int accumulate) {
     GRID_STRIDE(e, M * n_p) {
         const long long m = e / n_p, c = e % n_p;
-        const long long r = (pg.pass_m0 + m) % pg.R_pass;
-        const float v = (c == r % n_p) ? ((r < n_p) ? 1.f : -1.f) : 0.f;
+        float sg;
+        const long long j = start_neuron(pg, n_p, m, &sg);
+        const float v = (c == j) ? sg : 0.f;
         float* o = out + m * ld + c;
         *o = accumulate ? (*o + v) : v;
     }
@@ -85,9 +85,8 @@ __global__ void conv_start_rows_k(float* __restrict__ out, long long ld, long lo
             for (long long c = threadIdx.x; c < nin; c += blockDim.x) o[c] = 0.f;
             __syncthreads();
         }
-        const long long r = (pg.pass_m0 + m) % pg.R_pass;
-        const long long j = r % n_p;
-        const float sg = (r < n_p) ? 1.f : -1.f;
+        float sg;
+        const long long j = start_neuron(pg, n_p, m, &sg);
         const int co = (int)(j / (g.ho * g.wo));
         const int oi = (int)((j / g.wo) % g.ho);
         const int oj = (int)(j % g.wo);
@@ -187,6 +186,81 @@ __global__ void intersect_k(float* __restrict__ l, float* __restrict__ u, const 
             l[i] = fmaxf(l0, pass_out[b * 2 * n + j]);
             u[i] = fminf(u0, -pass_out[b * 2 * n + n + j]);
         }
+    }
+}
+
+// Unstable-neuron compaction (rows of an intermediate pass only for IBP-unstable neurons: the others keep
+// their IBP bounds, so their rows are never used). One CTA of 256 threads per centre.
+__global__ void __launch_bounds__(256) unstable_count_k(const float* __restrict__ l, const float* __restrict__ u,
+                                                        long long n, int* __restrict__ counts) {
+    __shared__ int red[8];
+    const long long b = blockIdx.x;
+    int c = 0;
+    for (long long j = threadIdx.x; j < n; j += 256) c += (l[b * n + j] < 0.f && u[b * n + j] > 0.f) ? 1 : 0;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int t = 0;
+        for (int i = 0; i < 8; ++i) t += red[i];
+        counts[b] = t;
+    }
+}
+
+// idx[b * half + i] = the i-th unstable neuron of centre b (increasing order), -1 for i >= its count.
+// Each 256-neuron chunk is ranked with warp ballots and a prefix over the 8 warps.
+__global__ void __launch_bounds__(256) unstable_list_k(const float* __restrict__ l, const float* __restrict__ u,
+                                                       long long n, int half, int* __restrict__ idx) {
+    __shared__ int wcount[8];
+    __shared__ int base_sh;
+    const long long b = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) base_sh = 0;
+    __syncthreads();
+    for (long long j0 = 0; j0 < n; j0 += 256) {
+        const long long j = j0 + threadIdx.x;
+        const bool un = j < n && l[b * n + j] < 0.f && u[b * n + j] > 0.f;
+        const unsigned bal = __ballot_sync(0xffffffffu, un);
+        if (lane == 0) wcount[warp] = __popc(bal);
+        __syncthreads();
+        int before = base_sh;
+        for (int w = 0; w < warp; ++w) before += wcount[w];
+        const int pos = before + __popc(bal & ((1u << lane) - 1u));
+        if (un && pos < half) idx[b * half + pos] = (int)j;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int t = 0;
+            for (int w = 0; w < 8; ++w) t += wcount[w];
+            base_sh += t;
+        }
+        __syncthreads();
+    }
+    for (int i = base_sh + threadIdx.x; i < half; i += 256) idx[b * half + i] = -1;
+}
+
+// Intersection after a compacted pass (2 * half rows per centre: +e_j for the listed j, then -e_j).
+__global__ void intersect_compact_k(float* __restrict__ l, float* __restrict__ u, const float* __restrict__ pass_out,
+                                    const int* __restrict__ idx, int B, long long n, int half) {
+    GRID_STRIDE(e, (long long)B * half) {
+        const long long b = e / half, i = e % half;
+        const int j = idx[e];
+        if (j < 0) continue;
+        const long long k = b * n + j;
+        l[k] = fmaxf(l[k], pass_out[b * 2 * half + i]);
+        u[k] = fminf(u[k], -pass_out[b * 2 * half + half + i]);
+    }
+}
+
+// out[m, :] = sg * W[j, :] for the start neuron j of row m (compacted pass over a dense node).
+__global__ void gather_start_rows_k(float* __restrict__ out, long long ld, long long M, PassGeom pg,
+                                    const float* __restrict__ W, long long n_p, long long n_src) {
+    for (long long m = blockIdx.x; m < M; m += gridDim.x) {
+        float sg;
+        const long long j = start_neuron(pg, n_p, m, &sg);
+        const float* w = W + j * n_src;
+        float* o = out + m * ld;
+        for (long long c = threadIdx.x; c < n_src; c += blockDim.x) o[c] = sg * w[c];
     }
 }
 
@@ -323,6 +397,32 @@ cudaError_t launch_intersect(float* l, float* u, const float* l_ibp, const float
     (void)l_ibp;
     (void)u_ibp;
     intersect_k<<<grid_for((long long)B * n, 256), 256, 0, s>>>(l, u, pass_out, B, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_unstable_count(const float* l, const float* u, int B, long long n, int* counts, cudaStream_t s) {
+    if (B <= 0) return cudaSuccess;
+    unstable_count_k<<<B, 256, 0, s>>>(l, u, n, counts);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_unstable_list(const float* l, const float* u, int B, long long n, int half, int* idx, cudaStream_t s) {
+    if (B <= 0 || half <= 0) return cudaSuccess;
+    unstable_list_k<<<B, 256, 0, s>>>(l, u, n, half, idx);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_intersect_compact(float* l, float* u, const float* pass_out, const int* idx, int B, long long n,
+                                     int half, cudaStream_t s) {
+    if (B <= 0 || half <= 0) return cudaSuccess;
+    intersect_compact_k<<<grid_for((long long)B * half, 256), 256, 0, s>>>(l, u, pass_out, idx, B, n, half);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_start_rows(float* out, long long ld, long long M, PassGeom pg, const float* W, long long n_p,
+                                     long long n_src, cudaStream_t s) {
+    if (M <= 0) return cudaSuccess;
+    gather_start_rows_k<<<rows_grid(M), 256, 0, s>>>(out, ld, M, pg, W, n_p, n_src);
     return cudaGetLastError();
 }
 

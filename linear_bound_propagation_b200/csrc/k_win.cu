@@ -25,10 +25,8 @@ struct StartPos {
 
 __device__ __forceinline__ StartPos start_pos(const PassStart& ps, const PassGeom& pg, long long m) {
     const long long g = pg.pass_m0 + m;
-    const long long r = g % pg.R_pass;
-    const long long j = r % ps.n;
     StartPos s;
-    s.sg = (r < ps.n) ? 1.f : -1.f;
+    const long long j = start_neuron(pg, ps.n, m, &s.sg);
     s.xj = (int)(j % ps.w);
     s.yj = (int)((j / ps.w) % ps.h);
     s.cj = (int)(j / ((long long)ps.h * ps.w));

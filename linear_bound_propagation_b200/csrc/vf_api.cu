@@ -96,6 +96,7 @@ struct vf_net {
     int windows = 1;        // receptive-field windows in passes that start at a convolution (VF_CONV_WINDOWS=0: off)
     int conv_whole_warp = 0;  // whole-map rows through the one-warp-per-row kernel (VF_CONV_KERNEL=warp)
     int conv_win_per_position = 0;  // windowed rows without position blocking (VF_CONV_WIN_KERNEL=1)
+    int compact = 1;        // intermediate passes over IBP-unstable neurons only (VF_COMPACT=0: off)
     bool prof = false;
     std::vector<cudaEvent_t> ev_free;
     struct Timed {
@@ -235,6 +236,7 @@ struct Walker {
     const std::vector<const float4*>* relax;  // per node: relaxation params of ReLU nodes
     std::vector<Entry> pend;
     bool win_on = false;      // rows may be held as receptive-field windows (pass starts at a convolution)
+    bool compact = false;     // identity-trick pass over the listed unstable neurons only (pg.idx)
     PassStart ps{1, 1, 1};    // the pass's start node
     long long max_len = 0;    // longest row a pool buffer has held
 
@@ -472,6 +474,12 @@ struct Walker {
                 }
                 if (e.kind == E_IDENT) {
                     if (!dry) LAUNCH(net, launch_cst_identity_bias(cst, M, pg, nd.b, nd.n, 1, s));
+                    if (compact) {  // the listed neurons' rows +-W[j] are gathered into a buffer
+                        int nb;
+                        TRY(alloc_buf(&nb, sn.n));
+                        if (!dry) LAUNCH(net, launch_gather_start_rows(bufs[nb], ld_buf, M, pg, nd.W, nd.n, sn.n, s));
+                        return add_into(nd.src, buf_entry(nb));
+                    }
                     Entry x;
                     x.kind = E_VIRT;
                     x.ref = RowRef{nd.pmW, 0, sn.n, 2 * nd.n, pg.pass_m0};
@@ -616,7 +624,7 @@ bool input_buffered(const vf_net* net) {
 
 // Buffers a pass needs at once and the longest row they hold, by a dry run of the walker.
 int pool_size(vf_net* net, int start, Entry init, const std::vector<const float4*>* relax, bool ext, bool win_on,
-              int* nb, long long* max_len) {
+              bool compact, int* nb, long long* max_len) {
     Walker w;
     w.net = net;
     w.s = nullptr;
@@ -628,6 +636,7 @@ int pool_size(vf_net* net, int start, Entry init, const std::vector<const float4
     w.ld_buf = 1;
     w.relax = relax;
     w.win_on = win_on;
+    w.compact = compact;
     float dummy = 0.f;
     w.ext_in = ext ? &dummy : nullptr;
     TRY(w.run(start, init));
@@ -684,24 +693,23 @@ long long offset_of(const vf_net* net, int v, int B) {
     return o * B;
 }
 
-int check_finite_dev(vf_net* net, const std::vector<std::pair<const float*, long long>>& arrays, Arena& ar,
-                     cudaStream_t s) {
+// Enqueues the NaN/Inf scan of the arrays into a device flag; the flag is read back (with the
+// compaction counts) by prepare_bounds, so a call synchronises its stream once.
+int scan_finite_dev(vf_net* net, const std::vector<std::pair<const float*, long long>>& arrays, Arena& ar,
+                    cudaStream_t s, int** flag_out) {
     int* flag = ar.take<int>(1);
     if (!flag) return fail(VF_ERR_WORKSPACE, "workspace too small");
     CU(cudaMemsetAsync(flag, 0, sizeof(int), s));
     for (auto& a : arrays)
         if (a.first != nullptr) LAUNCH(net, launch_finite_scan(a.first, a.second, flag, s));
-    int h = 0;
-    CU(cudaMemcpyAsync(&h, flag, sizeof(int), cudaMemcpyDeviceToHost, s));
-    CU(cudaStreamSynchronize(s));
-    if (h) return fail(VF_ERR_NONFINITE, "NaN or Inf in centres, C or alpha");
+    *flag_out = flag;
     return VF_OK;
 }
 
 // Runs every row block of one pass. `init` describes the start rows (global addressing).
 int run_pass(vf_net* net, int start, Entry init, long long rows, long long R_pass, Arena& ar,
              const std::vector<const float4*>& relax, const float* centres, float eps, float* pass_out, float* ext_in,
-             float* const_out, cudaStream_t s) {
+             float* const_out, cudaStream_t s, const int* idx = nullptr) {
     const bool ext = ext_in != nullptr;
     const Node& sn = net->nodes[start];
     // rows held as receptive-field windows: identity-trick passes that start at a convolution or a residual add
@@ -709,7 +717,7 @@ int run_pass(vf_net* net, int start, Entry init, long long rows, long long R_pas
         net->windows && !ext && init.kind == E_IDENT && (sn.op == VF_CONV2D || sn.op == VF_ADD) && sn.h > 1;
     int nb = 0;
     long long max_len = 0;
-    TRY(pool_size(net, start, init, &relax, ext, win_on, &nb, &max_len));
+    TRY(pool_size(net, start, init, &relax, ext, win_on, idx != nullptr, &nb, &max_len));
     long long nmax = (max_node_size(net, input_buffered(net)) + 31) / 32 * 32;  // 128-byte rows
     if (win_on) nmax = std::max<long long>(32, (max_len + 31) / 32 * 32);
     int tiles = std::max(dense_back_tiles_n((int)net->nodes[0].n), dense_back_tc_tiles_n((int)net->nodes[0].n));
@@ -739,10 +747,11 @@ int run_pass(vf_net* net, int start, Entry init, long long rows, long long R_pas
     w.eps = eps;
     w.n_centres = rows / R_pass;
     w.win_on = win_on;
+    w.compact = idx != nullptr;
     w.ps = PassStart{sn.n, sn.h, sn.w};
     for (long long m0 = 0; m0 < rows; m0 += chunk) {
         w.M = std::min(chunk, rows - m0);
-        w.pg = PassGeom{m0, R_pass};
+        w.pg = PassGeom{m0, R_pass, idx};
         Entry e = init;
         if (e.kind == E_VIRT) e.ref.m0 = m0;
         w.ext_in = ext ? ext_in + m0 * net->nodes[0].n : nullptr;
@@ -784,7 +793,7 @@ struct Bounds {
 };
 
 int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf_opts& o, Arena& ar, IbpState& st,
-                   Bounds& bd, cudaStream_t s) {
+                   Bounds& bd, cudaStream_t s, const int* finite_flag = nullptr) {
     const int nn = (int)net->nodes.size();
     TRY(run_ibp(net, centres, B, eps, ar, st, s));
     bd.Lw.assign(nn, nullptr);
@@ -808,6 +817,37 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
             bd.relax[v] = P[v];
             max_pass_rows = std::max(max_pass_rows, 2 * net->nodes[v].n);
         }
+    // Unstable-neuron compaction: only IBP-unstable neurons change at the intersection, so a pass needs
+    // rows for those alone. The number per centre is read back once (one host synchronisation) and each
+    // pass is sized for the largest count; a pass whose largest count is above 7/8 of the node stays plain.
+    // The finite-check flag (if any) is read back in the same copy, before any pass runs.
+    std::vector<int> half(nn, -1);  // -1: plain pass, 0: nothing to refine, > 0: compacted rows per sign
+    std::vector<int> ps;
+    if (net->compact)
+        for (int k = 0; k < nn; ++k) {
+            const int p = net->nodes[k].src;
+            if (net->nodes[k].op == VF_RELU && ((o.relu_crown == nullptr) || (o.relu_crown[k] != 0)) &&
+                !exact_source(net, p))
+                ps.push_back(p);
+        }
+    if (!ps.empty() || finite_flag != nullptr) {
+        int* counts = ar.take<int>(1 + (size_t)B * ps.size());  // [0]: finite flag, then [pass][centre]
+        if (!counts) return fail(VF_ERR_WORKSPACE, "workspace too small");
+        if (finite_flag != nullptr)
+            CU(cudaMemcpyAsync(counts, finite_flag, sizeof(int), cudaMemcpyDeviceToDevice, s));
+        else
+            CU(cudaMemsetAsync(counts, 0, sizeof(int), s));
+        for (size_t i = 0; i < ps.size(); ++i)
+            LAUNCH(net, launch_unstable_count(bd.Lw[ps[i]], bd.Uw[ps[i]], B, net->nodes[ps[i]].n, counts + 1 + i * B, s));
+        std::vector<int> h(1 + (size_t)B * ps.size());
+        CU(cudaMemcpyAsync(h.data(), counts, sizeof(int) * h.size(), cudaMemcpyDeviceToHost, s));
+        CU(cudaStreamSynchronize(s));
+        if (h[0]) return fail(VF_ERR_NONFINITE, "NaN or Inf in centres, C or alpha");
+        for (size_t i = 0; i < ps.size(); ++i) {
+            const int u_max = *std::max_element(h.begin() + 1 + i * B, h.begin() + 1 + (i + 1) * B);
+            half[ps[i]] = (8LL * u_max <= 7LL * net->nodes[ps[i]].n) ? u_max : -1;
+        }
+    }
     Arena tmp = ar;  // pass outputs are transient
     float* pass_out = tmp.take<float>((size_t)B * max_pass_rows);
     if (!pass_out) return fail(VF_ERR_WORKSPACE, "workspace too small");
@@ -816,7 +856,18 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
         if (nd.op != VF_RELU) continue;
         const int p = nd.src;
         const bool crown = (o.relu_crown == nullptr) || (o.relu_crown[k] != 0);
-        if (crown && !exact_source(net, p)) {
+        if (crown && !exact_source(net, p) && half[p] > 0) {
+            const long long np = net->nodes[p].n;
+            const int hp = half[p];
+            int* idx = tmp.take<int>((size_t)B * hp);
+            if (!idx) return fail(VF_ERR_WORKSPACE, "workspace too small");
+            LAUNCH(net, launch_unstable_list(bd.Lw[p], bd.Uw[p], B, np, hp, idx, s));
+            Entry init;
+            init.kind = E_IDENT;
+            TRY(run_pass(net, p, init, (long long)B * 2 * hp, 2 * hp, tmp, bd.relax, centres, eps, pass_out, nullptr,
+                         nullptr, s, idx));
+            LAUNCH(net, launch_intersect_compact(bd.Lw[p], bd.Uw[p], pass_out, idx, B, np, hp, s));
+        } else if (crown && !exact_source(net, p) && half[p] < 0) {
             Entry init;
             init.kind = E_IDENT;
             const long long np = net->nodes[p].n;
@@ -1027,6 +1078,7 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
     if (const char* f = getenv("VF_CONV_WINDOWS")) net->windows = atoi(f) != 0;
     if (const char* f = getenv("VF_CONV_KERNEL")) net->conv_whole_warp = (strcmp(f, "warp") == 0) ? 1 : 0;
     if (const char* f = getenv("VF_CONV_WIN_KERNEL")) net->conv_win_per_position = (strcmp(f, "1") == 0) ? 1 : 0;
+    if (const char* f = getenv("VF_COMPACT")) net->compact = atoi(f) != 0;
     CU(cudaMalloc(&net->d_err, sizeof(int)));
     CU(cudaMemset(net->d_err, 0, sizeof(int)));
     net->nodes.resize(n_nodes);
@@ -1272,19 +1324,19 @@ int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const f
     const int BC = C_bstride > 0 ? B : 1;
     Arena ar{net->ws, net->ws_bytes};
 
+    int* finite_flag = nullptr;
     if (!o.skip_finite_check) {
         std::vector<std::pair<const float*, long long>> arrs = {{centres, (long long)B * n0},
                                                                 {C, (long long)(BC - 1) * C_bstride + (long long)R * nL}};
         if (o.alpha)
             for (int v = 0; v < nn; ++v)
                 if (net->nodes[v].op == VF_RELU && o.alpha[v]) arrs.push_back({o.alpha[v], (long long)B * net->nodes[v].n});
-        Arena tmp = ar;
-        TRY(check_finite_dev(net, arrs, tmp, s));
+        TRY(scan_finite_dev(net, arrs, ar, s, &finite_flag));
     }
 
     IbpState st;
     Bounds bd;
-    TRY(prepare_bounds(net, centres, B, eps, o, ar, st, bd, s));
+    TRY(prepare_bounds(net, centres, B, eps, o, ar, st, bd, s, finite_flag));
     std::vector<float*>& Lw = bd.Lw;
     std::vector<float*>& Uw = bd.Uw;
     std::vector<const float4*>& relax = bd.relax;

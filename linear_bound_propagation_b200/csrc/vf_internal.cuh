@@ -35,7 +35,24 @@ struct Relax {
 struct PassGeom {
     long long pass_m0;
     long long R_pass;
+    const int* idx = nullptr;  // compacted identity-trick pass: start neurons, see start_neuron
 };
+
+// Start neuron of local row m of an identity-trick pass over a node with n_start neurons. Plain pass:
+// rows [I; -I] per centre. Compacted pass (pg.idx set): rows [e_j; -e_j] for the neurons listed in
+// idx[b * (R_pass / 2) + i]; a padding slot holds -1 and stands for neuron 0 (its result is unused).
+__device__ __forceinline__ long long start_neuron(const PassGeom& pg, long long n_start, long long m, float* sg) {
+    const long long g = pg.pass_m0 + m;
+    const long long r = g % pg.R_pass;
+    if (pg.idx == nullptr) {
+        *sg = (r < n_start) ? 1.f : -1.f;
+        return r % n_start;
+    }
+    const long long half = pg.R_pass >> 1;
+    *sg = (r < half) ? 1.f : -1.f;
+    const int j = pg.idx[(g / pg.R_pass) * half + (r % half)];
+    return j < 0 ? 0 : j;
+}
 
 enum OutMode { OUT_STORE = 0, OUT_ACCUM = 1, OUT_CONCRETIZE = 2 };
 
@@ -153,6 +170,16 @@ cudaError_t launch_finish_rows(const float* cst, const float* part, int ntiles, 
 cudaError_t launch_add_partials(float* cst, const float* part, int ntiles, long long M, cudaStream_t s);
 cudaError_t launch_intersect(float* l, float* u, const float* l_ibp, const float* u_ibp, const float* pass_out,
                              int B, long long n, cudaStream_t s);
+// Unstable-neuron compaction of an intermediate pass (IBP bounds l < 0 < u): counts[b] = number of such
+// neurons of centre b; idx[b * half + i] = the i-th of them in increasing order, -1 past the count.
+cudaError_t launch_unstable_count(const float* l, const float* u, int B, long long n, int* counts, cudaStream_t s);
+cudaError_t launch_unstable_list(const float* l, const float* u, int B, long long n, int half, int* idx, cudaStream_t s);
+// Intersection for a compacted pass: rows [e_j; -e_j] of the listed neurons, R = 2 * half rows per centre.
+cudaError_t launch_intersect_compact(float* l, float* u, const float* pass_out, const int* idx, int B, long long n,
+                                     int half, cudaStream_t s);
+// Rows +-W[j, :] (W is [n_p, n_src], row-major) for the start neurons of a compacted pass over a dense node.
+cudaError_t launch_gather_start_rows(float* out, long long ld, long long M, PassGeom pg, const float* W, long long n_p,
+                                     long long n_src, cudaStream_t s);
 cudaError_t launch_spec_rows(const float* C, long long C_bstride, int BC, int R, int nL, float* S, cudaStream_t s);
 cudaError_t launch_spec_ibp(const float* C, long long C_bstride, int B, int R, int nL, const float* zc, const float* zr,
                             float* lb, float* ub, cudaStream_t s);

@@ -158,6 +158,26 @@ def test_receptive_field_windows_through_residual_adds(monkeypatch, kernel):
     assert res["1"] < 0.7 * res["0"], res
 
 
+@pytest.mark.parametrize("compact", ["1", "0"])
+@pytest.mark.parametrize("eps", [0.3 / 255, 1e-6])
+def test_unstable_compaction_dense(monkeypatch, compact, eps):
+    """Intermediate passes over the IBP-unstable neurons only (gathered +-W rows for a dense start): at
+    eps 0.3/255 the first refined layer is ~37% unstable and compacted, the second stays plain; at 1e-6
+    almost no neuron is unstable and the compacted passes are a few rows per centre."""
+    monkeypatch.setenv("VF_COMPACT", compact)
+    w = synth.workload(2, B=7, eps=eps)
+    g, ora, out = run_both(w.net, w.centres, w.eps, w.C)
+    assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out)
+
+
+@pytest.mark.parametrize("compact", ["1", "0"])
+def test_unstable_compaction_conv(monkeypatch, compact):
+    monkeypatch.setenv("VF_COMPACT", compact)
+    w = synth.workload(3, B=2)
+    g, ora, out = run_both(w.net, w.centres, w.eps, w.C)
+    assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out)
+
+
 @pytest.mark.parametrize("eps", [0.5 / 255, 1.0 / 255, 2.0 / 255])
 def test_cfg5_subset_each_eps(eps):
     w = synth.workload(5, B=2, eps=eps)
