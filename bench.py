@@ -304,6 +304,28 @@ def run_ours(args):
     h2d = h_centres.numel() * 4 + h_C.numel() * 4
     d2h = h_lb.numel() * 4 + h_ver.numel()
 
+    graph = None
+    if args.graph:
+        # the same verify call captured once in a CUDA graph (no host synchronisation inside) and replayed
+        vg = vf.VerifyGraph(net, centres, w.eps, C, crown_relus=w.crown_relus, both_sides=w.both_sides)
+        for _ in range(args.warmup):
+            vg.replay()
+        torch.cuda.synchronize()
+        g_ms = 0.0
+        for i in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            vg.replay()
+            e1.record(stream)
+            e1.synchronize()
+            g_ms += e0.elapsed_time(e1)
+        g_ms = max_over_ranks(g_ms, dev)
+        graph = {"value": weak_throughput(world, B * Rs, args.steps, g_ms), "unit": UNIT,
+                 "ms_per_step": g_ms / args.steps,
+                 "note": "vf.VerifyGraph: the verify call captured in a CUDA graph and replayed (no NaN/Inf scan, "
+                         "no unstable-neuron compaction)"}
+        del vg
     roof = roofline(kstats, total_ms, torch.cuda.get_device_properties(dev).multi_processor_count,
                     w.name if args.centres is None else None)
     alpha = None
@@ -334,7 +356,7 @@ def run_ours(args):
                 "e2e": None if args.no_e2e else {"value": weak_throughput(world, B * Rs, args.steps, e2e_ms), "unit": UNIT,
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches, "clocks": clocks, "verified_specs": verified, "total_specs": B * Rs,
-                "alpha_crown": alpha}
+                "alpha_crown": alpha, "graph": graph}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = oracle_sample(w, args.cpu_sample_s)[0]
         print(json.dumps(line), flush=True)
@@ -356,6 +378,7 @@ def main():
     ap.add_argument("--centres", type=int, default=None,
                     help="use only the first N centres of the workload (profiling captures of a small case)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-staged end-to-end leg")
+    ap.add_argument("--graph", action="store_true", help="also time the verify call replayed from a CUDA graph")
     ap.add_argument("--alpha-iters", type=int, default=10,
                     help="also time vf_alpha_crown with this many Adam steps (dense chains; 0 = skip)")
     args = ap.parse_args()

@@ -124,6 +124,9 @@ typedef struct {
      * bounds used for each ReLU source after refinement (other nodes: IBP bounds). */
     float* pre_lb;
     float* pre_ub;
+    /* 1: the call never synchronises `stream` (no NaN/Inf scan, no unstable-neuron compaction;
+     * the bounds are the same numbers), so it can be captured in a CUDA graph. */
+    int no_host_sync;
 } vf_opts;
 
 /* Whole verification step (section 1): IBP, CROWN intermediate bounds, specification

@@ -823,7 +823,7 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
     // The finite-check flag (if any) is read back in the same copy, before any pass runs.
     std::vector<int> half(nn, -1);  // -1: plain pass, 0: nothing to refine, > 0: compacted rows per sign
     std::vector<int> ps;
-    if (net->compact)
+    if (net->compact && !o.no_host_sync)
         for (int k = 0; k < nn; ++k) {
             const int p = net->nodes[k].src;
             if (net->nodes[k].op == VF_RELU && ((o.relu_crown == nullptr) || (o.relu_crown[k] != 0)) &&
@@ -1325,7 +1325,7 @@ int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const f
     Arena ar{net->ws, net->ws_bytes};
 
     int* finite_flag = nullptr;
-    if (!o.skip_finite_check) {
+    if (!o.skip_finite_check && !o.no_host_sync) {
         std::vector<std::pair<const float*, long long>> arrs = {{centres, (long long)B * n0},
                                                                 {C, (long long)(BC - 1) * C_bstride + (long long)R * nL}};
         if (o.alpha)

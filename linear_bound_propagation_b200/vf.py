@@ -45,7 +45,7 @@ class NodeDesc(ctypes.Structure):
 class Opts(ctypes.Structure):
     _fields_ = [("relu_crown", ctypes.POINTER(ctypes.c_int)), ("alpha", ctypes.POINTER(ctypes.c_void_p)),
                 ("both_sides", ctypes.c_int), ("skip_finite_check", ctypes.c_int),
-                ("pre_lb", ctypes.c_void_p), ("pre_ub", ctypes.c_void_p)]
+                ("pre_lb", ctypes.c_void_p), ("pre_ub", ctypes.c_void_p), ("no_host_sync", ctypes.c_int)]
 
 
 _lib = None
@@ -188,7 +188,7 @@ class Net:
 
     def verify(self, centres: torch.Tensor, eps: float, C: torch.Tensor, crown_relus: Optional[Sequence[int]] = None,
                alpha: Optional[Dict[int, torch.Tensor]] = None, both_sides: bool = False, want_pre: bool = False,
-               skip_finite_check: bool = False, stream=None, out=None):
+               skip_finite_check: bool = False, no_host_sync: bool = False, stream=None, out=None):
         """vf_verify_batch. C: [B or 1, R, n_L]. Returns dict of device tensors."""
         B = centres.shape[0]
         R = C.shape[1]
@@ -216,6 +216,7 @@ class Net:
             keep.append(arr)
         o.both_sides = 1 if both_sides else 0
         o.skip_finite_check = 1 if skip_finite_check else 0
+        o.no_host_sync = 1 if no_host_sync else 0
         o.pre_lb = out["pre_lb"].data_ptr() if "pre_lb" in out else None
         o.pre_ub = out["pre_ub"].data_ptr() if "pre_ub" in out else None
         _check(lib().vf_verify_batch(self.h, _ptr(centres), B, float(eps), _ptr(C), R, bstride, ctypes.byref(o),
@@ -281,6 +282,37 @@ class Net:
 
     def launch_count(self) -> int:
         return lib().vf_launch_count(self.h)
+
+
+class VerifyGraph:
+    """One vf_verify_batch call captured in a CUDA graph and replayed.
+
+    Shapes, eps, options and the device buffers are fixed at capture: write the next batch into
+    ``self.centres`` / ``self.C`` in place, call ``replay()`` and read ``self.out``. The captured call
+    never synchronises its stream (``no_host_sync``: no NaN/Inf scan, no unstable-neuron compaction),
+    which leaves the bounds unchanged. It uses the handle's workspace, so no other call on the same
+    handle may run while a replay is in flight.
+    """
+
+    def __init__(self, net: Net, centres: torch.Tensor, eps: float, C: torch.Tensor,
+                 crown_relus: Optional[Sequence[int]] = None, both_sides: bool = False):
+        self.net = net
+        self.centres = centres.clone()
+        self.C = C.clone()
+        kw = dict(crown_relus=crown_relus, both_sides=both_sides, no_host_sync=True)
+        side = torch.cuda.Stream(device=centres.device)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):  # warm-up outside the capture: host caches, kernel attributes
+            self.out = net.verify(self.centres, eps, self.C, **kw)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize(centres.device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, capture_error_mode="relaxed"):
+            net.verify(self.centres, eps, self.C, out=self.out, **kw)
+
+    def replay(self):
+        self.graph.replay()
+        return self.out
 
 
 def concretize(lam: torch.Tensor, cst: Optional[torch.Tensor], centres: torch.Tensor, eps: float, stream=None):

@@ -178,6 +178,38 @@ def test_unstable_compaction_conv(monkeypatch, compact):
     assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out)
 
 
+def test_verify_graph_replays_match_plain_calls():
+    """A verify call captured in a CUDA graph gives the plain call's bounds, also after new inputs are
+    written into its buffers."""
+    w = synth.workload(2, B=38)
+    net = vf.Net(w.net)
+    c_all, C = _dev(w.centres), _dev(w.C)
+    a, b = c_all[:19].contiguous(), c_all[19:].contiguous()
+    vg = vf.VerifyGraph(net, a, w.eps, C)
+    for batch in (a, b, a):
+        vg.centres.copy_(batch)
+        got = {k: v.clone() for k, v in vg.replay().items()}
+        ref = net.verify(batch, w.eps, C)
+        torch.cuda.synchronize()
+        net.check()
+        for k in ("lb", "lb_ibp", "verified"):
+            assert torch.equal(got[k], ref[k]), k
+
+
+def test_verify_graph_cnn_with_windows_and_compaction_off():
+    """The captured call runs plain (uncompacted) passes; on a CNN its bounds match the plain call's
+    compacted ones and the oracle."""
+    w = synth.workload(3, B=2)
+    net = vf.Net(w.net)
+    c, C = _dev(w.centres), _dev(w.C)
+    vg = vf.VerifyGraph(net, c, w.eps, C)
+    got = {k: v.cpu().numpy() for k, v in vg.replay().items()}
+    ref = {k: v.cpu().numpy() for k, v in net.verify(c, w.eps, C).items()}
+    np.testing.assert_allclose(got["lb"], ref["lb"], rtol=1e-6, atol=1e-6)
+    ora = O.verify(w.net, w.centres, w.eps, w.C)
+    assert max_violation(got["lb"], ora.lb) <= 1.0
+
+
 @pytest.mark.parametrize("eps", [0.5 / 255, 1.0 / 255, 2.0 / 255])
 def test_cfg5_subset_each_eps(eps):
     w = synth.workload(5, B=2, eps=eps)
