@@ -360,14 +360,10 @@ cudaError_t launch_conv_back(const RowRef& A, Relax rx, const float* W, const fl
     if (M <= 0) return cudaSuccess;
     const ConvTiling t = make_tiling(g);
     const size_t smem = conv_back_smem_bytes(g);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(conv_back_ffma, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = allow_dyn_smem((const void*)conv_back_ffma, 200 * 1024);
+    if (e != cudaSuccess) return e;
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, conv_back_ffma, kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, conv_back_ffma, kThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
     const long long items = ((M + RG - 1) / RG) * (long long)(t.ntx * t.nty);

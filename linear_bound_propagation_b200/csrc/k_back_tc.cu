@@ -526,15 +526,14 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (fn == nullptr) {
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {  // thread-safe one-time lookup
         void* ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
             q != cudaDriverEntryPointSuccess)
             return nullptr;
-        fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
+        return reinterpret_cast<EncodeTiledFn>(ptr);
+    }();
     return fn;
 }
 
@@ -639,18 +638,11 @@ cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, 
     p.count_const = rx.count_const;
     p.err = err;
     p.test_stall = test_stall;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(dense_back_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
-    static int num_sms = 0;
-    if (num_sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    }
+    cudaError_t e = allow_dyn_smem((const void*)dense_back_tc, 220 * 1024);
+    if (e != cudaSuccess) return e;
+    int dev = 0, num_sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const long long grid = std::min<long long>(p.ntiles, num_sms);  // persistent: one CTA per SM
     dense_back_tc<<<(unsigned)grid, NUM_THREADS, smem, s>>>(ta, tp, tbh, tbl, p);
     return cudaGetLastError();

@@ -6,6 +6,10 @@
 // §2.1 (ReLU relaxation slopes from intermediate bounds; IBP as their substitute) and §3/§4.3
 // (per-neuron alpha slopes). Every row reduction here runs in a fixed order, so repeated calls
 // give bitwise-identical results.
+#include <mutex>
+#include <set>
+#include <tuple>
+
 #include "vf_internal.cuh"
 
 namespace vf {
@@ -454,6 +458,20 @@ cudaError_t launch_concretize_api(const float* lambda, const float* cst, const f
                                   int n0, float* lb, cudaStream_t s) {
     concretize_api_k<<<rows_grid(((long long)B * R + 7) / 8), 256, 0, s>>>(lambda, cst, centres, eps, B, R, n0, lb);
     return cudaGetLastError();
+}
+
+cudaError_t allow_dyn_smem(const void* func, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static std::mutex mu;
+    static std::set<std::tuple<const void*, int, int>> done;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_tuple(func, dev, bytes);
+    if (done.count(key)) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.insert(key);
+    return e;
 }
 
 }  // namespace vf

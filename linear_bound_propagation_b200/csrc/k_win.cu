@@ -468,13 +468,8 @@ cudaError_t launch_back_cb(const RowRef& A, Relax rx, const WinWeights& ww, cons
                            const ConvGeom& g, PassGeom pg, PassStart ps, const Win& wa, const Win& wd, int out_mode,
                            float* out, long long ld_out, float* cst, const float* centres, float eps,
                            const WinLaunch& L, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(conv_back_win_k<CB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kWinSmemLimit);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    const cudaError_t e = allow_dyn_smem((const void*)conv_back_win_k<CB>, kWinSmemLimit);
+    if (e != cudaSuccess) return e;
     conv_back_win_k<CB><<<warp_rows_grid(M, L.nwarps, L.ctas_per_sm), 32 * L.nwarps, L.smem, s>>>(
         A, rx, ww.Wt, ww.tap_stride, ww.ci_pad, L.w_in_smem, bias, M, g, pg, ps, wa, wd, out_mode, out, ld_out, cst,
         centres, eps, L.nwarps, L.stage_floats);
@@ -486,16 +481,11 @@ cudaError_t launch_back2(const RowRef& A, Relax rx, const WinWeights& ww, const 
                          const ConvGeom& g, PassGeom pg, PassStart ps, const Win& wa, const Win& wd, int out_mode,
                          float* out, long long ld_out, float* cst, const float* centres, float eps,
                          const Win2Launch& L, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(conv_back_win2_k<S, KS, CB, PM>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kWinSmemLimit);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    cudaError_t e = allow_dyn_smem((const void*)conv_back_win2_k<S, KS, CB, PM>, kWinSmemLimit);
+    if (e != cudaSuccess) return e;
     const float inv_hwd = 1.f / (float)wd.hw;
     int per_sm = 0;  // resident CTAs per SM (registers and shared memory)
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, conv_back_win2_k<S, KS, CB, PM>,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, conv_back_win2_k<S, KS, CB, PM>,
                                                                   32 * L.nwarps, L.smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;

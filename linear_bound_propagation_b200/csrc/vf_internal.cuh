@@ -205,6 +205,10 @@ cudaError_t launch_alpha_init(float* alpha, float* m1, float* m2, long long M, i
                               cudaStream_t s);
 cudaError_t launch_best_update(float* best, const float* cur, long long M, int first, cudaStream_t s);
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per (kernel,
+// device, size); safe to call from several threads.
+cudaError_t allow_dyn_smem(const void* func, int bytes);
+
 // Records `msg` as this thread's vf_last_error() text and returns `code`.
 int set_last_error(int code, const char* msg);
 
