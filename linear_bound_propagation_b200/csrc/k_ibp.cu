@@ -100,7 +100,7 @@ __global__ void ibp_conv_k(const float* __restrict__ hc, const float* __restrict
         float sc = 0.f, sr = 0.f;
         for (int ci = 0; ci < g.ci; ++ci) {
             const float* xc = hc + (b * g.ci + ci) * (long long)g.h * g.w;
-            const float* xr = hr + (b * g.ci + ci) * (long long)g.h * g.w;
+            const float* xr = hr != nullptr ? hr + (b * g.ci + ci) * (long long)g.h * g.w : nullptr;
             const float* wp = W + ((long long)co * g.ci + ci) * g.k * g.k;
             const float* wa = Wabs + ((long long)co * g.ci + ci) * g.k * g.k;
             for (int p = 0; p < g.k; ++p) {
@@ -110,12 +110,12 @@ __global__ void ibp_conv_k(const float* __restrict__ hc, const float* __restrict
                     const int x = oj * g.stride - g.pad + q;
                     if (x < 0 || x >= g.w) continue;
                     sc = fmaf(wp[p * g.k + q], xc[y * g.w + x], sc);
-                    sr = fmaf(wa[p * g.k + q], xr[y * g.w + x], sr);
+                    if (xr != nullptr) sr = fmaf(wa[p * g.k + q], xr[y * g.w + x], sr);
                 }
             }
         }
         zc[idx] = sc + bias[co];
-        zr[idx] = sr;
+        if (zr != nullptr) zr[idx] = sr;
     }
 }
 

@@ -883,13 +883,14 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
     return VF_OK;
 }
 
-// A ReLU MLP laid out input -> dense -> relu -> dense -> ... -> dense (nodes in that order).
+// A ReLU chain laid out input -> affine -> relu -> affine -> ... -> dense (nodes in that order), each
+// affine node dense or a convolution.
 bool dense_chain(const vf_net* net) {
     const int nn = (int)net->nodes.size();
     for (int v = 1; v < nn; ++v) {
         const Node& nd = net->nodes[v];
         if (nd.src != v - 1) return false;
-        if (nd.op != ((v % 2 == 1) ? VF_DENSE : VF_RELU)) return false;
+        if (v % 2 == 1 ? (nd.op != VF_DENSE && nd.op != VF_CONV2D) : nd.op != VF_RELU) return false;
     }
     return net->nodes[nn - 1].op == VF_DENSE;
 }
@@ -923,8 +924,12 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
     const long long rows = (long long)B * R;
     // per-row floats: H (sum_n) + Z (nmax) + lam_in (n0) + two gradient buffers (gmax) + cst + lb
     // (+ slopes and two Adam moments, 3 * sum_n, when optimising)
-    const size_t per_row = sizeof(float) * (sum_n + nmax + n0 + 2 * gmax + 2 + (grad_mode ? 0 : 3 * sum_n)) +
-                           64 * (relus.size() + 8);
+    int ctiles_max = 0;
+    for (int v = 1; v < L; v += 2)
+        if (net->nodes[v].op == VF_CONV2D) ctiles_max = std::max(ctiles_max, conv_back_tiles(conv_geom(net, net->nodes[v])));
+    const size_t per_row =
+        sizeof(float) * (sum_n + nmax + n0 + 2 * gmax + 2 + ctiles_max + (grad_mode ? 0 : 3 * sum_n)) +
+        64 * (relus.size() + 8);
     long long chunk = (long long)(ar.left() / per_row);
     if (chunk > rows) chunk = rows;
     if (chunk < 1) return fail(VF_ERR_WORKSPACE, "workspace too small for alpha optimisation");
@@ -943,7 +948,12 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
     float* G1 = ar.take<float>((size_t)chunk * gmax);
     float* cst = ar.take<float>(chunk);
     float* lbc = ar.take<float>(chunk);
-    if (!Z || !lam_in || !G0 || !G1 || !cst || !lbc) return fail(VF_ERR_WORKSPACE, "workspace too small");
+    int ctiles = 0;  // per-tile partials written by the convolution kernel (unused here: no bias, no relaxation)
+    for (int v = 1; v < L; v += 2)
+        if (net->nodes[v].op == VF_CONV2D) ctiles = std::max(ctiles, conv_back_tiles(conv_geom(net, net->nodes[v])));
+    float* cpart = ctiles ? ar.take<float>((size_t)chunk * ctiles) : nullptr;
+    if (!Z || !lam_in || !G0 || !G1 || !cst || !lbc || (ctiles && !cpart))
+        return fail(VF_ERR_WORKSPACE, "workspace too small");
     for (int u : relus)
         if (!H[u] || (!grad_mode && (!A[u] || !M1[u] || !M2[u]))) return fail(VF_ERR_WORKSPACE, "workspace too small");
 
@@ -974,8 +984,14 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
                 const int nd_in = (int)net->nodes[u - 2].n;
                 LAUNCH(net, launch_relax_alpha_rows(H[u], Mc, nu, bd.relax[u], pg, al[u], Z, cst, s));
                 float* out = (u - 2 == 0) ? lam_in : H[u - 2];
-                LAUNCH(net, launch_dense_back(RowRef{Z, 0, nu, kHugeRows, 0}, Relax{nullptr, 0}, d.W, nullptr, Mc, nu,
-                                              nd_in, pg, OUT_STORE, out, nd_in, nullptr, nullptr, 0.f, nullptr, s));
+                if (d.op == VF_CONV2D)
+                    LAUNCH(net, launch_conv_back(RowRef{Z, 0, nu, kHugeRows, 0}, Relax{nullptr, 0}, d.W, nullptr, Mc,
+                                                 conv_geom(net, d), pg, OUT_STORE, out, nd_in, cpart, nullptr, 0.f,
+                                                 net->num_sms, s));
+                else
+                    LAUNCH(net, launch_dense_back(RowRef{Z, 0, nu, kHugeRows, 0}, Relax{nullptr, 0}, d.W, nullptr, Mc,
+                                                  nu, nd_in, pg, OUT_STORE, out, nd_in, nullptr, nullptr, 0.f, nullptr,
+                                                  s));
             }
             LAUNCH(net, launch_concretize_grad(lam_in, Mc, (int)n0, pg, centres, eps, cst, lbc, G0, s));
             if (it == 0 && lb_start) CU(cudaMemcpyAsync(lb_start + m0, lbc, sizeof(float) * Mc, cudaMemcpyDeviceToDevice, s));
@@ -988,7 +1004,11 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
                 const Node& dn = net->nodes[d];
                 const int u = d + 1;
                 const int nu = (int)net->nodes[u].n;
-                LAUNCH(net, launch_rows_times_wt(G, dn.W, dn.b, (int)Mc, (int)net->nodes[d - 1].n, nu, Gn, s));
+                if (dn.op == VF_CONV2D)
+                    LAUNCH(net, launch_ibp_conv(G, nullptr, dn.W, dn.Wabs, dn.b, (int)Mc, conv_geom(net, dn), Gn,
+                                                nullptr, s));
+                else
+                    LAUNCH(net, launch_rows_times_wt(G, dn.W, dn.b, (int)Mc, (int)net->nodes[d - 1].n, nu, Gn, s));
                 float* gout = grad_mode ? grad_out + aoff[u] + m0 * nu : nullptr;
                 LAUNCH(net, launch_relax_grad_adam(Gn, H[u], Mc, nu, bd.relax[u], pg, al[u], gout, M1[u], M2[u],
                                                    grad_mode ? 0 : it + 1, lr, s));
@@ -1387,7 +1407,7 @@ int vf_alpha_crown(vf_net* net, const float* centres, int B, float eps, const fl
     if (B < 0 || R < 0 || C_bstride < 0 || iters < 0) return fail(VF_ERR_ARG, "negative size");
     if (!std::isfinite(eps) || eps < 0.f || !std::isfinite(lr) || lr < 0.f)
         return fail(VF_ERR_NONFINITE, "eps and lr must be finite and >= 0");
-    if (!dense_chain(net)) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation needs a dense ReLU chain");
+    if (!dense_chain(net)) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation needs a ReLU chain of dense/conv layers");
     if (o.both_sides) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation bounds the lower side; pass -C for upper");
     if (B == 0 || R == 0) return VF_OK;
     return spec_alpha(net, centres, B, eps, C, R, C_bstride, o, iters, lr, false, nullptr, nullptr, lb, lb_start,
@@ -1402,7 +1422,7 @@ int vf_alpha_grad(vf_net* net, const float* centres, int B, float eps, const flo
     if (!centres || !C || !lb || !alpha || !grad) return fail(VF_ERR_ARG, "NULL pointer");
     if (B < 0 || R < 0 || C_bstride < 0) return fail(VF_ERR_ARG, "negative size");
     if (!std::isfinite(eps) || eps < 0.f) return fail(VF_ERR_NONFINITE, "eps must be finite and >= 0");
-    if (!dense_chain(net)) return fail(VF_ERR_UNSUPPORTED, "alpha gradients need a dense ReLU chain");
+    if (!dense_chain(net)) return fail(VF_ERR_UNSUPPORTED, "alpha gradients need a ReLU chain of dense/conv layers");
     if (B == 0 || R == 0) return VF_OK;
     return spec_alpha(net, centres, B, eps, C, R, C_bstride, o, 0, 0.f, true, alpha, grad, lb, nullptr, nullptr,
                       (cudaStream_t)stream);

@@ -141,6 +141,7 @@ cudaError_t launch_rewin_rows(const RowRef& A, Relax rx, long long M, int C, int
 cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
                              const float* rowsum_abs, float eps, int B, int K, int N, float* zc, float* zr,
                              cudaStream_t s);
+// hr and zr may both be NULL: then only the centre map W * hc + b is computed (the alpha-CROWN gradient).
 cudaError_t launch_ibp_conv(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
                             int B, const ConvGeom& g, float* zc, float* zr, cudaStream_t s);
 cudaError_t launch_ibp_relu(const float* c, const float* r, long long n, float* oc, float* orad, cudaStream_t s);

@@ -370,16 +370,17 @@ def verify(net, centres, eps, C, crown_relus: Optional[Sequence[int]] = None,
 # ----------------------------------------------------------------------------- alpha-CROWN
 
 def _dense_chain(net):
-    """Node ids of a ReLU MLP written as input -> dense -> relu -> ... -> dense, else None."""
-    if net[0].op != "input":
+    """Node ids of the affine nodes of a chain input -> affine -> relu -> ... -> dense, where each affine
+    node is dense or a convolution, else None."""
+    if net[0].op != "input" or net[-1].op != "dense":
         return None
     for v in range(1, len(net)):
         nd = net[v]
-        if nd.src != v - 1 or nd.op not in ("dense", "relu"):
+        if nd.src != v - 1 or nd.op not in ("dense", "conv", "relu"):
             return None
-        if (nd.op == "dense") == (v % 2 == 0):
+        if (nd.op != "relu") == (v % 2 == 0):
             return None
-    return [v for v in range(len(net)) if net[v].op == "dense"]
+    return [v for v in range(len(net)) if net[v].op != "relu" and v > 0]
 
 
 def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows):
@@ -395,12 +396,14 @@ def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows):
     to the coefficients over a node's output,
       input:   G = centre - eps * sign(lam_in)             (from lam . centre - eps |lam|)
       dense:   G_z = G_h W^T + b                           (lam_h = lam_z W,  const += lam_z . b)
+      conv:    G_z = conv(G_h) + b per channel             (lam_h = conv^T(lam_z), const += sum lam_z b)
       relu:    dlb/dalpha_i = G_z,i * lam_h,i * [lam_h,i >= 0]   for unstable i
                G_h = G_z * slope + [lam_h < 0] * t         (lam_z = slope * lam_h, const += min(lam_h, 0) t)
     """
     chain = _dense_chain(net)
     if chain is None:
-        raise ValueError("alpha optimisation is defined here for dense ReLU chains")
+        raise ValueError("alpha optimisation is defined here for ReLU chains of dense and convolution layers")
+    sh = shapes(net)
     L = len(net) - 1
     lam = np.asarray(rows, F)
     R = lam.shape[0]
@@ -411,6 +414,10 @@ def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows):
         if nd.op == "dense":
             const = const + lam @ nd.b.astype(F)
             lam = lam @ nd.W.astype(F)
+        elif nd.op == "conv":
+            lam4 = lam.reshape((R,) + sh[v])
+            const = const + lam4.reshape(R, nd.W.shape[0], -1).sum(axis=2) @ nd.b.astype(F)
+            lam = conv2d_adjoint(lam4, nd.W, nd.stride, nd.pad, sh[nd.src][1:]).reshape(R, -1)
         else:
             lo, up, t = relax[v]
             unst = (up > 0.0) & (up < 1.0)
@@ -427,6 +434,9 @@ def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows):
         nd = net[v]
         if nd.op == "dense":
             G = G @ nd.W.astype(F).T + nd.b.astype(F)[None, :]
+        elif nd.op == "conv":
+            Gz = conv2d(G.reshape((R,) + sh[nd.src]), nd.W, nd.stride, nd.pad) + nd.b.astype(F)[None, :, None, None]
+            G = Gz.reshape(R, -1)
         else:
             lam_h, slope, unst = saved[v]
             t = relax[v][2]

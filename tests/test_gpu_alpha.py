@@ -27,7 +27,7 @@ def _oracle_relax(net, res, b):
             for k, nd in enumerate(net) if nd.op == "relu"}
 
 
-@pytest.mark.parametrize("config,B", [(1, 16), (2, 6)])
+@pytest.mark.parametrize("config,B", [(1, 16), (2, 6), (3, 2)])
 def test_alpha_grad_matches_oracle(config, B):
     w = synth.workload(config, B=B)
     net, R = w.net, w.C.shape[1]
@@ -66,7 +66,7 @@ def test_alpha_grad_matches_oracle(config, B):
     assert checked >= B // 2
 
 
-@pytest.mark.parametrize("config,B", [(1, 64), (2, 16)])
+@pytest.mark.parametrize("config,B", [(1, 64), (2, 16), (3, 3)])
 def test_alpha_crown_improves_soundly_and_tracks_oracle(config, B):
     w = synth.workload(config, B=B)
     net = w.net
@@ -89,8 +89,11 @@ def test_alpha_crown_improves_soundly_and_tracks_oracle(config, B):
 
 
 def test_alpha_rejects_non_chains():
-    w = synth.workload(3, B=2)
-    g = vf.Net(w.net)
+    rng = np.random.default_rng(7)
+    net = synth.resnet_cfg4(rng, image=(3, 8, 8), widths=(3, 4, 5), fc=6, classes=4)
+    centres = rng.random((2, 3 * 8 * 8)).astype(np.float32)
+    C = synth.margin_spec(np.array([0, 1]), 4)
+    g = vf.Net(net)
     with pytest.raises(vf.VfError) as e:
-        g.alpha_crown(_dev(w.centres), w.eps, _dev(w.C), iters=1)
+        g.alpha_crown(_dev(centres), 0.01, _dev(C), iters=1)
     assert e.value.code == vf.VF_ERR_UNSUPPORTED

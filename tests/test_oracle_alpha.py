@@ -45,6 +45,57 @@ def check_fd_gradient(seed=0):
     return True, ""
 
 
+def _setup_conv(seed=0, eps=0.15):
+    """A small convolutional chain: conv 3x3 s1 p1, ReLU, conv 2x2 s2, ReLU, dense, ReLU, dense."""
+    rng = np.random.default_rng(100 + seed)
+    net = [synth.Node(synth.INPUT, shape=(2, 6, 6))]
+    v = synth._relu(net, synth._conv(net, rng, 0, 2, 3, 3, 1, 1))
+    v = synth._relu(net, synth._conv(net, rng, v, 3, 4, 2, 2, 0))
+    v = synth._relu(net, synth._dense(net, rng, v, 4 * 3 * 3, 5))
+    synth._dense(net, rng, v, 5, 3)
+    c = rng.random((1, 2 * 6 * 6)).astype(np.float32)
+    C = synth.margin_spec(np.array([0]), 3)
+    res = O.verify(net, c, eps, C)
+    relax = {k: O.relax_params(res.pre_bounds[k][0][0], res.pre_bounds[k][1][0]) for k in relu_ids(net)}
+    return rng, net, c, C, eps, res, relax
+
+
+def check_fd_gradient_conv(seed=0):
+    rng, net, c, C, eps, res, relax = _setup_conv(seed)
+    R = C.shape[1]
+    a = {k: rng.random((R, relax[k][0].size)) for k in relax}
+    lb, g = O.spec_bound_alpha(net, c[0], eps, C[0], relax, a)
+    h = 1e-6
+    n_checked = 0
+    for k in relax:
+        unst = (relax[k][1] > 0) & (relax[k][1] < 1)
+        for i in range(a[k].shape[1]):
+            for r in range(R):
+                ap = {kk: v.copy() for kk, v in a.items()}
+                am = {kk: v.copy() for kk, v in a.items()}
+                ap[k][r, i] += h
+                am[k][r, i] -= h
+                fd = (O.spec_bound_alpha(net, c[0], eps, C[0], relax, ap)[0][r] -
+                      O.spec_bound_alpha(net, c[0], eps, C[0], relax, am)[0][r]) / (2 * h)
+                if abs(fd - g[k][r, i]) > 1e-6 * (1 + abs(fd)):
+                    return False, f"conv gradient mismatch relu {k} row {r} neuron {i}: {g[k][r, i]} vs {fd}"
+                if not unst[i] and g[k][r, i] != 0.0:
+                    return False, "nonzero gradient on a stable neuron"
+                n_checked += int(unst[i])
+    if n_checked < 10:
+        return False, "too few unstable neurons for the check to mean anything"
+    return True, ""
+
+
+def check_adaptive_start_is_crown_conv(seed=1):
+    rng, net, c, C, eps, res, relax = _setup_conv(seed)
+    a = {k: np.repeat(relax[k][0][None, :], C.shape[1], axis=0) for k in relax}
+    lb, _ = O.spec_bound_alpha(net, c[0], eps, C[0], relax, a)
+    if not np.allclose(lb, res.lb_crown[0], rtol=1e-12, atol=1e-12):
+        return False, "adaptive slopes do not reproduce the CROWN bound on a convolutional chain"
+    return True, ""
+
+
 def check_adaptive_start_is_crown(seed=1):
     rng, net, c, C, eps, res, relax = _setup(seed)
     a = {k: np.repeat(relax[k][0][None, :], C.shape[1], axis=0) for k in relax}
@@ -83,7 +134,8 @@ def check_optimised_sound(seed=2):
     return True, ""
 
 
-CHECKS = [check_fd_gradient, check_adaptive_start_is_crown, check_hand_optimum, check_optimised_sound]
+CHECKS = [check_fd_gradient, check_adaptive_start_is_crown, check_hand_optimum, check_optimised_sound,
+          check_fd_gradient_conv, check_adaptive_start_is_crown_conv]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=[c.__name__ for c in CHECKS])
@@ -93,15 +145,19 @@ def test_alpha_pin(check):
 
 
 MUTATIONS = [
-    ("G = G @ nd.W.astype(F).T + nd.b.astype(F)[None, :]", "G = G @ nd.W.astype(F).T"),
-    ("G = G * slope + np.where(lam_h < 0.0, t[None, :], 0.0)", "G = G * slope"),
-    ("G = c[None, :] - F(eps) * np.sign(lam)", "G = c[None, :] + F(eps) * np.sign(lam)"),
-    ("np.where(unst[None, :] & (lam_h >= 0.0), G * lam_h, 0.0)", "np.where(unst[None, :], G * lam_h, 0.0)"),
+    ("G = G @ nd.W.astype(F).T + nd.b.astype(F)[None, :]", "G = G @ nd.W.astype(F).T", check_fd_gradient),
+    ("G = G * slope + np.where(lam_h < 0.0, t[None, :], 0.0)", "G = G * slope", check_fd_gradient),
+    ("G = c[None, :] - F(eps) * np.sign(lam)", "G = c[None, :] + F(eps) * np.sign(lam)", check_fd_gradient),
+    ("np.where(unst[None, :] & (lam_h >= 0.0), G * lam_h, 0.0)", "np.where(unst[None, :], G * lam_h, 0.0)",
+     check_fd_gradient),
+    ("nd.pad) + nd.b.astype(F)[None, :, None, None]", "nd.pad)", check_fd_gradient_conv),
+    ("Gz = conv2d(G.reshape((R,) + sh[nd.src]), nd.W, nd.stride, nd.pad)",
+     "Gz = conv2d(G.reshape((R,) + sh[nd.src]), nd.W[:, :, ::-1, ::-1], nd.stride, nd.pad)", check_fd_gradient_conv),
 ]
 
 
-@pytest.mark.parametrize("old,new", MUTATIONS)
-def test_gradient_mutation_is_caught(monkeypatch, old, new):
+@pytest.mark.parametrize("old,new,check", MUTATIONS)
+def test_gradient_mutation_is_caught(monkeypatch, old, new, check):
     src = textwrap.dedent(inspect.getsource(O.spec_bound_alpha))
     assert src.count(old) == 1
     ns = {}
@@ -109,6 +165,6 @@ def test_gradient_mutation_is_caught(monkeypatch, old, new):
     monkeypatch.setattr(O, "spec_bound_alpha", ns["spec_bound_alpha"])
     caught = False
     for seed in range(3):
-        ok, _ = check_fd_gradient(seed)
+        ok, _ = check(seed)
         caught |= not ok
     assert caught
