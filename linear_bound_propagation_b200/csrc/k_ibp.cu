@@ -14,74 +14,81 @@ namespace vf {
 namespace {
 
 // z[m, n] = sum_k h[m, k] * W[n, k]: blockIdx.z = 0 computes the centre (h = centre, W, + bias), 1 the
-// radius (h = radius, |W|). Tiles of 16 rows x 64 columns, 256 threads (one row x 4 columns each), the next
-// k-slice prefetched into registers while the current one is used. With rowsum_abs != nullptr the source is
-// the input box with radius eps in every coordinate: the radius is eps * sum_k |W[n, k]| without a product.
+// radius (h = radius, |W|). Tiles of 64 rows x 64 columns, 256 threads each owning a 4 x 4 block of
+// outputs; per k the thread reads one float4 of the staged h tile and one of the staged W tile for 16
+// FMAs. The next 16-wide k-slice is prefetched into registers while the current one is used. With
+// rowsum_abs != nullptr the source is the input box with radius eps in every coordinate: the radius is
+// eps * sum_k |W[n, k]| without a product.
 __global__ void __launch_bounds__(256)
 ibp_dense_k(const float* __restrict__ hc, const float* __restrict__ hr, const float* __restrict__ W,
             const float* __restrict__ Wabs, const float* __restrict__ bias, const float* __restrict__ rowsum_abs,
             float eps, int B, int K, int N, float* __restrict__ zc, float* __restrict__ zr) {
-    constexpr int TM = 16, TN = 64, KB = 32;
-    __shared__ float As[KB][TM + 1], Bs[KB][TN + 1];
+    constexpr int TM = 64, TN = 64, KB = 16, LDA = TM + 4, LDB = TN + 4;
+    __shared__ __align__(16) float As[KB][LDA];
+    __shared__ __align__(16) float Bs[KB][LDB];
     const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
     const int m0 = blockIdx.x * TM, n0 = blockIdx.y * TN;
     const bool rad = blockIdx.z == 1;
     if (rad && rowsum_abs != nullptr) {
-        const int m = m0 + ty;
-        for (int j = 0; j < 4; ++j) {
-            const int n = n0 + tx + 16 * j;
+        for (int e = tid; e < TM * TN; e += 256) {
+            const int m = m0 + e / TN, n = n0 + e % TN;
             if (m < B && n < N) zr[(long long)m * N + n] = eps * rowsum_abs[n];
         }
         return;
     }
     const float* h = rad ? hr : hc;
     const float* w = rad ? Wabs : W;
-    float a_reg[2], b_reg[8];
+    // loader mapping: 64 rows x 16 k per tile = 1024 values, 4 per thread (k fastest for coalescing)
+    float a_reg[4], b_reg[4];
     auto load = [&](int k0) {
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int e = tid + 256 * i, row = e / KB, kk = e % KB, m = m0 + row, k = k0 + kk;
+        for (int i = 0; i < 4; ++i) {
+            const int e = tid + 256 * i, row = e / KB, kk = e % KB, k = k0 + kk;
+            const int m = m0 + row, n = n0 + row;
             a_reg[i] = (m < B && k < K) ? h[(long long)m * K + k] : 0.f;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int e = tid + 256 * i, row = e / KB, kk = e % KB, n = n0 + row, k = k0 + kk;
             b_reg[i] = (n < N && k < K) ? w[(long long)n * K + k] : 0.f;
         }
     };
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
     load(0);
     for (int k0 = 0; k0 < K; k0 += KB) {
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 4; ++i) {
             const int e = tid + 256 * i;
             As[e % KB][e / KB] = a_reg[i];
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int e = tid + 256 * i;
             Bs[e % KB][e / KB] = b_reg[i];
         }
         __syncthreads();
         if (k0 + KB < K) load(k0 + KB);
 #pragma unroll
         for (int kk = 0; kk < KB; ++kk) {
-            const float a = As[kk][ty];
+            const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+            const float4 bb = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[j] = fmaf(a, Bs[kk][tx + 16 * j], acc[j]);
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
         __syncthreads();
     }
-    const int m = m0 + ty;
-    if (m >= B) return;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int n = n0 + tx + 16 * j;
-        if (n >= N) continue;
-        if (rad)
-            zr[(long long)m * N + n] = acc[j];
-        else
-            zc[(long long)m * N + n] = acc[j] + bias[n];
+    for (int i = 0; i < 4; ++i) {
+        const int m = m0 + ty * 4 + i;
+        if (m >= B) break;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = n0 + tx * 4 + j;
+            if (n >= N) continue;
+            if (rad)
+                zr[(long long)m * N + n] = acc[i][j];
+            else
+                zc[(long long)m * N + n] = acc[i][j] + bias[n];
+        }
     }
 }
 
@@ -161,14 +168,14 @@ unsigned grid_for(long long n, int threads) {
 cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
                              const float* rowsum_abs, float eps, int B, int K, int N, float* zc, float* zr,
                              cudaStream_t s) {
-    dim3 grid((B + 15) / 16, (N + 63) / 64, 2);
+    dim3 grid((B + 63) / 64, (N + 63) / 64, 2);
     ibp_dense_k<<<grid, 256, 0, s>>>(hc, hr, W, Wabs, bias, rowsum_abs, eps, B, K, N, zc, zr);
     return cudaGetLastError();
 }
 
 cudaError_t launch_rows_times_wt(const float* A, const float* W, const float* bias, int M, int K, int N, float* out,
                                  cudaStream_t s) {
-    dim3 grid((M + 15) / 16, (N + 63) / 64, 1);  // only the centre product: out = A W^T + bias
+    dim3 grid((M + 63) / 64, (N + 63) / 64, 1);  // only the centre product: out = A W^T + bias
     ibp_dense_k<<<grid, 256, 0, s>>>(A, A, W, W, bias, nullptr, 0.f, M, K, N, out, out);
     return cudaGetLastError();
 }
