@@ -397,51 +397,68 @@ def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows):
       input:   G = centre - eps * sign(lam_in)             (from lam . centre - eps |lam|)
       dense:   G_z = G_h W^T + b                           (lam_h = lam_z W,  const += lam_z . b)
       conv:    G_z = conv(G_h) + b per channel             (lam_h = conv^T(lam_z), const += sum lam_z b)
+      add:     G_y = G_a + G_b                             (lam_a += lam_y, lam_b += lam_y)
       relu:    dlb/dalpha_i = G_z,i * lam_h,i * [lam_h,i >= 0]   for unstable i
                G_h = G_z * slope + [lam_h < 0] * t         (lam_z = slope * lam_h, const += min(lam_h, 0) t)
     """
-    chain = _dense_chain(net)
-    if chain is None:
-        raise ValueError("alpha optimisation is defined here for ReLU chains of dense and convolution layers")
     sh = shapes(net)
     L = len(net) - 1
-    lam = np.asarray(rows, F)
-    R = lam.shape[0]
+    R = np.asarray(rows).shape[0]
     const = np.zeros(R, F)
-    saved = {}  # relu node -> (lam_h, slope) used on the way down
+    pend: Dict[int, np.ndarray] = {L: np.asarray(rows, F)}
+    saved = {}  # relu node -> (lam_h, slope, unstable) used on the way down
+
+    def put(v, m):
+        pend[v] = pend[v] + m if v in pend else m
+
     for v in range(L, 0, -1):
+        if v not in pend:
+            continue
+        lam = pend.pop(v)
         nd = net[v]
         if nd.op == "dense":
             const = const + lam @ nd.b.astype(F)
-            lam = lam @ nd.W.astype(F)
+            put(nd.src, lam @ nd.W.astype(F))
         elif nd.op == "conv":
             lam4 = lam.reshape((R,) + sh[v])
             const = const + lam4.reshape(R, nd.W.shape[0], -1).sum(axis=2) @ nd.b.astype(F)
-            lam = conv2d_adjoint(lam4, nd.W, nd.stride, nd.pad, sh[nd.src][1:]).reshape(R, -1)
-        else:
+            put(nd.src, conv2d_adjoint(lam4, nd.W, nd.stride, nd.pad, sh[nd.src][1:]).reshape(R, -1))
+        elif nd.op == "relu":
             lo, up, t = relax[v]
             unst = (up > 0.0) & (up < 1.0)
             lo_rows = np.where(unst[None, :], np.asarray(alpha_rows[v], F), lo[None, :])
             slope = np.where(lam >= 0.0, lo_rows, up[None, :])
             const = const + np.minimum(lam, 0.0) @ t
             saved[v] = (lam, slope, unst)
-            lam = lam * slope
+            put(nd.src, lam * slope)
+        else:  # add: both branches receive the rows
+            put(nd.src, lam)
+            put(nd.src2, lam)
+    lam_in = pend[0]
     c = np.asarray(centre, F)
-    lb = lam @ c - F(eps) * np.abs(lam).sum(axis=1) + const
-    G = c[None, :] - F(eps) * np.sign(lam)
+    lb = lam_in @ c - F(eps) * np.abs(lam_in).sum(axis=1) + const
+    # G[v]: gradient of lb with respect to the coefficients over node v's output, in topological order
+    G = {0: c[None, :] - F(eps) * np.sign(lam_in)}
     grads = {}
     for v in range(1, L + 1):
         nd = net[v]
         if nd.op == "dense":
-            G = G @ nd.W.astype(F).T + nd.b.astype(F)[None, :]
+            G[v] = G[nd.src] @ nd.W.astype(F).T + nd.b.astype(F)[None, :]
         elif nd.op == "conv":
-            Gz = conv2d(G.reshape((R,) + sh[nd.src]), nd.W, nd.stride, nd.pad) + nd.b.astype(F)[None, :, None, None]
-            G = Gz.reshape(R, -1)
-        else:
+            Gz = conv2d(G[nd.src].reshape((R,) + sh[nd.src]), nd.W, nd.stride, nd.pad) + nd.b.astype(F)[None, :, None, None]
+            G[v] = Gz.reshape(R, -1)
+        elif nd.op == "relu":
+            Gz = G[nd.src]
+            if v not in saved:  # not an ancestor of the last node: its slopes do not enter lb
+                grads[v] = np.zeros((R, _size(sh[v])), F)
+                G[v] = np.zeros_like(Gz)
+                continue
             lam_h, slope, unst = saved[v]
             t = relax[v][2]
-            grads[v] = np.where(unst[None, :] & (lam_h >= 0.0), G * lam_h, 0.0)
-            G = G * slope + np.where(lam_h < 0.0, t[None, :], 0.0)
+            grads[v] = np.where(unst[None, :] & (lam_h >= 0.0), Gz * lam_h, 0.0)
+            G[v] = Gz * slope + np.where(lam_h < 0.0, t[None, :], 0.0)
+        else:
+            G[v] = G[nd.src] + G[nd.src2]
     return lb, grads
 
 

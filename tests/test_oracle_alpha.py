@@ -87,6 +87,47 @@ def check_fd_gradient_conv(seed=0):
     return True, ""
 
 
+def _setup_residual(seed=0, eps=0.05):
+    rng = np.random.default_rng(200 + seed)
+    net = synth.resnet_cfg4(rng, image=(2, 8, 8), widths=(2, 3, 3), fc=4, classes=3)
+    c = rng.random((1, 2 * 8 * 8)).astype(np.float32)
+    C = synth.margin_spec(np.array([1]), 3)
+    res = O.verify(net, c, eps, C)
+    relax = {k: O.relax_params(res.pre_bounds[k][0][0], res.pre_bounds[k][1][0]) for k in relu_ids(net)}
+    return rng, net, c, C, eps, res, relax
+
+
+def check_fd_gradient_residual(seed=0, samples=40):
+    """Central differences on a residual net (identity and 1x1-convolution shortcuts) for a seeded sample
+    of (row, unstable neuron) pairs of every ReLU layer."""
+    rng, net, c, C, eps, res, relax = _setup_residual(seed)
+    R = C.shape[1]
+    a = {k: rng.random((R, relax[k][0].size)) for k in relax}
+    lb, g = O.spec_bound_alpha(net, c[0], eps, C[0], relax, a)
+    if not np.allclose(O.spec_bound_alpha(net, c[0], eps, C[0], relax,
+                                          {k: np.repeat(relax[k][0][None, :], R, axis=0) for k in relax})[0],
+                       res.lb_crown[0], rtol=1e-12, atol=1e-12):
+        return False, "adaptive slopes do not reproduce the CROWN bound on a residual net"
+    h = 1e-6
+    n_checked = 0
+    for k in relax:
+        unst = np.nonzero((relax[k][1] > 0) & (relax[k][1] < 1))[0]
+        for i in rng.permutation(unst)[:samples]:
+            for r in range(R):
+                ap = {kk: v.copy() for kk, v in a.items()}
+                am = {kk: v.copy() for kk, v in a.items()}
+                ap[k][r, i] += h
+                am[k][r, i] -= h
+                fd = (O.spec_bound_alpha(net, c[0], eps, C[0], relax, ap)[0][r] -
+                      O.spec_bound_alpha(net, c[0], eps, C[0], relax, am)[0][r]) / (2 * h)
+                if abs(fd - g[k][r, i]) > 1e-6 * (1 + abs(fd)):
+                    return False, f"residual gradient mismatch relu {k} row {r} neuron {i}: {g[k][r, i]} vs {fd}"
+                n_checked += 1
+    if n_checked < 20:
+        return False, "too few unstable neurons for the check to mean anything"
+    return True, ""
+
+
 def check_adaptive_start_is_crown_conv(seed=1):
     rng, net, c, C, eps, res, relax = _setup_conv(seed)
     a = {k: np.repeat(relax[k][0][None, :], C.shape[1], axis=0) for k in relax}
@@ -135,7 +176,7 @@ def check_optimised_sound(seed=2):
 
 
 CHECKS = [check_fd_gradient, check_adaptive_start_is_crown, check_hand_optimum, check_optimised_sound,
-          check_fd_gradient_conv, check_adaptive_start_is_crown_conv]
+          check_fd_gradient_conv, check_adaptive_start_is_crown_conv, check_fd_gradient_residual]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=[c.__name__ for c in CHECKS])
@@ -145,14 +186,18 @@ def test_alpha_pin(check):
 
 
 MUTATIONS = [
-    ("G = G @ nd.W.astype(F).T + nd.b.astype(F)[None, :]", "G = G @ nd.W.astype(F).T", check_fd_gradient),
-    ("G = G * slope + np.where(lam_h < 0.0, t[None, :], 0.0)", "G = G * slope", check_fd_gradient),
-    ("G = c[None, :] - F(eps) * np.sign(lam)", "G = c[None, :] + F(eps) * np.sign(lam)", check_fd_gradient),
-    ("np.where(unst[None, :] & (lam_h >= 0.0), G * lam_h, 0.0)", "np.where(unst[None, :], G * lam_h, 0.0)",
+    ("G[v] = G[nd.src] @ nd.W.astype(F).T + nd.b.astype(F)[None, :]", "G[v] = G[nd.src] @ nd.W.astype(F).T",
+     check_fd_gradient),
+    ("G[v] = Gz * slope + np.where(lam_h < 0.0, t[None, :], 0.0)", "G[v] = Gz * slope", check_fd_gradient),
+    ("G = {0: c[None, :] - F(eps) * np.sign(lam_in)}", "G = {0: c[None, :] + F(eps) * np.sign(lam_in)}",
+     check_fd_gradient),
+    ("np.where(unst[None, :] & (lam_h >= 0.0), Gz * lam_h, 0.0)", "np.where(unst[None, :], Gz * lam_h, 0.0)",
      check_fd_gradient),
     ("nd.pad) + nd.b.astype(F)[None, :, None, None]", "nd.pad)", check_fd_gradient_conv),
-    ("Gz = conv2d(G.reshape((R,) + sh[nd.src]), nd.W, nd.stride, nd.pad)",
-     "Gz = conv2d(G.reshape((R,) + sh[nd.src]), nd.W[:, :, ::-1, ::-1], nd.stride, nd.pad)", check_fd_gradient_conv),
+    ("Gz = conv2d(G[nd.src].reshape((R,) + sh[nd.src]), nd.W, nd.stride, nd.pad)",
+     "Gz = conv2d(G[nd.src].reshape((R,) + sh[nd.src]), nd.W[:, :, ::-1, ::-1], nd.stride, nd.pad)",
+     check_fd_gradient_conv),
+    ("G[v] = G[nd.src] + G[nd.src2]", "G[v] = G[nd.src]", check_fd_gradient_residual),
 ]
 
 
