@@ -353,7 +353,7 @@ def run_ours(args):
     roof = roofline(kstats, total_ms, torch.cuda.get_device_properties(dev).multi_processor_count,
                     w.name if args.centres is None else None)
     alpha = None
-    if args.alpha_iters > 0 and all(nd.op in ("input", "dense", "conv", "relu") for nd in w.net) and not w.both_sides:
+    if args.alpha_iters > 0 and not w.both_sides:
         # alpha-CROWN leg: the same workload, intermediate bounds as above, then per-row slope optimisation
         net.alpha_crown(centres, w.eps, C, iters=args.alpha_iters, crown_relus=w.crown_relus)  # warm-up
         torch.cuda.synchronize()

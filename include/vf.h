@@ -149,8 +149,9 @@ int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const f
  * within [0, 1], by `iters` steps of projected gradient ascent with Adam (betas 0.9, 0.999, step `lr`)
  * from the adaptive slopes. Intermediate bounds are computed as in vf_verify_batch (opts->relu_crown,
  * opts->alpha) and stay fixed. Any slope in [0, 1] gives a sound bound, so every iterate is sound.
- * Networks: ReLU chains (input, affine, relu, ..., dense) whose affine nodes are dense or convolutions;
- * residual nets return VF_ERR_UNSUPPORTED, as does opts->both_sides (pass -C for upper bounds).
+ * Networks: any graph of this library whose last node is dense (chains of dense/convolution layers take
+ * a fused path; residual graphs keep every node's coefficients); opts->both_sides returns
+ * VF_ERR_UNSUPPORTED (pass -C for upper bounds).
  * Outputs [device]: lb [B, R] the best CROWN lower bound over the iterates (not intersected with IBP);
  * lb_start [B, R] (or NULL) the bound at the adaptive start; alpha_out (or NULL) the final slopes, one
  * [B, R, n_v] block per ReLU node v in node order. C [device] [B or 1, R, n_L] with centre stride C_bstride. */

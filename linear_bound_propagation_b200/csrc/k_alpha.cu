@@ -39,11 +39,13 @@ __device__ __forceinline__ float block_sum256(float v, float* red) {
     return t;
 }
 
-// Z[m, :] = slope * H[m, :] with per-row slopes for unstable neurons (alpha == nullptr: the table's
-// own lower slope); cst[m] += sum min(H, 0) * t + Z * bias (bias in P.w). One CTA per row.
+// Z[m, :] (=, += with accumulate) slope * H[m, :] with per-row slopes for unstable neurons (alpha ==
+// nullptr: the table's own lower slope); cst[m] += sum min(H, 0) * t (+ Z * bias, bias in P.w, when
+// with_bias). One CTA per row.
 __global__ void __launch_bounds__(256)
 relax_alpha_rows_k(const float* __restrict__ H, long long M, int n, const float4* __restrict__ P, PassGeom pg,
-                   const float* __restrict__ alpha, float* __restrict__ Z, float* __restrict__ cst) {
+                   const float* __restrict__ alpha, float* __restrict__ Z, float* __restrict__ cst, int with_bias,
+                   int accumulate) {
     __shared__ float red[8];
     for (long long m = blockIdx.x; m < M; m += gridDim.x) {
         const long long b = (pg.pass_m0 + m) / pg.R_pass;
@@ -56,8 +58,8 @@ relax_alpha_rows_k(const float* __restrict__ H, long long M, int n, const float4
             const float lo = (alpha != nullptr && unstable(p)) ? alpha[m * n + i] : p.x;
             const float r = (x >= 0.f) ? x * lo : x * p.y;
             cs = fmaf(fminf(x, 0.f), p.z, cs);
-            cs = fmaf(r, p.w, cs);
-            z[i] = r;
+            if (with_bias) cs = fmaf(r, p.w, cs);
+            z[i] = accumulate ? z[i] + r : r;
         }
         const float t = block_sum256(cs, red);
         if (threadIdx.x == 0) cst[m] += t;
@@ -136,9 +138,10 @@ __global__ void best_update_k(float* __restrict__ best, const float* __restrict_
 }  // namespace
 
 cudaError_t launch_relax_alpha_rows(const float* H, long long M, int n, const float4* P, PassGeom pg,
-                                    const float* alpha, float* Z, float* cst, cudaStream_t s) {
+                                    const float* alpha, float* Z, float* cst, cudaStream_t s, int with_bias,
+                                    int accumulate) {
     long long g = M < 148LL * 16 ? M : 148LL * 16;
-    relax_alpha_rows_k<<<(unsigned)(g < 1 ? 1 : g), 256, 0, s>>>(H, M, n, P, pg, alpha, Z, cst);
+    relax_alpha_rows_k<<<(unsigned)(g < 1 ? 1 : g), 256, 0, s>>>(H, M, n, P, pg, alpha, Z, cst, with_bias, accumulate);
     return cudaGetLastError();
 }
 

@@ -1025,6 +1025,174 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
     return VF_OK;
 }
 
+// alpha-CROWN on any node graph (residual adds included): the same computation as spec_alpha with every
+// node's coefficients materialised. Down: pending rows per node (the first contribution stores, later
+// ones add), affine nodes add their bias to the row constant, ReLUs apply per-row slopes and keep the
+// rows over their output for the gradient. Up, in topological order: G over each node's output from its
+// sources' G (affine: forward product plus bias; ReLU: the slope chain rule and the slope gradient /
+// Adam step; add: sum of the two sources).
+int spec_alpha_graph(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
+                     const vf_opts& o, int iters, float lr, bool grad_mode, const float* alpha_in, float* grad_out,
+                     float* lb, float* lb_start, float* alpha_out, cudaStream_t s) {
+    const int nn = (int)net->nodes.size();
+    const int L = nn - 1;
+    const long long n0 = net->nodes[0].n;
+    const int nL = (int)net->nodes[L].n;
+    if (net->nodes[L].op != VF_DENSE) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation needs a dense last node");
+    Arena ar{net->ws, net->ws_bytes};
+    IbpState st;
+    Bounds bd;
+    TRY(prepare_bounds(net, centres, B, eps, o, ar, st, bd, s));
+    std::vector<int> relus;
+    long long sum_relu = 0, sum_all = 0;
+    std::vector<long long> aoff(nn, 0);
+    int ctiles = 0;
+    for (int v = 0; v < nn; ++v) {
+        const Node& nd = net->nodes[v];
+        sum_all += nd.n;
+        if (nd.op == VF_RELU) {
+            relus.push_back(v);
+            aoff[v] = (long long)B * R * sum_relu;
+            sum_relu += nd.n;
+        }
+        if (nd.op == VF_CONV2D) ctiles = std::max(ctiles, conv_back_tiles(conv_geom(net, nd)));
+    }
+    const long long rows = (long long)B * R;
+    // per row: pending rows and gradients of every node, the per-ReLU slopes and Adam moments, constants
+    const size_t per_row = sizeof(float) * (2 * sum_all + (grad_mode ? 0 : 3 * sum_relu) + 2 + ctiles) +
+                           64 * (2 * nn + 3 * relus.size() + 8);
+    long long chunk = (long long)(ar.left() / per_row);
+    if (chunk > rows) chunk = rows;
+    if (chunk < 1) return fail(VF_ERR_WORKSPACE, "workspace too small for alpha optimisation");
+    std::vector<float*> P(nn, nullptr), G(nn, nullptr), A(nn, nullptr), M1(nn, nullptr), M2(nn, nullptr);
+    for (int v = 0; v < nn; ++v) {
+        P[v] = ar.take<float>((size_t)chunk * net->nodes[v].n);
+        G[v] = ar.take<float>((size_t)chunk * net->nodes[v].n);
+        if (!P[v] || !G[v]) return fail(VF_ERR_WORKSPACE, "workspace too small");
+    }
+    for (int u : relus)
+        if (!grad_mode) {
+            A[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+            M1[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+            M2[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+            if (!A[u] || !M1[u] || !M2[u]) return fail(VF_ERR_WORKSPACE, "workspace too small");
+        }
+    float* cst = ar.take<float>(chunk);
+    float* lbc = ar.take<float>(chunk);
+    float* cpart = ctiles ? ar.take<float>((size_t)chunk * ctiles) : nullptr;
+    if (!cst || !lbc || (ctiles && !cpart)) return fail(VF_ERR_WORKSPACE, "workspace too small");
+
+    for (long long m0 = 0; m0 < rows; m0 += chunk) {
+        const long long Mc = std::min(chunk, rows - m0);
+        const PassGeom pg{m0, R};
+        std::vector<float*> al(nn, nullptr);
+        for (int u : relus) {
+            const long long nu = net->nodes[u].n;
+            if (grad_mode) {
+                al[u] = const_cast<float*>(alpha_in) + aoff[u] + m0 * nu;
+            } else {
+                al[u] = A[u];
+                LAUNCH(net, launch_alpha_init(A[u], M1[u], M2[u], Mc, (int)nu, bd.relax[u], pg, s));
+            }
+        }
+        const int evals = grad_mode ? 1 : iters + 1;
+        for (int it = 0; it < evals; ++it) {
+            // ---- down: pending rows per node; written[v]: P[v] holds a first contribution
+            std::vector<char> written(nn, 0);
+            CU(cudaMemsetAsync(cst, 0, sizeof(float) * Mc, s));
+            const Node& last = net->nodes[L];
+            LAUNCH(net, launch_dense_back(RowRef{C, C_bstride, nL, R, m0}, Relax{nullptr, 0}, last.W, last.b, Mc, nL,
+                                          (int)net->nodes[last.src].n, pg, OUT_STORE, P[last.src],
+                                          net->nodes[last.src].n, cst, nullptr, 0.f, nullptr, s));
+            written[last.src] = 1;
+            for (int v = L - 1; v >= 1; --v) {
+                if (!written[v]) continue;
+                const Node& nd = net->nodes[v];
+                const int nv = (int)nd.n;
+                const RowRef rv{P[v], 0, nv, kHugeRows, 0};
+                auto mode_of = [&](int src) { return written[src] ? OUT_ACCUM : OUT_STORE; };
+                switch (nd.op) {
+                    case VF_DENSE: {
+                        const int ns = (int)net->nodes[nd.src].n;
+                        LAUNCH(net, launch_dense_back(rv, Relax{nullptr, 0}, nd.W, nd.b, Mc, nv, ns, pg, mode_of(nd.src),
+                                                      P[nd.src], ns, cst, nullptr, 0.f, nullptr, s));
+                        written[nd.src] = 1;
+                        break;
+                    }
+                    case VF_CONV2D: {
+                        const ConvGeom g = conv_geom(net, nd);
+                        LAUNCH(net, launch_conv_back(rv, Relax{nullptr, 0}, nd.W, nd.b, Mc, g, pg, mode_of(nd.src),
+                                                     P[nd.src], net->nodes[nd.src].n, cpart, nullptr, 0.f,
+                                                     net->num_sms, s));
+                        LAUNCH(net, launch_add_partials(cst, cpart, conv_back_tiles(g), Mc, s));
+                        written[nd.src] = 1;
+                        break;
+                    }
+                    case VF_RELU:
+                        LAUNCH(net, launch_relax_alpha_rows(P[v], Mc, nv, bd.relax[v], pg, al[v], P[nd.src], cst, s,
+                                                            0, written[nd.src] ? 1 : 0));
+                        written[nd.src] = 1;
+                        break;
+                    case VF_ADD:
+                        for (int src : {nd.src, nd.src2}) {
+                            LAUNCH(net, launch_relax_rows(rv, Relax{nullptr, 0}, Mc, nv, pg, P[src], nv,
+                                                          written[src] ? 1 : 0, nullptr, s));
+                            written[src] = 1;
+                        }
+                        break;
+                    default:
+                        return fail(VF_ERR_ARG, "bad node kind");
+                }
+            }
+            if (!written[0]) return fail(VF_ERR_ARG, "internal: the input was not reached");
+            LAUNCH(net, launch_concretize_grad(P[0], Mc, (int)n0, pg, centres, eps, cst, lbc, G[0], s));
+            if (it == 0 && lb_start) CU(cudaMemcpyAsync(lb_start + m0, lbc, sizeof(float) * Mc, cudaMemcpyDeviceToDevice, s));
+            LAUNCH(net, launch_best_update(lb + m0, lbc, Mc, it == 0 ? 1 : 0, s));
+            if (!grad_mode && it == iters) break;
+            // ---- up: gradient over every node's output, in topological order
+            for (int v = 1; v < L; ++v) {
+                const Node& nd = net->nodes[v];
+                const int nv = (int)nd.n;
+                switch (nd.op) {
+                    case VF_DENSE:
+                        LAUNCH(net, launch_rows_times_wt(G[nd.src], nd.W, nd.b, (int)Mc, (int)net->nodes[nd.src].n, nv,
+                                                         G[v], s));
+                        break;
+                    case VF_CONV2D:
+                        LAUNCH(net, launch_ibp_conv(G[nd.src], nullptr, nd.W, nd.Wabs, nd.b, (int)Mc, conv_geom(net, nd),
+                                                    G[v], nullptr, s));
+                        break;
+                    case VF_RELU: {
+                        CU(cudaMemcpyAsync(G[v], G[nd.src], sizeof(float) * Mc * nv, cudaMemcpyDeviceToDevice, s));
+                        float* gout = grad_mode ? grad_out + aoff[v] + m0 * nv : nullptr;
+                        if (written[v])
+                            LAUNCH(net, launch_relax_grad_adam(G[v], P[v], Mc, nv, bd.relax[v], pg, al[v], gout, M1[v],
+                                                               M2[v], grad_mode ? 0 : it + 1, lr, s));
+                        else if (gout != nullptr)  // not an ancestor of the last node: zero gradient
+                            CU(cudaMemsetAsync(gout, 0, sizeof(float) * Mc * nv, s));
+                        break;
+                    }
+                    case VF_ADD: {
+                        const RowRef r1{G[nd.src], 0, nv, kHugeRows, 0}, r2{G[nd.src2], 0, nv, kHugeRows, 0};
+                        LAUNCH(net, launch_relax_rows(r1, Relax{nullptr, 0}, Mc, nv, pg, G[v], nv, 0, nullptr, s));
+                        LAUNCH(net, launch_relax_rows(r2, Relax{nullptr, 0}, Mc, nv, pg, G[v], nv, 1, nullptr, s));
+                        break;
+                    }
+                    default:
+                        return fail(VF_ERR_ARG, "bad node kind");
+                }
+            }
+        }
+        if (!grad_mode && alpha_out)
+            for (int u : relus) {
+                const long long nu = net->nodes[u].n;
+                CU(cudaMemcpyAsync(alpha_out + aoff[u] + m0 * nu, A[u], sizeof(float) * Mc * nu,
+                                   cudaMemcpyDeviceToDevice, s));
+            }
+    }
+    return VF_OK;
+}
+
 }  // namespace
 
 int vf::set_last_error(int code, const char* msg) {
@@ -1407,9 +1575,11 @@ int vf_alpha_crown(vf_net* net, const float* centres, int B, float eps, const fl
     if (B < 0 || R < 0 || C_bstride < 0 || iters < 0) return fail(VF_ERR_ARG, "negative size");
     if (!std::isfinite(eps) || eps < 0.f || !std::isfinite(lr) || lr < 0.f)
         return fail(VF_ERR_NONFINITE, "eps and lr must be finite and >= 0");
-    if (!dense_chain(net)) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation needs a ReLU chain of dense/conv layers");
     if (o.both_sides) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation bounds the lower side; pass -C for upper");
     if (B == 0 || R == 0) return VF_OK;
+    if (!dense_chain(net))
+        return spec_alpha_graph(net, centres, B, eps, C, R, C_bstride, o, iters, lr, false, nullptr, nullptr, lb,
+                                lb_start, alpha_out, (cudaStream_t)stream);
     return spec_alpha(net, centres, B, eps, C, R, C_bstride, o, iters, lr, false, nullptr, nullptr, lb, lb_start,
                       alpha_out, (cudaStream_t)stream);
 }
@@ -1422,8 +1592,10 @@ int vf_alpha_grad(vf_net* net, const float* centres, int B, float eps, const flo
     if (!centres || !C || !lb || !alpha || !grad) return fail(VF_ERR_ARG, "NULL pointer");
     if (B < 0 || R < 0 || C_bstride < 0) return fail(VF_ERR_ARG, "negative size");
     if (!std::isfinite(eps) || eps < 0.f) return fail(VF_ERR_NONFINITE, "eps must be finite and >= 0");
-    if (!dense_chain(net)) return fail(VF_ERR_UNSUPPORTED, "alpha gradients need a ReLU chain of dense/conv layers");
     if (B == 0 || R == 0) return VF_OK;
+    if (!dense_chain(net))
+        return spec_alpha_graph(net, centres, B, eps, C, R, C_bstride, o, 0, 0.f, true, alpha, grad, lb, nullptr,
+                                nullptr, (cudaStream_t)stream);
     return spec_alpha(net, centres, B, eps, C, R, C_bstride, o, 0, 0.f, true, alpha, grad, lb, nullptr, nullptr,
                       (cudaStream_t)stream);
 }

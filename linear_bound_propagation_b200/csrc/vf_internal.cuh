@@ -196,7 +196,8 @@ cudaError_t launch_rows_times_wt(const float* A, const float* W, const float* bi
 
 // ---- alpha-CROWN (k_alpha.cu) -----------------------------------------------------------
 cudaError_t launch_relax_alpha_rows(const float* H, long long M, int n, const float4* P, PassGeom pg,
-                                    const float* alpha, float* Z, float* cst, cudaStream_t s);
+                                    const float* alpha, float* Z, float* cst, cudaStream_t s, int with_bias = 1,
+                                    int accumulate = 0);
 cudaError_t launch_concretize_grad(const float* lam, long long M, int n0, PassGeom pg, const float* centres, float eps,
                                    const float* cst, float* lb, float* G, cudaStream_t s);
 cudaError_t launch_relax_grad_adam(float* G, const float* H, long long M, int n, const float4* P, PassGeom pg,

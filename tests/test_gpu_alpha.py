@@ -88,12 +88,70 @@ def test_alpha_crown_improves_soundly_and_tracks_oracle(config, B):
     assert sound_on_samples(net, w.centres[:4], w.eps, w.C[:4] if w.C.shape[0] > 1 else w.C, lb[:4], None, n=2000)
 
 
-def test_alpha_rejects_non_chains():
-    rng = np.random.default_rng(7)
+def _small_residual(seed=7, B=2):
+    rng = np.random.default_rng(seed)
     net = synth.resnet_cfg4(rng, image=(3, 8, 8), widths=(3, 4, 5), fc=6, classes=4)
-    centres = rng.random((2, 3 * 8 * 8)).astype(np.float32)
-    C = synth.margin_spec(np.array([0, 1]), 4)
+    centres = rng.random((B, 3 * 8 * 8)).astype(np.float32)
+    C = synth.margin_spec(rng.integers(0, 4, B), 4)
+    return net, centres, C, 0.02
+
+
+def test_alpha_grad_matches_oracle_residual():
+    """The graph form of the slope gradient (residual adds, identity and 1x1-convolution shortcuts)."""
+    net, centres, C, eps = _small_residual()
+    B, R = centres.shape[0], C.shape[1]
     g = vf.Net(net)
-    with pytest.raises(vf.VfError) as e:
-        g.alpha_crown(_dev(centres), 0.01, _dev(C), iters=1)
-    assert e.value.code == vf.VF_ERR_UNSUPPORTED
+    rng = np.random.default_rng(9)
+    alpha = rng.random(g.alpha_size(B, R)).astype(np.float32)
+    lb, grad = g.alpha_grad(_dev(centres), eps, _dev(C), _dev(alpha))
+    torch.cuda.synchronize()
+    g.check()
+    lb, grad = lb.cpu().numpy(), grad.cpu().numpy()
+    res = O.verify(net, centres, eps, C)
+    amb = ambiguous_centres(res, net)
+    off, checked = 0, 0
+    blocks = {}
+    for k in g.relu_ids:
+        blocks[k] = (off, g.sizes[k])
+        off += B * R * g.sizes[k]
+    for b in range(B):
+        if amb[b]:
+            continue
+        relax = _oracle_relax(net, res, b)
+        a = {k: alpha[o + b * R * n: o + (b + 1) * R * n].reshape(R, n).astype(np.float64) for k, (o, n) in blocks.items()}
+        olb, og = O.spec_bound_alpha(net, centres[b], eps, C[b], relax, a)
+        assert _viol(lb[b], olb).max() <= 1.0, f"centre {b}"
+        for k, (o, n) in blocks.items():
+            gg = grad[o + b * R * n: o + (b + 1) * R * n].reshape(R, n)
+            assert _viol(gg, og[k]).max() <= 10.0, f"centre {b} relu {k}: {_viol(gg, og[k]).max()}"
+        checked += 1
+    assert checked >= 1
+
+
+def test_alpha_crown_residual_improves_soundly():
+    net, centres, C, eps = _small_residual(B=3)
+    g = vf.Net(net)
+    out = g.alpha_crown(_dev(centres), eps, _dev(C), iters=5, lr=0.1)
+    torch.cuda.synchronize()
+    g.check()
+    lb, lb0 = out["lb"].cpu().numpy(), out["lb_start"].cpu().numpy()
+    assert np.all(lb >= lb0)
+    res = O.verify(net, centres, eps, C)
+    ok = ~ambiguous_centres(res, net)
+    assert _viol(lb0[ok], res.lb_crown[ok]).max() <= 1.0
+    best, start = O.alpha_crown(net, centres, eps, C, iters=5, lr=0.1)
+    v = _viol(lb[ok], best[ok])
+    assert (v > 1.0).mean() <= 0.1, f"{(v > 1.0).mean():.3f} of rows off the oracle trajectory"
+    assert sound_on_samples(net, centres, eps, C, lb, None, n=2000)
+
+
+def test_alpha_rejects_both_sides():
+    w = synth.workload(2, B=2)
+    g = vf.Net(w.net)
+    o, keep = g._opts()
+    o.both_sides = 1
+    B, R = 2, w.C.shape[1]
+    lb = torch.empty(B, R, device="cuda")
+    code = vf.lib().vf_alpha_crown(g.h, vf._ptr(_dev(w.centres)), B, float(w.eps), vf._ptr(_dev(w.C)), R, 0,
+                                   vf.ctypes.byref(o), 1, 0.1, vf._ptr(lb), None, None, vf._stream_ptr())
+    assert code == vf.VF_ERR_UNSUPPORTED
