@@ -885,7 +885,7 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
 
 // A ReLU chain laid out input -> affine -> relu -> affine -> ... -> dense (nodes in that order), each
 // affine node dense or a convolution.
-bool dense_chain(const vf_net* net) {
+bool affine_chain(const vf_net* net) {
     const int nn = (int)net->nodes.size();
     for (int v = 1; v < nn; ++v) {
         const Node& nd = net->nodes[v];
@@ -1577,7 +1577,7 @@ int vf_alpha_crown(vf_net* net, const float* centres, int B, float eps, const fl
         return fail(VF_ERR_NONFINITE, "eps and lr must be finite and >= 0");
     if (o.both_sides) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation bounds the lower side; pass -C for upper");
     if (B == 0 || R == 0) return VF_OK;
-    if (!dense_chain(net))
+    if (!affine_chain(net))
         return spec_alpha_graph(net, centres, B, eps, C, R, C_bstride, o, iters, lr, false, nullptr, nullptr, lb,
                                 lb_start, alpha_out, (cudaStream_t)stream);
     return spec_alpha(net, centres, B, eps, C, R, C_bstride, o, iters, lr, false, nullptr, nullptr, lb, lb_start,
@@ -1593,7 +1593,7 @@ int vf_alpha_grad(vf_net* net, const float* centres, int B, float eps, const flo
     if (B < 0 || R < 0 || C_bstride < 0) return fail(VF_ERR_ARG, "negative size");
     if (!std::isfinite(eps) || eps < 0.f) return fail(VF_ERR_NONFINITE, "eps must be finite and >= 0");
     if (B == 0 || R == 0) return VF_OK;
-    if (!dense_chain(net))
+    if (!affine_chain(net))
         return spec_alpha_graph(net, centres, B, eps, C, R, C_bstride, o, 0, 0.f, true, alpha, grad, lb, nullptr,
                                 nullptr, (cudaStream_t)stream);
     return spec_alpha(net, centres, B, eps, C, R, C_bstride, o, 0, 0.f, true, alpha, grad, lb, nullptr, nullptr,
