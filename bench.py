@@ -189,7 +189,9 @@ def run_reference(args):
     if rank != 0:
         return
     w = synth.workload(args.config)
-    base, n, t = oracle_sample(w, args.cpu_sample_s)
+    # each step a bounded sample: about two minutes for the whole --warmup + --steps run (at least one centre)
+    per_step_s = min(args.cpu_sample_s, 120.0 / max(1, args.warmup + args.steps))
+    base, n, t = oracle_sample(w, per_step_s)
     R = w.C.shape[1] * (2 if w.both_sides else 1)
     import oracle.lbp as O
     times = []
