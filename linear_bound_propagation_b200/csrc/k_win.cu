@@ -598,6 +598,12 @@ bool conv_back_win_plan(const ConvGeom& g, const WinWeights& ww, const Win& wa, 
     return true;
 }
 
+bool conv_back_win_whole_map_fits(const ConvGeom& g, const WinWeights& ww, const Win& wa, const Win& wd) {
+    Win2Launch L;
+    int pm = 1;
+    return !ww.per_position && conv_back_win2_plan(g, ww, wa, wd, OUT_STORE, &L, &pm) && L.nwarps == 8 && L.w_all;
+}
+
 cudaError_t launch_conv_start_rows_win(float* out, long long ld, long long M, PassGeom pg, PassStart ps, const float* W,
                                        const ConvGeom& g, const Win& wd, int accumulate, cudaStream_t s) {
     if (M <= 0) return cudaSuccess;

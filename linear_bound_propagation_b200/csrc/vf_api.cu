@@ -94,7 +94,9 @@ struct vf_net {
     int* d_err = nullptr;   // device flag raised by a kernel whose bounded wait expired
     int tc_stall = 0;       // test hook: VF_TEST_TC_STALL=1 makes one tensor-core launch time out
     int windows = 1;        // receptive-field windows in passes that start at a convolution (VF_CONV_WINDOWS=0: off)
-    int conv_whole_warp = 0;  // whole-map rows through the one-warp-per-row kernel (VF_CONV_KERNEL=warp)
+    // whole-map rows through the one-warp-per-row windowed kernel: 0 never (VF_CONV_KERNEL=tile), 1 whenever
+    // its staging fits (VF_CONV_KERNEL=warp), 2 (default) when it fits with a full CTA and staged weights
+    int conv_whole_warp = 2;
     int conv_win_per_position = 0;  // windowed rows without position blocking (VF_CONV_WIN_KERNEL=1)
     int compact = 1;        // intermediate passes over IBP-unstable neurons only (VF_COMPACT=0: off)
     bool prof = false;
@@ -535,7 +537,9 @@ struct Walker {
                 }
                 WinLaunch wl;
                 if (!e.windowed && e.kind != E_IDENT && net->conv_whole_warp &&
-                    conv_back_win_plan(g, nd.ww, full_win(nd), &wl)) {  // whole-map rows as one full window
+                    conv_back_win_plan(g, nd.ww, full_win(nd), &wl) &&
+                    (net->conv_whole_warp == 1 ||
+                     conv_back_win_whole_map_fits(g, nd.ww, full_win(nd), full_win(sn)))) {  // rows as one full window
                     e.windowed = true;
                     e.win = full_win(nd);
                 }
@@ -1264,7 +1268,8 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
     if (const char* f = getenv("VF_DENSE_KERNEL")) net->dense_kernel = (strcmp(f, "ffma") == 0) ? 1 : 0;
     if (const char* f = getenv("VF_TEST_TC_STALL")) net->tc_stall = atoi(f) != 0;
     if (const char* f = getenv("VF_CONV_WINDOWS")) net->windows = atoi(f) != 0;
-    if (const char* f = getenv("VF_CONV_KERNEL")) net->conv_whole_warp = (strcmp(f, "warp") == 0) ? 1 : 0;
+    if (const char* f = getenv("VF_CONV_KERNEL"))
+        net->conv_whole_warp = (strcmp(f, "warp") == 0) ? 1 : (strcmp(f, "tile") == 0 ? 0 : 2);
     if (const char* f = getenv("VF_CONV_WIN_KERNEL")) net->conv_win_per_position = (strcmp(f, "1") == 0) ? 1 : 0;
     if (const char* f = getenv("VF_COMPACT")) net->compact = atoi(f) != 0;
     CU(cudaMalloc(&net->d_err, sizeof(int)));

@@ -130,6 +130,10 @@ cudaError_t launch_conv_back_win(const RowRef& A, Relax rx, const WinWeights& ww
 // the start node's shape.
 cudaError_t launch_ident_rows_win(float* out, long long ld, long long M, PassGeom pg, PassStart ps, const Win& wd,
                                   int accumulate, cudaStream_t s);
+// True when rows over the whole map (`wa` = the whole output map, `wd` = the whole input map) fit the
+// position-blocked windowed kernel with a full CTA of 8 rows and all weights in shared memory; such
+// convolutions run faster there than in the tiled whole-map kernel.
+bool conv_back_win_whole_map_fits(const ConvGeom& g, const WinWeights& ww, const Win& wa, const Win& wd);
 // Re-windowing of rows over one map of C x H x W: out (=, +=) relax(A) moved from window `wa` into `wd`
 // (which must contain `wa`); relaxation constants (rx.count_const) go to cst.
 cudaError_t launch_rewin_rows(const RowRef& A, Relax rx, long long M, int C, int H, int W, PassGeom pg, PassStart ps,

@@ -107,6 +107,23 @@ def _conv_flops(net, centres, eps, C, both):
     return fl, {k: v.cpu().numpy() for k, v in out.items()}
 
 
+@pytest.mark.parametrize("kernel", ["tile", "warp", "auto"])
+def test_whole_map_convolution_kernels(monkeypatch, kernel):
+    """Whole-map rows (windows off) through the tiled kernel, through the windowed kernel with the whole map as
+    the window, and the default choice between them: all match the oracle on a CNN and a residual net."""
+    monkeypatch.setenv("VF_CONV_WINDOWS", "0")
+    monkeypatch.setenv("VF_CONV_KERNEL", kernel)
+    w = synth.workload(3, B=2)
+    g, ora, out = run_both(w.net, w.centres, w.eps, w.C)
+    assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out)
+    rng = np.random.default_rng(45)
+    net = synth.resnet_cfg4(rng, image=(3, 16, 16), widths=(4, 5, 6), fc=10, classes=5)
+    centres = rng.random((2, 3 * 16 * 16)).astype(np.float32)
+    C = synth.margin_spec(rng.integers(0, 5, 2), 5)
+    g, ora, out = run_both(net, centres, 0.01, C, both=True)
+    assert_parity(net, centres, 0.01, C, g, ora, out, both=True)
+
+
 def test_window_kernels_on_mixed_geometries(monkeypatch):
     """Convolutions with 5x5 stride-1, 3x3 stride-2 and 4x4 stride-4 kernels: the stride/tap combinations
     without a position-blocked instance take the per-position windowed kernel, the others the blocked
