@@ -91,14 +91,20 @@ def start_clocks():
     try:
         f = open(path, "w")
         p = subprocess.Popen(["nvidia-smi", "-i", str(dev), f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                              "-lms", "200"], stdout=f, stderr=subprocess.DEVNULL)
-        return p, f, path
+                              "-lms", "20"], stdout=f, stderr=subprocess.DEVNULL)
+        # start timing only once the sampler is running, so that its samples fall inside the timed region
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and p.poll() is None and os.path.getsize(path) == 0:
+            time.sleep(0.01)
+        with open(path) as fh:
+            first = len(fh.readlines())
+        return p, f, path, first
     except Exception:
-        return None, None, path
+        return None, None, path, 0
 
 
 def stop_clocks(handle):
-    p, f, path = handle
+    p, f, path, first = handle
     if p is None:
         return None
     p.terminate()
@@ -110,18 +116,21 @@ def stop_clocks(handle):
     sm, mx, reasons = [], 0.0, set()
     names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
     with open(path) as fh:
-        for line in fh:
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = max(mx, float(parts[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
+        lines = fh.readlines()
+    if len(lines) > first:  # drop the samples taken before the timed region started
+        lines = lines[first:]
+    for line in lines:
+        parts = [x.strip() for x in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            mx = max(mx, float(parts[2]))
+        except ValueError:
+            continue
+        for nm, v in zip(names, parts[5:9]):
+            if v.lower().startswith("active"):
+                reasons.add(nm)
     os.unlink(path)
     if not sm:
         return None

@@ -34,6 +34,9 @@ __device__ __forceinline__ StartPos start_pos(const PassStart& ps, const PassGeo
     return s;
 }
 
+// n / d for 0 <= n < 2^22 and small d, exact: (n + 0.5) / d is at least 1/(2d) from an integer
+__device__ __forceinline__ int fdiv(int n, float inv) { return __float2int_rz(((float)n + 0.5f) * inv); }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -52,6 +55,8 @@ __global__ void __launch_bounds__(256)
 conv_start_rows_win_k(float* __restrict__ out, long long ld, long long M, PassGeom pg, PassStart ps,
                       const float* __restrict__ W, ConvGeom g, Win wd, int accumulate) {
     const int nwin = wd.C * wd.hh * wd.hw;
+    const int plane = wd.hh * wd.hw;
+    const float inv_plane = 1.f / (float)plane, inv_hw = 1.f / (float)wd.hw;
     const int lane = threadIdx.x & 31;
     for (long long m = blockIdx.x * 8LL + (threadIdx.x >> 5); m < M; m += (long long)gridDim.x * 8) {
         const StartPos sp = start_pos(ps, pg, m);
@@ -59,7 +64,9 @@ conv_start_rows_win_k(float* __restrict__ out, long long ld, long long M, PassGe
         const int fy = sp.yj * g.stride - g.pad, fx = sp.xj * g.stride - g.pad;
         float* o = out + m * ld;
         for (int e = lane; e < nwin; e += 32) {
-            const int dx = e % wd.hw, dy = (e / wd.hw) % wd.hh, ci = e / (wd.hw * wd.hh);
+            const int ci = fdiv(e, inv_plane);
+            const int r2 = e - ci * plane;
+            const int dy = fdiv(r2, inv_hw), dx = r2 - dy * wd.hw;
             const int y = oy + dy, x = ox + dx;
             const int p = y - fy, q = x - fx;
             float v = 0.f;
@@ -252,7 +259,6 @@ struct WinClasses {
     int ny[4], nx[4], G[4];
 };
 
-__device__ __forceinline__ int fdiv(int n, float inv) { return __float2int_rz(((float)n + 0.5f) * inv); }
 
 // a[i] for a small runtime i, by selects (keeps the parameter arrays out of local memory)
 template <int N>
