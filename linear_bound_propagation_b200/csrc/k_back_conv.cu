@@ -131,7 +131,10 @@ conv_back_ffma(RowRef A, Relax rx, const float* __restrict__ W, const float* __r
                 // Element indices are split with float reciprocals (exact for these small sizes).
                 const int nwin = cc * wh * ww;
                 const float inv_ww = 1.f / (float)ww, inv_wh = 1.f / (float)wh;
-                const bool shared_p = (rx.P != nullptr) && rowb[0] == rowb[RG - 1];
+                // the item's valid rows are consecutive, so they share a centre iff the first and the last
+                // valid row do (rows past M are padding and carry no centre)
+                const int nvalid = (int)((M - m0) < RG ? (M - m0) : RG);
+                const bool shared_p = (rx.P != nullptr) && rowb[0] == rowb[nvalid - 1];
                 if (shared_p) {
                     const float4* P0 = rx.P + rowb[0] * nOut;
                     for (int e = tid; e < nwin; e += kThreads) {

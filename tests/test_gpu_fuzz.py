@@ -1,0 +1,92 @@
+"""GPU parity on seeded random small networks: plain and residual CNNs with random kernel sizes, strides and
+paddings, dense heads, random radii and both bound sides. Each network exercises a different mix of the
+executor's paths (receptive-field windows and their merges at residual adds, whole-map rows, unstable-only
+compaction, tensor-core and FFMA contractions); every result is compared with the fp64 oracle."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.lbp as O
+from linear_bound_propagation_b200 import synth
+from tests._parity import ambiguous_centres, max_violation, sound_on_samples
+
+pytestmark = pytest.mark.gpu
+
+vf = pytest.importorskip("linear_bound_propagation_b200.vf")
+
+SEEDS = list(range(24))
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _out_hw(h, k, s, p):
+    return (h + 2 * p - k) // s + 1
+
+
+def random_net(seed):
+    """A random network of this library's node kinds; returns (net, input shape, classes)."""
+    rng = np.random.default_rng(10_000 + seed)
+    c, h = int(rng.integers(1, 4)), int(rng.integers(6, 13))
+    net = [synth.Node(synth.INPUT, shape=(c, h, h))]
+    v = 0
+    for _ in range(int(rng.integers(1, 4))):
+        if rng.random() < 0.35 and h >= 4:  # residual block: conv-relu-conv + shortcut, add, relu
+            co = int(rng.integers(1, 5))
+            s = int(rng.choice([1, 2]))
+            ho = _out_hw(h, 3, s, 1)
+            a = synth._relu(net, synth._conv(net, rng, v, c, co, 3, s, 1, 0.7))
+            b = synth._conv(net, rng, a, co, co, 3, 1, 1, 0.7)
+            sc = v if (s == 1 and co == c) else synth._conv(net, rng, v, c, co, 1, s, 0, 0.7)
+            net.append(synth.Node(synth.ADD, src=b, src2=sc))
+            v = synth._relu(net, len(net) - 1)
+            c, h = co, ho
+        else:
+            k = int(rng.integers(1, min(5, h) + 1))
+            s = int(rng.choice([1, 2])) if h > k else 1
+            p = int(rng.integers(0, k))
+            if _out_hw(h, k, s, p) < 1 or s * (_out_hw(h, k, s, p) - 1) > h - 1 + p:
+                p = 0
+            co = int(rng.integers(1, 6))
+            v = synth._relu(net, synth._conv(net, rng, v, c, co, k, s, p))
+            c, h = co, _out_hw(h, k, s, p)
+    hidden, classes = int(rng.integers(3, 12)), int(rng.integers(2, 6))
+    v = synth._relu(net, synth._dense(net, rng, v, c * h * h, hidden))
+    synth._dense(net, rng, v, hidden, classes)
+    return net, net[0].shape, classes
+
+
+@pytest.mark.parametrize("seed", SEEDS)
+def test_random_network_matches_oracle(seed):
+    net, shape, classes = random_net(seed)
+    rng = np.random.default_rng(20_000 + seed)
+    B = int(rng.integers(1, 4))
+    n0 = int(np.prod(shape))
+    centres = rng.random((B, n0)).astype(np.float32)
+    eps = float(np.float32(rng.choice([0.002, 0.01, 0.03])))
+    C = synth.margin_spec(rng.integers(0, classes, B), classes)
+    both = bool(rng.random() < 0.5)
+    ora = O.verify(net, centres, eps, C, both_sides=both)
+    g = vf.Net(net)
+    out = g.verify(_dev(centres), eps, _dev(C), both_sides=both, want_pre=True)
+    torch.cuda.synchronize()
+    g.check()
+    out = {k: v.cpu().numpy() for k, v in out.items()}
+    assert max_violation(out["lb_ibp"], ora.lb_ibp) <= 1.0
+    amb = ambiguous_centres(ora, net)
+    for b in range(B):
+        viol = max_violation(out["lb"][b], ora.lb[b])
+        if both:
+            viol = max(viol, max_violation(out["ub"][b], ora.ub[b]))
+        for k in [v for v, nd in enumerate(net) if nd.op == "relu"]:
+            p = net[k].src
+            gl = g.node_block(torch.from_numpy(out["pre_lb"]), p, B).numpy()[b]
+            gu = g.node_block(torch.from_numpy(out["pre_ub"]), p, B).numpy()[b]
+            viol = max(viol, max_violation(gl, ora.pre_bounds[k][0][b]), max_violation(gu, ora.pre_bounds[k][1][b]))
+        if viol > 1.0:
+            assert amb[b], f"seed {seed} centre {b}: violation {viol:.2f} without an adaptive-slope tie"
+            assert sound_on_samples(net, centres[b:b + 1], eps, C[b:b + 1], out["lb"][b:b + 1],
+                                    out["ub"][b:b + 1] if both else None)
