@@ -1,5 +1,6 @@
 """GPU parity on seeded random small networks: plain and residual CNNs with random kernel sizes, strides and
-paddings, dense heads, random radii and both bound sides. Each network exercises a different mix of the
+paddings, dense heads, and dense ReLU chains of random widths, with random batch sizes, radii, CROWN-refined
+layer subsets and bound sides. Each network exercises a different mix of the
 executor's paths (receptive-field windows and their merges at residual adds, whole-map rows, unstable-only
 compaction, tensor-core and FFMA contractions); every result is compared with the fp64 oracle."""
 from __future__ import annotations
@@ -82,6 +83,53 @@ def test_random_network_matches_oracle(seed):
         if both:
             viol = max(viol, max_violation(out["ub"][b], ora.ub[b]))
         for k in [v for v, nd in enumerate(net) if nd.op == "relu"]:
+            p = net[k].src
+            gl = g.node_block(torch.from_numpy(out["pre_lb"]), p, B).numpy()[b]
+            gu = g.node_block(torch.from_numpy(out["pre_ub"]), p, B).numpy()[b]
+            viol = max(viol, max_violation(gl, ora.pre_bounds[k][0][b]), max_violation(gu, ora.pre_bounds[k][1][b]))
+        if viol > 1.0:
+            assert amb[b], f"seed {seed} centre {b}: violation {viol:.2f} without an adaptive-slope tie"
+            assert sound_on_samples(net, centres[b:b + 1], eps, C[b:b + 1], out["lb"][b:b + 1],
+                                    out["ub"][b:b + 1] if both else None)
+
+
+def random_mlp(seed):
+    rng = np.random.default_rng(30_000 + seed)
+    widths = [int(rng.choice([5, 8, 13, 32, 48, 64, 100]))]
+    for _ in range(int(rng.integers(1, 5))):
+        widths.append(int(rng.choice([4, 7, 16, 32, 36, 64, 96, 128])))
+    widths.append(int(rng.integers(2, 8)))
+    return synth.mlp(widths, rng), widths
+
+
+@pytest.mark.parametrize("seed", list(range(16)))
+def test_random_mlp_matches_oracle(seed):
+    """Random dense ReLU chains (widths that do and do not meet the tensor-core shape rules), random batch
+    sizes that leave ragged tiles, random subsets of layers refined by CROWN (the rest keep IBP bounds)
+    and both bound sides."""
+    net, widths = random_mlp(seed)
+    rng = np.random.default_rng(40_000 + seed)
+    B = int(rng.integers(1, 41))
+    centres = rng.random((B, widths[0])).astype(np.float32)
+    eps = float(np.float32(rng.choice([0.005, 0.02, 0.08])))
+    classes = widths[-1]
+    C = synth.margin_spec(rng.integers(0, classes, B), classes)
+    both = bool(rng.random() < 0.5)
+    relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
+    crown = [v for v in relus if rng.random() < 0.7]
+    ora = O.verify(net, centres, eps, C, crown_relus=crown, both_sides=both)
+    g = vf.Net(net)
+    out = g.verify(_dev(centres), eps, _dev(C), crown_relus=crown, both_sides=both, want_pre=True)
+    torch.cuda.synchronize()
+    g.check()
+    out = {k: v.cpu().numpy() for k, v in out.items()}
+    assert max_violation(out["lb_ibp"], ora.lb_ibp) <= 1.0
+    amb = ambiguous_centres(ora, net)
+    for b in range(B):
+        viol = max_violation(out["lb"][b], ora.lb[b])
+        if both:
+            viol = max(viol, max_violation(out["ub"][b], ora.ub[b]))
+        for k in relus:
             p = net[k].src
             gl = g.node_block(torch.from_numpy(out["pre_lb"]), p, B).numpy()[b]
             gu = g.node_block(torch.from_numpy(out["pre_ub"]), p, B).numpy()[b]
