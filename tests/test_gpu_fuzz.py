@@ -47,7 +47,7 @@ def random_net(seed):
             c, h = co, ho
         else:
             k = int(rng.integers(1, min(5, h) + 1))
-            s = int(rng.choice([1, 2])) if h > k else 1
+            s = int(rng.choice([1, 2, 2, 4])) if h > k else 1
             p = int(rng.integers(0, k))
             if _out_hw(h, k, s, p) < 1 or s * (_out_hw(h, k, s, p) - 1) > h - 1 + p:
                 p = 0
@@ -138,3 +138,46 @@ def test_random_mlp_matches_oracle(seed):
             assert amb[b], f"seed {seed} centre {b}: violation {viol:.2f} without an adaptive-slope tie"
             assert sound_on_samples(net, centres[b:b + 1], eps, C[b:b + 1], out["lb"][b:b + 1],
                                     out["ub"][b:b + 1] if both else None)
+
+
+def _alpha_blocks(g, B, R):
+    off, blocks = 0, {}
+    for k in g.relu_ids:
+        blocks[k] = (off, g.sizes[k])
+        off += B * R * g.sizes[k]
+    return blocks
+
+
+@pytest.mark.parametrize("seed", list(range(12)))
+def test_random_alpha_gradient_matches_oracle(seed):
+    """alpha-CROWN bound and slope gradient at random slopes on random networks (CNN chains, residual
+    graphs and dense chains alike), against the oracle's reverse-mode gradient."""
+    net = random_net(seed)[0] if seed % 2 == 0 else random_mlp(seed)[0]
+    rng = np.random.default_rng(50_000 + seed)
+    B = int(rng.integers(1, 4))
+    n0 = int(np.prod(net[0].shape))
+    classes = int(net[-1].W.shape[0])
+    centres = rng.random((B, n0)).astype(np.float32)
+    eps = float(np.float32(rng.choice([0.005, 0.02])))
+    C = synth.margin_spec(rng.integers(0, classes, B), classes)
+    R = C.shape[1]
+    g = vf.Net(net)
+    alpha = rng.random(g.alpha_size(B, R)).astype(np.float32)
+    lb, grad = g.alpha_grad(_dev(centres), eps, _dev(C), _dev(alpha))
+    torch.cuda.synchronize()
+    g.check()
+    lb, grad = lb.cpu().numpy(), grad.cpu().numpy()
+    res = O.verify(net, centres, eps, C)
+    amb = ambiguous_centres(res, net)
+    blocks = _alpha_blocks(g, B, R)
+    for b in range(B):
+        if amb[b]:
+            continue
+        relax = {k: O.relax_params(res.pre_bounds[k][0][b], res.pre_bounds[k][1][b]) for k in g.relu_ids}
+        a = {k: alpha[o + b * R * n: o + (b + 1) * R * n].reshape(R, n).astype(np.float64) for k, (o, n) in blocks.items()}
+        olb, og = O.spec_bound_alpha(net, centres[b], eps, C[b], relax, a)
+        assert max_violation(lb[b], olb) <= 1.0, f"seed {seed} centre {b}"
+        for k, (o, n) in blocks.items():
+            gg = grad[o + b * R * n: o + (b + 1) * R * n].reshape(R, n)
+            v = np.abs(gg - og[k]) / (1e-4 * (np.abs(og[k]) + 1.0))
+            assert v.max() <= 10.0, f"seed {seed} centre {b} relu {k}: {v.max():.2f}"
