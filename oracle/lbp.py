@@ -129,14 +129,34 @@ def forward(net, x: np.ndarray) -> List[np.ndarray]:
 
 # ----------------------------------------------------------------------------- IBP
 
-def ibp(net, centres: np.ndarray, eps: float):
+def split_clamp(l: np.ndarray, u: np.ndarray, s: Optional[np.ndarray]):
+    """Pre-activation interval of ReLU neurons inside a branch-and-bound subdomain [SNNV §2.2, §3, §4.3:
+    complete verification by beta-CROWN with branch-and-bound; the page names the method only].
+
+    Reading: a split fixes the sign of one ReLU's pre-activation z_i on a subdomain of the input box.
+    s[i] = +1 is the subdomain where z_i >= 0 (its interval becomes [max(l, 0), u]); s[i] = -1 the one
+    where z_i <= 0 (interval [l, min(u, 0)]); 0 leaves the neuron free. Nothing else changes: bounds
+    computed over the whole box stay valid on any part of it. An interval left empty (l > u) means
+    the subdomain holds no input, so every bound on it is vacuously sound.
+    """
+    l = np.asarray(l, F)
+    u = np.asarray(u, F)
+    if s is None:
+        return l, u
+    s = np.asarray(s)
+    return np.where(s > 0, np.maximum(l, 0.0), l), np.where(s < 0, np.minimum(u, 0.0), u)
+
+
+def ibp(net, centres: np.ndarray, eps: float, splits: Optional[Dict[int, np.ndarray]] = None):
     """Interval bound propagation in centre/radius form [SNNV §2.1, §4.2].
 
     The input box is centre c, radius eps (no clipping to any data range: the page
     only speaks of "a specified domain" [SNNV §1]; the plain reading is the L-inf ball).
     Affine node: centre' = W c + b, radius' = |W| r (the exact image of a box under an
     affine map, coordinate-wise). ReLU: clamp both ends, then back to centre/radius.
-    Add: centres add, radii add.
+    Add: centres add, radii add. Under split constraints (relu node -> [B, n] signs, see
+    ``split_clamp``) a ReLU first clamps its input interval; a neuron split to z <= 0 outputs
+    exactly 0.
 
     Returns (centre, radius) lists over nodes, each [B, n_v] float64.
     """
@@ -158,8 +178,13 @@ def ibp(net, centres: np.ndarray, eps: float):
             c = (conv2d(ci, nd.W, nd.stride, nd.pad) + nd.b.astype(F)[None, :, None, None]).reshape(B, -1)
             r = conv2d(ri, np.abs(nd.W.astype(F)), nd.stride, nd.pad).reshape(B, -1)
         elif nd.op == "relu":
-            lo = np.maximum(cs[nd.src] - rs[nd.src], 0.0)
-            hi = np.maximum(cs[nd.src] + rs[nd.src], 0.0)
+            sp = None if splits is None else splits.get(v)
+            l, u = split_clamp(cs[nd.src] - rs[nd.src], cs[nd.src] + rs[nd.src], sp)
+            lo = np.maximum(l, 0.0)
+            hi = np.maximum(u, 0.0)
+            if sp is not None:
+                off = np.asarray(sp) < 0
+                lo, hi = np.where(off, 0.0, lo), np.where(off, 0.0, hi)
             c, r = (hi + lo) / 2.0, (hi - lo) / 2.0
         elif nd.op == "add":
             c, r = cs[nd.src] + cs[nd.src2], rs[nd.src] + rs[nd.src2]
@@ -301,7 +326,7 @@ def _first_affine_on_input(net, p: int) -> bool:
 
 def verify(net, centres, eps, C, crown_relus: Optional[Sequence[int]] = None,
            alphas: Optional[Dict[int, np.ndarray]] = None, both_sides: bool = False,
-           row_block: int = 4096) -> OracleResult:
+           row_block: int = 4096, splits: Optional[Dict[int, np.ndarray]] = None) -> OracleResult:
     """IBP, then CROWN intermediate bounds, then the specification pass and decision.
 
     Readings taken where the page is silent (it names the methods only, [SNNV §1, §2.1]):
@@ -319,7 +344,10 @@ def verify(net, centres, eps, C, crown_relus: Optional[Sequence[int]] = None,
         node's interval, C c - |C| r; the final lower bound is the larger (both are sound)
         and a row is verified iff it is > 0 [SNNV §1]. Upper bounds, when asked for,
         are -lower(-C) and C c + |C| r, the final one the smaller;
-      * alpha (relu node -> [B, n]) is shared by all rows and passes; missing = adaptive.
+      * alpha (relu node -> [B, n]) is shared by all rows and passes; missing = adaptive;
+      * splits (relu node -> [B, n] in {-1, 0, +1}): each centre's row is one subdomain; the IBP
+        pass and the IBP bounds of split neurons are clamped (``split_clamp``), which makes those
+        neurons IBP-stable, so they take no CROWN refinement and their relaxation is exact.
     """
     centres = np.asarray(centres, F)
     B = centres.shape[0]
@@ -327,13 +355,14 @@ def verify(net, centres, eps, C, crown_relus: Optional[Sequence[int]] = None,
     R = C.shape[1]
     sh = shapes(net)
     L = len(net) - 1
-    cs, rs = ibp(net, centres, eps)
+    cs, rs = ibp(net, centres, eps, splits)
     ibp_b = {v: (cs[v] - rs[v], cs[v] + rs[v]) for v in range(len(net))}
     relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
     crown_set = set(relus if crown_relus is None else crown_relus)
     alphas = alphas or {}
+    splits = splits or {}
 
-    pre = {k: (ibp_b[net[k].src][0].copy(), ibp_b[net[k].src][1].copy()) for k in relus}
+    pre = {k: tuple(x.copy() for x in split_clamp(*ibp_b[net[k].src], splits.get(k))) for k in relus}
     lb_cr = np.empty((B, R), F)
     ub_cr = np.empty((B, R), F) if both_sides else None
     for b in range(B):
@@ -383,13 +412,19 @@ def _dense_chain(net):
     return [v for v in range(len(net)) if net[v].op != "relu" and v > 0]
 
 
-def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows):
+def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows, split_signs=None, beta_rows=None):
     """Lower bounds of `rows` (R x n_L) over the box, with one lower slope per (row, unstable neuron)
     [SNNV §3, §4.3: per-neuron alpha tensors], and their gradients with respect to those slopes.
 
     relax: relu node -> (lo, up, t) vectors (the intermediate-bound relaxation); alpha_rows: relu node
     -> [R, n] slopes in [0, 1], used in place of `lo` for unstable neurons (0 < up < 1). Returns
     (lb [R], grads {relu node: [R, n]}, zero where the neuron is stable).
+
+    Split constraints (beta-CROWN [SNNV §2.2, §4.3], reading: the Lagrangian form of a split): on a
+    subdomain where s_i z_i >= 0 (split_signs: relu node -> [n] signs, 0 = free) the rows' function is
+    bounded below by itself minus beta_i s_i z_i for any beta_i >= 0 (beta_rows: relu node -> [R, n]), so
+    the coefficients over the ReLU's input z gain -beta_i s_i before the back-substitution goes on. With
+    beta_rows given the return is (lb, grads, beta_grads), d lb / d beta_i = -s_i G_z,i.
 
     Forward: the back-substitution of `backward` with row-specific lower slopes. Gradient: reverse
     mode through that chain (layer order from the input up): with G the gradient of lb with respect
@@ -430,7 +465,10 @@ def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows):
             slope = np.where(lam >= 0.0, lo_rows, up[None, :])
             const = const + np.minimum(lam, 0.0) @ t
             saved[v] = (lam, slope, unst)
-            put(nd.src, lam * slope)
+            lam_z = lam * slope
+            if beta_rows is not None and v in split_signs:
+                lam_z = lam_z - np.asarray(beta_rows[v], F) * np.asarray(split_signs[v], F)[None, :]
+            put(nd.src, lam_z)
         else:  # add: both branches receive the rows
             put(nd.src, lam)
             put(nd.src2, lam)
@@ -439,7 +477,7 @@ def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows):
     lb = lam_in @ c - F(eps) * np.abs(lam_in).sum(axis=1) + const
     # G[v]: gradient of lb with respect to the coefficients over node v's output, in topological order
     G = {0: c[None, :] - F(eps) * np.sign(lam_in)}
-    grads = {}
+    grads, bgrads = {}, {}
     for v in range(1, L + 1):
         nd = net[v]
         if nd.op == "dense":
@@ -451,38 +489,61 @@ def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows):
             Gz = G[nd.src]
             if v not in saved:  # not an ancestor of the last node: its slopes do not enter lb
                 grads[v] = np.zeros((R, _size(sh[v])), F)
+                bgrads[v] = np.zeros((R, _size(sh[v])), F)
                 G[v] = np.zeros_like(Gz)
                 continue
             lam_h, slope, unst = saved[v]
             t = relax[v][2]
             grads[v] = np.where(unst[None, :] & (lam_h >= 0.0), Gz * lam_h, 0.0)
+            sg = np.zeros(Gz.shape[1], F) if split_signs is None or v not in split_signs else \
+                np.asarray(split_signs[v], F)
+            bgrads[v] = -Gz * sg[None, :]
             G[v] = Gz * slope + np.where(lam_h < 0.0, t[None, :], 0.0)
         else:
             G[v] = G[nd.src] + G[nd.src2]
+    if beta_rows is not None:
+        return lb, grads, bgrads
     return lb, grads
 
 
-def alpha_crown(net, centres, eps, C, iters=10, lr=0.1, crown_relus=None, betas=(0.9, 0.999)):
+def alpha_crown(net, centres, eps, C, iters=10, lr=0.1, crown_relus=None, betas=(0.9, 0.999), splits=None):
     """Projected gradient ascent (Adam) on per-row lower slopes of the specification pass, starting
     from the adaptive slopes, keeping each row's best bound [SNNV §1 alpha-CROWN; §3 alpha tensors].
     Intermediate bounds are those of `verify` (adaptive slopes). Returns (best lb [B, R], lb at the
-    adaptive start [B, R])."""
-    res = verify(net, centres, eps, C, crown_relus=crown_relus)
+    adaptive start [B, R]).
+
+    With split constraints (relu node -> [B, n] signs) the multipliers beta of the split neurons
+    (beta-CROWN, see ``spec_bound_alpha``) are optimised together with the slopes: one per (row, split
+    neuron), starting at 0, the same Adam step, projected to beta >= 0."""
+    res = verify(net, centres, eps, C, crown_relus=crown_relus, splits=splits)
     B, R = res.lb.shape
     C = np.asarray(C, F)
     relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
     best = np.empty((B, R), F)
     start = np.empty((B, R), F)
     b1, b2 = betas
+
+    def adam(x, m1, m2, g, it):
+        m1 = b1 * m1 + (1 - b1) * g
+        m2 = b2 * m2 + (1 - b2) * g * g
+        mh = m1 / (1 - b1 ** (it + 1))
+        vh = m2 / (1 - b2 ** (it + 1))
+        return x + lr * mh / (np.sqrt(vh) + 1e-8), m1, m2
+
     for b in range(B):
         relax = {k: relax_params(res.pre_bounds[k][0][b], res.pre_bounds[k][1][b]) for k in relus}
         rows = C[b if C.shape[0] > 1 else 0]
         alpha = {k: np.repeat(relax[k][0][None, :], R, axis=0) for k in relus}
         m1 = {k: np.zeros_like(a) for k, a in alpha.items()}
         m2 = {k: np.zeros_like(a) for k, a in alpha.items()}
+        sg = None if not splits else {k: np.asarray(splits[k][b]) for k in relus if k in splits}
+        beta = None if sg is None else {k: np.zeros((R, len(sg[k])), F) for k in sg}
+        bm1 = None if sg is None else {k: np.zeros_like(x) for k, x in beta.items()}
+        bm2 = None if sg is None else {k: np.zeros_like(x) for k, x in beta.items()}
         best_b = None
         for it in range(iters + 1):
-            lb, g = spec_bound_alpha(net, centres[b], eps, rows, relax, alpha)
+            out = spec_bound_alpha(net, centres[b], eps, rows, relax, alpha, sg, beta)
+            lb, g = out[0], out[1]
             if it == 0:
                 start[b] = lb
                 best_b = lb.copy()
@@ -491,10 +552,122 @@ def alpha_crown(net, centres, eps, C, iters=10, lr=0.1, crown_relus=None, betas=
             if it == iters:
                 break
             for k in relus:
-                m1[k] = b1 * m1[k] + (1 - b1) * g[k]
-                m2[k] = b2 * m2[k] + (1 - b2) * g[k] * g[k]
-                mh = m1[k] / (1 - b1 ** (it + 1))
-                vh = m2[k] / (1 - b2 ** (it + 1))
-                alpha[k] = np.clip(alpha[k] + lr * mh / (np.sqrt(vh) + 1e-8), 0.0, 1.0)
+                a, m1[k], m2[k] = adam(alpha[k], m1[k], m2[k], g[k], it)
+                alpha[k] = np.clip(a, 0.0, 1.0)
+            if beta is not None:
+                for k in beta:
+                    gb = np.where(sg[k][None, :] != 0, out[2][k], 0.0)
+                    x, bm1[k], bm2[k] = adam(beta[k], bm1[k], bm2[k], gb, it)
+                    beta[k] = np.maximum(x, 0.0)
         best[b] = best_b
     return best, start
+
+
+# ----------------------------------------------------------------------------- branch and bound
+
+def branch_scores(l: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """Branching score of ReLU neurons from their pre-activation bounds (reading: the page names
+    branch-and-bound only [SNNV §3, §4.3]). An unstable neuron (l < 0 < u) scores the intercept of its
+    upper relaxation, -u l / (u - l), the widest vertical gap between the chord and the ReLU; a stable
+    one scores -inf and is never split."""
+    l = np.asarray(l, F)
+    u = np.asarray(u, F)
+    sc = np.full(l.shape, -np.inf)
+    un = (l < 0.0) & (u > 0.0)
+    sc[un] = -u[un] * l[un] / (u[un] - l[un])
+    return sc
+
+
+@dataclasses.dataclass
+class BabResult:
+    status: str       # "verified", "falsified" or "unknown"
+    domains: int      # subdomains whose bounds were computed, the whole box included
+    iterations: int   # batched evaluations after the whole box
+    max_depth: int    # most splits in one evaluated subdomain
+    lb: float         # lowest row bound over the subdomains still open at the end (+inf if none)
+
+
+def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_relus=None, iters: int = 20,
+        lr: float = 0.1) -> BabResult:
+    """Branch and bound over ReLU splits on top of ``verify`` [SNNV §2.2, §3, §4.3: beta-CROWN with
+    branch-and-bound for complete verification; the page names the method only].
+
+    Property: every row of C [R, n_L] is positive at every input of the box centre +- eps.
+    A subdomain's row bound is the larger of ``verify``'s bound and the best bound of ``alpha_crown``
+    (``iters`` Adam steps of size ``lr`` on the slopes and on the split multipliers beta).
+    Reading of the search (one plain best-first variant):
+      1. the centre is evaluated first; a row < 0 there is a counterexample ("falsified");
+      2. the whole box is bounded; if every row's lower bound is > 0 it is "verified";
+      3. otherwise the open subdomains are kept with their lowest row bound; each round takes the
+         (at most batch // 2) open subdomains with the lowest bound (ties: created first), splits each
+         on its highest-scoring neuron (``branch_scores`` over all ReLU layers, ties: first layer, then
+         lowest index) into z <= 0 and z >= 0 (in that order), and bounds all children together;
+      4. a child is closed when its bounds are contradictory (some l > u: it holds no input) or all its
+         rows are > 0; a child with no unstable neuron left and a row <= 0 cannot be split further and
+         ends the search ("unknown"), as does a spent budget of ``max_domains`` bounded subdomains;
+      5. no open subdomain left: "verified".
+    """
+    C = np.asarray(C, F)
+    centre = np.asarray(centre, F)
+    relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
+    sizes = [_size(shapes(net)[net[k].src]) for k in relus]
+    y = forward(net, centre[None, :])[-1][0] @ C.T
+    if np.any(y < 0.0):
+        return BabResult("falsified", 0, 0, 0, float(y.min()))
+
+    def evaluate(domains):
+        sp = {k: np.zeros((len(domains), n), np.int8) for k, n in zip(relus, sizes)}
+        for i, d in enumerate(domains):
+            for (k, j), sign in d.items():
+                sp[k][i, j] = sign
+        cen = np.repeat(centre[None, :], len(domains), axis=0)
+        res = verify(net, cen, eps, C[None], crown_relus=crown_relus, splits=sp)
+        lb = res.lb
+        if iters > 0:
+            lb = np.maximum(lb, alpha_crown(net, cen, eps, C[None], iters=iters, lr=lr, crown_relus=crown_relus,
+                                            splits=sp)[0])
+        out = []
+        for i in range(len(domains)):
+            empty = any(np.any(res.pre_bounds[k][0][i] > res.pre_bounds[k][1][i]) for k in relus)
+            best, choice = -np.inf, None
+            for k in relus:
+                sc = branch_scores(res.pre_bounds[k][0][i], res.pre_bounds[k][1][i])
+                j = int(np.argmax(sc))
+                if sc[j] > best:
+                    best, choice = sc[j], (k, j)
+            out.append((float(lb[i].min()), empty, choice))
+        return out
+
+    (lb0, _, choice0), = evaluate([{}])
+    if lb0 > 0.0:
+        return BabResult("verified", 1, 0, 0, np.inf)
+    if choice0 is None:
+        return BabResult("unknown", 1, 0, 0, lb0)
+    open_ = [(lb0, 0, {}, choice0)]  # (lowest row bound, creation number, splits, branching neuron)
+    domains, iters, depth, seq = 1, 0, 0, 1
+    while open_:
+        take = min(len(open_), batch // 2, (max_domains - domains) // 2)
+        if take <= 0:
+            break
+        open_.sort(key=lambda d: (d[0], d[1]))
+        parents, open_ = open_[:take], open_[take:]
+        children = []
+        for _, _, sp, nb in parents:
+            for sign in (-1, 1):
+                d = dict(sp)
+                d[nb] = sign
+                children.append(d)
+        results = evaluate(children)
+        domains += len(children)
+        iters += 1
+        for d, (lbd, empty, nb) in zip(children, results):
+            depth = max(depth, len(d))
+            num, seq = seq, seq + 1
+            if empty or lbd > 0.0:
+                continue
+            if nb is None:
+                return BabResult("unknown", domains, iters, depth, lbd)
+            open_.append((lbd, num, d, nb))
+    if not open_:
+        return BabResult("verified", domains, iters, depth, np.inf)
+    return BabResult("unknown", domains, iters, depth, min(d[0] for d in open_))
