@@ -82,6 +82,9 @@ void vf_net_destroy(vf_net* net);
 int vf_net_node_size(const vf_net* net, int v);
 /* Sum of vf_net_node_size over all nodes: the row length of vf_ibp's bound arrays per centre block. */
 long long vf_net_total_size(const vf_net* net);
+/* Kind (VF_DENSE, ...), sources and size of node v; any output pointer may be NULL. VF_ERR_ARG if v is
+ * out of range. */
+int vf_net_node_info(const vf_net* net, int v, int* op, int* src, int* src2, long long* n);
 
 /* IBP pass (technical summary, section 2.1: the cheap, sound interval substitute).
  * Box: centres[b] +/- eps (no clipping). For every node v, writes its interval bounds
@@ -127,6 +130,15 @@ typedef struct {
     /* 1: the call never synchronises `stream` (no NaN/Inf scan, no unstable-neuron compaction;
      * the bounds are the same numbers), so it can be captured in a CUDA graph. */
     int no_host_sync;
+    /* [host] n_nodes entries of [device] [B, n_v] signs, or NULL: branch-and-bound split constraints
+     * (technical summary, sections 2.2 and 4.3: beta-CROWN with branch-and-bound). Each centre row b is
+     * one subdomain of its box; for ReLU node v, +1 restricts it to the inputs where the ReLU's input
+     * z_i >= 0, -1 to those where z_i <= 0, 0 leaves neuron i free. The IBP interval of a split neuron
+     * is clamped to its sign (z >= 0: l = max(l, 0); z <= 0: u = min(u, 0), and the ReLU outputs 0),
+     * which makes it stable, so its relaxation is exact on the subdomain. Every bound is then valid on
+     * the subdomain only. A subdomain that holds no input shows up as some pre_lb > pre_ub.
+     * vf_alpha_crown also optimises the split multipliers beta (see vf_alpha_beta_grad). */
+    const signed char* const* split;
 } vf_opts;
 
 /* Whole verification step (section 1): IBP, CROWN intermediate bounds, specification
@@ -165,6 +177,53 @@ int vf_alpha_crown(vf_net* net, const float* centres, int B, float eps, const fl
  * ReLU output is negative). Same networks and options as vf_alpha_crown. */
 int vf_alpha_grad(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
                   const vf_opts* opts, const float* alpha, float* lb, float* grad, void* stream);
+
+/* vf_alpha_grad with split constraints (opts->split) and their multipliers (beta-CROWN, technical summary
+ * sections 2.2 and 4.3; the Lagrangian reading): on a subdomain where s_i z_i >= 0, the bound of a row may
+ * subtract beta_i s_i z_i for any beta_i >= 0, so the row's coefficient over z_i gains -beta_i s_i when
+ * the back-substitution passes the ReLU. beta [device] and grad_beta [device] have alpha's layout (one
+ * [B, R, n_v] block per ReLU node v); entries of free neurons are ignored (beta) and zero (grad_beta):
+ * d lb / d beta_i = -s_i * (d lb / d coefficient over z_i). beta = NULL means all zero; grad_beta may be
+ * NULL. vf_alpha_crown starts beta at 0 and takes the slopes' Adam step on it, projected to beta >= 0. */
+int vf_alpha_beta_grad(vf_net* net, const float* centres, int B, float eps, const float* C, int R,
+                       long long C_bstride, const vf_opts* opts, const float* alpha, const float* beta, float* lb,
+                       float* grad_alpha, float* grad_beta, void* stream);
+
+/* Branch and bound over ReLU splits for one property (technical summary, sections 2.2, 3 and 4.3:
+ * complete verification by beta-CROWN with branch-and-bound; the page names the method only). The
+ * property: every row of C [device] [R, n_L] is positive at every input of the box centre [device] [n0]
+ * +/- eps. The search, run on the host with every bound computed on the device:
+ *   1. a row < 0 at the centre itself is a counterexample (VF_BAB_FALSIFIED);
+ *   2. a subdomain's row bound is the larger of vf_verify_batch's and vf_alpha_crown's (alpha_iters Adam
+ *      steps of size lr on the slopes and the split multipliers); the whole box is bounded first;
+ *   3. each round takes the open subdomains with the lowest bound (ties: created first), at most
+ *      batch / 2 of them, splits each on its neuron with the largest upper-relaxation intercept
+ *      -u l / (u - l) over all ReLU layers (ties: first layer, lowest index) into z <= 0 and z >= 0, and
+ *      bounds all children in one batch;
+ *   4. a child closes when some pre-activation bound has l > u (it holds no input) or all its rows are
+ *      > 0; a child with no unstable neuron left and a row <= 0 ends the search (VF_BAB_UNKNOWN), as does
+ *      a spent budget of max_domains bounded subdomains;
+ *   5. no open subdomain: VF_BAB_VERIFIED.
+ * The call synchronises `stream` once per round. It allocates its own device buffers for the round
+ * (batch subdomains) and uses the handle's workspace for the bounds. */
+enum { VF_BAB_FALSIFIED = -1, VF_BAB_UNKNOWN = 0, VF_BAB_VERIFIED = 1 };
+typedef struct {
+    int max_domains;        /* budget of bounded subdomains, the whole box included (>= 1) */
+    int batch;              /* subdomains bounded per round (even, >= 2) */
+    int alpha_iters;        /* Adam steps per bound (0: vf_verify_batch's bound alone) */
+    float lr;               /* Adam step size */
+    const int* relu_crown;  /* as vf_opts.relu_crown */
+} vf_bab_opts;
+typedef struct {
+    int status;             /* VF_BAB_VERIFIED, VF_BAB_FALSIFIED or VF_BAB_UNKNOWN */
+    long long domains;      /* subdomains bounded, the whole box included (0 when falsified at the centre) */
+    int rounds;             /* batched rounds after the whole box */
+    int max_depth;          /* most splits in one bounded subdomain */
+    float lb;               /* lowest row bound of the subdomains open at the end (+inf if none); when
+                               falsified, the lowest row value at the centre */
+} vf_bab_result;
+int vf_bab_verify(vf_net* net, const float* centre, float eps, const float* C, int R, const vf_bab_opts* opts,
+                  vf_bab_result* result /*[host]*/, void* stream);
 
 /* Synchronise `stream` and report any pending asynchronous CUDA error. */
 int vf_sync(void* stream);

@@ -11,6 +11,10 @@
 // the other direction: at the input G = c - eps * sign(lam_in); through a dense node G_z = G_h W^T + b;
 // at a ReLU d lb / d alpha_i = G_z,i * lam_h,i for lam_h,i >= 0 (unstable i), and
 // G_h = G_z * slope + [lam_h < 0] * t.
+//
+// Split constraints (beta-CROWN with branch-and-bound, same page §2.2 and §4.3): on a subdomain where
+// s_i z_i >= 0, lb may add -beta_i s_i z_i for any beta_i >= 0, so lam_z gains -beta_i s_i at the ReLU;
+// d lb / d beta_i = -s_i G_z,i, and beta takes the same Adam step, projected to beta >= 0.
 #include <math.h>
 
 #include "vf_internal.cuh"
@@ -45,7 +49,7 @@ __device__ __forceinline__ float block_sum256(float v, float* red) {
 __global__ void __launch_bounds__(256)
 relax_alpha_rows_k(const float* __restrict__ H, long long M, int n, const float4* __restrict__ P, PassGeom pg,
                    const float* __restrict__ alpha, float* __restrict__ Z, float* __restrict__ cst, int with_bias,
-                   int accumulate) {
+                   int accumulate, const signed char* __restrict__ split, const float* __restrict__ beta) {
     __shared__ float red[8];
     for (long long m = blockIdx.x; m < M; m += gridDim.x) {
         const long long b = (pg.pass_m0 + m) / pg.R_pass;
@@ -56,7 +60,11 @@ relax_alpha_rows_k(const float* __restrict__ H, long long M, int n, const float4
             const float x = h[i];
             const float4 p = P[b * n + i];
             const float lo = (alpha != nullptr && unstable(p)) ? alpha[m * n + i] : p.x;
-            const float r = (x >= 0.f) ? x * lo : x * p.y;
+            float r = (x >= 0.f) ? x * lo : x * p.y;
+            if (beta != nullptr) {
+                const signed char sg = split[b * n + i];
+                if (sg != 0) r -= (float)sg * beta[m * n + i];
+            }
             cs = fmaf(fminf(x, 0.f), p.z, cs);
             if (with_bias) cs = fmaf(r, p.w, cs);
             z[i] = accumulate ? z[i] + r : r;
@@ -89,16 +97,25 @@ concretize_grad_k(const float* __restrict__ lam, long long M, int n0, PassGeom p
 // Through one ReLU of the chain, in place: g = d lb / d alpha (unstable, lam_h >= 0), then
 // G <- G * slope + [H < 0] * t (slope from the current alpha), then (adam_step > 0) one Adam ascent step
 // on alpha, projected to [0, 1]. grad_out (optional) receives g.
+__device__ __forceinline__ float adam_ascent(float x, float g, float* m1, float* m2, float lr, float c1, float c2) {
+    const float v1 = 0.9f * *m1 + 0.1f * g;
+    const float v2 = 0.999f * *m2 + 0.001f * g * g;
+    *m1 = v1;
+    *m2 = v2;
+    return x + lr * (v1 * c1) / (sqrtf(v2 * c2) + 1e-8f);
+}
+
 __global__ void relax_grad_adam_k(float* __restrict__ G, const float* __restrict__ H, long long M, int n,
                                   const float4* __restrict__ P, PassGeom pg, float* __restrict__ alpha,
                                   float* __restrict__ grad_out, float* __restrict__ m1, float* __restrict__ m2,
-                                  int adam_step, float lr, float c1, float c2) {
+                                  int adam_step, float lr, float c1, float c2, BetaRows bt) {
     const long long total = M * n;
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
          e += (long long)gridDim.x * blockDim.x) {
         const long long m = e / n;
         const int i = (int)(e % n);
-        const float4 p = P[((pg.pass_m0 + m) / pg.R_pass) * n + i];
+        const long long bi = ((pg.pass_m0 + m) / pg.R_pass) * n + i;
+        const float4 p = P[bi];
         const bool un = unstable(p);
         const float x = H[e];
         const float a = (alpha != nullptr && un) ? alpha[e] : p.x;
@@ -106,14 +123,24 @@ __global__ void relax_grad_adam_k(float* __restrict__ G, const float* __restrict
         const float g = (un && x >= 0.f) ? gz * x : 0.f;
         G[e] = gz * ((x >= 0.f) ? a : p.y) + ((x < 0.f) ? p.z : 0.f);
         if (grad_out != nullptr) grad_out[e] = g;
-        if (adam_step > 0 && un && alpha != nullptr) {
-            const float v1 = 0.9f * m1[e] + 0.1f * g;
-            const float v2 = 0.999f * m2[e] + 0.001f * g * g;
-            m1[e] = v1;
-            m2[e] = v2;
-            const float step = lr * (v1 * c1) / (sqrtf(v2 * c2) + 1e-8f);
-            alpha[e] = fminf(fmaxf(a + step, 0.f), 1.f);
+        if (adam_step > 0 && un && alpha != nullptr)
+            alpha[e] = fminf(fmaxf(adam_ascent(a, g, &m1[e], &m2[e], lr, c1, c2), 0.f), 1.f);
+        if (bt.split != nullptr) {
+            const signed char sg = bt.split[bi];
+            const float gb = (sg != 0) ? -(float)sg * gz : 0.f;
+            if (bt.grad_out != nullptr) bt.grad_out[e] = gb;
+            if (adam_step > 0 && sg != 0 && bt.beta != nullptr)
+                bt.beta[e] = fmaxf(adam_ascent(bt.beta[e], gb, &bt.m1[e], &bt.m2[e], lr, c1, c2), 0.f);
         }
+    }
+}
+
+__global__ void zero3_k(float* __restrict__ a, float* __restrict__ b, float* __restrict__ c, long long count) {
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < count;
+         e += (long long)gridDim.x * blockDim.x) {
+        a[e] = 0.f;
+        b[e] = 0.f;
+        c[e] = 0.f;
     }
 }
 
@@ -139,9 +166,10 @@ __global__ void best_update_k(float* __restrict__ best, const float* __restrict_
 
 cudaError_t launch_relax_alpha_rows(const float* H, long long M, int n, const float4* P, PassGeom pg,
                                     const float* alpha, float* Z, float* cst, cudaStream_t s, int with_bias,
-                                    int accumulate) {
+                                    int accumulate, BetaRows bt) {
     long long g = M < 148LL * 16 ? M : 148LL * 16;
-    relax_alpha_rows_k<<<(unsigned)(g < 1 ? 1 : g), 256, 0, s>>>(H, M, n, P, pg, alpha, Z, cst, with_bias, accumulate);
+    relax_alpha_rows_k<<<(unsigned)(g < 1 ? 1 : g), 256, 0, s>>>(H, M, n, P, pg, alpha, Z, cst, with_bias, accumulate,
+                                                                 bt.split, bt.split != nullptr ? bt.beta : nullptr);
     return cudaGetLastError();
 }
 
@@ -155,14 +183,19 @@ cudaError_t launch_concretize_grad(const float* lam, long long M, int n0, PassGe
 
 cudaError_t launch_relax_grad_adam(float* G, const float* H, long long M, int n, const float4* P, PassGeom pg,
                                    float* alpha, float* grad_out, float* m1, float* m2, int adam_step, float lr,
-                                   cudaStream_t s) {
+                                   cudaStream_t s, BetaRows bt) {
     float c1 = 1.f, c2 = 1.f;
     if (adam_step > 0) {
         c1 = 1.f / (1.f - powf(0.9f, (float)adam_step));
         c2 = 1.f / (1.f - powf(0.999f, (float)adam_step));
     }
     relax_grad_adam_k<<<grid_for(M * n, 256), 256, 0, s>>>(G, H, M, n, P, pg, alpha, grad_out, m1, m2, adam_step, lr,
-                                                            c1, c2);
+                                                            c1, c2, bt);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_zero_moments(float* beta, float* m1, float* m2, long long count, cudaStream_t s) {
+    zero3_k<<<grid_for(count, 256), 256, 0, s>>>(beta, m1, m2, count);
     return cudaGetLastError();
 }
 

@@ -7,6 +7,8 @@
 //   affine:  centre' = W c + b,   radius' = |W| r     (both products in one pass)
 //   ReLU:    [max(c - r, 0), max(c + r, 0)] back to centre/radius
 //   add:     centres add, radii add
+//   splits:  branch-and-bound subdomains fix the sign of some pre-activations (same page, §2.2 and
+//            §4.3: beta-CROWN with branch-and-bound); their intervals are clamped to that sign
 #include "vf_internal.cuh"
 
 namespace vf {
@@ -126,11 +128,14 @@ __global__ void ibp_conv_k(const float* __restrict__ hc, const float* __restrict
     }
 }
 
-__global__ void ibp_relu_k(const float* __restrict__ c, const float* __restrict__ r, long long n, float* __restrict__ oc,
-                           float* __restrict__ orad) {
+// ReLU of an interval. Under split constraints (split != nullptr, one sign per neuron): a neuron split
+// to z <= 0 outputs exactly 0; one split to z >= 0 keeps [max(l, 0), max(u, 0)], the plain result.
+__global__ void ibp_relu_k(const float* __restrict__ c, const float* __restrict__ r, long long n,
+                           const signed char* __restrict__ split, float* __restrict__ oc, float* __restrict__ orad) {
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-        const float lo = fmaxf(c[i] - r[i], 0.f);
-        const float hi = fmaxf(c[i] + r[i], 0.f);
+        float lo = fmaxf(c[i] - r[i], 0.f);
+        float hi = fmaxf(c[i] + r[i], 0.f);
+        if (split != nullptr && split[i] < 0) lo = hi = 0.f;
         oc[i] = 0.5f * (hi + lo);
         orad[i] = 0.5f * (hi - lo);
     }
@@ -149,11 +154,19 @@ __global__ void fill_k(float* __restrict__ p, long long n, float v) {
         p[i] = v;
 }
 
-__global__ void bounds_k(const float* __restrict__ c, const float* __restrict__ r, long long n, float* __restrict__ lb,
-                         float* __restrict__ ub) {
+// l = c - r, u = c + r; under split constraints a neuron split to z >= 0 takes l = max(l, 0) and one
+// split to z <= 0 takes u = min(u, 0) (an empty interval marks a subdomain with no input).
+__global__ void bounds_k(const float* __restrict__ c, const float* __restrict__ r, long long n,
+                         const signed char* __restrict__ split, float* __restrict__ lb, float* __restrict__ ub) {
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-        lb[i] = c[i] - r[i];
-        ub[i] = c[i] + r[i];
+        float l = c[i] - r[i], u = c[i] + r[i];
+        if (split != nullptr) {
+            const signed char sg = split[i];
+            if (sg > 0) l = fmaxf(l, 0.f);
+            if (sg < 0) u = fminf(u, 0.f);
+        }
+        lb[i] = l;
+        ub[i] = u;
     }
 }
 
@@ -187,8 +200,9 @@ cudaError_t launch_ibp_conv(const float* hc, const float* hr, const float* W, co
     return cudaGetLastError();
 }
 
-cudaError_t launch_ibp_relu(const float* c, const float* r, long long n, float* oc, float* orad, cudaStream_t s) {
-    ibp_relu_k<<<grid_for(n, 256), 256, 0, s>>>(c, r, n, oc, orad);
+cudaError_t launch_ibp_relu(const float* c, const float* r, long long n, float* oc, float* orad, cudaStream_t s,
+                            const signed char* split) {
+    ibp_relu_k<<<grid_for(n, 256), 256, 0, s>>>(c, r, n, split, oc, orad);
     return cudaGetLastError();
 }
 
@@ -203,8 +217,9 @@ cudaError_t launch_fill(float* p, long long n, float v, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_bounds_from_cr(const float* c, const float* r, long long n, float* lb, float* ub, cudaStream_t s) {
-    bounds_k<<<grid_for(n, 256), 256, 0, s>>>(c, r, n, lb, ub);
+cudaError_t launch_bounds_from_cr(const float* c, const float* r, long long n, float* lb, float* ub, cudaStream_t s,
+                                  const signed char* split) {
+    bounds_k<<<grid_for(n, 256), 256, 0, s>>>(c, r, n, split, lb, ub);
     return cudaGetLastError();
 }
 

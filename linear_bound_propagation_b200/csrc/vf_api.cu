@@ -653,7 +653,8 @@ struct IbpState {
     std::vector<float*> c, r;
 };
 
-int run_ibp(vf_net* net, const float* centres, int B, float eps, Arena& ar, IbpState& st, cudaStream_t s) {
+int run_ibp(vf_net* net, const float* centres, int B, float eps, Arena& ar, IbpState& st, cudaStream_t s,
+            const signed char* const* split = nullptr) {
     const size_t N = net->nodes.size();
     st.c.assign(N, nullptr);
     st.r.assign(N, nullptr);
@@ -681,7 +682,7 @@ int run_ibp(vf_net* net, const float* centres, int B, float eps, Arena& ar, IbpS
                                             st.r[v], s));
                 break;
             case VF_RELU:
-                LAUNCH(net, launch_ibp_relu(st.c[sv], st.r[sv], cnt, st.c[v], st.r[v], s));
+                LAUNCH(net, launch_ibp_relu(st.c[sv], st.r[sv], cnt, st.c[v], st.r[v], s, split ? split[v] : nullptr));
                 break;
             case VF_ADD:
                 LAUNCH(net, launch_ibp_add(st.c[sv], st.r[sv], st.c[nd.src2], st.r[nd.src2], cnt, st.c[v], st.r[v], s));
@@ -799,7 +800,7 @@ struct Bounds {
 int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf_opts& o, Arena& ar, IbpState& st,
                    Bounds& bd, cudaStream_t s, const int* finite_flag = nullptr) {
     const int nn = (int)net->nodes.size();
-    TRY(run_ibp(net, centres, B, eps, ar, st, s));
+    TRY(run_ibp(net, centres, B, eps, ar, st, s, o.split));
     bd.Lw.assign(nn, nullptr);
     bd.Uw.assign(nn, nullptr);
     for (int v = 0; v < nn; ++v) {
@@ -809,7 +810,7 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
         bd.Lw[p] = ar.take<float>(cnt);
         bd.Uw[p] = ar.take<float>(cnt);
         if (!bd.Lw[p] || !bd.Uw[p]) return fail(VF_ERR_WORKSPACE, "workspace too small for intermediate bounds");
-        LAUNCH(net, launch_bounds_from_cr(st.c[p], st.r[p], cnt, bd.Lw[p], bd.Uw[p], s));
+        LAUNCH(net, launch_bounds_from_cr(st.c[p], st.r[p], cnt, bd.Lw[p], bd.Uw[p], s, o.split ? o.split[v] : nullptr));
     }
     bd.relax.assign(nn, nullptr);
     std::vector<float4*> P(nn, nullptr);
@@ -906,7 +907,8 @@ bool affine_chain(const vf_net* net) {
 // Slope arrays: for each ReLU node in order, a [B, R, n] block.
 int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
                const vf_opts& o, int iters, float lr, bool grad_mode, const float* alpha_in, float* grad_out,
-               float* lb, float* lb_start, float* alpha_out, cudaStream_t s) {
+               float* lb, float* lb_start, float* alpha_out, cudaStream_t s, const float* beta_in = nullptr,
+               float* beta_grad_out = nullptr) {
     const int nn = (int)net->nodes.size();
     const int L = nn - 1;
     const long long n0 = net->nodes[0].n;
@@ -931,19 +933,29 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
     int ctiles_max = 0;
     for (int v = 1; v < L; v += 2)
         if (net->nodes[v].op == VF_CONV2D) ctiles_max = std::max(ctiles_max, conv_back_tiles(conv_geom(net, net->nodes[v])));
+    long long sum_split = 0;  // neurons of ReLUs with split constraints (their beta rows)
+    for (int u : relus)
+        if (o.split && o.split[u]) sum_split += net->nodes[u].n;
     const size_t per_row =
-        sizeof(float) * (sum_n + nmax + n0 + 2 * gmax + 2 + ctiles_max + (grad_mode ? 0 : 3 * sum_n)) +
-        64 * (relus.size() + 8);
+        sizeof(float) * (sum_n + nmax + n0 + 2 * gmax + 2 + ctiles_max + (grad_mode ? 0 : 3 * (sum_n + sum_split))) +
+        64 * (2 * relus.size() + 8);
     long long chunk = (long long)(ar.left() / per_row);
     if (chunk > rows) chunk = rows;
     if (chunk < 1) return fail(VF_ERR_WORKSPACE, "workspace too small for alpha optimisation");
     std::vector<float*> H(nn, nullptr), A(nn, nullptr), M1(nn, nullptr), M2(nn, nullptr);
+    std::vector<float*> Bt(nn, nullptr), BM1(nn, nullptr), BM2(nn, nullptr);
     for (int u : relus) {
         H[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
         if (!grad_mode) {
             A[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
             M1[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
             M2[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+            if (o.split && o.split[u]) {
+                Bt[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+                BM1[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+                BM2[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+                if (!Bt[u] || !BM1[u] || !BM2[u]) return fail(VF_ERR_WORKSPACE, "workspace too small");
+            }
         }
     }
     float* Z = ar.take<float>((size_t)chunk * nmax);
@@ -974,6 +986,21 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
                 LAUNCH(net, launch_alpha_init(A[u], M1[u], M2[u], Mc, (int)nu, bd.relax[u], pg, s));
             }
         }
+        std::vector<BetaRows> bt(nn);
+        for (int u : relus) {
+            if (!(o.split && o.split[u])) continue;
+            const long long nu = net->nodes[u].n;
+            bt[u].split = o.split[u];
+            if (grad_mode) {
+                bt[u].beta = beta_in ? const_cast<float*>(beta_in) + aoff[u] + m0 * nu : nullptr;
+                bt[u].grad_out = beta_grad_out ? beta_grad_out + aoff[u] + m0 * nu : nullptr;
+            } else {
+                bt[u].beta = Bt[u];
+                bt[u].m1 = BM1[u];
+                bt[u].m2 = BM2[u];
+                LAUNCH(net, launch_zero_moments(Bt[u], BM1[u], BM2[u], Mc * nu, s));
+            }
+        }
         const int evals = grad_mode ? 1 : iters + 1;
         for (int it = 0; it < evals; ++it) {
             // down: back-substitution of the rows with the current slopes, keeping lam over every ReLU
@@ -986,7 +1013,7 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
                 const int nu = (int)net->nodes[u].n;
                 const Node& d = net->nodes[u - 1];
                 const int nd_in = (int)net->nodes[u - 2].n;
-                LAUNCH(net, launch_relax_alpha_rows(H[u], Mc, nu, bd.relax[u], pg, al[u], Z, cst, s));
+                LAUNCH(net, launch_relax_alpha_rows(H[u], Mc, nu, bd.relax[u], pg, al[u], Z, cst, s, 1, 0, bt[u]));
                 float* out = (u - 2 == 0) ? lam_in : H[u - 2];
                 if (d.op == VF_CONV2D)
                     LAUNCH(net, launch_conv_back(RowRef{Z, 0, nu, kHugeRows, 0}, Relax{nullptr, 0}, d.W, nullptr, Mc,
@@ -1015,7 +1042,7 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
                     LAUNCH(net, launch_rows_times_wt(G, dn.W, dn.b, (int)Mc, (int)net->nodes[d - 1].n, nu, Gn, s));
                 float* gout = grad_mode ? grad_out + aoff[u] + m0 * nu : nullptr;
                 LAUNCH(net, launch_relax_grad_adam(Gn, H[u], Mc, nu, bd.relax[u], pg, al[u], gout, M1[u], M2[u],
-                                                   grad_mode ? 0 : it + 1, lr, s));
+                                                   grad_mode ? 0 : it + 1, lr, s, bt[u]));
                 std::swap(G, Gn);
             }
         }
@@ -1037,7 +1064,8 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
 // Adam step; add: sum of the two sources).
 int spec_alpha_graph(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
                      const vf_opts& o, int iters, float lr, bool grad_mode, const float* alpha_in, float* grad_out,
-                     float* lb, float* lb_start, float* alpha_out, cudaStream_t s) {
+                     float* lb, float* lb_start, float* alpha_out, cudaStream_t s, const float* beta_in = nullptr,
+                     float* beta_grad_out = nullptr) {
     const int nn = (int)net->nodes.size();
     const int L = nn - 1;
     const long long n0 = net->nodes[0].n;
@@ -1062,9 +1090,13 @@ int spec_alpha_graph(vf_net* net, const float* centres, int B, float eps, const 
         if (nd.op == VF_CONV2D) ctiles = std::max(ctiles, conv_back_tiles(conv_geom(net, nd)));
     }
     const long long rows = (long long)B * R;
-    // per row: pending rows and gradients of every node, the per-ReLU slopes and Adam moments, constants
-    const size_t per_row = sizeof(float) * (2 * sum_all + (grad_mode ? 0 : 3 * sum_relu) + 2 + ctiles) +
-                           64 * (2 * nn + 3 * relus.size() + 8);
+    long long sum_split = 0;  // neurons of ReLUs with split constraints (their beta rows)
+    for (int u : relus)
+        if (o.split && o.split[u]) sum_split += net->nodes[u].n;
+    // per row: pending rows and gradients of every node, the per-ReLU slopes and Adam moments (and the
+    // multipliers of split ReLUs with theirs), constants
+    const size_t per_row = sizeof(float) * (2 * sum_all + (grad_mode ? 0 : 3 * (sum_relu + sum_split)) + 2 + ctiles) +
+                           64 * (2 * nn + 6 * relus.size() + 8);
     long long chunk = (long long)(ar.left() / per_row);
     if (chunk > rows) chunk = rows;
     if (chunk < 1) return fail(VF_ERR_WORKSPACE, "workspace too small for alpha optimisation");
@@ -1074,12 +1106,19 @@ int spec_alpha_graph(vf_net* net, const float* centres, int B, float eps, const 
         G[v] = ar.take<float>((size_t)chunk * net->nodes[v].n);
         if (!P[v] || !G[v]) return fail(VF_ERR_WORKSPACE, "workspace too small");
     }
+    std::vector<float*> Bt(nn, nullptr), BM1(nn, nullptr), BM2(nn, nullptr);
     for (int u : relus)
         if (!grad_mode) {
             A[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
             M1[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
             M2[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
             if (!A[u] || !M1[u] || !M2[u]) return fail(VF_ERR_WORKSPACE, "workspace too small");
+            if (o.split && o.split[u]) {
+                Bt[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+                BM1[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+                BM2[u] = ar.take<float>((size_t)chunk * net->nodes[u].n);
+                if (!Bt[u] || !BM1[u] || !BM2[u]) return fail(VF_ERR_WORKSPACE, "workspace too small");
+            }
         }
     float* cst = ar.take<float>(chunk);
     float* lbc = ar.take<float>(chunk);
@@ -1097,6 +1136,21 @@ int spec_alpha_graph(vf_net* net, const float* centres, int B, float eps, const 
             } else {
                 al[u] = A[u];
                 LAUNCH(net, launch_alpha_init(A[u], M1[u], M2[u], Mc, (int)nu, bd.relax[u], pg, s));
+            }
+        }
+        std::vector<BetaRows> bt(nn);
+        for (int u : relus) {
+            if (!(o.split && o.split[u])) continue;
+            const long long nu = net->nodes[u].n;
+            bt[u].split = o.split[u];
+            if (grad_mode) {
+                bt[u].beta = beta_in ? const_cast<float*>(beta_in) + aoff[u] + m0 * nu : nullptr;
+                bt[u].grad_out = beta_grad_out ? beta_grad_out + aoff[u] + m0 * nu : nullptr;
+            } else {
+                bt[u].beta = Bt[u];
+                bt[u].m1 = BM1[u];
+                bt[u].m2 = BM2[u];
+                LAUNCH(net, launch_zero_moments(Bt[u], BM1[u], BM2[u], Mc * nu, s));
             }
         }
         const int evals = grad_mode ? 1 : iters + 1;
@@ -1134,7 +1188,7 @@ int spec_alpha_graph(vf_net* net, const float* centres, int B, float eps, const 
                     }
                     case VF_RELU:
                         LAUNCH(net, launch_relax_alpha_rows(P[v], Mc, nv, bd.relax[v], pg, al[v], P[nd.src], cst, s,
-                                                            0, written[nd.src] ? 1 : 0));
+                                                            0, written[nd.src] ? 1 : 0, bt[v]));
                         written[nd.src] = 1;
                         break;
                     case VF_ADD:
@@ -1169,11 +1223,14 @@ int spec_alpha_graph(vf_net* net, const float* centres, int B, float eps, const 
                     case VF_RELU: {
                         CU(cudaMemcpyAsync(G[v], G[nd.src], sizeof(float) * Mc * nv, cudaMemcpyDeviceToDevice, s));
                         float* gout = grad_mode ? grad_out + aoff[v] + m0 * nv : nullptr;
-                        if (written[v])
+                        if (written[v]) {
                             LAUNCH(net, launch_relax_grad_adam(G[v], P[v], Mc, nv, bd.relax[v], pg, al[v], gout, M1[v],
-                                                               M2[v], grad_mode ? 0 : it + 1, lr, s));
-                        else if (gout != nullptr)  // not an ancestor of the last node: zero gradient
-                            CU(cudaMemsetAsync(gout, 0, sizeof(float) * Mc * nv, s));
+                                                               M2[v], grad_mode ? 0 : it + 1, lr, s, bt[v]));
+                        } else {  // not an ancestor of the last node: zero gradients
+                            if (gout != nullptr) CU(cudaMemsetAsync(gout, 0, sizeof(float) * Mc * nv, s));
+                            if (bt[v].grad_out != nullptr)
+                                CU(cudaMemsetAsync(bt[v].grad_out, 0, sizeof(float) * Mc * nv, s));
+                        }
                         break;
                     }
                     case VF_ADD: {
@@ -1591,18 +1648,36 @@ int vf_alpha_crown(vf_net* net, const float* centres, int B, float eps, const fl
 
 int vf_alpha_grad(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
                   const vf_opts* opts, const float* alpha, float* lb, float* grad, void* stream) {
+    return vf_alpha_beta_grad(net, centres, B, eps, C, R, C_bstride, opts, alpha, nullptr, lb, grad, nullptr, stream);
+}
+
+int vf_alpha_beta_grad(vf_net* net, const float* centres, int B, float eps, const float* C, int R,
+                       long long C_bstride, const vf_opts* opts, const float* alpha, const float* beta, float* lb,
+                       float* grad_alpha, float* grad_beta, void* stream) {
     TRY(check_net(net));
     vf_opts o{};
     if (opts) o = *opts;
-    if (!centres || !C || !lb || !alpha || !grad) return fail(VF_ERR_ARG, "NULL pointer");
+    if (!centres || !C || !lb || !alpha || !grad_alpha) return fail(VF_ERR_ARG, "NULL pointer");
     if (B < 0 || R < 0 || C_bstride < 0) return fail(VF_ERR_ARG, "negative size");
     if (!std::isfinite(eps) || eps < 0.f) return fail(VF_ERR_NONFINITE, "eps must be finite and >= 0");
+    if (o.both_sides) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation bounds one side: pass -C for upper bounds");
     if (B == 0 || R == 0) return VF_OK;
     if (!affine_chain(net))
-        return spec_alpha_graph(net, centres, B, eps, C, R, C_bstride, o, 0, 0.f, true, alpha, grad, lb, nullptr,
-                                nullptr, (cudaStream_t)stream);
-    return spec_alpha(net, centres, B, eps, C, R, C_bstride, o, 0, 0.f, true, alpha, grad, lb, nullptr, nullptr,
-                      (cudaStream_t)stream);
+        return spec_alpha_graph(net, centres, B, eps, C, R, C_bstride, o, 0, 0.f, true, alpha, grad_alpha, lb, nullptr,
+                                nullptr, (cudaStream_t)stream, beta, grad_beta);
+    return spec_alpha(net, centres, B, eps, C, R, C_bstride, o, 0, 0.f, true, alpha, grad_alpha, lb, nullptr, nullptr,
+                      (cudaStream_t)stream, beta, grad_beta);
+}
+
+int vf_net_node_info(const vf_net* net, int v, int* op, int* src, int* src2, long long* n) {
+    TRY(check_net(net));
+    if (v < 0 || v >= (int)net->nodes.size()) return fail(VF_ERR_ARG, "node index out of range");
+    const Node& nd = net->nodes[v];
+    if (op) *op = nd.op;
+    if (src) *src = nd.src;
+    if (src2) *src2 = nd.src2;
+    if (n) *n = nd.n;
+    return VF_OK;
 }
 
 int vf_profile_enable(vf_net* net, int enable) {

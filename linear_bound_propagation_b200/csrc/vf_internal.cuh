@@ -148,11 +148,13 @@ cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, c
 // hr and zr may both be NULL: then only the centre map W * hc + b is computed (the alpha-CROWN gradient).
 cudaError_t launch_ibp_conv(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
                             int B, const ConvGeom& g, float* zc, float* zr, cudaStream_t s);
-cudaError_t launch_ibp_relu(const float* c, const float* r, long long n, float* oc, float* orad, cudaStream_t s);
+cudaError_t launch_ibp_relu(const float* c, const float* r, long long n, float* oc, float* orad, cudaStream_t s,
+                            const signed char* split = nullptr);
 cudaError_t launch_ibp_add(const float* c1, const float* r1, const float* c2, const float* r2, long long n,
                            float* oc, float* orad, cudaStream_t s);
 cudaError_t launch_fill(float* p, long long n, float v, cudaStream_t s);
-cudaError_t launch_bounds_from_cr(const float* c, const float* r, long long n, float* lb, float* ub, cudaStream_t s);
+cudaError_t launch_bounds_from_cr(const float* c, const float* r, long long n, float* lb, float* ub, cudaStream_t s,
+                                  const signed char* split = nullptr);
 
 // ---- relaxation, pass bookkeeping, decision (k_misc.cu) ------------------------------
 // P[i] = {lo, up, t, bias of the affine source}; bias may be null (then 0); neuron j = i % n_per_centre
@@ -199,17 +201,44 @@ cudaError_t launch_rows_times_wt(const float* A, const float* W, const float* bi
                                  cudaStream_t s);
 
 // ---- alpha-CROWN (k_alpha.cu) -----------------------------------------------------------
+// Split constraints of one ReLU for the beta terms of the specification bound: the sign of each
+// (centre, neuron) [B, n] (0 = free), the per-row multipliers [M, n], their Adam moments and the
+// gradient output [M, n]. All null: no split constraint.
+struct BetaRows {
+    const signed char* split = nullptr;
+    float* beta = nullptr;
+    float* m1 = nullptr;
+    float* m2 = nullptr;
+    float* grad_out = nullptr;
+};
 cudaError_t launch_relax_alpha_rows(const float* H, long long M, int n, const float4* P, PassGeom pg,
                                     const float* alpha, float* Z, float* cst, cudaStream_t s, int with_bias = 1,
-                                    int accumulate = 0);
+                                    int accumulate = 0, BetaRows bt = BetaRows{});
 cudaError_t launch_concretize_grad(const float* lam, long long M, int n0, PassGeom pg, const float* centres, float eps,
                                    const float* cst, float* lb, float* G, cudaStream_t s);
 cudaError_t launch_relax_grad_adam(float* G, const float* H, long long M, int n, const float4* P, PassGeom pg,
                                    float* alpha, float* grad_out, float* m1, float* m2, int adam_step, float lr,
-                                   cudaStream_t s);
+                                   cudaStream_t s, BetaRows bt = BetaRows{});
+cudaError_t launch_zero_moments(float* beta, float* m1, float* m2, long long count, cudaStream_t s);
 cudaError_t launch_alpha_init(float* alpha, float* m1, float* m2, long long M, int n, const float4* P, PassGeom pg,
                               cudaStream_t s);
 cudaError_t launch_best_update(float* best, const float* cur, long long M, int first, cudaStream_t s);
+
+// ---- branch and bound (k_bab.cu) ------------------------------------------------------------
+// Per subdomain: the neuron to split next (search-wide index, -1 if none is unstable), whether some
+// pre-activation bound has l > u, the lowest row bound (max of two bound arrays when both are given)
+// and the branching score of the chosen neuron.
+struct BabPick {
+    int best;
+    int empty;
+    float minlb;
+    float score;
+};
+cudaError_t launch_bab_pick(const float* pre_lb, const float* pre_ub, int D, const long long* blk_off, const int* blk_n,
+                            const int* gbase, int nl, const float* lb_a, const float* lb_b, int R, BabPick* out,
+                            cudaStream_t s);
+// dst[d, :] = src[:] for d < D (n floats per row).
+cudaError_t launch_repeat_row(const float* src, long long n, int D, float* dst, cudaStream_t s);
 
 // Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per (kernel,
 // device, size); safe to call from several threads.

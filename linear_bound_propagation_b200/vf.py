@@ -45,7 +45,21 @@ class NodeDesc(ctypes.Structure):
 class Opts(ctypes.Structure):
     _fields_ = [("relu_crown", ctypes.POINTER(ctypes.c_int)), ("alpha", ctypes.POINTER(ctypes.c_void_p)),
                 ("both_sides", ctypes.c_int), ("skip_finite_check", ctypes.c_int),
-                ("pre_lb", ctypes.c_void_p), ("pre_ub", ctypes.c_void_p), ("no_host_sync", ctypes.c_int)]
+                ("pre_lb", ctypes.c_void_p), ("pre_ub", ctypes.c_void_p), ("no_host_sync", ctypes.c_int),
+                ("split", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class BabOpts(ctypes.Structure):
+    _fields_ = [("max_domains", ctypes.c_int), ("batch", ctypes.c_int), ("alpha_iters", ctypes.c_int),
+                ("lr", ctypes.c_float), ("relu_crown", ctypes.POINTER(ctypes.c_int))]
+
+
+class BabResult(ctypes.Structure):
+    _fields_ = [("status", ctypes.c_int), ("domains", ctypes.c_longlong), ("rounds", ctypes.c_int),
+                ("max_depth", ctypes.c_int), ("lb", ctypes.c_float)]
+
+
+BAB_STATUS = {1: "verified", -1: "falsified", 0: "unknown"}
 
 
 _lib = None
@@ -79,6 +93,9 @@ def lib() -> ctypes.CDLL:
     L.vf_concretize_dense_noalloc.argtypes = [P, LL, I, P, P, P, F, I, I, I, P, P]
     L.vf_alpha_crown.argtypes = [P, P, I, F, P, I, LL, ctypes.POINTER(Opts), I, F, P, P, P, P]
     L.vf_alpha_grad.argtypes = [P, P, I, F, P, I, LL, ctypes.POINTER(Opts), P, P, P, P]
+    L.vf_alpha_beta_grad.argtypes = [P, P, I, F, P, I, LL, ctypes.POINTER(Opts), P, P, P, P, P, P]
+    L.vf_net_node_info.argtypes = [P, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(LL)]
+    L.vf_bab_verify.argtypes = [P, P, F, P, I, ctypes.POINTER(BabOpts), ctypes.POINTER(BabResult), P]
     L.vf_launch_count.argtypes = [P]
     L.vf_launch_count.restype = LL
     _lib = L
@@ -188,8 +205,10 @@ class Net:
 
     def verify(self, centres: torch.Tensor, eps: float, C: torch.Tensor, crown_relus: Optional[Sequence[int]] = None,
                alpha: Optional[Dict[int, torch.Tensor]] = None, both_sides: bool = False, want_pre: bool = False,
-               skip_finite_check: bool = False, no_host_sync: bool = False, stream=None, out=None):
-        """vf_verify_batch. C: [B or 1, R, n_L]. Returns dict of device tensors."""
+               skip_finite_check: bool = False, no_host_sync: bool = False, stream=None, out=None,
+               splits: Optional[Dict[int, torch.Tensor]] = None):
+        """vf_verify_batch. C: [B or 1, R, n_L]. splits: ReLU node -> int8 [B, n] signs (+1: z >= 0,
+        -1: z <= 0, 0: free), one subdomain per centre row. Returns dict of device tensors."""
         B = centres.shape[0]
         R = C.shape[1]
         dev = centres.device
@@ -217,6 +236,10 @@ class Net:
         o.both_sides = 1 if both_sides else 0
         o.skip_finite_check = 1 if skip_finite_check else 0
         o.no_host_sync = 1 if no_host_sync else 0
+        sarr = self._split_array(splits)
+        if sarr is not None:
+            o.split = ctypes.cast(sarr, ctypes.POINTER(ctypes.c_void_p))
+            keep.append(sarr)
         o.pre_lb = out["pre_lb"].data_ptr() if "pre_lb" in out else None
         o.pre_ub = out["pre_ub"].data_ptr() if "pre_ub" in out else None
         _check(lib().vf_verify_batch(self.h, _ptr(centres), B, float(eps), _ptr(C), R, bstride, ctypes.byref(o),
@@ -224,14 +247,28 @@ class Net:
                                      _ptr(out.get("verified")), _stream_ptr(stream)))
         return out
 
-    def _opts(self, crown_relus=None):
+    def _split_array(self, splits):
+        if not splits:
+            return None
+        arr = (ctypes.c_void_p * self.n_nodes)()
+        for v, sg in splits.items():
+            assert sg.dtype == torch.int8 and sg.is_cuda and sg.is_contiguous(), "splits: contiguous CUDA int8"
+            arr[v] = sg.data_ptr()
+        return arr
+
+    def _opts(self, crown_relus=None, splits=None):
         o = Opts()
-        keep = None
+        keep = []
         if crown_relus is not None:
-            keep = (ctypes.c_int * self.n_nodes)()
+            flags = (ctypes.c_int * self.n_nodes)()
             for v in crown_relus:
-                keep[v] = 1
-            o.relu_crown = ctypes.cast(keep, ctypes.POINTER(ctypes.c_int))
+                flags[v] = 1
+            o.relu_crown = ctypes.cast(flags, ctypes.POINTER(ctypes.c_int))
+            keep.append(flags)
+        sarr = self._split_array(splits)
+        if sarr is not None:
+            o.split = ctypes.cast(sarr, ctypes.POINTER(ctypes.c_void_p))
+            keep.append(sarr)
         return o, keep
 
     def alpha_size(self, B: int, R: int) -> int:
@@ -239,14 +276,15 @@ class Net:
         return B * R * sum(self.sizes[v] for v in self.relu_ids)
 
     def alpha_crown(self, centres: torch.Tensor, eps: float, C: torch.Tensor, iters: int = 20, lr: float = 0.1,
-                    crown_relus=None, want_alpha: bool = False, stream=None):
-        """vf_alpha_crown: returns dict(lb=best bound [B, R], lb_start=[B, R], alpha=final slopes or None)."""
+                    crown_relus=None, want_alpha: bool = False, stream=None, splits=None):
+        """vf_alpha_crown: returns dict(lb=best bound [B, R], lb_start=[B, R], alpha=final slopes or None).
+        With splits (see verify) the split multipliers beta are optimised with the slopes."""
         B, R = centres.shape[0], C.shape[1]
         bstride = 0 if C.shape[0] == 1 else R * C.shape[2]
         lb = torch.empty(B, R, device=centres.device)
         lb0 = torch.empty(B, R, device=centres.device)
         al = torch.empty(self.alpha_size(B, R), device=centres.device) if want_alpha else None
-        o, keep = self._opts(crown_relus)
+        o, keep = self._opts(crown_relus, splits)
         _check(lib().vf_alpha_crown(self.h, _ptr(centres), B, float(eps), _ptr(C), R, bstride, ctypes.byref(o), iters,
                                     float(lr), _ptr(lb), _ptr(lb0), _ptr(al), _stream_ptr(stream)))
         return {"lb": lb, "lb_start": lb0, "alpha": al}
@@ -262,6 +300,38 @@ class Net:
         _check(lib().vf_alpha_grad(self.h, _ptr(centres), B, float(eps), _ptr(C), R, bstride, ctypes.byref(o),
                                    _ptr(alpha), _ptr(lb), _ptr(grad), _stream_ptr(stream)))
         return lb, grad
+
+    def alpha_beta_grad(self, centres: torch.Tensor, eps: float, C: torch.Tensor, alpha: torch.Tensor,
+                        beta: Optional[torch.Tensor], splits, crown_relus=None, stream=None):
+        """vf_alpha_beta_grad: (lb [B, R], d lb / d alpha, d lb / d beta) at the given slopes and split
+        multipliers (both in alpha's layout)."""
+        B, R = centres.shape[0], C.shape[1]
+        bstride = 0 if C.shape[0] == 1 else R * C.shape[2]
+        lb = torch.empty(B, R, device=centres.device)
+        ga = torch.empty_like(alpha)
+        gb = torch.empty_like(alpha)
+        o, keep = self._opts(crown_relus, splits)
+        _check(lib().vf_alpha_beta_grad(self.h, _ptr(centres), B, float(eps), _ptr(C), R, bstride, ctypes.byref(o),
+                                        _ptr(alpha), _ptr(beta), _ptr(lb), _ptr(ga), _ptr(gb), _stream_ptr(stream)))
+        return lb, ga, gb
+
+    def bab(self, centre: torch.Tensor, eps: float, C: torch.Tensor, max_domains: int = 1000, batch: int = 16,
+            alpha_iters: int = 20, lr: float = 0.1, crown_relus=None, stream=None):
+        """vf_bab_verify on one box: centre [n0], C [R, n_L] (device). Returns dict(status, domains, rounds,
+        max_depth, lb)."""
+        o = BabOpts(max_domains=max_domains, batch=batch, alpha_iters=alpha_iters, lr=float(lr))
+        keep = None
+        if crown_relus is not None:
+            keep = (ctypes.c_int * self.n_nodes)()
+            for v in crown_relus:
+                keep[v] = 1
+            o.relu_crown = ctypes.cast(keep, ctypes.POINTER(ctypes.c_int))
+        r = BabResult()
+        C2 = C.reshape(-1, C.shape[-1]).contiguous()
+        _check(lib().vf_bab_verify(self.h, _ptr(centre.contiguous()), float(eps), _ptr(C2), C2.shape[0],
+                                   ctypes.byref(o), ctypes.byref(r), _stream_ptr(stream)))
+        return {"status": BAB_STATUS[r.status], "domains": r.domains, "rounds": r.rounds, "max_depth": r.max_depth,
+                "lb": r.lb}
 
     def profile(self, enable: bool):
         _check(lib().vf_profile_enable(self.h, 1 if enable else 0))
