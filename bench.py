@@ -383,6 +383,9 @@ def run_ours(args):
                  "unit": UNIT, "ms_per_step": a_ms / args.steps, "mean_lb_gain": float(gain.mean().item()),
                  "rows_improved": float((gain > 0).float().mean().item()),
                  "note": "vf_alpha_crown: intermediate bounds as in the verify step, then per-row lower-slope Adam ascent"}
+    bab = None
+    if args.bab_domains > 0 and not w.both_sides and w.C.shape[1] > 1:
+        bab = bab_leg(args, w, net, centres, dev, stream, world, rank)
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -393,13 +396,66 @@ def run_ours(args):
                         "pipeline": "double-buffered: the H2D of step i+1 and the D2H of step i overlap compute on a "
                                     "copy stream; all copies of every step are inside the timed region"},
                 "gpu_launches": launches, "clocks": clocks, "verified_specs": verified, "total_specs": B * Rs,
-                "alpha_crown": alpha, "graph": graph}
+                "alpha_crown": alpha, "graph": graph, "bab": bab}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = oracle_sample(w, args.cpu_sample_s)[0]
+            if bab is not None:
+                line["cpu_baseline"]["bab"] = oracle_bab_sample(args, w, bab["label0"])
         print(json.dumps(line), flush=True)
     net.close()
     if world > 1:
         dist.destroy_process_group()
+
+
+def bab_leg(args, w, net, centres, dev, stream, world, rank):
+    """Branch and bound (vf_bab_verify) on the workload's network: for the first --bab-centres centres,
+    the margin rows of the class the network gives the centre (so the centre is no counterexample), at
+    the workload's radius, a budget of --bab-domains subdomains bounded --bab-batch at a time with
+    alpha-beta ascent steps. Reports subdomains bounded per second (device-timed, max over ranks)."""
+    import torch
+    from linear_bound_propagation_b200 import vf
+    K = min(args.bab_centres, centres.shape[0])
+    lbI, _ = net.ibp(centres[:K].contiguous(), 0.0)
+    logits = net.node_block(lbI, len(w.net) - 1, K)
+    labels = logits.argmax(dim=1).cpu().numpy()
+    nL = logits.shape[1]
+    specs = [torch.from_numpy(synth.margin_spec(np.array([y]), nL)[0]).to(dev) for y in labels]
+    kw = dict(batch=args.bab_batch, alpha_iters=args.bab_alpha_iters, lr=0.1, crown_relus=w.crown_relus)
+    net.bab(centres[0], w.eps, specs[0], max_domains=min(args.bab_batch + 1, args.bab_domains), **kw)  # warm-up
+    torch.cuda.synchronize()
+    ms, domains, statuses = 0.0, 0, []
+    for k in range(K):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        r = net.bab(centres[k], w.eps, specs[k], max_domains=args.bab_domains, **kw)
+        e1.record(stream)
+        e1.synchronize()
+        ms += e0.elapsed_time(e1)
+        domains += r["domains"]
+        statuses.append(r["status"])
+    ms = max_over_ranks(ms, dev)
+    out = {"value": world * domains / (ms / 1e3) if ms > 0 else None, "unit": "subdomains/s", "subdomains": domains,
+           "ms": ms, "centres": K, "statuses": statuses, "budget": args.bab_domains, "batch": args.bab_batch,
+           "alpha_iters": args.bab_alpha_iters, "eps": w.eps,
+           "note": "vf_bab_verify: best-first ReLU-split search; every subdomain bound by vf_verify_batch plus "
+                   "alpha-beta ascent, decisions on the device, one host synchronisation per round"}
+    out["label0"] = int(labels[0])
+    return out
+
+
+def oracle_bab_sample(args, w, label):
+    """The oracle's search on the first centre of the same problem as the device's branch-and-bound leg,
+    with a small budget (two rounds), timed on the host cores."""
+    import oracle.lbp as O
+    nL = w.net[-1].W.shape[0]
+    budget = min(args.bab_domains, 2 * args.bab_batch + 1)
+    C0 = synth.margin_spec(np.array([label]), nL)[0]
+    t0 = time.perf_counter()
+    o = O.bab(w.net, w.centres[0], w.eps, C0, max_domains=budget, batch=args.bab_batch, iters=args.bab_alpha_iters,
+              lr=0.1, crown_relus=w.crown_relus)
+    dt = time.perf_counter() - t0
+    return {"value": o.domains / dt, "unit": "subdomains/s", "cores": threads_used(), "kind": "oracle",
+            "sample": f"first centre, budget {budget} subdomains ({o.domains} bounded, {o.status}), {dt:.2f} s"}
 
 
 def main():
@@ -418,6 +474,11 @@ def main():
     ap.add_argument("--graph", action="store_true", help="also time the verify call replayed from a CUDA graph")
     ap.add_argument("--alpha-iters", type=int, default=10,
                     help="also time vf_alpha_crown with this many Adam steps (dense chains; 0 = skip)")
+    ap.add_argument("--bab-domains", type=int, default=512,
+                    help="also time vf_bab_verify with this budget of subdomains per centre (0 = skip)")
+    ap.add_argument("--bab-centres", type=int, default=2)
+    ap.add_argument("--bab-batch", type=int, default=64)
+    ap.add_argument("--bab-alpha-iters", type=int, default=10)
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
