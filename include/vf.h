@@ -139,6 +139,14 @@ typedef struct {
      * the subdomain only. A subdomain that holds no input shows up as some pre_lb > pre_ub.
      * vf_alpha_crown also optimises the split multipliers beta (see vf_alpha_beta_grad). */
     const signed char* const* split;
+    /* 1: sound in fp32 (vf_verify_batch only; VF_ERR_UNSUPPORTED elsewhere). Every bound is widened by a
+     * rigorous budget for its own rounding, so lb never exceeds the exact-arithmetic minimum over the
+     * box (technical summary, section 4.2: soundness as a one-sided over-approximation). Interval ends
+     * are rounded outwards with a gamma_K = K u / (1 - K u) term per dot product of K terms; the ReLU
+     * intercept is rounded up; each back-substituted row's result is lowered by |row| . A, where A is a
+     * per-centre error-weight vector accumulated forward through |W|, the ReLU slopes and the node's
+     * rounding weights. Contractions take the FFMA kernels (IEEE rounding), not the tensor cores. */
+    int sound;
 } vf_opts;
 
 /* Whole verification step (section 1): IBP, CROWN intermediate bounds, specification

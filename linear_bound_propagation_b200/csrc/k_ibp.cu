@@ -24,13 +24,13 @@ namespace {
 __global__ void __launch_bounds__(256)
 ibp_dense_k(const float* __restrict__ hc, const float* __restrict__ hr, const float* __restrict__ W,
             const float* __restrict__ Wabs, const float* __restrict__ bias, const float* __restrict__ rowsum_abs,
-            float eps, int B, int K, int N, float* __restrict__ zc, float* __restrict__ zr) {
+            float eps, int B, int K, int N, float* __restrict__ zc, float* __restrict__ zr, int z0) {
     constexpr int TM = 64, TN = 64, KB = 16, LDA = TM + 4, LDB = TN + 4;
     __shared__ __align__(16) float As[KB][LDA];
     __shared__ __align__(16) float Bs[KB][LDB];
     const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
     const int m0 = blockIdx.x * TM, n0 = blockIdx.y * TN;
-    const bool rad = blockIdx.z == 1;
+    const bool rad = blockIdx.z + z0 == 1;
     if (rad && rowsum_abs != nullptr) {
         for (int e = tid; e < TM * TN; e += 256) {
             const int m = m0 + e / TN, n = n0 + e % TN;
@@ -123,7 +123,7 @@ __global__ void ibp_conv_k(const float* __restrict__ hc, const float* __restrict
                 }
             }
         }
-        zc[idx] = sc + bias[co];
+        zc[idx] = bias != nullptr ? sc + bias[co] : sc;
         if (zr != nullptr) zr[idx] = sr;
     }
 }
@@ -157,9 +157,11 @@ __global__ void fill_k(float* __restrict__ p, long long n, float v) {
 // l = c - r, u = c + r; under split constraints a neuron split to z >= 0 takes l = max(l, 0) and one
 // split to z <= 0 takes u = min(u, 0) (an empty interval marks a subdomain with no input).
 __global__ void bounds_k(const float* __restrict__ c, const float* __restrict__ r, long long n,
-                         const signed char* __restrict__ split, float* __restrict__ lb, float* __restrict__ ub) {
+                         const signed char* __restrict__ split, float* __restrict__ lb, float* __restrict__ ub,
+                         int sound) {
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-        float l = c[i] - r[i], u = c[i] + r[i];
+        float l = sound ? __fsub_rd(c[i], r[i]) : c[i] - r[i];
+        float u = sound ? __fadd_ru(c[i], r[i]) : c[i] + r[i];
         if (split != nullptr) {
             const signed char sg = split[i];
             if (sg > 0) l = fmaxf(l, 0.f);
@@ -182,14 +184,20 @@ cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, c
                              const float* rowsum_abs, float eps, int B, int K, int N, float* zc, float* zr,
                              cudaStream_t s) {
     dim3 grid((B + 63) / 64, (N + 63) / 64, 2);
-    ibp_dense_k<<<grid, 256, 0, s>>>(hc, hr, W, Wabs, bias, rowsum_abs, eps, B, K, N, zc, zr);
+    ibp_dense_k<<<grid, 256, 0, s>>>(hc, hr, W, Wabs, bias, rowsum_abs, eps, B, K, N, zc, zr, 0);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_abs_rows_times_wt(const float* A, const float* Wabs, int M, int K, int N, float* out, cudaStream_t s) {
+    dim3 grid((M + 63) / 64, (N + 63) / 64, 1);  // only the radius product: out = A |W|^T
+    ibp_dense_k<<<grid, 256, 0, s>>>(A, A, Wabs, Wabs, nullptr, nullptr, 0.f, M, K, N, out, out, 1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_rows_times_wt(const float* A, const float* W, const float* bias, int M, int K, int N, float* out,
                                  cudaStream_t s) {
     dim3 grid((M + 63) / 64, (N + 63) / 64, 1);  // only the centre product: out = A W^T + bias
-    ibp_dense_k<<<grid, 256, 0, s>>>(A, A, W, W, bias, nullptr, 0.f, M, K, N, out, out);
+    ibp_dense_k<<<grid, 256, 0, s>>>(A, A, W, W, bias, nullptr, 0.f, M, K, N, out, out, 0);
     return cudaGetLastError();
 }
 
@@ -218,8 +226,8 @@ cudaError_t launch_fill(float* p, long long n, float v, cudaStream_t s) {
 }
 
 cudaError_t launch_bounds_from_cr(const float* c, const float* r, long long n, float* lb, float* ub, cudaStream_t s,
-                                  const signed char* split) {
-    bounds_k<<<grid_for(n, 256), 256, 0, s>>>(c, r, n, split, lb, ub);
+                                  const signed char* split, int sound) {
+    bounds_k<<<grid_for(n, 256), 256, 0, s>>>(c, r, n, split, lb, ub, sound);
     return cudaGetLastError();
 }
 

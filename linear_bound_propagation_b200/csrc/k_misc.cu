@@ -32,7 +32,8 @@ unsigned grid_for(long long n, int threads) {
 // the row constant together with the relaxation intercept.
 __global__ void relax_params_k(const float* __restrict__ l, const float* __restrict__ u,
                                const float* __restrict__ alpha, long long n, float4* __restrict__ P,
-                               const float* __restrict__ bias, long long n_per_centre, long long per_channel) {
+                               const float* __restrict__ bias, long long n_per_centre, long long per_channel,
+                               int sound) {
     GRID_STRIDE(i, n) {
         const float lo_b = l[i], up_b = u[i];
         float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -43,7 +44,8 @@ __global__ void relax_params_k(const float* __restrict__ l, const float* __restr
         } else {
             const float s = up_b / (up_b - lo_b);
             p.y = s;
-            p.z = -s * lo_b;
+            // sound: the line s z + t lies above the ReLU at both ends (hence on [l, u]) in exact arithmetic
+            p.z = sound ? fmaxf(__fmul_ru(s, -lo_b), __fmul_ru(up_b, __fsub_ru(1.f, s))) : -s * lo_b;
             if (alpha != nullptr)
                 p.x = fminf(fmaxf(alpha[i], 0.f), 1.f);
             else
@@ -181,14 +183,20 @@ __global__ void add_partials_k(float* __restrict__ cst, const float* __restrict_
 
 // Intermediate bounds after a pass over node p (rows [I; -I] per centre): IBP-unstable neurons
 // take l = max(l, lb_j), u = min(u, -lb_{n + j}); IBP-stable ones keep their (exact) relaxation.
+// corr (optional, [B, n]): an error budget taken off both rows' lower bounds, rounded outwards.
 __global__ void intersect_k(float* __restrict__ l, float* __restrict__ u, const float* __restrict__ pass_out, int B,
-                            long long n) {
+                            long long n, const float* __restrict__ corr) {
     GRID_STRIDE(i, (long long)B * n) {
         const long long b = i / n, j = i % n;
         const float l0 = l[i], u0 = u[i];
         if (l0 < 0.f && u0 > 0.f) {
-            l[i] = fmaxf(l0, pass_out[b * 2 * n + j]);
-            u[i] = fminf(u0, -pass_out[b * 2 * n + n + j]);
+            float lc = pass_out[b * 2 * n + j], uc = -pass_out[b * 2 * n + n + j];
+            if (corr != nullptr) {
+                lc = __fsub_rd(lc, corr[i]);
+                uc = __fadd_ru(uc, corr[i]);
+            }
+            l[i] = fmaxf(l0, lc);
+            u[i] = fminf(u0, uc);
         }
     }
 }
@@ -245,14 +253,20 @@ __global__ void __launch_bounds__(256) unstable_list_k(const float* __restrict__
 
 // Intersection after a compacted pass (2 * half rows per centre: +e_j for the listed j, then -e_j).
 __global__ void intersect_compact_k(float* __restrict__ l, float* __restrict__ u, const float* __restrict__ pass_out,
-                                    const int* __restrict__ idx, int B, long long n, int half) {
+                                    const int* __restrict__ idx, int B, long long n, int half,
+                                    const float* __restrict__ corr) {
     GRID_STRIDE(e, (long long)B * half) {
         const long long b = e / half, i = e % half;
         const int j = idx[e];
         if (j < 0) continue;
         const long long k = b * n + j;
-        l[k] = fmaxf(l[k], pass_out[b * 2 * half + i]);
-        u[k] = fminf(u[k], -pass_out[b * 2 * half + half + i]);
+        float lc = pass_out[b * 2 * half + i], uc = -pass_out[b * 2 * half + half + i];
+        if (corr != nullptr) {
+            lc = __fsub_rd(lc, corr[k]);
+            uc = __fadd_ru(uc, corr[k]);
+        }
+        l[k] = fmaxf(l[k], lc);
+        u[k] = fminf(u[k], uc);
     }
 }
 
@@ -282,25 +296,33 @@ __global__ void spec_rows_k(const float* __restrict__ C, long long C_bstride, in
 // IBP bound of the specification: C applied to the last node's interval, C c -+ |C| r.
 __global__ void __launch_bounds__(256)
 spec_ibp_k(const float* __restrict__ C, long long C_bstride, int B, int R, int nL, const float* __restrict__ zc,
-           const float* __restrict__ zr, float* __restrict__ lb, float* __restrict__ ub) {
+           const float* __restrict__ zr, float* __restrict__ lb, float* __restrict__ ub, float gam) {
     const int lane = threadIdx.x & 31;
     const long long rows = (long long)B * R;
     for (long long w = blockIdx.x * 8LL + (threadIdx.x >> 5); w < rows; w += (long long)gridDim.x * 8) {
         const long long b = w / R, r = w % R;
         const float* cr = C + b * C_bstride + r * nL;
-        float sc = 0.f, sr = 0.f;
+        float sc = 0.f, sr = 0.f, sa = 0.f;
         for (int j = lane; j < nL; j += 32) {
             sc = fmaf(cr[j], zc[b * nL + j], sc);
             sr = fmaf(fabsf(cr[j]), zr[b * nL + j], sr);
+            if (gam > 0.f) sa = __fmaf_ru(fabsf(cr[j]), __fadd_ru(fabsf(zc[b * nL + j]), zr[b * nL + j]), sa);
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
             sc += __shfl_xor_sync(0xffffffffu, sc, off);
             sr += __shfl_xor_sync(0xffffffffu, sr, off);
+            sa = __fadd_ru(sa, __shfl_xor_sync(0xffffffffu, sa, off));
         }
         if (lane == 0) {
-            lb[w] = sc - sr;
-            ub[w] = sc + sr;
+            if (gam > 0.f) {  // sound: both sums err by at most gam * sum |C| (|zc| + zr)
+                const float e = __fmul_ru(gam, sa);
+                lb[w] = __fsub_rd(__fsub_rd(sc, sr), e);
+                ub[w] = __fadd_ru(__fadd_ru(sc, sr), e);
+            } else {
+                lb[w] = sc - sr;
+                ub[w] = sc + sr;
+            }
         }
     }
 }
@@ -350,8 +372,9 @@ unsigned rows_grid(long long rows_per_cta_units) {
 }  // namespace
 
 cudaError_t launch_relax_params(const float* l, const float* u, const float* alpha, long long n, float4* P,
-                                const float* bias, long long n_per_centre, long long per_channel, cudaStream_t s) {
-    relax_params_k<<<grid_for(n, 256), 256, 0, s>>>(l, u, alpha, n, P, bias, n_per_centre, per_channel);
+                                const float* bias, long long n_per_centre, long long per_channel, cudaStream_t s,
+                                int sound) {
+    relax_params_k<<<grid_for(n, 256), 256, 0, s>>>(l, u, alpha, n, P, bias, n_per_centre, per_channel, sound);
     return cudaGetLastError();
 }
 
@@ -397,10 +420,10 @@ cudaError_t launch_add_partials(float* cst, const float* part, int ntiles, long 
 }
 
 cudaError_t launch_intersect(float* l, float* u, const float* l_ibp, const float* u_ibp, const float* pass_out, int B,
-                             long long n, cudaStream_t s) {
+                             long long n, cudaStream_t s, const float* corr) {
     (void)l_ibp;
     (void)u_ibp;
-    intersect_k<<<grid_for((long long)B * n, 256), 256, 0, s>>>(l, u, pass_out, B, n);
+    intersect_k<<<grid_for((long long)B * n, 256), 256, 0, s>>>(l, u, pass_out, B, n, corr);
     return cudaGetLastError();
 }
 
@@ -417,9 +440,9 @@ cudaError_t launch_unstable_list(const float* l, const float* u, int B, long lon
 }
 
 cudaError_t launch_intersect_compact(float* l, float* u, const float* pass_out, const int* idx, int B, long long n,
-                                     int half, cudaStream_t s) {
+                                     int half, cudaStream_t s, const float* corr) {
     if (B <= 0 || half <= 0) return cudaSuccess;
-    intersect_compact_k<<<grid_for((long long)B * half, 256), 256, 0, s>>>(l, u, pass_out, idx, B, n, half);
+    intersect_compact_k<<<grid_for((long long)B * half, 256), 256, 0, s>>>(l, u, pass_out, idx, B, n, half, corr);
     return cudaGetLastError();
 }
 
@@ -436,8 +459,8 @@ cudaError_t launch_spec_rows(const float* C, long long C_bstride, int BC, int R,
 }
 
 cudaError_t launch_spec_ibp(const float* C, long long C_bstride, int B, int R, int nL, const float* zc, const float* zr,
-                            float* lb, float* ub, cudaStream_t s) {
-    spec_ibp_k<<<rows_grid(((long long)B * R + 7) / 8), 256, 0, s>>>(C, C_bstride, B, R, nL, zc, zr, lb, ub);
+                            float* lb, float* ub, cudaStream_t s, float gam) {
+    spec_ibp_k<<<rows_grid(((long long)B * R + 7) / 8), 256, 0, s>>>(C, C_bstride, B, R, nL, zc, zr, lb, ub, gam);
     return cudaGetLastError();
 }
 

@@ -99,6 +99,7 @@ struct vf_net {
     int conv_whole_warp = 2;
     int conv_win_per_position = 0;  // windowed rows without position blocking (VF_CONV_WIN_KERNEL=1)
     int compact = 1;        // intermediate passes over IBP-unstable neurons only (VF_COMPACT=0: off)
+    int call_sound = 0;     // set for the duration of a vf_opts.sound call: contractions take FFMA kernels
     bool prof = false;
     std::vector<cudaEvent_t> ev_free;
     struct Timed {
@@ -241,6 +242,7 @@ struct Walker {
     bool compact = false;     // identity-trick pass over the listed unstable neurons only (pg.idx)
     PassStart ps{1, 1, 1};    // the pass's start node
     long long max_len = 0;    // longest row a pool buffer has held
+    const std::vector<float*>* sw = nullptr;  // sound mode: per-node rounding weights [B, n_v]
 
     int alloc_buf(int* out, long long len) {
         max_len = std::max(max_len, len);
@@ -425,6 +427,9 @@ struct Walker {
         pend[v] = Entry();
         if (e.kind == E_NONE) return VF_OK;
         const Node& nd = net->nodes[v];
+        // sound mode: the rounding budget of these rows at this node (identity starts are exact)
+        if (sw != nullptr && !dry && e.kind != E_IDENT && (*sw)[v] != nullptr)
+            LAUNCH(net, launch_row_budget(e.ref, e.rx, M, (int)nd.n, pg, (*sw)[v], cst, s));
         switch (nd.op) {
             case VF_INPUT: {
                 if (e.kind == E_IDENT || e.rx.P != nullptr || e.windowed) {
@@ -487,13 +492,13 @@ struct Walker {
                     x.ref = RowRef{nd.pmW, 0, sn.n, 2 * nd.n, pg.pass_m0};
                     return add_into(nd.src, x);
                 }
-                const bool fuse = (nd.src == 0 && ext_in == nullptr && net->nodes[0].consumers == 1 &&
+                const bool fuse = (nd.src == 0 && ext_in == nullptr && net->nodes[0].consumers == 1 && sw == nullptr &&
                                    pend[0].kind == E_NONE);
                 float* out = nullptr;
                 long long ld = 0;
                 int mode = OUT_CONCRETIZE;
                 if (!fuse) TRY(target(nd.src, &out, &ld, &mode));
-                const bool tc = net->dense_kernel == 0 && nd.WtHi != nullptr &&
+                const bool tc = net->dense_kernel == 0 && !net->call_sound && nd.WtHi != nullptr &&
                                 dense_back_tc_supported(e.ref, e.rx, M, (int)nd.n, (int)sn.n, pg);
                 if (fuse) part_tiles = tc ? dense_back_tc_tiles_n((int)sn.n) : dense_back_tiles_n((int)sn.n);
                 if (!dry) {
@@ -550,7 +555,7 @@ struct Walker {
                     e = pend[v];
                     pend[v] = Entry();
                 }
-                const bool fuse = (nd.src == 0 && ext_in == nullptr && net->nodes[0].consumers == 1 &&
+                const bool fuse = (nd.src == 0 && ext_in == nullptr && net->nodes[0].consumers == 1 && sw == nullptr &&
                                    pend[0].kind == E_NONE);
                 float* out = nullptr;
                 long long ld = 0;
@@ -628,7 +633,7 @@ bool input_buffered(const vf_net* net) {
 
 // Buffers a pass needs at once and the longest row they hold, by a dry run of the walker.
 int pool_size(vf_net* net, int start, Entry init, const std::vector<const float4*>* relax, bool ext, bool win_on,
-              bool compact, int* nb, long long* max_len) {
+              bool compact, int* nb, long long* max_len, const std::vector<float*>* sw = nullptr) {
     Walker w;
     w.net = net;
     w.s = nullptr;
@@ -641,6 +646,7 @@ int pool_size(vf_net* net, int start, Entry init, const std::vector<const float4
     w.relax = relax;
     w.win_on = win_on;
     w.compact = compact;
+    w.sw = sw;  // the same fusion decisions as the real walk
     float dummy = 0.f;
     w.ext_in = ext ? &dummy : nullptr;
     TRY(w.run(start, init));
@@ -654,7 +660,7 @@ struct IbpState {
 };
 
 int run_ibp(vf_net* net, const float* centres, int B, float eps, Arena& ar, IbpState& st, cudaStream_t s,
-            const signed char* const* split = nullptr) {
+            const signed char* const* split = nullptr, int sound = 0) {
     const size_t N = net->nodes.size();
     st.c.assign(N, nullptr);
     st.r.assign(N, nullptr);
@@ -672,20 +678,43 @@ int run_ibp(vf_net* net, const float* centres, int B, float eps, Arena& ar, IbpS
         st.r[v] = ar.take<float>(cnt);
         if (!st.c[v] || !st.r[v]) return fail(VF_ERR_WORKSPACE, "workspace too small for IBP buffers");
         const int sv = nd.src;
+        const long long cnt_src = (long long)B * net->nodes[sv].n;
+        Arena tmp = ar;  // sound mode: |c| + r of the source and |W| (|c| + r), used at once
+        float* T = sound ? tmp.take<float>(cnt_src) : nullptr;
+        float* S = sound ? tmp.take<float>(cnt) : nullptr;
+        if (sound && (!T || !S)) return fail(VF_ERR_WORKSPACE, "workspace too small for sound IBP");
         switch (nd.op) {
             case VF_DENSE:
                 LAUNCH(net, launch_ibp_dense(st.c[sv], st.r[sv], nd.W, nd.Wabs, nd.b, sv == 0 ? nd.rowsum_abs : nullptr,
                                              eps, B, (int)net->nodes[sv].n, (int)nd.n, st.c[v], st.r[v], s));
+                if (sound) {  // every dot product of K terms errs by at most gamma_K (|W| (|c| + r) + |b|)
+                    LAUNCH(net, launch_abs_plus(st.c[sv], st.r[sv], cnt_src, T, s));
+                    LAUNCH(net, launch_abs_rows_times_wt(T, nd.Wabs, B, (int)net->nodes[sv].n, (int)nd.n, S, s));
+                    LAUNCH(net, launch_sound_radius(st.r[v], S, nd.b, cnt, nd.n, 1, gamma_up(2 * net->nodes[sv].n + 64), s));
+                }
                 break;
-            case VF_CONV2D:
-                LAUNCH(net, launch_ibp_conv(st.c[sv], st.r[sv], nd.W, nd.Wabs, nd.b, B, conv_geom(net, nd), st.c[v],
-                                            st.r[v], s));
+            case VF_CONV2D: {
+                const ConvGeom g = conv_geom(net, nd);
+                LAUNCH(net, launch_ibp_conv(st.c[sv], st.r[sv], nd.W, nd.Wabs, nd.b, B, g, st.c[v], st.r[v], s));
+                if (sound) {
+                    LAUNCH(net, launch_abs_plus(st.c[sv], st.r[sv], cnt_src, T, s));
+                    LAUNCH(net, launch_ibp_conv(T, nullptr, nd.Wabs, nd.Wabs, nullptr, B, g, S, nullptr, s));
+                    LAUNCH(net, launch_sound_radius(st.r[v], S, nd.b, cnt, nd.n, (long long)g.ho * g.wo,
+                                                    gamma_up(2LL * g.ci * g.k * g.k + 64), s));
+                }
                 break;
+            }
             case VF_RELU:
-                LAUNCH(net, launch_ibp_relu(st.c[sv], st.r[sv], cnt, st.c[v], st.r[v], s, split ? split[v] : nullptr));
+                if (sound)
+                    LAUNCH(net, launch_sound_relu(st.c[sv], st.r[sv], cnt, split ? split[v] : nullptr, st.c[v], st.r[v], s));
+                else
+                    LAUNCH(net, launch_ibp_relu(st.c[sv], st.r[sv], cnt, st.c[v], st.r[v], s, split ? split[v] : nullptr));
                 break;
             case VF_ADD:
-                LAUNCH(net, launch_ibp_add(st.c[sv], st.r[sv], st.c[nd.src2], st.r[nd.src2], cnt, st.c[v], st.r[v], s));
+                if (sound)
+                    LAUNCH(net, launch_sound_add(st.c[sv], st.r[sv], st.c[nd.src2], st.r[nd.src2], cnt, st.c[v], st.r[v], s));
+                else
+                    LAUNCH(net, launch_ibp_add(st.c[sv], st.r[sv], st.c[nd.src2], st.r[nd.src2], cnt, st.c[v], st.r[v], s));
                 break;
         }
     }
@@ -714,16 +743,17 @@ int scan_finite_dev(vf_net* net, const std::vector<std::pair<const float*, long 
 // Runs every row block of one pass. `init` describes the start rows (global addressing).
 int run_pass(vf_net* net, int start, Entry init, long long rows, long long R_pass, Arena& ar,
              const std::vector<const float4*>& relax, const float* centres, float eps, float* pass_out, float* ext_in,
-             float* const_out, cudaStream_t s, const int* idx = nullptr) {
+             float* const_out, cudaStream_t s, const int* idx = nullptr, const std::vector<float*>* sw = nullptr) {
     const bool ext = ext_in != nullptr;
     const Node& sn = net->nodes[start];
-    // rows held as receptive-field windows: identity-trick passes that start at a convolution or a residual add
-    const bool win_on =
-        net->windows && !ext && init.kind == E_IDENT && (sn.op == VF_CONV2D || sn.op == VF_ADD) && sn.h > 1;
+    // rows held as receptive-field windows: identity-trick passes that start at a convolution or a residual
+    // add (not in sound mode, whose rounding budget reads plain rows)
+    const bool win_on = net->windows && !ext && sw == nullptr && init.kind == E_IDENT &&
+                        (sn.op == VF_CONV2D || sn.op == VF_ADD) && sn.h > 1;
     int nb = 0;
     long long max_len = 0;
-    TRY(pool_size(net, start, init, &relax, ext, win_on, idx != nullptr, &nb, &max_len));
-    long long nmax = (max_node_size(net, input_buffered(net)) + 31) / 32 * 32;  // 128-byte rows
+    TRY(pool_size(net, start, init, &relax, ext, win_on, idx != nullptr, &nb, &max_len, sw));
+    long long nmax = (max_node_size(net, input_buffered(net) || sw != nullptr) + 31) / 32 * 32;  // 128-byte rows
     if (win_on) nmax = std::max<long long>(32, (max_len + 31) / 32 * 32);
     int tiles = std::max(dense_back_tiles_n((int)net->nodes[0].n), dense_back_tc_tiles_n((int)net->nodes[0].n));
     for (size_t v = 1; v < net->nodes.size(); ++v)  // per-tile partials of every convolution step
@@ -753,6 +783,7 @@ int run_pass(vf_net* net, int start, Entry init, long long rows, long long R_pas
     w.n_centres = rows / R_pass;
     w.win_on = win_on;
     w.compact = idx != nullptr;
+    w.sw = sw;
     w.ps = PassStart{sn.n, sn.h, sn.w};
     for (long long m0 = 0; m0 < rows; m0 += chunk) {
         w.M = std::min(chunk, rows - m0);
@@ -795,12 +826,90 @@ int build_relax(vf_net* net, int B, const std::vector<const float*>& L, const st
 struct Bounds {
     std::vector<float*> Lw, Uw;
     std::vector<const float4*> relax;
+    // sound mode: A[v] [B, n_v], the rounding weights of node v (per unit of a row's coefficient magnitude
+    // over v's output; computed for nodes [0, a_next))
+    std::vector<float*> A;
+    int a_next = 0;
 };
+
+// Magnitude bound M_v >= |value of node v| over the box (sound bounds): from refined bounds where a node
+// feeds a ReLU, max(u, 0) of the source for a ReLU output, |c| + r from interval propagation otherwise.
+int magnitude_of(vf_net* net, int v, int B, const IbpState& st, const Bounds& bd, float* M, cudaStream_t s) {
+    const Node& nd = net->nodes[v];
+    const long long cnt = (long long)B * nd.n;
+    if (nd.op == VF_RELU && bd.Lw[nd.src] != nullptr) {
+        LAUNCH(net, launch_magnitude(bd.Lw[nd.src], bd.Uw[nd.src], cnt, 1, M, s));
+    } else if (bd.Lw[v] != nullptr) {
+        LAUNCH(net, launch_magnitude(bd.Lw[v], bd.Uw[v], cnt, 0, M, s));
+    } else {
+        LAUNCH(net, launch_abs_plus(st.c[v], st.r[v], cnt, M, s));
+    }
+    return VF_OK;
+}
+
+// Rounding weights w_v of nodes [bd.a_next, upto] (k_sound.cu states the analysis) into the arrays bd.A
+// (allocated by the caller); `scratch` holds transient vectors. A ReLU's weight needs its final bounds and
+// relaxation; other nodes' weights may use bounds refined later (earlier bounds are valid, only wider).
+int sound_weights(vf_net* net, int B, float eps, const float* centres, const IbpState& st, Bounds& bd, int upto,
+                  Arena scratch, cudaStream_t s) {
+    const float gN = gamma_up(net->total + 64);  // a row constant sums at most one term per neuron of the net
+    for (int v = bd.a_next; v <= upto; ++v) {
+        const Node& nd = net->nodes[v];
+        const long long cnt = (long long)B * nd.n;
+        float* w = bd.A[v];
+        Arena tmp = scratch;
+        switch (nd.op) {
+            case VF_INPUT:
+                LAUNCH(net, launch_input_weight(centres, eps, cnt, gamma_up(2 * nd.n + 64), w, s));
+                break;
+            case VF_DENSE:
+            case VF_CONV2D: {
+                const Node& sn = net->nodes[nd.src];
+                const long long cs = (long long)B * sn.n;
+                float* Ms = tmp.take<float>(cs);
+                float* Mv = tmp.take<float>(cnt);
+                if (!Ms || !Mv) return fail(VF_ERR_WORKSPACE, "workspace too small for rounding weights");
+                TRY(magnitude_of(net, nd.src, B, st, bd, Ms, s));
+                TRY(magnitude_of(net, v, B, st, bd, Mv, s));
+                long long kb, kf, per_channel = 1;  // terms of one backward / forward dot product
+                ConvGeom g{};
+                if (nd.op == VF_DENSE) {
+                    kb = nd.n;
+                    kf = sn.n;
+                    LAUNCH(net, launch_abs_rows_times_wt(Ms, nd.Wabs, B, (int)sn.n, (int)nd.n, w, s));
+                } else {
+                    g = conv_geom(net, nd);
+                    kb = (long long)g.co * g.k * g.k;
+                    kf = (long long)g.ci * g.k * g.k;
+                    per_channel = (long long)g.ho * g.wo;
+                    LAUNCH(net, launch_ibp_conv(Ms, nullptr, nd.Wabs, nd.Wabs, nullptr, B, g, w, nullptr, s));
+                }
+                const float gb = gamma_up(kb + 64);
+                const float gQ = nextafterf(gb * (1.f + 2.f * gamma_up(kf + 64)), INFINITY);
+                LAUNCH(net, launch_affine_weight(w, nd.b, Mv, cnt, nd.n, per_channel, gQ, gN, s));
+                break;
+            }
+            case VF_RELU:
+                LAUNCH(net, launch_relu_weight(bd.relax[v], bd.Lw[nd.src], bd.Uw[nd.src], cnt, gN, w, s));
+                break;
+            default: {  // add: the rows' sums at its sources are charged there
+                float* Mv = tmp.take<float>(cnt);
+                if (!Mv) return fail(VF_ERR_WORKSPACE, "workspace too small for rounding weights");
+                TRY(magnitude_of(net, v, B, st, bd, Mv, s));
+                LAUNCH(net, launch_scale_up(Mv, cnt, 0x1p-23f, w, s));
+                break;
+            }
+        }
+    }
+    bd.a_next = std::max(bd.a_next, upto + 1);
+    return VF_OK;
+}
 
 int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf_opts& o, Arena& ar, IbpState& st,
                    Bounds& bd, cudaStream_t s, const int* finite_flag = nullptr) {
     const int nn = (int)net->nodes.size();
-    TRY(run_ibp(net, centres, B, eps, ar, st, s, o.split));
+    const int sound = o.sound ? 1 : 0;
+    TRY(run_ibp(net, centres, B, eps, ar, st, s, o.split, sound));
     bd.Lw.assign(nn, nullptr);
     bd.Uw.assign(nn, nullptr);
     for (int v = 0; v < nn; ++v) {
@@ -810,7 +919,16 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
         bd.Lw[p] = ar.take<float>(cnt);
         bd.Uw[p] = ar.take<float>(cnt);
         if (!bd.Lw[p] || !bd.Uw[p]) return fail(VF_ERR_WORKSPACE, "workspace too small for intermediate bounds");
-        LAUNCH(net, launch_bounds_from_cr(st.c[p], st.r[p], cnt, bd.Lw[p], bd.Uw[p], s, o.split ? o.split[v] : nullptr));
+        LAUNCH(net, launch_bounds_from_cr(st.c[p], st.r[p], cnt, bd.Lw[p], bd.Uw[p], s, o.split ? o.split[v] : nullptr,
+                                          sound));
+    }
+    if (sound) {  // error weights of every node, kept for the specification pass
+        bd.A.assign(nn, nullptr);
+        bd.a_next = 0;
+        for (int v = 0; v < nn; ++v) {
+            bd.A[v] = ar.take<float>((size_t)B * net->nodes[v].n);
+            if (!bd.A[v]) return fail(VF_ERR_WORKSPACE, "workspace too small for error weights");
+        }
     }
     bd.relax.assign(nn, nullptr);
     std::vector<float4*> P(nn, nullptr);
@@ -861,6 +979,9 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
         if (nd.op != VF_RELU) continue;
         const int p = nd.src;
         const bool crown = (o.relu_crown == nullptr) || (o.relu_crown[k] != 0);
+        const bool run = crown && !exact_source(net, p) && half[p] != 0;
+        if (sound && run) TRY(sound_weights(net, B, eps, centres, st, bd, p, tmp, s));
+        const std::vector<float*>* sw = sound ? &bd.A : nullptr;
         if (crown && !exact_source(net, p) && half[p] > 0) {
             const long long np = net->nodes[p].n;
             const int hp = half[p];
@@ -870,20 +991,21 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
             Entry init;
             init.kind = E_IDENT;
             TRY(run_pass(net, p, init, (long long)B * 2 * hp, 2 * hp, tmp, bd.relax, centres, eps, pass_out, nullptr,
-                         nullptr, s, idx));
+                         nullptr, s, idx, sw));
             LAUNCH(net, launch_intersect_compact(bd.Lw[p], bd.Uw[p], pass_out, idx, B, np, hp, s));
         } else if (crown && !exact_source(net, p) && half[p] < 0) {
             Entry init;
             init.kind = E_IDENT;
             const long long np = net->nodes[p].n;
             TRY(run_pass(net, p, init, (long long)B * 2 * np, 2 * np, tmp, bd.relax, centres, eps, pass_out, nullptr,
-                         nullptr, s));
+                         nullptr, s, nullptr, sw));
             LAUNCH(net, launch_intersect(bd.Lw[p], bd.Uw[p], nullptr, nullptr, pass_out, B, np, s));
         }
         const Node& sn = net->nodes[p];
         const bool aff = sn.op == VF_DENSE || sn.op == VF_CONV2D;
         LAUNCH(net, launch_relax_params(bd.Lw[p], bd.Uw[p], o.alpha ? o.alpha[k] : nullptr, (long long)B * nd.n, P[k],
-                                        aff ? sn.b : nullptr, nd.n, sn.op == VF_CONV2D ? (long long)sn.h * sn.w : 1, s));
+                                        aff ? sn.b : nullptr, nd.n, sn.op == VF_CONV2D ? (long long)sn.h * sn.w : 1, s,
+                                        sound));
     }
     return VF_OK;
 }
@@ -1584,9 +1706,15 @@ int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const f
         TRY(scan_finite_dev(net, arrs, ar, s, &finite_flag));
     }
 
+    struct SoundScope {  // contractions take the FFMA kernels (whose rounding the error analysis models)
+        vf_net* n;
+        SoundScope(vf_net* n_, int on) : n(n_) { n->call_sound = on; }
+        ~SoundScope() { n->call_sound = 0; }
+    } scope(net, o.sound ? 1 : 0);
     IbpState st;
     Bounds bd;
     TRY(prepare_bounds(net, centres, B, eps, o, ar, st, bd, s, finite_flag));
+    if (o.sound) TRY(sound_weights(net, B, eps, centres, st, bd, last, ar, s));
     std::vector<float*>& Lw = bd.Lw;
     std::vector<float*>& Uw = bd.Uw;
     std::vector<const float4*>& relax = bd.relax;
@@ -1606,8 +1734,10 @@ int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const f
     } else {
         init.ref = RowRef{C, C_bstride, nL, R, 0};
     }
-    TRY(run_pass(net, last, init, (long long)B * Rp, Rp, ar, relax, centres, eps, pass_out, nullptr, nullptr, s));
-    LAUNCH(net, launch_spec_ibp(C, C_bstride, B, R, nL, st.c[last], st.r[last], lbI, ubI, s));
+    TRY(run_pass(net, last, init, (long long)B * Rp, Rp, ar, relax, centres, eps, pass_out, nullptr, nullptr, s,
+                 nullptr, o.sound ? &bd.A : nullptr));
+    LAUNCH(net, launch_spec_ibp(C, C_bstride, B, R, nL, st.c[last], st.r[last], lbI, ubI, s,
+                                o.sound ? gamma_up(2LL * nL + 64) : 0.f));
     LAUNCH(net, launch_decide(lbI, ubI, pass_out, B, R, o.both_sides, lb, ub, lb_ibp, verified, s));
 
     if (o.pre_lb || o.pre_ub) {
@@ -1620,7 +1750,7 @@ int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const f
             } else {
                 float* tl = o.pre_lb ? o.pre_lb + off : nullptr;
                 float* tu = o.pre_ub ? o.pre_ub + off : nullptr;
-                if (tl && tu) LAUNCH(net, launch_bounds_from_cr(st.c[v], st.r[v], cnt, tl, tu, s));
+                if (tl && tu) LAUNCH(net, launch_bounds_from_cr(st.c[v], st.r[v], cnt, tl, tu, s, nullptr, o.sound ? 1 : 0));
             }
         }
     }
@@ -1638,6 +1768,7 @@ int vf_alpha_crown(vf_net* net, const float* centres, int B, float eps, const fl
     if (!std::isfinite(eps) || eps < 0.f || !std::isfinite(lr) || lr < 0.f)
         return fail(VF_ERR_NONFINITE, "eps and lr must be finite and >= 0");
     if (o.both_sides) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation bounds the lower side; pass -C for upper");
+    if (o.sound) return fail(VF_ERR_UNSUPPORTED, "the sound-in-fp32 mode covers vf_verify_batch only");
     if (B == 0 || R == 0) return VF_OK;
     if (!affine_chain(net))
         return spec_alpha_graph(net, centres, B, eps, C, R, C_bstride, o, iters, lr, false, nullptr, nullptr, lb,
@@ -1661,6 +1792,7 @@ int vf_alpha_beta_grad(vf_net* net, const float* centres, int B, float eps, cons
     if (B < 0 || R < 0 || C_bstride < 0) return fail(VF_ERR_ARG, "negative size");
     if (!std::isfinite(eps) || eps < 0.f) return fail(VF_ERR_NONFINITE, "eps must be finite and >= 0");
     if (o.both_sides) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation bounds one side: pass -C for upper bounds");
+    if (o.sound) return fail(VF_ERR_UNSUPPORTED, "the sound-in-fp32 mode covers vf_verify_batch only");
     if (B == 0 || R == 0) return VF_OK;
     if (!affine_chain(net))
         return spec_alpha_graph(net, centres, B, eps, C, R, C_bstride, o, 0, 0.f, true, alpha, grad_alpha, lb, nullptr,

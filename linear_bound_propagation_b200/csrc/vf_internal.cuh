@@ -154,13 +154,17 @@ cudaError_t launch_ibp_add(const float* c1, const float* r1, const float* c2, co
                            float* oc, float* orad, cudaStream_t s);
 cudaError_t launch_fill(float* p, long long n, float v, cudaStream_t s);
 cudaError_t launch_bounds_from_cr(const float* c, const float* r, long long n, float* lb, float* ub, cudaStream_t s,
-                                  const signed char* split = nullptr);
+                                  const signed char* split = nullptr, int sound = 0);
+// out = A |W|^T (A [M, K], Wabs [N, K] = |W|): the radius half of the dense interval product.
+cudaError_t launch_abs_rows_times_wt(const float* A, const float* Wabs, int M, int K, int N, float* out, cudaStream_t s);
 
 // ---- relaxation, pass bookkeeping, decision (k_misc.cu) ------------------------------
 // P[i] = {lo, up, t, bias of the affine source}; bias may be null (then 0); neuron j = i % n_per_centre
 // takes bias[j / per_channel] (per_channel = H*W for a convolution, 1 for a dense node).
+// sound != 0: the intercept t is rounded up so that the upper line stays above the ReLU at both ends.
 cudaError_t launch_relax_params(const float* l, const float* u, const float* alpha, long long n, float4* P,
-                                const float* bias, long long n_per_centre, long long per_channel, cudaStream_t s);
+                                const float* bias, long long n_per_centre, long long per_channel, cudaStream_t s,
+                                int sound = 0);
 cudaError_t launch_cst_identity_bias(float* cst, long long M, PassGeom pg, const float* bias, long long n_p,
                                      long long per_channel, cudaStream_t s);
 cudaError_t launch_ident_rows(float* out, long long ld, long long M, PassGeom pg, long long n_p, int accumulate,
@@ -175,21 +179,23 @@ cudaError_t launch_finish_rows(const float* cst, const float* part, int ntiles, 
                                cudaStream_t s);
 // cst[m] += sum_{t < ntiles} part[t * M + m], in increasing t.
 cudaError_t launch_add_partials(float* cst, const float* part, int ntiles, long long M, cudaStream_t s);
+// corr (optional, [B, n]): error budget subtracted from the pass's lower bounds of +-z_j (rounded outwards).
 cudaError_t launch_intersect(float* l, float* u, const float* l_ibp, const float* u_ibp, const float* pass_out,
-                             int B, long long n, cudaStream_t s);
+                             int B, long long n, cudaStream_t s, const float* corr = nullptr);
 // Unstable-neuron compaction of an intermediate pass (IBP bounds l < 0 < u): counts[b] = number of such
 // neurons of centre b; idx[b * half + i] = the i-th of them in increasing order, -1 past the count.
 cudaError_t launch_unstable_count(const float* l, const float* u, int B, long long n, int* counts, cudaStream_t s);
 cudaError_t launch_unstable_list(const float* l, const float* u, int B, long long n, int half, int* idx, cudaStream_t s);
 // Intersection for a compacted pass: rows [e_j; -e_j] of the listed neurons, R = 2 * half rows per centre.
 cudaError_t launch_intersect_compact(float* l, float* u, const float* pass_out, const int* idx, int B, long long n,
-                                     int half, cudaStream_t s);
+                                     int half, cudaStream_t s, const float* corr = nullptr);
 // Rows +-W[j, :] (W is [n_p, n_src], row-major) for the start neurons of a compacted pass over a dense node.
 cudaError_t launch_gather_start_rows(float* out, long long ld, long long M, PassGeom pg, const float* W, long long n_p,
                                      long long n_src, cudaStream_t s);
 cudaError_t launch_spec_rows(const float* C, long long C_bstride, int BC, int R, int nL, float* S, cudaStream_t s);
+// gam > 0: sound mode, both bounds widened by gam * sum |C| (|zc| + zr) and rounded outwards.
 cudaError_t launch_spec_ibp(const float* C, long long C_bstride, int B, int R, int nL, const float* zc, const float* zr,
-                            float* lb, float* ub, cudaStream_t s);
+                            float* lb, float* ub, cudaStream_t s, float gam = 0.f);
 cudaError_t launch_decide(const float* lb_ibp, const float* ub_ibp, const float* pass_out, int B, int R, int both,
                           float* lb, float* ub, float* lb_ibp_out, uint8_t* verified, cudaStream_t s);
 cudaError_t launch_finite_scan(const float* p, long long n, int* flag, cudaStream_t s);
@@ -223,6 +229,26 @@ cudaError_t launch_zero_moments(float* beta, float* m1, float* m2, long long cou
 cudaError_t launch_alpha_init(float* alpha, float* m1, float* m2, long long M, int n, const float4* P, PassGeom pg,
                               cudaStream_t s);
 cudaError_t launch_best_update(float* best, const float* cur, long long M, int first, cudaStream_t s);
+
+// ---- sound-in-fp32 mode (k_sound.cu) ----------------------------------------------------------
+float gamma_up(long long K);
+cudaError_t launch_sound_radius(float* zr, const float* S, const float* bias, long long total, long long n,
+                                long long per_channel, float g, cudaStream_t s);
+cudaError_t launch_abs_plus(const float* c, const float* r, long long total, float* T, cudaStream_t s);
+cudaError_t launch_sound_relu(const float* c, const float* r, long long total, const signed char* split, float* oc,
+                              float* orad, cudaStream_t s);
+cudaError_t launch_sound_add(const float* c1, const float* r1, const float* c2, const float* r2, long long total,
+                             float* oc, float* orad, cudaStream_t s);
+cudaError_t launch_magnitude(const float* l, const float* u, long long total, int pos_only, float* M, cudaStream_t s);
+cudaError_t launch_input_weight(const float* c, float eps, long long total, float g0, float* w, cudaStream_t s);
+cudaError_t launch_affine_weight(float* w, const float* bias, const float* Mv, long long total, long long n,
+                                 long long per_channel, float gQ, float gN, cudaStream_t s);
+cudaError_t launch_relu_weight(const float4* P, const float* l, const float* u, long long total, float gN, float* w,
+                               cudaStream_t s);
+cudaError_t launch_scale_up(const float* M, long long total, float g, float* w, cudaStream_t s);
+// cst[m] -= sum_j |row_j| w[b, j] (rows over one node, relaxed by rx when given), rounded down.
+cudaError_t launch_row_budget(const RowRef& A, Relax rx, long long M, int n, PassGeom pg, const float* w, float* cst,
+                              cudaStream_t s);
 
 // ---- branch and bound (k_bab.cu) ------------------------------------------------------------
 // Per subdomain: the neuron to split next (search-wide index, -1 if none is unstable), whether some

@@ -46,7 +46,7 @@ class Opts(ctypes.Structure):
     _fields_ = [("relu_crown", ctypes.POINTER(ctypes.c_int)), ("alpha", ctypes.POINTER(ctypes.c_void_p)),
                 ("both_sides", ctypes.c_int), ("skip_finite_check", ctypes.c_int),
                 ("pre_lb", ctypes.c_void_p), ("pre_ub", ctypes.c_void_p), ("no_host_sync", ctypes.c_int),
-                ("split", ctypes.POINTER(ctypes.c_void_p))]
+                ("split", ctypes.POINTER(ctypes.c_void_p)), ("sound", ctypes.c_int)]
 
 
 class BabOpts(ctypes.Structure):
@@ -206,9 +206,10 @@ class Net:
     def verify(self, centres: torch.Tensor, eps: float, C: torch.Tensor, crown_relus: Optional[Sequence[int]] = None,
                alpha: Optional[Dict[int, torch.Tensor]] = None, both_sides: bool = False, want_pre: bool = False,
                skip_finite_check: bool = False, no_host_sync: bool = False, stream=None, out=None,
-               splits: Optional[Dict[int, torch.Tensor]] = None):
+               splits: Optional[Dict[int, torch.Tensor]] = None, sound: bool = False):
         """vf_verify_batch. C: [B or 1, R, n_L]. splits: ReLU node -> int8 [B, n] signs (+1: z >= 0,
-        -1: z <= 0, 0: free), one subdomain per centre row. Returns dict of device tensors."""
+        -1: z <= 0, 0: free), one subdomain per centre row. sound: bounds that hold despite fp32 rounding.
+        Returns dict of device tensors."""
         B = centres.shape[0]
         R = C.shape[1]
         dev = centres.device
@@ -236,6 +237,7 @@ class Net:
         o.both_sides = 1 if both_sides else 0
         o.skip_finite_check = 1 if skip_finite_check else 0
         o.no_host_sync = 1 if no_host_sync else 0
+        o.sound = 1 if sound else 0
         sarr = self._split_array(splits)
         if sarr is not None:
             o.split = ctypes.cast(sarr, ctypes.POINTER(ctypes.c_void_p))
