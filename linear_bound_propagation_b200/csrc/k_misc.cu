@@ -183,20 +183,14 @@ __global__ void add_partials_k(float* __restrict__ cst, const float* __restrict_
 
 // Intermediate bounds after a pass over node p (rows [I; -I] per centre): IBP-unstable neurons
 // take l = max(l, lb_j), u = min(u, -lb_{n + j}); IBP-stable ones keep their (exact) relaxation.
-// corr (optional, [B, n]): an error budget taken off both rows' lower bounds, rounded outwards.
 __global__ void intersect_k(float* __restrict__ l, float* __restrict__ u, const float* __restrict__ pass_out, int B,
-                            long long n, const float* __restrict__ corr) {
+                            long long n) {
     GRID_STRIDE(i, (long long)B * n) {
         const long long b = i / n, j = i % n;
         const float l0 = l[i], u0 = u[i];
         if (l0 < 0.f && u0 > 0.f) {
-            float lc = pass_out[b * 2 * n + j], uc = -pass_out[b * 2 * n + n + j];
-            if (corr != nullptr) {
-                lc = __fsub_rd(lc, corr[i]);
-                uc = __fadd_ru(uc, corr[i]);
-            }
-            l[i] = fmaxf(l0, lc);
-            u[i] = fminf(u0, uc);
+            l[i] = fmaxf(l0, pass_out[b * 2 * n + j]);
+            u[i] = fminf(u0, -pass_out[b * 2 * n + n + j]);
         }
     }
 }
@@ -253,20 +247,14 @@ __global__ void __launch_bounds__(256) unstable_list_k(const float* __restrict__
 
 // Intersection after a compacted pass (2 * half rows per centre: +e_j for the listed j, then -e_j).
 __global__ void intersect_compact_k(float* __restrict__ l, float* __restrict__ u, const float* __restrict__ pass_out,
-                                    const int* __restrict__ idx, int B, long long n, int half,
-                                    const float* __restrict__ corr) {
+                                    const int* __restrict__ idx, int B, long long n, int half) {
     GRID_STRIDE(e, (long long)B * half) {
         const long long b = e / half, i = e % half;
         const int j = idx[e];
         if (j < 0) continue;
         const long long k = b * n + j;
-        float lc = pass_out[b * 2 * half + i], uc = -pass_out[b * 2 * half + half + i];
-        if (corr != nullptr) {
-            lc = __fsub_rd(lc, corr[k]);
-            uc = __fadd_ru(uc, corr[k]);
-        }
-        l[k] = fmaxf(l[k], lc);
-        u[k] = fminf(u[k], uc);
+        l[k] = fmaxf(l[k], pass_out[b * 2 * half + i]);
+        u[k] = fminf(u[k], -pass_out[b * 2 * half + half + i]);
     }
 }
 
@@ -420,10 +408,10 @@ cudaError_t launch_add_partials(float* cst, const float* part, int ntiles, long 
 }
 
 cudaError_t launch_intersect(float* l, float* u, const float* l_ibp, const float* u_ibp, const float* pass_out, int B,
-                             long long n, cudaStream_t s, const float* corr) {
+                             long long n, cudaStream_t s) {
     (void)l_ibp;
     (void)u_ibp;
-    intersect_k<<<grid_for((long long)B * n, 256), 256, 0, s>>>(l, u, pass_out, B, n, corr);
+    intersect_k<<<grid_for((long long)B * n, 256), 256, 0, s>>>(l, u, pass_out, B, n);
     return cudaGetLastError();
 }
 
@@ -440,9 +428,9 @@ cudaError_t launch_unstable_list(const float* l, const float* u, int B, long lon
 }
 
 cudaError_t launch_intersect_compact(float* l, float* u, const float* pass_out, const int* idx, int B, long long n,
-                                     int half, cudaStream_t s, const float* corr) {
+                                     int half, cudaStream_t s) {
     if (B <= 0 || half <= 0) return cudaSuccess;
-    intersect_compact_k<<<grid_for((long long)B * half, 256), 256, 0, s>>>(l, u, pass_out, idx, B, n, half, corr);
+    intersect_compact_k<<<grid_for((long long)B * half, 256), 256, 0, s>>>(l, u, pass_out, idx, B, n, half);
     return cudaGetLastError();
 }
 

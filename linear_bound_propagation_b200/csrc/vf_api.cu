@@ -826,9 +826,9 @@ int build_relax(vf_net* net, int B, const std::vector<const float*>& L, const st
 struct Bounds {
     std::vector<float*> Lw, Uw;
     std::vector<const float4*> relax;
-    // sound mode: A[v] [B, n_v], the rounding weights of node v (per unit of a row's coefficient magnitude
+    // sound mode: sw[v] [B, n_v], the rounding weights of node v (per unit of a row's coefficient magnitude
     // over v's output; computed for nodes [0, a_next))
-    std::vector<float*> A;
+    std::vector<float*> sw;
     int a_next = 0;
 };
 
@@ -847,7 +847,7 @@ int magnitude_of(vf_net* net, int v, int B, const IbpState& st, const Bounds& bd
     return VF_OK;
 }
 
-// Rounding weights w_v of nodes [bd.a_next, upto] (k_sound.cu states the analysis) into the arrays bd.A
+// Rounding weights w_v of nodes [bd.a_next, upto] (k_sound.cu states the analysis) into the arrays bd.sw
 // (allocated by the caller); `scratch` holds transient vectors. A ReLU's weight needs its final bounds and
 // relaxation; other nodes' weights may use bounds refined later (earlier bounds are valid, only wider).
 int sound_weights(vf_net* net, int B, float eps, const float* centres, const IbpState& st, Bounds& bd, int upto,
@@ -856,7 +856,7 @@ int sound_weights(vf_net* net, int B, float eps, const float* centres, const Ibp
     for (int v = bd.a_next; v <= upto; ++v) {
         const Node& nd = net->nodes[v];
         const long long cnt = (long long)B * nd.n;
-        float* w = bd.A[v];
+        float* w = bd.sw[v];
         Arena tmp = scratch;
         switch (nd.op) {
             case VF_INPUT:
@@ -923,11 +923,11 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
                                           sound));
     }
     if (sound) {  // error weights of every node, kept for the specification pass
-        bd.A.assign(nn, nullptr);
+        bd.sw.assign(nn, nullptr);
         bd.a_next = 0;
         for (int v = 0; v < nn; ++v) {
-            bd.A[v] = ar.take<float>((size_t)B * net->nodes[v].n);
-            if (!bd.A[v]) return fail(VF_ERR_WORKSPACE, "workspace too small for error weights");
+            bd.sw[v] = ar.take<float>((size_t)B * net->nodes[v].n);
+            if (!bd.sw[v]) return fail(VF_ERR_WORKSPACE, "workspace too small for error weights");
         }
     }
     bd.relax.assign(nn, nullptr);
@@ -981,7 +981,7 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
         const bool crown = (o.relu_crown == nullptr) || (o.relu_crown[k] != 0);
         const bool run = crown && !exact_source(net, p) && half[p] != 0;
         if (sound && run) TRY(sound_weights(net, B, eps, centres, st, bd, p, tmp, s));
-        const std::vector<float*>* sw = sound ? &bd.A : nullptr;
+        const std::vector<float*>* sw = sound ? &bd.sw : nullptr;
         if (crown && !exact_source(net, p) && half[p] > 0) {
             const long long np = net->nodes[p].n;
             const int hp = half[p];
@@ -1735,7 +1735,7 @@ int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const f
         init.ref = RowRef{C, C_bstride, nL, R, 0};
     }
     TRY(run_pass(net, last, init, (long long)B * Rp, Rp, ar, relax, centres, eps, pass_out, nullptr, nullptr, s,
-                 nullptr, o.sound ? &bd.A : nullptr));
+                 nullptr, o.sound ? &bd.sw : nullptr));
     LAUNCH(net, launch_spec_ibp(C, C_bstride, B, R, nL, st.c[last], st.r[last], lbI, ubI, s,
                                 o.sound ? gamma_up(2LL * nL + 64) : 0.f));
     LAUNCH(net, launch_decide(lbI, ubI, pass_out, B, R, o.both_sides, lb, ub, lb_ibp, verified, s));

@@ -179,16 +179,15 @@ cudaError_t launch_finish_rows(const float* cst, const float* part, int ntiles, 
                                cudaStream_t s);
 // cst[m] += sum_{t < ntiles} part[t * M + m], in increasing t.
 cudaError_t launch_add_partials(float* cst, const float* part, int ntiles, long long M, cudaStream_t s);
-// corr (optional, [B, n]): error budget subtracted from the pass's lower bounds of +-z_j (rounded outwards).
 cudaError_t launch_intersect(float* l, float* u, const float* l_ibp, const float* u_ibp, const float* pass_out,
-                             int B, long long n, cudaStream_t s, const float* corr = nullptr);
+                             int B, long long n, cudaStream_t s);
 // Unstable-neuron compaction of an intermediate pass (IBP bounds l < 0 < u): counts[b] = number of such
 // neurons of centre b; idx[b * half + i] = the i-th of them in increasing order, -1 past the count.
 cudaError_t launch_unstable_count(const float* l, const float* u, int B, long long n, int* counts, cudaStream_t s);
 cudaError_t launch_unstable_list(const float* l, const float* u, int B, long long n, int half, int* idx, cudaStream_t s);
 // Intersection for a compacted pass: rows [e_j; -e_j] of the listed neurons, R = 2 * half rows per centre.
 cudaError_t launch_intersect_compact(float* l, float* u, const float* pass_out, const int* idx, int B, long long n,
-                                     int half, cudaStream_t s, const float* corr = nullptr);
+                                     int half, cudaStream_t s);
 // Rows +-W[j, :] (W is [n_p, n_src], row-major) for the start neurons of a compacted pass over a dense node.
 cudaError_t launch_gather_start_rows(float* out, long long ld, long long M, PassGeom pg, const float* W, long long n_p,
                                      long long n_src, cudaStream_t s);
