@@ -383,6 +383,31 @@ def run_ours(args):
                  "unit": UNIT, "ms_per_step": a_ms / args.steps, "mean_lb_gain": float(gain.mean().item()),
                  "rows_improved": float((gain > 0).float().mean().item()),
                  "note": "vf_alpha_crown: intermediate bounds as in the verify step, then per-row lower-slope Adam ascent"}
+    sound = None
+    if args.sound_steps > 0:
+        # sound-in-fp32 leg: the same verify call with vf_opts.sound (FFMA contractions, rounding budgets)
+        plain_lb = out["lb"].clone()
+        so = {k: torch.empty_like(v) for k, v in out.items()}
+        skw = dict(kw, out=so, sound=True)
+        net.verify(centres, w.eps, C, **skw)  # warm-up
+        torch.cuda.synchronize()
+        s_ms = 0.0
+        for i in range(args.sound_steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            net.verify(centres, w.eps, C, **skw)
+            e1.record(stream)
+            e1.synchronize()
+            s_ms += e0.elapsed_time(e1)
+        s_ms = max_over_ranks(s_ms, dev)
+        gap = plain_lb - so["lb"]
+        sound = {"value": weak_throughput(world, B * Rs, args.sound_steps, s_ms), "unit": UNIT,
+                 "steps": args.sound_steps, "ms_per_step": s_ms / args.sound_steps,
+                 "lb_below_plain_mean": float(gap.mean().item()), "lb_below_plain_max": float(gap.max().item()),
+                 "verified_specs": int(so["verified"].sum().item()),
+                 "note": "vf_verify_batch with vf_opts.sound: directed-rounding IBP, rounded-up intercepts and a "
+                         "per-row rounding budget at every node; FFMA contractions"}
     bab = None
     if args.bab_domains > 0 and not w.both_sides and w.C.shape[1] > 1:
         bab = bab_leg(args, w, net, centres, dev, stream, world, rank)
@@ -396,7 +421,7 @@ def run_ours(args):
                         "pipeline": "double-buffered: the H2D of step i+1 and the D2H of step i overlap compute on a "
                                     "copy stream; all copies of every step are inside the timed region"},
                 "gpu_launches": launches, "clocks": clocks, "verified_specs": verified, "total_specs": B * Rs,
-                "alpha_crown": alpha, "graph": graph, "bab": bab}
+                "alpha_crown": alpha, "graph": graph, "bab": bab, "sound": sound}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = oracle_sample(w, args.cpu_sample_s)[0]
             if bab is not None:
@@ -474,6 +499,8 @@ def main():
     ap.add_argument("--graph", action="store_true", help="also time the verify call replayed from a CUDA graph")
     ap.add_argument("--alpha-iters", type=int, default=10,
                     help="also time vf_alpha_crown with this many Adam steps (dense chains; 0 = skip)")
+    ap.add_argument("--sound-steps", type=int, default=5,
+                    help="also time the sound-in-fp32 verify call for this many steps (0 = skip)")
     ap.add_argument("--bab-domains", type=int, default=512,
                     help="also time vf_bab_verify with this budget of subdomains per centre (0 = skip)")
     ap.add_argument("--bab-centres", type=int, default=2)
