@@ -39,3 +39,16 @@ def test_every_declared_symbol_is_exported():
 def test_last_error_without_gpu_call():
     L = vf.lib()
     assert isinstance(L.vf_last_error(), bytes)
+
+
+def test_new_entry_points_reject_null_arguments_without_a_gpu():
+    """Branch and bound, the split multipliers' gradient and the node query validate their arguments on the
+    host before any device work: a NULL handle or missing option block is an error code, not a crash."""
+    L = vf.lib()
+    res = vf.BabResult()
+    o = vf.BabOpts(max_domains=10, batch=4, alpha_iters=0, lr=0.1)
+    assert L.vf_bab_verify(None, None, 0.1, None, 1, vf.ctypes.byref(o), vf.ctypes.byref(res), None) == vf.VF_ERR_ARG
+    assert b"NULL" in L.vf_last_error()
+    assert L.vf_alpha_beta_grad(None, None, 1, 0.1, None, 1, 0, None, None, None, None, None, None, None) == vf.VF_ERR_ARG
+    op = vf.ctypes.c_int()
+    assert L.vf_net_node_info(None, 0, vf.ctypes.byref(op), None, None, None) == vf.VF_ERR_ARG
