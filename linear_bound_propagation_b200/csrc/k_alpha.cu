@@ -157,6 +157,11 @@ __global__ void alpha_init_k(float* __restrict__ alpha, float* __restrict__ m1, 
     }
 }
 
+__global__ void identity_relax_k(float4* __restrict__ P, long long n) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        P[i] = make_float4(1.f, 1.f, 0.f, 0.f);
+}
+
 __global__ void best_update_k(float* __restrict__ best, const float* __restrict__ cur, long long M, int first) {
     for (long long m = blockIdx.x * (long long)blockDim.x + threadIdx.x; m < M; m += (long long)gridDim.x * blockDim.x)
         best[m] = first ? cur[m] : fmaxf(best[m], cur[m]);
@@ -202,6 +207,11 @@ cudaError_t launch_zero_moments(float* beta, float* m1, float* m2, long long cou
 cudaError_t launch_alpha_init(float* alpha, float* m1, float* m2, long long M, int n, const float4* P, PassGeom pg,
                               cudaStream_t s) {
     alpha_init_k<<<grid_for(M * n, 256), 256, 0, s>>>(alpha, m1, m2, M, n, P, pg);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_identity_relax(float4* P, long long n, cudaStream_t s) {
+    identity_relax_k<<<grid_for(n, 256), 256, 0, s>>>(P, n);
     return cudaGetLastError();
 }
 

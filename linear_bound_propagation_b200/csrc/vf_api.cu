@@ -1050,6 +1050,14 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
     }
     const long long gmax = std::max<long long>(nmax, n0);
     const long long rows = (long long)B * R;
+    // identity relaxation table [B, nmax]: the slopes are applied by relax_alpha_rows_k, so the contraction
+    // that follows may run on the tensor cores, which read every row through such a table
+    float4* ident = nullptr;
+    if (net->dense_kernel == 0 && !net->call_sound) {
+        ident = ar.take<float4>((size_t)B * nmax);
+        if (!ident) return fail(VF_ERR_WORKSPACE, "workspace too small for alpha optimisation");
+        LAUNCH(net, launch_identity_relax(ident, (long long)B * nmax, s));
+    }
     // per-row floats: H (sum_n) + Z (nmax) + lam_in (n0) + two gradient buffers (gmax) + cst + lb
     // (+ slopes and two Adam moments, 3 * sum_n, when optimising)
     int ctiles_max = 0;
@@ -1141,6 +1149,11 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
                     LAUNCH(net, launch_conv_back(RowRef{Z, 0, nu, kHugeRows, 0}, Relax{nullptr, 0}, d.W, nullptr, Mc,
                                                  conv_geom(net, d), pg, OUT_STORE, out, nd_in, cpart, nullptr, 0.f,
                                                  net->num_sms, s));
+                else if (ident != nullptr && d.WtHi != nullptr &&
+                         dense_back_tc_supported(RowRef{Z, 0, nu, kHugeRows, 0}, Relax{ident, 0}, Mc, nu, nd_in, pg))
+                    LAUNCH(net, launch_dense_back_tc(RowRef{Z, 0, nu, kHugeRows, 0}, Relax{ident, 0}, d.WtHi, d.WtLo, B,
+                                                     Mc, nu, nd_in, pg, OUT_STORE, out, nd_in, cst, nullptr, 0.f,
+                                                     nullptr, net->d_err, 0, s));
                 else
                     LAUNCH(net, launch_dense_back(RowRef{Z, 0, nu, kHugeRows, 0}, Relax{nullptr, 0}, d.W, nullptr, Mc,
                                                   nu, nd_in, pg, OUT_STORE, out, nd_in, nullptr, nullptr, 0.f, nullptr,

@@ -228,6 +228,9 @@ cudaError_t launch_zero_moments(float* beta, float* m1, float* m2, long long cou
 cudaError_t launch_alpha_init(float* alpha, float* m1, float* m2, long long M, int n, const float4* P, PassGeom pg,
                               cudaStream_t s);
 cudaError_t launch_best_update(float* best, const float* cur, long long M, int first, cudaStream_t s);
+// P[i] = {1, 1, 0, 0}: a relaxation table that passes rows through unchanged (slopes 1, no intercept, no
+// bias), so rows whose slopes were applied already can take the tensor-core contraction.
+cudaError_t launch_identity_relax(float4* P, long long n, cudaStream_t s);
 
 // ---- sound-in-fp32 mode (k_sound.cu) ----------------------------------------------------------
 float gamma_up(long long K);
