@@ -569,12 +569,15 @@ def branch_scores(l: np.ndarray, u: np.ndarray) -> np.ndarray:
     """Branching score of ReLU neurons from their pre-activation bounds (reading: the page names
     branch-and-bound only [SNNV §3, §4.3]). An unstable neuron (l < 0 < u) scores the intercept of its
     upper relaxation, -u l / (u - l), the widest vertical gap between the chord and the ReLU; a stable
-    one scores -inf and is never split."""
-    l = np.asarray(l, F)
-    u = np.asarray(u, F)
-    sc = np.full(l.shape, -np.inf)
+    one scores -inf and is never split.
+
+    The score decides an index (the neuron to split), so it is taken in the precision the device takes
+    it in: the bounds rounded to fp32 and the score evaluated in fp32 arithmetic, in the same order."""
+    l = np.asarray(l, F).astype(np.float32)
+    u = np.asarray(u, F).astype(np.float32)
+    sc = np.full(l.shape, -np.inf, np.float32)
     un = (l < 0.0) & (u > 0.0)
-    sc[un] = -u[un] * l[un] / (u[un] - l[un])
+    sc[un] = (-u[un] * l[un]) / (u[un] - l[un])
     return sc
 
 
@@ -611,7 +614,7 @@ def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_rel
     centre = np.asarray(centre, F)
     relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
     sizes = [_size(shapes(net)[net[k].src]) for k in relus]
-    y = forward(net, centre[None, :])[-1][0] @ C.T
+    y = (forward(net, centre[None, :])[-1][0] @ C.T).astype(np.float32)  # a decision: fp32, as on the device
     if np.any(y < 0.0):
         return BabResult("falsified", 0, 0, 0, float(y.min()))
 
@@ -635,7 +638,8 @@ def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_rel
                 j = int(np.argmax(sc))
                 if sc[j] > best:
                     best, choice = sc[j], (k, j)
-            out.append((float(lb[i].min()), empty, choice))
+            # the closing test and the best-first order are decisions too: taken on fp32 values
+            out.append((float(np.float32(lb[i].min())), empty, choice))
         return out
 
     (lb0, _, choice0), = evaluate([{}])
