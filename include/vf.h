@@ -233,6 +233,19 @@ typedef struct {
 int vf_bab_verify(vf_net* net, const float* centre, float eps, const float* C, int R, const vf_bab_opts* opts,
                   vf_bab_result* result /*[host]*/, void* stream);
 
+/* The search of vf_bab_verify (steps 2-5) with a caller-supplied bound function, so other bounding
+ * methods can drive it; vf_bab_verify is the centre check plus this search with the device bound function.
+ * bound(user, n, ...) bounds n subdomains: subdomain i holds split_count[i] splits, listed from
+ * split_offset[i] in split_neuron (search-wide neuron index: ReLU layers in node order, neurons in order)
+ * and split_sign (+1: z >= 0, -1: z <= 0); it writes lb[i] (lowest row bound), branch[i] (the neuron to split
+ * next, -1 if none is unstable) and empty[i] (1 if the subdomain holds no input), all [host], and returns
+ * VF_OK or an error code, which ends the search with that code. A subdomain's splits are its parent's in
+ * order, then the new one. Runs on the host only; the search itself touches no device. */
+typedef int (*vf_bab_bound_fn)(void* user, int n, const int* split_offset, const int* split_count,
+                               const int* split_neuron, const signed char* split_sign, float* lb, int* branch,
+                               int* empty);
+int vf_bab_search(vf_bab_bound_fn bound, void* user, int max_domains, int batch, vf_bab_result* result /*[host]*/);
+
 /* Synchronise `stream` and report any pending asynchronous CUDA error. */
 int vf_sync(void* stream);
 

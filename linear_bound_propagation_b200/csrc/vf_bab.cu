@@ -70,6 +70,73 @@ struct ReluLayer {
     int gbase;      // search-wide index of its first neuron
 };
 
+// Everything the device bound function needs: the handle, the options, and the round's buffers.
+struct DeviceBound {
+    vf_net* net;
+    const vf_bab_opts* opts;
+    float eps;
+    const float* C;
+    int R;
+    void* stream;
+    int nn, sum_n;
+    const std::vector<ReluLayer>* layers;
+    float *cen, *lbv, *lba, *plb, *pub;
+    signed char* spl;
+    BabPick* pick;
+    const long long* meta_off;
+    const int *meta_n, *meta_g;
+    std::vector<signed char> hsplit;
+    std::vector<BabPick> hpick;
+};
+
+// vf_bab_bound_fn on the device: one vf_verify_batch (bounds and pre-activation bounds of all n subdomains
+// with their split constraints) and, with alpha_iters, one vf_alpha_crown (slopes and split multipliers),
+// then bab_pick_k and one copy back.
+int device_bound(void* user, int n, const int* split_offset, const int* split_count, const int* split_neuron,
+                 const signed char* split_sign, float* lb, int* branch, int* empty) {
+    DeviceBound& d = *static_cast<DeviceBound*>(user);
+    const std::vector<ReluLayer>& layers = *d.layers;
+    const int nl = (int)layers.size();
+    cudaStream_t s = (cudaStream_t)d.stream;
+    d.hsplit.assign((size_t)n * d.sum_n, 0);
+    for (int i = 0; i < n; ++i)
+        for (int k = 0; k < split_count[i]; ++k) {
+            const int g = split_neuron[split_offset[i] + k];
+            int q = 0;
+            while (q + 1 < nl && layers[q + 1].gbase <= g) ++q;
+            if (g < layers[q].gbase || g >= layers[q].gbase + layers[q].n)
+                return vf::set_last_error(VF_ERR_ARG, "split neuron index out of range");
+            d.hsplit[(size_t)n * layers[q].gbase + (size_t)i * layers[q].n + (g - layers[q].gbase)] =
+                split_sign[split_offset[i] + k];
+        }
+    if (d.sum_n > 0) BAB_CU(cudaMemcpyAsync(d.spl, d.hsplit.data(), d.hsplit.size(), cudaMemcpyHostToDevice, s));
+    std::vector<const signed char*> sp(d.nn, nullptr);
+    for (const auto& L : layers) sp[L.node] = d.spl + (size_t)n * L.gbase;
+    vf_opts o{};
+    o.relu_crown = d.opts->relu_crown;
+    o.split = sp.data();
+    o.pre_lb = d.plb;
+    o.pre_ub = d.pub;
+    BAB_TRY(vf_verify_batch(d.net, d.cen, n, d.eps, d.C, d.R, 0, &o, d.lbv, nullptr, nullptr, nullptr, d.stream));
+    if (d.opts->alpha_iters > 0) {
+        vf_opts oa{};
+        oa.relu_crown = d.opts->relu_crown;
+        oa.split = sp.data();
+        BAB_TRY(vf_alpha_crown(d.net, d.cen, n, d.eps, d.C, d.R, 0, &oa, d.opts->alpha_iters, d.opts->lr, d.lba, nullptr,
+                               nullptr, d.stream));
+    }
+    BAB_CU(vf::launch_bab_pick(d.plb, d.pub, n, d.meta_off, d.meta_n, d.meta_g, nl, d.lbv,
+                               d.opts->alpha_iters > 0 ? d.lba : nullptr, d.R, d.pick, s));
+    BAB_CU(cudaMemcpyAsync(d.hpick.data(), d.pick, sizeof(BabPick) * n, cudaMemcpyDeviceToHost, s));
+    BAB_CU(cudaStreamSynchronize(s));
+    for (int i = 0; i < n; ++i) {
+        lb[i] = d.hpick[i].minlb;
+        branch[i] = d.hpick[i].best;
+        empty[i] = d.hpick[i].empty;
+    }
+    return VF_OK;
+}
+
 }  // namespace
 
 extern "C" int vf_bab_verify(vf_net* net, const float* centre, float eps, const float* C, int R,
@@ -150,78 +217,91 @@ extern "C" int vf_bab_verify(vf_net* net, const float* centre, float eps, const 
         }
     }
 
-    // ---- bound a batch of subdomains; one host synchronisation
-    std::vector<signed char> hsplit;
-    std::vector<BabPick> hpick(D);
-    auto evaluate = [&](const std::vector<const std::vector<std::pair<int, signed char>>*>& doms) -> int {
-        const int Dn = (int)doms.size();
-        hsplit.assign((size_t)Dn * sum_n, 0);
-        for (int i = 0; i < Dn; ++i)
-            for (const auto& gs : *doms[i]) {
-                int q = 0;
-                while (q + 1 < nl && layers[q + 1].gbase <= gs.first) ++q;
-                const int j = gs.first - layers[q].gbase;
-                hsplit[(size_t)Dn * layers[q].gbase + (size_t)i * layers[q].n + j] = gs.second;
+    // ---- bound a batch of subdomains on the device; one host synchronisation
+    DeviceBound db;
+    db.net = net;
+    db.opts = opts;
+    db.eps = eps;
+    db.C = C;
+    db.R = R;
+    db.stream = stream;
+    db.nn = nn;
+    db.sum_n = sum_n;
+    db.layers = &layers;
+    db.cen = cen.get<float>();
+    db.spl = spl.get<signed char>();
+    db.lbv = lbv.get<float>();
+    db.lba = lba.get<float>();
+    db.plb = plb.get<float>();
+    db.pub = pub.get<float>();
+    db.pick = pick.get<BabPick>();
+    db.meta_off = meta_off.get<long long>();
+    db.meta_n = meta_n.get<int>();
+    db.meta_g = meta_g.get<int>();
+    db.hpick.resize(D);
+    return vf_bab_search(device_bound, &db, opts->max_domains, opts->batch, result);
+}
+
+extern "C" int vf_bab_search(vf_bab_bound_fn bound, void* user, int max_domains, int batch, vf_bab_result* result) {
+    if (!bound || !result) return vf::set_last_error(VF_ERR_ARG, "NULL pointer");
+    if (max_domains < 1 || batch < 2 || batch % 2 != 0)
+        return vf::set_last_error(VF_ERR_ARG, "need max_domains >= 1 and an even batch >= 2");
+    using Splits = std::vector<std::pair<int, signed char>>;
+    std::vector<int> off, cnt, nid, br(batch), em(batch);
+    std::vector<signed char> sg;
+    std::vector<float> lb(batch);
+    auto evaluate = [&](const std::vector<const Splits*>& doms) -> int {
+        off.clear();
+        cnt.clear();
+        nid.clear();
+        sg.clear();
+        for (const Splits* d : doms) {
+            off.push_back((int)nid.size());
+            cnt.push_back((int)d->size());
+            for (const auto& p : *d) {
+                nid.push_back(p.first);
+                sg.push_back(p.second);
             }
-        if (sum_n > 0)
-            BAB_CU(cudaMemcpyAsync(spl.p, hsplit.data(), hsplit.size(), cudaMemcpyHostToDevice, s));
-        std::vector<const signed char*> sp(nn, nullptr);
-        for (const auto& L : layers) sp[L.node] = spl.get<signed char>() + (size_t)Dn * L.gbase;
-        vf_opts o{};
-        o.relu_crown = opts->relu_crown;
-        o.split = sp.data();
-        o.pre_lb = plb.get<float>();
-        o.pre_ub = pub.get<float>();
-        BAB_TRY(vf_verify_batch(net, cen.get<float>(), Dn, eps, C, R, 0, &o, lbv.get<float>(), nullptr, nullptr, nullptr,
-                                stream));
-        if (opts->alpha_iters > 0) {
-            vf_opts oa{};
-            oa.relu_crown = opts->relu_crown;
-            oa.split = sp.data();
-            BAB_TRY(vf_alpha_crown(net, cen.get<float>(), Dn, eps, C, R, 0, &oa, opts->alpha_iters, opts->lr,
-                                   lba.get<float>(), nullptr, nullptr, stream));
         }
-        BAB_CU(vf::launch_bab_pick(plb.get<float>(), pub.get<float>(), Dn, meta_off.get<long long>(), meta_n.get<int>(),
-                                   meta_g.get<int>(), nl, lbv.get<float>(),
-                                   opts->alpha_iters > 0 ? lba.get<float>() : nullptr, R, pick.get<BabPick>(), s));
-        BAB_CU(cudaMemcpyAsync(hpick.data(), pick.p, sizeof(BabPick) * Dn, cudaMemcpyDeviceToHost, s));
-        BAB_CU(cudaStreamSynchronize(s));
-        return VF_OK;
+        nid.push_back(0);  // keep the arrays non-empty
+        sg.push_back(0);
+        return bound(user, (int)doms.size(), off.data(), cnt.data(), nid.data(), sg.data(), lb.data(), br.data(),
+                     em.data());
     };
 
     // ---- 2. the whole box
-    const std::vector<std::pair<int, signed char>> none;
+    const Splits none;
     BAB_TRY(evaluate({&none}));
-    if (hpick[0].minlb > 0.f) {
+    if (lb[0] > 0.f) {
         *result = vf_bab_result{VF_BAB_VERIFIED, 1, 0, 0, INFINITY};
         return VF_OK;
     }
-    if (hpick[0].best < 0) {
-        *result = vf_bab_result{VF_BAB_UNKNOWN, 1, 0, 0, hpick[0].minlb};
+    if (br[0] < 0) {
+        *result = vf_bab_result{VF_BAB_UNKNOWN, 1, 0, 0, lb[0]};
         return VF_OK;
     }
     std::vector<Domain> open;
-    open.push_back(Domain{hpick[0].minlb, 0, {}, hpick[0].best});
+    open.push_back(Domain{lb[0], 0, {}, br[0]});
     long long domains = 1, seq = 1;
     int rounds = 0, depth = 0;
 
     // ---- 3-5. rounds of splitting
     while (!open.empty()) {
-        const long long take = std::min<long long>({(long long)open.size(), (long long)D / 2,
-                                                    (opts->max_domains - domains) / 2});
+        const long long take =
+            std::min<long long>({(long long)open.size(), (long long)batch / 2, (max_domains - domains) / 2});
         if (take <= 0) break;
         std::sort(open.begin(), open.end(),
                   [](const Domain& a, const Domain& b) { return a.lb < b.lb || (a.lb == b.lb && a.seq < b.seq); });
         std::vector<Domain> parents(open.begin(), open.begin() + take);
         open.erase(open.begin(), open.begin() + take);
-        std::vector<std::vector<std::pair<int, signed char>>> children;
+        std::vector<Splits> children;
         children.reserve(2 * take);
         for (const Domain& p : parents)
             for (signed char sign : {(signed char)-1, (signed char)1}) {
                 children.push_back(p.splits);
                 children.back().push_back({p.branch, sign});
             }
-        std::vector<const std::vector<std::pair<int, signed char>>*> ptrs;
+        std::vector<const Splits*> ptrs;
         for (const auto& c : children) ptrs.push_back(&c);
         BAB_TRY(evaluate(ptrs));
         domains += (long long)children.size();
@@ -229,13 +309,12 @@ extern "C" int vf_bab_verify(vf_net* net, const float* centre, float eps, const 
         for (size_t i = 0; i < children.size(); ++i) {
             depth = std::max(depth, (int)children[i].size());
             const long long num = seq++;
-            const BabPick& pk = hpick[i];
-            if (pk.empty || pk.minlb > 0.f) continue;
-            if (pk.best < 0) {
-                *result = vf_bab_result{VF_BAB_UNKNOWN, domains, rounds, depth, pk.minlb};
+            if (em[i] || lb[i] > 0.f) continue;
+            if (br[i] < 0) {
+                *result = vf_bab_result{VF_BAB_UNKNOWN, domains, rounds, depth, lb[i]};
                 return VF_OK;
             }
-            open.push_back(Domain{pk.minlb, num, std::move(children[i]), pk.best});
+            open.push_back(Domain{lb[i], num, std::move(children[i]), br[i]});
         }
     }
     if (open.empty()) {

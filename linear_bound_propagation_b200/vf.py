@@ -26,7 +26,7 @@ SYMBOLS = ["vf_net_create", "vf_net_destroy", "vf_net_node_size", "vf_net_total_
            "vf_crown_backward", "vf_concretize", "vf_verify_batch", "vf_sync", "vf_last_error",
            "vf_profile_enable", "vf_profile_read", "vf_launch_count", "vf_net_check",
            "vf_concretize_dense_noalloc", "vf_alpha_crown", "vf_alpha_grad", "vf_alpha_beta_grad",
-           "vf_net_node_info", "vf_bab_verify"]
+           "vf_net_node_info", "vf_bab_verify", "vf_bab_search"]
 NOALLOC_SCRATCH_FLOATS = 1 << 22
 
 
@@ -61,6 +61,9 @@ class BabResult(ctypes.Structure):
 
 
 BAB_STATUS = {1: "verified", -1: "falsified", 0: "unknown"}
+BOUND_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                            ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_byte),
+                            ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int))
 
 
 _lib = None
@@ -97,6 +100,7 @@ def lib() -> ctypes.CDLL:
     L.vf_alpha_beta_grad.argtypes = [P, P, I, F, P, I, LL, ctypes.POINTER(Opts), P, P, P, P, P, P]
     L.vf_net_node_info.argtypes = [P, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(LL)]
     L.vf_bab_verify.argtypes = [P, P, F, P, I, ctypes.POINTER(BabOpts), ctypes.POINTER(BabResult), P]
+    L.vf_bab_search.argtypes = [BOUND_FN, P, I, I, ctypes.POINTER(BabResult)]
     L.vf_launch_count.argtypes = [P]
     L.vf_launch_count.restype = LL
     _lib = L
@@ -410,6 +414,34 @@ def concretize_dense_noalloc(lam: torch.Tensor, W: torch.Tensor, b: torch.Tensor
     _check(lib().vf_concretize_dense_noalloc(_ptr(lam), bstride, R, _ptr(W), _ptr(b), _ptr(centres), float(eps), B,
                                              n_in, n_out, _ptr(out), _stream_ptr(stream)))
     return out
+
+
+def bab_search(evaluate, max_domains: int, batch: int):
+    """vf_bab_search with a Python bound function: evaluate(list of subdomains, each a dict neuron -> sign in
+    the order its splits were made) -> one (lowest row bound, holds no input, neuron to split next or None)
+    per subdomain. Returns dict(status, domains, rounds, max_depth, lb). Runs on the host."""
+    err = []
+
+    def cb(user, n, off, cnt, nid, sg, lb, branch, empty):
+        try:
+            doms = [{nid[off[i] + k]: sg[off[i] + k] for k in range(cnt[i])} for i in range(n)]
+            for i, (l, e, b) in enumerate(evaluate(doms)):
+                lb[i] = l
+                branch[i] = -1 if b is None else int(b)
+                empty[i] = 1 if e else 0
+            return VF_OK
+        except Exception as ex:  # reported after the call returns
+            err.append(ex)
+            return VF_ERR_ARG
+
+    fn = BOUND_FN(cb)
+    r = BabResult()
+    code = lib().vf_bab_search(fn, None, max_domains, batch, ctypes.byref(r))
+    if err:
+        raise err[0]
+    _check(code)
+    return {"status": BAB_STATUS[r.status], "domains": r.domains, "rounds": r.rounds, "max_depth": r.max_depth,
+            "lb": r.lb}
 
 
 def sync(stream=None):

@@ -642,6 +642,13 @@ def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_rel
             out.append((float(np.float32(lb[i].min())), empty, choice))
         return out
 
+    return bab_search(evaluate, max_domains, batch)
+
+
+def bab_search(evaluate, max_domains: int, batch: int) -> BabResult:
+    """Steps 2-5 of ``bab`` with any bound function: evaluate(list of subdomains) -> one (lowest row bound,
+    holds no input, neuron to split next or None) per subdomain. A subdomain is a dict neuron -> sign in
+    the order its splits were made (its parent's, then the new one)."""
     (lb0, _, choice0), = evaluate([{}])
     if lb0 > 0.0:
         return BabResult("verified", 1, 0, 0, np.inf)
