@@ -28,12 +28,12 @@ Parity status per function (what pins it, all in tests/test_oracle_*.py):
   split_clamp, splits in ibp / verify,  -- pinned (soundness on the subdomain by sampling, the
   beta in spec_bound_alpha / alpha_crown   full-split affine closed form, weak and strong LP
                                            duality, central differences for beta)
-  branch_scores, bab                    -- pinned (exact 2-D ranges and sampling: never a wrong
+  branch_scores, bab, bab_search        -- pinned (exact 2-D ranges and sampling: never a wrong
                                            "verified" or "falsified"; splitting verifies
                                            properties the whole-box bound leaves open)
 """
 from .lbp import (  # noqa: F401
     shapes, conv2d, conv2d_adjoint, forward, ibp, relax_params, backward, concretize,
     crown_pass, verify, OracleResult, spec_bound_alpha, alpha_crown, split_clamp, branch_scores, bab,
-    BabResult,
+    bab_search, BabResult,
 )
