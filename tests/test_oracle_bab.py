@@ -284,3 +284,24 @@ def test_split_mutation_is_caught(monkeypatch, fname, old, new, check):
     except Exception:
         ok = False
     assert not ok, f"{check.__name__} did not catch {old!r} -> {new!r}"
+
+
+def test_every_subdomain_bound_takes_the_requested_ascent_steps(monkeypatch):
+    """Regression: the search's bound for every subdomain, the whole box and every child alike, runs
+    alpha_crown with the requested number of Adam steps (a loop counter once shadowed it)."""
+    seen = []
+    real = O.alpha_crown
+
+    def spy(*a, **kw):
+        seen.append(kw.get("iters"))
+        return real(*a, **kw)
+
+    monkeypatch.setattr(O, "alpha_crown", spy)
+    rng = np.random.default_rng(0)
+    net = synth.mlp([4, 10, 10, 3], rng)
+    c = rng.random(4).astype(np.float32)
+    y = O.forward(net, c[None].astype(np.float64))[-1][0]
+    C = synth.margin_spec(np.array([int(np.argmax(y))]), 3)[0]
+    r = O.bab(net, c, float(np.float32(0.2)), C, max_domains=40, batch=8, iters=7, lr=0.1)
+    assert r.iterations >= 2 and len(seen) == r.iterations + 1
+    assert set(seen) == {7}
