@@ -21,6 +21,7 @@ import pytest
 import oracle.lbp as O
 from linear_bound_propagation_b200 import synth
 from tests._helpers import box_samples, exact_range_2d, net_from_layers, relu_ids
+from tests._random_nets import random_mlp, random_net
 
 
 def _signs_at(net, x, frac, rng):
@@ -305,3 +306,33 @@ def test_every_subdomain_bound_takes_the_requested_ascent_steps(monkeypatch):
     r = O.bab(net, c, float(np.float32(0.2)), C, max_domains=40, batch=8, iters=7, lr=0.1)
     assert r.iterations >= 2 and len(seen) == r.iterations + 1
     assert set(seen) == {7}
+
+
+@pytest.mark.parametrize("seed", list(range(12)))
+def test_split_bounds_sound_on_random_architectures(seed):
+    """Subdomain soundness of split-constrained bounds (both sides, every intermediate bound) on the random
+    CNN / residual / dense networks of the GPU fuzz suite: every sampled input that satisfies the splits
+    stays inside every bound."""
+    net = random_net(seed)[0] if seed % 2 == 0 else random_mlp(seed)[0]
+    rng = np.random.default_rng(60_000 + seed)
+    n0 = int(np.prod(net[0].shape))
+    classes = int(net[-1].W.shape[0])
+    eps = float(np.float32(rng.choice([0.01, 0.05])))
+    c = rng.random(n0).astype(np.float32)
+    x0 = c + eps * (2 * rng.random(n0) - 1)
+    sp = _signs_at(net, x0, 0.3, rng)
+    C = synth.margin_spec(np.array([int(rng.integers(0, classes))]), classes)
+    res = O.verify(net, c[None], eps, C, both_sides=True, splits={k: s[None] for k, s in sp.items()})
+    xs = np.concatenate([box_samples(c, eps, 3000, 300, rng), x0[None, :]])
+    outs = O.forward(net, xs)
+    keep = np.ones(xs.shape[0], bool)
+    for k, s in sp.items():
+        keep &= np.all((s[None, :] == 0) | (s[None, :] * outs[net[k].src] >= 0.0), axis=1)
+    assert keep[-1], "the point the splits were taken from lies in the subdomain"
+    y = outs[-1][keep] @ C[0].astype(np.float64).T
+    tol = 1e-9 * (1 + np.abs(y).max())
+    assert np.all(y >= res.lb[0] - tol) and np.all(y <= res.ub[0] + tol)
+    for k in relu_ids(net):
+        z = outs[net[k].src][keep]
+        l, u = res.pre_bounds[k]
+        assert np.all(z >= l[0] - tol) and np.all(z <= u[0] + tol), f"relu {k}"
