@@ -336,3 +336,29 @@ def test_split_bounds_sound_on_random_architectures(seed):
         z = outs[net[k].src][keep]
         l, u = res.pre_bounds[k]
         assert np.all(z >= l[0] - tol) and np.all(z <= u[0] + tol), f"relu {k}"
+
+
+@pytest.mark.parametrize("seed", list(range(6)))
+def test_beta_gradient_central_differences_on_random_architectures(seed):
+    """d lb / d beta against central differences on random CNN / residual / dense networks, for a seeded
+    sample of (row, split neuron) pairs of every ReLU layer with splits."""
+    net = random_net(seed)[0] if seed % 2 == 0 else random_mlp(seed)[0]
+    rng = np.random.default_rng(70_000 + seed)
+    n0 = int(np.prod(net[0].shape))
+    classes = int(net[-1].W.shape[0])
+    eps = float(np.float32(0.03))
+    c = rng.random(n0).astype(np.float32)
+    x0 = c + eps * (2 * rng.random(n0) - 1)
+    sp = _signs_at(net, x0, 0.4, rng)
+    C = synth.margin_spec(np.array([int(rng.integers(0, classes))]), classes)
+    res = O.verify(net, c[None], eps, C, splits={k: s[None] for k, s in sp.items()})
+    relax = {k: O.relax_params(res.pre_bounds[k][0][0], res.pre_bounds[k][1][0]) for k in relu_ids(net)}
+    R = C.shape[1]
+    a = {k: rng.random((R, relax[k][0].size)) for k in relax}
+    beta = {k: rng.exponential(0.5, (R, sp[k].size)) for k in sp}
+    pairs = [(k, int(r), int(i)) for k in sp for i in rng.permutation(np.nonzero(sp[k])[0])[:4]
+             for r in rng.permutation(R)[:2]]
+    if not pairs:
+        pytest.skip("no split neuron drawn")
+    ok, det = _fd_beta(net, c, eps, C[0], relax, a, sp, beta, pairs)
+    assert ok, det
