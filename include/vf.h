@@ -143,9 +143,10 @@ typedef struct {
      * rigorous budget for its own rounding, so lb never exceeds the exact-arithmetic minimum over the
      * box (technical summary, section 4.2: soundness as a one-sided over-approximation). Interval ends
      * are rounded outwards with a gamma_K = K u / (1 - K u) term per dot product of K terms; the ReLU
-     * intercept is rounded up; each back-substituted row's result is lowered by |row| . A, where A is a
-     * per-centre error-weight vector accumulated forward through |W|, the ReLU slopes and the node's
-     * rounding weights. Contractions take the FFMA kernels (IEEE rounding), not the tensor cores. */
+     * intercept is rounded up; at every node a back-substituted row passes, its constant is lowered by
+     * sum_i |row_i| w_i, with w that node's rounding weights (contraction gamma_K |W| M, bias, relaxation and
+     * intercept terms, concretisation), rounded down. Contractions take the FFMA kernels (IEEE rounding),
+     * not the tensor cores; receptive-field windows and the fused concretisation are off. */
     int sound;
 } vf_opts;
 
