@@ -2,9 +2,12 @@
 """Throughput benchmark: verified specs/sec of one full bound-propagation step on B200.
 
 A step is one vf_verify_batch call over the whole batch: IBP over every node, CROWN passes
-for the intermediate bounds, the specification pass and the decision. Default workload:
-ReLU MLP 784-256-256-256-10, 1024 centres, eps = 2/255, 9 margin rows per centre, CROWN
-intermediate bounds for z2 and z3 (synthetic, seeded; see linear_bound_propagation_b200.synth).
+for the intermediate bounds, the specification pass and the decision. Headline workload:
+ReLU MLP 3072-(1024 x 8)-100, 4096 centres, eps = 1/255, 99 margin rows per centre, IBP
+intermediate bounds for z1..z6 and CROWN for z7, z8 and the output (synthetic, seeded; see
+linear_bound_propagation_b200.synth). The same line carries that network at eps 0.5/255 and
+2/255 (`eps_sweep`) and the other four workloads (`workloads`: value, ms per step, the
+dominant kernel's roofline and the oracle's CPU baseline each).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1..5]
 
@@ -64,9 +67,14 @@ def workload_config(w, cfg):
 
 
 def oracle_sample(w, target_s):
-    """Time the oracle on the first n centres of the workload, n sized to about target_s seconds."""
+    """Time the oracle on the first n centres of the workload, n sized to about target_s seconds.
+    Workloads whose single centre already takes minutes on the host (the residual network: 148,480
+    intermediate-pass rows per centre) are timed on a row sample of one centre instead (see
+    oracle_row_sample)."""
     import oracle.lbp as O
     R = w.C.shape[1] * (2 if w.both_sides else 1)
+    if intermediate_rows(w) > 20000:
+        return oracle_row_sample(w)
 
     def run(n):
         t0 = time.perf_counter()
@@ -80,6 +88,64 @@ def oracle_sample(w, target_s):
     t = run(n) if n > 1 else t1
     return {"value": n * R / t, "unit": UNIT, "cores": threads_used(), "kind": "oracle",
             "sample": f"first {n} of {B} centres of {w.name} ({n * R} specs), fp64 numpy oracle, {t:.2f} s"}, n, t
+
+
+def crown_passes(w):
+    """(relu node, pre-activation node, neurons) of every intermediate CROWN pass the oracle runs."""
+    import oracle.lbp as O
+    sh = O.shapes(w.net)
+    relus = [v for v, nd in enumerate(w.net) if nd.op == "relu"]
+    sel = set(relus if w.crown_relus is None else w.crown_relus)
+    out = []
+    for k in relus:
+        p = w.net[k].src
+        first_affine = w.net[p].op in ("dense", "conv") and w.net[p].src == 0
+        if k in sel and not first_affine:
+            out.append((k, p, int(np.prod(sh[p]))))
+    return out
+
+
+def intermediate_rows(w):
+    return sum(2 * n for _, _, n in crown_passes(w))
+
+
+def oracle_row_sample(w, rows_per_pass=32):
+    """The oracle's per-centre time on one centre, from its own functions: the IBP pass and the
+    specification pass in full, and for every intermediate pass the first rows_per_pass / 2 rows of
+    [I] and of [-I] through crown_pass, scaled to the pass's 2n rows. A pass's cost is linear in its
+    rows (rows are independent and each takes the same operations), and the relaxation values do not
+    change the work, so the earlier layers' relaxations are taken from the IBP bounds."""
+    import oracle.lbp as O
+    R = w.C.shape[1] * (2 if w.both_sides else 1)
+    c = w.centres[:1]
+    t0 = time.perf_counter()
+    cs, rs = O.ibp(w.net, c, w.eps)
+    t_ibp = time.perf_counter() - t0
+    relax = {}
+    relus = [v for v, nd in enumerate(w.net) if nd.op == "relu"]
+    passes = {k: (p, n) for k, p, n in crown_passes(w)}
+    t_passes, sampled = 0.0, 0
+    for k in relus:
+        p = w.net[k].src
+        if k in passes:
+            n = passes[k][1]
+            h = min(n, rows_per_pass // 2)
+            eye = np.eye(n)[:h]
+            t0 = time.perf_counter()
+            O.crown_pass(w.net, p, np.concatenate([eye, -eye]), relax, c[0], w.eps)
+            t_passes += (time.perf_counter() - t0) * (2 * n) / (2 * h)
+            sampled += 2 * h
+        relax[k] = O.relax_params(cs[p][0] - rs[p][0], cs[p][0] + rs[p][0])
+    Cb = w.C[0]
+    rows = np.concatenate([Cb, -Cb]) if w.both_sides else Cb
+    t0 = time.perf_counter()
+    O.crown_pass(w.net, len(w.net) - 1, rows, relax, c[0], w.eps)
+    t_spec = time.perf_counter() - t0
+    t = t_ibp + t_passes + t_spec
+    return {"value": R / t, "unit": UNIT, "cores": threads_used(), "kind": "oracle",
+            "sample": f"one centre of {w.name}: IBP and the {R}-row specification pass in full, and {sampled} of "
+                      f"the {intermediate_rows(w)} intermediate-pass rows ({rows_per_pass} per pass) scaled "
+                      f"linearly to each pass's rows; {t:.1f} s per centre, fp64 numpy oracle"}, 1, t
 
 
 def start_clocks():
@@ -203,13 +269,18 @@ def run_reference(args):
     base, n, t = oracle_sample(w, per_step_s)
     R = w.C.shape[1] * (2 if w.both_sides else 1)
     import oracle.lbp as O
+    row_sampled = intermediate_rows(w) > 20000
     times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        O.verify(w.net, w.centres[:n], w.eps, w.C[:n] if w.C.shape[0] > 1 else w.C, crown_relus=w.crown_relus,
-                 both_sides=w.both_sides)
+        if row_sampled:  # one centre's time from a row sample (see oracle_row_sample)
+            dt = oracle_row_sample(w)[2]
+        else:
+            O.verify(w.net, w.centres[:n], w.eps, w.C[:n] if w.C.shape[0] > 1 else w.C, crown_relus=w.crown_relus,
+                     both_sides=w.both_sides)
+            dt = time.perf_counter() - t0
         if i >= args.warmup:
-            times.append(time.perf_counter() - t0)
+            times.append(dt)
     value = n * R * len(times) / sum(times)
     base["value"] = value
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
@@ -223,7 +294,6 @@ def run_reference(args):
 def run_ours(args):
     import torch
     import torch.distributed as dist
-    from linear_bound_propagation_b200 import vf
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -232,16 +302,56 @@ def run_ours(args):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    ctx = {"world": world, "rank": rank, "dev": dev,
+           "flush": torch.empty(L2_FLUSH_BYTES // 4, device=dev)}
+
+    # the headline: the configured workload at its own radius, every step timed, with the e2e leg
+    line = measure_workload(args, ctx, args.config, None, args.steps, args.warmup, headline=True)
+    if args.eps_sweep and args.config == 5:
+        # the same network and batch at the other two radii of the benchmark definition
+        sweep = []
+        for e in (0.5 / 255.0, 2.0 / 255.0):
+            sweep.append(measure_workload(args, ctx, 5, e, min(args.steps, args.sub_steps), min(args.warmup, 3),
+                                          headline=False))
+        if line is not None:
+            line["eps_sweep"] = sweep
+    if args.all_workloads:
+        subs = {}
+        for cfg in (1, 2, 3, 4, 5):
+            if cfg == args.config:
+                continue
+            subs[synth.WORKLOAD_NAMES[cfg]] = measure_workload(
+                args, ctx, cfg, None, min(args.steps, args.sub_steps), min(args.warmup, 3), headline=False,
+                legs=(cfg == 2))
+        if line is not None:
+            line["workloads"] = subs
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def measure_workload(args, ctx, cfg, eps, steps, warmup, headline, legs=None):
+    """Time `steps` vf_verify_batch calls on workload `cfg` (radius `eps`, or the workload's own). The
+    headline adds the end-to-end leg, the clocks and the launch count; `legs` the alpha-CROWN, sound and
+    branch-and-bound legs. Returns the JSON object on rank 0 (None elsewhere)."""
+    import torch
+    import torch.distributed as dist
+    from linear_bound_propagation_b200 import vf
+
+    world, rank, dev, flush = ctx["world"], ctx["rank"], ctx["dev"], ctx["flush"]
+    if legs is None:
+        legs = headline and cfg == 2
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    w = synth.workload(args.config, B=args.centres)
+    w = synth.workload(cfg, B=args.centres if headline else None, eps=eps)
     B, R = w.centres.shape[0], w.C.shape[1]
     Rs = R * (2 if w.both_sides else 1)
     net = vf.Net(w.net, workspace_bytes=int(args.workspace_gb * (1 << 30)))
-    dev = torch.device("cuda", local)
     centres = torch.from_numpy(w.centres).to(dev)
     C = torch.from_numpy(w.C).to(dev)
     stream = torch.cuda.current_stream()
@@ -249,10 +359,9 @@ def run_ours(args):
            "verified": torch.empty(B, R, device=dev, dtype=torch.uint8)}
     if w.both_sides:
         out["ub"] = torch.empty(B, R, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev)
     kw = dict(crown_relus=w.crown_relus, both_sides=w.both_sides, out=out)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         net.verify(centres, w.eps, C, **kw)
     torch.cuda.synchronize()
     barrier()
@@ -262,8 +371,8 @@ def run_ours(args):
     launches0 = net.launch_count()
     net.profile(True)
     net.profile_read(reset=True)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
         flush.zero_()
         ev[i][0].record(stream)
         net.verify(centres, w.eps, C, **kw)
@@ -279,12 +388,55 @@ def run_ours(args):
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = float(sum(step_ms))
     total_ms = max_over_ranks(total_ms, dev)
-    value = weak_throughput(world, B * Rs, args.steps, total_ms)
+    value = weak_throughput(world, B * Rs, steps, total_ms)
     verified = int(out["verified"].sum().item())
+    roof = roofline(kstats, total_ms, torch.cuda.get_device_properties(dev).multi_processor_count,
+                    w.name if (args.centres is None or not headline) else None)
 
-    # End to end through the public API with host buffers, every step's copies inside the timed region:
-    # pinned H2D of the step's centres and C, the verify call, D2H of lb and verified. Two buffer sets and a
-    # copy stream: the H2D of step i+1 and the D2H of step i run while step i+1 / i+2 compute.
+    e2e = None
+    if headline and not args.no_e2e:
+        e2e = e2e_leg(args, w, net, centres, C, out, kw, stream, flush, dev, world, steps)
+    graph = graph_leg(args, w, net, centres, C, stream, flush, dev, world, steps, warmup, B * Rs) \
+        if (headline and args.graph) else None
+    alpha = sound = bab = None
+    if legs:
+        alpha = alpha_leg(args, w, net, centres, C, stream, flush, dev, world, steps)
+        sound = sound_leg(args, w, net, centres, C, out, kw, stream, flush, dev, world, B * Rs)
+        if args.bab_domains > 0 and not w.both_sides and w.C.shape[1] > 1:
+            bab = bab_leg(args, w, net, centres, dev, stream, world, rank)
+    net.close()
+    del net
+    torch.cuda.empty_cache()
+    if rank != 0:
+        return None
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+            "warmup": warmup, "ms_per_step": total_ms / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(w, cfg), "roofline": roof, "gpu_launches": launches, "clocks": clocks,
+            "verified_specs": verified, "total_specs": B * Rs}
+    if headline:
+        line["e2e"] = e2e
+        line["graph"] = graph
+    if legs:
+        line.update({"alpha_crown": alpha, "bab": bab, "sound": sound})
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(w, args.cpu_sample_s if headline else args.sub_cpu_sample_s)[0]
+        if bab is not None:
+            line["cpu_baseline"]["bab"] = oracle_bab_sample(args, w, bab["label0"])
+    if not headline:  # sub-lines keep only what identifies and measures them
+        for k in ("metric", "unit", "n_gpus", "higher_is_better", "scaling", "vs_baseline", "dtype", "data"):
+            line.pop(k, None)
+    return line
+
+
+def e2e_leg(args, w, net, centres, C, out, kw, stream, flush, dev, world, steps):
+    """End to end through the public API with host buffers, every step's copies inside the timed region:
+    pinned H2D of the step's centres and C, the verify call, D2H of lb and verified. Two buffer sets and a
+    copy stream: the H2D of step i+1 and the D2H of step i run while step i+1 / i+2 compute."""
+    import torch
+    import torch.distributed as dist
+    B, R = w.centres.shape[0], w.C.shape[1]
+    Rs = R * (2 if w.both_sides else 1)
     h_centres = torch.from_numpy(w.centres).pin_memory()
     h_C = torch.from_numpy(w.C).pin_memory()
     h_lb = [torch.empty(B, R).pin_memory() for _ in range(2)]
@@ -330,106 +482,94 @@ def run_ours(args):
         torch.cuda.synchronize()
         return t0.elapsed_time(t1)
 
-    if not args.no_e2e:
-        e2e_run(2)
+    e2e_run(2)
     torch.cuda.synchronize()
-    barrier()
-    e2e_ms = 0.0 if args.no_e2e else e2e_run(args.steps)
-    e2e_ms = max_over_ranks(e2e_ms, dev)
-    h2d = h_centres.numel() * 4 + h_C.numel() * 4
-    d2h = h_lb[0].numel() * 4 + h_ver[0].numel()
-
-    graph = None
-    if args.graph:
-        # the same verify call captured once in a CUDA graph (no host synchronisation inside) and replayed
-        vg = vf.VerifyGraph(net, centres, w.eps, C, crown_relus=w.crown_relus, both_sides=w.both_sides)
-        for _ in range(args.warmup):
-            vg.replay()
-        torch.cuda.synchronize()
-        g_ms = 0.0
-        for i in range(args.steps):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            vg.replay()
-            e1.record(stream)
-            e1.synchronize()
-            g_ms += e0.elapsed_time(e1)
-        g_ms = max_over_ranks(g_ms, dev)
-        graph = {"value": weak_throughput(world, B * Rs, args.steps, g_ms), "unit": UNIT,
-                 "ms_per_step": g_ms / args.steps,
-                 "note": "vf.VerifyGraph: the verify call captured in a CUDA graph and replayed (no NaN/Inf scan, "
-                         "no unstable-neuron compaction)"}
-        del vg
-    roof = roofline(kstats, total_ms, torch.cuda.get_device_properties(dev).multi_processor_count,
-                    w.name if args.centres is None else None)
-    alpha = None
-    if args.alpha_iters > 0 and not w.both_sides:
-        # alpha-CROWN leg: the same workload, intermediate bounds as above, then per-row slope optimisation
-        net.alpha_crown(centres, w.eps, C, iters=args.alpha_iters, crown_relus=w.crown_relus)  # warm-up
-        torch.cuda.synchronize()
-        a_ms = 0.0
-        for i in range(args.steps):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            res = net.alpha_crown(centres, w.eps, C, iters=args.alpha_iters, crown_relus=w.crown_relus)
-            e1.record(stream)
-            e1.synchronize()
-            a_ms += e0.elapsed_time(e1)
-        a_ms = max_over_ranks(a_ms, dev)
-        gain = (res["lb"] - res["lb_start"])
-        alpha = {"iters": args.alpha_iters, "lr": 0.1, "value": weak_throughput(world, B * R, args.steps, a_ms),
-                 "unit": UNIT, "ms_per_step": a_ms / args.steps, "mean_lb_gain": float(gain.mean().item()),
-                 "rows_improved": float((gain > 0).float().mean().item()),
-                 "note": "vf_alpha_crown: intermediate bounds as in the verify step, then per-row lower-slope Adam ascent"}
-    sound = None
-    if args.sound_steps > 0:
-        # sound-in-fp32 leg: the same verify call with vf_opts.sound (FFMA contractions, rounding budgets)
-        plain_lb = out["lb"].clone()
-        so = {k: torch.empty_like(v) for k, v in out.items()}
-        skw = dict(kw, out=so, sound=True)
-        net.verify(centres, w.eps, C, **skw)  # warm-up
-        torch.cuda.synchronize()
-        s_ms = 0.0
-        for i in range(args.sound_steps):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            net.verify(centres, w.eps, C, **skw)
-            e1.record(stream)
-            e1.synchronize()
-            s_ms += e0.elapsed_time(e1)
-        s_ms = max_over_ranks(s_ms, dev)
-        gap = plain_lb - so["lb"]
-        sound = {"value": weak_throughput(world, B * Rs, args.sound_steps, s_ms), "unit": UNIT,
-                 "steps": args.sound_steps, "ms_per_step": s_ms / args.sound_steps,
-                 "lb_below_plain_mean": float(gap.mean().item()), "lb_below_plain_max": float(gap.max().item()),
-                 "verified_specs": int(so["verified"].sum().item()),
-                 "note": "vf_verify_batch with vf_opts.sound: directed-rounding IBP, rounded-up intercepts and a "
-                         "per-row rounding budget at every node; FFMA contractions"}
-    bab = None
-    if args.bab_domains > 0 and not w.both_sides and w.C.shape[1] > 1:
-        bab = bab_leg(args, w, net, centres, dev, stream, world, rank)
-    if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": workload_config(w, args.config), "roofline": roof,
-                "e2e": None if args.no_e2e else {"value": weak_throughput(world, B * Rs, args.steps, e2e_ms), "unit": UNIT,
-                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                        "pipeline": "double-buffered: the H2D of step i+1 and the D2H of step i overlap compute on a "
-                                    "copy stream; all copies of every step are inside the timed region"},
-                "gpu_launches": launches, "clocks": clocks, "verified_specs": verified, "total_specs": B * Rs,
-                "alpha_crown": alpha, "graph": graph, "bab": bab, "sound": sound}
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = oracle_sample(w, args.cpu_sample_s)[0]
-            if bab is not None:
-                line["cpu_baseline"]["bab"] = oracle_bab_sample(args, w, bab["label0"])
-        print(json.dumps(line), flush=True)
-    net.close()
     if world > 1:
-        dist.destroy_process_group()
+        dist.barrier()
+    e2e_ms = max_over_ranks(e2e_run(steps), dev)
+    return {"value": weak_throughput(world, B * Rs, steps, e2e_ms), "unit": UNIT,
+            "h2d_bytes_per_step": h_centres.numel() * 4 + h_C.numel() * 4,
+            "d2h_bytes_per_step": h_lb[0].numel() * 4 + h_ver[0].numel(),
+            "pipeline": "double-buffered: the H2D of step i+1 and the D2H of step i overlap compute on a "
+                        "copy stream; all copies of every step are inside the timed region"}
+
+
+def graph_leg(args, w, net, centres, C, stream, flush, dev, world, steps, warmup, specs):
+    """The same verify call captured once in a CUDA graph (no host synchronisation inside) and replayed."""
+    import torch
+    from linear_bound_propagation_b200 import vf
+    vg = vf.VerifyGraph(net, centres, w.eps, C, crown_relus=w.crown_relus, both_sides=w.both_sides)
+    for _ in range(warmup):
+        vg.replay()
+    torch.cuda.synchronize()
+    g_ms = 0.0
+    for i in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        vg.replay()
+        e1.record(stream)
+        e1.synchronize()
+        g_ms += e0.elapsed_time(e1)
+    g_ms = max_over_ranks(g_ms, dev)
+    del vg
+    return {"value": weak_throughput(world, specs, steps, g_ms), "unit": UNIT, "ms_per_step": g_ms / steps,
+            "note": "vf.VerifyGraph: the verify call captured in a CUDA graph and replayed (no NaN/Inf scan, "
+                    "no unstable-neuron compaction)"}
+
+
+def alpha_leg(args, w, net, centres, C, stream, flush, dev, world, steps):
+    """alpha-CROWN: the same workload, intermediate bounds as in verify, then per-row slope optimisation."""
+    import torch
+    if args.alpha_iters <= 0 or w.both_sides:
+        return None
+    B, R = w.centres.shape[0], w.C.shape[1]
+    net.alpha_crown(centres, w.eps, C, iters=args.alpha_iters, crown_relus=w.crown_relus)  # warm-up
+    torch.cuda.synchronize()
+    a_ms = 0.0
+    for i in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        res = net.alpha_crown(centres, w.eps, C, iters=args.alpha_iters, crown_relus=w.crown_relus)
+        e1.record(stream)
+        e1.synchronize()
+        a_ms += e0.elapsed_time(e1)
+    a_ms = max_over_ranks(a_ms, dev)
+    gain = (res["lb"] - res["lb_start"])
+    return {"iters": args.alpha_iters, "lr": 0.1, "value": weak_throughput(world, B * R, steps, a_ms),
+            "unit": UNIT, "ms_per_step": a_ms / steps, "mean_lb_gain": float(gain.mean().item()),
+            "rows_improved": float((gain > 0).float().mean().item()),
+            "note": "vf_alpha_crown: intermediate bounds as in the verify step, then per-row lower-slope Adam ascent"}
+
+
+def sound_leg(args, w, net, centres, C, out, kw, stream, flush, dev, world, specs):
+    """The same verify call with vf_opts.sound (FFMA contractions, rounding budgets)."""
+    import torch
+    if args.sound_steps <= 0:
+        return None
+    plain_lb = out["lb"].clone()
+    so = {k: torch.empty_like(v) for k, v in out.items()}
+    skw = dict(kw, out=so, sound=True)
+    net.verify(centres, w.eps, C, **skw)  # warm-up
+    torch.cuda.synchronize()
+    s_ms = 0.0
+    for i in range(args.sound_steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        net.verify(centres, w.eps, C, **skw)
+        e1.record(stream)
+        e1.synchronize()
+        s_ms += e0.elapsed_time(e1)
+    s_ms = max_over_ranks(s_ms, dev)
+    gap = plain_lb - so["lb"]
+    return {"value": weak_throughput(world, specs, args.sound_steps, s_ms), "unit": UNIT,
+            "steps": args.sound_steps, "ms_per_step": s_ms / args.sound_steps,
+            "lb_below_plain_mean": float(gap.mean().item()), "lb_below_plain_max": float(gap.max().item()),
+            "verified_specs": int(so["verified"].sum().item()),
+            "note": "vf_verify_batch with vf_opts.sound: directed-rounding IBP, rounded-up intercepts and a "
+                    "per-row rounding budget at every node; FFMA contractions"}
 
 
 def bab_leg(args, w, net, centres, dev, stream, world, rank):
@@ -489,7 +629,15 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--config", type=int, default=5,
+                    help="headline workload (5: MLP 3072-1024x8-100, 4096 centres, eps 1/255)")
+    ap.add_argument("--no-eps-sweep", dest="eps_sweep", action="store_false",
+                    help="skip workload 5 at eps 0.5/255 and 2/255 (reported under eps_sweep)")
+    ap.add_argument("--no-all-workloads", dest="all_workloads", action="store_false",
+                    help="skip the other four workloads (reported under workloads)")
+    ap.add_argument("--sub-steps", type=int, default=5, help="timed steps of each eps_sweep / workloads entry")
+    ap.add_argument("--sub-cpu-sample-s", type=float, default=6.0,
+                    help="seconds of oracle time behind each workloads entry's cpu_baseline")
     ap.add_argument("--workspace-gb", type=float, default=16.0)
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -202,7 +202,11 @@ int vf_alpha_beta_grad(vf_net* net, const float* centres, int B, float eps, cons
  * complete verification by beta-CROWN with branch-and-bound; the page names the method only). The
  * property: every row of C [device] [R, n_L] is positive at every input of the box centre [device] [n0]
  * +/- eps. The search, run on the host with every bound computed on the device:
- *   1. a row < 0 at the centre itself is a counterexample (VF_BAB_FALSIFIED);
+ *   1. a row < 0 at the centre itself is a counterexample (VF_BAB_FALSIFIED). The fp32 value at the centre
+ *      is only a rounded evaluation, so a negative row is confirmed by the sound-in-fp32 mode (vf_opts.sound,
+ *      both sides, eps = 0): FALSIFIED needs that mode's upper bound, which the exact value on the fp32
+ *      weights cannot exceed, to be < 0 on some row; a row within rounding of 0 is not a counterexample
+ *      and the search goes on;
  *   2. a subdomain's row bound is the larger of vf_verify_batch's and vf_alpha_crown's (alpha_iters Adam
  *      steps of size lr on the slopes and the split multipliers); the whole box is bounded first;
  *   3. each round takes the open subdomains with the lowest bound (ties: created first), at most
@@ -222,6 +226,10 @@ typedef struct {
     int alpha_iters;        /* Adam steps per bound (0: vf_verify_batch's bound alone) */
     float lr;               /* Adam step size */
     const int* relu_crown;  /* as vf_opts.relu_crown */
+    int* trace;             /* [host] or NULL: for every bounded subdomain in the order bounded (the whole box
+                               first), the search-wide index of the neuron it would be split on (-1: none is
+                               unstable); at most trace_cap entries are written, result->domains are bounded */
+    int trace_cap;
 } vf_bab_opts;
 typedef struct {
     int status;             /* VF_BAB_VERIFIED, VF_BAB_FALSIFIED or VF_BAB_UNKNOWN */
@@ -291,7 +299,9 @@ int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms
  * the library's device code), so make that first call before any stream capture. All calls share the
  * one array and it keeps the last call's contents (the row constants are cleared by each call): calls
  * whose execution overlaps on the GPU -- on different streams, or from different threads -- race and
- * must be serialised by the caller. Errors: VF_ERR_ARG, VF_ERR_NONFINITE (eps), VF_ERR_WORKSPACE,
+ * must be serialised by the caller. The looked-up address is kept for the life of the process, so a
+ * caller that resets a device (cudaDeviceReset) must not use this entry point on it afterwards.
+ * lambda_bstride is 0 or at least R * n_out. Errors: VF_ERR_ARG, VF_ERR_NONFINITE (eps), VF_ERR_WORKSPACE,
  * VF_ERR_CUDA, described by vf_last_error(). */
 int vf_concretize_dense_noalloc(const float* lambda, long long lambda_bstride, int R, const float* W, const float* b,
                                 const float* centres, float eps, int B, int n_in, int n_out, float* lb, void* stream);

@@ -16,18 +16,20 @@
 // network creation. Three MMAs accumulate r_hi W_hi + r_hi W_lo + r_lo W_hi in fp32, which
 // leaves an error near 2^-21 relative per product instead of tf32's 2^-11.
 //
-// Roles in a CTA of 6 warps (one 128-row x BN-column output tile, BN <= 256):
-//   warp 0: TMA producer and TMEM allocator. Two smem rings: raw A tiles (128 x 32 fp32, 128-byte
-//           swizzle) together with the relaxation table slice of the tile's centres, and the
-//           W^T head/remainder tiles (BN x 32 each);
-//   warp 1: one thread issues kind::tf32 MMAs with A read from TMEM and B from smem, committing
-//           each k-block to the barriers that release its A and B stages;
-//   warps 2-5: one thread per tile row (= TMEM lane): relax the row's 32 coefficients of the
-//           k-block, keep the row constant, split into head/remainder and store both into a TMEM
-//           A stage (4 stages of 64 columns); afterwards read the accumulator (TMEM columns
-//           0..BN-1) and write the epilogue, staged through smem so global stores are coalesced.
-// TMEM: 512 columns per CTA (one CTA per SM). All waits are bounded: on expiry a shared abort
-// flag stops every role, the producer waits (also bounded) for its copies in flight, the MMA
+// Roles in a CTA of 11 warps (one CTA per SM, persistent over 128-row x BN-column output tiles, BN <= 256):
+//   warp 0:    TMA producer of the raw A tiles (128 x 32 fp32, 128-byte swizzle) together with the
+//              relaxation-table slice of the tile's centres, and owner of the TMEM allocation;
+//   warp 10:   TMA producer of the W^T head/remainder tiles (BN x 32 each) into a second ring;
+//   warp 1:    one thread issues the kind::tf32 MMAs, A read from TMEM and B from shared memory, and
+//              commits each k-block to the barriers that release its A and B stages;
+//   warps 2-5: one thread per tile row (= TMEM lane): relax the row's 32 coefficients of the k-block,
+//              keep the row constant, split into head/remainder and store both into one of four TMEM A
+//              stages (64 columns each);
+//   warps 6-9: drain the accumulator (TMEM columns 0..BN-1), hand it back to the MMA and write the
+//              epilogue: stores staged through shared memory so global stores are coalesced, or the
+//              concretisation against the centre into a per-N-tile partial.
+// TMEM: 512 columns per CTA. All waits are bounded: on expiry a shared abort
+// flag stops every role, the producers wait (also bounded) for their copies in flight, the MMA
 // thread for its MMAs, TMEM is freed and the kernel reports through *err.
 #include <cuda.h>
 

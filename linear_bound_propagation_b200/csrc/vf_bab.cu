@@ -87,6 +87,7 @@ struct DeviceBound {
     const int *meta_n, *meta_g;
     std::vector<signed char> hsplit;
     std::vector<BabPick> hpick;
+    long long traced = 0;  // entries of opts->trace written so far
 };
 
 // vf_bab_bound_fn on the device: one vf_verify_batch (bounds and pre-activation bounds of all n subdomains
@@ -133,6 +134,7 @@ int device_bound(void* user, int n, const int* split_offset, const int* split_co
         lb[i] = d.hpick[i].minlb;
         branch[i] = d.hpick[i].best;
         empty[i] = d.hpick[i].empty;
+        if (d.opts->trace != nullptr && d.traced < d.opts->trace_cap) d.opts->trace[d.traced++] = branch[i];
     }
     return VF_OK;
 }
@@ -212,8 +214,23 @@ extern "C" int vf_bab_verify(vf_net* net, const float* centre, float eps, const 
         BAB_CU(cudaStreamSynchronize(s));
         const float ymin = *std::min_element(y.begin(), y.end());
         if (ymin < 0.f) {
-            *result = vf_bab_result{VF_BAB_FALSIFIED, 0, 0, 0, ymin};
-            return VF_OK;
+            // a rounded evaluation: confirm with the sound mode's upper bound at the centre, which the exact
+            // value C f(centre) on the fp32 weights cannot exceed
+            DeviceBuffer ub;
+            BAB_CU(cudaMalloc(&ub.p, sizeof(float) * R));
+            vf_opts so{};
+            so.relu_crown = opts->relu_crown;
+            so.both_sides = 1;
+            so.sound = 1;
+            BAB_TRY(vf_verify_batch(net, cen.get<float>(), 1, 0.f, C, R, 0, &so, lbv.get<float>(), ub.get<float>(),
+                                    nullptr, nullptr, stream));
+            std::vector<float> yu(R);
+            BAB_CU(cudaMemcpyAsync(yu.data(), ub.p, sizeof(float) * R, cudaMemcpyDeviceToHost, s));
+            BAB_CU(cudaStreamSynchronize(s));
+            if (*std::min_element(yu.begin(), yu.end()) < 0.f) {
+                *result = vf_bab_result{VF_BAB_FALSIFIED, 0, 0, 0, ymin};
+                return VF_OK;
+            }
         }
     }
 

@@ -29,7 +29,9 @@ constexpr long long kScratchFloats = VF_NOALLOC_SCRATCH_FLOATS;
 static __device__ __align__(256) float g_noalloc_scratch[kScratchFloats];
 
 // Device address of g_noalloc_scratch per device. In host code the symbol's name is only a host-side
-// stand-in, so the address must be looked up on each device (with that device current) before use.
+// stand-in, so the address must be looked up on each device (with that device current) before use. The
+// address is cached for the life of the process: a caller that resets a device (cudaDeviceReset) destroys
+// the module the array lives in, and must not call this entry point on that device afterwards.
 constexpr int kMaxDevices = 64;
 float* g_scratch_dev[kMaxDevices] = {};
 std::mutex g_scratch_mu;
@@ -71,6 +73,9 @@ int vf_concretize_dense_noalloc(const float* lambda, long long lambda_bstride, i
     if (!lambda || !W || !b || !centres || !lb) return noalloc_fail(VF_ERR_ARG, "NULL pointer");
     if (B < 0 || R < 0 || n_in <= 0 || n_out <= 0 || lambda_bstride < 0)
         return noalloc_fail(VF_ERR_ARG, "bad sizes");
+    if (lambda_bstride > 0 && lambda_bstride < (long long)R * n_out)
+        return noalloc_fail(VF_ERR_ARG, "lambda_bstride %lld is below one centre's R * n_out = %lld elements",
+                            lambda_bstride, (long long)R * n_out);
     if (!std::isfinite(eps) || eps < 0.f) return noalloc_fail(VF_ERR_NONFINITE, "eps must be finite and >= 0");
     if (B == 0 || R == 0) return VF_OK;
     const long long M = (long long)B * R;

@@ -52,7 +52,8 @@ class Opts(ctypes.Structure):
 
 class BabOpts(ctypes.Structure):
     _fields_ = [("max_domains", ctypes.c_int), ("batch", ctypes.c_int), ("alpha_iters", ctypes.c_int),
-                ("lr", ctypes.c_float), ("relu_crown", ctypes.POINTER(ctypes.c_int))]
+                ("lr", ctypes.c_float), ("relu_crown", ctypes.POINTER(ctypes.c_int)),
+                ("trace", ctypes.POINTER(ctypes.c_int)), ("trace_cap", ctypes.c_int)]
 
 
 class BabResult(ctypes.Structure):
@@ -323,10 +324,16 @@ class Net:
         return lb, ga, gb
 
     def bab(self, centre: torch.Tensor, eps: float, C: torch.Tensor, max_domains: int = 1000, batch: int = 16,
-            alpha_iters: int = 20, lr: float = 0.1, crown_relus=None, stream=None):
+            alpha_iters: int = 20, lr: float = 0.1, crown_relus=None, stream=None, trace: bool = False):
         """vf_bab_verify on one box: centre [n0], C [R, n_L] (device). Returns dict(status, domains, rounds,
-        max_depth, lb)."""
+        max_depth, lb), plus, with trace, the branching neuron of every bounded subdomain in the order bounded
+        (search-wide index, -1 if none)."""
         o = BabOpts(max_domains=max_domains, batch=batch, alpha_iters=alpha_iters, lr=float(lr))
+        tbuf = None
+        if trace:
+            tbuf = (ctypes.c_int * max_domains)()
+            o.trace = ctypes.cast(tbuf, ctypes.POINTER(ctypes.c_int))
+            o.trace_cap = max_domains
         keep = None
         if crown_relus is not None:
             keep = (ctypes.c_int * self.n_nodes)()
@@ -337,8 +344,11 @@ class Net:
         C2 = C.reshape(-1, C.shape[-1]).contiguous()
         _check(lib().vf_bab_verify(self.h, _ptr(centre.contiguous()), float(eps), _ptr(C2), C2.shape[0],
                                    ctypes.byref(o), ctypes.byref(r), _stream_ptr(stream)))
-        return {"status": BAB_STATUS[r.status], "domains": r.domains, "rounds": r.rounds, "max_depth": r.max_depth,
-                "lb": r.lb}
+        out = {"status": BAB_STATUS[r.status], "domains": r.domains, "rounds": r.rounds, "max_depth": r.max_depth,
+               "lb": r.lb}
+        if trace:
+            out["trace"] = [tbuf[i] for i in range(min(r.domains, max_domains))]
+        return out
 
     def profile(self, enable: bool):
         _check(lib().vf_profile_enable(self.h, 1 if enable else 0))
@@ -405,12 +415,24 @@ def concretize_dense_noalloc(lam: torch.Tensor, W: torch.Tensor, b: torch.Tensor
     """vf_concretize_dense_noalloc: rows lam [B or 1, R, n_out] over z = W x + b, x in centres +/- eps.
     The library allocates nothing for this call (its scratch is a fixed device array); `out` may be
     passed to keep the call free of any allocation on the Python side too."""
+    for name, t in (("lam", lam), ("W", W), ("b", b), ("centres", centres)):
+        if t.dtype != torch.float32:
+            raise ValueError(f"{name} must be float32, got {t.dtype}")
+    if W.dim() != 2 or centres.dim() != 2 or lam.dim() not in (2, 3):
+        raise ValueError("W [n_out, n_in], centres [B, n_in] and lam [B or 1, R, n_out] (or [R, n_out]) expected")
     B = centres.shape[0]
     R = lam.shape[-2]
     n_out, n_in = W.shape
+    if centres.shape[1] != n_in or lam.shape[-1] != n_out or b.numel() != n_out:
+        raise ValueError(f"shapes do not match W [{n_out}, {n_in}]: centres {tuple(centres.shape)}, "
+                         f"lam {tuple(lam.shape)}, b {tuple(b.shape)}")
+    if lam.dim() == 3 and lam.shape[0] not in (1, B):
+        raise ValueError(f"lam has {lam.shape[0]} centre blocks for {B} centres")
     bstride = 0 if lam.dim() == 2 or lam.shape[0] == 1 else R * n_out
     if out is None:
         out = torch.empty(B, R, device=centres.device)
+    elif out.dtype != torch.float32 or tuple(out.shape) != (B, R):
+        raise ValueError(f"out must be float32 [{B}, {R}], got {out.dtype} {tuple(out.shape)}")
     _check(lib().vf_concretize_dense_noalloc(_ptr(lam), bstride, R, _ptr(W), _ptr(b), _ptr(centres), float(eps), B,
                                              n_in, n_out, _ptr(out), _stream_ptr(stream)))
     return out

@@ -17,7 +17,7 @@ from tests import test_oracle_pins as P
 FAST_FIRST = [P.check_hand_examples, P.check_linear_network, P.check_first_layer_exact, P.check_relax_valid,
               P.check_conv_vs_torch, P.check_forward_vs_torch, P.check_all_stable_exact,
               P.check_one_hidden_alpha0, P.check_eps_monotone, P.check_exact_2d, P.check_lp_sandwich,
-              P.check_soundness_small_configs]
+              P.check_adam_closed_form, P.check_crown_subset, P.check_soundness_small_configs]
 
 MUTATIONS = [
     ("relax_params", "t[unstable] = -s * l[unstable]", "t[unstable] = s * l[unstable]"),
@@ -43,6 +43,16 @@ MUTATIONS = [
     ("verify", "np.einsum(\"brn,bn->br\", np.abs(Cfull), zr)\n    ub_ibp", "np.einsum(\"brn,bn->br\", Cfull, zr)\n    ub_ibp"),
     ("verify", "ub_cr[b] = -lbs[R:]", "ub_cr[b] = lbs[R:]"),
     ("verify", "lb = np.maximum(lb_ibp, lb_cr)", "lb = np.minimum(lb_ibp, lb_cr)"),
+    ("verify", "if k in crown_set and not _first_affine_on_input(net, p):",
+     "if k not in crown_set and not _first_affine_on_input(net, p):"),
+    ("verify", "crown_set = set(relus if crown_relus is None else crown_relus)",
+     "crown_set = set(relus if crown_relus is None else [r - 2 for r in crown_relus])"),
+    ("verify", "pre[k][0][b] = np.where(unst, np.maximum(l0, l_cr), l0)", "pass"),
+    ("alpha_crown", "mh = m1 / (1 - b1 ** (it + 1))", "mh = m1 / (1 - b1 ** it)"),
+    ("alpha_crown", "mh = m1 / (1 - b1 ** (it + 1))", "mh = m1 / (1 - b1 ** (it + 2))"),
+    ("alpha_crown", "np.sqrt(vh) + 1e-8", "np.sqrt(vh + 1e-8)"),
+    ("alpha_crown", "lr * mh / (np.sqrt(vh) + 1e-8)", "lr * mh / (vh + 1e-8)"),
+    ("alpha_crown", "m2 = b2 * m2 + (1 - b2) * g * g", "m2 = b2 * m2 + (1 - b2) * np.abs(g)"),
 ]
 
 

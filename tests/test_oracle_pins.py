@@ -258,7 +258,7 @@ def check_soundness_small_configs(seed=7):
         n0 = int(np.prod(net[0].shape))
         centres = rng.random((C.shape[0] if C.shape[0] > 1 else 2, n0)).astype(np.float32)
         crown = relu_ids(net)[-2:] if mode == "last2" else None
-        ok, det = _sound_on(net, centres, eps, C, 3000, 300, seed + i, crown)
+        ok, det = _sound_on(net, centres, eps, C, 10000, 1000, seed + i, crown)
         if not ok:
             return False, f"case {i}: {det}"
     return True, ""
@@ -329,9 +329,80 @@ def check_eps_monotone(seed=10):
     return True, ""
 
 
+def _one_neuron_net(w):
+    """y = ReLU(w x) on x in [-1, 1]: input -> dense [[w]] -> ReLU -> dense [[1]], zero biases."""
+    return net_from_layers([{"W": [[w]], "b": [0.0]}, {"W": [[1.0]], "b": [0.0]}])
+
+
+def check_adam_closed_form():
+    """alpha-CROWN's ascent against Adam's closed form (Kingma & Ba 2015, Algorithm 1, bias-corrected).
+
+    On y = ReLU(w x), x in [-1, 1], the pre-activation interval [-w, w] sits at the adaptive tie, so the
+    start slope is 1, and the specification bound is lb(alpha) = -w alpha, whose gradient -w does not
+    change while alpha stays in [0, 1]. With a constant gradient g the bias-corrected moments are exactly
+    m_hat = g and v_hat = g^2 after every step k (m_k = (1 - b1^k) g, v_k = (1 - b2^k) g^2), so each step
+    moves alpha by lr * g / (|g| + 1e-8) and after k steps alpha_k = 1 - k lr w / (w + 1e-8). The bound
+    improves with every step, so the best over the iterates is -w alpha_k. w = 1e-4 makes the 1e-8
+    term visible (|g| is comparable to it), which fixes where the epsilon sits."""
+    for w, lr in ((2.0, 0.1), (1e-4, 0.1), (0.5, 0.25)):
+        net = _one_neuron_net(w)
+        w32 = float(np.float32(w))
+        c = np.zeros((1, 1), np.float32)
+        C = np.ones((1, 1, 1), np.float32)
+        for k in range(0, 4):
+            best, start = O.alpha_crown(net, c, 1.0, C, iters=k, lr=lr)
+            a_k = max(0.0, 1.0 - k * lr * w32 / (w32 + 1e-8))
+            want = -w32 * a_k
+            if not abs(start[0, 0] + w32) <= 1e-15:
+                return False, f"w={w}: adaptive start {start[0, 0]} != {-w32}"
+            if not abs(best[0, 0] - want) <= 1e-12 * (1.0 + abs(want)):
+                return False, f"w={w} lr={lr} after {k} steps: best {best[0, 0]} != closed form {want}"
+    return True, ""
+
+
+def check_crown_subset(seed=11):
+    """IBP substitution for the unselected ReLUs: a ReLU outside crown_relus keeps its IBP bounds bit for
+    bit, and a selected one takes, on its IBP-unstable neurons, the intersection with a standalone CROWN
+    pass from rows [I; -I] over its pre-activation node, run with the relaxations of the earlier ReLUs.
+    The selected passes must also change something (else 'refine nothing' would pass)."""
+    rng = np.random.default_rng(seed)
+    net = synth.mlp([12] + [10] * 5 + [6], rng)
+    relus = relu_ids(net)
+    sel = relus[-2:]
+    c = rng.random((2, 12)).astype(np.float32)
+    C = synth.margin_spec(np.array([1, 4]), 6)
+    eps = 0.05
+    res = O.verify(net, c, eps, C, crown_relus=sel)
+    tightened = 0
+    for b in range(2):
+        relax = {}
+        for k in relus:
+            p = net[k].src
+            l_ibp, u_ibp = res.ibp_bounds[p][0][b], res.ibp_bounds[p][1][b]
+            l, u = res.pre_bounds[k][0][b], res.pre_bounds[k][1][b]
+            if k not in sel:
+                if not (np.array_equal(l, l_ibp) and np.array_equal(u, u_ibp)):
+                    return False, f"unselected relu {k} does not keep its IBP bounds"
+            else:
+                n = l.size
+                eye = np.eye(n)
+                lbs = O.crown_pass(net, p, np.concatenate([eye, -eye]), relax, c[b], eps)
+                unst = (l_ibp < 0) & (u_ibp > 0)
+                l_want = np.where(unst, np.maximum(l_ibp, lbs[:n]), l_ibp)
+                u_want = np.where(unst, np.minimum(u_ibp, -lbs[n:]), u_ibp)
+                if not (np.allclose(l, l_want, rtol=0, atol=1e-12) and np.allclose(u, u_want, rtol=0, atol=1e-12)):
+                    return False, f"selected relu {k}: bounds differ from a standalone CROWN pass"
+                tightened += int(np.sum((l > l_ibp) | (u < u_ibp)))
+            relax[k] = O.relax_params(l, u)
+    if tightened == 0:
+        return False, "no selected bound was tightened"
+    return True, ""
+
+
 ALL_CHECKS = [check_conv_vs_torch, check_forward_vs_torch, check_hand_examples, check_linear_network,
               check_first_layer_exact, check_relax_valid, check_one_hidden_alpha0, check_all_stable_exact,
-              check_soundness_small_configs, check_exact_2d, check_lp_sandwich, check_eps_monotone]
+              check_soundness_small_configs, check_exact_2d, check_lp_sandwich, check_eps_monotone,
+              check_adam_closed_form, check_crown_subset]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=[c.__name__ for c in ALL_CHECKS])
@@ -343,3 +414,13 @@ def test_oracle_pin(check):
 def test_alpha_nan_rejected():
     with pytest.raises(ValueError):
         O.relax_params(np.array([-1.0]), np.array([1.0]), np.array([np.nan]))
+
+
+def test_wide_mlp_crown_layers_are_the_last_two():
+    """The wide MLP workload refines z7 and z8 (the last two of its eight hidden ReLU layers) by CROWN and
+    keeps IBP for z1..z6 (IBP substitution for the middle layers)."""
+    w = synth.workload(5, B=1)
+    dense = [v for v, nd in enumerate(w.net) if nd.op == "dense"]
+    assert len(dense) == 9
+    want = [v for v, nd in enumerate(w.net) if nd.op == "relu" and nd.src in (dense[6], dense[7])]
+    assert w.crown_relus == want and len(want) == 2

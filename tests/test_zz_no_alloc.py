@@ -2,8 +2,9 @@
 device memory belongs to another allocator, or they run under a fixed budget, or they must avoid the
 synchronisation that cudaMalloc/cudaFree can cause). Its scratch is a fixed array inside the library.
 
-It must give the same bounds as the handle-based path -- vf_crown_backward from the dense layer followed
-by vf_concretize -- within the parity tolerance, on two calls in a row (the shared scratch keeps the
+It must give the same bounds as the fp64 oracle's back-substitution through the layer followed by its
+concretisation, and as the handle-based path -- vf_crown_backward from the dense layer followed by
+vf_concretize -- within the parity tolerance, on two calls in a row (the shared scratch keeps the
 previous call's contents, so the second call checks that nothing stale leaks in). This file is named so
 that pytest collects it last; it also passes when run alone in a fresh process.
 """
@@ -13,6 +14,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle.lbp as O
 from linear_bound_propagation_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -42,6 +44,12 @@ def test_noalloc_matches_crown_backward_then_concretize_twice(shared_rows):
     torch.cuda.synchronize()
     ref = ref.cpu().numpy()
 
+    # the oracle: rows over z = W x + b back to the input (one dense node on the input), then concretised
+    c_np = centres.cpu().numpy()
+    ora = np.stack([O.concretize(*O.backward(net[:2], 1, lam_np[0 if shared_rows else i].astype(np.float64), {}),
+                                 c_np[i], eps) for i in range(B)])
+    assert _rel_violation(ref, ora) <= 1.0
+
     W = torch.from_numpy(np.ascontiguousarray(net[1].W)).cuda()
     b = torch.from_numpy(np.ascontiguousarray(net[1].b)).cuda()
     out = torch.empty(B, R, device="cuda")
@@ -51,7 +59,8 @@ def test_noalloc_matches_crown_backward_then_concretize_twice(shared_rows):
         torch.cuda.synchronize()
         got = out.cpu().numpy()
         assert np.isfinite(got).all(), f"call {call}: unwritten outputs"
-        assert _rel_violation(got, ref) <= 1.0, f"call {call}"
+        assert _rel_violation(got, ora) <= 1.0, f"call {call}: against the oracle"
+        assert _rel_violation(got, ref) <= 1.0, f"call {call}: against the handle path"
 
 
 def test_noalloc_rejects_requests_beyond_its_fixed_scratch():
