@@ -213,25 +213,30 @@ TF32_OVER_BF16 = 1.1 / 2.25
 TRAFFIC_PER_LAUNCH = {("mlp_784-256x3-10_B1024", 1): 1099.0e6 / 6}
 
 
-def roofline(kstats, step_total_ms, n_sms, workload=None):
+def roofline(kstats, step_total_ms, n_sms, workload=None, step_ms=None):
     """Roofline entry for the dominant contraction kind of the step.
 
-    Tensor-core dense steps (3xTF32): algorithmic flops 2*M*K*N per launch against the tf32 peak
-    divided by 3 (three tf32 MMAs per fp32-accurate product); the tf32 peak is the measured bf16
-    burst peak times the nominal tf32/bf16 ratio. FFMA and convolution kernels: fp32 FFMA peak =
-    SMs x 128 lanes x 2 flop x max SM clock ("alu")."""
+    Tensor-core steps (3xTF32, dense and convolution): algorithmic flops per launch (2*M*K*N dense;
+    2*M*positions*C_in*C_out*k*k/s^2 convolution) against the tf32 peak divided by 3 (three tf32 products per
+    fp32-accurate one); the tf32 peak is the measured bf16 peak times the nominal tf32/bf16 ratio, the burst
+    figure for short steps and the sustained (power-capped) one for steps of 100 ms and longer. FFMA kernels:
+    fp32 FFMA peak = SMs x 128 lanes x 2 flop x max SM clock ("alu")."""
     p, src = peaks()
     kind = max(kstats, key=lambda k: kstats[k][1])
     n_k, k_ms, k_flops = kstats[kind]
     avg_ms = k_ms / max(n_k, 1)
     achieved = (k_flops / max(n_k, 1)) / (avg_ms / 1000.0) / 1e12 if n_k else 0.0
     sm_mhz = float(p.get("sm_max_mhz", 1965.0))
-    if kind == 1:
-        tf32 = float(p["bf16_tflops"]) * TF32_OVER_BF16
+    if kind in (1, 5):
+        sustained = step_ms is not None and step_ms >= 100.0 and "bf16_tflops_sustained" in p
+        bf16 = float(p["bf16_tflops_sustained"] if sustained else p["bf16_tflops"])
+        tf32 = bf16 * TF32_OVER_BF16
         peak = tf32 / 3.0
-        bound, name = "tensor", "dense_back_tc (tcgen05 kind::tf32, 3xTF32 CROWN Lambda.W contraction)"
-        psrc = (f"tf32 = {src} bf16 burst {p['bf16_tflops']:.0f} TFLOP/s x nominal 1.1/2.25 = {tf32:.0f}; "
-                f"3xTF32 effective = tf32 / 3")
+        bound = "tensor"
+        name = {1: "dense_back_tc (tcgen05 kind::tf32, 3xTF32 CROWN Lambda.W contraction)",
+                5: "conv_back_tc (tcgen05 kind::tf32 implicit GEMM, 3xTF32 transposed convolution)"}[kind]
+        psrc = (f"tf32 = {src} bf16 {'sustained' if sustained else 'burst'} {bf16:.0f} TFLOP/s x nominal "
+                f"1.1/2.25 = {tf32:.0f}; 3xTF32 effective = tf32 / 3")
     else:
         peak = n_sms * 128 * 2 * sm_mhz * 1e6 / 1e12
         bound = "alu"
@@ -382,7 +387,7 @@ def measure_workload(args, ctx, cfg, eps, steps, warmup, headline, legs=None):
     torch.cuda.synchronize()
     clocks = stop_clocks(clk)
     launches = net.launch_count() - launches0
-    kstats = {k: net.profile_read(kind=k, reset=False) for k in (1, 2, 3, 4)}
+    kstats = {k: net.profile_read(kind=k, reset=False) for k in (1, 2, 3, 4, 5)}
     net.profile_read(reset=True)
     net.profile(False)
     step_ms = [a.elapsed_time(b) for a, b in ev]
@@ -391,7 +396,7 @@ def measure_workload(args, ctx, cfg, eps, steps, warmup, headline, legs=None):
     value = weak_throughput(world, B * Rs, steps, total_ms)
     verified = int(out["verified"].sum().item())
     roof = roofline(kstats, total_ms, torch.cuda.get_device_properties(dev).multi_processor_count,
-                    w.name if (args.centres is None or not headline) else None)
+                    w.name if (args.centres is None or not headline) else None, total_ms / steps)
 
     e2e = None
     if headline and not args.no_e2e:

@@ -272,7 +272,14 @@ const char* vf_last_error(void);
  * their summed device time in ms and their summed algorithmic flops (2*M*K*N for dense steps;
  * 2*M*n_in*C_out*k*k/stride^2 for whole-map convolutions, 2*M*(window positions on the map)*C_in*C_out*
  * k*k/stride^2 for receptive-field windows) since the last reset (reset != 0 clears all kinds). */
-enum { VF_KERNEL_ALL = 0, VF_KERNEL_DENSE_TC = 1, VF_KERNEL_DENSE_FFMA = 2, VF_KERNEL_CONV = 3, VF_KERNEL_CONV_WIN = 4 };
+enum {
+    VF_KERNEL_ALL = 0,
+    VF_KERNEL_DENSE_TC = 1,
+    VF_KERNEL_DENSE_FFMA = 2,
+    VF_KERNEL_CONV = 3,
+    VF_KERNEL_CONV_WIN = 4,
+    VF_KERNEL_CONV_TC = 5 /* tensor-core implicit GEMM, whole maps and windows; flops as for windows */
+};
 int vf_profile_enable(vf_net* net, int enable);
 int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms, double* flops, int reset);
 

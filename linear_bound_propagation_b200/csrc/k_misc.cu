@@ -30,29 +30,89 @@ unsigned grid_for(long long n, int threads) {
 // to [0, 1], or the adaptive choice 1 if u >= -l else 0. The fourth lane carries the bias of
 // the affine node that produced z (0 if none), which the next back-substitution step adds to
 // the row constant together with the relaxation intercept.
+__device__ __forceinline__ float4 relax_one(float lo_b, float up_b, const float* __restrict__ alpha, long long i,
+                                            float bias_v, int sound) {
+    float4 p = make_float4(0.f, 0.f, 0.f, bias_v);
+    if (up_b <= 0.f) {
+    } else if (lo_b >= 0.f) {
+        p.x = 1.f;
+        p.y = 1.f;
+    } else {
+        const float s = up_b / (up_b - lo_b);
+        p.y = s;
+        // sound: the line s z + t lies above the ReLU at both ends (hence on [l, u]) in exact arithmetic
+        p.z = sound ? fmaxf(__fmul_ru(s, -lo_b), __fmul_ru(up_b, __fsub_ru(1.f, s))) : -s * lo_b;
+        if (alpha != nullptr)
+            p.x = fminf(fmaxf(alpha[i], 0.f), 1.f);
+        else
+            p.x = (up_b >= -lo_b) ? 1.f : 0.f;
+    }
+    return p;
+}
+
 __global__ void relax_params_k(const float* __restrict__ l, const float* __restrict__ u,
                                const float* __restrict__ alpha, long long n, float4* __restrict__ P,
                                const float* __restrict__ bias, long long n_per_centre, long long per_channel,
                                int sound) {
     GRID_STRIDE(i, n) {
-        const float lo_b = l[i], up_b = u[i];
-        float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (up_b <= 0.f) {
-        } else if (lo_b >= 0.f) {
-            p.x = 1.f;
-            p.y = 1.f;
+        const float bv = (bias != nullptr) ? bias[(i % n_per_centre) / per_channel] : 0.f;
+        P[i] = relax_one(l[i], u[i], alpha, i, bv, sound);
+    }
+}
+
+// One ReLU layer (n = B * n_layer neurons): its bounds and its relaxation in one pass, four neurons per
+// thread (n_layer % 4 == 0). from_cr: l, u = c -/+ r as bounds_k takes them (split clamp, sound rounding)
+// and stored; otherwise l, u are read and, with pass_out (the rows [I; -I] of a plain intermediate pass,
+// [B, 2 n_layer]), intersected as intersect_k does on the IBP-unstable neurons and stored back. Then P as
+// relax_params_k, with the same arithmetic (relax_one), so the result is bitwise the unfused one.
+__global__ void relu_bounds_relax_k(const float* __restrict__ c, const float* __restrict__ r,
+                                    const signed char* __restrict__ split, const float* __restrict__ pass_out,
+                                    float* __restrict__ l, float* __restrict__ u, const float* __restrict__ alpha,
+                                    long long n4, long long n_layer, float4* __restrict__ P,
+                                    const float* __restrict__ bias, long long per_channel, int sound) {
+    GRID_STRIDE(q, n4) {
+        const long long i0 = 4 * q;
+        float lv[4], uv[4];
+        if (c != nullptr) {
+            const float4 c4 = reinterpret_cast<const float4*>(c)[q], r4 = reinterpret_cast<const float4*>(r)[q];
+            const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, rr[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                lv[j] = sound ? __fsub_rd(cc[j], rr[j]) : cc[j] - rr[j];
+                uv[j] = sound ? __fadd_ru(cc[j], rr[j]) : cc[j] + rr[j];
+                if (split != nullptr) {
+                    const signed char sg = split[i0 + j];
+                    if (sg > 0) lv[j] = fmaxf(lv[j], 0.f);
+                    if (sg < 0) uv[j] = fminf(uv[j], 0.f);
+                }
+            }
         } else {
-            const float s = up_b / (up_b - lo_b);
-            p.y = s;
-            // sound: the line s z + t lies above the ReLU at both ends (hence on [l, u]) in exact arithmetic
-            p.z = sound ? fmaxf(__fmul_ru(s, -lo_b), __fmul_ru(up_b, __fsub_ru(1.f, s))) : -s * lo_b;
-            if (alpha != nullptr)
-                p.x = fminf(fmaxf(alpha[i], 0.f), 1.f);
-            else
-                p.x = (up_b >= -lo_b) ? 1.f : 0.f;
+            const float4 l4 = reinterpret_cast<const float4*>(l)[q], u4 = reinterpret_cast<const float4*>(u)[q];
+            lv[0] = l4.x; lv[1] = l4.y; lv[2] = l4.z; lv[3] = l4.w;
+            uv[0] = u4.x; uv[1] = u4.y; uv[2] = u4.z; uv[3] = u4.w;
+            if (pass_out != nullptr) {
+                const long long b = i0 / n_layer, j0 = i0 - b * n_layer;
+                const float4 pl = *reinterpret_cast<const float4*>(pass_out + b * 2 * n_layer + j0);
+                const float4 pu = *reinterpret_cast<const float4*>(pass_out + b * 2 * n_layer + n_layer + j0);
+                const float ql[4] = {pl.x, pl.y, pl.z, pl.w}, qu[4] = {pu.x, pu.y, pu.z, pu.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (lv[j] < 0.f && uv[j] > 0.f) {
+                        lv[j] = fmaxf(lv[j], ql[j]);
+                        uv[j] = fminf(uv[j], -qu[j]);
+                    }
+            }
         }
-        p.w = (bias != nullptr) ? bias[(i % n_per_centre) / per_channel] : 0.f;
-        P[i] = p;
+        if (c != nullptr || pass_out != nullptr) {
+            reinterpret_cast<float4*>(l)[q] = make_float4(lv[0], lv[1], lv[2], lv[3]);
+            reinterpret_cast<float4*>(u)[q] = make_float4(uv[0], uv[1], uv[2], uv[3]);
+        }
+        const long long j0 = i0 % n_layer;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float bv = (bias != nullptr) ? bias[(j0 + j) / per_channel] : 0.f;
+            P[i0 + j] = relax_one(lv[j], uv[j], alpha, i0 + j, bv, sound);
+        }
     }
 }
 
@@ -363,6 +423,25 @@ cudaError_t launch_relax_params(const float* l, const float* u, const float* alp
                                 const float* bias, long long n_per_centre, long long per_channel, cudaStream_t s,
                                 int sound) {
     relax_params_k<<<grid_for(n, 256), 256, 0, s>>>(l, u, alpha, n, P, bias, n_per_centre, per_channel, sound);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_relu_bounds_relax(const float* c, const float* r, const signed char* split, const float* pass_out,
+                                     float* l, float* u, const float* alpha, int B, long long n_layer, float4* P,
+                                     const float* bias, long long per_channel, int sound, cudaStream_t s) {
+    const long long n = (long long)B * n_layer;
+    if (n_layer % 4 != 0 || (reinterpret_cast<uintptr_t>(l) & 15) || (reinterpret_cast<uintptr_t>(u) & 15) ||
+        (c && ((reinterpret_cast<uintptr_t>(c) & 15) || (reinterpret_cast<uintptr_t>(r) & 15))) ||
+        (pass_out && (reinterpret_cast<uintptr_t>(pass_out) & 15))) {
+        // unvectorisable layout: the two unfused steps
+        cudaError_t e = cudaSuccess;
+        if (c != nullptr) e = launch_bounds_from_cr(c, r, n, l, u, s, split, sound);
+        else if (pass_out != nullptr) e = launch_intersect(l, u, nullptr, nullptr, pass_out, B, n_layer, s);
+        if (e != cudaSuccess) return e;
+        return launch_relax_params(l, u, alpha, n, P, bias, n_layer, per_channel, s, sound);
+    }
+    relu_bounds_relax_k<<<grid_for(n / 4, 256), 256, 0, s>>>(c, r, split, pass_out, l, u, alpha, n / 4, n_layer, P,
+                                                            bias, per_channel, sound);
     return cudaGetLastError();
 }
 

@@ -75,6 +75,7 @@ struct Node {
     float* WtLo = nullptr; // dense only: W^T - WtHi (3xTF32 remainder)
     float* rowsum_abs = nullptr;  // dense only: sum_k |W[n, k]| (IBP radius of a layer fed by the input box)
     float* Wwin = nullptr;        // conv only: weights in the tap-major layout of the windowed kernel
+    float* Wtc = nullptr;         // conv only: 3xTF32 operand images of the tensor-core kernel (or null)
     WinWeights ww{nullptr, 0, 0, 4, 0};
     int consumers = 0;
 };
@@ -99,6 +100,7 @@ struct vf_net {
     int conv_whole_warp = 2;
     int conv_win_per_position = 0;  // windowed rows without position blocking (VF_CONV_WIN_KERNEL=1)
     int compact = 1;        // intermediate passes over IBP-unstable neurons only (VF_COMPACT=0: off)
+    int conv_tc = 1;        // convolution steps on the tensor cores where the shapes allow (VF_CONV_TC=0: off)
     int call_sound = 0;     // set for the duration of a vf_opts.sound call: contractions take FFMA kernels
     bool prof = false;
     std::vector<cudaEvent_t> ev_free;
@@ -108,9 +110,9 @@ struct vf_net {
         double flops;
     };
     std::vector<Timed> ev_used;
-    double prof_flops[5] = {0, 0, 0, 0, 0};
-    long long prof_launches[5] = {0, 0, 0, 0, 0};
-    double prof_ms[5] = {0, 0, 0, 0, 0};
+    double prof_flops[6] = {0, 0, 0, 0, 0, 0};
+    long long prof_launches[6] = {0, 0, 0, 0, 0, 0};
+    double prof_ms[6] = {0, 0, 0, 0, 0, 0};
 };
 
 namespace {
@@ -540,6 +542,40 @@ struct Walker {
                         LAUNCH(net, launch_conv_start_rows(out, ld, M, pg, nd.W, g, mode == OUT_ACCUM ? 1 : 0, s));
                     return VF_OK;
                 }
+                const bool fuse_in = (nd.src == 0 && ext_in == nullptr && net->nodes[0].consumers == 1 &&
+                                      sw == nullptr && pend[0].kind == E_NONE);
+                const Win wa_tc = e.windowed ? e.win : full_win(nd);
+                if (net->conv_tc && !net->call_sound && sw == nullptr && nd.Wtc != nullptr &&
+                    conv_back_tc_supported(g, wa_tc, full_win(sn), OUT_CONCRETIZE)) {
+                    // tensor-core implicit GEMM, for whole-map and windowed rows alike
+                    float* out = nullptr;
+                    long long ld = 0;
+                    int mode = OUT_CONCRETIZE;
+                    Win dst = full_win(sn);
+                    if (!fuse_in) {
+                        if (e.windowed) {
+                            const Win nat = win_back(e.win, g);
+                            dst = win_small(nat, sn) ? nat : full_win(sn);
+                            TRY(target(nd.src, &out, &ld, &mode, &nat, &dst));
+                        } else {
+                            TRY(target(nd.src, &out, &ld, &mode));
+                        }
+                    }
+                    if (!dry) {
+                        if (mode == OUT_STORE && !conv_back_tc_covers(g, wa_tc, dst))
+                            CU(cudaMemset2DAsync(out, sizeof(float) * ld, 0, sizeof(float) * win_len(dst), M, s));
+                        cudaEvent_t e0 = nullptr;
+                        prof_begin(&e0);
+                        LAUNCH(net, launch_conv_back_tc(e.ref, e.rx, nd.Wtc, nd.b, M, g, pg, ps, wa_tc, dst, mode, out,
+                                                        ld, cst, centres, eps, net->d_err, net->num_sms, s));
+                        const Win nat = win_back(wa_tc, g);
+                        const double pos = (double)std::min<long long>((long long)nat.hh * nat.hw, (long long)g.h * g.w);
+                        prof_end(e0, VF_KERNEL_CONV_TC, 2.0 * (double)M * pos * g.ci * g.co * g.k * g.k /
+                                                            ((double)g.stride * g.stride));
+                    }
+                    release(e);
+                    return VF_OK;
+                }
                 WinLaunch wl;
                 if (!e.windowed && e.kind != E_IDENT && net->conv_whole_warp &&
                     conv_back_win_plan(g, nd.ww, full_win(nd), &wl) &&
@@ -912,24 +948,6 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
     TRY(run_ibp(net, centres, B, eps, ar, st, s, o.split, sound));
     bd.Lw.assign(nn, nullptr);
     bd.Uw.assign(nn, nullptr);
-    for (int v = 0; v < nn; ++v) {
-        if (net->nodes[v].op != VF_RELU) continue;
-        const int p = net->nodes[v].src;
-        const long long cnt = (long long)B * net->nodes[p].n;
-        bd.Lw[p] = ar.take<float>(cnt);
-        bd.Uw[p] = ar.take<float>(cnt);
-        if (!bd.Lw[p] || !bd.Uw[p]) return fail(VF_ERR_WORKSPACE, "workspace too small for intermediate bounds");
-        LAUNCH(net, launch_bounds_from_cr(st.c[p], st.r[p], cnt, bd.Lw[p], bd.Uw[p], s, o.split ? o.split[v] : nullptr,
-                                          sound));
-    }
-    if (sound) {  // error weights of every node, kept for the specification pass
-        bd.sw.assign(nn, nullptr);
-        bd.a_next = 0;
-        for (int v = 0; v < nn; ++v) {
-            bd.sw[v] = ar.take<float>((size_t)B * net->nodes[v].n);
-            if (!bd.sw[v]) return fail(VF_ERR_WORKSPACE, "workspace too small for error weights");
-        }
-    }
     bd.relax.assign(nn, nullptr);
     std::vector<float4*> P(nn, nullptr);
     long long max_pass_rows = 1;
@@ -940,6 +958,45 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
             bd.relax[v] = P[v];
             max_pass_rows = std::max(max_pass_rows, 2 * net->nodes[v].n);
         }
+    // A ReLU whose bounds no CROWN pass refines (IBP substitution, or an exact source) takes its
+    // relaxation in the same pass that forms its bounds from the IBP centre and radius.
+    auto refined = [&](int k) {
+        const bool crown = (o.relu_crown == nullptr) || (o.relu_crown[k] != 0);
+        return crown && !exact_source(net, net->nodes[k].src);
+    };
+    auto relax_args = [&](int k, const float** bias, long long* per_channel) {
+        const Node& sn = net->nodes[net->nodes[k].src];
+        const bool aff = sn.op == VF_DENSE || sn.op == VF_CONV2D;
+        *bias = aff ? sn.b : nullptr;
+        *per_channel = sn.op == VF_CONV2D ? (long long)sn.h * sn.w : 1;
+    };
+    for (int v = 0; v < nn; ++v) {
+        if (net->nodes[v].op != VF_RELU) continue;
+        const int p = net->nodes[v].src;
+        const long long cnt = (long long)B * net->nodes[p].n;
+        bd.Lw[p] = ar.take<float>(cnt);
+        bd.Uw[p] = ar.take<float>(cnt);
+        if (!bd.Lw[p] || !bd.Uw[p]) return fail(VF_ERR_WORKSPACE, "workspace too small for intermediate bounds");
+        if (!refined(v)) {
+            const float* bias;
+            long long pc;
+            relax_args(v, &bias, &pc);
+            LAUNCH(net, launch_relu_bounds_relax(st.c[p], st.r[p], o.split ? o.split[v] : nullptr, nullptr, bd.Lw[p],
+                                                 bd.Uw[p], o.alpha ? o.alpha[v] : nullptr, B, net->nodes[p].n, P[v],
+                                                 bias, pc, sound, s));
+        } else {
+            LAUNCH(net, launch_bounds_from_cr(st.c[p], st.r[p], cnt, bd.Lw[p], bd.Uw[p], s,
+                                              o.split ? o.split[v] : nullptr, sound));
+        }
+    }
+    if (sound) {  // error weights of every node, kept for the specification pass
+        bd.sw.assign(nn, nullptr);
+        bd.a_next = 0;
+        for (int v = 0; v < nn; ++v) {
+            bd.sw[v] = ar.take<float>((size_t)B * net->nodes[v].n);
+            if (!bd.sw[v]) return fail(VF_ERR_WORKSPACE, "workspace too small for error weights");
+        }
+    }
     // Unstable-neuron compaction: only IBP-unstable neurons change at the intersection, so a pass needs
     // rows for those alone. The number per centre is read back once (one host synchronisation) and each
     // pass is sized for the largest count; a pass whose largest count is above 7/8 of the node stays plain.
@@ -999,8 +1056,15 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
             const long long np = net->nodes[p].n;
             TRY(run_pass(net, p, init, (long long)B * 2 * np, 2 * np, tmp, bd.relax, centres, eps, pass_out, nullptr,
                          nullptr, s, nullptr, sw));
-            LAUNCH(net, launch_intersect(bd.Lw[p], bd.Uw[p], nullptr, nullptr, pass_out, B, np, s));
+            // the intersection and the relaxation in one pass over the layer
+            const float* bias;
+            long long pc;
+            relax_args(k, &bias, &pc);
+            LAUNCH(net, launch_relu_bounds_relax(nullptr, nullptr, nullptr, pass_out, bd.Lw[p], bd.Uw[p],
+                                                 o.alpha ? o.alpha[k] : nullptr, B, np, P[k], bias, pc, sound, s));
+            continue;
         }
+        if (!refined(k)) continue;  // relaxed together with its bounds above
         const Node& sn = net->nodes[p];
         const bool aff = sn.op == VF_DENSE || sn.op == VF_CONV2D;
         LAUNCH(net, launch_relax_params(bd.Lw[p], bd.Uw[p], o.alpha ? o.alpha[k] : nullptr, (long long)B * nd.n, P[k],
@@ -1430,6 +1494,7 @@ void vf_net_destroy(vf_net* net) {
         cudaFree(nd.WtLo);
         cudaFree(nd.rowsum_abs);
         cudaFree(nd.Wwin);
+        cudaFree(nd.Wtc);
     }
     cudaFree(net->d_err);
     for (auto e : net->ev_free) cudaEventDestroy(e);
@@ -1464,6 +1529,7 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
         net->conv_whole_warp = (strcmp(f, "warp") == 0) ? 1 : (strcmp(f, "tile") == 0 ? 0 : 2);
     if (const char* f = getenv("VF_CONV_WIN_KERNEL")) net->conv_win_per_position = (strcmp(f, "1") == 0) ? 1 : 0;
     if (const char* f = getenv("VF_COMPACT")) net->compact = atoi(f) != 0;
+    if (const char* f = getenv("VF_CONV_TC")) net->conv_tc = atoi(f) != 0;
     CU(cudaMalloc(&net->d_err, sizeof(int)));
     CU(cudaMemset(net->d_err, 0, sizeof(int)));
     net->nodes.resize(n_nodes);
@@ -1569,6 +1635,13 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
                     CU(cudaMalloc(&nd.Wwin, sizeof(float) * wt.size()));
                     CU(cudaMemcpy(nd.Wwin, wt.data(), sizeof(float) * wt.size(), cudaMemcpyHostToDevice));
                     nd.ww = WinWeights{nd.Wwin, ts, ci_pad, cb, net->conv_win_per_position};
+                }
+                if (conv_tc_weights_supported(g)) {  // operand images of the tensor-core kernel
+                    std::vector<float> w0((size_t)cnt), wt((size_t)conv_tc_wtc_floats(g));
+                    CU(cudaMemcpy(w0.data(), nd.W, sizeof(float) * cnt, cudaMemcpyDeviceToHost));
+                    conv_tc_pack_weights(g, w0.data(), wt.data());
+                    CU(cudaMalloc(&nd.Wtc, sizeof(float) * wt.size()));
+                    CU(cudaMemcpy(nd.Wtc, wt.data(), sizeof(float) * wt.size(), cudaMemcpyHostToDevice));
                 }
                 if (!conv_back_supported(g))
                     return fail(VF_ERR_UNSUPPORTED,
@@ -1833,7 +1906,7 @@ int vf_profile_enable(vf_net* net, int enable) {
 
 int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms, double* flops, int reset) {
     TRY(check_net(net));
-    if (kind < 0 || kind > 4) return fail(VF_ERR_ARG, "bad kernel kind");
+    if (kind < 0 || kind > 5) return fail(VF_ERR_ARG, "bad kernel kind");
     for (auto& t : net->ev_used) {
         CU(cudaEventSynchronize(t.e1));
         float ms = 0.f;
@@ -1851,7 +1924,7 @@ int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms
     if (total_ms) *total_ms = net->prof_ms[kind];
     if (flops) *flops = net->prof_flops[kind];
     if (reset)
-        for (int k = 0; k < 5; ++k) {
+        for (int k = 0; k < 6; ++k) {
             net->prof_launches[k] = 0;
             net->prof_ms[k] = 0.0;
             net->prof_flops[k] = 0.0;

@@ -140,6 +140,23 @@ cudaError_t launch_rewin_rows(const RowRef& A, Relax rx, long long M, int C, int
                               const Win& wa, const Win& wd, float* out, long long ld_out, int accumulate, float* cst,
                               cudaStream_t s);
 
+// ---- tensor-core convolution (k_back_conv_tc.cu) ----------------------------------------
+// The same step as launch_conv_back_win (rows over the conv output in window wa, relaxed on load, bias into
+// cst; out in window wd, or concretised into cst), as a tcgen05 implicit GEMM (3xTF32). Whole-map rows are
+// the window of the whole map (ay = ax = by = bx = 0). Conditions: C_in a multiple of 16 up to 128, k <= 8,
+// stride 1 or 2, and one row's shifted slabs within the TMEM and shared-memory plan. A STORE writes every entry
+// of wd only when conv_back_tc_covers(g, wa, wd); otherwise the caller clears the rows first. Writes *err on
+// a bounded-wait expiry.
+bool conv_tc_weights_supported(const ConvGeom& g);
+int conv_tc_wtc_floats(const ConvGeom& g);
+void conv_tc_pack_weights(const ConvGeom& g, const float* W, float* out);
+bool conv_back_tc_supported(const ConvGeom& g, const Win& wa, const Win& wd, int out_mode);
+bool conv_back_tc_covers(const ConvGeom& g, const Win& wa, const Win& wd);
+cudaError_t launch_conv_back_tc(const RowRef& A, Relax rx, const float* Wtc, const float* bias, long long M,
+                                const ConvGeom& g, PassGeom pg, PassStart ps, const Win& wa, const Win& wd,
+                                int out_mode, float* out, long long ld_out, float* cst, const float* centres,
+                                float eps, int* err, int num_sms, cudaStream_t s);
+
 // ---- IBP (k_ibp.cu) -------------------------------------------------------------------
 // rowsum_abs (optional): sum_k |W[n, k]|, used with `eps` when the source is the input box (radius eps everywhere).
 cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
@@ -165,6 +182,13 @@ cudaError_t launch_abs_rows_times_wt(const float* A, const float* Wabs, int M, i
 cudaError_t launch_relax_params(const float* l, const float* u, const float* alpha, long long n, float4* P,
                                 const float* bias, long long n_per_centre, long long per_channel, cudaStream_t s,
                                 int sound = 0);
+// One ReLU layer's bounds and relaxation in one pass over its B * n_layer neurons: bounds from the IBP
+// centre/radius (c, r given; as launch_bounds_from_cr) or read from l, u and intersected with a plain
+// pass's rows (pass_out given; as launch_intersect), then P as launch_relax_params. Falls back to those
+// launches when n_layer is not a multiple of 4 or an array is not 16-byte aligned.
+cudaError_t launch_relu_bounds_relax(const float* c, const float* r, const signed char* split, const float* pass_out,
+                                     float* l, float* u, const float* alpha, int B, long long n_layer, float4* P,
+                                     const float* bias, long long per_channel, int sound, cudaStream_t s);
 cudaError_t launch_cst_identity_bias(float* cst, long long M, PassGeom pg, const float* bias, long long n_p,
                                      long long per_channel, cudaStream_t s);
 cudaError_t launch_ident_rows(float* out, long long ld, long long M, PassGeom pg, long long n_p, int accumulate,

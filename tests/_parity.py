@@ -59,3 +59,23 @@ def sound_on_samples(net, centres, eps, C, lb, ub=None, n=2000, seed=0):
         if ub is not None and np.any(y > ub[b] + tol(y)):
             return False
     return True
+
+
+def kink_sensitive_rows(run, centres, eps, rows, rel=1e-6):
+    """Rows (centre b, row r) at a kink of an iterative computation: `run(centre_batch, eps)` -> [b, R] is the
+    oracle's result (fp64). A row whose result moves by more than the parity tolerance when eps changes by a
+    relative `rel` -- a change far below any tolerance, about the size of fp32 rounding in the inputs -- has a
+    discontinuity there (a branch of a decision flips), so fp32 and fp64 may legitimately end on different
+    branches. Returns a boolean mask over `rows` (a list of (b, r))."""
+    out = np.zeros(len(rows), bool)
+    by_centre = {}
+    for i, (b, r) in enumerate(rows):
+        by_centre.setdefault(b, []).append((i, r))
+    for b, items in by_centre.items():
+        base = run(centres[b:b + 1], eps)[0]
+        hi = run(centres[b:b + 1], eps * (1 + rel))[0]
+        lo = run(centres[b:b + 1], eps * (1 - rel))[0]
+        for i, r in items:
+            t = REL_TOL * (abs(base[r]) + 1.0)
+            out[i] = abs(hi[r] - base[r]) > t or abs(lo[r] - base[r]) > t
+    return out

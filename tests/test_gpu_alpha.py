@@ -5,7 +5,7 @@ import torch
 
 import oracle.lbp as O
 from linear_bound_propagation_b200 import synth
-from tests._parity import ambiguous_centres, sound_on_samples
+from tests._parity import ambiguous_centres, kink_sensitive_rows, sound_on_samples
 
 pytestmark = pytest.mark.gpu
 
@@ -59,9 +59,9 @@ def test_alpha_grad_matches_oracle(config, B):
         assert _viol(lb[b], olb).max() <= 1.0, f"centre {b}"
         for k, (o, n) in blocks.items():
             gg = grad[o + b * R * n: o + (b + 1) * R * n].reshape(R, n)
-            # gradient entries: compare where the oracle's coefficient sign is clear (the kink of the
-            # |.| and of the slope choice makes the gradient one-sided at lam = 0)
-            assert _viol(gg, og[k]).max() <= 10.0, f"centre {b} relu {k}: {_viol(gg, og[k]).max()}"
+            # every gradient entry at the parity tolerance (the gradient is a chain of fp32 contractions
+            # like the bound itself; the measured worst entry is well inside it)
+            assert _viol(gg, og[k]).max() <= 1.0, f"centre {b} relu {k}: {_viol(gg, og[k]).max()}"
         checked += 1
     assert checked >= B // 2
 
@@ -81,11 +81,33 @@ def test_alpha_crown_improves_soundly_and_tracks_oracle(config, B):
     amb = ambiguous_centres(res, net)
     ok = ~amb
     assert _viol(lb0[ok], res.lb_crown[ok]).max() <= 1.0
-    # the same 5 Adam steps in fp64 end within tolerance on all but a few rows (kinks may split them)
+    # the same 5 Adam steps in fp64 end within tolerance on every row that is not at a kink of the
+    # trajectory: a row may leave the oracle's value only if the oracle's own value jumps under a 1e-6
+    # relative change of eps (a slope step or a slope choice flips there)
     best, start = O.alpha_crown(net, w.centres, w.eps, w.C, iters=5, lr=0.1)
-    v = _viol(lb[ok], best[ok])
-    assert (v > 1.0).mean() <= 0.05, f"{(v > 1.0).mean():.3f} of rows off the oracle trajectory"
+    _assert_off_rows_at_kinks(net, w.centres, w.eps, w.C, lb, best, ok, iters=5)
     assert sound_on_samples(net, w.centres[:4], w.eps, w.C[:4] if w.C.shape[0] > 1 else w.C, lb[:4], None, n=2000)
+
+
+def _assert_off_rows_at_kinks(net, centres, eps, C, lb, best, ok, iters, splits=None):
+    """Every row of a centre without an adaptive-slope near-tie matches the oracle's optimised bound, or
+    sits at a kink of the optimisation (kink_sensitive_rows)."""
+    off = [(b, r) for b in range(lb.shape[0]) if ok[b] for r in range(lb.shape[1])
+           if _viol(lb[b, r], best[b, r]) > 1.0]
+    if not off:
+        return
+
+    by_b = {}
+    for b, r in off:
+        by_b.setdefault(b, []).append(r)
+    bad = []
+    for b, rs in by_b.items():
+        Cb = C[b:b + 1] if C.shape[0] > 1 else C
+        sp = None if splits is None else {k: v[b:b + 1] for k, v in splits.items()}
+        kink = kink_sensitive_rows(lambda c, e: O.alpha_crown(net, c, e, Cb, iters=iters, lr=0.1, splits=sp)[0],
+                                   centres[b:b + 1], eps, [(0, r) for r in rs])
+        bad += [(b, r) for r, k in zip(rs, kink) if not k]
+    assert not bad, f"rows off the oracle's trajectory without a kink: {bad[:8]} (of {len(off)} off)"
 
 
 def _small_residual(seed=7, B=2):
@@ -123,7 +145,7 @@ def test_alpha_grad_matches_oracle_residual():
         assert _viol(lb[b], olb).max() <= 1.0, f"centre {b}"
         for k, (o, n) in blocks.items():
             gg = grad[o + b * R * n: o + (b + 1) * R * n].reshape(R, n)
-            assert _viol(gg, og[k]).max() <= 10.0, f"centre {b} relu {k}: {_viol(gg, og[k]).max()}"
+            assert _viol(gg, og[k]).max() <= 1.0, f"centre {b} relu {k}: {_viol(gg, og[k]).max()}"
         checked += 1
     assert checked >= 1
 
@@ -140,8 +162,7 @@ def test_alpha_crown_residual_improves_soundly():
     ok = ~ambiguous_centres(res, net)
     assert _viol(lb0[ok], res.lb_crown[ok]).max() <= 1.0
     best, start = O.alpha_crown(net, centres, eps, C, iters=5, lr=0.1)
-    v = _viol(lb[ok], best[ok])
-    assert (v > 1.0).mean() <= 0.1, f"{(v > 1.0).mean():.3f} of rows off the oracle trajectory"
+    _assert_off_rows_at_kinks(net, centres, eps, C, lb, best, ok, iters=5)
     assert sound_on_samples(net, centres, eps, C, lb, None, n=2000)
 
 

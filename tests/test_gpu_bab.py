@@ -10,6 +10,7 @@ import torch
 import oracle.lbp as O
 from linear_bound_propagation_b200 import synth
 from tests._parity import ambiguous_centres, max_violation
+from tests.test_gpu_alpha import _assert_off_rows_at_kinks
 
 pytestmark = pytest.mark.gpu
 
@@ -132,8 +133,8 @@ def test_alpha_beta_gradient_matches_oracle(kind):
         olb, og, obg = O.spec_bound_alpha(net, centres[b], eps, C[b], relax, a, {k: sp[k][b] for k in sp}, bt)
         assert _viol(lb[b], olb).max() <= 1.0, f"centre {b}"
         for k, (o, n) in blocks.items():
-            assert _viol(cut(ga, o, n), og[k]).max() <= 10.0, f"centre {b} relu {k}: slope gradient"
-            assert _viol(cut(gb, o, n), obg[k]).max() <= 10.0, f"centre {b} relu {k}: beta gradient"
+            assert _viol(cut(ga, o, n), og[k]).max() <= 1.0, f"centre {b} relu {k}: slope gradient"
+            assert _viol(cut(gb, o, n), obg[k]).max() <= 1.0, f"centre {b} relu {k}: beta gradient"
             assert np.all(cut(gb, o, n)[:, sp[k][b] == 0] == 0.0)
         checked += 1
     assert checked >= 1
@@ -153,8 +154,9 @@ def test_alpha_crown_with_splits_tracks_oracle():
     ok = ~ambiguous_centres(res, net)
     assert _viol(lb0[ok], res.lb_crown[ok]).max() <= 1.0
     best, _ = O.alpha_crown(net, centres, eps, C, iters=10, lr=0.1, splits=sp)
-    v = _viol(lb[ok], best[ok])
-    assert (v > 1.0).mean() <= 0.1, f"{(v > 1.0).mean():.3f} of rows off the oracle trajectory"
+    # every row matches the oracle's trajectory or sits at a kink of it (its oracle value jumps under a 1e-6
+    # relative change of eps)
+    _assert_off_rows_at_kinks(net, centres, eps, C, lb, best, ok, iters=10, splits=sp)
     # sound on the subdomains: sampled inputs that satisfy a centre's splits stay above its bound
     for b in range(centres.shape[0]):
         xs = centres[b] + eps * (2 * rng.random((20000, centres.shape[1])) - 1)
