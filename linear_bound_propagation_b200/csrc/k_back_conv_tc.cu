@@ -86,6 +86,7 @@ struct ConvTcParams {
     int wpi, items;           // warps per row in the staging, staging items per row and chunk
     int abuf, acc_cols;       // accumulator sets, TMEM columns per set
     int a_stage_bytes, w_stage_bytes, w_off, rc_off, rt_off, cp_off;  // shared-memory plan
+    int w_resident;  // 1: every chunk's weights loaded once per CTA (w region = all of Wtc), else per chunk
     float inv_plane, inv_wa, inv_npos, inv_p;  // 1 / (Ha Wa), 1 / Wa, 1 / npos_img, 1 / P (exact quotients, fdiv)
     int out_mode;
     float* out;
@@ -169,13 +170,15 @@ __device__ __forceinline__ void epi_block16(const ConvTcParams& p, bool act, boo
     }
 }
 
-// Stage U items of one row for output-channel chunk c: item e = (4-channel half h, window position) holds the
-// row's four coefficients of that half at that position, relaxed, split into tf32 head and remainder and
-// written to the operand stage `sa`; the row-constant terms go to *cs. Items at or past p.items are skipped.
+// Stage U items for output-channel chunk c; item u belongs to row slot iu[u] (table entry rgu[u], relaxation
+// base Pbu[u]) and has index eu[u] in that row: e = (4-channel half h, window position). Each holds the row's
+// four coefficients of that half at that position, relaxed, split into tf32 head and remainder and written to
+// the operand stage `sa`; its row-constant terms go to *csu[u]. Items at or past p.items are skipped. All loads
+// of the U items are issued before any is used.
 template <int U>
-__device__ __forceinline__ void stage_items(const ConvTcParams& p, int c, int i, int e0, int step, const RowGeo& rg,
-                                            const float* arow, const float4* Pb, int hw_o, uint8_t* sa,
-                                            int stage_half, float* cs) {
+__device__ __forceinline__ void stage_items(const ConvTcParams& p, int c, const int (&iu)[U], const int (&eu)[U],
+                                            const RowGeo* const (&rgu)[U], const float4* const (&Pbu)[U], int hw_o,
+                                            uint8_t* sa, int stage_half, float* const (&csu)[U]) {
     const int Wa = p.wa.hw, plane_a = p.wa.hh * p.wa.hw;
     float xv[U][4];
     float4 pr[U][4];
@@ -183,37 +186,40 @@ __device__ __forceinline__ void stage_items(const ConvTcParams& p, int c, int i,
     bool live[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-        const int e = e0 + u * step;
+        const int e = eu[u];
         live[u] = e < p.items;
         const int h = live[u] ? fdiv(e, p.inv_plane) : 0, pos = live[u] ? e - h * plane_a : 0;
         const int a = fdiv(pos, p.inv_wa), bb = pos - a * Wa;
-        const int oy = rg.aoy + a, ox = rg.aox + bb;
+        const int oy = rgu[u]->aoy + a, ox = rgu[u]->aox + bb;
         const bool on = live[u] && oy >= 0 && oy < p.g.ho && ox >= 0 && ox < p.g.wo;
         hh[u] = h;
-        tpos[u] = i * p.npos_img + (p.gy + a) * p.P + (p.gx + bb);
+        tpos[u] = iu[u] * p.npos_img + (p.gy + a) * p.P + (p.gx + bb);
+        const float* arow = rgu[u]->arow;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int co = 8 * c + 4 * h + j;
             const bool ld = on && co < p.g.co;
             xv[u][j] = ld ? __ldg(&arow[(long long)co * plane_a + pos]) : 0.f;
-            pr[u][j] = (ld && Pb != nullptr) ? __ldg(&Pb[(long long)co * hw_o + oy * p.g.wo + ox])
-                                             : make_float4(1.f, 1.f, 0.f, 0.f);
+            pr[u][j] = (ld && Pbu[u] != nullptr) ? __ldg(&Pbu[u][(long long)co * hw_o + oy * p.g.wo + ox])
+                                                 : make_float4(1.f, 1.f, 0.f, 0.f);
         }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         if (!live[u]) continue;
         float r[4];
+        float cs = *csu[u];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int co = 8 * c + 4 * hh[u] + j;
             const float x = xv[u][j];
             // off-map entries and padding channels hold x = 0, so they add nothing
             const float v = (x >= 0.f) ? x * pr[u][j].x : x * pr[u][j].y;
-            if (p.rx.count_const) *cs = fmaf(fminf(x, 0.f), pr[u][j].z, *cs);
-            if (p.bias != nullptr && co < p.g.co) *cs = fmaf(v, __ldg(&p.bias[co]), *cs);
+            if (p.rx.count_const) cs = fmaf(fminf(x, 0.f), pr[u][j].z, cs);
+            if (p.bias != nullptr && co < p.g.co) cs = fmaf(v, __ldg(&p.bias[co]), cs);
             r[j] = v;
         }
+        *csu[u] = cs;
         const float h0 = tf32_hi(r[0]), h1 = tf32_hi(r[1]), h2 = tf32_hi(r[2]), h3 = tf32_hi(r[3]);
         float4* hi = reinterpret_cast<float4*>(sa + (size_t)hh[u] * stage_half) + tpos[u];
         float4* lo = reinterpret_cast<float4*>(sa + (size_t)(2 + hh[u]) * stage_half) + tpos[u];
@@ -228,6 +234,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) conv_back_tc(const __grid_cons
     __shared__ uint64_t a_full[2], a_empty[2], acc_full[2], acc_empty[2], rc_full[2], rc_empty[2], done_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
+    __shared__ uint32_t tap_a16[MAX_TAPS], tap_b16[MAX_TAPS];  // per tap: operand offsets in 16-byte units
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long ngroups = (p.M + p.G - 1) / p.G;
@@ -235,6 +242,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) conv_back_tc(const __grid_cons
     float* cp = reinterpret_cast<float*>(base + p.cp_off);  // [nact * T * 128] concretised per position
     RowGeo* rt = reinterpret_cast<RowGeo*>(base + p.rt_off);  // [2][G] row table, by group parity
 
+    if (threadIdx.x < MAX_TAPS) {
+        const int tap = threadIdx.x;
+        tap_a16[tap] = (uint32_t)p.tap_shift[tap];
+        // B operand of tap w (chunk 0): resident weights are [tap][chunk][2 Np 4], a chunk stage [tap][2 Np 4]
+        tap_b16[tap] = (uint32_t)(p.tap_w[tap] * (p.w_resident ? p.nchunk : 1) * p.Np * 2);
+    }
     if (threadIdx.x == 0) {
         abort_sh = 0;
         for (int s = 0; s < 2; ++s) {
@@ -253,6 +266,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) conv_back_tc(const __grid_cons
         float4* z = reinterpret_cast<float4*>(base);
         const int n4 = p.a_stage_bytes / 16;  // two stages, each hi and lo, back to back
         for (int i = threadIdx.x; i < n4; i += NUM_THREADS) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (p.w_resident) {  // every chunk's weights, once
+            const float4* src = reinterpret_cast<const float4*>(p.Wtc);
+            float4* dst = reinterpret_cast<float4*>(base + p.w_off);
+            const int nw4 = p.g.k * p.g.k * p.nchunk * p.Np * 2;
+            for (int i = threadIdx.x; i < nw4; i += NUM_THREADS) dst[i] = __ldg(&src[i]);
+        }
         fence_proxy_async_smem();
     }
     if (warp == W_EPI0) {
@@ -297,8 +316,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) conv_back_tc(const __grid_cons
                                        mbar_wait(&a_empty[st], (uint32_t)((gc >> 1) - 1) & 1, abort_flag));
                 if (dead) continue;
                 uint8_t* sa = base + (size_t)st * 2 * 2 * stage_half;  // [hi: 2 halves][lo: 2 halves]
-                // this chunk's weights, every tap
-                {
+                // this chunk's weights, every tap (unless all chunks are resident)
+                if (!p.w_resident) {
                     const int per_tap4 = p.Np * 2;  // float4 per tap: [2][Np][4]
                     const float4* src = reinterpret_cast<const float4*>(p.Wtc);
                     float4* dst = reinterpret_cast<float4*>(base + p.w_off + (size_t)st * p.w_stage_bytes);
@@ -308,26 +327,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) conv_back_tc(const __grid_cons
                         dst[i] = __ldg(&src[((size_t)tap * p.nchunk + c) * per_tap4 + e]);
                     }
                 }
-                for (int i = warp / p.wpi; i < p.G; i += ngrp_par) {
-                    const long long m = m0 + i;
-                    if (m >= p.M) break;
-                    const RowGeo rg = tab[i];
-                    const float* arow = rg.arow;
-                    const float4* Pb = p.rx.P != nullptr ? p.rx.P + rg.b * nOut : nullptr;
-                    float cs = 0.f;
-                    // two items per lane per iteration (all sixteen loads issued before any is used) while the
-                    // row has them; the last iteration takes one when no lane has a second
-                    const int step = p.wpi * 32;
-                    for (int e0 = part * 32 + lane; __any_sync(0xffffffffu, e0 < p.items); e0 += 2 * step) {
-                        if (__any_sync(0xffffffffu, e0 + step < p.items))
-                            stage_items<2>(p, c, i, e0, step, rg, arow, Pb, hw_o, sa, stage_half, &cs);
-                        else
-                            stage_items<1>(p, c, i, e0, step, rg, arow, Pb, hw_o, sa, stage_half, &cs);
+                const int step = p.wpi * 32;
+                const int e0 = part * 32 + lane;
+                float* rcs = rc + (size_t)rs * p.G * p.wpi + part;
+                if (p.items <= step) {
+                    // one item per lane and row: two rows at a time, so sixteen loads are in flight per lane
+                    for (int i = warp / p.wpi; i < p.G; i += 2 * ngrp_par) {
+                        if (m0 + i >= p.M) break;
+                        const int i2 = i + ngrp_par;
+                        const bool two = i2 < p.G && m0 + i2 < p.M;
+                        float cs0 = 0.f, cs1 = 0.f;
+                        if (two) {
+                            const RowGeo* r0 = &tab[i];
+                            const RowGeo* r1 = &tab[i2];
+                            const float4* P0 = p.rx.P != nullptr ? p.rx.P + r0->b * nOut : nullptr;
+                            const float4* P1 = p.rx.P != nullptr ? p.rx.P + r1->b * nOut : nullptr;
+                            stage_items<2>(p, c, {i, i2}, {e0, e0}, {r0, r1}, {P0, P1}, hw_o, sa, stage_half,
+                                           {&cs0, &cs1});
+                        } else {
+                            const RowGeo* r0 = &tab[i];
+                            const float4* P0 = p.rx.P != nullptr ? p.rx.P + r0->b * nOut : nullptr;
+                            stage_items<1>(p, c, {i}, {e0}, {r0}, {P0}, hw_o, sa, stage_half, {&cs0});
+                        }
+                        cs0 = warp_sum32(cs0);
+                        cs1 = warp_sum32(cs1);
+                        if (lane == 0) {
+                            rcs[(size_t)i * p.wpi] = (c == 0) ? cs0 : rcs[(size_t)i * p.wpi] + cs0;
+                            if (two) rcs[(size_t)i2 * p.wpi] = (c == 0) ? cs1 : rcs[(size_t)i2 * p.wpi] + cs1;
+                        }
                     }
-                    cs = warp_sum32(cs);
-                    if (lane == 0) {
-                        float* slot = rc + ((size_t)rs * p.G + i) * p.wpi + part;
-                        *slot = (c == 0) ? cs : *slot + cs;
+                } else {
+                    for (int i = warp / p.wpi; i < p.G; i += ngrp_par) {
+                        if (m0 + i >= p.M) break;
+                        const RowGeo* r0 = &tab[i];
+                        const float4* P0 = p.rx.P != nullptr ? p.rx.P + r0->b * nOut : nullptr;
+                        float cs = 0.f;
+                        // two items of the row per lane and iteration while it has them, then one
+                        for (int e = e0; __any_sync(0xffffffffu, e < p.items); e += 2 * step) {
+                            if (__any_sync(0xffffffffu, e + step < p.items))
+                                stage_items<2>(p, c, {i, i}, {e, e + step}, {r0, r0}, {P0, P0}, hw_o, sa, stage_half,
+                                               {&cs, &cs});
+                            else
+                                stage_items<1>(p, c, {i}, {e}, {r0}, {P0}, hw_o, sa, stage_half, {&cs});
+                        }
+                        cs = warp_sum32(cs);
+                        if (lane == 0) rcs[(size_t)i * p.wpi] = (c == 0) ? cs : rcs[(size_t)i * p.wpi] + cs;
                     }
                 }
                 fence_proxy_async_smem();
@@ -340,6 +384,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) conv_back_tc(const __grid_cons
         if (lane == 0) {
             const uint32_t id_full = idesc_tf32(BM, p.Np), id_half = idesc_tf32(BM, p.C);
             const uint32_t lbo_a = (uint32_t)stage_half, lbo_b = (uint32_t)(p.Np * 16);
+            const uint64_t lo16 = (uint64_t)(2 * stage_half) >> 4;  // head -> remainder buffer, 16-byte units
             long long gc = 0;
             int it = 0;
             bool alive = true;
@@ -355,21 +400,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) conv_back_tc(const __grid_cons
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_u32(base + (size_t)st * 2 * 2 * stage_half);
-                    const uint32_t sw = smem_u32(base + p.w_off + (size_t)st * p.w_stage_bytes);
-                    for (int k = 0; k < p.nact; ++k)
-                        for (int t = 0; t < p.T; ++t) {
-                            const uint32_t d = acc0 + (uint32_t)((k * p.T + t) * p.Np);
-                            for (int j = 0; j < p.cls_nt[k]; ++j) {
-                                const int tap = p.cls_t0[k] + j;
-                                const uint32_t row = (uint32_t)(t * BM + p.tap_shift[tap]) * 16u;
-                                const uint64_t a_hi = noswz_desc(sa + row, lbo_a, 128);
-                                const uint64_t a_lo = noswz_desc(sa + 2 * stage_half + row, lbo_a, 128);
-                                const uint64_t b = noswz_desc(sw + (uint32_t)(p.tap_w[tap] * p.Np * 32), lbo_b, 128);
-                                mma_tf32_ss(d, a_hi, b, id_full, (c > 0 || j > 0) ? 1u : 0u);
-                                mma_tf32_ss(d, a_lo, b, id_half, 1u);
-                            }
+                    // descriptors of this stage; a tap or tile moves only the 14-bit start-address field (the
+                    // shared-memory window is below 256 KB, so the sum never carries out of it)
+                    const uint64_t da = noswz_desc(smem_u32(base + (size_t)st * 2 * 2 * stage_half), lbo_a, 128);
+                    const uint64_t db =
+                        p.w_resident ? noswz_desc(smem_u32(base + p.w_off), lbo_b, 128) + (uint64_t)(c * p.Np * 2)
+                                     : noswz_desc(smem_u32(base + p.w_off + (size_t)st * p.w_stage_bytes), lbo_b, 128);
+                    // taps outermost, tiles innermost: consecutive MMAs go to different accumulators, so
+                    // they overlap in the tensor pipe instead of each waiting for the previous one's result
+                    for (int k = 0; k < p.nact; ++k) {
+                        const int t0 = p.cls_t0[k], nt = p.cls_nt[k];
+                        const uint32_t dk = acc0 + (uint32_t)(k * p.T * p.Np);
+                        for (int j = 0; j < nt; ++j) {
+                            const uint64_t a_tap = da + tap_a16[t0 + j];
+                            const uint64_t b = db + tap_b16[t0 + j];
+                            const uint32_t acc = (c > 0 || j > 0) ? 1u : 0u;
+                            for (int t = 0; t < p.T; ++t)
+                                mma_tf32_ss(dk + (uint32_t)(t * p.Np), a_tap + (uint64_t)(t * BM), b, id_full, acc);
+                            for (int t = 0; t < p.T; ++t)
+                                mma_tf32_ss(dk + (uint32_t)(t * p.Np), a_tap + (uint64_t)(t * BM) + lo16, b, id_half, 1u);
                         }
+                    }
                     mma_commit(&a_empty[st]);
                 }
                 if (!alive) break;
@@ -555,6 +606,9 @@ bool plan(const ConvGeom& g, const Win& wa, const Win& wd, int out_mode, ConvTcP
     int vt = (p.items + 31) / 32;
     p.wpi = vt >= 8 ? 8 : (vt >= 4 ? 4 : (vt >= 2 ? 2 : 1));
     p.w_stage_bytes = g.k * g.k * p.Np * 32;
+    const int w_all = p.w_stage_bytes * p.nchunk;
+    p.w_resident = w_all <= 64 * 1024 ? 1 : 0;
+    const int w_bytes = p.w_resident ? w_all : 2 * p.w_stage_bytes;
     // largest group (rows per CTA round) that fits TMEM and shared memory; two accumulator sets if possible
     for (int abuf = 2; abuf >= 1; --abuf) {
         const int cols = (int)TMEM_COLS / abuf;
@@ -566,7 +620,7 @@ bool plan(const ConvGeom& g, const Win& wa, const Win& wd, int out_mode, ConvTcP
             const int rc_bytes = 2 * G * p.wpi * 4;
             const int rt_bytes = 2 * G * (int)sizeof(RowGeo);
             const int cp_bytes = out_mode == OUT_CONCRETIZE ? p.nact * T * BM * 4 : 0;
-            const int total = 2 * a_stage + 2 * p.w_stage_bytes + rc_bytes + rt_bytes + 64 + cp_bytes + 1024;
+            const int total = 2 * a_stage + w_bytes + rc_bytes + rt_bytes + 64 + cp_bytes + 1024;
             if (total > SMEM_LIMIT || NPOS * 16 >= (1 << 18)) continue;
             p.G = G;
             p.T = T;
@@ -575,7 +629,7 @@ bool plan(const ConvGeom& g, const Win& wa, const Win& wd, int out_mode, ConvTcP
             p.acc_cols = cols;
             p.a_stage_bytes = 2 * a_stage;  // both stages
             p.w_off = 2 * a_stage;
-            p.rc_off = p.w_off + 2 * p.w_stage_bytes;
+            p.rc_off = p.w_off + w_bytes;
             p.rt_off = p.rc_off + (rc_bytes + 15) / 16 * 16;
             p.cp_off = p.rt_off + (rt_bytes + 63) / 64 * 64;
             p.inv_plane = 1.f / (float)(wa.hh * wa.hw);
