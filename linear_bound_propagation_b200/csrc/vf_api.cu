@@ -76,6 +76,7 @@ struct Node {
     float* rowsum_abs = nullptr;  // dense only: sum_k |W[n, k]| (IBP radius of a layer fed by the input box)
     float* Wwin = nullptr;        // conv only: weights in the tap-major layout of the windowed kernel
     float* Wtc = nullptr;         // conv only: 3xTF32 operand images of the tensor-core kernel (or null)
+    float* Wtn = nullptr;         // conv only: the same with the taps in N (k_back_conv_tcn.cu), or null
     WinWeights ww{nullptr, 0, 0, 4, 0};
     int consumers = 0;
 };
@@ -101,6 +102,7 @@ struct vf_net {
     int conv_win_per_position = 0;  // windowed rows without position blocking (VF_CONV_WIN_KERNEL=1)
     int compact = 1;        // intermediate passes over IBP-unstable neurons only (VF_COMPACT=0: off)
     int conv_tc = 1;        // convolution steps on the tensor cores where the shapes allow (VF_CONV_TC=0: off)
+    int conv_tcn = 0;       // ... with the taps-in-N kernel where its shapes allow (VF_CONV_TC=tapn; measured slower)
     int call_sound = 0;     // set for the duration of a vf_opts.sound call: contractions take FFMA kernels
     bool prof = false;
     std::vector<cudaEvent_t> ev_free;
@@ -545,8 +547,10 @@ struct Walker {
                 const bool fuse_in = (nd.src == 0 && ext_in == nullptr && net->nodes[0].consumers == 1 &&
                                       sw == nullptr && pend[0].kind == E_NONE);
                 const Win wa_tc = e.windowed ? e.win : full_win(nd);
-                if (net->conv_tc && !net->call_sound && sw == nullptr && nd.Wtc != nullptr &&
-                    conv_back_tc_supported(g, wa_tc, full_win(sn), OUT_CONCRETIZE)) {
+                const bool tcn = net->conv_tc && net->conv_tcn && !net->call_sound && sw == nullptr &&
+                                 nd.Wtn != nullptr && conv_back_tcn_supported(g, wa_tc, full_win(sn), OUT_CONCRETIZE);
+                if (tcn || (net->conv_tc && !net->call_sound && sw == nullptr && nd.Wtc != nullptr &&
+                            conv_back_tc_supported(g, wa_tc, full_win(sn), OUT_CONCRETIZE))) {
                     // tensor-core implicit GEMM, for whole-map and windowed rows alike
                     float* out = nullptr;
                     long long ld = 0;
@@ -566,8 +570,12 @@ struct Walker {
                             CU(cudaMemset2DAsync(out, sizeof(float) * ld, 0, sizeof(float) * win_len(dst), M, s));
                         cudaEvent_t e0 = nullptr;
                         prof_begin(&e0);
-                        LAUNCH(net, launch_conv_back_tc(e.ref, e.rx, nd.Wtc, nd.b, M, g, pg, ps, wa_tc, dst, mode, out,
-                                                        ld, cst, centres, eps, net->d_err, net->num_sms, s));
+                        if (tcn)
+                            LAUNCH(net, launch_conv_back_tcn(e.ref, e.rx, nd.Wtn, nd.b, M, g, pg, ps, wa_tc, dst, mode,
+                                                             out, ld, cst, centres, eps, net->d_err, net->num_sms, s));
+                        else
+                            LAUNCH(net, launch_conv_back_tc(e.ref, e.rx, nd.Wtc, nd.b, M, g, pg, ps, wa_tc, dst, mode,
+                                                            out, ld, cst, centres, eps, net->d_err, net->num_sms, s));
                         const Win nat = win_back(wa_tc, g);
                         const double pos = (double)std::min<long long>((long long)nat.hh * nat.hw, (long long)g.h * g.w);
                         prof_end(e0, VF_KERNEL_CONV_TC, 2.0 * (double)M * pos * g.ci * g.co * g.k * g.k /
@@ -1495,6 +1503,7 @@ void vf_net_destroy(vf_net* net) {
         cudaFree(nd.rowsum_abs);
         cudaFree(nd.Wwin);
         cudaFree(nd.Wtc);
+        cudaFree(nd.Wtn);
     }
     cudaFree(net->d_err);
     for (auto e : net->ev_free) cudaEventDestroy(e);
@@ -1529,7 +1538,10 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
         net->conv_whole_warp = (strcmp(f, "warp") == 0) ? 1 : (strcmp(f, "tile") == 0 ? 0 : 2);
     if (const char* f = getenv("VF_CONV_WIN_KERNEL")) net->conv_win_per_position = (strcmp(f, "1") == 0) ? 1 : 0;
     if (const char* f = getenv("VF_COMPACT")) net->compact = atoi(f) != 0;
-    if (const char* f = getenv("VF_CONV_TC")) net->conv_tc = atoi(f) != 0;
+    if (const char* f = getenv("VF_CONV_TC")) {
+        net->conv_tc = strcmp(f, "0") != 0;
+        net->conv_tcn = strcmp(f, "tapn") == 0;
+    }
     CU(cudaMalloc(&net->d_err, sizeof(int)));
     CU(cudaMemset(net->d_err, 0, sizeof(int)));
     net->nodes.resize(n_nodes);
@@ -1642,6 +1654,12 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
                     conv_tc_pack_weights(g, w0.data(), wt.data());
                     CU(cudaMalloc(&nd.Wtc, sizeof(float) * wt.size()));
                     CU(cudaMemcpy(nd.Wtc, wt.data(), sizeof(float) * wt.size(), cudaMemcpyHostToDevice));
+                    if (const int nwn = conv_tcn_wtn_floats(g)) {  // the taps-in-N operand images
+                        std::vector<float> wn((size_t)nwn);
+                        conv_tcn_pack_weights(g, w0.data(), wn.data());
+                        CU(cudaMalloc(&nd.Wtn, sizeof(float) * wn.size()));
+                        CU(cudaMemcpy(nd.Wtn, wn.data(), sizeof(float) * wn.size(), cudaMemcpyHostToDevice));
+                    }
                 }
                 if (!conv_back_supported(g))
                     return fail(VF_ERR_UNSUPPORTED,

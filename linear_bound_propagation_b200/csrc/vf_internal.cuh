@@ -157,6 +157,20 @@ cudaError_t launch_conv_back_tc(const RowRef& A, Relax rx, const float* Wtc, con
                                 int out_mode, float* out, long long ld_out, float* cst, const float* centres,
                                 float eps, int* err, int num_sms, cudaStream_t s);
 
+// ---- tensor-core convolution with the taps in N (k_back_conv_tcn.cu) ------------------------
+// The same step as launch_conv_back_tc with one GEMM column per (tap, input channel): three large MMAs per tile
+// and 8 output channels; the taps are summed in shared memory. Conditions: C_in a multiple of 16, C_in k^2 <= 512
+// in at most four groups of <= 256 columns, k <= 8, and one row's natural window within shared memory.
+// conv_tcn_wtn_floats is 0 when the weights do not fit the scheme. The same coverage rule as
+// conv_back_tc_covers applies to STOREs.
+int conv_tcn_wtn_floats(const ConvGeom& g);
+void conv_tcn_pack_weights(const ConvGeom& g, const float* W, float* out);
+bool conv_back_tcn_supported(const ConvGeom& g, const Win& wa, const Win& wd, int out_mode);
+cudaError_t launch_conv_back_tcn(const RowRef& A, Relax rx, const float* Wtn, const float* bias, long long M,
+                                 const ConvGeom& g, PassGeom pg, PassStart ps, const Win& wa, const Win& wd,
+                                 int out_mode, float* out, long long ld_out, float* cst, const float* centres,
+                                 float eps, int* err, int num_sms, cudaStream_t s);
+
 // ---- IBP (k_ibp.cu) -------------------------------------------------------------------
 // rowsum_abs (optional): sum_k |W[n, k]|, used with `eps` when the source is the input box (radius eps everywhere).
 cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,

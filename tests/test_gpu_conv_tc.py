@@ -1,5 +1,6 @@
-"""GPU parity of the tensor-core convolution step (conv_back_tc: tcgen05 implicit GEMM, 3xTF32) against the
-fp64 oracle, through the C ABI.
+"""GPU parity of the tensor-core convolution step against the fp64 oracle, through the C ABI. Two kernels do it,
+both tcgen05 implicit GEMMs with the 3xTF32 split: conv_back_tc (tap shifts, the default) and conv_back_tcn (taps
+in the N dimension, chosen with VF_CONV_TC=tapn where its shapes allow; measured slower, kept tested).
 
 The kernel takes every convolution back-substitution whose input has a multiple of 16 channels (up to 128),
 kernel size up to 8 and stride 1 or 2: whole-map rows, receptive-field windows, stored, accumulated (residual
@@ -71,12 +72,14 @@ def _run(net, centres, eps, C, both=True, workspace=0):
     return g, {k: v.cpu().numpy() for k, v in out.items()}, tc
 
 
+@pytest.mark.parametrize("kernel", ["1", "tapn"])
 @pytest.mark.parametrize("compact", ["1", "0"])
 @pytest.mark.parametrize("windows", ["1", "0"])
 @pytest.mark.parametrize("case", list(CASES))
-def test_conv_tc_matches_oracle(monkeypatch, case, windows, compact):
+def test_conv_tc_matches_oracle(monkeypatch, case, windows, compact, kernel):
     monkeypatch.setenv("VF_CONV_WINDOWS", windows)
     monkeypatch.setenv("VF_COMPACT", compact)
+    monkeypatch.setenv("VF_CONV_TC", kernel)
     net, centres, C, eps = CASES[case]()
     ora = O.verify(net, centres, eps, C, both_sides=True)
     g, out, tc = _run(net, centres, eps, C)
@@ -84,11 +87,13 @@ def test_conv_tc_matches_oracle(monkeypatch, case, windows, compact):
     assert_parity(net, centres, eps, C, g, ora, out, both=True)
 
 
+@pytest.mark.parametrize("kernel", ["1", "tapn"])
 @pytest.mark.parametrize("case", list(CASES))
-def test_conv_tc_row_blocks_are_bitwise_stable(case):
+def test_conv_tc_row_blocks_are_bitwise_stable(monkeypatch, case, kernel):
     """Each row's arithmetic depends only on its own window: the same bounds, bit for bit, when a pass is
     cut into many small row blocks (a small workspace), i.e. when rows share tensor-core groups with other
     rows and sit at other places in them."""
+    monkeypatch.setenv("VF_CONV_TC", kernel)
     net, centres, C, eps = CASES[case]()
     _, a, _ = _run(net, centres, eps, C)
     _, b, _ = _run(net, centres, eps, C, workspace=6 << 20)
@@ -102,14 +107,15 @@ def test_conv_tc_and_ffma_agree_on_workloads(monkeypatch, config, B):
     parity tolerance, and the oracle's on the centres it finishes quickly."""
     w = synth.workload(config, B=B)
     res = {}
-    for on in ("1", "0"):
+    for on in ("1", "tapn", "0"):
         monkeypatch.setenv("VF_CONV_TC", on)
         _, out, tc = _run(w.net, w.centres, w.eps, w.C, both=False)
-        assert (tc > 0) == (on == "1")
+        assert (tc > 0) == (on != "0")
         res[on] = out
-    assert max_violation(res["1"]["lb"], res["0"]["lb"]) <= 1.0
-    assert max_violation(res["1"]["pre_lb"], res["0"]["pre_lb"]) <= 1.0
-    assert max_violation(res["1"]["pre_ub"], res["0"]["pre_ub"]) <= 1.0
+    for on in ("1", "tapn"):
+        assert max_violation(res[on]["lb"], res["0"]["lb"]) <= 1.0
+        assert max_violation(res[on]["pre_lb"], res["0"]["pre_lb"]) <= 1.0
+        assert max_violation(res[on]["pre_ub"], res["0"]["pre_ub"]) <= 1.0
     if config == 3:
         ora = O.verify(w.net, w.centres[:2], w.eps, w.C[:2])
         assert max_violation(res["1"]["lb"][:2], ora.lb) <= 1.0
