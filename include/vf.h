@@ -202,11 +202,15 @@ int vf_alpha_beta_grad(vf_net* net, const float* centres, int B, float eps, cons
  * complete verification by beta-CROWN with branch-and-bound; the page names the method only). The
  * property: every row of C [device] [R, n_L] is positive at every input of the box centre [device] [n0]
  * +/- eps. The search, run on the host with every bound computed on the device:
- *   1. a row < 0 at the centre itself is a counterexample (VF_BAB_FALSIFIED). The fp32 value at the centre
- *      is only a rounded evaluation, so a negative row is confirmed by the sound-in-fp32 mode (vf_opts.sound,
- *      both sides, eps = 0): FALSIFIED needs that mode's upper bound, which the exact value on the fp32
- *      weights cannot exceed, to be < 0 on some row; a row within rounding of 0 is not a counterexample
- *      and the search goes on;
+ *   1. candidate counterexamples, before any subdomain is bounded: the centre, then (when some row's bound
+ *      over the whole box is <= 0) every row r's CROWN minimiser vertex x*_r = centre - eps * sign(lam_r),
+ *      lam_r the row's back-substituted input coefficients (vf_crown_backward with the whole box's
+ *      intermediate bounds), where the row's linear lower bound is attained; each coordinate is rounded
+ *      towards the centre so every point lies inside the box. A row < 0 at one of these inputs is a
+ *      counterexample (VF_BAB_FALSIFIED). The fp32 value there is only a rounded evaluation, so a negative
+ *      row is confirmed by the sound-in-fp32 mode (vf_opts.sound, both sides, eps = 0): FALSIFIED needs that
+ *      mode's upper bound, which the exact value on the fp32 weights cannot exceed, to be < 0 on some row; a
+ *      row within rounding of 0 is not a counterexample and the search goes on;
  *   2. a subdomain's row bound is the larger of vf_verify_batch's and vf_alpha_crown's (alpha_iters Adam
  *      steps of size lr on the slopes and the split multipliers); the whole box is bounded first;
  *   3. each round takes the open subdomains with the lowest bound (ties: created first), at most
@@ -233,11 +237,11 @@ typedef struct {
 } vf_bab_opts;
 typedef struct {
     int status;             /* VF_BAB_VERIFIED, VF_BAB_FALSIFIED or VF_BAB_UNKNOWN */
-    long long domains;      /* subdomains bounded, the whole box included (0 when falsified at the centre) */
+    long long domains;      /* subdomains bounded, the whole box included (0 when falsified by step 1) */
     int rounds;             /* batched rounds after the whole box */
     int max_depth;          /* most splits in one bounded subdomain */
     float lb;               /* lowest row bound of the subdomains open at the end (+inf if none); when
-                               falsified, the lowest row value at the centre */
+                               falsified, the lowest fp32 row value at the candidate inputs that decided */
 } vf_bab_result;
 int vf_bab_verify(vf_net* net, const float* centre, float eps, const float* C, int R, const vf_bab_opts* opts,
                   vf_bab_result* result /*[host]*/, void* stream);

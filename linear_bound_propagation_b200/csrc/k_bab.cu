@@ -92,7 +92,28 @@ __global__ void repeat_row_k(const float* __restrict__ src, long long n, int D, 
         dst[e] = src[e % n];
 }
 
+// x[r, i] = the vertex of the box centre +/- eps where row r's linear lower bound lam[r, :] . x + const is
+// smallest: centre - eps where lam > 0, centre + eps where lam < 0, the centre where lam = 0. The fp32 sum or
+// difference is rounded towards the centre (__fsub_ru / __fadd_rd), so every point lies inside the box.
+__global__ void minimiser_points_k(const float* __restrict__ centre, const float* __restrict__ lam, float eps,
+                                   long long n, int R, float* __restrict__ x) {
+    const long long total = n * R;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const float c = centre[e % n], l = lam[e];
+        x[e] = l > 0.f ? __fsub_ru(c, eps) : (l < 0.f ? __fadd_rd(c, eps) : c);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_minimiser_points(const float* centre, const float* lam, float eps, long long n, int R, float* x,
+                                    cudaStream_t s) {
+    long long g = (n * R + 255) / 256;
+    if (g > 148LL * 32) g = 148LL * 32;
+    minimiser_points_k<<<(unsigned)(g < 1 ? 1 : g), 256, 0, s>>>(centre, lam, eps, n, R, x);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_bab_pick(const float* pre_lb, const float* pre_ub, int D, const long long* blk_off, const int* blk_n,
                             const int* gbase, int nl, const float* lb_a, const float* lb_b, int R, BabPick* out,

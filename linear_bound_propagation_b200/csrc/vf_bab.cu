@@ -203,31 +203,65 @@ extern "C" int vf_bab_verify(vf_net* net, const float* centre, float eps, const 
     }
     BAB_CU(vf::launch_repeat_row(centre, n0, D, cen.get<float>(), s));
 
-    // ---- 1. the centre itself
-    {
+    // ---- 1. candidate counterexamples: the centre, then every row's CROWN minimiser vertex of the box.
+    // A negative row at a point is a rounded evaluation: it counts only when the sound mode's upper bound
+    // there (both sides, eps = 0), which the exact value C f(x) on the fp32 weights cannot exceed, is < 0.
+    auto falsified_at = [&](const float* xs, int P, float* ymin_out, bool* hit) -> int {
+        *hit = false;
+        DeviceBuffer y, yub;
+        BAB_CU(cudaMalloc(&y.p, sizeof(float) * (size_t)P * R));
+        BAB_CU(cudaMalloc(&yub.p, sizeof(float) * (size_t)P * R));
         vf_opts o{};
         o.relu_crown = opts->relu_crown;
-        BAB_TRY(vf_verify_batch(net, cen.get<float>(), 1, 0.f, C, R, 0, &o, lbv.get<float>(), nullptr, nullptr, nullptr,
-                                stream));
-        std::vector<float> y(R);
-        BAB_CU(cudaMemcpyAsync(y.data(), lbv.p, sizeof(float) * R, cudaMemcpyDeviceToHost, s));
+        BAB_TRY(vf_verify_batch(net, xs, P, 0.f, C, R, 0, &o, y.get<float>(), nullptr, nullptr, nullptr, stream));
+        std::vector<float> h((size_t)P * R);
+        BAB_CU(cudaMemcpyAsync(h.data(), y.p, sizeof(float) * h.size(), cudaMemcpyDeviceToHost, s));
         BAB_CU(cudaStreamSynchronize(s));
-        const float ymin = *std::min_element(y.begin(), y.end());
-        if (ymin < 0.f) {
-            // a rounded evaluation: confirm with the sound mode's upper bound at the centre, which the exact
-            // value C f(centre) on the fp32 weights cannot exceed
-            DeviceBuffer ub;
-            BAB_CU(cudaMalloc(&ub.p, sizeof(float) * R));
-            vf_opts so{};
-            so.relu_crown = opts->relu_crown;
-            so.both_sides = 1;
-            so.sound = 1;
-            BAB_TRY(vf_verify_batch(net, cen.get<float>(), 1, 0.f, C, R, 0, &so, lbv.get<float>(), ub.get<float>(),
-                                    nullptr, nullptr, stream));
-            std::vector<float> yu(R);
-            BAB_CU(cudaMemcpyAsync(yu.data(), ub.p, sizeof(float) * R, cudaMemcpyDeviceToHost, s));
-            BAB_CU(cudaStreamSynchronize(s));
-            if (*std::min_element(yu.begin(), yu.end()) < 0.f) {
+        *ymin_out = *std::min_element(h.begin(), h.end());
+        if (!(*ymin_out < 0.f)) return VF_OK;
+        vf_opts so = o;
+        so.both_sides = 1;
+        so.sound = 1;
+        BAB_TRY(vf_verify_batch(net, xs, P, 0.f, C, R, 0, &so, y.get<float>(), yub.get<float>(), nullptr, nullptr,
+                                stream));
+        BAB_CU(cudaMemcpyAsync(h.data(), yub.p, sizeof(float) * h.size(), cudaMemcpyDeviceToHost, s));
+        BAB_CU(cudaStreamSynchronize(s));
+        *hit = *std::min_element(h.begin(), h.end()) < 0.f;
+        return VF_OK;
+    };
+    {
+        float ymin = 0.f;
+        bool hit = false;
+        BAB_TRY(falsified_at(cen.get<float>(), 1, &ymin, &hit));
+        if (hit) {
+            *result = vf_bab_result{VF_BAB_FALSIFIED, 0, 0, 0, ymin};
+            return VF_OK;
+        }
+    }
+    {
+        // the whole box's bounds (no split); only a row the box does not already prove positive can fall below
+        // 0 at its vertex, so the attack is skipped when every row's bound is > 0
+        vf_opts o{};
+        o.relu_crown = opts->relu_crown;
+        o.pre_lb = plb.get<float>();
+        o.pre_ub = pub.get<float>();
+        BAB_TRY(vf_verify_batch(net, cen.get<float>(), 1, eps, C, R, 0, &o, lbv.get<float>(), nullptr, nullptr, nullptr,
+                                stream));
+        std::vector<float> h(R);
+        BAB_CU(cudaMemcpyAsync(h.data(), lbv.p, sizeof(float) * R, cudaMemcpyDeviceToHost, s));
+        BAB_CU(cudaStreamSynchronize(s));
+        if (!(*std::min_element(h.begin(), h.end()) > 0.f)) {
+            DeviceBuffer lam, cst, xs;
+            BAB_CU(cudaMalloc(&lam.p, sizeof(float) * (size_t)R * n0));
+            BAB_CU(cudaMalloc(&cst.p, sizeof(float) * (size_t)R));
+            BAB_CU(cudaMalloc(&xs.p, sizeof(float) * (size_t)R * n0));
+            BAB_TRY(vf_crown_backward(net, nn - 1, C, R, 0, plb.get<float>(), pub.get<float>(), nullptr, 1,
+                                      lam.get<float>(), cst.get<float>(), stream));
+            BAB_CU(vf::launch_minimiser_points(centre, lam.get<float>(), eps, n0, R, xs.get<float>(), s));
+            float ymin = 0.f;
+            bool hit = false;
+            BAB_TRY(falsified_at(xs.get<float>(), R, &ymin, &hit));
+            if (hit) {
                 *result = vf_bab_result{VF_BAB_FALSIFIED, 0, 0, 0, ymin};
                 return VF_OK;
             }

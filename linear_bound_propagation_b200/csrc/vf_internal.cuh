@@ -305,6 +305,10 @@ cudaError_t launch_bab_pick(const float* pre_lb, const float* pre_ub, int D, con
                             cudaStream_t s);
 // dst[d, :] = src[:] for d < D (n floats per row).
 cudaError_t launch_repeat_row(const float* src, long long n, int D, float* dst, cudaStream_t s);
+// Row r's CROWN minimiser vertex of the box centre +/- eps: x[r, :] = centre - eps * sign(lam[r, :]), each
+// coordinate rounded towards the centre so it stays inside the box. centre [n], lam and x [R, n], device.
+cudaError_t launch_minimiser_points(const float* centre, const float* lam, float eps, long long n, int R, float* x,
+                                    cudaStream_t s);
 
 // Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per (kernel,
 // device, size); safe to call from several threads.

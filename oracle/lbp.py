@@ -599,7 +599,8 @@ def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_rel
     A subdomain's row bound is the larger of ``verify``'s bound and the best bound of ``alpha_crown``
     (``iters`` Adam steps of size ``lr`` on the slopes and on the split multipliers beta).
     Reading of the search (one plain best-first variant):
-      1. the centre is evaluated first; a row < 0 there is a counterexample ("falsified");
+      1. the centre is evaluated first, then every row's CROWN minimiser vertex of the whole box
+         (``minimiser_attack``); a row < 0 at any of these inputs is a counterexample ("falsified");
       2. the whole box is bounded; if every row's lower bound is > 0 it is "verified";
       3. otherwise the open subdomains are kept with their lowest row bound; each round takes the
          (at most batch // 2) open subdomains with the lowest bound (ties: created first), splits each
@@ -617,6 +618,9 @@ def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_rel
     y = (forward(net, centre[None, :])[-1][0] @ C.T).astype(np.float32)  # a decision: fp32, as on the device
     if np.any(y < 0.0):
         return BabResult("falsified", 0, 0, 0, float(y.min()))
+    ya = minimiser_attack(net, centre, eps, C, crown_relus)
+    if ya.size and np.any(ya < 0.0):
+        return BabResult("falsified", 0, 0, 0, float(ya.min()))
 
     def evaluate(domains):
         sp = {k: np.zeros((len(domains), n), np.int8) for k, n in zip(relus, sizes)}
@@ -643,6 +647,33 @@ def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_rel
         return out
 
     return bab_search(evaluate, max_domains, batch)
+
+
+def minimiser_vertices(net, centre, eps, C, crown_relus=None):
+    """Each row's CROWN minimiser vertex of the box centre +- eps (reading; the page names branch-and-bound
+    only [SNNV §3, §4.3]): back-substituting row r of C with the relaxations of ``verify``'s intermediate
+    bounds gives C_r f(x) >= lam_r . x + const_r on the box, and the linear function is smallest at
+    x*_r = centre - eps * sign(lam_r) (sign(0) = 0: the centre's coordinate). Returns (lb, lam_in [R, n0],
+    const [R], x* [R, n0]) with lb [R] the whole box's row bounds (larger of IBP and CROWN)."""
+    centre = np.asarray(centre, F)
+    C = np.asarray(C, F)
+    res = verify(net, centre[None, :], eps, C[None], crown_relus=crown_relus)
+    relax = {k: relax_params(res.pre_bounds[k][0][0], res.pre_bounds[k][1][0])
+             for k, nd in enumerate(net) if nd.op == "relu"}
+    lam_in, const = backward(net, len(net) - 1, C, relax)
+    return res.lb[0], lam_in, const, centre[None, :] - F(eps) * np.sign(lam_in)
+
+
+def minimiser_attack(net, centre, eps, C, crown_relus=None) -> np.ndarray:
+    """Candidate counterexamples of a property: the fp32 values C f(x*_r) [R candidates, R rows] at every
+    row's minimiser vertex (``minimiser_vertices``). A negative entry is a genuine counterexample, an input of
+    the box with a negative row. Only a row that the whole box does not prove positive can be negative at its
+    vertex, so when every row's bound is > 0 nothing is evaluated (an empty result). The values decide, so
+    they are taken in fp32 as on the device."""
+    lb, _, _, xs = minimiser_vertices(net, centre, eps, C, crown_relus)
+    if np.all(lb > 0.0):
+        return np.zeros((0, len(lb)), np.float32)
+    return (forward(net, xs)[-1] @ np.asarray(C, F).T).astype(np.float32)
 
 
 def bab_search(evaluate, max_domains: int, batch: int) -> BabResult:

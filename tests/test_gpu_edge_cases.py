@@ -128,7 +128,7 @@ def test_first_alpha_step_elementwise(config, B):
 def _bab_problems():
     rng = np.random.default_rng(0)
     out = []
-    for t in range(12):
+    for t in range(24):
         net = synth.mlp([4, 10, 10, 3], rng)
         c = rng.random(4).astype(np.float32)
         y = O.forward(net, c[None].astype(np.float64))[-1][0]
@@ -148,8 +148,20 @@ def _oracle_search_log(monkeypatch, net, c, eps, C, max_domains, batch):
     relus = relu_ids(net)
     sizes = [int(np.prod(O.shapes(net)[net[k].src])) for k in relus]
     base = {k: int(sum(sizes[:i])) for i, k in enumerate(relus)}
-    verify_log, results = [], []
+    verify_log, results, attack = [], [], {}
     real_verify, real_search = O.verify, O.bab_search
+    real_vertices, real_attack = O.minimiser_vertices, O.minimiser_attack
+
+    def vertices(*a, **kw):
+        out = real_vertices(*a, **kw)
+        attack["lb"], attack["lam"] = out[0], out[1]
+        attack["amb"] = bool(ambiguous_centres(verify_log[-1], net)[0])
+        return out
+
+    def attack_values(*a, **kw):
+        y = real_attack(*a, **kw)
+        attack["y"] = y
+        return y
 
     def verify(*a, **kw):
         res = real_verify(*a, **kw)
@@ -172,13 +184,33 @@ def _oracle_search_log(monkeypatch, net, c, eps, C, max_domains, batch):
 
     monkeypatch.setattr(O, "verify", verify)
     monkeypatch.setattr(O, "bab_search", search)
+    monkeypatch.setattr(O, "minimiser_vertices", vertices)
+    monkeypatch.setattr(O, "minimiser_attack", attack_values)
     try:
         o = O.bab(net, c, eps, C, max_domains=max_domains, batch=batch, iters=0)
     finally:
         monkeypatch.setattr(O, "verify", real_verify)
         monkeypatch.setattr(O, "bab_search", real_search)
+        monkeypatch.setattr(O, "minimiser_vertices", real_vertices)
+        monkeypatch.setattr(O, "minimiser_attack", real_attack)
     trace = [-1 if r["choice"] is None else base[r["choice"][0]] + r["choice"][1] for r in results]
-    return o, results, trace
+    return o, results, trace, attack
+
+
+def _attack_near_tie(attack):
+    """The vertex attack's decision sits near a tie: a whole-box row bound (which decides whether the attack
+    runs) or a row value at a vertex within the tolerance of 0, an adaptive slope of the whole box near its
+    tie, or a coefficient of lam_in so small against its row that the device's fp32 sign of it may differ."""
+    if "lb" not in attack:
+        return False
+    if attack["amb"] or np.any(np.abs(attack["lb"]) <= NEAR * (1 + np.abs(attack["lb"]))):
+        return True
+    y = attack.get("y")
+    if y is None or y.size == 0:
+        return False
+    lam = attack["lam"]
+    small = np.abs(lam) <= NEAR * np.abs(lam).max(axis=1, keepdims=True)
+    return bool(np.any(np.abs(y) <= NEAR * (1 + np.abs(y).max())) or np.any(small & (lam != 0.0)))
 
 
 def _near_tie(results):
@@ -195,20 +227,28 @@ def _near_tie(results):
 
 def test_bab_decisions_bit_exact(monkeypatch):
     """vf_bab_verify (bounds of vf_verify_batch alone, no ascent) against the oracle's search: on every
-    property whose decisions all sit clear of their ties, the same neuron is chosen for every bounded
-    subdomain in the same order, and the subdomain count, rounds and depth are equal (index work: exact)."""
-    compared = deep = 0
+    property whose decisions all sit clear of their ties, the same status; when falsified, by the same step
+    (the centre or the vertex attack, both before any subdomain is bounded); otherwise the same neuron is
+    chosen for every bounded subdomain in the same order, and the subdomain count, rounds and depth are
+    equal (index work: exact)."""
+    compared = deep = falsified = 0
     for name, net, c, eps, C in _bab_problems():
-        o, results, trace = _oracle_search_log(monkeypatch, net, c, eps, C, max_domains=120, batch=8)
+        o, results, trace, attack = _oracle_search_log(monkeypatch, net, c, eps, C, max_domains=120, batch=8)
         g = vf.Net(net)
         r = g.bab(_dev(c), eps, _dev(C), max_domains=120, batch=8, alpha_iters=0, lr=0.1, trace=True)
         torch.cuda.synchronize()
         g.check()
-        assert r["status"] == o.status or _near_tie(results), f"{name}: device {r['status']} vs oracle {o.status}"
-        if o.status == "falsified" or _near_tie(results):
+        tie = _near_tie(results) or _attack_near_tie(attack)
+        assert r["status"] == o.status or tie, f"{name}: device {r['status']} vs oracle {o.status}"
+        if o.status == "falsified":
+            falsified += not tie
+            assert r["domains"] == o.domains or tie, name
+            continue
+        if tie:
             continue
         assert r["trace"] == trace, f"{name}: branching sequence differs"
         assert (r["domains"], r["rounds"], r["max_depth"]) == (o.domains, o.iterations, o.max_depth), name
         compared += 1
         deep += r["rounds"] >= 2
     assert compared >= 8 and deep >= 2, f"only {compared} properties free of near-ties ({deep} with 2+ rounds)"
+    assert falsified >= 8, f"only {falsified} falsified properties free of near-ties"

@@ -13,6 +13,7 @@ other than the oracle itself:
 from __future__ import annotations
 
 import inspect
+import itertools
 import textwrap
 
 import numpy as np
@@ -249,8 +250,68 @@ def check_bab_sampled(seed=0):
     return True, ""
 
 
+def check_minimiser_vertex(seed=25):
+    """4-8-8-3 nets at three radii, every margin row: the vertex x*_r lies in the box, the row's linear lower
+    bound lam_r . x + const_r takes there its minimum over all 16 vertices of the box (brute force), that
+    minimum is the CROWN bound ``verify`` reports, and the row's exact value at x*_r is not below it."""
+    rng = np.random.default_rng(seed)
+    for t in range(6):
+        net = synth.mlp([4, 8, 8, 3], rng)
+        c = rng.random(4).astype(np.float32)
+        y = O.forward(net, c[None].astype(np.float64))[-1][0]
+        C = synth.margin_spec(np.array([int(np.argmax(y))]), 3)[0]
+        for eps in (0.05, 0.2, 0.5):
+            eps = float(np.float32(eps))
+            _, lam, cst, xs = O.minimiser_vertices(net, c, eps, C)
+            crown = O.verify(net, c[None], eps, C[None]).lb_crown[0]
+            cen = c.astype(np.float64)
+            V = np.array(list(itertools.product(*[(ci - eps, ci + eps) for ci in cen])))
+            brute = (V @ lam.T + cst[None, :]).min(axis=0)
+            at = np.einsum("ri,ri->r", lam, xs) + cst
+            val = np.einsum("ri,ri->r", O.forward(net, xs)[-1], C.astype(np.float64))
+            tol = 1e-12 * (1 + np.abs(brute))
+            if np.abs(xs - cen[None, :]).max() > eps * (1 + 1e-15):
+                return False, f"net {t} eps {eps}: a vertex outside the box"
+            if np.any(np.abs(at - brute) > tol) or np.any(np.abs(at - crown) > tol):
+                return False, f"net {t} eps {eps}: vertex value {at} vs brute force {brute} vs CROWN {crown}"
+            if np.any(val < at - tol):
+                return False, f"net {t} eps {eps}: the linear bound exceeds the row at its vertex"
+    return True, ""
+
+
+def check_attack_exact_2d(seed=26):
+    """Random 2-w-w-3 nets, margin rows of the centre's class, radii 0.1-0.8, the search given one subdomain
+    (so only the centre and the vertices can decide): it says "falsified" only when the exact minimum over the
+    box (enumerated activation regions) is < 0, and does so for at least 3/4 of the properties whose exact
+    minimum is below -0.02 (the vertex is a heuristic; 34 of 38 here)."""
+    rng = np.random.default_rng(seed)
+    hits = false_props = 0
+    for trial in range(40):
+        w = 3 + trial % 2
+        dims = [2, w, w, 3]
+        layers = [{"W": (rng.standard_normal((dims[i + 1], dims[i])) * 0.8).astype(np.float32),
+                   "b": (rng.standard_normal(dims[i + 1]) * 0.3).astype(np.float32)} for i in range(3)]
+        net = net_from_layers(layers)
+        c = rng.random(2).astype(np.float32)
+        y = O.forward(net, c[None].astype(np.float64))[-1][0]
+        C = synth.margin_spec(np.array([int(np.argmax(y))]), 3)[0]
+        for eps in (0.1, 0.2, 0.4, 0.8):
+            eps = float(np.float32(eps))
+            lo, _ = exact_range_2d(layers, C, c, eps)
+            r = O.bab(net, c, eps, C, max_domains=1, batch=2, iters=0)
+            if r.status == "falsified" and lo.min() >= 0.0:
+                return False, f"trial {trial} eps {eps}: falsified a property whose exact minimum is {lo.min()}"
+            if lo.min() < -0.02:
+                false_props += 1
+                hits += r.status == "falsified" and r.domains == 0
+    if hits * 4 < false_props * 3:
+        return False, f"only {hits} of {false_props} false properties falsified without splitting"
+    return True, ""
+
+
 CHECKS = [check_split_subdomain_sound, check_full_split_closed_form, check_beta_duality_lp,
-          check_beta_fd_gradient, check_bab_exact_2d, check_bab_sampled]
+          check_beta_fd_gradient, check_bab_exact_2d, check_bab_sampled, check_minimiser_vertex,
+          check_attack_exact_2d]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=[c.__name__ for c in CHECKS])
@@ -270,6 +331,15 @@ MUTATIONS = [
     ("alpha_crown", "beta[k] = np.maximum(x, 0.0)", "beta[k] = x", check_beta_duality_lp),
     ("verify", "split_clamp(*ibp_b[net[k].src], splits.get(k))", "split_clamp(*ibp_b[net[k].src], None)",
      check_full_split_closed_form),
+    ("minimiser_vertices", "centre[None, :] - F(eps) * np.sign(lam_in)", "centre[None, :] + F(eps) * np.sign(lam_in)",
+     check_minimiser_vertex),
+    ("minimiser_vertices", "centre[None, :] - F(eps) * np.sign(lam_in)", "centre[None, :] - F(eps) * lam_in",
+     check_minimiser_vertex),
+    ("minimiser_vertices", "backward(net, len(net) - 1, C, relax)", "backward(net, len(net) - 1, -C, relax)",
+     check_minimiser_vertex),
+    ("minimiser_attack", "forward(net, xs)[-1] @ np.asarray(C, F).T", "forward(net, xs)[-1] @ np.asarray(-C, F).T",
+     check_attack_exact_2d),
+    ("bab", "if ya.size and np.any(ya < 0.0):", "if ya.size and np.all(ya < 0.0):", check_attack_exact_2d),
 ]
 
 
@@ -298,12 +368,12 @@ def test_every_subdomain_bound_takes_the_requested_ascent_steps(monkeypatch):
         return real(*a, **kw)
 
     monkeypatch.setattr(O, "alpha_crown", spy)
-    rng = np.random.default_rng(0)
+    rng = np.random.default_rng(3)
     net = synth.mlp([4, 10, 10, 3], rng)
     c = rng.random(4).astype(np.float32)
     y = O.forward(net, c[None].astype(np.float64))[-1][0]
     C = synth.margin_spec(np.array([int(np.argmax(y))]), 3)[0]
-    r = O.bab(net, c, float(np.float32(0.2)), C, max_domains=40, batch=8, iters=7, lr=0.1)
+    r = O.bab(net, c, float(np.float32(0.3)), C, max_domains=40, batch=8, iters=7, lr=0.1)
     assert r.iterations >= 2 and len(seen) == r.iterations + 1
     assert set(seen) == {7}
 
