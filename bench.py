@@ -388,6 +388,7 @@ def measure_workload(args, ctx, cfg, eps, steps, warmup, headline, legs=None):
     clocks = stop_clocks(clk)
     launches = net.launch_count() - launches0
     kstats = {k: net.profile_read(kind=k, reset=False) for k in (1, 2, 3, 4, 5)}
+    fwd = net.profile_read(kind=vf.VF_KERNEL_DENSE_FWD_TC, reset=False)
     net.profile_read(reset=True)
     net.profile(False)
     step_ms = [a.elapsed_time(b) for a, b in ev]
@@ -397,6 +398,9 @@ def measure_workload(args, ctx, cfg, eps, steps, warmup, headline, legs=None):
     verified = int(out["verified"].sum().item())
     roof = roofline(kstats, total_ms, torch.cuda.get_device_properties(dev).multi_processor_count,
                     w.name if (args.centres is None or not headline) else None, total_ms / steps)
+    if fwd[0]:  # IBP forward products on the tensor cores (not the dominant kernel; reported beside it)
+        roof["forward_products_tc"] = {"launches": fwd[0], "ms": fwd[1], "share_of_step": fwd[1] / total_ms,
+                                       "achieved_tflops": fwd[2] / (fwd[1] / 1000.0) / 1e12 if fwd[1] else None}
 
     e2e = None
     if headline and not args.no_e2e:
@@ -591,7 +595,8 @@ def bab_leg(args, w, net, centres, dev, stream, world, rank):
     nL = logits.shape[1]
     specs = [torch.from_numpy(synth.margin_spec(np.array([y]), nL)[0]).to(dev) for y in labels]
     kw = dict(batch=args.bab_batch, alpha_iters=args.bab_alpha_iters, lr=0.1, crown_relus=w.crown_relus)
-    net.bab(centres[0], w.eps, specs[0], max_domains=min(args.bab_batch + 1, args.bab_domains), **kw)  # warm-up
+    for k in range(K):  # warm-up on every timed problem (a property falsified at once warms nothing else)
+        net.bab(centres[k], w.eps, specs[k], max_domains=min(args.bab_batch + 1, args.bab_domains), **kw)
     torch.cuda.synchronize()
     ms, domains, statuses = 0.0, 0, []
     for k in range(K):

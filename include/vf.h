@@ -282,7 +282,9 @@ enum {
     VF_KERNEL_DENSE_FFMA = 2,
     VF_KERNEL_CONV = 3,
     VF_KERNEL_CONV_WIN = 4,
-    VF_KERNEL_CONV_TC = 5 /* tensor-core implicit GEMM, whole maps and windows; flops as for windows */
+    VF_KERNEL_CONV_TC = 5, /* tensor-core implicit GEMM, whole maps and windows; flops as for windows */
+    VF_KERNEL_DENSE_FWD_TC = 6 /* forward products on the tensor cores: IBP W c + b and |W| r, the alpha
+                                  gradient's G W^T + b; 2*M*K*N flops */
 };
 int vf_profile_enable(vf_net* net, int enable);
 int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms, double* flops, int reset);

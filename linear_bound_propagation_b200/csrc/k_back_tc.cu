@@ -93,6 +93,7 @@ struct TcParams {
     const float* centres;
     float eps;
     float* part;
+    const float* col_bias;  // OUT_STORE only: added to every stored output column (nullptr: none)
     int count_const;
     int* err;
     int test_stall;  // test hook: CTA 0 never issues its first raw-tile copy, so a bounded wait expires
@@ -371,13 +372,14 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                         __syncwarp();
                         const int n = n0 + cu + lane;
                         const bool col_ok = (cu + lane < p.BN) && (n < p.N);
+                        const float cb = (col_ok && p.col_bias != nullptr) ? __ldg(&p.col_bias[n]) : 0.f;
 #pragma unroll 4
                         for (int j = 0; j < 32; ++j) {
                             const long long mr = row0 + j;
                             if (col_ok && mr < p.M) {
                                 float* o = p.out + mr * p.ld_out + n;
                                 const float val = stg[j * 33 + lane];
-                                *o = (p.out_mode == OUT_ACCUM) ? (*o + val) : val;
+                                *o = (p.out_mode == OUT_ACCUM) ? (*o + val) : val + cb;
                             }
                         }
                         __syncwarp();
@@ -459,10 +461,12 @@ bool dense_back_tc_supported(const RowRef& A, Relax rx, long long M, int K, int 
     return false;
 }
 
-cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, const float* Wt_lo, long long B,
-                                 long long M, int K, int N, PassGeom pg, int out_mode, float* out, long long ld_out,
-                                 float* cst, const float* centres, float eps, float* part, int* err, int test_stall,
-                                 cudaStream_t s) {
+namespace {
+
+cudaError_t launch_tc(const RowRef& A, Relax rx, const float* Wt_hi, const float* Wt_lo, long long B, long long M,
+                     int K, int N, PassGeom pg, int out_mode, float* out, long long ld_out, float* cst,
+                     const float* centres, float eps, float* part, const float* col_bias, int* err, int test_stall,
+                     cudaStream_t s) {
     if (M <= 0) return cudaSuccess;
     TcParams p{};
     p.M = M;
@@ -512,6 +516,7 @@ cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, 
     p.centres = centres;
     p.eps = eps;
     p.part = part;
+    p.col_bias = col_bias;
     p.count_const = rx.count_const;
     p.err = err;
     p.test_stall = test_stall;
@@ -523,6 +528,30 @@ cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, 
     const long long grid = std::min<long long>(p.ntiles, num_sms);  // persistent: one CTA per SM
     dense_back_tc<<<(unsigned)grid, NUM_THREADS, smem, s>>>(ta, tp, tbh, tbl, p);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, const float* Wt_lo, long long B,
+                                 long long M, int K, int N, PassGeom pg, int out_mode, float* out, long long ld_out,
+                                 float* cst, const float* centres, float eps, float* part, int* err, int test_stall,
+                                 cudaStream_t s) {
+    return launch_tc(A, rx, Wt_hi, Wt_lo, B, M, K, N, pg, out_mode, out, ld_out, cst, centres, eps, part, nullptr,
+                     err, test_stall, s);
+}
+
+bool dense_fwd_tc_supported(const float* A, long long M, int K, int N) {
+    if (K % 4 != 0 || K < 32 || N < 16) return false;  // TMA rows of A and W: 16-byte strides
+    if ((reinterpret_cast<uintptr_t>(A) & 15) != 0) return false;
+    return M >= BM && M < (1LL << 31);
+}
+
+cudaError_t launch_dense_fwd_tc(const float* A, long long M, int K, int N, const float* W_hi, const float* W_lo,
+                                const float* bias, const float4* ident, float* out, int* err, cudaStream_t s) {
+    // the same kernel with every row read through one identity relaxation row (slopes 1, intercept 0, no row
+    // constant) and the bias added per output column in the store epilogue
+    return launch_tc(RowRef{A, 0, K, kHugeRows, 0}, Relax{ident, 0}, W_hi, W_lo, 1, M, K, N, PassGeom{0, kHugeRows},
+                     OUT_STORE, out, N, nullptr, nullptr, 0.f, nullptr, bias, err, 0, s);
 }
 
 }  // namespace vf

@@ -188,6 +188,13 @@ cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, c
     return cudaGetLastError();
 }
 
+cudaError_t launch_ibp_radius_rowsum(const float* rowsum_abs, float eps, int B, int N, float* zr, cudaStream_t s) {
+    dim3 grid((B + 63) / 64, (N + 63) / 64, 1);  // only the radius of a layer fed by the input box
+    ibp_dense_k<<<grid, 256, 0, s>>>(nullptr, nullptr, nullptr, nullptr, nullptr, rowsum_abs, eps, B, 0, N, nullptr,
+                                     zr, 1);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_abs_rows_times_wt(const float* A, const float* Wabs, int M, int K, int N, float* out, cudaStream_t s) {
     dim3 grid((M + 63) / 64, (N + 63) / 64, 1);  // only the radius product: out = A |W|^T
     ibp_dense_k<<<grid, 256, 0, s>>>(A, A, Wabs, Wabs, nullptr, nullptr, 0.f, M, K, N, out, out, 1);

@@ -73,6 +73,10 @@ struct Node {
     float* pmW = nullptr;  // dense only: [W; -W], the rows of the identity-trick first step
     float* WtHi = nullptr; // dense only: W^T [n_in, n_out] truncated to tf32 (3xTF32 head)
     float* WtLo = nullptr; // dense only: W^T - WtHi (3xTF32 remainder)
+    float* WfHi = nullptr; // dense only: W [n_out, n_in] split the same way (forward products W c, G W^T)
+    float* WfLo = nullptr;
+    float* WaHi = nullptr; // dense only: |W| split: |WfHi| and |WfLo| (|w| truncates to |head|, remainder keeps sign)
+    float* WaLo = nullptr;
     float* rowsum_abs = nullptr;  // dense only: sum_k |W[n, k]| (IBP radius of a layer fed by the input box)
     float* Wwin = nullptr;        // conv only: weights in the tap-major layout of the windowed kernel
     float* Wtc = nullptr;         // conv only: 3xTF32 operand images of the tensor-core kernel (or null)
@@ -104,6 +108,10 @@ struct vf_net {
     int conv_tc = 1;        // convolution steps on the tensor cores where the shapes allow (VF_CONV_TC=0: off)
     int conv_tcn = 0;       // ... with the taps-in-N kernel where its shapes allow (VF_CONV_TC=tapn; measured slower)
     int call_sound = 0;     // set for the duration of a vf_opts.sound call: contractions take FFMA kernels
+    // forward products (IBP, alpha up pass) on the tensor cores: 0 never (VF_FWD_TC=0), 1 (default) when the product
+    // has at least kFwdTcMinTiles output tiles, 2 whenever the shapes allow (VF_FWD_TC=all)
+    int fwd_tc = 1;
+    float4* ident_row = nullptr;  // identity relaxation row {1, 1, 0, 0} x (largest node size), for forward products
     bool prof = false;
     std::vector<cudaEvent_t> ev_free;
     struct Timed {
@@ -112,9 +120,9 @@ struct vf_net {
         double flops;
     };
     std::vector<Timed> ev_used;
-    double prof_flops[6] = {0, 0, 0, 0, 0, 0};
-    long long prof_launches[6] = {0, 0, 0, 0, 0, 0};
-    double prof_ms[6] = {0, 0, 0, 0, 0, 0};
+    double prof_flops[7] = {0, 0, 0, 0, 0, 0, 0};
+    long long prof_launches[7] = {0, 0, 0, 0, 0, 0, 0};
+    double prof_ms[7] = {0, 0, 0, 0, 0, 0, 0};
 };
 
 namespace {
@@ -699,6 +707,48 @@ int pool_size(vf_net* net, int start, Entry init, const std::vector<const float4
     return VF_OK;
 }
 
+// Fewest 128 x (<= 256) output tiles for which a forward product takes the tensor-core kernel by default: it runs
+// one persistent CTA per tile, so a product of a few tiles (the IBP of 1024 centres through 256 neurons: 8 tiles;
+// the ascent of 64 branch-and-bound subdomains: 5) leaves most SMs idle and is slower than the FFMA kernel's 64 x 64
+// tiles (measured on the 784-256x3-10 network). Products measured faster on the tensor cores had 72 tiles (the
+// alpha ascent at 1024 centres) and 128 (the IBP of the 3072-1024x8-100 network at 4096 centres); the threshold
+// sits between the two groups.
+constexpr long long kFwdTcMinTiles = 32;
+
+bool fwd_tc_ok(const vf_net* net, const Node& nd, const float* A, long long M, int K) {
+    const int N = (int)nd.n;
+    if (net->dense_kernel != 0 || net->fwd_tc == 0 || net->call_sound || nd.WfHi == nullptr) return false;
+    if (!dense_fwd_tc_supported(A, M, K, N)) return false;
+    return net->fwd_tc == 2 || ((M + 127) / 128) * dense_back_tc_tiles_n(N) >= kFwdTcMinTiles;
+}
+
+// out [M, N] = A [M, K] W^T + bias (absw: A |W|^T, no bias) for dense node nd: the tensor-core kernel where
+// fwd_tc_ok (profiled as VF_KERNEL_DENSE_FWD_TC), else the FFMA kernel.
+int fwd_product(vf_net* net, const Node& nd, const float* A, long long M, int K, bool absw, const float* bias,
+                float* out, cudaStream_t s) {
+    const int N = (int)nd.n;
+    if (fwd_tc_ok(net, nd, A, M, K)) {
+        cudaEvent_t e0 = nullptr;
+        if (net->prof) {
+            e0 = take_event(net);
+            cudaEventRecord(e0, s);
+        }
+        LAUNCH(net, launch_dense_fwd_tc(A, M, K, N, absw ? nd.WaHi : nd.WfHi, absw ? nd.WaLo : nd.WfLo,
+                                        absw ? nullptr : bias, net->ident_row, out, net->d_err, s));
+        if (net->prof) {
+            cudaEvent_t e1 = take_event(net);
+            cudaEventRecord(e1, s);
+            net->ev_used.push_back({e0, e1, VF_KERNEL_DENSE_FWD_TC, 2.0 * (double)M * K * N});
+        }
+        return VF_OK;
+    }
+    if (absw)
+        LAUNCH(net, launch_abs_rows_times_wt(A, nd.Wabs, (int)M, K, N, out, s));
+    else
+        LAUNCH(net, launch_rows_times_wt(A, nd.W, bias, (int)M, K, N, out, s));
+    return VF_OK;
+}
+
 struct IbpState {
     std::vector<float*> c, r;
 };
@@ -729,6 +779,16 @@ int run_ibp(vf_net* net, const float* centres, int B, float eps, Arena& ar, IbpS
         if (sound && (!T || !S)) return fail(VF_ERR_WORKSPACE, "workspace too small for sound IBP");
         switch (nd.op) {
             case VF_DENSE:
+                if (!sound && fwd_tc_ok(net, nd, st.c[sv], B, (int)net->nodes[sv].n) &&
+                    (sv == 0 || fwd_tc_ok(net, nd, st.r[sv], B, (int)net->nodes[sv].n))) {
+                    // centre W c + b and radius |W| r on the tensor cores (the input box: eps * sum_k |W[n, k]|)
+                    TRY(fwd_product(net, nd, st.c[sv], B, (int)net->nodes[sv].n, false, nd.b, st.c[v], s));
+                    if (sv == 0)
+                        LAUNCH(net, launch_ibp_radius_rowsum(nd.rowsum_abs, eps, B, (int)nd.n, st.r[v], s));
+                    else
+                        TRY(fwd_product(net, nd, st.r[sv], B, (int)net->nodes[sv].n, true, nullptr, st.r[v], s));
+                    break;
+                }
                 LAUNCH(net, launch_ibp_dense(st.c[sv], st.r[sv], nd.W, nd.Wabs, nd.b, sv == 0 ? nd.rowsum_abs : nullptr,
                                              eps, B, (int)net->nodes[sv].n, (int)nd.n, st.c[v], st.r[v], s));
                 if (sound) {  // every dot product of K terms errs by at most gamma_K (|W| (|c| + r) + |b|)
@@ -1246,7 +1306,7 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
                     LAUNCH(net, launch_ibp_conv(G, nullptr, dn.W, dn.Wabs, dn.b, (int)Mc, conv_geom(net, dn), Gn,
                                                 nullptr, s));
                 else
-                    LAUNCH(net, launch_rows_times_wt(G, dn.W, dn.b, (int)Mc, (int)net->nodes[d - 1].n, nu, Gn, s));
+                    TRY(fwd_product(net, dn, G, Mc, (int)net->nodes[d - 1].n, false, dn.b, Gn, s));
                 float* gout = grad_mode ? grad_out + aoff[u] + m0 * nu : nullptr;
                 LAUNCH(net, launch_relax_grad_adam(Gn, H[u], Mc, nu, bd.relax[u], pg, al[u], gout, M1[u], M2[u],
                                                    grad_mode ? 0 : it + 1, lr, s, bt[u]));
@@ -1420,8 +1480,7 @@ int spec_alpha_graph(vf_net* net, const float* centres, int B, float eps, const 
                 const int nv = (int)nd.n;
                 switch (nd.op) {
                     case VF_DENSE:
-                        LAUNCH(net, launch_rows_times_wt(G[nd.src], nd.W, nd.b, (int)Mc, (int)net->nodes[nd.src].n, nv,
-                                                         G[v], s));
+                        TRY(fwd_product(net, nd, G[nd.src], Mc, (int)net->nodes[nd.src].n, false, nd.b, G[v], s));
                         break;
                     case VF_CONV2D:
                         LAUNCH(net, launch_ibp_conv(G[nd.src], nullptr, nd.W, nd.Wabs, nd.b, (int)Mc, conv_geom(net, nd),
@@ -1500,12 +1559,17 @@ void vf_net_destroy(vf_net* net) {
         cudaFree(nd.pmW);
         cudaFree(nd.WtHi);
         cudaFree(nd.WtLo);
+        cudaFree(nd.WfHi);
+        cudaFree(nd.WfLo);
+        cudaFree(nd.WaHi);
+        cudaFree(nd.WaLo);
         cudaFree(nd.rowsum_abs);
         cudaFree(nd.Wwin);
         cudaFree(nd.Wtc);
         cudaFree(nd.Wtn);
     }
     cudaFree(net->d_err);
+    cudaFree(net->ident_row);
     for (auto e : net->ev_free) cudaEventDestroy(e);
     for (auto& p : net->ev_used) {
         cudaEventDestroy(p.e0);
@@ -1542,6 +1606,7 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
         net->conv_tc = strcmp(f, "0") != 0;
         net->conv_tcn = strcmp(f, "tapn") == 0;
     }
+    if (const char* f = getenv("VF_FWD_TC")) net->fwd_tc = strcmp(f, "0") == 0 ? 0 : (strcmp(f, "all") == 0 ? 2 : 1);
     CU(cudaMalloc(&net->d_err, sizeof(int)));
     CU(cudaMemset(net->d_err, 0, sizeof(int)));
     net->nodes.resize(n_nodes);
@@ -1611,6 +1676,28 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
                     CU(cudaMalloc(&nd.WtLo, sizeof(float) * cnt));
                     CU(cudaMemcpy(nd.WtHi, hi.data(), sizeof(float) * cnt, cudaMemcpyHostToDevice));
                     CU(cudaMemcpy(nd.WtLo, lo.data(), sizeof(float) * cnt, cudaMemcpyHostToDevice));
+                }
+                if (s.n % 4 == 0) {  // TMA rows of W (forward products) need a 16-byte stride
+                    std::vector<float> hi((size_t)cnt), lo((size_t)cnt);
+                    for (long long i = 0; i < cnt; ++i) {
+                        uint32_t bits;
+                        std::memcpy(&bits, &pm[i], 4);
+                        bits &= 0xFFFFE000u;
+                        std::memcpy(&hi[i], &bits, 4);
+                        lo[i] = pm[i] - hi[i];
+                    }
+                    CU(cudaMalloc(&nd.WfHi, sizeof(float) * cnt));
+                    CU(cudaMalloc(&nd.WfLo, sizeof(float) * cnt));
+                    CU(cudaMemcpy(nd.WfHi, hi.data(), sizeof(float) * cnt, cudaMemcpyHostToDevice));
+                    CU(cudaMemcpy(nd.WfLo, lo.data(), sizeof(float) * cnt, cudaMemcpyHostToDevice));
+                    for (long long i = 0; i < cnt; ++i) {
+                        hi[i] = std::fabs(hi[i]);
+                        lo[i] = std::fabs(lo[i]);
+                    }
+                    CU(cudaMalloc(&nd.WaHi, sizeof(float) * cnt));
+                    CU(cudaMalloc(&nd.WaLo, sizeof(float) * cnt));
+                    CU(cudaMemcpy(nd.WaHi, hi.data(), sizeof(float) * cnt, cudaMemcpyHostToDevice));
+                    CU(cudaMemcpy(nd.WaLo, lo.data(), sizeof(float) * cnt, cudaMemcpyHostToDevice));
                 }
                 break;
             }
@@ -1693,7 +1780,16 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
     if (net->nodes[last].op != VF_DENSE && net->nodes[last].op != VF_CONV2D)
         return fail(VF_ERR_UNSUPPORTED, "the last node must be dense or conv");
     net->total = 0;
-    for (auto& nd : net->nodes) net->total += nd.n;
+    long long nmax = 0;
+    for (auto& nd : net->nodes) {
+        net->total += nd.n;
+        nmax = std::max(nmax, nd.n);
+    }
+    {
+        std::vector<float4> id((size_t)nmax, make_float4(1.f, 1.f, 0.f, 0.f));
+        CU(cudaMalloc(&net->ident_row, sizeof(float4) * nmax));
+        CU(cudaMemcpy(net->ident_row, id.data(), sizeof(float4) * nmax, cudaMemcpyHostToDevice));
+    }
     net->ws_bytes = ws_bytes ? ws_bytes : (size_t(4) << 30);
     CU(cudaMalloc(&net->ws, net->ws_bytes));
     return VF_OK;
@@ -1924,7 +2020,7 @@ int vf_profile_enable(vf_net* net, int enable) {
 
 int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms, double* flops, int reset) {
     TRY(check_net(net));
-    if (kind < 0 || kind > 5) return fail(VF_ERR_ARG, "bad kernel kind");
+    if (kind < 0 || kind > 6) return fail(VF_ERR_ARG, "bad kernel kind");
     for (auto& t : net->ev_used) {
         CU(cudaEventSynchronize(t.e1));
         float ms = 0.f;
@@ -1942,7 +2038,7 @@ int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms
     if (total_ms) *total_ms = net->prof_ms[kind];
     if (flops) *flops = net->prof_flops[kind];
     if (reset)
-        for (int k = 0; k < 6; ++k) {
+        for (int k = 0; k < 7; ++k) {
             net->prof_launches[k] = 0;
             net->prof_ms[k] = 0.0;
             net->prof_flops[k] = 0.0;

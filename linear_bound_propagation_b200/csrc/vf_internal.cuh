@@ -177,6 +177,8 @@ cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, c
                              const float* rowsum_abs, float eps, int B, int K, int N, float* zc, float* zr,
                              cudaStream_t s);
 // hr and zr may both be NULL: then only the centre map W * hc + b is computed (the alpha-CROWN gradient).
+// zr[m, n] = eps * rowsum_abs[n] for m < B: the IBP radius of a dense layer fed by the input box.
+cudaError_t launch_ibp_radius_rowsum(const float* rowsum_abs, float eps, int B, int N, float* zr, cudaStream_t s);
 cudaError_t launch_ibp_conv(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
                             int B, const ConvGeom& g, float* zc, float* zr, cudaStream_t s);
 cudaError_t launch_ibp_relu(const float* c, const float* r, long long n, float* oc, float* orad, cudaStream_t s,

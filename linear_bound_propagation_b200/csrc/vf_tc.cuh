@@ -18,4 +18,11 @@ cudaError_t launch_dense_back_tc(const RowRef& A, Relax rx, const float* Wt_hi, 
                                  float* cst, const float* centres, float eps, float* part, int* err, int test_stall,
                                  cudaStream_t s);
 
+// Forward product out[M, N] = A[M, K] W^T (+ bias[n]) on the same kernel: W_hi / W_lo hold W in its own
+// [N, K] layout (K contiguous) split into tf32 head and fp32 remainder; ident is an identity relaxation row
+// ({1, 1, 0, 0}) of at least K entries. A: M rows K floats apart, 16-byte aligned; needs M >= 128.
+bool dense_fwd_tc_supported(const float* A, long long M, int K, int N);
+cudaError_t launch_dense_fwd_tc(const float* A, long long M, int K, int N, const float* W_hi, const float* W_lo,
+                                const float* bias, const float4* ident, float* out, int* err, cudaStream_t s);
+
 }  // namespace vf

@@ -27,17 +27,25 @@ def _oracle_relax(net, res, b):
             for k, nd in enumerate(net) if nd.op == "relu"}
 
 
-@pytest.mark.parametrize("config,B", [(1, 16), (2, 6), (3, 2)])
-def test_alpha_grad_matches_oracle(config, B):
+@pytest.mark.parametrize("config,B", [(1, 16), (2, 6), (2, 16), (3, 2)])
+def test_alpha_grad_matches_oracle(monkeypatch, config, B):
+    """Bound and slope gradient element-wise. Workload 2 at 16 centres has 144 rows per pass, so with the forward
+    products on the tensor cores whenever the shapes allow (VF_FWD_TC=all) the gradient's G W^T + b runs there
+    (at 6 centres, 54 rows, on the FFMA kernel)."""
+    monkeypatch.setenv("VF_FWD_TC", "all")
     w = synth.workload(config, B=B)
     net, R = w.net, w.C.shape[1]
     rng = np.random.default_rng(5)
     g = vf.Net(net)
     relus = g.relu_ids
     alpha = rng.random(g.alpha_size(B, R)).astype(np.float32)  # seeded slopes, from the test
+    g.profile(True)
+    g.profile_read(reset=True)
     lb, grad = g.alpha_grad(_dev(w.centres), w.eps, _dev(w.C), _dev(alpha))
     torch.cuda.synchronize()
     g.check()
+    fwd_tc = g.profile_read(kind=vf.VF_KERNEL_DENSE_FWD_TC)[0]
+    assert (fwd_tc > 0) == (config == 2 and B * R >= 128), fwd_tc
     lb, grad = lb.cpu().numpy(), grad.cpu().numpy()
     res = O.verify(net, w.centres, w.eps, w.C)
     amb = ambiguous_centres(res, net)
