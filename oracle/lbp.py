@@ -326,7 +326,8 @@ def _first_affine_on_input(net, p: int) -> bool:
 
 def verify(net, centres, eps, C, crown_relus: Optional[Sequence[int]] = None,
            alphas: Optional[Dict[int, np.ndarray]] = None, both_sides: bool = False,
-           row_block: int = 4096, splits: Optional[Dict[int, np.ndarray]] = None) -> OracleResult:
+           row_block: int = 4096, splits: Optional[Dict[int, np.ndarray]] = None,
+           alpha_inter_iters: int = 0, alpha_inter_lr: float = 0.1) -> OracleResult:
     """IBP, then CROWN intermediate bounds, then the specification pass and decision.
 
     Readings taken where the page is silent (it names the methods only, [SNNV §1, §2.1]):
@@ -347,7 +348,15 @@ def verify(net, centres, eps, C, crown_relus: Optional[Sequence[int]] = None,
       * alpha (relu node -> [B, n]) is shared by all rows and passes; missing = adaptive;
       * splits (relu node -> [B, n] in {-1, 0, +1}): each centre's row is one subdomain; the IBP
         pass and the IBP bounds of split neurons are clamped (``split_clamp``), which makes those
-        neurons IBP-stable, so they take no CROWN refinement and their relaxation is exact.
+        neurons IBP-stable, so they take no CROWN refinement and their relaxation is exact;
+      * alpha_inter_iters > 0 (alpha-CROWN for the intermediate bounds; the page names the per-neuron alpha
+        tensors [SNNV §3, §4.3], the reading is ours): right after the CROWN pass of a ReLU k whose source p
+        is a dense node, the neurons of p still unstable (l < 0 < u) take rows [e_j; -e_j] over p and
+        ``ascend`` (alpha_inter_iters Adam steps of size alpha_inter_lr, per-row slopes of every earlier
+        ReLU, split multipliers where splits are given) on the network up to p with the relaxations of the
+        earlier ReLUs; l_j = max(l_j, best of e_j), u_j = min(u_j, -best of -e_j). The ascent starts at the
+        relaxation's slopes, so its best is never below the pass it refines. Layers after k relax with the
+        refined bounds.
     """
     centres = np.asarray(centres, F)
     B = centres.shape[0]
@@ -378,6 +387,17 @@ def verify(net, centres, eps, C, crown_relus: Optional[Sequence[int]] = None,
                 unst = (l0 < 0.0) & (u0 > 0.0)
                 pre[k][0][b] = np.where(unst, np.maximum(l0, l_cr), l0)
                 pre[k][1][b] = np.where(unst, np.minimum(u0, u_cr), u0)
+                if alpha_inter_iters > 0 and net[p].op == "dense":
+                    l1, u1 = pre[k][0][b], pre[k][1][b]
+                    idx = np.nonzero((l1 < 0.0) & (u1 > 0.0))[0]
+                    if idx.size:
+                        sub = net[:p + 1]
+                        sg = {j: np.asarray(splits[j][b]) for j in relus if j < p and j in splits} or None
+                        best, _ = ascend(sub, centres[b], eps, np.concatenate([eye[idx], -eye[idx]]), relax,
+                                         alpha_inter_iters, alpha_inter_lr, sg)
+                        m = idx.size
+                        l1[idx] = np.maximum(l1[idx], best[:m])
+                        u1[idx] = np.minimum(u1[idx], -best[m:])
             a = alphas.get(k)
             relax[k] = relax_params(pre[k][0][b], pre[k][1][b], None if a is None else a[b])
         Cb = C[b if C.shape[0] > 1 else 0]
@@ -506,22 +526,15 @@ def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows, split_signs=None
     return lb, grads
 
 
-def alpha_crown(net, centres, eps, C, iters=10, lr=0.1, crown_relus=None, betas=(0.9, 0.999), splits=None):
-    """Projected gradient ascent (Adam) on per-row lower slopes of the specification pass, starting
-    from the adaptive slopes, keeping each row's best bound [SNNV §1 alpha-CROWN; §3 alpha tensors].
-    Intermediate bounds are those of `verify` (adaptive slopes). Returns (best lb [B, R], lb at the
-    adaptive start [B, R]).
-
-    With split constraints (relu node -> [B, n] signs) the multipliers beta of the split neurons
-    (beta-CROWN, see ``spec_bound_alpha``) are optimised together with the slopes: one per (row, split
-    neuron), starting at 0, the same Adam step, projected to beta >= 0."""
-    res = verify(net, centres, eps, C, crown_relus=crown_relus, splits=splits)
-    B, R = res.lb.shape
-    C = np.asarray(C, F)
-    relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
-    best = np.empty((B, R), F)
-    start = np.empty((B, R), F)
+def ascend(net, centre, eps, rows, relax, iters, lr, split_signs=None, betas=(0.9, 0.999)):
+    """Projected gradient ascent (Adam, step lr, moments ``betas``) on per-row lower slopes of the bound of
+    ``rows`` over ``net``'s last node for one centre [SNNV §1 alpha-CROWN; §3 alpha tensors], starting from the
+    slopes of ``relax``; with split signs (relu node -> [n]) the split multipliers beta are optimised with them
+    (from 0, projected to beta >= 0; see ``spec_bound_alpha``). Returns (best lb over the iterates [R], lb at
+    the start [R])."""
     b1, b2 = betas
+    R = np.asarray(rows).shape[0]
+    relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
 
     def adam(x, m1, m2, g, it):
         m1 = b1 * m1 + (1 - b1) * g
@@ -530,36 +543,56 @@ def alpha_crown(net, centres, eps, C, iters=10, lr=0.1, crown_relus=None, betas=
         vh = m2 / (1 - b2 ** (it + 1))
         return x + lr * mh / (np.sqrt(vh) + 1e-8), m1, m2
 
+    alpha = {k: np.repeat(relax[k][0][None, :], R, axis=0) for k in relus}
+    m1 = {k: np.zeros_like(a) for k, a in alpha.items()}
+    m2 = {k: np.zeros_like(a) for k, a in alpha.items()}
+    sg = split_signs or None
+    beta = None if sg is None else {k: np.zeros((R, len(sg[k])), F) for k in sg}
+    bm1 = None if sg is None else {k: np.zeros_like(x) for k, x in beta.items()}
+    bm2 = None if sg is None else {k: np.zeros_like(x) for k, x in beta.items()}
+    start = best = None
+    for it in range(iters + 1):
+        out = spec_bound_alpha(net, centre, eps, rows, relax, alpha, sg, beta)
+        lb, g = out[0], out[1]
+        if it == 0:
+            start, best = lb, lb.copy()
+        else:
+            best = np.maximum(best, lb)
+        if it == iters:
+            break
+        for k in relus:
+            a, m1[k], m2[k] = adam(alpha[k], m1[k], m2[k], g[k], it)
+            alpha[k] = np.clip(a, 0.0, 1.0)
+        if beta is not None:
+            for k in beta:
+                gb = np.where(sg[k][None, :] != 0, out[2][k], 0.0)
+                x, bm1[k], bm2[k] = adam(beta[k], bm1[k], bm2[k], gb, it)
+                beta[k] = np.maximum(x, 0.0)
+    return best, start
+
+
+def alpha_crown(net, centres, eps, C, iters=10, lr=0.1, crown_relus=None, betas=(0.9, 0.999), splits=None,
+                alpha_inter_iters=0, alpha_inter_lr=0.1):
+    """Projected gradient ascent (Adam) on per-row lower slopes of the specification pass, starting
+    from the adaptive slopes, keeping each row's best bound [SNNV §1 alpha-CROWN; §3 alpha tensors]
+    (``ascend`` per centre). Intermediate bounds are those of `verify` (with ``alpha_inter_iters`` > 0, those of
+    its intermediate ascent). Returns (best lb [B, R], lb at the adaptive start [B, R]).
+
+    With split constraints (relu node -> [B, n] signs) the multipliers beta of the split neurons
+    (beta-CROWN, see ``spec_bound_alpha``) are optimised together with the slopes: one per (row, split
+    neuron), starting at 0, the same Adam step, projected to beta >= 0."""
+    res = verify(net, centres, eps, C, crown_relus=crown_relus, splits=splits, alpha_inter_iters=alpha_inter_iters,
+                 alpha_inter_lr=alpha_inter_lr)
+    B, R = res.lb.shape
+    C = np.asarray(C, F)
+    relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
+    best = np.empty((B, R), F)
+    start = np.empty((B, R), F)
     for b in range(B):
         relax = {k: relax_params(res.pre_bounds[k][0][b], res.pre_bounds[k][1][b]) for k in relus}
         rows = C[b if C.shape[0] > 1 else 0]
-        alpha = {k: np.repeat(relax[k][0][None, :], R, axis=0) for k in relus}
-        m1 = {k: np.zeros_like(a) for k, a in alpha.items()}
-        m2 = {k: np.zeros_like(a) for k, a in alpha.items()}
         sg = None if not splits else {k: np.asarray(splits[k][b]) for k in relus if k in splits}
-        beta = None if sg is None else {k: np.zeros((R, len(sg[k])), F) for k in sg}
-        bm1 = None if sg is None else {k: np.zeros_like(x) for k, x in beta.items()}
-        bm2 = None if sg is None else {k: np.zeros_like(x) for k, x in beta.items()}
-        best_b = None
-        for it in range(iters + 1):
-            out = spec_bound_alpha(net, centres[b], eps, rows, relax, alpha, sg, beta)
-            lb, g = out[0], out[1]
-            if it == 0:
-                start[b] = lb
-                best_b = lb.copy()
-            else:
-                best_b = np.maximum(best_b, lb)
-            if it == iters:
-                break
-            for k in relus:
-                a, m1[k], m2[k] = adam(alpha[k], m1[k], m2[k], g[k], it)
-                alpha[k] = np.clip(a, 0.0, 1.0)
-            if beta is not None:
-                for k in beta:
-                    gb = np.where(sg[k][None, :] != 0, out[2][k], 0.0)
-                    x, bm1[k], bm2[k] = adam(beta[k], bm1[k], bm2[k], gb, it)
-                    beta[k] = np.maximum(x, 0.0)
-        best[b] = best_b
+        best[b], start[b] = ascend(net, centres[b], eps, rows, relax, iters, lr, sg, betas)
     return best, start
 
 

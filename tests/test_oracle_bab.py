@@ -328,7 +328,7 @@ MUTATIONS = [
      check_full_split_closed_form),
     ("split_clamp", "np.where(s < 0, np.minimum(u, 0.0), u)", "np.where(s < 0, np.maximum(u, 0.0), u)",
      check_full_split_closed_form),
-    ("alpha_crown", "beta[k] = np.maximum(x, 0.0)", "beta[k] = x", check_beta_duality_lp),
+    ("ascend", "beta[k] = np.maximum(x, 0.0)", "beta[k] = x", check_beta_duality_lp),
     ("verify", "split_clamp(*ibp_b[net[k].src], splits.get(k))", "split_clamp(*ibp_b[net[k].src], None)",
      check_full_split_closed_form),
     ("minimiser_vertices", "centre[None, :] - F(eps) * np.sign(lam_in)", "centre[None, :] + F(eps) * np.sign(lam_in)",

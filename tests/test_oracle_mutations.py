@@ -48,11 +48,11 @@ MUTATIONS = [
     ("verify", "crown_set = set(relus if crown_relus is None else crown_relus)",
      "crown_set = set(relus if crown_relus is None else [r - 2 for r in crown_relus])"),
     ("verify", "pre[k][0][b] = np.where(unst, np.maximum(l0, l_cr), l0)", "pass"),
-    ("alpha_crown", "mh = m1 / (1 - b1 ** (it + 1))", "mh = m1 / (1 - b1 ** it)"),
-    ("alpha_crown", "mh = m1 / (1 - b1 ** (it + 1))", "mh = m1 / (1 - b1 ** (it + 2))"),
-    ("alpha_crown", "np.sqrt(vh) + 1e-8", "np.sqrt(vh + 1e-8)"),
-    ("alpha_crown", "lr * mh / (np.sqrt(vh) + 1e-8)", "lr * mh / (vh + 1e-8)"),
-    ("alpha_crown", "m2 = b2 * m2 + (1 - b2) * g * g", "m2 = b2 * m2 + (1 - b2) * np.abs(g)"),
+    ("ascend", "mh = m1 / (1 - b1 ** (it + 1))", "mh = m1 / (1 - b1 ** it)"),
+    ("ascend", "mh = m1 / (1 - b1 ** (it + 1))", "mh = m1 / (1 - b1 ** (it + 2))"),
+    ("ascend", "np.sqrt(vh) + 1e-8", "np.sqrt(vh + 1e-8)"),
+    ("ascend", "lr * mh / (np.sqrt(vh) + 1e-8)", "lr * mh / (vh + 1e-8)"),
+    ("ascend", "m2 = b2 * m2 + (1 - b2) * g * g", "m2 = b2 * m2 + (1 - b2) * np.abs(g)"),
 ]
 
 
