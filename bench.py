@@ -546,10 +546,41 @@ def alpha_leg(args, w, net, centres, C, stream, flush, dev, world, steps):
         a_ms += e0.elapsed_time(e1)
     a_ms = max_over_ranks(a_ms, dev)
     gain = (res["lb"] - res["lb_start"])
-    return {"iters": args.alpha_iters, "lr": 0.1, "value": weak_throughput(world, B * R, steps, a_ms),
-            "unit": UNIT, "ms_per_step": a_ms / steps, "mean_lb_gain": float(gain.mean().item()),
-            "rows_improved": float((gain > 0).float().mean().item()),
-            "note": "vf_alpha_crown: intermediate bounds as in the verify step, then per-row lower-slope Adam ascent"}
+    out = {"iters": args.alpha_iters, "lr": 0.1, "value": weak_throughput(world, B * R, steps, a_ms),
+           "unit": UNIT, "ms_per_step": a_ms / steps, "mean_lb_gain": float(gain.mean().item()),
+           "rows_improved": float((gain > 0).float().mean().item()),
+           "note": "vf_alpha_crown: intermediate bounds as in the verify step, then per-row lower-slope Adam ascent"}
+    if args.alpha_inter_iters > 0:
+        kw = dict(crown_relus=w.crown_relus, want_pre=True)
+        plain = net.verify(centres, w.eps, C, **kw)
+        net.verify(centres, w.eps, C, alpha_inter_iters=args.alpha_inter_iters, **kw)  # warm-up
+        torch.cuda.synchronize()
+        i_ms = 0.0
+        for i in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            ri = net.verify(centres, w.eps, C, alpha_inter_iters=args.alpha_inter_iters, **kw)
+            e1.record(stream)
+            e1.synchronize()
+            i_ms += e0.elapsed_time(e1)
+        i_ms = max_over_ranks(i_ms, dev)
+        srcs = [nd.src for k, nd in enumerate(w.net) if nd.op == "relu" and
+                (w.crown_relus is None or k in w.crown_relus) and k > 2]  # refined ReLUs (the first is exact)
+        width = sum((net.node_block(plain["pre_ub"], v, B) - net.node_block(plain["pre_lb"], v, B)).sum().item()
+                    for v in srcs)
+        width_i = sum((net.node_block(ri["pre_ub"], v, B) - net.node_block(ri["pre_lb"], v, B)).sum().item()
+                      for v in srcs)
+        out["intermediate"] = {
+            "iters": args.alpha_inter_iters, "lr": 0.1, "value": weak_throughput(world, B * R, steps, i_ms),
+            "unit": UNIT, "ms_per_step": i_ms / steps,
+            "mean_lb_gain": float((ri["lb"] - plain["lb"]).mean().item()),
+            "verified_plain": int(plain["verified"].sum().item()), "verified": int(ri["verified"].sum().item()),
+            "refined_width_ratio": width_i / width if width else None,
+            "note": "vf_verify_batch with vf_opts.alpha_inter_iters: alpha-CROWN on every refined intermediate "
+                    "bound (rows [e_j; -e_j] of the neurons still unstable after the CROWN pass), then the plain "
+                    "specification pass"}
+    return out
 
 
 def sound_leg(args, w, net, centres, C, out, kw, stream, flush, dev, world, specs):
@@ -661,6 +692,8 @@ def main():
                     help="also time the sound-in-fp32 verify call for this many steps (0 = skip)")
     ap.add_argument("--bab-domains", type=int, default=512,
                     help="also time vf_bab_verify with this budget of subdomains per centre (0 = skip)")
+    ap.add_argument("--alpha-inter-iters", type=int, default=5,
+                    help="Adam steps of the intermediate-bound alpha leg (0: skip it)")
     ap.add_argument("--bab-centres", type=int, default=2)
     ap.add_argument("--bab-batch", type=int, default=64)
     ap.add_argument("--bab-alpha-iters", type=int, default=10)

@@ -148,6 +148,16 @@ typedef struct {
      * intercept terms, concretisation), rounded down. Contractions take the FFMA kernels (IEEE rounding),
      * not the tensor cores; receptive-field windows and the fused concretisation are off. */
     int sound;
+    /* alpha-CROWN for the intermediate bounds (technical summary, sections 3 and 4.3: the per-neuron alpha
+     * tensors; the reading is this library's): alpha_inter_iters > 0 runs, right after the CROWN pass of every
+     * refined ReLU whose source p is a dense node, alpha_inter_iters Adam steps of size alpha_inter_lr (the
+     * ascent of vf_alpha_crown: per-row slopes of every earlier ReLU, split multipliers where `split` is set)
+     * on rows [e_j; -e_j] over p for the neurons j still unstable (l < 0 < u); l_j = max(l_j, best lower bound),
+     * u_j = min(u_j, -best bound of -e_j), and the ReLU's relaxation is formed again before later layers use it.
+     * Chain networks only (VF_ERR_UNSUPPORTED otherwise); reads unstable counts back (synchronises `stream`),
+     * so not with no_host_sync; not with sound. 0 = off. */
+    int alpha_inter_iters;
+    float alpha_inter_lr;
 } vf_opts;
 
 /* Whole verification step (section 1): IBP, CROWN intermediate bounds, specification

@@ -1009,6 +1009,12 @@ int sound_weights(vf_net* net, int B, float eps, const float* centres, const Ibp
     return VF_OK;
 }
 
+bool affine_chain(const vf_net* net);
+int alpha_chain(vf_net* net, int L, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
+                const vf_opts& o, int iters, float lr, bool grad_mode, const float* alpha_in, float* grad_out,
+                float* lb, float* lb_start, float* alpha_out, const Bounds& bd, Arena ar, cudaStream_t s,
+                const float* beta_in, float* beta_grad_out);
+
 int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf_opts& o, Arena& ar, IbpState& st,
                    Bounds& bd, cudaStream_t s, const int* finite_flag = nullptr) {
     const int nn = (int)net->nodes.size();
@@ -1099,6 +1105,41 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
     Arena tmp = ar;  // pass outputs are transient
     float* pass_out = tmp.take<float>((size_t)B * max_pass_rows);
     if (!pass_out) return fail(VF_ERR_WORKSPACE, "workspace too small");
+    // alpha-CROWN for the bounds of ReLU k's dense source p, right after its CROWN pass: the neurons still
+    // unstable take rows [e_j; -e_j] over p, ascended (per-row slopes of the earlier ReLUs, split multipliers
+    // where splits are given) on the network up to p; their bounds become max / min with the best iterate, and
+    // the relaxation of k is formed again.
+    const bool chain = affine_chain(net);
+    auto inter_alpha = [&](int k) -> int {
+        const int p = net->nodes[k].src;
+        if (o.alpha_inter_iters <= 0 || sound || !refined(k) || net->nodes[p].op != VF_DENSE) return VF_OK;
+        if (!chain) return fail(VF_ERR_UNSUPPORTED, "intermediate alpha optimisation covers chain networks");
+        const long long np = net->nodes[p].n;
+        Arena t2 = tmp;
+        int* cnt = t2.take<int>(B);
+        if (!cnt) return fail(VF_ERR_WORKSPACE, "workspace too small");
+        LAUNCH(net, launch_unstable_count(bd.Lw[p], bd.Uw[p], B, np, cnt, s));
+        std::vector<int> h(B);
+        CU(cudaMemcpyAsync(h.data(), cnt, sizeof(int) * B, cudaMemcpyDeviceToHost, s));
+        CU(cudaStreamSynchronize(s));
+        const int hp = *std::max_element(h.begin(), h.end());
+        if (hp == 0) return VF_OK;
+        int* idx = t2.take<int>((size_t)B * hp);
+        float* rows = t2.take<float>((size_t)B * 2 * hp * np);
+        float* best = t2.take<float>((size_t)B * 2 * hp);
+        if (!idx || !rows || !best) return fail(VF_ERR_WORKSPACE, "workspace too small for intermediate alpha rows");
+        LAUNCH(net, launch_unstable_list(bd.Lw[p], bd.Uw[p], B, np, hp, idx, s));
+        LAUNCH(net, launch_unit_rows(idx, B, hp, np, rows, s));
+        TRY(alpha_chain(net, p, centres, B, eps, rows, 2 * hp, 2LL * hp * np, o, o.alpha_inter_iters,
+                        o.alpha_inter_lr, false, nullptr, nullptr, best, nullptr, nullptr, bd, t2, s, nullptr, nullptr));
+        LAUNCH(net, launch_intersect_compact(bd.Lw[p], bd.Uw[p], best, idx, B, np, hp, s));
+        const float* bias;
+        long long pc;
+        relax_args(k, &bias, &pc);
+        LAUNCH(net, launch_relax_params(bd.Lw[p], bd.Uw[p], o.alpha ? o.alpha[k] : nullptr, (long long)B * net->nodes[k].n,
+                                        P[k], bias, net->nodes[k].n, pc, s, sound));
+        return VF_OK;
+    };
     for (int k = 0; k < nn; ++k) {
         const Node& nd = net->nodes[k];
         if (nd.op != VF_RELU) continue;
@@ -1130,6 +1171,7 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
             relax_args(k, &bias, &pc);
             LAUNCH(net, launch_relu_bounds_relax(nullptr, nullptr, nullptr, pass_out, bd.Lw[p], bd.Uw[p],
                                                  o.alpha ? o.alpha[k] : nullptr, B, np, P[k], bias, pc, sound, s));
+            TRY(inter_alpha(k));
             continue;
         }
         if (!refined(k)) continue;  // relaxed together with its bounds above
@@ -1138,6 +1180,7 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
         LAUNCH(net, launch_relax_params(bd.Lw[p], bd.Uw[p], o.alpha ? o.alpha[k] : nullptr, (long long)B * nd.n, P[k],
                                         aff ? sn.b : nullptr, nd.n, sn.op == VF_CONV2D ? (long long)sn.h * sn.w : 1, s,
                                         sound));
+        TRY(inter_alpha(k));
     }
     return VF_OK;
 }
@@ -1159,18 +1202,18 @@ bool affine_chain(const vf_net* net) {
 // Otherwise: iters Adam ascent steps from the adaptive slopes, lb = best bound seen per row,
 // lb_start (optional) = the bound at the adaptive start, alpha_out (optional) = the final slopes.
 // Slope arrays: for each ReLU node in order, a [B, R, n] block.
-int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
-               const vf_opts& o, int iters, float lr, bool grad_mode, const float* alpha_in, float* grad_out,
-               float* lb, float* lb_start, float* alpha_out, cudaStream_t s, const float* beta_in = nullptr,
-               float* beta_grad_out = nullptr) {
+// alpha-CROWN on a chain network (affine_chain) up to its node L, which is dense: rows C [B or 1, R, n_L] over
+// node L's output, per-row slopes of every ReLU before L (and split multipliers where o.split is set), the
+// relaxations of bd, scratch from ar. The specification pass (L = last node) and the intermediate passes of
+// prepare_bounds (L = a ReLU's dense source, rows [e_j; -e_j]) both run here.
+int alpha_chain(vf_net* net, int L, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
+                const vf_opts& o, int iters, float lr, bool grad_mode, const float* alpha_in, float* grad_out,
+                float* lb, float* lb_start, float* alpha_out, const Bounds& bd, Arena ar, cudaStream_t s,
+                const float* beta_in, float* beta_grad_out) {
     const int nn = (int)net->nodes.size();
-    const int L = nn - 1;
     const long long n0 = net->nodes[0].n;
     const int nL = (int)net->nodes[L].n;
-    Arena ar{net->ws, net->ws_bytes};
-    IbpState st;
-    Bounds bd;
-    TRY(prepare_bounds(net, centres, B, eps, o, ar, st, bd, s));
+    if (net->nodes[L].op != VF_DENSE) return fail(VF_ERR_UNSUPPORTED, "alpha optimisation needs rows over a dense node");
     std::vector<int> relus;
     long long sum_n = 0, nmax = 1;
     std::vector<long long> aoff(nn, 0);  // offset of each ReLU's [B, R, n] slope block
@@ -1321,6 +1364,18 @@ int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float*
             }
     }
     return VF_OK;
+}
+
+int spec_alpha(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
+               const vf_opts& o, int iters, float lr, bool grad_mode, const float* alpha_in, float* grad_out,
+               float* lb, float* lb_start, float* alpha_out, cudaStream_t s, const float* beta_in = nullptr,
+               float* beta_grad_out = nullptr) {
+    Arena ar{net->ws, net->ws_bytes};
+    IbpState st;
+    Bounds bd;
+    TRY(prepare_bounds(net, centres, B, eps, o, ar, st, bd, s));
+    return alpha_chain(net, (int)net->nodes.size() - 1, centres, B, eps, C, R, C_bstride, o, iters, lr, grad_mode,
+                       alpha_in, grad_out, lb, lb_start, alpha_out, bd, ar, s, beta_in, beta_grad_out);
 }
 
 // alpha-CROWN on any node graph (residual adds included): the same computation as spec_alpha with every
@@ -1878,11 +1933,23 @@ int vf_concretize(const float* lambda, const float* cst, const float* centres, f
     return VF_OK;
 }
 
+// The intermediate alpha options (vf_opts.alpha_inter_iters / alpha_inter_lr) of any call.
+int check_inter_opts(const vf_opts& o) {
+    if (o.alpha_inter_iters < 0) return fail(VF_ERR_ARG, "alpha_inter_iters must be >= 0");
+    if (o.alpha_inter_iters == 0) return VF_OK;
+    if (!std::isfinite(o.alpha_inter_lr) || o.alpha_inter_lr < 0.f)
+        return fail(VF_ERR_NONFINITE, "alpha_inter_lr must be finite and >= 0");
+    if (o.no_host_sync) return fail(VF_ERR_UNSUPPORTED, "intermediate alpha optimisation synchronises the stream");
+    if (o.sound) return fail(VF_ERR_UNSUPPORTED, "intermediate alpha optimisation is not part of the sound mode");
+    return VF_OK;
+}
+
 int vf_verify_batch(vf_net* net, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
                     const vf_opts* opts, float* lb, float* ub, float* lb_ibp, uint8_t* verified, void* stream) {
     TRY(check_net(net));
     vf_opts o{};
     if (opts) o = *opts;
+    TRY(check_inter_opts(o));
     if (!centres || !C || !lb) return fail(VF_ERR_ARG, "centres, C and lb must not be NULL");
     if (o.both_sides && !ub) return fail(VF_ERR_ARG, "both_sides needs ub");
     if (B < 0 || R < 0 || C_bstride < 0) return fail(VF_ERR_ARG, "negative size");
@@ -1963,6 +2030,7 @@ int vf_alpha_crown(vf_net* net, const float* centres, int B, float eps, const fl
     TRY(check_net(net));
     vf_opts o{};
     if (opts) o = *opts;
+    TRY(check_inter_opts(o));
     if (!centres || !C || !lb) return fail(VF_ERR_ARG, "centres, C and lb must not be NULL");
     if (B < 0 || R < 0 || C_bstride < 0 || iters < 0) return fail(VF_ERR_ARG, "negative size");
     if (!std::isfinite(eps) || eps < 0.f || !std::isfinite(lr) || lr < 0.f)
@@ -1988,6 +2056,7 @@ int vf_alpha_beta_grad(vf_net* net, const float* centres, int B, float eps, cons
     TRY(check_net(net));
     vf_opts o{};
     if (opts) o = *opts;
+    TRY(check_inter_opts(o));
     if (!centres || !C || !lb || !alpha || !grad_alpha) return fail(VF_ERR_ARG, "NULL pointer");
     if (B < 0 || R < 0 || C_bstride < 0) return fail(VF_ERR_ARG, "negative size");
     if (!std::isfinite(eps) || eps < 0.f) return fail(VF_ERR_NONFINITE, "eps must be finite and >= 0");

@@ -48,7 +48,8 @@ class Opts(ctypes.Structure):
     _fields_ = [("relu_crown", ctypes.POINTER(ctypes.c_int)), ("alpha", ctypes.POINTER(ctypes.c_void_p)),
                 ("both_sides", ctypes.c_int), ("skip_finite_check", ctypes.c_int),
                 ("pre_lb", ctypes.c_void_p), ("pre_ub", ctypes.c_void_p), ("no_host_sync", ctypes.c_int),
-                ("split", ctypes.POINTER(ctypes.c_void_p)), ("sound", ctypes.c_int)]
+                ("split", ctypes.POINTER(ctypes.c_void_p)), ("sound", ctypes.c_int),
+                ("alpha_inter_iters", ctypes.c_int), ("alpha_inter_lr", ctypes.c_float)]
 
 
 class BabOpts(ctypes.Structure):
@@ -213,10 +214,11 @@ class Net:
     def verify(self, centres: torch.Tensor, eps: float, C: torch.Tensor, crown_relus: Optional[Sequence[int]] = None,
                alpha: Optional[Dict[int, torch.Tensor]] = None, both_sides: bool = False, want_pre: bool = False,
                skip_finite_check: bool = False, no_host_sync: bool = False, stream=None, out=None,
-               splits: Optional[Dict[int, torch.Tensor]] = None, sound: bool = False):
+               splits: Optional[Dict[int, torch.Tensor]] = None, sound: bool = False, alpha_inter_iters: int = 0,
+               alpha_inter_lr: float = 0.1):
         """vf_verify_batch. C: [B or 1, R, n_L]. splits: ReLU node -> int8 [B, n] signs (+1: z >= 0,
         -1: z <= 0, 0: free), one subdomain per centre row. sound: bounds that hold despite fp32 rounding.
-        Returns dict of device tensors."""
+        alpha_inter_iters > 0: alpha-CROWN for the intermediate bounds (vf_opts). Returns dict of device tensors."""
         B = centres.shape[0]
         R = C.shape[1]
         dev = centres.device
@@ -245,6 +247,8 @@ class Net:
         o.skip_finite_check = 1 if skip_finite_check else 0
         o.no_host_sync = 1 if no_host_sync else 0
         o.sound = 1 if sound else 0
+        o.alpha_inter_iters = int(alpha_inter_iters)
+        o.alpha_inter_lr = float(alpha_inter_lr)
         sarr = self._split_array(splits)
         if sarr is not None:
             o.split = ctypes.cast(sarr, ctypes.POINTER(ctypes.c_void_p))
@@ -265,8 +269,10 @@ class Net:
             arr[v] = sg.data_ptr()
         return arr
 
-    def _opts(self, crown_relus=None, splits=None):
+    def _opts(self, crown_relus=None, splits=None, alpha_inter_iters=0, alpha_inter_lr=0.1):
         o = Opts()
+        o.alpha_inter_iters = int(alpha_inter_iters)
+        o.alpha_inter_lr = float(alpha_inter_lr)
         keep = []
         if crown_relus is not None:
             flags = (ctypes.c_int * self.n_nodes)()
@@ -285,15 +291,17 @@ class Net:
         return B * R * sum(self.sizes[v] for v in self.relu_ids)
 
     def alpha_crown(self, centres: torch.Tensor, eps: float, C: torch.Tensor, iters: int = 20, lr: float = 0.1,
-                    crown_relus=None, want_alpha: bool = False, stream=None, splits=None):
+                    crown_relus=None, want_alpha: bool = False, stream=None, splits=None, alpha_inter_iters: int = 0,
+                    alpha_inter_lr: float = 0.1):
         """vf_alpha_crown: returns dict(lb=best bound [B, R], lb_start=[B, R], alpha=final slopes or None).
-        With splits (see verify) the split multipliers beta are optimised with the slopes."""
+        With splits (see verify) the split multipliers beta are optimised with the slopes; alpha_inter_iters > 0
+        optimises the intermediate bounds first (vf_opts)."""
         B, R = centres.shape[0], C.shape[1]
         bstride = 0 if C.shape[0] == 1 else R * C.shape[2]
         lb = torch.empty(B, R, device=centres.device)
         lb0 = torch.empty(B, R, device=centres.device)
         al = torch.empty(self.alpha_size(B, R), device=centres.device) if want_alpha else None
-        o, keep = self._opts(crown_relus, splits)
+        o, keep = self._opts(crown_relus, splits, alpha_inter_iters, alpha_inter_lr)
         _check(lib().vf_alpha_crown(self.h, _ptr(centres), B, float(eps), _ptr(C), R, bstride, ctypes.byref(o), iters,
                                     float(lr), _ptr(lb), _ptr(lb0), _ptr(al), _stream_ptr(stream)))
         return {"lb": lb, "lb_start": lb0, "alpha": al}
