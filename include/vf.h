@@ -244,6 +244,9 @@ typedef struct {
                                first), the search-wide index of the neuron it would be split on (-1: none is
                                unstable); at most trace_cap entries are written, result->domains are bounded */
     int trace_cap;
+    int alpha_inter_iters;  /* as vf_opts.alpha_inter_iters for every bound of the search (0: off): the subdomains'
+                               intermediate bounds by alpha-CROWN, with the split multipliers of earlier layers */
+    float alpha_inter_lr;
 } vf_bab_opts;
 typedef struct {
     int status;             /* VF_BAB_VERIFIED, VF_BAB_FALSIFIED or VF_BAB_UNKNOWN */

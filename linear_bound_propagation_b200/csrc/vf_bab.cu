@@ -118,11 +118,15 @@ int device_bound(void* user, int n, const int* split_offset, const int* split_co
     o.split = sp.data();
     o.pre_lb = d.plb;
     o.pre_ub = d.pub;
+    o.alpha_inter_iters = d.opts->alpha_inter_iters;
+    o.alpha_inter_lr = d.opts->alpha_inter_lr;
     BAB_TRY(vf_verify_batch(d.net, d.cen, n, d.eps, d.C, d.R, 0, &o, d.lbv, nullptr, nullptr, nullptr, d.stream));
     if (d.opts->alpha_iters > 0) {
         vf_opts oa{};
         oa.relu_crown = d.opts->relu_crown;
         oa.split = sp.data();
+        oa.alpha_inter_iters = d.opts->alpha_inter_iters;
+        oa.alpha_inter_lr = d.opts->alpha_inter_lr;
         BAB_TRY(vf_alpha_crown(d.net, d.cen, n, d.eps, d.C, d.R, 0, &oa, d.opts->alpha_iters, d.opts->lr, d.lba, nullptr,
                                nullptr, d.stream));
     }
@@ -149,6 +153,7 @@ extern "C" int vf_bab_verify(vf_net* net, const float* centre, float eps, const 
         return vf::set_last_error(VF_ERR_ARG, "need max_domains >= 1, an even batch >= 2 and alpha_iters >= 0");
     if (!std::isfinite(eps) || eps < 0.f) return vf::set_last_error(VF_ERR_NONFINITE, "eps must be finite and >= 0");
     if (!std::isfinite(opts->lr)) return vf::set_last_error(VF_ERR_NONFINITE, "lr must be finite");
+    if (opts->alpha_inter_iters < 0) return vf::set_last_error(VF_ERR_ARG, "alpha_inter_iters must be >= 0");
     cudaStream_t s = (cudaStream_t)stream;
 
     // ---- the graph: ReLU layers, their input blocks and search-wide neuron indices

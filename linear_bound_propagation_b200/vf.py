@@ -55,7 +55,8 @@ class Opts(ctypes.Structure):
 class BabOpts(ctypes.Structure):
     _fields_ = [("max_domains", ctypes.c_int), ("batch", ctypes.c_int), ("alpha_iters", ctypes.c_int),
                 ("lr", ctypes.c_float), ("relu_crown", ctypes.POINTER(ctypes.c_int)),
-                ("trace", ctypes.POINTER(ctypes.c_int)), ("trace_cap", ctypes.c_int)]
+                ("trace", ctypes.POINTER(ctypes.c_int)), ("trace_cap", ctypes.c_int),
+                ("alpha_inter_iters", ctypes.c_int), ("alpha_inter_lr", ctypes.c_float)]
 
 
 class BabResult(ctypes.Structure):
@@ -333,11 +334,14 @@ class Net:
         return lb, ga, gb
 
     def bab(self, centre: torch.Tensor, eps: float, C: torch.Tensor, max_domains: int = 1000, batch: int = 16,
-            alpha_iters: int = 20, lr: float = 0.1, crown_relus=None, stream=None, trace: bool = False):
+            alpha_iters: int = 20, lr: float = 0.1, crown_relus=None, stream=None, trace: bool = False,
+            alpha_inter_iters: int = 0, alpha_inter_lr: float = 0.1):
         """vf_bab_verify on one box: centre [n0], C [R, n_L] (device). Returns dict(status, domains, rounds,
         max_depth, lb), plus, with trace, the branching neuron of every bounded subdomain in the order bounded
-        (search-wide index, -1 if none)."""
-        o = BabOpts(max_domains=max_domains, batch=batch, alpha_iters=alpha_iters, lr=float(lr))
+        (search-wide index, -1 if none). alpha_inter_iters > 0: intermediate bounds of every subdomain by
+        alpha-CROWN with the split multipliers (vf_opts)."""
+        o = BabOpts(max_domains=max_domains, batch=batch, alpha_iters=alpha_iters, lr=float(lr),
+                    alpha_inter_iters=int(alpha_inter_iters), alpha_inter_lr=float(alpha_inter_lr))
         tbuf = None
         if trace:
             tbuf = (ctypes.c_int * max_domains)()

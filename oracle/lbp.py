@@ -624,13 +624,15 @@ class BabResult:
 
 
 def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_relus=None, iters: int = 20,
-        lr: float = 0.1) -> BabResult:
+        lr: float = 0.1, alpha_inter_iters: int = 0, alpha_inter_lr: float = 0.1) -> BabResult:
     """Branch and bound over ReLU splits on top of ``verify`` [SNNV §2.2, §3, §4.3: beta-CROWN with
     branch-and-bound for complete verification; the page names the method only].
 
     Property: every row of C [R, n_L] is positive at every input of the box centre +- eps.
     A subdomain's row bound is the larger of ``verify``'s bound and the best bound of ``alpha_crown``
-    (``iters`` Adam steps of size ``lr`` on the slopes and on the split multipliers beta).
+    (``iters`` Adam steps of size ``lr`` on the slopes and on the split multipliers beta); with
+    ``alpha_inter_iters`` > 0 both take their intermediate bounds from ``verify``'s intermediate ascent (slopes
+    and the split multipliers of earlier layers).
     Reading of the search (one plain best-first variant):
       1. the centre is evaluated first, then every row's CROWN minimiser vertex of the whole box
          (``minimiser_attack``); a row < 0 at any of these inputs is a counterexample ("falsified");
@@ -661,11 +663,13 @@ def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_rel
             for (k, j), sign in d.items():
                 sp[k][i, j] = sign
         cen = np.repeat(centre[None, :], len(domains), axis=0)
-        res = verify(net, cen, eps, C[None], crown_relus=crown_relus, splits=sp)
+        res = verify(net, cen, eps, C[None], crown_relus=crown_relus, splits=sp, alpha_inter_iters=alpha_inter_iters,
+                     alpha_inter_lr=alpha_inter_lr)
         lb = res.lb
         if iters > 0:
             lb = np.maximum(lb, alpha_crown(net, cen, eps, C[None], iters=iters, lr=lr, crown_relus=crown_relus,
-                                            splits=sp)[0])
+                                            splits=sp, alpha_inter_iters=alpha_inter_iters,
+                                            alpha_inter_lr=alpha_inter_lr)[0])
         out = []
         for i in range(len(domains)):
             empty = any(np.any(res.pre_bounds[k][0][i] > res.pre_bounds[k][1][i]) for k in relus)

@@ -225,3 +225,28 @@ def test_bab_rejects_bad_options():
         with pytest.raises(vf.VfError) as e:
             g.bab(_dev(centres[0]), eps, _dev(C[0]), **kw)
         assert e.value.code == vf.VF_ERR_ARG
+
+
+def test_bab_with_intermediate_alpha():
+    """Branch and bound with alpha-CROWN intermediate bounds (slopes and the split multipliers of earlier layers)
+    in every subdomain, on the 72 small properties of the decision test: the device ends with the oracle's status
+    (same options) on at least 90% of them, every "verified" holds on sampled inputs, and the properties that the
+    option turns from "unknown" to "verified" in the oracle are verified on the device as well."""
+    from tests.test_gpu_edge_cases import _bab_problems
+    agree = total = 0
+    gained = []
+    for name, net, c, eps, C in _bab_problems():
+        g = vf.Net(net)
+        r = g.bab(_dev(c), eps, _dev(C), max_domains=120, batch=8, alpha_iters=0, alpha_inter_iters=5)
+        torch.cuda.synchronize()
+        g.check()
+        o = O.bab(net, c, eps, C, max_domains=120, batch=8, iters=0, alpha_inter_iters=5)
+        total += 1
+        agree += r["status"] == o.status
+        if r["status"] == "verified":
+            xs = c + eps * (2 * np.random.default_rng(2).random((20000, c.size)) - 1)
+            assert (O.forward(net, xs)[-1] @ C.astype(np.float64).T).min() > 0.0, name
+        if o.status == "verified" and O.bab(net, c, eps, C, max_domains=120, batch=8, iters=0).status == "unknown":
+            gained.append((name, r["status"]))
+    assert agree >= 0.9 * total, f"{agree} of {total} statuses agree"
+    assert gained and all(s == "verified" for _, s in gained), gained
