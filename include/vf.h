@@ -296,8 +296,8 @@ enum {
     VF_KERNEL_CONV = 3,
     VF_KERNEL_CONV_WIN = 4,
     VF_KERNEL_CONV_TC = 5, /* tensor-core implicit GEMM, whole maps and windows; flops as for windows */
-    VF_KERNEL_DENSE_FWD_TC = 6 /* forward products on the tensor cores: IBP W c + b and |W| r, the alpha
-                                  gradient's G W^T + b; 2*M*K*N flops */
+    VF_KERNEL_DENSE_FWD_TC = 6 /* forward products on the tensor cores: the alpha gradient's G W^T + b (and with
+                                  VF_FWD_TC=ibp at vf_net_create the IBP W c + b, |W| r); 2*M*K*N flops */
 };
 int vf_profile_enable(vf_net* net, int enable);
 int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms, double* flops, int reset);

@@ -108,8 +108,9 @@ struct vf_net {
     int conv_tc = 1;        // convolution steps on the tensor cores where the shapes allow (VF_CONV_TC=0: off)
     int conv_tcn = 0;       // ... with the taps-in-N kernel where its shapes allow (VF_CONV_TC=tapn; measured slower)
     int call_sound = 0;     // set for the duration of a vf_opts.sound call: contractions take FFMA kernels
-    // forward products (IBP, alpha up pass) on the tensor cores: 0 never (VF_FWD_TC=0), 1 (default) when the product
-    // has at least kFwdTcMinTiles output tiles, 2 whenever the shapes allow (VF_FWD_TC=all)
+    // forward products of the alpha ascent (G W^T + b) on the tensor cores: 0 never (VF_FWD_TC=0), 1 (default) when
+    // the product has at least kFwdTcMinTiles output tiles, 2 whenever the shapes allow (VF_FWD_TC=all); 3 also the
+    // IBP products W c + b, |W| r (VF_FWD_TC=ibp; less accurate on deep wide networks, see run_ibp)
     int fwd_tc = 1;
     float4* ident_row = nullptr;  // identity relaxation row {1, 1, 0, 0} x (largest node size), for forward products
     bool prof = false;
@@ -719,7 +720,7 @@ bool fwd_tc_ok(const vf_net* net, const Node& nd, const float* A, long long M, i
     const int N = (int)nd.n;
     if (net->dense_kernel != 0 || net->fwd_tc == 0 || net->call_sound || nd.WfHi == nullptr) return false;
     if (!dense_fwd_tc_supported(A, M, K, N)) return false;
-    return net->fwd_tc == 2 || ((M + 127) / 128) * dense_back_tc_tiles_n(N) >= kFwdTcMinTiles;
+    return net->fwd_tc >= 2 || ((M + 127) / 128) * dense_back_tc_tiles_n(N) >= kFwdTcMinTiles;
 }
 
 // out [M, N] = A [M, K] W^T + bias (absw: A |W|^T, no bias) for dense node nd: the tensor-core kernel where
@@ -779,9 +780,11 @@ int run_ibp(vf_net* net, const float* centres, int B, float eps, Arena& ar, IbpS
         if (sound && (!T || !S)) return fail(VF_ERR_WORKSPACE, "workspace too small for sound IBP");
         switch (nd.op) {
             case VF_DENSE:
-                if (!sound && fwd_tc_ok(net, nd, st.c[sv], B, (int)net->nodes[sv].n) &&
+                // IBP products stay on the FFMA kernel: on the tensor cores (3xTF32) the bounds of the
+                // 3072-1024x8-100 network drifted from the fp64 oracle by up to 1.06x the parity tolerance after
+                // eight layers (FFMA: 0.02x), and they are under 0.5% of any step
+                if (!sound && net->fwd_tc == 3 && fwd_tc_ok(net, nd, st.c[sv], B, (int)net->nodes[sv].n) &&
                     (sv == 0 || fwd_tc_ok(net, nd, st.r[sv], B, (int)net->nodes[sv].n))) {
-                    // centre W c + b and radius |W| r on the tensor cores (the input box: eps * sum_k |W[n, k]|)
                     TRY(fwd_product(net, nd, st.c[sv], B, (int)net->nodes[sv].n, false, nd.b, st.c[v], s));
                     if (sv == 0)
                         LAUNCH(net, launch_ibp_radius_rowsum(nd.rowsum_abs, eps, B, (int)nd.n, st.r[v], s));
@@ -1661,7 +1664,8 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
         net->conv_tc = strcmp(f, "0") != 0;
         net->conv_tcn = strcmp(f, "tapn") == 0;
     }
-    if (const char* f = getenv("VF_FWD_TC")) net->fwd_tc = strcmp(f, "0") == 0 ? 0 : (strcmp(f, "all") == 0 ? 2 : 1);
+    if (const char* f = getenv("VF_FWD_TC"))
+        net->fwd_tc = strcmp(f, "0") == 0 ? 0 : (strcmp(f, "all") == 0 ? 2 : (strcmp(f, "ibp") == 0 ? 3 : 1));
     CU(cudaMalloc(&net->d_err, sizeof(int)));
     CU(cudaMemset(net->d_err, 0, sizeof(int)));
     net->nodes.resize(n_nodes);

@@ -65,7 +65,9 @@ def test_cfg3_full_size_sampled():
 @pytest.mark.parametrize("eps", [0.5 / 255, 1.0 / 255, 2.0 / 255])
 def test_cfg5_full_size_sampled(eps):
     w = synth.workload(5, eps=eps)
-    _check_sampled(w, [0, 4095])
+    # eight centres (about a second of oracle time each): with 8 x 1024 IBP-substituted neurons per centre, a
+    # centre often holds an adaptive-slope near-tie, and at most a quarter of the sample may sit there
+    _check_sampled(w, [0, 1, 1023, 2047, 2048, 3071, 4094, 4095])
 
 
 @pytest.mark.slow
