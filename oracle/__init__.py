@@ -23,17 +23,23 @@ Parity status per function (what pins it, all in tests/test_oracle_*.py):
                                            pointwise L(x) <= f(x))
   verify (intermediate + spec passes)   -- pinned (2-D exact ranges, soundness,
                                            one-hidden-layer ordering, monotonicity in eps)
-  spec_bound_alpha, alpha_crown         -- pinned (central differences, hand optimum,
-                                           soundness of optimised bounds)
+  spec_bound_alpha, ascend, alpha_crown -- pinned (central differences, hand optimum, Adam's closed-form
+                                           first steps, soundness of optimised bounds)
+  verify(alpha_inter_iters=...)         -- pinned (one-neuron closed form of the ascent, the triangle LP
+                                           bounding and reached by the optimised intermediate bounds,
+                                           soundness by sampling, never looser than plain)
   split_clamp, splits in ibp / verify,  -- pinned (soundness on the subdomain by sampling, the
   beta in spec_bound_alpha / alpha_crown   full-split affine closed form, weak and strong LP
                                            duality, central differences for beta)
   branch_scores, bab, bab_search        -- pinned (exact 2-D ranges and sampling: never a wrong
                                            "verified" or "falsified"; splitting verifies
                                            properties the whole-box bound leaves open)
+  minimiser_vertices, minimiser_attack  -- pinned (brute force over the box's vertices: the vertex attains
+                                           the CROWN bound; exact 2-D ranges: only false properties are
+                                           falsified, most clearly false ones without a split)
 """
 from .lbp import (  # noqa: F401
     shapes, conv2d, conv2d_adjoint, forward, ibp, relax_params, backward, concretize,
-    crown_pass, verify, OracleResult, spec_bound_alpha, alpha_crown, split_clamp, branch_scores, bab,
-    bab_search, BabResult,
+    crown_pass, verify, OracleResult, spec_bound_alpha, ascend, alpha_crown, split_clamp, branch_scores, bab,
+    bab_search, BabResult, minimiser_vertices, minimiser_attack,
 )
