@@ -318,17 +318,6 @@ __global__ void intersect_compact_k(float* __restrict__ l, float* __restrict__ u
     }
 }
 
-// rows[b, i, :] = e_j and rows[b, half + i, :] = -e_j for j = idx[b * half + i] (a padding slot, j < 0: zero rows).
-__global__ void unit_rows_k(const int* __restrict__ idx, int B, int half, long long n, float* __restrict__ rows) {
-    GRID_STRIDE(e, (long long)B * 2 * half * n) {
-        const long long r = e / n, col = e % n;
-        const long long b = r / (2 * half);
-        const int i = (int)(r % (2 * half));
-        const int j = idx[b * half + (i < half ? i : i - half)];
-        rows[e] = (j >= 0 && col == j) ? (i < half ? 1.f : -1.f) : 0.f;
-    }
-}
-
 // out[m, :] = sg * W[j, :] for the start neuron j of row m (compacted pass over a dense node).
 __global__ void gather_start_rows_k(float* __restrict__ out, long long ld, long long M, PassGeom pg,
                                     const float* __restrict__ W, long long n_p, long long n_src) {
@@ -521,13 +510,6 @@ cudaError_t launch_intersect_compact(float* l, float* u, const float* pass_out, 
                                      int half, cudaStream_t s) {
     if (B <= 0 || half <= 0) return cudaSuccess;
     intersect_compact_k<<<grid_for((long long)B * half, 256), 256, 0, s>>>(l, u, pass_out, idx, B, n, half);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_unit_rows(const int* idx, int B, int half, long long n, float* rows, cudaStream_t s) {
-    const long long total = (long long)B * 2 * half * n;
-    if (total <= 0) return cudaSuccess;
-    unit_rows_k<<<grid_for(total, 256), 256, 0, s>>>(idx, B, half, n, rows);
     return cudaGetLastError();
 }
 

@@ -1016,7 +1016,7 @@ bool affine_chain(const vf_net* net);
 int alpha_chain(vf_net* net, int L, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
                 const vf_opts& o, int iters, float lr, bool grad_mode, const float* alpha_in, float* grad_out,
                 float* lb, float* lb_start, float* alpha_out, const Bounds& bd, Arena ar, cudaStream_t s,
-                const float* beta_in, float* beta_grad_out);
+                const float* beta_in, float* beta_grad_out, const int* unit_idx = nullptr);
 
 int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf_opts& o, Arena& ar, IbpState& st,
                    Bounds& bd, cudaStream_t s, const int* finite_flag = nullptr) {
@@ -1128,13 +1128,11 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
         const int hp = *std::max_element(h.begin(), h.end());
         if (hp == 0) return VF_OK;
         int* idx = t2.take<int>((size_t)B * hp);
-        float* rows = t2.take<float>((size_t)B * 2 * hp * np);
         float* best = t2.take<float>((size_t)B * 2 * hp);
-        if (!idx || !rows || !best) return fail(VF_ERR_WORKSPACE, "workspace too small for intermediate alpha rows");
+        if (!idx || !best) return fail(VF_ERR_WORKSPACE, "workspace too small for intermediate alpha rows");
         LAUNCH(net, launch_unstable_list(bd.Lw[p], bd.Uw[p], B, np, hp, idx, s));
-        LAUNCH(net, launch_unit_rows(idx, B, hp, np, rows, s));
-        TRY(alpha_chain(net, p, centres, B, eps, rows, 2 * hp, 2LL * hp * np, o, o.alpha_inter_iters,
-                        o.alpha_inter_lr, false, nullptr, nullptr, best, nullptr, nullptr, bd, t2, s, nullptr, nullptr));
+        TRY(alpha_chain(net, p, centres, B, eps, nullptr, 2 * hp, 0, o, o.alpha_inter_iters, o.alpha_inter_lr, false,
+                        nullptr, nullptr, best, nullptr, nullptr, bd, t2, s, nullptr, nullptr, idx));
         LAUNCH(net, launch_intersect_compact(bd.Lw[p], bd.Uw[p], best, idx, B, np, hp, s));
         const float* bias;
         long long pc;
@@ -1208,11 +1206,12 @@ bool affine_chain(const vf_net* net) {
 // alpha-CROWN on a chain network (affine_chain) up to its node L, which is dense: rows C [B or 1, R, n_L] over
 // node L's output, per-row slopes of every ReLU before L (and split multipliers where o.split is set), the
 // relaxations of bd, scratch from ar. The specification pass (L = last node) and the intermediate passes of
-// prepare_bounds (L = a ReLU's dense source, rows [e_j; -e_j]) both run here.
+// prepare_bounds (L = a ReLU's dense source) both run here. unit_idx (or null): the rows are [e_j; -e_j] per
+// centre for the neurons listed as in a compacted identity-trick pass (R = 2 x entries per centre; C unused).
 int alpha_chain(vf_net* net, int L, const float* centres, int B, float eps, const float* C, int R, long long C_bstride,
                 const vf_opts& o, int iters, float lr, bool grad_mode, const float* alpha_in, float* grad_out,
                 float* lb, float* lb_start, float* alpha_out, const Bounds& bd, Arena ar, cudaStream_t s,
-                const float* beta_in, float* beta_grad_out) {
+                const float* beta_in, float* beta_grad_out, const int* unit_idx) {
     const int nn = (int)net->nodes.size();
     const long long n0 = net->nodes[0].n;
     const int nL = (int)net->nodes[L].n;
@@ -1314,9 +1313,16 @@ int alpha_chain(vf_net* net, int L, const float* centres, int B, float eps, cons
             // down: back-substitution of the rows with the current slopes, keeping lam over every ReLU
             CU(cudaMemsetAsync(cst, 0, sizeof(float) * Mc, s));
             const Node& last = net->nodes[L];
-            LAUNCH(net, launch_dense_back(RowRef{C, C_bstride, nL, R, m0}, Relax{nullptr, 0}, last.W, last.b, Mc, nL,
-                                          (int)net->nodes[L - 1].n, pg, OUT_STORE, H[L - 1], net->nodes[L - 1].n, cst,
-                                          nullptr, 0.f, nullptr, s));
+            if (unit_idx != nullptr) {  // rows [e_j; -e_j]: the first step gathers +-W[j, :] and adds +-b[j]
+                const PassGeom pgi{m0, R, unit_idx};
+                LAUNCH(net, launch_gather_start_rows(H[L - 1], net->nodes[L - 1].n, Mc, pgi, last.W, nL,
+                                                     net->nodes[L - 1].n, s));
+                LAUNCH(net, launch_cst_identity_bias(cst, Mc, pgi, last.b, nL, 1, s));
+            } else {
+                LAUNCH(net, launch_dense_back(RowRef{C, C_bstride, nL, R, m0}, Relax{nullptr, 0}, last.W, last.b, Mc,
+                                              nL, (int)net->nodes[L - 1].n, pg, OUT_STORE, H[L - 1],
+                                              net->nodes[L - 1].n, cst, nullptr, 0.f, nullptr, s));
+            }
             for (int u = L - 1; u >= 2; u -= 2) {
                 const int nu = (int)net->nodes[u].n;
                 const Node& d = net->nodes[u - 1];

@@ -226,9 +226,6 @@ cudaError_t launch_intersect(float* l, float* u, const float* l_ibp, const float
 cudaError_t launch_unstable_count(const float* l, const float* u, int B, long long n, int* counts, cudaStream_t s);
 cudaError_t launch_unstable_list(const float* l, const float* u, int B, long long n, int half, int* idx, cudaStream_t s);
 // Intersection for a compacted pass: rows [e_j; -e_j] of the listed neurons, R = 2 * half rows per centre.
-// rows [B, 2 * half, n]: per centre b, rows e_j (first half) and -e_j (second half) for j = idx[b * half + i];
-// padding slots (j < 0) give zero rows.
-cudaError_t launch_unit_rows(const int* idx, int B, int half, long long n, float* rows, cudaStream_t s);
 cudaError_t launch_intersect_compact(float* l, float* u, const float* pass_out, const int* idx, int B, long long n,
                                      int half, cudaStream_t s);
 // Rows +-W[j, :] (W is [n_p, n_src], row-major) for the start neurons of a compacted pass over a dense node.
