@@ -526,12 +526,14 @@ def spec_bound_alpha(net, centre, eps, rows, relax, alpha_rows, split_signs=None
     return lb, grads
 
 
-def ascend(net, centre, eps, rows, relax, iters, lr, split_signs=None, betas=(0.9, 0.999)):
+def ascend(net, centre, eps, rows, relax, iters, lr, split_signs=None, betas=(0.9, 0.999), alpha0=None, beta0=None,
+           return_state=False):
     """Projected gradient ascent (Adam, step lr, moments ``betas``) on per-row lower slopes of the bound of
     ``rows`` over ``net``'s last node for one centre [SNNV §1 alpha-CROWN; §3 alpha tensors], starting from the
-    slopes of ``relax``; with split signs (relu node -> [n]) the split multipliers beta are optimised with them
-    (from 0, projected to beta >= 0; see ``spec_bound_alpha``). Returns (best lb over the iterates [R], lb at
-    the start [R])."""
+    slopes of ``relax`` (or from ``alpha0``: relu node -> [R, n], clamped to [0, 1]); with split signs (relu node
+    -> [n]) the split multipliers beta are optimised with them (from 0, or from ``beta0`` where it has the node,
+    projected to beta >= 0; see ``spec_bound_alpha``). Adam's moments start at zero. Returns (best lb over the
+    iterates [R], lb at the start [R]), plus the last iterate's (slopes, multipliers) with ``return_state``."""
     b1, b2 = betas
     R = np.asarray(rows).shape[0]
     relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
@@ -543,11 +545,13 @@ def ascend(net, centre, eps, rows, relax, iters, lr, split_signs=None, betas=(0.
         vh = m2 / (1 - b2 ** (it + 1))
         return x + lr * mh / (np.sqrt(vh) + 1e-8), m1, m2
 
-    alpha = {k: np.repeat(relax[k][0][None, :], R, axis=0) for k in relus}
+    alpha = {k: (np.repeat(relax[k][0][None, :], R, axis=0) if alpha0 is None else
+                 np.clip(np.asarray(alpha0[k], F), 0.0, 1.0)) for k in relus}
     m1 = {k: np.zeros_like(a) for k, a in alpha.items()}
     m2 = {k: np.zeros_like(a) for k, a in alpha.items()}
     sg = split_signs or None
-    beta = None if sg is None else {k: np.zeros((R, len(sg[k])), F) for k in sg}
+    beta = None if sg is None else {k: (np.maximum(np.asarray(beta0[k], F), 0.0) if beta0 is not None and k in beta0
+                                        else np.zeros((R, len(sg[k])), F)) for k in sg}
     bm1 = None if sg is None else {k: np.zeros_like(x) for k, x in beta.items()}
     bm2 = None if sg is None else {k: np.zeros_like(x) for k, x in beta.items()}
     start = best = None
@@ -568,11 +572,13 @@ def ascend(net, centre, eps, rows, relax, iters, lr, split_signs=None, betas=(0.
                 gb = np.where(sg[k][None, :] != 0, out[2][k], 0.0)
                 x, bm1[k], bm2[k] = adam(beta[k], bm1[k], bm2[k], gb, it)
                 beta[k] = np.maximum(x, 0.0)
+    if return_state:
+        return best, start, alpha, beta
     return best, start
 
 
 def alpha_crown(net, centres, eps, C, iters=10, lr=0.1, crown_relus=None, betas=(0.9, 0.999), splits=None,
-                alpha_inter_iters=0, alpha_inter_lr=0.1):
+                alpha_inter_iters=0, alpha_inter_lr=0.1, starts=None, return_state=False):
     """Projected gradient ascent (Adam) on per-row lower slopes of the specification pass, starting
     from the adaptive slopes, keeping each row's best bound [SNNV §1 alpha-CROWN; §3 alpha tensors]
     (``ascend`` per centre). Intermediate bounds are those of `verify` (with ``alpha_inter_iters`` > 0, those of
@@ -580,7 +586,10 @@ def alpha_crown(net, centres, eps, C, iters=10, lr=0.1, crown_relus=None, betas=
 
     With split constraints (relu node -> [B, n] signs) the multipliers beta of the split neurons
     (beta-CROWN, see ``spec_bound_alpha``) are optimised together with the slopes: one per (row, split
-    neuron), starting at 0, the same Adam step, projected to beta >= 0."""
+    neuron), starting at 0, the same Adam step, projected to beta >= 0.
+
+    starts (or None): per centre None or (slopes, multipliers) to start from instead (``ascend``'s alpha0 and
+    beta0); with ``return_state`` the last iterates per centre are returned as a third element."""
     res = verify(net, centres, eps, C, crown_relus=crown_relus, splits=splits, alpha_inter_iters=alpha_inter_iters,
                  alpha_inter_lr=alpha_inter_lr)
     B, R = res.lb.shape
@@ -588,11 +597,17 @@ def alpha_crown(net, centres, eps, C, iters=10, lr=0.1, crown_relus=None, betas=
     relus = [v for v, nd in enumerate(net) if nd.op == "relu"]
     best = np.empty((B, R), F)
     start = np.empty((B, R), F)
+    state = []
     for b in range(B):
         relax = {k: relax_params(res.pre_bounds[k][0][b], res.pre_bounds[k][1][b]) for k in relus}
         rows = C[b if C.shape[0] > 1 else 0]
         sg = None if not splits else {k: np.asarray(splits[k][b]) for k in relus if k in splits}
-        best[b], start[b] = ascend(net, centres[b], eps, rows, relax, iters, lr, sg, betas)
+        a0, b0 = starts[b] if starts is not None and starts[b] is not None else (None, None)
+        best[b], start[b], a_fin, b_fin = ascend(net, centres[b], eps, rows, relax, iters, lr, sg, betas, a0, b0,
+                                                 return_state=True)
+        state.append((a_fin, b_fin))
+    if return_state:
+        return best, start, state
     return best, start
 
 
@@ -624,7 +639,7 @@ class BabResult:
 
 
 def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_relus=None, iters: int = 20,
-        lr: float = 0.1, alpha_inter_iters: int = 0, alpha_inter_lr: float = 0.1) -> BabResult:
+        lr: float = 0.1, alpha_inter_iters: int = 0, alpha_inter_lr: float = 0.1, warm_start: bool = True) -> BabResult:
     """Branch and bound over ReLU splits on top of ``verify`` [SNNV §2.2, §3, §4.3: beta-CROWN with
     branch-and-bound for complete verification; the page names the method only].
 
@@ -632,7 +647,9 @@ def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_rel
     A subdomain's row bound is the larger of ``verify``'s bound and the best bound of ``alpha_crown``
     (``iters`` Adam steps of size ``lr`` on the slopes and on the split multipliers beta); with
     ``alpha_inter_iters`` > 0 both take their intermediate bounds from ``verify``'s intermediate ascent (slopes
-    and the split multipliers of earlier layers).
+    and the split multipliers of earlier layers). With ``warm_start`` (reading; the page names the method only) a
+    child's ascent starts from its parent's last slopes and multipliers (its new split's multiplier from 0); the
+    whole box starts from the adaptive slopes.
     Reading of the search (one plain best-first variant):
       1. the centre is evaluated first, then every row's CROWN minimiser vertex of the whole box
          (``minimiser_attack``); a row < 0 at any of these inputs is a counterexample ("falsified");
@@ -657,6 +674,8 @@ def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_rel
     if ya.size and np.any(ya < 0.0):
         return BabResult("falsified", 0, 0, 0, float(ya.min()))
 
+    saved = {}  # a bounded subdomain's splits, in the order made -> its last slopes and multipliers
+
     def evaluate(domains):
         sp = {k: np.zeros((len(domains), n), np.int8) for k, n in zip(relus, sizes)}
         for i, d in enumerate(domains):
@@ -667,9 +686,14 @@ def bab(net, centre, eps, C, max_domains: int = 1000, batch: int = 16, crown_rel
                      alpha_inter_lr=alpha_inter_lr)
         lb = res.lb
         if iters > 0:
-            lb = np.maximum(lb, alpha_crown(net, cen, eps, C[None], iters=iters, lr=lr, crown_relus=crown_relus,
-                                            splits=sp, alpha_inter_iters=alpha_inter_iters,
-                                            alpha_inter_lr=alpha_inter_lr)[0])
+            keys = [tuple(d.items()) for d in domains]
+            starts = [saved.get(key[:-1]) if warm_start and key else None for key in keys]
+            best, _, state = alpha_crown(net, cen, eps, C[None], iters=iters, lr=lr, crown_relus=crown_relus,
+                                         splits=sp, alpha_inter_iters=alpha_inter_iters, alpha_inter_lr=alpha_inter_lr,
+                                         starts=starts, return_state=True)
+            lb = np.maximum(lb, best)
+            for key, st in zip(keys, state):
+                saved[key] = st
         out = []
         for i in range(len(domains)):
             empty = any(np.any(res.pre_bounds[k][0][i] > res.pre_bounds[k][1][i]) for k in relus)

@@ -432,3 +432,56 @@ def test_beta_gradient_central_differences_on_random_architectures(seed):
         pytest.skip("no split neuron drawn")
     ok, det = _fd_beta(net, c, eps, C[0], relax, a, sp, beta, pairs)
     assert ok, det
+
+
+def _small_props():
+    rng = np.random.default_rng(0)
+    out = []
+    for t in range(24):
+        net = synth.mlp([4, 10, 10, 3], rng)
+        c = rng.random(4).astype(np.float32)
+        y = O.forward(net, c[None].astype(np.float64))[-1][0]
+        C = synth.margin_spec(np.array([int(np.argmax(y))]), 3)[0]
+        for eps in (0.1, 0.2, 0.3):
+            out.append((net, c, float(np.float32(eps)), C))
+    return out
+
+
+def check_warm_start_settles_more():
+    """72 properties of 4-10-10-3 nets, 3 ascent steps per subdomain, 200 subdomains: children that start from
+    their parent's slopes and multipliers settle more properties than children that start afresh (36 against 31
+    verified), and every "verified" of either holds on sampled inputs (sound whatever the start)."""
+    counts = {}
+    for warm in (False, True):
+        n = 0
+        for net, c, eps, C in _small_props():
+            r = O.bab(net, c, eps, C, max_domains=200, batch=8, iters=3, lr=0.1, warm_start=warm)
+            if r.status == "verified":
+                n += 1
+                xs = box_samples(c, eps, 4000, 400, np.random.default_rng(1))
+                if (O.forward(net, xs)[-1] @ C.astype(np.float64).T).min() <= 0.0:
+                    return False, f"warm={warm}: verified a property with a negative sample"
+        counts[warm] = n
+    if counts[True] < counts[False] + 3:
+        return False, f"warm start verified {counts[True]}, cold {counts[False]}"
+    return True, counts
+
+
+def test_warm_start_settles_more():
+    ok, detail = check_warm_start_settles_more()
+    assert ok, detail
+
+
+@pytest.mark.parametrize("old,new", [
+    ("starts = [saved.get(key[:-1]) if warm_start and key else None for key in keys]",
+     "starts = [saved.get(key) if warm_start and key else None for key in keys]"),
+    ("saved[key] = st", "saved[key] = (st[0], None)"),
+])
+def test_warm_start_mutation_is_caught(monkeypatch, old, new):
+    src = textwrap.dedent(inspect.getsource(O.bab))
+    assert src.count(old) == 1
+    ns = {}
+    exec(compile(src.replace(old, new), "<mutant bab>", "exec"), O.__dict__, ns)
+    monkeypatch.setattr(O, "bab", ns["bab"])
+    ok, _ = check_warm_start_settles_more()
+    assert not ok
