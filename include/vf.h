@@ -158,6 +158,14 @@ typedef struct {
      * so not with no_host_sync; not with sound. 0 = off. */
     int alpha_inter_iters;
     float alpha_inter_lr;
+    /* vf_alpha_crown only (NULL = off), [device], each one [B, R, n_v] block per ReLU node v in node order (the
+     * layout of alpha_out): start slopes of the ascent (an entry < 0 starts from the adaptive slope; others are
+     * clamped to [0, 1]), start split multipliers (clamped to >= 0; free neurons' entries do not enter the bound
+     * and keep their start value), and the last iterate's split multipliers (0 for a layer without splits).
+     * Adam's moments always start at zero. */
+    const float* alpha_rows_init;
+    const float* beta_rows_init;
+    float* beta_rows_out;
 } vf_opts;
 
 /* Whole verification step (section 1): IBP, CROWN intermediate bounds, specification
@@ -247,6 +255,10 @@ typedef struct {
     int alpha_inter_iters;  /* as vf_opts.alpha_inter_iters for every bound of the search (0: off): the subdomains'
                                intermediate bounds by alpha-CROWN, with the split multipliers of earlier layers */
     float alpha_inter_lr;
+    int cold_start;         /* 0 (default): a child's ascent starts from its parent's last slopes and multipliers
+                               (its new split's multiplier from 0), kept on the device for every open subdomain
+                               while a pool of at most 1 GiB has room; 1: every ascent starts from the adaptive
+                               slopes and zero multipliers */
 } vf_bab_opts;
 typedef struct {
     int status;             /* VF_BAB_VERIFIED, VF_BAB_FALSIFIED or VF_BAB_UNKNOWN */

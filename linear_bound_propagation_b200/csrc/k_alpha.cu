@@ -135,23 +135,28 @@ __global__ void relax_grad_adam_k(float* __restrict__ G, const float* __restrict
     }
 }
 
-__global__ void zero3_k(float* __restrict__ a, float* __restrict__ b, float* __restrict__ c, long long count) {
+// a = max(init, 0) (or 0 without init), b = c = 0: split multipliers and their Adam moments at the start.
+__global__ void zero3_k(float* __restrict__ a, float* __restrict__ b, float* __restrict__ c, long long count,
+                        const float* __restrict__ init) {
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < count;
          e += (long long)gridDim.x * blockDim.x) {
-        a[e] = 0.f;
+        a[e] = init != nullptr ? fmaxf(init[e], 0.f) : 0.f;
         b[e] = 0.f;
         c[e] = 0.f;
     }
 }
 
 // alpha[m, i] = P[b, i].x (the adaptive start) and zero Adam moments.
+// Start slopes: the relaxation's lower slope, or init[e] clamped to [0, 1] where init is given and init[e] >= 0
+// (a negative entry: no start for that entry). Adam's moments start at zero.
 __global__ void alpha_init_k(float* __restrict__ alpha, float* __restrict__ m1, float* __restrict__ m2, long long M,
-                             int n, const float4* __restrict__ P, PassGeom pg) {
+                             int n, const float4* __restrict__ P, PassGeom pg, const float* __restrict__ init) {
     const long long total = M * n;
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
          e += (long long)gridDim.x * blockDim.x) {
         const long long m = e / n;
-        alpha[e] = P[((pg.pass_m0 + m) / pg.R_pass) * n + (e % n)].x;
+        const float a0 = init != nullptr ? init[e] : -1.f;
+        alpha[e] = a0 >= 0.f ? fminf(a0, 1.f) : P[((pg.pass_m0 + m) / pg.R_pass) * n + (e % n)].x;
         m1[e] = 0.f;
         m2[e] = 0.f;
     }
@@ -199,14 +204,14 @@ cudaError_t launch_relax_grad_adam(float* G, const float* H, long long M, int n,
     return cudaGetLastError();
 }
 
-cudaError_t launch_zero_moments(float* beta, float* m1, float* m2, long long count, cudaStream_t s) {
-    zero3_k<<<grid_for(count, 256), 256, 0, s>>>(beta, m1, m2, count);
+cudaError_t launch_zero_moments(float* beta, float* m1, float* m2, long long count, cudaStream_t s, const float* init) {
+    zero3_k<<<grid_for(count, 256), 256, 0, s>>>(beta, m1, m2, count, init);
     return cudaGetLastError();
 }
 
 cudaError_t launch_alpha_init(float* alpha, float* m1, float* m2, long long M, int n, const float4* P, PassGeom pg,
-                              cudaStream_t s) {
-    alpha_init_k<<<grid_for(M * n, 256), 256, 0, s>>>(alpha, m1, m2, M, n, P, pg);
+                              cudaStream_t s, const float* init) {
+    alpha_init_k<<<grid_for(M * n, 256), 256, 0, s>>>(alpha, m1, m2, M, n, P, pg, init);
     return cudaGetLastError();
 }
 

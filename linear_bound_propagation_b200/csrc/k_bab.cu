@@ -105,7 +105,42 @@ __global__ void minimiser_points_k(const float* __restrict__ centre, const float
     }
 }
 
+// Per-subdomain ascent states (slopes or split multipliers) between a batch, in the alpha_out layout (per ReLU
+// layer q a block [n, R, n_q] at n R gbase_q), and a pool of slots ([R, sum_n] each, layer q at R gbase_q).
+// Gather: batch <- pool[slot[i]], or -1 (no start) where slot[i] < 0. Scatter: pool[slot[i]] <- batch where
+// slot[i] >= 0.
+__global__ void bab_state_k(float* __restrict__ pool, const int* __restrict__ slot, int n, int R, long long sum_n,
+                            const int* __restrict__ meta_n, const int* __restrict__ meta_g, int nl,
+                            float* __restrict__ batch, int scatter) {
+    for (int q = 0; q < nl; ++q) {
+        const long long nq = meta_n[q], gq = meta_g[q];
+        const long long per = (long long)R * nq;
+        const long long total = (long long)n * per;
+        for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+             e += (long long)gridDim.x * blockDim.x) {
+            const long long i = e / per, w = e - i * per;
+            const int sl = slot[i];
+            float* b = batch + (long long)n * R * gq + e;
+            float* pp = pool + (long long)(sl < 0 ? 0 : sl) * R * sum_n + (long long)R * gq + w;
+            if (scatter) {
+                if (sl >= 0) *pp = *b;
+            } else {
+                *b = sl >= 0 ? *pp : -1.f;
+            }
+        }
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_bab_state(float* pool, const int* slot, int n, int R, long long sum_n, const int* meta_n,
+                             const int* meta_g, int nl, float* batch, int scatter, cudaStream_t s) {
+    if (n <= 0 || nl <= 0) return cudaSuccess;
+    long long g = ((long long)n * R * sum_n + 255) / 256;
+    if (g > 148LL * 16) g = 148LL * 16;
+    bab_state_k<<<(unsigned)(g < 1 ? 1 : g), 256, 0, s>>>(pool, slot, n, R, sum_n, meta_n, meta_g, nl, batch, scatter);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_minimiser_points(const float* centre, const float* lam, float eps, long long n, int R, float* x,
                                     cudaStream_t s) {

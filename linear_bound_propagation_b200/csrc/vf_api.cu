@@ -1131,7 +1131,11 @@ int prepare_bounds(vf_net* net, const float* centres, int B, float eps, const vf
         float* best = t2.take<float>((size_t)B * 2 * hp);
         if (!idx || !best) return fail(VF_ERR_WORKSPACE, "workspace too small for intermediate alpha rows");
         LAUNCH(net, launch_unstable_list(bd.Lw[p], bd.Uw[p], B, np, hp, idx, s));
-        TRY(alpha_chain(net, p, centres, B, eps, nullptr, 2 * hp, 0, o, o.alpha_inter_iters, o.alpha_inter_lr, false,
+        vf_opts oi = o;  // the start states and outputs of a specification ascent do not apply here
+        oi.alpha_rows_init = nullptr;
+        oi.beta_rows_init = nullptr;
+        oi.beta_rows_out = nullptr;
+        TRY(alpha_chain(net, p, centres, B, eps, nullptr, 2 * hp, 0, oi, o.alpha_inter_iters, o.alpha_inter_lr, false,
                         nullptr, nullptr, best, nullptr, nullptr, bd, t2, s, nullptr, nullptr, idx));
         LAUNCH(net, launch_intersect_compact(bd.Lw[p], bd.Uw[p], best, idx, B, np, hp, s));
         const float* bias;
@@ -1290,7 +1294,8 @@ int alpha_chain(vf_net* net, int L, const float* centres, int B, float eps, cons
                 al[u] = const_cast<float*>(alpha_in) + aoff[u] + m0 * nu;
             } else {
                 al[u] = A[u];
-                LAUNCH(net, launch_alpha_init(A[u], M1[u], M2[u], Mc, (int)nu, bd.relax[u], pg, s));
+                const float* ai = o.alpha_rows_init ? o.alpha_rows_init + aoff[u] + m0 * nu : nullptr;
+                LAUNCH(net, launch_alpha_init(A[u], M1[u], M2[u], Mc, (int)nu, bd.relax[u], pg, s, ai));
             }
         }
         std::vector<BetaRows> bt(nn);
@@ -1305,7 +1310,8 @@ int alpha_chain(vf_net* net, int L, const float* centres, int B, float eps, cons
                 bt[u].beta = Bt[u];
                 bt[u].m1 = BM1[u];
                 bt[u].m2 = BM2[u];
-                LAUNCH(net, launch_zero_moments(Bt[u], BM1[u], BM2[u], Mc * nu, s));
+                const float* bi = o.beta_rows_init ? o.beta_rows_init + aoff[u] + m0 * nu : nullptr;
+                LAUNCH(net, launch_zero_moments(Bt[u], BM1[u], BM2[u], Mc * nu, s, bi));
             }
         }
         const int evals = grad_mode ? 1 : iters + 1;
@@ -1370,6 +1376,15 @@ int alpha_chain(vf_net* net, int L, const float* centres, int B, float eps, cons
                 const long long nu = net->nodes[u].n;
                 CU(cudaMemcpyAsync(alpha_out + aoff[u] + m0 * nu, A[u], sizeof(float) * Mc * nu,
                                    cudaMemcpyDeviceToDevice, s));
+            }
+        if (!grad_mode && o.beta_rows_out)
+            for (int u : relus) {
+                const long long nu = net->nodes[u].n;
+                if (Bt[u] != nullptr)
+                    CU(cudaMemcpyAsync(o.beta_rows_out + aoff[u] + m0 * nu, Bt[u], sizeof(float) * Mc * nu,
+                                       cudaMemcpyDeviceToDevice, s));
+                else
+                    CU(cudaMemsetAsync(o.beta_rows_out + aoff[u] + m0 * nu, 0, sizeof(float) * Mc * nu, s));
             }
     }
     return VF_OK;
@@ -1466,7 +1481,8 @@ int spec_alpha_graph(vf_net* net, const float* centres, int B, float eps, const 
                 al[u] = const_cast<float*>(alpha_in) + aoff[u] + m0 * nu;
             } else {
                 al[u] = A[u];
-                LAUNCH(net, launch_alpha_init(A[u], M1[u], M2[u], Mc, (int)nu, bd.relax[u], pg, s));
+                const float* ai = o.alpha_rows_init ? o.alpha_rows_init + aoff[u] + m0 * nu : nullptr;
+                LAUNCH(net, launch_alpha_init(A[u], M1[u], M2[u], Mc, (int)nu, bd.relax[u], pg, s, ai));
             }
         }
         std::vector<BetaRows> bt(nn);
@@ -1481,7 +1497,8 @@ int spec_alpha_graph(vf_net* net, const float* centres, int B, float eps, const 
                 bt[u].beta = Bt[u];
                 bt[u].m1 = BM1[u];
                 bt[u].m2 = BM2[u];
-                LAUNCH(net, launch_zero_moments(Bt[u], BM1[u], BM2[u], Mc * nu, s));
+                const float* bi = o.beta_rows_init ? o.beta_rows_init + aoff[u] + m0 * nu : nullptr;
+                LAUNCH(net, launch_zero_moments(Bt[u], BM1[u], BM2[u], Mc * nu, s, bi));
             }
         }
         const int evals = grad_mode ? 1 : iters + 1;
@@ -1579,6 +1596,15 @@ int spec_alpha_graph(vf_net* net, const float* centres, int B, float eps, const 
                 const long long nu = net->nodes[u].n;
                 CU(cudaMemcpyAsync(alpha_out + aoff[u] + m0 * nu, A[u], sizeof(float) * Mc * nu,
                                    cudaMemcpyDeviceToDevice, s));
+            }
+        if (!grad_mode && o.beta_rows_out)
+            for (int u : relus) {
+                const long long nu = net->nodes[u].n;
+                if (Bt[u] != nullptr)
+                    CU(cudaMemcpyAsync(o.beta_rows_out + aoff[u] + m0 * nu, Bt[u], sizeof(float) * Mc * nu,
+                                       cudaMemcpyDeviceToDevice, s));
+                else
+                    CU(cudaMemsetAsync(o.beta_rows_out + aoff[u] + m0 * nu, 0, sizeof(float) * Mc * nu, s));
             }
     }
     return VF_OK;

@@ -13,6 +13,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <utility>
 #include <vector>
 
@@ -88,6 +89,15 @@ struct DeviceBound {
     std::vector<signed char> hsplit;
     std::vector<BabPick> hpick;
     long long traced = 0;  // entries of opts->trace written so far
+    // warm starts: each bounded subdomain's last slopes and multipliers in a pool slot, found by its split list
+    bool warm = false;
+    int pool_cap = 0;
+    float *pool_a = nullptr, *pool_b = nullptr;  // [pool_cap, R, sum_n]
+    float *init_a, *init_b, *out_a, *out_b;      // [D, R, sum_n] in the alpha_out layout of a batch
+    int* dslots = nullptr;                       // [2 D]: parents' slots, then the children's
+    std::map<std::vector<int>, int> slot_of;
+    std::vector<int> free_slots;
+    int next_slot = 0;
 };
 
 // vf_bab_bound_fn on the device: one vf_verify_batch (bounds and pre-activation bounds of all n subdomains
@@ -127,8 +137,51 @@ int device_bound(void* user, int n, const int* split_offset, const int* split_co
         oa.split = sp.data();
         oa.alpha_inter_iters = d.opts->alpha_inter_iters;
         oa.alpha_inter_lr = d.opts->alpha_inter_lr;
+        std::vector<int> slots(2 * (size_t)n, -1), keyv;
+        std::vector<std::vector<int>> keys(n);
+        if (d.warm) {
+            // a child's splits are its parent's followed by one more: the parent's key drops the last entry
+            for (int i = 0; i < n; ++i) {
+                for (int k = 0; k < split_count[i]; ++k)
+                    keys[i].push_back(2 * split_neuron[split_offset[i] + k] + (split_sign[split_offset[i] + k] > 0));
+                if (!keys[i].empty()) {
+                    keyv.assign(keys[i].begin(), keys[i].end() - 1);
+                    auto it = d.slot_of.find(keyv);
+                    if (it != d.slot_of.end()) slots[i] = it->second;
+                }
+                if (!d.free_slots.empty()) {
+                    slots[n + i] = d.free_slots.back();
+                    d.free_slots.pop_back();
+                } else if (d.next_slot < d.pool_cap) {
+                    slots[n + i] = d.next_slot++;
+                }
+            }
+            BAB_CU(cudaMemcpyAsync(d.dslots, slots.data(), sizeof(int) * 2 * n, cudaMemcpyHostToDevice, s));
+            BAB_CU(vf::launch_bab_state(d.pool_a, d.dslots, n, d.R, d.sum_n, d.meta_n, d.meta_g, nl, d.init_a, 0, s));
+            BAB_CU(vf::launch_bab_state(d.pool_b, d.dslots, n, d.R, d.sum_n, d.meta_n, d.meta_g, nl, d.init_b, 0, s));
+            oa.alpha_rows_init = d.init_a;
+            oa.beta_rows_init = d.init_b;
+            oa.beta_rows_out = d.out_b;
+        }
         BAB_TRY(vf_alpha_crown(d.net, d.cen, n, d.eps, d.C, d.R, 0, &oa, d.opts->alpha_iters, d.opts->lr, d.lba, nullptr,
-                               nullptr, d.stream));
+                               d.warm ? d.out_a : nullptr, d.stream));
+        if (d.warm) {
+            BAB_CU(vf::launch_bab_state(d.pool_a, d.dslots + n, n, d.R, d.sum_n, d.meta_n, d.meta_g, nl, d.out_a, 1, s));
+            BAB_CU(vf::launch_bab_state(d.pool_b, d.dslots + n, n, d.R, d.sum_n, d.meta_n, d.meta_g, nl, d.out_b, 1, s));
+            // both children of a parent are bounded in the same round: its slot is free again (the copies above
+            // are ordered before any later gather or scatter on the stream)
+            for (int i = 0; i < n; ++i) {
+                if (!keys[i].empty()) {
+                    keyv.assign(keys[i].begin(), keys[i].end() - 1);
+                    auto it = d.slot_of.find(keyv);
+                    if (it != d.slot_of.end()) {
+                        d.free_slots.push_back(it->second);
+                        d.slot_of.erase(it);
+                    }
+                }
+                if (slots[n + i] >= 0) d.slot_of[keys[i]] = slots[n + i];
+            }
+        }
     }
     BAB_CU(vf::launch_bab_pick(d.plb, d.pub, n, d.meta_off, d.meta_n, d.meta_g, nl, d.lbv,
                                d.opts->alpha_iters > 0 ? d.lba : nullptr, d.R, d.pick, s));
@@ -295,6 +348,27 @@ extern "C" int vf_bab_verify(vf_net* net, const float* centre, float eps, const 
     db.meta_n = meta_n.get<int>();
     db.meta_g = meta_g.get<int>();
     db.hpick.resize(D);
+    DeviceBuffer pool_a, pool_b, init_a, init_b, out_a, out_b, dslots;
+    db.warm = opts->alpha_iters > 0 && !opts->cold_start && sum_n > 0;
+    if (db.warm) {
+        const size_t per = (size_t)R * sum_n;  // floats of one subdomain's slopes (and of its multipliers)
+        const size_t cap_mem = (size_t(1) << 30) / (2 * per * sizeof(float));
+        db.pool_cap = (int)std::min<size_t>((size_t)opts->max_domains, cap_mem);
+        BAB_CU(cudaMalloc(&pool_a.p, sizeof(float) * per * std::max(db.pool_cap, 1)));
+        BAB_CU(cudaMalloc(&pool_b.p, sizeof(float) * per * std::max(db.pool_cap, 1)));
+        BAB_CU(cudaMalloc(&init_a.p, sizeof(float) * per * D));
+        BAB_CU(cudaMalloc(&init_b.p, sizeof(float) * per * D));
+        BAB_CU(cudaMalloc(&out_a.p, sizeof(float) * per * D));
+        BAB_CU(cudaMalloc(&out_b.p, sizeof(float) * per * D));
+        BAB_CU(cudaMalloc(&dslots.p, sizeof(int) * 2 * D));
+        db.pool_a = pool_a.get<float>();
+        db.pool_b = pool_b.get<float>();
+        db.init_a = init_a.get<float>();
+        db.init_b = init_b.get<float>();
+        db.out_a = out_a.get<float>();
+        db.out_b = out_b.get<float>();
+        db.dslots = dslots.get<int>();
+    }
     return vf_bab_search(device_bound, &db, opts->max_domains, opts->batch, result);
 }
 

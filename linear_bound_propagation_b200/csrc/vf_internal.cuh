@@ -264,9 +264,12 @@ cudaError_t launch_concretize_grad(const float* lam, long long M, int n0, PassGe
 cudaError_t launch_relax_grad_adam(float* G, const float* H, long long M, int n, const float4* P, PassGeom pg,
                                    float* alpha, float* grad_out, float* m1, float* m2, int adam_step, float lr,
                                    cudaStream_t s, BetaRows bt = BetaRows{});
-cudaError_t launch_zero_moments(float* beta, float* m1, float* m2, long long count, cudaStream_t s);
+// Split multipliers max(init, 0) (0 without init) and zero Adam moments.
+cudaError_t launch_zero_moments(float* beta, float* m1, float* m2, long long count, cudaStream_t s,
+                                const float* init = nullptr);
+// Start slopes: P's lower slope per (centre, neuron), or init clamped to [0, 1] where init >= 0; zero moments.
 cudaError_t launch_alpha_init(float* alpha, float* m1, float* m2, long long M, int n, const float4* P, PassGeom pg,
-                              cudaStream_t s);
+                              cudaStream_t s, const float* init = nullptr);
 cudaError_t launch_best_update(float* best, const float* cur, long long M, int first, cudaStream_t s);
 // P[i] = {1, 1, 0, 0}: a relaxation table that passes rows through unchanged (slopes 1, no intercept, no
 // bias), so rows whose slopes were applied already can take the tensor-core contraction.
@@ -307,6 +310,11 @@ cudaError_t launch_bab_pick(const float* pre_lb, const float* pre_ub, int D, con
                             cudaStream_t s);
 // dst[d, :] = src[:] for d < D (n floats per row).
 cudaError_t launch_repeat_row(const float* src, long long n, int D, float* dst, cudaStream_t s);
+// Branch-and-bound ascent states between a batch (alpha_out layout: per ReLU layer q a block [n, R, n_q] at
+// n R gbase_q) and a pool of [R, sum_n] slots: scatter = 0 gathers batch <- pool[slot[i]] (-1 where slot[i] < 0),
+// scatter = 1 writes pool[slot[i]] <- batch where slot[i] >= 0. meta_n / meta_g [device]: per layer n_q, gbase_q.
+cudaError_t launch_bab_state(float* pool, const int* slot, int n, int R, long long sum_n, const int* meta_n,
+                             const int* meta_g, int nl, float* batch, int scatter, cudaStream_t s);
 // Row r's CROWN minimiser vertex of the box centre +/- eps: x[r, :] = centre - eps * sign(lam[r, :]), each
 // coordinate rounded towards the centre so it stays inside the box. centre [n], lam and x [R, n], device.
 cudaError_t launch_minimiser_points(const float* centre, const float* lam, float eps, long long n, int R, float* x,

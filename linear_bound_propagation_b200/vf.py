@@ -49,14 +49,16 @@ class Opts(ctypes.Structure):
                 ("both_sides", ctypes.c_int), ("skip_finite_check", ctypes.c_int),
                 ("pre_lb", ctypes.c_void_p), ("pre_ub", ctypes.c_void_p), ("no_host_sync", ctypes.c_int),
                 ("split", ctypes.POINTER(ctypes.c_void_p)), ("sound", ctypes.c_int),
-                ("alpha_inter_iters", ctypes.c_int), ("alpha_inter_lr", ctypes.c_float)]
+                ("alpha_inter_iters", ctypes.c_int), ("alpha_inter_lr", ctypes.c_float),
+                ("alpha_rows_init", ctypes.c_void_p), ("beta_rows_init", ctypes.c_void_p),
+                ("beta_rows_out", ctypes.c_void_p)]
 
 
 class BabOpts(ctypes.Structure):
     _fields_ = [("max_domains", ctypes.c_int), ("batch", ctypes.c_int), ("alpha_iters", ctypes.c_int),
                 ("lr", ctypes.c_float), ("relu_crown", ctypes.POINTER(ctypes.c_int)),
                 ("trace", ctypes.POINTER(ctypes.c_int)), ("trace_cap", ctypes.c_int),
-                ("alpha_inter_iters", ctypes.c_int), ("alpha_inter_lr", ctypes.c_float)]
+                ("alpha_inter_iters", ctypes.c_int), ("alpha_inter_lr", ctypes.c_float), ("cold_start", ctypes.c_int)]
 
 
 class BabResult(ctypes.Structure):
@@ -293,19 +295,28 @@ class Net:
 
     def alpha_crown(self, centres: torch.Tensor, eps: float, C: torch.Tensor, iters: int = 20, lr: float = 0.1,
                     crown_relus=None, want_alpha: bool = False, stream=None, splits=None, alpha_inter_iters: int = 0,
-                    alpha_inter_lr: float = 0.1):
-        """vf_alpha_crown: returns dict(lb=best bound [B, R], lb_start=[B, R], alpha=final slopes or None).
-        With splits (see verify) the split multipliers beta are optimised with the slopes; alpha_inter_iters > 0
-        optimises the intermediate bounds first (vf_opts)."""
+                    alpha_inter_lr: float = 0.1, alpha_init: Optional[torch.Tensor] = None,
+                    beta_init: Optional[torch.Tensor] = None, want_beta: bool = False):
+        """vf_alpha_crown: returns dict(lb=best bound [B, R], lb_start=[B, R], alpha=final slopes or None,
+        beta=final split multipliers or None). With splits (see verify) the split multipliers beta are optimised
+        with the slopes; alpha_inter_iters > 0 optimises the intermediate bounds first; alpha_init / beta_init
+        (alpha_size(B, R) floats, device) are start states (a negative slope entry: the adaptive slope)."""
         B, R = centres.shape[0], C.shape[1]
         bstride = 0 if C.shape[0] == 1 else R * C.shape[2]
         lb = torch.empty(B, R, device=centres.device)
         lb0 = torch.empty(B, R, device=centres.device)
         al = torch.empty(self.alpha_size(B, R), device=centres.device) if want_alpha else None
+        be = torch.empty(self.alpha_size(B, R), device=centres.device) if want_beta else None
         o, keep = self._opts(crown_relus, splits, alpha_inter_iters, alpha_inter_lr)
+        for t in (alpha_init, beta_init):
+            if t is not None:
+                assert t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and t.numel() == self.alpha_size(B, R)
+        o.alpha_rows_init = alpha_init.data_ptr() if alpha_init is not None else None
+        o.beta_rows_init = beta_init.data_ptr() if beta_init is not None else None
+        o.beta_rows_out = be.data_ptr() if be is not None else None
         _check(lib().vf_alpha_crown(self.h, _ptr(centres), B, float(eps), _ptr(C), R, bstride, ctypes.byref(o), iters,
                                     float(lr), _ptr(lb), _ptr(lb0), _ptr(al), _stream_ptr(stream)))
-        return {"lb": lb, "lb_start": lb0, "alpha": al}
+        return {"lb": lb, "lb_start": lb0, "alpha": al, "beta": be}
 
     def alpha_grad(self, centres: torch.Tensor, eps: float, C: torch.Tensor, alpha: torch.Tensor, crown_relus=None,
                    stream=None):
@@ -335,13 +346,15 @@ class Net:
 
     def bab(self, centre: torch.Tensor, eps: float, C: torch.Tensor, max_domains: int = 1000, batch: int = 16,
             alpha_iters: int = 20, lr: float = 0.1, crown_relus=None, stream=None, trace: bool = False,
-            alpha_inter_iters: int = 0, alpha_inter_lr: float = 0.1):
+            alpha_inter_iters: int = 0, alpha_inter_lr: float = 0.1, warm_start: bool = True):
         """vf_bab_verify on one box: centre [n0], C [R, n_L] (device). Returns dict(status, domains, rounds,
         max_depth, lb), plus, with trace, the branching neuron of every bounded subdomain in the order bounded
         (search-wide index, -1 if none). alpha_inter_iters > 0: intermediate bounds of every subdomain by
-        alpha-CROWN with the split multipliers (vf_opts)."""
+        alpha-CROWN with the split multipliers (vf_opts). warm_start: children start their ascent from the
+        parent's last slopes and multipliers."""
         o = BabOpts(max_domains=max_domains, batch=batch, alpha_iters=alpha_iters, lr=float(lr),
-                    alpha_inter_iters=int(alpha_inter_iters), alpha_inter_lr=float(alpha_inter_lr))
+                    alpha_inter_iters=int(alpha_inter_iters), alpha_inter_lr=float(alpha_inter_lr),
+                    cold_start=0 if warm_start else 1)
         tbuf = None
         if trace:
             tbuf = (ctypes.c_int * max_domains)()

@@ -97,7 +97,7 @@ def test_alpha_crown_improves_soundly_and_tracks_oracle(config, B):
     assert sound_on_samples(net, w.centres[:4], w.eps, w.C[:4] if w.C.shape[0] > 1 else w.C, lb[:4], None, n=2000)
 
 
-def _assert_off_rows_at_kinks(net, centres, eps, C, lb, best, ok, iters, splits=None):
+def _assert_off_rows_at_kinks(net, centres, eps, C, lb, best, ok, iters, splits=None, starts=None):
     """Every row of a centre without an adaptive-slope near-tie matches the oracle's optimised bound, or
     sits at a kink of the optimisation (kink_sensitive_rows)."""
     off = [(b, r) for b in range(lb.shape[0]) if ok[b] for r in range(lb.shape[1])
@@ -112,7 +112,9 @@ def _assert_off_rows_at_kinks(net, centres, eps, C, lb, best, ok, iters, splits=
     for b, rs in by_b.items():
         Cb = C[b:b + 1] if C.shape[0] > 1 else C
         sp = None if splits is None else {k: v[b:b + 1] for k, v in splits.items()}
-        kink = kink_sensitive_rows(lambda c, e: O.alpha_crown(net, c, e, Cb, iters=iters, lr=0.1, splits=sp)[0],
+        st = None if starts is None else [starts[b]]
+        kink = kink_sensitive_rows(lambda c, e: O.alpha_crown(net, c, e, Cb, iters=iters, lr=0.1, splits=sp,
+                                                              starts=st)[0],
                                    centres[b:b + 1], eps, [(0, r) for r in rs])
         bad += [(b, r) for r, k in zip(rs, kink) if not k]
     assert not bad, f"rows off the oracle's trajectory without a kink: {bad[:8]} (of {len(off)} off)"

@@ -250,3 +250,99 @@ def test_bab_with_intermediate_alpha():
             gained.append((name, r["status"]))
     assert agree >= 0.9 * total, f"{agree} of {total} statuses agree"
     assert gained and all(s == "verified" for _, s in gained), gained
+
+
+def _starts(g, net, B, R, rng, sp):
+    """Seeded start slopes in [0, 1] with a fifth of the entries negative (no start), and start multipliers, in
+    the alpha_out layout; plus the same as the oracle's per-centre (slopes, multipliers) dicts."""
+    relus = g.relu_ids
+    a = rng.random(g.alpha_size(B, R)).astype(np.float32)
+    a[rng.random(a.size) < 0.2] = -1.0
+    bt = (rng.random(g.alpha_size(B, R)) * 0.5).astype(np.float32)
+    per_centre, off = [({}, {}) for _ in range(B)], 0
+    for k in relus:
+        n = g.sizes[k]
+        blk_a = a[off: off + B * R * n].reshape(B, R, n)
+        blk_b = bt[off: off + B * R * n].reshape(B, R, n)
+        for b in range(B):
+            per_centre[b][0][k] = blk_a[b].astype(np.float64)
+            if k in sp:
+                per_centre[b][1][k] = blk_b[b].astype(np.float64)
+        off += B * R * n
+    return a, bt, per_centre
+
+
+def test_alpha_crown_start_states_match_oracle():
+    """vf_alpha_crown from given start slopes and multipliers (the warm start of branch and bound) against the
+    oracle's ascent from the same start: at zero steps the bound element-wise (a negative slope entry starts from
+    the adaptive slope); after four steps every row, except at kinks of the ascent; the returned last multipliers
+    are >= 0, keep their start value on free neurons (their gradient is zero) and are zero on layers without
+    splits."""
+    net, centres, C, eps = _case("mlp", B=4, seed=3)
+    rng = np.random.default_rng(17)
+    sp = _signs(net, centres, eps, 0.3, rng)
+    g = vf.Net(net)
+    B, R = centres.shape[0], C.shape[1]
+    a, bt, starts = _starts(g, net, B, R, rng, sp)
+    oracle_starts = []
+    res = O.verify(net, centres, eps, C, splits=sp)
+    for b in range(B):
+        relax = {k: O.relax_params(res.pre_bounds[k][0][b], res.pre_bounds[k][1][b]) for k in g.relu_ids}
+        # the oracle takes a slope start per entry: a negative device entry means the relaxation's slope
+        a0 = {k: np.where(v < 0, np.repeat(relax[k][0][None, :], R, axis=0), v) for k, v in starts[b][0].items()}
+        oracle_starts.append((a0, starts[b][1]))
+    spd = {k: _dev(v) for k, v in sp.items()}
+    for iters in (0, 4):
+        out = g.alpha_crown(_dev(centres), eps, _dev(C), iters=iters, lr=0.1, splits=spd, alpha_init=_dev(a),
+                            beta_init=_dev(bt), want_beta=True)
+        torch.cuda.synchronize()
+        g.check()
+        lb = out["lb"].cpu().numpy()
+        best, start = O.alpha_crown(net, centres, eps, C, iters=iters, lr=0.1, splits=sp, starts=oracle_starts)
+        ok = ~ambiguous_centres(res, net)
+        assert ok.sum() >= 2
+        assert _viol(out["lb_start"].cpu().numpy()[ok], start[ok]).max() <= 1.0, iters
+        if iters == 0:
+            assert _viol(lb[ok], best[ok]).max() <= 1.0
+        else:
+            _assert_off_rows_at_kinks(net, centres, eps, C, lb, best, ok, iters=iters, splits=sp,
+                                      starts=oracle_starts)
+        beta = out["beta"].cpu().numpy()
+        assert np.all(beta >= 0.0)
+        off = 0
+        for k in g.relu_ids:
+            n = g.sizes[k]
+            blk = beta[off: off + B * R * n].reshape(B, R, n)
+            if k in sp:
+                free = np.broadcast_to((sp[k] == 0)[:, None, :], blk.shape)
+                start_b = np.maximum(bt[off: off + B * R * n].reshape(B, R, n), 0.0)
+                assert np.array_equal(blk[free], start_b[free]), k
+            else:
+                assert np.all(blk == 0.0), k
+            off += B * R * n
+
+
+def test_bab_warm_start_on_device():
+    """The 72 small properties with 3 ascent steps per subdomain: children that start from their parent's
+    slopes and multipliers settle more properties on the device than children that start afresh (as in the
+    oracle: 36 against 31), the device's statuses agree with the oracle's warm search on at least 90% of them,
+    and every "verified" holds on sampled inputs."""
+    from tests.test_gpu_edge_cases import _bab_problems
+    counts = {True: 0, False: 0}
+    agree = total = 0
+    for name, net, c, eps, C in _bab_problems():
+        g = vf.Net(net)
+        for warm in (True, False):
+            r = g.bab(_dev(c), eps, _dev(C), max_domains=200, batch=8, alpha_iters=3, lr=0.1, warm_start=warm)
+            torch.cuda.synchronize()
+            g.check()
+            if r["status"] == "verified":
+                counts[warm] += 1
+                xs = c + eps * (2 * np.random.default_rng(3).random((20000, c.size)) - 1)
+                assert (O.forward(net, xs)[-1] @ C.astype(np.float64).T).min() > 0.0, (name, warm)
+            if warm:
+                o = O.bab(net, c, eps, C, max_domains=200, batch=8, iters=3, lr=0.1)
+                total += 1
+                agree += r["status"] == o.status
+    assert counts[True] >= counts[False] + 3, counts
+    assert agree >= 0.9 * total, f"{agree} of {total}"
