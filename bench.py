@@ -227,14 +227,15 @@ def roofline(kstats, step_total_ms, n_sms, workload=None, step_ms=None):
     avg_ms = k_ms / max(n_k, 1)
     achieved = (k_flops / max(n_k, 1)) / (avg_ms / 1000.0) / 1e12 if n_k else 0.0
     sm_mhz = float(p.get("sm_max_mhz", 1965.0))
-    if kind in (1, 5):
+    if kind in (1, 5, 7):
         sustained = step_ms is not None and step_ms >= 100.0 and "bf16_tflops_sustained" in p
         bf16 = float(p["bf16_tflops_sustained"] if sustained else p["bf16_tflops"])
         tf32 = bf16 * TF32_OVER_BF16
         peak = tf32 / 3.0
         bound = "tensor"
         name = {1: "dense_back_tc (tcgen05 kind::tf32, 3xTF32 CROWN Lambda.W contraction)",
-                5: "conv_back_tc (tcgen05 kind::tf32 implicit GEMM, 3xTF32 transposed convolution)"}[kind]
+                5: "conv_back_tc (tcgen05 kind::tf32 implicit GEMM, 3xTF32 transposed convolution)",
+                7: "conv_back_tc on a 3-channel stem (input channels padded to 16)"}[kind]
         psrc = (f"tf32 = {src} bf16 {'sustained' if sustained else 'burst'} {bf16:.0f} TFLOP/s x nominal "
                 f"1.1/2.25 = {tf32:.0f}; 3xTF32 effective = tf32 / 3")
     else:
@@ -387,7 +388,7 @@ def measure_workload(args, ctx, cfg, eps, steps, warmup, headline, legs=None):
     torch.cuda.synchronize()
     clocks = stop_clocks(clk)
     launches = net.launch_count() - launches0
-    kstats = {k: net.profile_read(kind=k, reset=False) for k in (1, 2, 3, 4, 5)}
+    kstats = {k: net.profile_read(kind=k, reset=False) for k in (1, 2, 3, 4, 5, 7)}
     fwd = net.profile_read(kind=vf.VF_KERNEL_DENSE_FWD_TC, reset=False)
     net.profile_read(reset=True)
     net.profile(False)
@@ -398,7 +399,12 @@ def measure_workload(args, ctx, cfg, eps, steps, warmup, headline, legs=None):
     verified = int(out["verified"].sum().item())
     roof = roofline(kstats, total_ms, torch.cuda.get_device_properties(dev).multi_processor_count,
                     w.name if (args.centres is None or not headline) else None, total_ms / steps)
-    if fwd[0]:  # IBP forward products on the tensor cores (not the dominant kernel; reported beside it)
+    pad = kstats.get(7, (0, 0.0, 0.0))
+    if pad[0] and roof.get("kernel", "").startswith("conv_back_tc (") and pad[1] > 0:
+        # the stem on the tensor cores (its useful flops are 3/16 of the MMA work): reported beside the others
+        roof["stem_tc"] = {"launches": pad[0], "ms": pad[1], "share_of_step": pad[1] / total_ms,
+                           "achieved_tflops": pad[2] / (pad[1] / 1000.0) / 1e12}
+    if fwd[0]:  # the alpha ascent's forward products on the tensor cores (reported beside the dominant kernel)
         roof["forward_products_tc"] = {"launches": fwd[0], "ms": fwd[1], "share_of_step": fwd[1] / total_ms,
                                        "achieved_tflops": fwd[2] / (fwd[1] / 1000.0) / 1e12 if fwd[1] else None}
 

@@ -308,8 +308,10 @@ enum {
     VF_KERNEL_CONV = 3,
     VF_KERNEL_CONV_WIN = 4,
     VF_KERNEL_CONV_TC = 5, /* tensor-core implicit GEMM, whole maps and windows; flops as for windows */
-    VF_KERNEL_DENSE_FWD_TC = 6 /* forward products on the tensor cores: the alpha gradient's G W^T + b (and with
-                                  VF_FWD_TC=ibp at vf_net_create the IBP W c + b, |W| r); 2*M*K*N flops */
+    VF_KERNEL_DENSE_FWD_TC = 6, /* forward products on the tensor cores: the alpha gradient's G W^T + b (and with
+                                   VF_FWD_TC=ibp at vf_net_create the IBP W c + b, |W| r); 2*M*K*N flops */
+    VF_KERNEL_CONV_TC_PAD = 7  /* the tensor-core convolution on an input of fewer than 16 channels (padded to 16);
+                                  flops of the real channels */
 };
 int vf_profile_enable(vf_net* net, int enable);
 int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms, double* flops, int reset);

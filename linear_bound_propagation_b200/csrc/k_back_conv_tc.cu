@@ -78,7 +78,8 @@ struct ConvTcParams {
     PassGeom pg;
     PassStart ps;
     Win wa, wd;
-    int C, Np, nchunk;        // input channels (N), 2C, output-channel chunks of 8 (K)
+    int C, Np, nchunk;        // input channels padded to a multiple of 16 (N), 2C, output-channel chunks of 8 (K)
+    int Cr;                   // input channels of the map (C_in; the channels from Cr to C carry zero weights)
     int G, S, P, gy, gx;      // rows per group, slab lines, pitch, gap lines / columns
     int npos_img, T, NPOS;    // flat positions per row, M tiles per class, positions per stage buffer
     int ncls, nact;           // s*s classes, classes with at least one tap
@@ -113,27 +114,31 @@ __device__ __forceinline__ void epi_block16(const ConvTcParams& p, bool act, boo
         tmem_wait_ld();
     }
     if (!wr) return;
+    const int nc = min(16, p.Cr - cb);  // channels of the map in this block (padding channels are not written)
     float v[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) v[j] = act ? __uint_as_float(vh[j]) + __uint_as_float(vl[j]) : 0.f;
-    if (conc) {  // all sixteen centre loads in flight at once
+    if (conc) {  // all the block's centre loads in flight at once
         float cv[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) cv[j] = on ? __ldg(&crow[(long long)(cb + j) * S_in]) : 0.f;
+        for (int j = 0; j < 16; ++j) cv[j] = (on && j < nc) ? __ldg(&crow[(long long)(cb + j) * S_in]) : 0.f;
         float acc = 0.f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc += fmaf(v[j], cv[j], -p.eps * fabsf(v[j]));
+        for (int j = 0; j < 16; ++j)
+            if (j < nc) acc += fmaf(v[j], cv[j], -p.eps * fabsf(v[j]));
         *cpart += acc;
-    } else if (p.out_mode == OUT_ACCUM) {  // read all sixteen old values before the first store
+    } else if (p.out_mode == OUT_ACCUM) {  // read all the block's old values before the first store
         if (!on) return;
         float old[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) old[j] = orow[(long long)(cb + j) * wdp];
+        for (int j = 0; j < 16; ++j) old[j] = j < nc ? orow[(long long)(cb + j) * wdp] : 0.f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) orow[(long long)(cb + j) * wdp] = old[j] + v[j];
+        for (int j = 0; j < 16; ++j)
+            if (j < nc) orow[(long long)(cb + j) * wdp] = old[j] + v[j];
     } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) orow[(long long)(cb + j) * wdp] = on ? v[j] : 0.f;
+        for (int j = 0; j < 16; ++j)
+            if (j < nc) orow[(long long)(cb + j) * wdp] = on ? v[j] : 0.f;
     }
 }
 
@@ -450,7 +455,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) conv_back_tc(const __grid_cons
                     // off-map entries
                     const bool wr = on || (in_wd && p.out_mode == OUT_STORE);
                     float* orow = (valid && !conc) ? p.out + m * p.ld_out + (long long)dy * p.wd.hw + dx : nullptr;
-                    const float* crow = (valid && conc) ? p.centres + rg.b * (long long)p.C * S_in + (long long)Y * p.g.w + X
+                    const float* crow = (valid && conc) ? p.centres + rg.b * (long long)p.Cr * S_in + (long long)Y * p.g.w + X
                                                         : nullptr;
                     float cpart = 0.f;
                     const uint32_t col0 = lane_base + acc0 + (uint32_t)((k * p.T + t) * p.Np);
@@ -499,12 +504,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) conv_back_tc(const __grid_cons
 // ---------------------------------------------------------------------------------------- host side
 
 int conv_tc_wtc_floats(const ConvGeom& g) {
-    const int nchunk = (g.co + 7) / 8;
-    return g.k * g.k * nchunk * 2 * (2 * g.ci) * 4;
+    const int nchunk = (g.co + 7) / 8, C = (g.ci + 15) / 16 * 16;
+    return g.k * g.k * nchunk * 2 * (2 * C) * 4;
 }
 
 void conv_tc_pack_weights(const ConvGeom& g, const float* W, float* out) {
-    const int C = g.ci, Np = 2 * C, nchunk = (g.co + 7) / 8;
+    const int C = (g.ci + 15) / 16 * 16, Np = 2 * C, nchunk = (g.co + 7) / 8;
     for (int p = 0; p < g.k; ++p)
         for (int q = 0; q < g.k; ++q)
             for (int c = 0; c < nchunk; ++c)
@@ -513,7 +518,7 @@ void conv_tc_pack_weights(const ConvGeom& g, const float* W, float* out) {
                         for (int j = 0; j < 4; ++j) {
                             const int co = 8 * c + 4 * hk + j, ci = n % C;
                             float w = 0.f;
-                            if (co < g.co) w = W[(((size_t)co * g.ci + ci) * g.k + p) * g.k + q];
+                            if (co < g.co && ci < g.ci) w = W[(((size_t)co * g.ci + ci) * g.k + p) * g.k + q];
                             uint32_t bits;
                             std::memcpy(&bits, &w, 4);
                             bits &= 0xFFFFE000u;
@@ -524,7 +529,12 @@ void conv_tc_pack_weights(const ConvGeom& g, const float* W, float* out) {
 }
 
 bool conv_tc_weights_supported(const ConvGeom& g) {
-    return g.ci % 16 == 0 && g.ci <= 128 && g.k <= 8 && g.stride >= 1 && g.stride <= 2 && g.k * g.k <= MAX_TAPS;
+    // input channels a multiple of 16, or fewer than 16 at stride 1 (padded to 16 with zero weights: an MMA costs
+    // the same at N = 2 x 16 as at N = 2 x 3, so a 3-channel 3x3 stem runs like a 16-channel convolution, faster than
+    // the FFMA kernels on the residual network; the 4x4 stride-2 stem of the CNN measured slower than its windowed
+    // FFMA kernel and stays there)
+    return (g.ci % 16 == 0 || (g.ci < 16 && g.stride == 1)) && g.ci <= 128 && g.k <= 8 && g.stride >= 1 &&
+           g.stride <= 2 && g.k * g.k <= MAX_TAPS;
 }
 
 namespace {
@@ -533,8 +543,9 @@ bool plan(const ConvGeom& g, const Win& wa, const Win& wd, int out_mode, ConvTcP
     if (!conv_tc_weights_supported(g)) return false;
     ConvTcParams& p = *pp;
     const int s = g.stride, KS = (g.k + s - 1) / s;
-    p.C = g.ci;
-    p.Np = 2 * g.ci;
+    p.C = (g.ci + 15) / 16 * 16;
+    p.Cr = g.ci;
+    p.Np = 2 * p.C;
     p.nchunk = (g.co + 7) / 8;
     p.gy = p.gx = KS - 1;
     p.S = wa.hh + p.gy;

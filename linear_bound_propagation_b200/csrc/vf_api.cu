@@ -121,9 +121,9 @@ struct vf_net {
         double flops;
     };
     std::vector<Timed> ev_used;
-    double prof_flops[7] = {0, 0, 0, 0, 0, 0, 0};
-    long long prof_launches[7] = {0, 0, 0, 0, 0, 0, 0};
-    double prof_ms[7] = {0, 0, 0, 0, 0, 0, 0};
+    double prof_flops[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    long long prof_launches[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    double prof_ms[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 };
 
 namespace {
@@ -587,8 +587,8 @@ struct Walker {
                                                             out, ld, cst, centres, eps, net->d_err, net->num_sms, s));
                         const Win nat = win_back(wa_tc, g);
                         const double pos = (double)std::min<long long>((long long)nat.hh * nat.hw, (long long)g.h * g.w);
-                        prof_end(e0, VF_KERNEL_CONV_TC, 2.0 * (double)M * pos * g.ci * g.co * g.k * g.k /
-                                                            ((double)g.stride * g.stride));
+                        prof_end(e0, g.ci % 16 == 0 ? VF_KERNEL_CONV_TC : VF_KERNEL_CONV_TC_PAD,
+                                 2.0 * (double)M * pos * g.ci * g.co * g.k * g.k / ((double)g.stride * g.stride));
                     }
                     release(e);
                     return VF_OK;
@@ -2125,7 +2125,7 @@ int vf_profile_enable(vf_net* net, int enable) {
 
 int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms, double* flops, int reset) {
     TRY(check_net(net));
-    if (kind < 0 || kind > 6) return fail(VF_ERR_ARG, "bad kernel kind");
+    if (kind < 0 || kind > 7) return fail(VF_ERR_ARG, "bad kernel kind");
     for (auto& t : net->ev_used) {
         CU(cudaEventSynchronize(t.e1));
         float ms = 0.f;
@@ -2143,7 +2143,7 @@ int vf_profile_read(vf_net* net, int kind, long long* launches, double* total_ms
     if (total_ms) *total_ms = net->prof_ms[kind];
     if (flops) *flops = net->prof_flops[kind];
     if (reset)
-        for (int k = 0; k < 7; ++k) {
+        for (int k = 0; k < 8; ++k) {
             net->prof_launches[k] = 0;
             net->prof_ms[k] = 0.0;
             net->prof_flops[k] = 0.0;

@@ -21,7 +21,7 @@ VF_OK, VF_ERR_ARG, VF_ERR_SHAPE, VF_ERR_WORKSPACE, VF_ERR_NONFINITE, VF_ERR_CUDA
     VF_ERR_UNSUPPORTED = range(8)
 VF_INPUT, VF_DENSE, VF_CONV2D, VF_RELU, VF_ADD = range(5)
 (VF_KERNEL_ALL, VF_KERNEL_DENSE_TC, VF_KERNEL_DENSE_FFMA, VF_KERNEL_CONV, VF_KERNEL_CONV_WIN, VF_KERNEL_CONV_TC,
- VF_KERNEL_DENSE_FWD_TC) = range(7)
+ VF_KERNEL_DENSE_FWD_TC, VF_KERNEL_CONV_TC_PAD) = range(8)
 
 SYMBOLS = ["vf_net_create", "vf_net_destroy", "vf_net_node_size", "vf_net_total_size", "vf_ibp",
            "vf_crown_backward", "vf_concretize", "vf_verify_batch", "vf_sync", "vf_last_error",

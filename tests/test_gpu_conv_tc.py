@@ -2,7 +2,8 @@
 both tcgen05 implicit GEMMs with the 3xTF32 split: conv_back_tc (tap shifts, the default) and conv_back_tcn (taps
 in the N dimension, chosen with VF_CONV_TC=tapn where its shapes allow; measured slower, kept tested).
 
-The kernel takes every convolution back-substitution whose input has a multiple of 16 channels (up to 128),
+The kernel takes every convolution back-substitution whose input has a multiple of 16 channels (up to 128) or,
+at stride 1, fewer than 16 (a 3-channel stem, padded to 16 with zero weights),
 kernel size up to 8 and stride 1 or 2: whole-map rows, receptive-field windows, stored, accumulated (residual
 adds) and concretised against the input box (a convolution fed by a 16-channel input). The networks below
 are chosen so that each of those cases runs (1x1 stride-2 shortcuts leave whole stride classes empty; a 5x5
@@ -58,7 +59,26 @@ def _cnn(seed=62, B=2):
     return net, centres, C, float(np.float32(0.004))
 
 
-CASES = {"resnet16-32-64": _resnet, "conv5x5-conv3x3s2": _mixed, "cnn16-32-k4s2": _cnn}
+def _stem_cnn(seed=64, B=2):
+    """A 3-channel input whose 4x4 stride-2 stem stays on the FFMA kernels (the rest on the tensor cores)."""
+    rng = np.random.default_rng(seed)
+    net = synth.cnn_cfg3(rng, image=(3, 16, 16), c1=16, c2=32, hidden=20, classes=5)
+    centres = rng.random((B, 3 * 16 * 16)).astype(np.float32)
+    C = synth.margin_spec(rng.integers(0, 5, B), 5)
+    return net, centres, C, float(np.float32(0.004))
+
+
+def _stem_resnet(seed=65, B=2):
+    """A 3-channel 3x3 stride-1 stem before residual blocks of 16, 32 and 64 channels."""
+    rng = np.random.default_rng(seed)
+    net = synth.resnet_cfg4(rng, image=(3, 8, 8), widths=(16, 32, 64), fc=24, classes=5)
+    centres = rng.random((B, 3 * 8 * 8)).astype(np.float32)
+    C = synth.margin_spec(rng.integers(0, 5, B), 5)
+    return net, centres, C, float(np.float32(0.004))
+
+
+CASES = {"resnet16-32-64": _resnet, "conv5x5-conv3x3s2": _mixed, "cnn16-32-k4s2": _cnn, "stem3-cnn": _stem_cnn,
+         "stem3-resnet": _stem_resnet}
 
 
 def _run(net, centres, eps, C, both=True, workspace=0):
@@ -68,7 +88,7 @@ def _run(net, centres, eps, C, both=True, workspace=0):
     out = g.verify(_dev(centres), eps, _dev(C), both_sides=both, want_pre=True)
     torch.cuda.synchronize()
     g.check()
-    tc = g.profile_read(kind=vf.VF_KERNEL_CONV_TC, reset=True)[0]
+    tc = g.profile_read(kind=vf.VF_KERNEL_CONV_TC, reset=False)[0] + g.profile_read(kind=vf.VF_KERNEL_CONV_TC_PAD)[0]
     return g, {k: v.cpu().numpy() for k, v in out.items()}, tc
 
 
