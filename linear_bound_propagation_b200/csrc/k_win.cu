@@ -218,6 +218,7 @@ rewin_rows_k(RowRef A, Relax rx, long long M, int C, int H, int Wd, PassGeom pg,
     const int lane = threadIdx.x & 31;
     const long long n = (long long)C * H * Wd;
     const int nd = wd.C * wd.hh * wd.hw;
+    const float inv_hw = 1.f / (float)wd.hw, inv_hh = 1.f / (float)wd.hh;
     for (long long m = blockIdx.x * 8LL + (threadIdx.x >> 5); m < M; m += (long long)gridDim.x * 8) {
         const StartPos sp = start_pos(ps, pg, m);
         const int aoy = wa.ay * sp.yj + wa.by, aox = wa.ax * sp.xj + wa.bx;
@@ -225,21 +226,33 @@ rewin_rows_k(RowRef A, Relax rx, long long M, int C, int H, int Wd, PassGeom pg,
         const float* a = A.row(m);
         float* o = out + m * ld_out;
         float cs = 0.f;
-        for (int e = lane; e < nd; e += 32) {
-            const int dx = e % wd.hw, dy = (e / wd.hw) % wd.hh, c = e / (wd.hw * wd.hh);
-            const int Y = doy + dy, X = dox + dx;
-            const int ry = Y - aoy, rxx = X - aox;
-            float r = 0.f;
-            if (Y >= 0 && Y < H && X >= 0 && X < Wd && ry >= 0 && ry < wa.hh && rxx >= 0 && rxx < wa.hw) {
-                const float x = a[((long long)c * wa.hh + ry) * wa.hw + rxx];
-                r = x;
-                if (rx.P != nullptr) {
-                    const float4 p = rx.P[sp.b * n + ((long long)c * H + Y) * Wd + X];
-                    r = (x >= 0.f) ? x * p.x : x * p.y;
-                    if (rx.count_const) cs = fmaf(fminf(x, 0.f), p.z, cs);
-                }
+        // four entries per lane at a time, every load (coefficient, relaxation, old value) issued before any use
+        for (int e0 = lane; e0 < nd; e0 += 128) {
+            float x[4], old[4];
+            float4 p[4];
+            bool in[4], live[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + 32 * u;
+                live[u] = e < nd;
+                const int q = live[u] ? fdiv(e, inv_hw) : 0, dx = live[u] ? e - q * wd.hw : 0;
+                const int c = fdiv(q, inv_hh), dy = q - c * wd.hh;
+                const int Y = doy + dy, X = dox + dx;
+                const int ry = Y - aoy, rxx = X - aox;
+                in[u] = live[u] && Y >= 0 && Y < H && X >= 0 && X < Wd && ry >= 0 && ry < wa.hh && rxx >= 0 &&
+                        rxx < wa.hw;
+                x[u] = in[u] ? a[((long long)c * wa.hh + ry) * wa.hw + rxx] : 0.f;
+                p[u] = (in[u] && rx.P != nullptr) ? rx.P[sp.b * n + ((long long)c * H + Y) * Wd + X]
+                                                  : make_float4(1.f, 1.f, 0.f, 0.f);
+                old[u] = (live[u] && accumulate) ? o[e] : 0.f;
             }
-            o[e] = accumulate ? o[e] + r : r;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (!live[u]) continue;
+                const float r = (x[u] >= 0.f) ? x[u] * p[u].x : x[u] * p[u].y;
+                if (in[u] && rx.P != nullptr && rx.count_const) cs = fmaf(fminf(x[u], 0.f), p[u].z, cs);
+                o[e0 + 32 * u] = old[u] + r;
+            }
         }
         if (rx.P != nullptr && rx.count_const && cst != nullptr) {
             const float t = warp_sum(cs);
