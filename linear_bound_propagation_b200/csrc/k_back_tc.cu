@@ -354,6 +354,11 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 if (valid) p.part[(long long)n_tile * p.M + m] = conc;
                 __syncwarp();  // the staged centres are reused by the next tile
             } else {
+                // plain stores with 16-byte rows: each thread writes its own row's 32 columns as eight float4 (a short
+                // drain, so the accumulator goes back to the MMA sooner); otherwise through a shared-memory transpose
+                const bool vec = p.out_mode == OUT_STORE && (p.ld_out & 3) == 0 &&
+                                 (reinterpret_cast<uintptr_t>(p.out) & 15) == 0 &&
+                                 (p.col_bias == nullptr || (reinterpret_cast<uintptr_t>(p.col_bias) & 15) == 0);
                 for (int c0 = 0; c0 < p.BN; c0 += 64) {
                     uint32_t v[2][32];
                     tmem_ld32_nowait(tmem + lane_base + c0, v[0]);
@@ -367,6 +372,22 @@ dense_back_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                     for (int u = 0; u < 2; ++u) {
                         const int cu = c0 + 32 * u;
                         if (cu >= p.BN) break;
+                        if (vec && cu + 32 <= p.BN && n0 + cu + 32 <= p.N) {  // all 32 columns in the tile and the map
+                            if (valid) {
+                                float4* o4 = reinterpret_cast<float4*>(p.out + m * p.ld_out + n0 + cu);
+                                const float4* b4 =
+                                    p.col_bias != nullptr ? reinterpret_cast<const float4*>(p.col_bias + n0 + cu) : nullptr;
+#pragma unroll
+                                for (int q4 = 0; q4 < 8; ++q4) {
+                                    const float4 bb = b4 != nullptr ? __ldg(&b4[q4]) : make_float4(0.f, 0.f, 0.f, 0.f);
+                                    o4[q4] = make_float4(__uint_as_float(v[u][4 * q4]) + bb.x,
+                                                         __uint_as_float(v[u][4 * q4 + 1]) + bb.y,
+                                                         __uint_as_float(v[u][4 * q4 + 2]) + bb.z,
+                                                         __uint_as_float(v[u][4 * q4 + 3]) + bb.w);
+                                }
+                            }
+                            continue;
+                        }
 #pragma unroll
                         for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(v[u][j]);
                         __syncwarp();
