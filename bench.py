@@ -210,7 +210,12 @@ TF32_OVER_BF16 = 1.1 / 2.25
 # capture of the full-size workload, summed over the six contraction launches of one timed step and divided
 # by six. Keyed by workload name and kernel kind; reported only for that pair, and to be dropped whenever
 # the kernel changes.
-TRAFFIC_PER_LAUNCH = {("mlp_784-256x3-10_B1024", 1): 1099.0e6 / 6}
+# DRAM bytes (read + write) per dense_back_tc launch, from one-pass ncu captures of the current kernel
+# (profiles/dense_back_tc_wide_mlp_B4096.md section 3b): every launch of one verify call; the wide MLP measured at 256
+# centres (21 launches, 48.69 GB) and scaled by rows to 4096 centres (traffic grows with the rows), over its 73
+# full-size launches
+TRAFFIC_PER_LAUNCH = {("mlp_784-256x3-10_B1024", 1): 1.105e9 / 6,
+                      ("mlp_3072-1024x8-100_B4096", 1): 48.69e9 * 16 / 73}
 
 
 def roofline(kstats, step_total_ms, n_sms, workload=None, step_ms=None):
