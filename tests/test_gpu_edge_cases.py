@@ -252,3 +252,29 @@ def test_bab_decisions_bit_exact(monkeypatch):
         deep += r["rounds"] >= 2
     assert compared >= 8 and deep >= 2, f"only {compared} properties free of near-ties ({deep} with 2+ rounds)"
     assert falsified >= 8, f"only {falsified} falsified properties free of near-ties"
+
+
+def test_empty_batches_are_no_ops():
+    """No centres or no specification rows: every entry point returns VF_OK without touching its outputs (the
+    output buffers keep a sentinel), and the handle keeps working."""
+    import ctypes
+    w = synth.workload(2, B=2)
+    g = vf.Net(w.net)
+    L = vf.lib()
+    cen, C = _dev(w.centres), _dev(w.C)
+    sentinel = torch.full((64,), 7.0, device="cuda")
+    p = sentinel.data_ptr()
+    o = vf.Opts()
+    for B, R in ((0, 9), (2, 0), (0, 0)):
+        assert L.vf_verify_batch(g.h, cen.data_ptr(), B, w.eps, C.data_ptr(), R, 0, ctypes.byref(o), p, None, None,
+                                 None, None) == vf.VF_OK
+        assert L.vf_alpha_crown(g.h, cen.data_ptr(), B, w.eps, C.data_ptr(), R, 0, ctypes.byref(o), 3, 0.1, p, None,
+                                None, None) == vf.VF_OK
+        assert L.vf_concretize(p, None, cen.data_ptr(), w.eps, B, R, 784, p, None) == vf.VF_OK
+    assert L.vf_ibp(g.h, cen.data_ptr(), 0, w.eps, p, p, None) == vf.VF_OK
+    torch.cuda.synchronize()
+    g.check()
+    assert torch.all(sentinel == 7.0)
+    out = g.verify(cen, w.eps, C)  # still usable
+    torch.cuda.synchronize()
+    assert torch.isfinite(out["lb"]).all()
