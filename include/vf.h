@@ -271,6 +271,12 @@ typedef struct {
 int vf_bab_verify(vf_net* net, const float* centre, float eps, const float* C, int R, const vf_bab_opts* opts,
                   vf_bab_result* result /*[host]*/, void* stream);
 
+/* ABI self-description, for bindings that mirror the structs above (no device work): for struct `which`
+ * (0 vf_node_desc, 1 vf_opts, 2 vf_bab_opts, 3 vf_bab_result) and `field` (index in declaration order, each
+ * declarator counted once), writes the field's byte offset to *out; field = -1 writes the struct's size.
+ * VF_ERR_ARG for an unknown struct or a field index past the last one. */
+int vf_abi_layout(int which, int field, size_t* out);
+
 /* The search of vf_bab_verify (steps 2-5) with a caller-supplied bound function, so other bounding
  * methods can drive it; vf_bab_verify is the centre check plus this search with the device bound function.
  * bound(user, n, ...) bounds n subdomains: subdomain i holds split_count[i] splits, listed from

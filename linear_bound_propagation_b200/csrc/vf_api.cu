@@ -22,6 +22,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstddef>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -2104,6 +2105,37 @@ int vf_alpha_beta_grad(vf_net* net, const float* centres, int B, float eps, cons
                                 nullptr, (cudaStream_t)stream, beta, grad_beta);
     return spec_alpha(net, centres, B, eps, C, R, C_bstride, o, 0, 0.f, true, alpha, grad_alpha, lb, nullptr, nullptr,
                       (cudaStream_t)stream, beta, grad_beta);
+}
+
+int vf_abi_layout(int which, int field, size_t* out) {
+    if (!out) return fail(VF_ERR_ARG, "NULL pointer");
+#define VF_OFF(T, f) offsetof(T, f)
+    static const size_t node[] = {VF_OFF(vf_node_desc, op),     VF_OFF(vf_node_desc, src), VF_OFF(vf_node_desc, src2),
+                                  VF_OFF(vf_node_desc, c),      VF_OFF(vf_node_desc, h),   VF_OFF(vf_node_desc, w),
+                                  VF_OFF(vf_node_desc, n_out),  VF_OFF(vf_node_desc, k),   VF_OFF(vf_node_desc, stride),
+                                  VF_OFF(vf_node_desc, pad),    VF_OFF(vf_node_desc, W),   VF_OFF(vf_node_desc, b)};
+    static const size_t opts[] = {VF_OFF(vf_opts, relu_crown),      VF_OFF(vf_opts, alpha),
+                                  VF_OFF(vf_opts, both_sides),      VF_OFF(vf_opts, skip_finite_check),
+                                  VF_OFF(vf_opts, pre_lb),          VF_OFF(vf_opts, pre_ub),
+                                  VF_OFF(vf_opts, no_host_sync),    VF_OFF(vf_opts, split),
+                                  VF_OFF(vf_opts, sound),           VF_OFF(vf_opts, alpha_inter_iters),
+                                  VF_OFF(vf_opts, alpha_inter_lr),  VF_OFF(vf_opts, alpha_rows_init),
+                                  VF_OFF(vf_opts, beta_rows_init),  VF_OFF(vf_opts, beta_rows_out)};
+    static const size_t bopts[] = {VF_OFF(vf_bab_opts, max_domains),       VF_OFF(vf_bab_opts, batch),
+                                   VF_OFF(vf_bab_opts, alpha_iters),       VF_OFF(vf_bab_opts, lr),
+                                   VF_OFF(vf_bab_opts, relu_crown),        VF_OFF(vf_bab_opts, trace),
+                                   VF_OFF(vf_bab_opts, trace_cap),         VF_OFF(vf_bab_opts, alpha_inter_iters),
+                                   VF_OFF(vf_bab_opts, alpha_inter_lr),    VF_OFF(vf_bab_opts, cold_start)};
+    static const size_t bres[] = {VF_OFF(vf_bab_result, status), VF_OFF(vf_bab_result, domains),
+                                  VF_OFF(vf_bab_result, rounds), VF_OFF(vf_bab_result, max_depth),
+                                  VF_OFF(vf_bab_result, lb)};
+#undef VF_OFF
+    const size_t* tab[] = {node, opts, bopts, bres};
+    const int count[] = {12, 14, 10, 5};
+    const size_t size[] = {sizeof(vf_node_desc), sizeof(vf_opts), sizeof(vf_bab_opts), sizeof(vf_bab_result)};
+    if (which < 0 || which > 3 || field < -1 || field >= count[which]) return fail(VF_ERR_ARG, "no such struct field");
+    *out = field < 0 ? size[which] : tab[which][field];
+    return VF_OK;
 }
 
 int vf_net_node_info(const vf_net* net, int v, int* op, int* src, int* src2, long long* n) {

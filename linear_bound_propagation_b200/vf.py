@@ -27,7 +27,7 @@ SYMBOLS = ["vf_net_create", "vf_net_destroy", "vf_net_node_size", "vf_net_total_
            "vf_crown_backward", "vf_concretize", "vf_verify_batch", "vf_sync", "vf_last_error",
            "vf_profile_enable", "vf_profile_read", "vf_launch_count", "vf_net_check",
            "vf_concretize_dense_noalloc", "vf_alpha_crown", "vf_alpha_grad", "vf_alpha_beta_grad",
-           "vf_net_node_info", "vf_bab_verify", "vf_bab_search"]
+           "vf_net_node_info", "vf_bab_verify", "vf_bab_search", "vf_abi_layout"]
 NOALLOC_SCRATCH_FLOATS = 1 << 22
 
 

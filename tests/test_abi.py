@@ -52,3 +52,19 @@ def test_new_entry_points_reject_null_arguments_without_a_gpu():
     assert L.vf_alpha_beta_grad(None, None, 1, 0.1, None, 1, 0, None, None, None, None, None, None, None) == vf.VF_ERR_ARG
     op = vf.ctypes.c_int()
     assert L.vf_net_node_info(None, 0, vf.ctypes.byref(op), None, None, None) == vf.VF_ERR_ARG
+
+
+def test_struct_layouts_match_the_binding():
+    """Every ctypes mirror of a C struct (node descriptors, vf_opts, vf_bab_opts, vf_bab_result) has the C
+    struct's size and every field at the C offset, as the library reports them (vf_abi_layout, no device
+    work): a field added on one side only would shift every later one."""
+    L = vf.lib()
+    L.vf_abi_layout.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+    out = ctypes.c_size_t()
+    for which, S in enumerate((vf.NodeDesc, vf.Opts, vf.BabOpts, vf.BabResult)):
+        assert L.vf_abi_layout(which, -1, ctypes.byref(out)) == vf.VF_OK
+        assert out.value == ctypes.sizeof(S), S.__name__
+        for i, (name, _) in enumerate(S._fields_):
+            assert L.vf_abi_layout(which, i, ctypes.byref(out)) == vf.VF_OK, (S.__name__, name)
+            assert out.value == getattr(S, name).offset, (S.__name__, name)
+        assert L.vf_abi_layout(which, len(S._fields_), ctypes.byref(out)) == vf.VF_ERR_ARG, S.__name__
