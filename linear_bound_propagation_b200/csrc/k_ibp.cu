@@ -9,18 +9,25 @@
 //   add:     centres add, radii add
 //   splits:  branch-and-bound subdomains fix the sign of some pre-activations (same page, §2.2 and
 //            §4.3: beta-CROWN with branch-and-bound); their intervals are clamped to that sign
+#include <cooperative_groups.h>
+
 #include "vf_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace vf {
 
 namespace {
 
-// z[m, n] = sum_k h[m, k] * W[n, k]: blockIdx.z = 0 computes the centre (h = centre, W, + bias), 1 the
-// radius (h = radius, |W|). Tiles of 64 rows x 64 columns, 256 threads each owning a 4 x 4 block of
-// outputs; per k the thread reads one float4 of the staged h tile and one of the staged W tile for 16
-// FMAs. The next 16-wide k-slice is prefetched into registers while the current one is used. With
-// rowsum_abs != nullptr the source is the input box with radius eps in every coordinate: the radius is
-// eps * sum_k |W[n, k]| without a product.
+// z[m, n] = sum_k h[m, k] * W[n, k]: plane 0 computes the centre (h = centre, W, + bias), plane 1 the
+// radius (h = radius, |W|); the plane is blockIdx.z (/ the cluster size with SPLIT) + z0. Tiles of 64
+// rows x 64 columns, 256 threads each owning a 4 x 4 block of outputs; per k the thread reads one float4
+// of the staged h tile and one of the staged W tile for 16 FMAs. The next 16-wide k-slice is prefetched
+// into registers while the current one is used. With rowsum_abs != nullptr the source is the input box
+// with radius eps in every coordinate: the radius is eps * sum_k |W[n, k]| without a product.
+// SPLIT: a cluster of ks CTAs shares each output tile, rank r taking the r-th share of the k-slices; the
+// partial tiles meet in distributed shared memory and each rank sums 64 / ks of the rows in rank order.
+template <bool SPLIT>
 __global__ void __launch_bounds__(256)
 ibp_dense_k(const float* __restrict__ hc, const float* __restrict__ hr, const float* __restrict__ W,
             const float* __restrict__ Wabs, const float* __restrict__ bias, const float* __restrict__ rowsum_abs,
@@ -30,8 +37,11 @@ ibp_dense_k(const float* __restrict__ hc, const float* __restrict__ hr, const fl
     __shared__ __align__(16) float Bs[KB][LDB];
     const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
     const int m0 = blockIdx.x * TM, n0 = blockIdx.y * TN;
-    const bool rad = blockIdx.z + z0 == 1;
-    if (rad && rowsum_abs != nullptr) {
+    const int ks = SPLIT ? (int)cg::this_cluster().num_blocks() : 1;  // the cluster spans (1, 1, ks) CTAs
+    const int rank = SPLIT ? (int)blockIdx.z % ks : 0;
+    const bool rad = (int)blockIdx.z / ks + z0 == 1;
+    if (rad && rowsum_abs != nullptr) {  // the whole cluster leaves here together: no barrier is pending
+        if (rank != 0) return;
         for (int e = tid; e < TM * TN; e += 256) {
             const int m = m0 + e / TN, n = n0 + e % TN;
             if (m < B && n < N) zr[(long long)m * N + n] = eps * rowsum_abs[n];
@@ -40,6 +50,9 @@ ibp_dense_k(const float* __restrict__ hc, const float* __restrict__ hr, const fl
     }
     const float* h = rad ? hr : hc;
     const float* w = rad ? Wabs : W;
+    const int nk = (K + KB - 1) / KB;
+    const int k_begin = (int)((long long)rank * nk / ks) * KB;
+    const int k_end = min(K, (int)((long long)(rank + 1) * nk / ks) * KB);
     // loader mapping: 64 rows x 16 k per tile = 1024 values, 4 per thread (k fastest for coalescing)
     float a_reg[4], b_reg[4];
     auto load = [&](int k0) {
@@ -47,8 +60,8 @@ ibp_dense_k(const float* __restrict__ hc, const float* __restrict__ hr, const fl
         for (int i = 0; i < 4; ++i) {
             const int e = tid + 256 * i, row = e / KB, kk = e % KB, k = k0 + kk;
             const int m = m0 + row, n = n0 + row;
-            a_reg[i] = (m < B && k < K) ? h[(long long)m * K + k] : 0.f;
-            b_reg[i] = (n < N && k < K) ? w[(long long)n * K + k] : 0.f;
+            a_reg[i] = (m < B && k < k_end) ? h[(long long)m * K + k] : 0.f;
+            b_reg[i] = (n < N && k < k_end) ? w[(long long)n * K + k] : 0.f;
         }
     };
     float acc[4][4];
@@ -56,8 +69,8 @@ ibp_dense_k(const float* __restrict__ hc, const float* __restrict__ hr, const fl
     for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-    load(0);
-    for (int k0 = 0; k0 < K; k0 += KB) {
+    load(k_begin);
+    for (int k0 = k_begin; k0 < k_end; k0 += KB) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int e = tid + 256 * i;
@@ -65,7 +78,7 @@ ibp_dense_k(const float* __restrict__ hc, const float* __restrict__ hr, const fl
             Bs[e % KB][e / KB] = b_reg[i];
         }
         __syncthreads();
-        if (k0 + KB < K) load(k0 + KB);
+        if (k0 + KB < k_end) load(k0 + KB);
 #pragma unroll
         for (int kk = 0; kk < KB; ++kk) {
             const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
@@ -77,6 +90,29 @@ ibp_dense_k(const float* __restrict__ hc, const float* __restrict__ hr, const fl
                 for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
         __syncthreads();
+    }
+    if constexpr (SPLIT) {
+        __shared__ __align__(16) float Cs[TM][TN + 4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4*>(&Cs[ty * 4 + i][tx * 4]) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        cg::cluster_group cluster = cg::this_cluster();
+        cluster.sync();
+        const int rows_per = TM / ks;  // ks divides 64 (a power of two)
+        for (int e = tid; e < rows_per * TN; e += 256) {
+            const int row = rank * rows_per + e / TN, col = e % TN;
+            const int m = m0 + row, n = n0 + col;
+            float v = 0.f;
+            for (int q = 0; q < ks; ++q) v += cluster.map_shared_rank(&Cs[0][0], q)[row * (TN + 4) + col];
+            if (m < B && n < N) {
+                if (rad)
+                    zr[(long long)m * N + n] = v;
+                else
+                    zc[(long long)m * N + n] = v + bias[n];
+            }
+        }
+        cluster.sync();  // every rank's tile stays in shared memory until the others have read it
+        return;
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -180,32 +216,70 @@ unsigned grid_for(long long n, int threads) {
 
 }  // namespace
 
+namespace {
+
+// Forward products z = h . W^T over `planes` planes (centre and/or radius) starting at plane z0. When
+// the 64 x 64 tiles would not fill the SMs, K is split over a cluster of up to 8 CTAs per tile (a power
+// of two, at least two 16-wide k-slices per rank).
+cudaError_t launch_fwd(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
+                       const float* rowsum_abs, float eps, int B, int K, int N, float* zc, float* zr, int planes, int z0,
+                       cudaStream_t s) {
+    if (B <= 0) return cudaSuccess;
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0, v = 0;
+        sms = (cudaGetDevice(&dev) == cudaSuccess &&
+               cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+                  ? v
+                  : 148;
+    }
+    const long long tiles = (long long)((B + 63) / 64) * ((N + 63) / 64) * planes;
+    int ks = 1;
+    while (ks < 8 && tiles * ks * 2 <= 2LL * sms && ks * 2 * 2 * 16 <= K) ks *= 2;
+    if (ks == 1) {
+        dim3 grid((B + 63) / 64, (N + 63) / 64, planes);
+        ibp_dense_k<false><<<grid, 256, 0, s>>>(hc, hr, W, Wabs, bias, rowsum_abs, eps, B, K, N, zc, zr, z0);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)((B + 63) / 64), (unsigned)((N + 63) / 64), (unsigned)(planes * ks));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = (unsigned)ks;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ibp_dense_k<true>, hc, hr, W, Wabs, bias, rowsum_abs, eps, B, K, N, zc, zr, z0);
+}
+
+}  // namespace
+
 cudaError_t launch_ibp_dense(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
                              const float* rowsum_abs, float eps, int B, int K, int N, float* zc, float* zr,
                              cudaStream_t s) {
-    dim3 grid((B + 63) / 64, (N + 63) / 64, 2);
-    ibp_dense_k<<<grid, 256, 0, s>>>(hc, hr, W, Wabs, bias, rowsum_abs, eps, B, K, N, zc, zr, 0);
-    return cudaGetLastError();
+    return launch_fwd(hc, hr, W, Wabs, bias, rowsum_abs, eps, B, K, N, zc, zr, 2, 0, s);
 }
 
 cudaError_t launch_ibp_radius_rowsum(const float* rowsum_abs, float eps, int B, int N, float* zr, cudaStream_t s) {
     dim3 grid((B + 63) / 64, (N + 63) / 64, 1);  // only the radius of a layer fed by the input box
-    ibp_dense_k<<<grid, 256, 0, s>>>(nullptr, nullptr, nullptr, nullptr, nullptr, rowsum_abs, eps, B, 0, N, nullptr,
-                                     zr, 1);
+    ibp_dense_k<false><<<grid, 256, 0, s>>>(nullptr, nullptr, nullptr, nullptr, nullptr, rowsum_abs, eps, B, 0, N,
+                                            nullptr, zr, 1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_abs_rows_times_wt(const float* A, const float* Wabs, int M, int K, int N, float* out, cudaStream_t s) {
-    dim3 grid((M + 63) / 64, (N + 63) / 64, 1);  // only the radius product: out = A |W|^T
-    ibp_dense_k<<<grid, 256, 0, s>>>(A, A, Wabs, Wabs, nullptr, nullptr, 0.f, M, K, N, out, out, 1);
-    return cudaGetLastError();
+    // only the radius product: out = A |W|^T
+    return launch_fwd(A, A, Wabs, Wabs, nullptr, nullptr, 0.f, M, K, N, out, out, 1, 1, s);
 }
 
 cudaError_t launch_rows_times_wt(const float* A, const float* W, const float* bias, int M, int K, int N, float* out,
                                  cudaStream_t s) {
-    dim3 grid((M + 63) / 64, (N + 63) / 64, 1);  // only the centre product: out = A W^T + bias
-    ibp_dense_k<<<grid, 256, 0, s>>>(A, A, W, W, bias, nullptr, 0.f, M, K, N, out, out, 0);
-    return cudaGetLastError();
+    // only the centre product: out = A W^T + bias
+    return launch_fwd(A, A, W, W, bias, nullptr, 0.f, M, K, N, out, out, 1, 0, s);
 }
 
 cudaError_t launch_ibp_conv(const float* hc, const float* hr, const float* W, const float* Wabs, const float* bias,
