@@ -97,7 +97,11 @@ struct vf_net {
     size_t ws_bytes = 0;
     long long launches = 0;
     long long fail_at = 0;  // test hook: VF_TEST_FAIL_AT=<n> fails the n-th launch on the host
-    int dense_kernel = 0;   // 0: tensor cores where the shapes allow, 1: FFMA only (VF_DENSE_KERNEL=ffma)
+    // back-substitution through dense nodes: 0 (default) tensor cores where the shapes allow and the launch has at
+    // least dense_tc_min_tiles output tiles (fewer tiles leave most SMs idle, where the K-split FFMA kernel is
+    // faster), 1 FFMA only (VF_DENSE_KERNEL=ffma), 2 tensor cores whenever the shapes allow (VF_DENSE_KERNEL=tc)
+    int dense_kernel = 0;
+    long long dense_tc_min_tiles = 16;  // VF_DENSE_TC_MIN_TILES
     int* d_err = nullptr;   // device flag raised by a kernel whose bounded wait expired
     int tc_stall = 0;       // test hook: VF_TEST_TC_STALL=1 makes one tensor-core launch time out
     int windows = 1;        // receptive-field windows in passes that start at a convolution (VF_CONV_WINDOWS=0: off)
@@ -230,6 +234,13 @@ bool win_union(const Win& a, const Win& b, Win* u) {
     const int by = std::min(a.by, b.by), bx = std::min(a.bx, b.bx);
     *u = Win{a.C, std::max(a.by + a.hh, b.by + b.hh) - by, std::max(a.bx + a.hw, b.bx + b.hw) - bx, a.ay, by, a.ax, bx};
     return true;
+}
+
+// Dense back-substitution of M rows onto a node of N neurons on the tensor cores (the kernel's own shape
+// checks aside): not in FFMA-only or sound calls, and by default only when the launch has enough output tiles.
+bool back_tc_ok(const vf_net* net, long long M, int N) {
+    if (net->dense_kernel == 1 || net->call_sound) return false;
+    return net->dense_kernel == 2 || ((M + 127) / 128) * dense_back_tc_tiles_n(N) >= net->dense_tc_min_tiles;
 }
 
 struct Walker {
@@ -512,7 +523,7 @@ struct Walker {
                 long long ld = 0;
                 int mode = OUT_CONCRETIZE;
                 if (!fuse) TRY(target(nd.src, &out, &ld, &mode));
-                const bool tc = net->dense_kernel == 0 && !net->call_sound && nd.WtHi != nullptr &&
+                const bool tc = back_tc_ok(net, M, (int)sn.n) && nd.WtHi != nullptr &&
                                 dense_back_tc_supported(e.ref, e.rx, M, (int)nd.n, (int)sn.n, pg);
                 if (fuse) part_tiles = tc ? dense_back_tc_tiles_n((int)sn.n) : dense_back_tiles_n((int)sn.n);
                 if (!dry) {
@@ -719,7 +730,7 @@ constexpr long long kFwdTcMinTiles = 32;
 
 bool fwd_tc_ok(const vf_net* net, const Node& nd, const float* A, long long M, int K) {
     const int N = (int)nd.n;
-    if (net->dense_kernel != 0 || net->fwd_tc == 0 || net->call_sound || nd.WfHi == nullptr) return false;
+    if (net->dense_kernel == 1 || net->fwd_tc == 0 || net->call_sound || nd.WfHi == nullptr) return false;
     if (!dense_fwd_tc_supported(A, M, K, N)) return false;
     return net->fwd_tc >= 2 || ((M + 127) / 128) * dense_back_tc_tiles_n(N) >= kFwdTcMinTiles;
 }
@@ -1235,7 +1246,7 @@ int alpha_chain(vf_net* net, int L, const float* centres, int B, float eps, cons
     // identity relaxation table [B, nmax]: the slopes are applied by relax_alpha_rows_k, so the contraction
     // that follows may run on the tensor cores, which read every row through such a table
     float4* ident = nullptr;
-    if (net->dense_kernel == 0 && !net->call_sound) {
+    if (net->dense_kernel != 1 && !net->call_sound) {
         ident = ar.take<float4>((size_t)B * nmax);
         if (!ident) return fail(VF_ERR_WORKSPACE, "workspace too small for alpha optimisation");
         LAUNCH(net, launch_identity_relax(ident, (long long)B * nmax, s));
@@ -1340,7 +1351,7 @@ int alpha_chain(vf_net* net, int L, const float* centres, int B, float eps, cons
                     LAUNCH(net, launch_conv_back(RowRef{Z, 0, nu, kHugeRows, 0}, Relax{nullptr, 0}, d.W, nullptr, Mc,
                                                  conv_geom(net, d), pg, OUT_STORE, out, nd_in, cpart, nullptr, 0.f,
                                                  net->num_sms, s));
-                else if (ident != nullptr && d.WtHi != nullptr &&
+                else if (ident != nullptr && d.WtHi != nullptr && back_tc_ok(net, Mc, nd_in) &&
                          dense_back_tc_supported(RowRef{Z, 0, nu, kHugeRows, 0}, Relax{ident, 0}, Mc, nu, nd_in, pg))
                     LAUNCH(net, launch_dense_back_tc(RowRef{Z, 0, nu, kHugeRows, 0}, Relax{ident, 0}, d.WtHi, d.WtLo, B,
                                                      Mc, nu, nd_in, pg, OUT_STORE, out, nd_in, cst, nullptr, 0.f,
@@ -1686,7 +1697,9 @@ static int create_impl(const vf_node_desc* d, int n_nodes, size_t ws_bytes, vf_n
     CU(cudaGetDevice(&net->device));
     CU(cudaDeviceGetAttribute(&net->num_sms, cudaDevAttrMultiProcessorCount, net->device));
     if (const char* f = getenv("VF_TEST_FAIL_AT")) net->fail_at = atoll(f);
-    if (const char* f = getenv("VF_DENSE_KERNEL")) net->dense_kernel = (strcmp(f, "ffma") == 0) ? 1 : 0;
+    if (const char* f = getenv("VF_DENSE_KERNEL"))
+        net->dense_kernel = (strcmp(f, "ffma") == 0) ? 1 : (strcmp(f, "tc") == 0 ? 2 : 0);
+    if (const char* f = getenv("VF_DENSE_TC_MIN_TILES")) net->dense_tc_min_tiles = std::max(0LL, atoll(f));
     if (const char* f = getenv("VF_TEST_TC_STALL")) net->tc_stall = atoi(f) != 0;
     if (const char* f = getenv("VF_CONV_WINDOWS")) net->windows = atoi(f) != 0;
     if (const char* f = getenv("VF_CONV_KERNEL"))

@@ -382,7 +382,8 @@ class Net:
     def profile_read(self, kind: int = 0, reset: bool = True):
         """(launches, total device ms, algorithmic flops) of one contraction kind since the last reset:
         0 all, 1 dense tensor-core (3xTF32), 2 dense FFMA, 3 whole-map convolution, 4 windowed convolution,
-        5 tensor-core convolution (3xTF32, whole maps and windows)."""
+        5 tensor-core convolution (3xTF32, whole maps and windows), 6 dense tensor-core forward product,
+        7 tensor-core convolution of a stem with its channels padded to 16."""
         n = ctypes.c_longlong()
         ms = ctypes.c_double()
         fl = ctypes.c_double()

@@ -31,8 +31,10 @@ def _oracle_relax(net, res, b):
 def test_alpha_grad_matches_oracle(monkeypatch, config, B):
     """Bound and slope gradient element-wise. Workload 2 at 16 centres has 144 rows per pass, so with the forward
     products on the tensor cores whenever the shapes allow (VF_FWD_TC=all) the gradient's G W^T + b runs there
-    (at 6 centres, 54 rows, on the FFMA kernel)."""
+    (at 6 centres, 54 rows, on the FFMA kernel). The down pass's contractions take the tensor cores whenever the
+    shapes allow as well (VF_DENSE_KERNEL=tc)."""
     monkeypatch.setenv("VF_FWD_TC", "all")
+    monkeypatch.setenv("VF_DENSE_KERNEL", "tc")
     w = synth.workload(config, B=B)
     net, R = w.net, w.C.shape[1]
     rng = np.random.default_rng(5)

@@ -25,8 +25,18 @@ def _dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
+def _dense_kernel(monkeypatch, seed):
+    """Even seeds force the tensor cores on every dense launch the shapes allow (VF_DENSE_KERNEL=tc); odd
+    seeds keep the default choice, which sends launches of few tiles to the K-split FFMA kernel."""
+    if seed % 2 == 0:
+        monkeypatch.setenv("VF_DENSE_KERNEL", "tc")
+    else:
+        monkeypatch.delenv("VF_DENSE_KERNEL", raising=False)
+
+
 @pytest.mark.parametrize("seed", SEEDS)
-def test_random_network_matches_oracle(seed):
+def test_random_network_matches_oracle(monkeypatch, seed):
+    _dense_kernel(monkeypatch, seed)
     net, shape, classes = random_net(seed)
     rng = np.random.default_rng(20_000 + seed)
     B = int(rng.integers(1, 4))
@@ -59,10 +69,11 @@ def test_random_network_matches_oracle(seed):
 
 
 @pytest.mark.parametrize("seed", list(range(16)))
-def test_random_mlp_matches_oracle(seed):
+def test_random_mlp_matches_oracle(monkeypatch, seed):
     """Random dense ReLU chains (widths that do and do not meet the tensor-core shape rules), random batch
     sizes that leave ragged tiles, random subsets of layers refined by CROWN (the rest keep IBP bounds)
     and both bound sides."""
+    _dense_kernel(monkeypatch, seed)
     net, widths = random_mlp(seed)
     rng = np.random.default_rng(40_000 + seed)
     B = int(rng.integers(1, 41))

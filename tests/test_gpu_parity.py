@@ -234,18 +234,56 @@ def test_cfg5_subset_each_eps(eps):
     assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out)
 
 
-@pytest.mark.parametrize("kernel", ["tc", "ffma"])
+@pytest.mark.parametrize("kernel", ["tc", "ffma", "default"])
 def test_cfg2_both_dense_kernels(monkeypatch, kernel):
-    """The tensor-core (3xTF32) and FFMA contractions each match the oracle on the bench network."""
-    monkeypatch.setenv("VF_DENSE_KERNEL", kernel)
+    """The tensor-core (3xTF32) contraction on every launch the shapes allow, FFMA only, and the default choice
+    (launches of few tiles on the K-split FFMA kernel) each match the oracle on the bench network."""
+    if kernel == "default":
+        monkeypatch.delenv("VF_DENSE_KERNEL", raising=False)
+    else:
+        monkeypatch.setenv("VF_DENSE_KERNEL", kernel)
     w = synth.workload(2, B=11)
     g, ora, out = run_both(w.net, w.centres, w.eps, w.C, both=True)
     assert_parity(w.net, w.centres, w.eps, w.C, g, ora, out, both=True)
 
 
+@pytest.mark.parametrize("B,min_tiles,want_tc", [(2, "100000", False), (2, "0", True), (64, None, True)])
+def test_dense_kernel_choice_by_tile_count(monkeypatch, B, min_tiles, want_tc):
+    """A dense back-substitution takes the tensor cores only when its launch has at least VF_DENSE_TC_MIN_TILES
+    output tiles (128 rows x up to 256 columns): with an unreachable minimum every launch runs on the FFMA kernel,
+    with 0 every launch the shapes allow runs on the tensor cores, and with the default the intermediate passes of
+    64 centres of the 784-256x3-10 network (64 x 512 rows, 256 tiles and more) do. The bounds match the oracle
+    either way."""
+    monkeypatch.delenv("VF_DENSE_KERNEL", raising=False)
+    if min_tiles is None:
+        monkeypatch.delenv("VF_DENSE_TC_MIN_TILES", raising=False)
+    else:
+        monkeypatch.setenv("VF_DENSE_TC_MIN_TILES", min_tiles)
+    w = synth.workload(2, B=B)
+    g = vf.Net(w.net)
+    g.profile(True)
+    g.profile_read(reset=True)
+    out = g.verify(_dev(w.centres), w.eps, _dev(w.C))
+    torch.cuda.synchronize()
+    g.check()
+    n_tc = g.profile_read(kind=vf.VF_KERNEL_DENSE_TC, reset=False)[0]
+    n_ffma = g.profile_read(kind=vf.VF_KERNEL_DENSE_FFMA)[0]
+    assert (n_tc > 0) == want_tc, (n_tc, n_ffma)
+    assert n_ffma > 0  # the specification pass's first step (K = 10) is always FFMA
+    nb = min(B, 4)  # rows are independent across centres: the oracle checks the first few
+    ora = O.verify(w.net, w.centres[:nb], w.eps, w.C[:nb])
+    amb = ambiguous_centres(ora, w.net)
+    lb = out["lb"].cpu().numpy()
+    for b in range(nb):
+        if not amb[b]:
+            assert max_violation(lb[b], ora.lb[b]) <= 1.0, b
+
+
 def test_tc_path_wide_mlp_shapes(monkeypatch):
     """Shapes that hit the tensor-core tiling edge cases: K not a multiple of 32, N not a multiple
-    of the N tile, N below 16 (falls back), several N tiles with concretisation partials."""
+    of the N tile, N below 16 (falls back), several N tiles with concretisation partials. The launches here
+    have few tiles, so the tensor cores are forced (VF_DENSE_KERNEL=tc)."""
+    monkeypatch.setenv("VF_DENSE_KERNEL", "tc")
     rng = np.random.default_rng(11)
     net = synth.mlp([300, 196, 68, 260, 36, 12], rng)
     B = 3
@@ -359,6 +397,7 @@ def test_bounded_wait_expiry_is_reported_and_context_survives(monkeypatch):
     two seconds of clock, frees its resources and raises the device flag: vf_net_check reports
     VF_ERR_TIMEOUT. The context stays usable: a fresh handle then matches the oracle."""
     w = synth.workload(2, B=4)
+    monkeypatch.setenv("VF_DENSE_KERNEL", "tc")  # few tiles per launch: force the tensor-core kernel
     monkeypatch.setenv("VF_TEST_TC_STALL", "1")
     g = vf.Net(w.net)
     g.verify(_dev(w.centres), w.eps, _dev(w.C))
