@@ -270,6 +270,10 @@ def test_dense_kernel_choice_by_tile_count(monkeypatch, B, min_tiles, want_tc):
     n_ffma = g.profile_read(kind=vf.VF_KERNEL_DENSE_FFMA)[0]
     assert (n_tc > 0) == want_tc, (n_tc, n_ffma)
     assert n_ffma > 0  # the specification pass's first step (K = 10) is always FFMA
+    # the K-split FFMA launches reduce their partial tiles in a fixed order: a second call is bitwise identical
+    again = g.verify(_dev(w.centres), w.eps, _dev(w.C))
+    torch.cuda.synchronize()
+    assert torch.equal(again["lb"], out["lb"])
     nb = min(B, 4)  # rows are independent across centres: the oracle checks the first few
     ora = O.verify(w.net, w.centres[:nb], w.eps, w.C[:nb])
     amb = ambiguous_centres(ora, w.net)
