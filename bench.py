@@ -442,7 +442,7 @@ def measure_workload(args, ctx, cfg, eps, steps, warmup, headline, legs=None):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(w, args.cpu_sample_s if headline else args.sub_cpu_sample_s)[0]
         if bab is not None:
-            line["cpu_baseline"]["bab"] = oracle_bab_sample(args, w, bab["label0"])
+            line["cpu_baseline"]["bab"] = oracle_bab_sample(args, w, bab["sample_centre"], bab["sample_label"])
     if not headline:  # sub-lines keep only what identifies and measures them
         for k in ("metric", "unit", "n_gpus", "higher_is_better", "scaling", "vs_baseline", "dtype", "data"):
             line.pop(k, None)
@@ -640,7 +640,7 @@ def bab_leg(args, w, net, centres, dev, stream, world, rank):
     for k in range(K):  # warm-up on every timed problem (a property falsified at once warms nothing else)
         net.bab(centres[k], w.eps, specs[k], max_domains=min(args.bab_batch + 1, args.bab_domains), **kw)
     torch.cuda.synchronize()
-    ms, domains, statuses = 0.0, 0, []
+    ms, domains, statuses, per_centre = 0.0, 0, [], []
     for k in range(K):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -649,6 +649,7 @@ def bab_leg(args, w, net, centres, dev, stream, world, rank):
         e1.synchronize()
         ms += e0.elapsed_time(e1)
         domains += r["domains"]
+        per_centre.append(int(r["domains"]))
         statuses.append(r["status"])
     ms = max_over_ranks(ms, dev)
     out = {"value": world * domains / (ms / 1e3) if ms > 0 else None, "unit": "subdomains/s", "subdomains": domains,
@@ -656,23 +657,26 @@ def bab_leg(args, w, net, centres, dev, stream, world, rank):
            "alpha_iters": args.bab_alpha_iters, "eps": w.eps,
            "note": "vf_bab_verify: best-first ReLU-split search; every subdomain bound by vf_verify_batch plus "
                    "alpha-beta ascent, decisions on the device, one host synchronisation per round"}
-    out["label0"] = int(labels[0])
+    # the oracle's timed sample searches the first centre whose device search bounded subdomains (a property
+    # falsified at the root bounds none)
+    k0 = next((k for k in range(K) if per_centre[k] > 0), 0)
+    out["sample_centre"], out["sample_label"] = k0, int(labels[k0])
     return out
 
 
-def oracle_bab_sample(args, w, label):
-    """The oracle's search on the first centre of the same problem as the device's branch-and-bound leg,
-    with a small budget (two rounds), timed on the host cores."""
+def oracle_bab_sample(args, w, k, label):
+    """The oracle's search on centre k of the device's branch-and-bound leg (the first whose search bounded
+    subdomains), same property, with a small budget (two rounds), timed on the host cores."""
     import oracle.lbp as O
     nL = w.net[-1].W.shape[0]
     budget = min(args.bab_domains, 2 * args.bab_batch + 1)
     C0 = synth.margin_spec(np.array([label]), nL)[0]
     t0 = time.perf_counter()
-    o = O.bab(w.net, w.centres[0], w.eps, C0, max_domains=budget, batch=args.bab_batch, iters=args.bab_alpha_iters,
+    o = O.bab(w.net, w.centres[k], w.eps, C0, max_domains=budget, batch=args.bab_batch, iters=args.bab_alpha_iters,
               lr=0.1, crown_relus=w.crown_relus)
     dt = time.perf_counter() - t0
     return {"value": o.domains / dt, "unit": "subdomains/s", "cores": threads_used(), "kind": "oracle",
-            "sample": f"first centre, budget {budget} subdomains ({o.domains} bounded, {o.status}), {dt:.2f} s"}
+            "sample": f"centre {k}, budget {budget} subdomains ({o.domains} bounded, {o.status}), {dt:.2f} s"}
 
 
 def main():

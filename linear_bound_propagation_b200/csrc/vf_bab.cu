@@ -24,13 +24,21 @@ namespace {
 
 using vf::BabPick;
 
+// Scratch of one search, stream-ordered: allocated from the device's memory pool on the search's stream and
+// released on it when the buffer goes out of scope, after the work queued on that stream (no device-wide
+// synchronisation, as a plain free would take).
 struct DeviceBuffer {
     void* p = nullptr;
+    cudaStream_t s = nullptr;
     DeviceBuffer() = default;
     DeviceBuffer(const DeviceBuffer&) = delete;
     DeviceBuffer& operator=(const DeviceBuffer&) = delete;
     ~DeviceBuffer() {
-        if (p) cudaFree(p);
+        if (p) cudaFreeAsync(p, s);
+    }
+    cudaError_t alloc(size_t bytes, cudaStream_t stream) {
+        s = stream;
+        return cudaMallocAsync(&p, bytes, stream);
     }
     template <class T>
     T* get() const {
@@ -235,16 +243,16 @@ extern "C" int vf_bab_verify(vf_net* net, const float* centre, float eps, const 
 
     // ---- device buffers for one round of D subdomains
     DeviceBuffer cen, spl, lbv, lba, plb, pub, pick, meta_off, meta_n, meta_g;
-    BAB_CU(cudaMalloc(&cen.p, sizeof(float) * (size_t)D * n0));
-    BAB_CU(cudaMalloc(&spl.p, (size_t)D * std::max(sum_n, 1)));
-    BAB_CU(cudaMalloc(&lbv.p, sizeof(float) * (size_t)D * R));
-    BAB_CU(cudaMalloc(&lba.p, sizeof(float) * (size_t)D * R));
-    BAB_CU(cudaMalloc(&plb.p, sizeof(float) * (size_t)D * total));
-    BAB_CU(cudaMalloc(&pub.p, sizeof(float) * (size_t)D * total));
-    BAB_CU(cudaMalloc(&pick.p, sizeof(BabPick) * (size_t)D));
-    BAB_CU(cudaMalloc(&meta_off.p, sizeof(long long) * std::max(nl, 1)));
-    BAB_CU(cudaMalloc(&meta_n.p, sizeof(int) * std::max(nl, 1)));
-    BAB_CU(cudaMalloc(&meta_g.p, sizeof(int) * std::max(nl, 1)));
+    BAB_CU(cen.alloc(sizeof(float) * (size_t)D * n0, s));
+    BAB_CU(spl.alloc((size_t)D * std::max(sum_n, 1), s));
+    BAB_CU(lbv.alloc(sizeof(float) * (size_t)D * R, s));
+    BAB_CU(lba.alloc(sizeof(float) * (size_t)D * R, s));
+    BAB_CU(plb.alloc(sizeof(float) * (size_t)D * total, s));
+    BAB_CU(pub.alloc(sizeof(float) * (size_t)D * total, s));
+    BAB_CU(pick.alloc(sizeof(BabPick) * (size_t)D, s));
+    BAB_CU(meta_off.alloc(sizeof(long long) * std::max(nl, 1), s));
+    BAB_CU(meta_n.alloc(sizeof(int) * std::max(nl, 1), s));
+    BAB_CU(meta_g.alloc(sizeof(int) * std::max(nl, 1), s));
     {
         std::vector<long long> ho(nl);
         std::vector<int> hn(nl), hg(nl);
@@ -267,8 +275,8 @@ extern "C" int vf_bab_verify(vf_net* net, const float* centre, float eps, const 
     auto falsified_at = [&](const float* xs, int P, float* ymin_out, bool* hit) -> int {
         *hit = false;
         DeviceBuffer y, yub;
-        BAB_CU(cudaMalloc(&y.p, sizeof(float) * (size_t)P * R));
-        BAB_CU(cudaMalloc(&yub.p, sizeof(float) * (size_t)P * R));
+        BAB_CU(y.alloc(sizeof(float) * (size_t)P * R, s));
+        BAB_CU(yub.alloc(sizeof(float) * (size_t)P * R, s));
         vf_opts o{};
         o.relu_crown = opts->relu_crown;
         BAB_TRY(vf_verify_batch(net, xs, P, 0.f, C, R, 0, &o, y.get<float>(), nullptr, nullptr, nullptr, stream));
@@ -310,9 +318,9 @@ extern "C" int vf_bab_verify(vf_net* net, const float* centre, float eps, const 
         BAB_CU(cudaStreamSynchronize(s));
         if (!(*std::min_element(h.begin(), h.end()) > 0.f)) {
             DeviceBuffer lam, cst, xs;
-            BAB_CU(cudaMalloc(&lam.p, sizeof(float) * (size_t)R * n0));
-            BAB_CU(cudaMalloc(&cst.p, sizeof(float) * (size_t)R));
-            BAB_CU(cudaMalloc(&xs.p, sizeof(float) * (size_t)R * n0));
+            BAB_CU(lam.alloc(sizeof(float) * (size_t)R * n0, s));
+            BAB_CU(cst.alloc(sizeof(float) * (size_t)R, s));
+            BAB_CU(xs.alloc(sizeof(float) * (size_t)R * n0, s));
             BAB_TRY(vf_crown_backward(net, nn - 1, C, R, 0, plb.get<float>(), pub.get<float>(), nullptr, 1,
                                       lam.get<float>(), cst.get<float>(), stream));
             BAB_CU(vf::launch_minimiser_points(centre, lam.get<float>(), eps, n0, R, xs.get<float>(), s));
@@ -354,13 +362,13 @@ extern "C" int vf_bab_verify(vf_net* net, const float* centre, float eps, const 
         const size_t per = (size_t)R * sum_n;  // floats of one subdomain's slopes (and of its multipliers)
         const size_t cap_mem = (size_t(1) << 30) / (2 * per * sizeof(float));
         db.pool_cap = (int)std::min<size_t>((size_t)opts->max_domains, cap_mem);
-        BAB_CU(cudaMalloc(&pool_a.p, sizeof(float) * per * std::max(db.pool_cap, 1)));
-        BAB_CU(cudaMalloc(&pool_b.p, sizeof(float) * per * std::max(db.pool_cap, 1)));
-        BAB_CU(cudaMalloc(&init_a.p, sizeof(float) * per * D));
-        BAB_CU(cudaMalloc(&init_b.p, sizeof(float) * per * D));
-        BAB_CU(cudaMalloc(&out_a.p, sizeof(float) * per * D));
-        BAB_CU(cudaMalloc(&out_b.p, sizeof(float) * per * D));
-        BAB_CU(cudaMalloc(&dslots.p, sizeof(int) * 2 * D));
+        BAB_CU(pool_a.alloc(sizeof(float) * per * std::max(db.pool_cap, 1), s));
+        BAB_CU(pool_b.alloc(sizeof(float) * per * std::max(db.pool_cap, 1), s));
+        BAB_CU(init_a.alloc(sizeof(float) * per * D, s));
+        BAB_CU(init_b.alloc(sizeof(float) * per * D, s));
+        BAB_CU(out_a.alloc(sizeof(float) * per * D, s));
+        BAB_CU(out_b.alloc(sizeof(float) * per * D, s));
+        BAB_CU(dslots.alloc(sizeof(int) * 2 * D, s));
         db.pool_a = pool_a.get<float>();
         db.pool_b = pool_b.get<float>();
         db.init_a = init_a.get<float>();
