@@ -259,8 +259,9 @@ dense_back_ffma(RowRef A, Relax rx, const float* __restrict__ W, const float* __
     }
 }
 
-// Cluster size for the split-K kernel: enough CTAs to cover the SMs twice, at most 8 (the portable
-// cluster limit), a power of two (it divides the tile's 32 rows), and at least two BK slices per rank.
+// Cluster size for the split-K kernel: doubled while the launch stays within two CTAs per SM, at most 8
+// (the portable cluster limit), a power of two (it divides the tile's 32 rows), and at least two BK slices
+// per rank.
 int split_ways(long long ctas, int K, int num_sms) {
     int ks = 1;
     while (ks < 8 && ctas * ks * 2 <= 2LL * num_sms && (long long)(ks * 2) * 2 * BK <= K) ks *= 2;
