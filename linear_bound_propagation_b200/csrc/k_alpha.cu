@@ -31,46 +31,52 @@ unsigned grid_for(long long n, int threads) {
 
 __device__ __forceinline__ bool unstable(const float4& p) { return p.y > 0.f && p.y < 1.f; }
 
-__device__ __forceinline__ float block_sum256(float v, float* red) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-    __syncthreads();
-    float t = 0.f;
-    if (threadIdx.x == 0)
-        for (int i = 0; i < 8; ++i) t += red[i];
-    __syncthreads();
-    return t;
-}
-
 // Z[m, :] (=, += with accumulate) slope * H[m, :] with per-row slopes for unstable neurons (alpha ==
 // nullptr: the table's own lower slope); cst[m] += sum min(H, 0) * t (+ Z * bias, bias in P.w, when
-// with_bias). One CTA per row.
+// with_bias). One warp per row: each lane takes four columns 32 apart per step, so a warp's loads of a
+// step cover 4 x 128 contiguous bytes and are all issued before they are used; a warp reduction gives the
+// row constant.
 __global__ void __launch_bounds__(256)
 relax_alpha_rows_k(const float* __restrict__ H, long long M, int n, const float4* __restrict__ P, PassGeom pg,
                    const float* __restrict__ alpha, float* __restrict__ Z, float* __restrict__ cst, int with_bias,
                    int accumulate, const signed char* __restrict__ split, const float* __restrict__ beta) {
-    __shared__ float red[8];
-    for (long long m = blockIdx.x; m < M; m += gridDim.x) {
+    const int lane = threadIdx.x & 31;
+    for (long long m = blockIdx.x * 8LL + (threadIdx.x >> 5); m < M; m += (long long)gridDim.x * 8) {
         const long long b = (pg.pass_m0 + m) / pg.R_pass;
         const float* h = H + m * n;
+        const float* al = alpha != nullptr ? alpha + m * n : nullptr;
+        const float* be = beta != nullptr ? beta + m * n : nullptr;
+        const float4* Pb = P + b * n;
+        const signed char* sp = split != nullptr ? split + b * n : nullptr;
         float* z = Z + m * n;
         float cs = 0.f;
-        for (int i = threadIdx.x; i < n; i += 256) {
-            const float x = h[i];
-            const float4 p = P[b * n + i];
-            const float lo = (alpha != nullptr && unstable(p)) ? alpha[m * n + i] : p.x;
-            float r = (x >= 0.f) ? x * lo : x * p.y;
-            if (beta != nullptr) {
-                const signed char sg = split[b * n + i];
-                if (sg != 0) r -= (float)sg * beta[m * n + i];
+        for (int i0 = lane; i0 < n; i0 += 128) {
+            float x[4], a[4], old[4], bv[4];
+            float4 p[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + 32 * u;
+                const bool in = i < n;
+                x[u] = in ? h[i] : 0.f;
+                p[u] = in ? Pb[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                a[u] = (in && al != nullptr) ? al[i] : 0.f;
+                old[u] = (in && accumulate) ? z[i] : 0.f;
+                bv[u] = (in && be != nullptr && sp != nullptr && sp[i] != 0) ? (float)sp[i] * be[i] : 0.f;
             }
-            cs = fmaf(fminf(x, 0.f), p.z, cs);
-            if (with_bias) cs = fmaf(r, p.w, cs);
-            z[i] = accumulate ? z[i] + r : r;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + 32 * u;
+                if (i >= n) break;
+                const float lo = (al != nullptr && unstable(p[u])) ? a[u] : p[u].x;
+                const float r = ((x[u] >= 0.f) ? x[u] * lo : x[u] * p[u].y) - bv[u];
+                cs = fmaf(fminf(x[u], 0.f), p[u].z, cs);
+                if (with_bias) cs = fmaf(r, p[u].w, cs);
+                z[i] = accumulate ? old[u] + r : r;
+            }
         }
-        const float t = block_sum256(cs, red);
-        if (threadIdx.x == 0) cst[m] += t;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, off);
+        if (lane == 0) cst[m] += cs;
     }
 }
 
@@ -105,32 +111,51 @@ __device__ __forceinline__ float adam_ascent(float x, float g, float* m1, float*
     return x + lr * (v1 * c1) / (sqrtf(v2 * c2) + 1e-8f);
 }
 
-__global__ void relax_grad_adam_k(float* __restrict__ G, const float* __restrict__ H, long long M, int n,
-                                  const float4* __restrict__ P, PassGeom pg, float* __restrict__ alpha,
-                                  float* __restrict__ grad_out, float* __restrict__ m1, float* __restrict__ m2,
-                                  int adam_step, float lr, float c1, float c2, BetaRows bt) {
-    const long long total = M * n;
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-         e += (long long)gridDim.x * blockDim.x) {
-        const long long m = e / n;
-        const int i = (int)(e % n);
-        const long long bi = ((pg.pass_m0 + m) / pg.R_pass) * n + i;
-        const float4 p = P[bi];
-        const bool un = unstable(p);
-        const float x = H[e];
-        const float a = (alpha != nullptr && un) ? alpha[e] : p.x;
-        const float gz = G[e];
-        const float g = (un && x >= 0.f) ? gz * x : 0.f;
-        G[e] = gz * ((x >= 0.f) ? a : p.y) + ((x < 0.f) ? p.z : 0.f);
-        if (grad_out != nullptr) grad_out[e] = g;
-        if (adam_step > 0 && un && alpha != nullptr)
-            alpha[e] = fminf(fmaxf(adam_ascent(a, g, &m1[e], &m2[e], lr, c1, c2), 0.f), 1.f);
-        if (bt.split != nullptr) {
-            const signed char sg = bt.split[bi];
-            const float gb = (sg != 0) ? -(float)sg * gz : 0.f;
-            if (bt.grad_out != nullptr) bt.grad_out[e] = gb;
-            if (adam_step > 0 && sg != 0 && bt.beta != nullptr)
-                bt.beta[e] = fmaxf(adam_ascent(bt.beta[e], gb, &bt.m1[e], &bt.m2[e], lr, c1, c2), 0.f);
+// One warp per row, four columns 32 apart per lane and step (the row's centre, and so its relaxation and
+// split row, is found once per row rather than by a division per element).
+__global__ void __launch_bounds__(256)
+relax_grad_adam_k(float* __restrict__ G, const float* __restrict__ H, long long M, int n,
+                  const float4* __restrict__ P, PassGeom pg, float* __restrict__ alpha,
+                  float* __restrict__ grad_out, float* __restrict__ m1, float* __restrict__ m2,
+                  int adam_step, float lr, float c1, float c2, BetaRows bt) {
+    const int lane = threadIdx.x & 31;
+    for (long long m = blockIdx.x * 8LL + (threadIdx.x >> 5); m < M; m += (long long)gridDim.x * 8) {
+        const long long b = (pg.pass_m0 + m) / pg.R_pass;
+        const float4* Pb = P + b * n;
+        const signed char* sp = bt.split != nullptr ? bt.split + b * n : nullptr;
+        const long long r0 = m * n;
+        for (int i0 = lane; i0 < n; i0 += 128) {
+            float x[4], gz[4], a[4];
+            float4 p[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + 32 * u;
+                const bool in = i < n;
+                p[u] = in ? Pb[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                x[u] = in ? H[r0 + i] : 0.f;
+                gz[u] = in ? G[r0 + i] : 0.f;
+                a[u] = (in && alpha != nullptr) ? alpha[r0 + i] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + 32 * u;
+                if (i >= n) break;
+                const long long e = r0 + i;
+                const bool un = unstable(p[u]);
+                const float al = (alpha != nullptr && un) ? a[u] : p[u].x;
+                const float g = (un && x[u] >= 0.f) ? gz[u] * x[u] : 0.f;
+                G[e] = gz[u] * ((x[u] >= 0.f) ? al : p[u].y) + ((x[u] < 0.f) ? p[u].z : 0.f);
+                if (grad_out != nullptr) grad_out[e] = g;
+                if (adam_step > 0 && un && alpha != nullptr)
+                    alpha[e] = fminf(fmaxf(adam_ascent(al, g, &m1[e], &m2[e], lr, c1, c2), 0.f), 1.f);
+                if (sp != nullptr) {
+                    const signed char sg = sp[i];
+                    const float gb = (sg != 0) ? -(float)sg * gz[u] : 0.f;
+                    if (bt.grad_out != nullptr) bt.grad_out[e] = gb;
+                    if (adam_step > 0 && sg != 0 && bt.beta != nullptr)
+                        bt.beta[e] = fmaxf(adam_ascent(bt.beta[e], gb, &bt.m1[e], &bt.m2[e], lr, c1, c2), 0.f);
+                }
+            }
         }
     }
 }
@@ -177,7 +202,8 @@ __global__ void best_update_k(float* __restrict__ best, const float* __restrict_
 cudaError_t launch_relax_alpha_rows(const float* H, long long M, int n, const float4* P, PassGeom pg,
                                     const float* alpha, float* Z, float* cst, cudaStream_t s, int with_bias,
                                     int accumulate, BetaRows bt) {
-    long long g = M < 148LL * 16 ? M : 148LL * 16;
+    long long g = (M + 7) / 8;  // eight rows (warps) per CTA
+    if (g > 148LL * 16) g = 148LL * 16;
     relax_alpha_rows_k<<<(unsigned)(g < 1 ? 1 : g), 256, 0, s>>>(H, M, n, P, pg, alpha, Z, cst, with_bias, accumulate,
                                                                  bt.split, bt.split != nullptr ? bt.beta : nullptr);
     return cudaGetLastError();
@@ -199,8 +225,10 @@ cudaError_t launch_relax_grad_adam(float* G, const float* H, long long M, int n,
         c1 = 1.f / (1.f - powf(0.9f, (float)adam_step));
         c2 = 1.f / (1.f - powf(0.999f, (float)adam_step));
     }
-    relax_grad_adam_k<<<grid_for(M * n, 256), 256, 0, s>>>(G, H, M, n, P, pg, alpha, grad_out, m1, m2, adam_step, lr,
-                                                            c1, c2, bt);
+    long long g = (M + 7) / 8;  // eight rows (warps) per CTA
+    if (g > 148LL * 16) g = 148LL * 16;
+    relax_grad_adam_k<<<(unsigned)(g < 1 ? 1 : g), 256, 0, s>>>(G, H, M, n, P, pg, alpha, grad_out, m1, m2, adam_step,
+                                                                 lr, c1, c2, bt);
     return cudaGetLastError();
 }
 
